@@ -1,0 +1,364 @@
+"""Pins for the fp64 oracle: things fixed by the pages and by mathematics, not by
+the oracle itself.
+
+* closed forms worked out by hand (tests/golden/closed_forms.txt);
+* bf16 rounding against torch's fp32 -> bf16 conversion (a library routine);
+* the route-union against brute force (Python sets and sorts);
+* the deduplicated form equals the per-pair form bit for bit;
+* invariants: router-weight scaling, slot permutation, zero weights, token
+  independence;
+* E=1, k=1 reduces to a dense dequantised GEMV -> SwiGLU -> GEMV done with numpy
+  matmul (library routine);
+* a set of planted mistakes (in copies of the oracle source) each fail a pin.
+"""
+import math
+import os
+import subprocess
+import sys
+import tempfile
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.layers import draw_bank, make_layer, read_golden, tiny_layer
+
+GOLD = read_golden("closed_forms.txt")
+
+
+# ---------------------------------------------------------------- helpers ---
+def pack_nibbles(qmat: np.ndarray) -> np.ndarray:
+    """[rows, cols] ints in 0..15 -> [rows, cols/8] uint32, element c = nibble c%8 of word c/8."""
+    rows, cols = qmat.shape
+    q = qmat.astype(np.uint32).reshape(rows, cols // 8, 8)
+    out = np.zeros((rows, cols // 8), np.uint32)
+    for j in range(8):
+        out |= q[:, :, j] << np.uint32(4 * j)
+    return out
+
+
+def bf16_bits(v) -> np.ndarray:
+    return torch.tensor(np.asarray(v, np.float32)).to(torch.bfloat16).view(torch.int16).numpy() \
+        .astype(np.uint16)
+
+
+def const_matrix(rows, cols, q, s, b):
+    qm = np.full((rows, cols), q) if np.isscalar(q) else q
+    return (pack_nibbles(qm)[None], np.full((1, rows, cols // 64), bf16_bits(s), np.uint16),
+            np.full((1, rows, cols // 64), bf16_bits(b), np.uint16))
+
+
+def one_pair(x_vals, gate, up, down, w=0.5, lib=None):
+    H = len(x_vals)
+    x = bf16_bits(np.asarray(x_vals, np.float32))[None]
+    bank = {"gate": gate, "up": up, "down": down}
+    return oracle.switchglu(x, np.zeros((1, 1), np.int32), np.full((1, 1), w, np.float32), bank,
+                            1, want_h=True, lib=lib)
+
+
+def bf16_round_ref(v: np.ndarray) -> np.ndarray:
+    """torch's fp32 -> bf16 (round to nearest even) on values exact in fp32."""
+    return torch.tensor(np.asarray(v, np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+# ------------------------------------------------------------ bf16 rounding ---
+def test_round_bf16_matches_torch_on_fp32_values():
+    rng = np.random.default_rng(1)
+    v = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-30, 30, 20000),
+                        [1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 2 ** -133, 3 * 2 ** -134,
+                         3.3895313892515355e38, 3.3961e38, 0.7310585786300049]]).astype(np.float32)
+    got = np.array([oracle.round_bf16(float(a)) for a in v])
+    assert np.array_equal(got, bf16_round_ref(v))
+
+
+def test_round_bf16_overflow_and_ties():
+    assert oracle.round_bf16(1 + 2 ** -8) == 1.0              # tie -> even
+    assert oracle.round_bf16(1 + 3 * 2 ** -8) == 1 + 2 ** -6  # tie -> even (up)
+    assert oracle.round_bf16(255.5 * 2.0 ** 120) == math.inf  # tie at the top -> inf
+    assert oracle.round_bf16(255.25 * 2.0 ** 120) == 255 * 2.0 ** 120
+    assert oracle.round_bf16(2.0 ** -134) == 0.0              # half the smallest subnormal, tie -> 0
+    assert oracle.round_bf16(0.7310585786300049) == 0.73046875
+
+
+# ------------------------------------------------------------- closed forms ---
+def test_closed_form_all_ones():
+    m = const_matrix(64, 64, 1, 1.0, 0.0)
+    out, h = one_pair([1 / 64] * 64, m, m, m)
+    assert np.all(h[0] == 0.73046875)
+    assert np.all(out == GOLD["A_all_ones"][0])
+
+
+def test_closed_form_affine_scale_and_bias():
+    gu = const_matrix(64, 64, 3, 0.5, -1.0)
+    d = const_matrix(64, 64, 2, 0.25, 0.25)
+    out, _ = one_pair([1 / 32] * 64, gu, gu, d)
+    assert np.all(out == GOLD["B_affine"][0])
+
+
+def test_closed_form_pure_bias():
+    g = const_matrix(64, 64, 0, 1.0, 0.25)
+    u = const_matrix(64, 64, 0, 1.0, 0.5)
+    d = const_matrix(64, 64, 0, 1.0, 1 / 64)
+    out, h = one_pair([1 / 16] * 64, g, u, d)
+    assert np.all(h[0] == 1.4609375)
+    assert np.all(out == GOLD["C_pure_bias"][0])
+
+
+def test_closed_form_identity():
+    eye = const_matrix(64, 64, np.eye(64, dtype=np.int64), 1.0, 0.0)
+    xs = [2.0, -1.0, 0.5, -3.0, 0.0]
+    names = ["x2", "xm1", "x0p5", "xm3", "x0"]
+    x = np.zeros(64, np.float32)
+    x[:5] = xs
+    out, h = one_pair(x, eye, eye, eye, w=1.0)
+    for i, n in enumerate(names):
+        assert h[0][i] == GOLD["D_identity_h_" + n][0], n
+        assert out[0][i] == GOLD["D_identity_h_" + n][0], n
+    assert np.all(h[0][5:] == 0.0)
+
+
+@pytest.mark.parametrize("col", [0, 1, 5, 7, 8, 13, 63, 64, 71, 127])
+def test_nibble_and_group_probe(col):
+    """A single non-zero code at column `col` of row 0 moves G_0 to 5 * scale(group) * x_col."""
+    H = 128
+    qm = np.zeros((64, H), np.int64)
+    qm[0, col] = 5
+    s = np.ones((1, 64, H // 64), np.uint16) * bf16_bits(1.0)
+    s[0, :, 1] = bf16_bits(2.0)   # second group scaled by 2
+    gate = (pack_nibbles(qm)[None], s, np.zeros((1, 64, H // 64), np.uint16))
+    zero = const_matrix(H, 64, 0, 1.0, 0.0)
+    x = np.arange(1, H + 1, dtype=np.float32) / 8      # distinct, exact in bf16
+    out, h = one_pair(x, gate, gate, zero)
+    g = float(bf16_round_ref(np.float32(5 * (1.0 if col < 64 else 2.0) * x[col])))
+    expect = bf16_round_ref(np.float32(g * g / (1 + math.exp(-g))))
+    assert h[0][0] == expect
+    assert np.all(h[0][1:] == 0)
+
+
+# ---------------------------------------------------------------- union ---
+def brute_union(idx, E):
+    P = idx.size
+    flat = idx.ravel()
+    valid = [p for p in range(P) if 0 <= flat[p] < E]
+    uniq = sorted(set(int(flat[p]) for p in valid))
+    plist, offs = [], [0]
+    for e in uniq:
+        plist += [p for p in valid if flat[p] == e]
+        offs.append(len(plist))
+    return uniq, offs, plist + [-1] * (P - len(plist)), P - len(valid)
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_route_union_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    T, k, E = int(rng.integers(1, 20)), int(rng.integers(1, 9)), int(rng.integers(1, 300))
+    idx = rng.integers(-2, E + 2, size=(T, k)).astype(np.int32)   # duplicates and bad ids
+    uniq, offs, plist, u, bad = oracle.route_union(idx, E)
+    bu, bo, bp, bbad = brute_union(idx, E)
+    assert list(uniq) == bu and list(offs) == bo and list(plist) == bp and bad == bbad
+    assert u == len(set(int(e) for e in idx.ravel() if 0 <= e < E))
+
+
+def test_route_union_extremes():
+    T, k, E = 16, 8, 256
+    same = np.tile(np.arange(8, dtype=np.int32) * 3, (T, 1))
+    uniq, offs, plist, u, _ = oracle.route_union(same, E)
+    assert u == k and list(np.diff(offs)) == [T] * k
+    disjoint = np.arange(T * k, dtype=np.int32).reshape(T, k)
+    uniq, offs, plist, u, _ = oracle.route_union(disjoint, E)
+    assert u == T * k and list(plist) == list(range(T * k))
+
+
+# ------------------------------------------------------- dedup == per pair ---
+@pytest.mark.parametrize("cfg", [(2, 2, 16, 256, 128, "softmax"), (5, 4, 8, 128, 192, "uniform"),
+                                 (6, 3, 4, 64, 64, "uniform")])
+def test_dedup_equals_per_pair_bitwise(cfg):
+    T, k, E, H, I, routing = cfg
+    L = make_layer(T, k, E, H, I, seed=3, routing=routing)
+    out, h = oracle.switchglu(L.x, L.idx, L.w, L.bank, E, want_h=True)
+    out2, h2 = oracle.switchglu_union(L.x, L.idx, L.w, L.bank, E, want_h=True)
+    assert np.array_equal(out, out2) and np.array_equal(h, h2)
+
+
+def test_duplicate_expert_in_token_counts_twice():
+    L = make_layer(1, 2, 4, 64, 64, seed=5, idx=np.array([[2, 2]], np.int32),
+                   w=np.array([[0.25, 0.5]], np.float32))
+    single = make_layer(1, 1, 4, 64, 64, seed=5, idx=np.array([[2]], np.int32),
+                        w=np.array([[1.0]], np.float32))
+    out = oracle.switchglu(L.x, L.idx, L.w, L.bank, 4)
+    y = oracle.switchglu(single.x, single.idx, single.w, single.bank, 4)
+    assert np.allclose(out, 0.75 * y, rtol=1e-15, atol=0)
+
+
+# --------------------------------------------------------------- invariants ---
+def test_router_weight_scaling_and_zero():
+    L = make_layer(3, 4, 12, 128, 64, seed=7)
+    base = oracle.switchglu(L.x, L.idx, L.w, L.bank, L.E)
+    for a in (2.0, 0.5, 0.0):
+        got = oracle.switchglu(L.x, L.idx, L.w * np.float32(a), L.bank, L.E)
+        assert np.array_equal(got, a * base)
+
+
+def test_slot_permutation_invariance():
+    L = make_layer(3, 4, 12, 128, 64, seed=8)
+    base = oracle.switchglu(L.x, L.idx, L.w, L.bank, L.E)
+    perm = np.array([2, 0, 3, 1])
+    got = oracle.switchglu(L.x, L.idx[:, perm], L.w[:, perm], L.bank, L.E)
+    assert np.allclose(got, base, rtol=1e-13, atol=1e-12 * np.abs(base).max())
+
+
+def test_token_independence_and_token_subset():
+    L = make_layer(4, 3, 10, 128, 128, seed=9)
+    full = oracle.switchglu(L.x, L.idx, L.w, L.bank, L.E)
+    for t in range(L.T):
+        one = oracle.switchglu(L.x[t:t + 1], L.idx[t:t + 1], L.w[t:t + 1], L.bank, L.E)
+        assert np.array_equal(one[0], full[t])
+    sub = oracle.switchglu(L.x, L.idx, L.w, L.bank, L.E, tokens=[2])
+    assert np.array_equal(sub[2], full[2]) and np.isnan(sub[0]).all()
+
+
+def test_invalid_expert_contributes_nothing():
+    L = make_layer(2, 3, 6, 64, 64, seed=10, idx=np.array([[1, 7, 2], [-1, 3, 3]], np.int32))
+    out = oracle.switchglu(L.x, L.idx, L.w, L.bank, L.E)
+    w2 = L.w.copy()
+    w2[0, 1] = 0
+    w2[1, 0] = 0
+    idx2 = L.idx.copy()
+    idx2[0, 1] = 0
+    idx2[1, 0] = 0
+    ref = oracle.switchglu(L.x, idx2, w2, L.bank, L.E)
+    assert np.array_equal(out, ref)
+
+
+# ---------------------------------------------------- textbook special case ---
+def dense_dequant(q, s, b):
+    rows, words = q.shape
+    cols = words * 8
+    nib = np.stack([(q >> np.uint32(4 * j)) & np.uint32(15) for j in range(8)], axis=-1)
+    nib = nib.reshape(rows, cols).astype(np.float64)
+    sf = synth.bf16_bits_to_f32(s).astype(np.float64).repeat(64, axis=1)
+    bf = synth.bf16_bits_to_f32(b).astype(np.float64).repeat(64, axis=1)
+    return sf * nib + bf
+
+
+@pytest.mark.parametrize("HI", [(128, 64), (256, 192)])
+def test_single_expert_is_dense_swiglu(HI):
+    H, I = HI
+    L = make_layer(1, 1, 1, H, I, seed=11, idx=np.zeros((1, 1), np.int32),
+                   w=np.ones((1, 1), np.float32))
+    out, h = oracle.switchglu(L.x, L.idx, L.w, L.bank, 1, want_h=True)
+    Wg = dense_dequant(L.bank["gate"][0][0], L.bank["gate"][1][0], L.bank["gate"][2][0])
+    Wu = dense_dequant(L.bank["up"][0][0], L.bank["up"][1][0], L.bank["up"][2][0])
+    Wd = dense_dequant(L.bank["down"][0][0], L.bank["down"][1][0], L.bank["down"][2][0])
+    x = synth.bf16_bits_to_f32(L.x[0]).astype(np.float64)
+    g = bf16_round_ref(Wg @ x)
+    v = bf16_round_ref(Wu @ x)
+    href = bf16_round_ref(g * v / (1 + np.exp(-g)))
+    # library sums may differ from the oracle's ascending order in the last bits: allow one
+    # bf16 step where a value sits on a rounding boundary, and compare y tightly
+    ulp = np.abs(href) * 2.0 ** -7 + 1e-30
+    assert np.all(np.abs(h[0] - href) <= ulp)
+    assert np.mean(h[0] == href) > 0.97
+    yref = Wd @ h[0]
+    assert np.allclose(out[0], yref, rtol=1e-12, atol=1e-12 * np.abs(yref).max())
+
+
+def test_tiny_layer_runs_and_is_finite():
+    L = tiny_layer()
+    out = oracle.switchglu(L.x, L.idx, L.w, L.bank, L.E)
+    assert np.isfinite(out).all() and np.abs(out).max() > 0
+
+
+# ----------------------------------------------------------- planted mistakes ---
+MUTANTS = {
+    "nibble_msb_first": ("(word >> (4 * (col % 8)))", "(word >> (4 * (7 - col % 8)))"),
+    "bias_dropped": ("return bf16_value(s[g]) * nib + bf16_value(b[g]);",
+                     "return bf16_value(s[g]) * nib;"),
+    "gate_not_rounded": ("const double g = round_bf16(G), v = round_bf16(U);",
+                         "const double g = G, v = round_bf16(U);"),
+    "sigmoid_sign": ("std::exp(-g)", "std::exp(g)"),
+    "router_weight_dropped": ("acc += static_cast<double>(L.w[p]) * Y[",
+                              "acc += Y["),
+    "down_transposed": ("Y += L.down.at(e, c, r) * h[r];", "Y += L.down.at(e, r, c) * h[r];"),
+    "h_product_unrounded": ("h[r] = round_bf16(g * sigmoid(g) * v);", "h[r] = g * sigmoid(g) * v;"),
+}
+
+_MUTANT_CHECK = r"""
+import sys, numpy as np
+sys.path.insert(0, {root!r})
+import oracle
+from tests import test_oracle_pins as P
+lib = oracle.load({so!r})
+fails = 0
+def run(f):
+    global fails
+    try:
+        f(lib)
+    except AssertionError:
+        fails += 1
+run(P._pin_closed_forms)
+run(P._pin_textbook)
+print("FAILS", fails)
+"""
+
+
+def _pin_closed_forms(lib):
+    m = const_matrix(64, 64, 1, 1.0, 0.0)
+    out, _ = one_pair([1 / 64] * 64, m, m, m, lib=lib)
+    assert np.all(out == GOLD["A_all_ones"][0])
+    gu = const_matrix(64, 64, 3, 0.5, -1.0)
+    d = const_matrix(64, 64, 2, 0.25, 0.25)
+    out, _ = one_pair([1 / 32] * 64, gu, gu, d, lib=lib)
+    assert np.all(out == GOLD["B_affine"][0])
+    g = const_matrix(64, 64, 0, 1.0, 0.25)
+    u = const_matrix(64, 64, 0, 1.0, 0.5)
+    dd = const_matrix(64, 64, 0, 1.0, 1 / 64)
+    out, _ = one_pair([1 / 16] * 64, g, u, dd, lib=lib)
+    assert np.all(out == GOLD["C_pure_bias"][0])
+    eye = const_matrix(64, 64, np.eye(64, dtype=np.int64), 1.0, 0.0)
+    x = np.zeros(64, np.float32)
+    x[:4] = [2.0, -1.0, 0.5, -3.0]
+    out, h = one_pair(x, eye, eye, eye, w=1.0, lib=lib)
+    assert h[0][0] == GOLD["D_identity_h_x2"][0] and h[0][3] == GOLD["D_identity_h_xm3"][0]
+
+
+def _pin_textbook(lib):
+    H, I = 128, 64
+    L = make_layer(1, 1, 1, H, I, seed=11, idx=np.zeros((1, 1), np.int32),
+                   w=np.full((1, 1), 0.75, np.float32))
+    qidx = np.zeros((1, 1), np.int32)
+    out, h = oracle.switchglu(L.x, qidx, L.w, L.bank, 1, want_h=True, lib=lib)
+    Wg = dense_dequant(*[a[0] for a in L.bank["gate"]])
+    Wu = dense_dequant(*[a[0] for a in L.bank["up"]])
+    Wd = dense_dequant(*[a[0] for a in L.bank["down"]])
+    x = synth.bf16_bits_to_f32(L.x[0]).astype(np.float64)
+    g = bf16_round_ref(Wg @ x)
+    v = bf16_round_ref(Wu @ x)
+    href = bf16_round_ref(g * v / (1 + np.exp(-g)))
+    assert np.mean(h[0] == href) > 0.97
+    yref = 0.75 * (Wd @ href)
+    assert np.allclose(out[0], yref, rtol=0, atol=1e-3 * np.abs(yref).max())
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_fails_a_pin(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "oracle.cpp")).read()
+    assert old in src, "mutation site vanished: update the mutant"
+    mpath = tmp_path / "oracle_mut.cpp"
+    mpath.write_text(src.replace(old, new))
+    so = str(tmp_path / "liboracle_mut.so")
+    oracle.build(str(mpath), so)
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _MUTANT_CHECK.format(root=root, so=so)],
+                       capture_output=True, text=True, timeout=300)
+    assert "FAILS" in r.stdout, r.stderr[-2000:]
+    assert int(r.stdout.split("FAILS")[1].split()[0]) >= 1, f"mutant {name} passed every pin"
+
+
+def test_unmutated_oracle_passes_mutant_pins():
+    lib = oracle.load()
+    _pin_closed_forms(lib)
+    _pin_textbook(lib)

@@ -1,0 +1,108 @@
+"""Checks of the seeded input generators and of the byte model the metric uses.
+
+The byte model and the routing statistics are pinned by numbers the pages print
+(tests/golden/page_numbers.txt)."""
+import numpy as np
+import pytest
+
+import synth
+from tests.layers import read_golden
+
+PAGE = read_golden("page_numbers.txt")
+
+
+def bytes_per_expert(H: int, I: int) -> int:
+    """gate + up + down of one expert: 4-bit codes plus bf16 scale and bias per group of 64."""
+    per_matrix = I * H // 2 + 2 * 2 * I * H // 64
+    return 3 * per_matrix
+
+
+def test_byte_model_matches_page():
+    H, I = int(PAGE["hidden"][0]), int(PAGE["intermediate"][0])
+    be = bytes_per_expert(H, I)
+    assert be == 14_155_776
+    assert round(be / 1e6, 1) == PAGE["bytes_per_expert_MB"][0]
+    # the page's GB/s column counts M * TOPK blocks: recompute it from the printed times
+    for key in ("row_M1_isolated", "row_M1_chained", "row_M4_isolated", "row_M4_chained"):
+        ms, gbs, blocks = PAGE[key]
+        assert abs(blocks * be / (ms * 1e-3) / 1e9 - gbs) / gbs < 0.005, key
+
+
+def test_union_floor_arithmetic_matches_page():
+    k = 8
+    p = PAGE["overlap_mean"][0]
+    assert round(2 * k - k * p, 1) == PAGE["uniques_per_pair"][0]
+    assert abs(k / 256 - PAGE["random_overlap"][0]) < 0.002
+
+
+@pytest.mark.parametrize("p", [0.03, 0.21, 0.34, 0.45, 0.52])
+def test_verify_pair_overlap_statistics(p):
+    E, k, n = 256, 8, 3000
+    us, ov = [], []
+    for s in range(n):
+        idx, w = synth.route_verify_pair(E, k, p, 1000 * 3 + s)
+        assert len(set(idx[0])) == k and len(set(idx[1])) == k
+        assert np.allclose(w.sum(1), 1.0, atol=1e-6)
+        us.append(len(set(idx.ravel().tolist())))
+        ov.append(len(set(idx[0]) & set(idx[1])) / k)
+    # E[u] = 2k - k p ; standard error of the mean ~ sqrt(k p (1-p) / n) < 0.03
+    assert abs(np.mean(us) - (2 * k - k * p)) < 0.12
+    assert abs(np.mean(ov) - p) < 0.015
+
+
+def test_markov_chain_uniques_track_page_table():
+    """A p=0.34 chain reproduces the measured union-floor uniques at L=1..4 within
+    a unique or so (real routing has longer-range correlation; L=6 drifts up)."""
+    E, k = 256, 8
+    want = PAGE["chain_uniques"]
+    for L, target, tol in zip((1, 2, 3, 4, 6), want, (0.01, 0.5, 0.8, 1.0, 2.0)):
+        u = np.mean([len(set(synth.route_markov(L, E, k, 0.34, s)[0].ravel().tolist()))
+                     for s in range(800)])
+        assert abs(u - target) <= tol, (L, u, target)
+
+
+def test_softmax_topk_routing():
+    idx, w = synth.route_softmax_topk(2, 16, 2, 0)
+    assert idx.shape == (2, 2) and np.allclose(w.sum(1), 1)
+    assert np.all(w[:, 0] >= w[:, 1])
+
+
+def test_bank_is_deterministic_and_subset_consistent():
+    full = synth.fill_bank_host(6, 64, 128, 42, 1)
+    part = synth.fill_bank_host(6, 64, 128, 42, 1, experts=[4, 1])
+    for a, b in zip(full, part):
+        assert np.array_equal(a[[1, 4]], b[[1, 4]])
+        assert not b[[0, 2, 3, 5]].any()
+    other = synth.fill_bank_host(6, 64, 128, 43, 1)
+    assert not np.array_equal(full[0], other[0])
+
+
+def test_quantiser_round_trip():
+    """|dequant(quant(w)) - w| <= scale/2 + the bf16 rounding of scale and bias."""
+    E, rows, cols, seed, mid = 3, 16, 256, 5, 2
+    q, s, b = synth.fill_bank_host(E, rows, cols, seed, mid)
+    for e in range(E):
+        for r in range(rows):
+            w = synth.draw_row(E, rows, cols, seed, mid, e, r).astype(np.float64)
+            nib = np.array([(q[e, r, c // 8] >> (4 * (c % 8))) & 15 for c in range(cols)],
+                           np.float64)
+            sf = synth.bf16_bits_to_f32(s[e, r]).astype(np.float64).repeat(64)
+            bf = synth.bf16_bits_to_f32(b[e, r]).astype(np.float64).repeat(64)
+            wq = sf * nib + bf
+            g = w.reshape(-1, 64)
+            rng = (g.max(1) - g.min(1)).repeat(64)
+            # scale off by <= 2^-8 relative, bias by <= 2^-8 |min|, over 15 codes
+            bound = sf / 2 + 15 * rng / 15 * 2.0 ** -8 + np.abs(bf) * 2.0 ** -8 + 1e-6
+            assert np.all(np.abs(wq - w) <= bound)
+
+
+def test_normal_draw_moments():
+    r = np.concatenate([synth.draw_row(1, 64, 4096, 9, 0, 0, i) for i in range(64)])
+    assert abs(r.mean()) < 0.01 and abs(r.std() - 1) < 0.01
+    assert r.min() >= -6 and r.max() <= 6
+
+
+def test_x_bf16_rounding():
+    x = synth.x_bf16(3, 64, 2)
+    f = synth.bf16_bits_to_f32(x)
+    assert x.dtype == np.uint16 and np.isfinite(f).all() and abs(f.std() - 1) < 0.3
