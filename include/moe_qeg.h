@@ -1,0 +1,157 @@
+/*
+ * moe_qeg.h - union-of-experts 4-bit quantized MoE SwitchGLU layer for NVIDIA
+ * B200 (sm_100a).  C ABI; plain pointers and sizes only.
+ *
+ * What the layer computes (per window of T tokens routed top-k over E experts):
+ *   for every (token t, slot j) pair p = t*k + j with expert e = topk_idx[p]:
+ *     g = bf16(Wg[e] x_t), v = bf16(Wu[e] x_t)   (fp32 accumulation)
+ *     h = bf16(silu(g) * v)
+ *     y = Wd[e] h                               (fp32)
+ *   out[t] = bf16( sum_j topk_w[t, j] * y_(t, j) )
+ * where each weight matrix is 4-bit affine quantized with groups of 64 input
+ * columns: w = scale * q + bias, q in 0..15, scale and bias bf16.  This is the
+ * SwitchGLU of the moe_bench.py script in "gather_qmm at M=1 streams 4-bit
+ * expert weights at ~half the bandwidth of M=4" (mlx issue 4509, "Script":
+ * up, gate, silu(gate)*up, down, mx.quantize group 64, bits 4, affine), with
+ * the one-pass bf16(up)*silu(gate) epilogue of "Apple7/8 MoE gate and up in
+ * one decode pass" (splash PR 45, "What changed").
+ *
+ * How: instead of streaming one expert block per (token, expert) pair, the
+ * union of the routed experts is formed once and each distinct expert's
+ * gate/up/down block is read from HBM once and applied to every pair routed to
+ * it ("Small-L fused expert gather for fine-grained MoE decode", mlx discussion
+ * 3801, first post "Two implications" item 1, and the sort-by-expert /
+ * ragged-matmul framing of the second post).
+ *
+ * Layouts (row-major, all device memory, caller-owned):
+ *   x          bf16 [T, hidden]
+ *   topk_idx   int32 [T, k]       expert ids; ids outside [0, E) are skipped
+ *                                 and flagged (see moe_read_device_status)
+ *   topk_w     fp32 [T, k]        router weights, used as given
+ *   wg_q, wu_q uint32 [E, inter, hidden/8]  (gate, up: rows = output features)
+ *   wg_s/wg_b, wu_s/wu_b  bf16 [E, inter, hidden/64]
+ *   wd_q       uint32 [E, hidden, inter/8]
+ *   wd_s/wd_b  bf16 [E, hidden, inter/64]
+ *   out        bf16 [T, hidden]
+ * Element c of a weight row is nibble c % 8 (bits 4*(c%8) .. 4*(c%8)+3, least
+ * significant first) of 32-bit word c / 8.  bf16 values are passed as their
+ * raw 16-bit patterns (uint16_t).
+ *
+ * Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL is
+ * the legacy default stream).  They perform no host synchronisation, no
+ * device allocation (except where stated) and no host-device copies.
+ * Results are deterministic: the same inputs give the same bits on every run.
+ */
+#ifndef MOE_QEG_H
+#define MOE_QEG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad multiple */
+  MOE_ERR_UNSUPPORTED = 2,  /* shape outside the supported range, misaligned pointer */
+  MOE_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  MOE_ERR_DEVICE_INDEX = 4, /* a kernel met an expert id outside [0, E) */
+  MOE_ERR_TIMEOUT = 5,      /* a kernel's bounded wait ran out (internal error) */
+  MOE_ERR_WORKSPACE = 6     /* workspace too small, or growth needed during capture */
+} moe_status;
+
+/* Supported range (checked on the host; violations return MOE_ERR_UNSUPPORTED):
+ * hidden and inter multiples of 64 and <= 8192; E <= 1024; T*k <= 65536. */
+#define MOE_MAX_EXPERTS 1024
+#define MOE_MAX_DIM 8192
+#define MOE_MAX_PAIRS 65536
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_str(int status);
+
+/* Bytes of workspace that moe_switchglu_forward_ws needs for this shape
+ * (0 on invalid arguments).  The workspace holds the route-union arrays and
+ * h = bf16 [T*k, inter]; its contents are scratch between calls. */
+size_t moe_workspace_size(int T, int k, int E, int hidden, int inter);
+
+/*
+ * Route-union ("Small-L fused expert gather", mlx discussion 3801, second
+ * post: sort the (position, expert) pairs by expert and stream each unique
+ * expert once).  From topk_idx [T, k] (device) it writes (device):
+ *   unique[min(E, T*k)]     distinct expert ids, ascending
+ *   offsets[min(E, T*k)+1]  offsets[i] = number of pairs of unique[0..i);
+ *                           offsets[u] = number of valid pairs
+ *   pair_list[T*k]          pair ids p = t*k + j grouped by expert in the
+ *                           order of `unique`, ascending p within an expert;
+ *                           entries past offsets[u] are -1
+ *   num_unique[1]           u
+ * Entries of unique/offsets past u (resp. u+1) are left unchanged.  Pairs
+ * with an id outside [0, E) are left out and flag MOE_ERR_DEVICE_INDEX.
+ * All arrays must be 4-byte aligned.  Integer output, bit-exact.
+ */
+moe_status moe_route_union(const int32_t* topk_idx, int T, int k, int E, int32_t* unique,
+                           int32_t* offsets, int32_t* pair_list, int32_t* num_unique,
+                           void* stream);
+
+/*
+ * The fused union-of-experts SwitchGLU forward described at the top of this
+ * file, using caller-provided device workspace of at least
+ * moe_workspace_size(T, k, E, hidden, inter) bytes (16-byte aligned).
+ * x, the weight arrays, out and workspace must be 16-byte aligned; topk_idx
+ * and topk_w 4-byte aligned.  Tokens whose pairs are all invalid get a zero
+ * output row.  Capturable in a CUDA graph.
+ */
+moe_status moe_switchglu_forward_ws(const uint16_t* x, const int32_t* topk_idx,
+                                    const float* topk_w, const uint32_t* wg_q,
+                                    const uint16_t* wg_s, const uint16_t* wg_b,
+                                    const uint32_t* wu_q, const uint16_t* wu_s,
+                                    const uint16_t* wu_b, const uint32_t* wd_q,
+                                    const uint16_t* wd_s, const uint16_t* wd_b, int T, int k,
+                                    int E, int hidden, int inter, uint16_t* out, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/*
+ * Same as moe_switchglu_forward_ws with a library-owned workspace per device.
+ * The workspace is allocated (cudaMalloc) on the first call that needs more
+ * than the current one; such a call must not be made during stream capture
+ * (it returns MOE_ERR_WORKSPACE then).  The buffer lives until process exit.
+ * Calls on different streams of one device share it and must not overlap.
+ */
+moe_status moe_switchglu_forward(const uint16_t* x, const int32_t* topk_idx, const float* topk_w,
+                                 const uint32_t* wg_q, const uint16_t* wg_s,
+                                 const uint16_t* wg_b, const uint32_t* wu_q,
+                                 const uint16_t* wu_s, const uint16_t* wu_b,
+                                 const uint32_t* wd_q, const uint16_t* wd_s,
+                                 const uint16_t* wd_b, int T, int k, int E, int hidden,
+                                 int inter, uint16_t* out, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word that the
+ * kernels set instead of trapping: MOE_ERR_DEVICE_INDEX if an expert id was
+ * out of range, MOE_ERR_TIMEOUT if a bounded wait ran out, else MOE_OK (or
+ * MOE_ERR_CUDA if the synchronisation itself failed).
+ */
+moe_status moe_read_device_status(void* stream);
+
+/*
+ * Which kernel path a call with this shape takes, without launching anything:
+ * 1 = expert-major dequant-GEMV path (route-union, fused gate+up, down with
+ * combine), 2 = grouped tensor-core path, 0 = invalid/unsupported shape.
+ */
+int moe_select_path(int T, int k, int E, int hidden, int inter);
+
+/*
+ * Offsets (bytes) of the workspace regions for this shape, for inspection in
+ * tests: out[0] = num_unique (int32), out[1] = unique, out[2] = offsets,
+ * out[3] = pair_list, out[4] = h (bf16 [T*k, inter] in pair_list order),
+ * out[5] = total bytes.  Returns MOE_ERR_INVALID_ARG on bad shapes.
+ */
+moe_status moe_workspace_layout(int T, int k, int E, int hidden, int inter, size_t out[6]);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_QEG_H */

@@ -1,0 +1,199 @@
+"""Python binding of libmoe_qeg (include/moe_qeg.h): union-of-experts 4-bit
+quantized MoE SwitchGLU layer for B200 (sm_100a).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  The functions take torch CUDA tensors, check dtypes and shapes, and
+pass raw pointers plus the current CUDA stream to the C entry points of the
+same name.  If the compiled library is missing or cannot be loaded this module
+raises on import: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from ._build import SO, build as build_library, needs_build
+
+__all__ = ["MoeError", "MOE_OK", "moe_status_str", "moe_workspace_size", "moe_workspace_layout",
+           "moe_select_path", "moe_route_union", "moe_switchglu_forward",
+           "moe_switchglu_forward_ws", "moe_read_device_status", "library_path", "QuantBank"]
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_CUDA = 3
+MOE_ERR_DEVICE_INDEX = 4
+MOE_ERR_TIMEOUT = 5
+MOE_ERR_WORKSPACE = 6
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {moe_status_str(status)} ({status})")
+        self.status = status
+
+
+def _load():
+    if needs_build():
+        build_library()
+    lib = ctypes.CDLL(SO)
+    vp, ci, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.moe_status_str.restype = ctypes.c_char_p
+    lib.moe_status_str.argtypes = [ci]
+    lib.moe_workspace_size.restype = sz
+    lib.moe_workspace_size.argtypes = [ci] * 5
+    lib.moe_workspace_layout.restype = ci
+    lib.moe_workspace_layout.argtypes = [ci] * 5 + [vp]
+    lib.moe_select_path.restype = ci
+    lib.moe_select_path.argtypes = [ci] * 5
+    lib.moe_route_union.restype = ci
+    lib.moe_route_union.argtypes = [vp, ci, ci, ci, vp, vp, vp, vp, vp]
+    lib.moe_switchglu_forward.restype = ci
+    lib.moe_switchglu_forward.argtypes = [vp] * 12 + [ci] * 5 + [vp, vp]
+    lib.moe_switchglu_forward_ws.restype = ci
+    lib.moe_switchglu_forward_ws.argtypes = [vp] * 12 + [ci] * 5 + [vp, vp, sz, vp]
+    lib.moe_read_device_status.restype = ci
+    lib.moe_read_device_status.argtypes = [vp]
+    return lib
+
+
+_lib = _load()
+
+
+def library_path() -> str:
+    return SO
+
+
+def moe_status_str(status: int) -> str:
+    return _lib.moe_status_str(int(status)).decode()
+
+
+def _check(status: int, where: str, check: bool) -> int:
+    if check and status != MOE_OK:
+        raise MoeError(status, where)
+    return status
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: torch.Tensor, dtypes, name: str) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+_BF16 = (torch.bfloat16, torch.int16, torch.uint16)
+_Q = (torch.int32, torch.uint32)
+_I32 = (torch.int32,)
+_F32 = (torch.float32,)
+
+
+def moe_workspace_size(T: int, k: int, E: int, hidden: int, inter: int) -> int:
+    return int(_lib.moe_workspace_size(T, k, E, hidden, inter))
+
+
+def moe_workspace_layout(T: int, k: int, E: int, hidden: int, inter: int) -> dict:
+    out = (ctypes.c_size_t * 6)()
+    _check(_lib.moe_workspace_layout(T, k, E, hidden, inter, ctypes.addressof(out)),
+           "moe_workspace_layout", True)
+    return dict(zip(("num_unique", "unique", "offsets", "pair_list", "h", "total"), list(out)))
+
+
+def moe_select_path(T: int, k: int, E: int, hidden: int, inter: int) -> int:
+    return int(_lib.moe_select_path(T, k, E, hidden, inter))
+
+
+def moe_route_union(topk_idx: torch.Tensor, E: int, unique=None, offsets=None, pair_list=None,
+                    num_unique=None, stream=None, check: bool = True):
+    """Route-union of topk_idx [T, k] (int32, CUDA).  Returns (unique, offsets, pair_list,
+    num_unique) device tensors of sizes min(E,P), min(E,P)+1, P, 1."""
+    T, k = topk_idx.shape
+    P = T * k
+    m = max(1, min(E, P))
+    dev = topk_idx.device
+    unique = unique if unique is not None else torch.zeros(m, dtype=torch.int32, device=dev)
+    offsets = offsets if offsets is not None else torch.zeros(m + 1, dtype=torch.int32, device=dev)
+    pair_list = pair_list if pair_list is not None else torch.zeros(P, dtype=torch.int32,
+                                                                    device=dev)
+    num_unique = num_unique if num_unique is not None else torch.zeros(1, dtype=torch.int32,
+                                                                       device=dev)
+    st = _lib.moe_route_union(_ptr(topk_idx, _I32, "topk_idx"), T, k, E,
+                              _ptr(unique, _I32, "unique"), _ptr(offsets, _I32, "offsets"),
+                              _ptr(pair_list, _I32, "pair_list"),
+                              _ptr(num_unique, _I32, "num_unique"), _stream(stream))
+    _check(st, "moe_route_union", check)
+    return unique, offsets, pair_list, num_unique
+
+
+class QuantBank:
+    """Device tensors of one layer's expert bank: gate/up q [E, inter, hidden/8],
+    s/b [E, inter, hidden/64]; down q [E, hidden, inter/8], s/b [E, hidden, inter/64]."""
+
+    def __init__(self, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q, wd_s, wd_b):
+        self.wg_q, self.wg_s, self.wg_b = wg_q, wg_s, wg_b
+        self.wu_q, self.wu_s, self.wu_b = wu_q, wu_s, wu_b
+        self.wd_q, self.wd_s, self.wd_b = wd_q, wd_s, wd_b
+        self.E, self.inter, hw = wg_q.shape
+        self.hidden = hw * 8
+        for name, t, shape in (("wg_s", wg_s, (self.E, self.inter, self.hidden // 64)),
+                               ("wu_q", wu_q, wg_q.shape),
+                               ("wd_q", wd_q, (self.E, self.hidden, self.inter // 8)),
+                               ("wd_s", wd_s, (self.E, self.hidden, self.inter // 64))):
+            if tuple(t.shape) != tuple(shape):
+                raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+    def ptrs(self):
+        return [_ptr(self.wg_q, _Q, "wg_q"), _ptr(self.wg_s, _BF16, "wg_s"),
+                _ptr(self.wg_b, _BF16, "wg_b"), _ptr(self.wu_q, _Q, "wu_q"),
+                _ptr(self.wu_s, _BF16, "wu_s"), _ptr(self.wu_b, _BF16, "wu_b"),
+                _ptr(self.wd_q, _Q, "wd_q"), _ptr(self.wd_s, _BF16, "wd_s"),
+                _ptr(self.wd_b, _BF16, "wd_b")]
+
+
+def _fwd_args(x, topk_idx, topk_w, bank: QuantBank, out):
+    T, hidden = x.shape
+    k = topk_idx.shape[1]
+    if hidden != bank.hidden or tuple(topk_idx.shape) != (T, k) or tuple(topk_w.shape) != (T, k):
+        raise ValueError("x / topk_idx / topk_w shapes do not match the bank")
+    if out is None:
+        out = torch.empty((T, hidden), dtype=torch.bfloat16, device=x.device)
+    if tuple(out.shape) != (T, hidden):
+        raise ValueError("out has the wrong shape")
+    args = [_ptr(x, _BF16, "x"), _ptr(topk_idx, _I32, "topk_idx"), _ptr(topk_w, _F32, "topk_w"),
+            *bank.ptrs()]
+    return args, (T, k, bank.E, hidden, bank.inter), out
+
+
+def moe_switchglu_forward(x, topk_idx, topk_w, bank: QuantBank, out=None, stream=None,
+                          check: bool = True):
+    """out [T, hidden] bf16 = union-of-experts SwitchGLU of x [T, hidden] bf16."""
+    args, dims, out = _fwd_args(x, topk_idx, topk_w, bank, out)
+    st = _lib.moe_switchglu_forward(*args, *dims, _ptr(out, _BF16, "out"), _stream(stream))
+    _check(st, "moe_switchglu_forward", check)
+    return out
+
+
+def moe_switchglu_forward_ws(x, topk_idx, topk_w, bank: QuantBank, workspace: torch.Tensor,
+                             out=None, stream=None, check: bool = True):
+    """As moe_switchglu_forward, with a caller-owned uint8 device workspace tensor."""
+    args, dims, out = _fwd_args(x, topk_idx, topk_w, bank, out)
+    st = _lib.moe_switchglu_forward_ws(*args, *dims, _ptr(out, _BF16, "out"),
+                                       _ptr(workspace, (torch.uint8,), "workspace"),
+                                       workspace.numel(), _stream(stream))
+    _check(st, "moe_switchglu_forward_ws", check)
+    return out
+
+
+def moe_read_device_status(stream=None) -> int:
+    return int(_lib.moe_read_device_status(_stream(stream)))

@@ -1,0 +1,337 @@
+// C ABI of the union-of-experts quantized SwitchGLU library (include/moe_qeg.h):
+// argument validation, workspace layout, path selection and kernel launches.
+// Everything here is host code; the arithmetic is in the kernels.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe_qeg.h"
+#include "common.cuh"
+#include "gemv.cuh"
+#include "route_union.cuh"
+
+namespace qeg {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 0;
+  int smem_optin = 0;
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+// Per-device state: SM count, shared-memory limit, kernel attributes set once.
+moe_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (cudaFuncSetAttribute(gate_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             d.smem_optin) != cudaSuccess ||
+        cudaFuncSetAttribute(down_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             d.smem_optin) != cudaSuccess ||
+        cudaFuncSetAttribute(route_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             d.smem_optin) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    d.ready = true;
+  }
+  *out = &d;
+  return MOE_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool shape_ok(int T, int k, int E, int hidden, int inter) {
+  if (T <= 0 || k <= 0 || E <= 0 || hidden <= 0 || inter <= 0) return false;
+  if (hidden % 64 || inter % 64) return false;
+  if ((long long)T * k > MOE_MAX_PAIRS) return false;
+  return true;
+}
+
+bool shape_supported(int T, int k, int E, int hidden, int inter) {
+  return E <= MOE_MAX_EXPERTS && hidden <= 4096 && inter <= MOE_MAX_DIM;
+}
+
+struct WsLayout {
+  size_t num_unique, unique, offsets, pair_list, h, total;
+};
+
+WsLayout ws_layout(int T, int k, int E, int inter) {
+  const size_t P = (size_t)T * k;
+  const size_t m = P < (size_t)E ? P : (size_t)E;
+  WsLayout w;
+  w.num_unique = 0;
+  w.unique = 16;
+  w.offsets = align_up(w.unique + 4 * m, 16);
+  w.pair_list = align_up(w.offsets + 4 * (m + 1), 16);
+  w.h = align_up(w.pair_list + 4 * P, 256);
+  w.total = align_up(w.h + 2 * P * (size_t)inter, 256);
+  return w;
+}
+
+int next_pow2(int v) {
+  int p = 1;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+int gemv_ncw(int hidden) { return (hidden / 32 + 31) / 32; }
+int gemv_ncw3(int inter) { return next_pow2((inter / 32 + 31) / 32); }
+
+// Output rows per CTA of the down kernel: about one CTA per SM, a multiple of the
+// row count that keeps 1-D copies of scale/bias rows 16-byte aligned.
+int gemv_rows_per_cta(int hidden, int inter, int sms) {
+  const int sb_row = inter / 32;  // bytes of scales (or biases) per row
+  int g = 16;
+  for (int a = sb_row, b = 16; b;) {  // gcd(sb_row, 16)
+    const int t = a % b;
+    a = b;
+    b = t;
+    g = a;
+  }
+  const int gran = 16 / g;
+  const int cap = (kConsWarps / gemv_ncw3(inter)) * kRowsPerWarp3;
+  int rows = (hidden + sms - 1) / sms;
+  rows = (rows + gran - 1) / gran * gran;
+  if (rows > cap) rows = cap / gran * gran;
+  if (rows < gran) rows = gran;
+  return rows;
+}
+
+int select_path(int T, int k, int E, int hidden, int inter) {
+  if (!shape_ok(T, k, E, hidden, inter) || !shape_supported(T, k, E, hidden, inter)) return 0;
+  if (T <= kGemvMaxT && T * k <= kGemvMaxPairs) return 1;
+  return 0;  // the grouped tensor-core path is not available in this build
+}
+
+cudaError_t launch_gemv(const uint16_t* x, const int32_t* idx, const float* w, const uint32_t* gq,
+                        const uint16_t* gs, const uint16_t* gb, const uint32_t* uq,
+                        const uint16_t* us, const uint16_t* ub, const uint32_t* dq,
+                        const uint16_t* ds, const uint16_t* db, int T, int k, int E, int H, int I,
+                        uint16_t* out, unsigned char* ws, const DeviceInfo& d, cudaStream_t st,
+                        moe_status* why) {
+  const WsLayout wl = ws_layout(T, k, E, I);
+  const int P = T * k;
+  GateUpArgs ga;
+  ga.x = x;
+  ga.idx = idx;
+  ga.gq = gq;
+  ga.gs = gs;
+  ga.gb = gb;
+  ga.uq = uq;
+  ga.us = us;
+  ga.ub = ub;
+  ga.h = reinterpret_cast<uint16_t*>(ws + wl.h);
+  ga.ug = UnionGlobal{nullptr, nullptr, nullptr, nullptr};
+  ga.ex_u = reinterpret_cast<int*>(ws + wl.num_unique);
+  ga.ex_unique = reinterpret_cast<int*>(ws + wl.unique);
+  ga.ex_offsets = reinterpret_cast<int*>(ws + wl.offsets);
+  ga.ex_pair_list = reinterpret_cast<int*>(ws + wl.pair_list);
+  ga.T = T;
+  ga.k = k;
+  ga.E = E;
+  ga.H = H;
+  ga.I = I;
+  ga.ncw = gemv_ncw(H);
+  ga.wait_prior = 1;
+  const K2Layout L2 = k2_layout(H, E, P, ga.ncw);
+
+  DownArgs da;
+  da.idx = idx;
+  da.w = w;
+  da.dq = dq;
+  da.ds = ds;
+  da.db = db;
+  da.h = ga.h;
+  da.out = out;
+  da.ug = ga.ug;
+  da.T = T;
+  da.k = k;
+  da.E = E;
+  da.H = H;
+  da.I = I;
+  da.ncw3 = gemv_ncw3(I);
+  da.rows_per_cta = gemv_rows_per_cta(H, I, d.sms);
+  const K3Layout L3 = k3_layout(I, E, P, T, da.ncw3, da.rows_per_cta);
+  if (L2.total > (size_t)d.smem_optin || L3.total > (size_t)d.smem_optin) {
+    *why = MOE_ERR_UNSUPPORTED;
+    return cudaSuccess;
+  }
+
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+
+  cudaLaunchConfig_t c2 = {};
+  c2.gridDim = dim3(d.sms);
+  c2.blockDim = dim3(32 * (1 + 2 * ga.ncw));
+  c2.dynamicSmemBytes = L2.total;
+  c2.stream = st;
+  c2.attrs = attr;
+  c2.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&c2, gate_up_kernel, ga);
+  if (e != cudaSuccess) return e;
+
+  cudaLaunchConfig_t c3 = {};
+  c3.gridDim = dim3((H + da.rows_per_cta - 1) / da.rows_per_cta);
+  c3.blockDim = dim3(kThreads);
+  c3.dynamicSmemBytes = L3.total;
+  c3.stream = st;
+  c3.attrs = attr;
+  c3.numAttrs = 1;
+  return cudaLaunchKernelEx(&c3, down_combine_kernel, da);
+}
+
+struct OwnedWorkspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+OwnedWorkspace g_ws[kMaxDevices];
+
+}  // namespace
+}  // namespace qeg
+
+using namespace qeg;
+
+extern "C" {
+
+const char* moe_status_str(int s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE_INDEX: return "MOE_ERR_DEVICE_INDEX";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    default: return "MOE_ERR_UNKNOWN";
+  }
+}
+
+size_t moe_workspace_size(int T, int k, int E, int hidden, int inter) {
+  if (!shape_ok(T, k, E, hidden, inter)) return 0;
+  return ws_layout(T, k, E, inter).total;
+}
+
+moe_status moe_workspace_layout(int T, int k, int E, int hidden, int inter, size_t out[6]) {
+  if (!out || !shape_ok(T, k, E, hidden, inter)) return MOE_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(T, k, E, inter);
+  out[0] = w.num_unique;
+  out[1] = w.unique;
+  out[2] = w.offsets;
+  out[3] = w.pair_list;
+  out[4] = w.h;
+  out[5] = w.total;
+  return MOE_OK;
+}
+
+int moe_select_path(int T, int k, int E, int hidden, int inter) {
+  return select_path(T, k, E, hidden, inter);
+}
+
+moe_status moe_route_union(const int32_t* topk_idx, int T, int k, int E, int32_t* unique,
+                           int32_t* offsets, int32_t* pair_list, int32_t* num_unique,
+                           void* stream) {
+  if (!topk_idx || !unique || !offsets || !pair_list || !num_unique) return MOE_ERR_INVALID_ARG;
+  if (T <= 0 || k <= 0 || E <= 0) return MOE_ERR_INVALID_ARG;
+  if ((long long)T * k > MOE_MAX_PAIRS || E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  if (!aligned(topk_idx, 4) || !aligned(unique, 4) || !aligned(offsets, 4) ||
+      !aligned(pair_list, 4) || !aligned(num_unique, 4))
+    return MOE_ERR_UNSUPPORTED;
+  DeviceInfo* d = nullptr;
+  if (moe_status s = device_info(&d)) return s;
+  const size_t smem = route_union_smem_bytes(E);
+  if (smem > (size_t)d->smem_optin) return MOE_ERR_UNSUPPORTED;
+  route_union_kernel<<<1, 32 * kUnionWarps, smem, (cudaStream_t)stream>>>(
+      topk_idx, T * k, E, unique, offsets, pair_list, num_unique);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_switchglu_forward_ws(const uint16_t* x, const int32_t* topk_idx,
+                                    const float* topk_w, const uint32_t* wg_q,
+                                    const uint16_t* wg_s, const uint16_t* wg_b,
+                                    const uint32_t* wu_q, const uint16_t* wu_s,
+                                    const uint16_t* wu_b, const uint32_t* wd_q,
+                                    const uint16_t* wd_s, const uint16_t* wd_b, int T, int k,
+                                    int E, int hidden, int inter, uint16_t* out, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  if (!x || !topk_idx || !topk_w || !wg_q || !wg_s || !wg_b || !wu_q || !wu_s || !wu_b ||
+      !wd_q || !wd_s || !wd_b || !out || !workspace)
+    return MOE_ERR_INVALID_ARG;
+  if (!shape_ok(T, k, E, hidden, inter)) return MOE_ERR_INVALID_ARG;
+  const void* a16[] = {x, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q, wd_s, wd_b, out, workspace};
+  for (const void* p : a16)
+    if (!aligned(p, 16)) return MOE_ERR_UNSUPPORTED;
+  if (!aligned(topk_idx, 4) || !aligned(topk_w, 4)) return MOE_ERR_UNSUPPORTED;
+  const int path = select_path(T, k, E, hidden, inter);
+  if (path == 0) return MOE_ERR_UNSUPPORTED;
+  if (workspace_bytes < ws_layout(T, k, E, inter).total) return MOE_ERR_WORKSPACE;
+  DeviceInfo* d = nullptr;
+  if (moe_status s = device_info(&d)) return s;
+  moe_status why = MOE_OK;
+  const cudaError_t e = launch_gemv(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q,
+                                    wd_s, wd_b, T, k, E, hidden, inter, out,
+                                    static_cast<unsigned char*>(workspace), *d,
+                                    (cudaStream_t)stream, &why);
+  if (why != MOE_OK) return why;
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_switchglu_forward(const uint16_t* x, const int32_t* topk_idx, const float* topk_w,
+                                 const uint32_t* wg_q, const uint16_t* wg_s,
+                                 const uint16_t* wg_b, const uint32_t* wu_q,
+                                 const uint16_t* wu_s, const uint16_t* wu_b,
+                                 const uint32_t* wd_q, const uint16_t* wd_s,
+                                 const uint16_t* wd_b, int T, int k, int E, int hidden,
+                                 int inter, uint16_t* out, void* stream) {
+  if (!shape_ok(T, k, E, hidden, inter)) return MOE_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  const size_t need = ws_layout(T, k, E, inter).total;
+  OwnedWorkspace& w = g_ws[dev];
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (w.bytes < need) {
+      cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+      if (cudaStreamIsCapturing((cudaStream_t)stream, &cs) != cudaSuccess) return MOE_ERR_CUDA;
+      if (cs != cudaStreamCaptureStatusNone) return MOE_ERR_WORKSPACE;
+      // The old buffer may still be in use by queued work on some stream.
+      if (w.ptr) {
+        if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+        cudaFree(w.ptr);
+        w.ptr = nullptr;
+        w.bytes = 0;
+      }
+      if (cudaMalloc(&w.ptr, need) != cudaSuccess) return MOE_ERR_CUDA;
+      w.bytes = need;
+    }
+  }
+  return moe_switchglu_forward_ws(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q,
+                                  wd_s, wd_b, T, k, E, hidden, inter, out, w.ptr, w.bytes, stream);
+}
+
+moe_status moe_read_device_status(void* stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (word) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  if (word & kErrTimeout) return MOE_ERR_TIMEOUT;
+  if (word & kErrExpertIndex) return MOE_ERR_DEVICE_INDEX;
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,54 @@
+"""Helpers for the GPU tests: upload seeded layers and compare against the oracle."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import quantized_expert_gather_b200 as qeg
+
+# Parity bar for the bf16 layer output (the rel-L2 bound of the target; the
+# max-abs bound is taken on the unit-RMS scale of the reference).
+REL_L2_TOL = 5e-3
+MAX_ABS_TOL = 3e-2
+
+
+def to_dev_bank(L, device="cuda") -> qeg.QuantBank:
+    """Upload a host bank (tests.layers.Layer.bank) as a QuantBank of E experts."""
+    t = {}
+    for name, key in (("gate", "wg"), ("up", "wu"), ("down", "wd")):
+        q, s, b = L.bank[name]
+        t[key + "_q"] = torch.from_numpy(q.view(np.int32)).to(device)
+        t[key + "_s"] = torch.from_numpy(s.view(np.int16)).to(device).view(torch.bfloat16)
+        t[key + "_b"] = torch.from_numpy(b.view(np.int16)).to(device).view(torch.bfloat16)
+    return qeg.QuantBank(**t)
+
+
+def to_dev_inputs(L, device="cuda"):
+    x = torch.from_numpy(L.x.view(np.int16)).to(device).view(torch.bfloat16)
+    idx = torch.from_numpy(L.idx).to(device)
+    w = torch.from_numpy(L.w).to(device)
+    return x, idx, w
+
+
+def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def parity_errors(out: np.ndarray, ref: np.ndarray):
+    """(relative L2 error, max-abs error over rms(ref), raw max-abs error)."""
+    diff = out - ref
+    rms = float(np.sqrt(np.mean(ref ** 2))) if ref.size else 0.0
+    rel = float(np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300))
+    mx = float(np.abs(diff).max()) if diff.size else 0.0
+    return rel, (mx / rms if rms > 0 else mx), mx
+
+
+def assert_parity(out: np.ndarray, ref: np.ndarray, what: str = ""):
+    if not np.any(ref):
+        assert not np.any(out), f"{what}: expected an all-zero output"
+        return
+    rel, mxn, mx = parity_errors(out, ref)
+    assert np.isfinite(out).all(), f"{what}: non-finite output"
+    assert rel <= REL_L2_TOL and mxn <= MAX_ABS_TOL, (
+        f"{what}: rel-L2 {rel:.3e} (tol {REL_L2_TOL}), max-abs/rms {mxn:.3e} (tol {MAX_ABS_TOL}),"
+        f" raw max-abs {mx:.3e}")

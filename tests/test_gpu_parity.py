@@ -1,0 +1,248 @@
+"""Parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Integer outputs (route-union arrays) must match bit for bit; the bf16 layer
+output must be within rel-L2 5e-3 and max-abs/rms(ref) 3e-2 of the oracle on the
+same seeded inputs.  Shapes span several row blocks and a ragged tail; the
+full-size layers are the shapes the pages measure (GLM-5.3-Flash-shaped
+E=288 top-8 4096/2048; the E=256 verify pair and verify windows).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantized_expert_gather_b200 as qeg
+import synth
+from tests.gpu_util import assert_parity, bf16_to_f64, to_dev_bank, to_dev_inputs
+from tests.layers import make_layer, tiny_layer
+
+pytestmark = pytest.mark.gpu
+
+
+def run_forward(L, ws=False):
+    bank = to_dev_bank(L)
+    x, idx, w = to_dev_inputs(L)
+    if ws:
+        nbytes = qeg.moe_workspace_size(L.T, L.k, L.E, L.H, L.I)
+        work = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+        out = qeg.moe_switchglu_forward_ws(x, idx, w, bank, work)
+    else:
+        out = qeg.moe_switchglu_forward(x, idx, w, bank)
+    torch.cuda.synchronize()
+    return out, (bank, x, idx, w)
+
+
+def check_layer(L, what, tokens=None):
+    out, _ = run_forward(L)
+    assert qeg.moe_read_device_status() == qeg.MOE_OK
+    ref = oracle.switchglu(L.x, L.idx, L.w, L.bank, L.E, tokens=tokens)
+    got = bf16_to_f64(out)
+    if tokens is not None:
+        got, ref = got[tokens], ref[tokens]
+    assert_parity(got, ref, what)
+    return out
+
+
+# ------------------------------------------------------------- route-union ---
+@pytest.mark.parametrize("seed", range(8))
+def test_route_union_bit_exact_random(seed):
+    rng = np.random.default_rng(100 + seed)
+    T, k = int(rng.integers(1, 40)), int(rng.integers(1, 9))
+    E = int(rng.integers(1, 1025))
+    idx = rng.integers(0, E, size=(T, k)).astype(np.int32)
+    uq, of, pl, nu = qeg.moe_route_union(torch.from_numpy(idx).cuda(), E)
+    u_ref, o_ref, p_ref, n_ref, _ = oracle.route_union(idx, E)
+    n = int(nu.item())
+    assert n == n_ref
+    assert np.array_equal(uq.cpu().numpy()[:n], u_ref)
+    assert np.array_equal(of.cpu().numpy()[:n + 1], o_ref)
+    assert np.array_equal(pl.cpu().numpy(), p_ref)
+    assert qeg.moe_read_device_status() == qeg.MOE_OK
+
+
+@pytest.mark.parametrize("T,k,E", [(1, 8, 288), (4, 8, 288), (16, 8, 256), (512, 8, 256),
+                                   (2048, 8, 256), (8192, 8, 1024), (3, 1, 1)])
+def test_route_union_bit_exact_sizes(T, k, E):
+    idx, _ = synth.route_uniform(T, E, k, seed=T * 7 + E) if k <= E else (None, None)
+    if idx is None:
+        idx = np.zeros((T, k), np.int32)
+    uq, of, pl, nu = qeg.moe_route_union(torch.from_numpy(idx).cuda(), E)
+    u_ref, o_ref, p_ref, n_ref, _ = oracle.route_union(idx, E)
+    n = int(nu.item())
+    assert n == n_ref and np.array_equal(uq.cpu().numpy()[:n], u_ref)
+    assert np.array_equal(of.cpu().numpy()[:n + 1], o_ref)
+    assert np.array_equal(pl.cpu().numpy(), p_ref)
+
+
+def test_route_union_extremes_and_invalid_ids():
+    T, k, E = 16, 8, 256
+    for idx in (np.tile(np.arange(8, dtype=np.int32) * 5, (T, 1)),
+                np.arange(T * k, dtype=np.int32).reshape(T, k)):
+        uq, of, pl, nu = qeg.moe_route_union(torch.from_numpy(idx).cuda(), E)
+        u_ref, o_ref, p_ref, n_ref, _ = oracle.route_union(idx, E)
+        assert int(nu.item()) == n_ref and np.array_equal(pl.cpu().numpy(), p_ref)
+    assert qeg.moe_read_device_status() == qeg.MOE_OK
+    bad = np.array([[3, 300, 3], [-1, 7, 255]], np.int32)
+    uq, of, pl, nu = qeg.moe_route_union(torch.from_numpy(bad).cuda(), E)
+    u_ref, o_ref, p_ref, n_ref, nbad = oracle.route_union(bad, E)
+    assert nbad == 2 and int(nu.item()) == n_ref and np.array_equal(pl.cpu().numpy(), p_ref)
+    assert qeg.moe_read_device_status() == qeg.MOE_ERR_DEVICE_INDEX
+    assert qeg.moe_read_device_status() == qeg.MOE_OK  # cleared by the read
+
+
+# ----------------------------------------------------------------- forward ---
+def test_tiny_layer():
+    check_layer(tiny_layer(), "tiny E=16 top-2 256/128 T=2")
+
+
+@pytest.mark.parametrize("cfg", [
+    # T, k, E, H, I, routing
+    (7, 6, 40, 512, 384, "uniform"),     # ragged: several row blocks, odd T
+    (1, 8, 64, 256, 192, "uniform"),
+    (5, 3, 8, 1024, 512, "uniform"),     # heavy sharing: ~2 tokens per expert
+    (16, 8, 256, 512, 256, "markov"),
+    (3, 2, 4, 4096, 128, "uniform"),     # full hidden width, small inter
+    (9, 4, 30, 192, 1088, "uniform"),    # inter > 1024 (two chunk-warps), ragged
+])
+def test_forward_small_shapes(cfg):
+    T, k, E, H, I, routing = cfg
+    L = make_layer(T, k, E, H, I, seed=sum(cfg[:5]), routing=routing)
+    check_layer(L, f"T={T} k={k} E={E} H={H} I={I}")
+
+
+def test_forward_ws_variant_and_union_export():
+    L = make_layer(6, 4, 24, 256, 256, seed=21)
+    out, (bank, x, idx, w) = run_forward(L)
+    nbytes = qeg.moe_workspace_size(L.T, L.k, L.E, L.H, L.I)
+    work = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    out2 = qeg.moe_switchglu_forward_ws(x, idx, w, bank, work)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+    lay = qeg.moe_workspace_layout(L.T, L.k, L.E, L.H, L.I)
+    wsn = work.cpu().numpy()
+    u = int(wsn[lay["num_unique"]:lay["num_unique"] + 4].view(np.int32)[0])
+    u_ref, o_ref, p_ref, n_ref, _ = oracle.route_union(L.idx, L.E)
+    assert u == n_ref
+    assert np.array_equal(wsn[lay["unique"]:lay["unique"] + 4 * u].view(np.int32), u_ref)
+    P = L.T * L.k
+    assert np.array_equal(wsn[lay["pair_list"]:lay["pair_list"] + 4 * P].view(np.int32), p_ref)
+    # h in pair_list order vs the oracle's per-pair h (bf16 values; a flip of one bf16 step
+    # is allowed where fp32 and fp64 sums straddle a rounding boundary)
+    _, h_ref = oracle.switchglu(L.x, L.idx, L.w, L.bank, L.E, want_h=True)
+    h = torch.from_numpy(wsn[lay["h"]:lay["h"] + 2 * P * L.I].view(np.int16).copy()) \
+        .view(torch.bfloat16).float().numpy().reshape(P, L.I).astype(np.float64)
+    h_ref_sorted = h_ref[p_ref[:o_ref[-1]]]
+    step = np.abs(h_ref_sorted) * 2.0 ** -7 + 1e-30
+    assert np.all(np.abs(h[:o_ref[-1]] - h_ref_sorted) <= step * 1.01)
+    assert np.mean(h[:o_ref[-1]] == h_ref_sorted) > 0.97
+
+
+def test_deterministic_bitwise():
+    L = make_layer(8, 8, 64, 1024, 512, seed=31, routing="markov", p=0.5)
+    a, _ = run_forward(L)
+    b, _ = run_forward(L)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_token_independence():
+    L = make_layer(4, 8, 32, 512, 256, seed=41, routing="markov", p=0.6)
+    full, _ = run_forward(L)
+    for t in range(L.T):
+        one = make_layer(1, 8, 32, 512, 256, seed=41, idx=L.idx[t:t + 1], w=L.w[t:t + 1])
+        one.x = L.x[t:t + 1]
+        one.bank = L.bank
+        o, _ = run_forward(one)
+        assert_parity(bf16_to_f64(o)[0:1], bf16_to_f64(full)[t:t + 1], f"token {t}")
+
+
+def test_duplicate_experts_zero_weights_and_invalid_ids():
+    E = 12
+    idx = np.array([[2, 2, 5], [7, 13, 1], [-4, 3, 3], [0, 1, 2]], np.int32)
+    w = np.array([[0.5, 0.25, 0.25], [0.2, 0.3, 0.5], [1.0, 0.5, 0.5], [0, 0, 0]], np.float32)
+    L = make_layer(4, 3, E, 256, 128, seed=51, idx=idx, w=w)
+    out, _ = run_forward(L)
+    assert qeg.moe_read_device_status() == qeg.MOE_ERR_DEVICE_INDEX
+    ref = oracle.switchglu(L.x, L.idx, L.w, L.bank, E)
+    got = bf16_to_f64(out)
+    assert not np.any(got[3])  # zero router weights -> zero row
+    assert_parity(got, ref, "duplicates / invalid ids")
+
+
+def test_all_invalid_gives_zero_rows():
+    idx = np.full((3, 4), 99, np.int32)
+    L = make_layer(3, 4, 8, 128, 64, seed=52, idx=idx)
+    out, _ = run_forward(L)
+    assert qeg.moe_read_device_status() == qeg.MOE_ERR_DEVICE_INDEX
+    assert not torch.any(out.float() != 0)
+
+
+def test_all_identical_and_disjoint_routing():
+    T, k, E, H, I = 16, 8, 256, 512, 256
+    same = np.tile(np.arange(8, dtype=np.int32) * 9, (T, 1))
+    check_layer(make_layer(T, k, E, H, I, seed=61, idx=same), "all-identical routing")
+    disjoint = np.arange(T * k, dtype=np.int32).reshape(T, k)
+    check_layer(make_layer(T, k, E, H, I, seed=62, idx=disjoint), "disjoint routing")
+
+
+# ---------------------------------------------------------- full-size layers ---
+@pytest.mark.parametrize("T", [1, 4])
+def test_glm_flash_layer(T):
+    """E=288, top-8, hidden 4096, intermediate 2048, uniform routing (the moe_bench.py layer)."""
+    L = make_layer(T, 8, 288, 4096, 2048, seed=2000 + T, routing="uniform")
+    check_layer(L, f"GLM-5.3-Flash-shaped T={T}")
+
+
+@pytest.mark.parametrize("p", [0.03, 0.34, 0.52])
+def test_verify_pair_layer(p):
+    idx, w = synth.route_verify_pair(256, 8, p, seed=3000 + int(p * 100))
+    L = make_layer(2, 8, 256, 4096, 2048, seed=3000 + int(p * 100), idx=idx, w=w)
+    check_layer(L, f"verify pair p={p}")
+
+
+@pytest.mark.parametrize("T", [3, 16])
+def test_verify_window_layer(T):
+    L = make_layer(T, 8, 256, 4096, 2048, seed=4000 + T, routing="markov", p=0.40)
+    check_layer(L, f"verify window T={T}")
+
+
+# ------------------------------------------------------------ generator twin ---
+def test_device_generator_matches_host():
+    E, rows, cols, seed = 5, 64, 512, 77
+    q = torch.zeros((E, rows, cols // 8), dtype=torch.int32, device="cuda")
+    s = torch.zeros((E, rows, cols // 64), dtype=torch.int16, device="cuda")
+    b = torch.zeros_like(s)
+    synth.fill_bank_device(q, s, b, rows, cols, seed, synth.MATRIX_UP)
+    torch.cuda.synchronize()
+    qh, sh, bh = synth.fill_bank_host(E, rows, cols, seed, synth.MATRIX_UP)
+    assert np.array_equal(q.cpu().numpy().view(np.uint32), qh)
+    assert np.array_equal(s.cpu().numpy().view(np.uint16), sh)
+    assert np.array_equal(b.cpu().numpy().view(np.uint16), bh)
+
+
+# ------------------------------------------------------------ argument errors ---
+def test_rejected_arguments_launch_nothing():
+    L = make_layer(2, 2, 4, 128, 64, seed=71)
+    bank = to_dev_bank(L)
+    x, idx, w = to_dev_inputs(L)
+    # misaligned activation pointer (2 bytes into a real allocation)
+    xbig = torch.zeros(2 * 128 + 8, dtype=torch.bfloat16, device="cuda")
+    xmis = xbig[1:1 + 2 * 128].view(2, 128)
+    assert qeg.moe_switchglu_forward(xmis, idx, w, bank, check=False) is not None
+    st = qeg._lib.moe_switchglu_forward(xmis.data_ptr(), idx.data_ptr(), w.data_ptr(),
+                                        *bank.ptrs(), 2, 2, 4, 128, 64,
+                                        torch.empty(2, 128, dtype=torch.bfloat16,
+                                                    device="cuda").data_ptr(),
+                                        torch.cuda.current_stream().cuda_stream)
+    assert st == qeg.MOE_ERR_UNSUPPORTED
+    # workspace too small
+    work = torch.zeros(64, dtype=torch.uint8, device="cuda")
+    with pytest.raises(qeg.MoeError) as ei:
+        qeg.moe_switchglu_forward_ws(x, idx, w, bank, work)
+    assert ei.value.status == qeg.MOE_ERR_WORKSPACE
+    # hidden not a multiple of 64 is an invalid shape, rejected before any launch
+    st = qeg._lib.moe_switchglu_forward(x.data_ptr(), idx.data_ptr(), w.data_ptr(), *bank.ptrs(),
+                                        2, 2, 4, 96, 64, x.data_ptr(),
+                                        torch.cuda.current_stream().cuda_stream)
+    assert st == qeg.MOE_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert qeg.moe_read_device_status() == qeg.MOE_OK

@@ -1,0 +1,101 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point the
+header declares, and its pure host logic (path selection, workspace sizing,
+argument validation before any launch) behaves as documented.  No kernel runs."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+import quantized_expert_gather_b200 as qeg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_qeg.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("moe_route_union", "moe_switchglu_forward", "moe_switchglu_forward_ws",
+              "moe_workspace_size", "moe_read_device_status", "moe_status_str",
+              "moe_select_path", "moe_workspace_layout"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", qeg.library_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (moe_\w+)", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    lib = ctypes.CDLL(qeg.library_path())
+    for n in declared_functions():
+        assert hasattr(lib, n)
+
+
+def test_status_strings():
+    assert qeg.moe_status_str(0) == "MOE_OK"
+    assert qeg.moe_status_str(4) == "MOE_ERR_DEVICE_INDEX"
+    assert qeg.moe_status_str(99) == "MOE_ERR_UNKNOWN"
+
+
+def test_path_selection_without_launch():
+    # small windows -> expert-major GEMV path
+    for T in (1, 2, 4, 16, 64, 256):
+        assert qeg.moe_select_path(T, 8, 256, 4096, 2048) == 1
+    assert qeg.moe_select_path(2, 2, 16, 256, 128) == 1
+    # invalid shapes
+    assert qeg.moe_select_path(0, 8, 256, 4096, 2048) == 0
+    assert qeg.moe_select_path(4, 8, 256, 4000, 2048) == 0
+    assert qeg.moe_select_path(4, 8, 256, 4096, 2000) == 0
+    assert qeg.moe_select_path(4, 8, 2048, 4096, 2048) == 0  # too many experts
+
+
+def test_workspace_size_and_layout():
+    T, k, E, H, I = 4, 8, 288, 4096, 2048
+    n = qeg.moe_workspace_size(T, k, E, H, I)
+    lay = qeg.moe_workspace_layout(T, k, E, H, I)
+    assert lay["total"] == n
+    assert lay["h"] % 256 == 0 and lay["h"] + 2 * T * k * I <= n
+    assert lay["unique"] % 16 == 0 and lay["offsets"] % 16 == 0 and lay["pair_list"] % 16 == 0
+    assert qeg.moe_workspace_size(0, 8, E, H, I) == 0
+    with pytest.raises(qeg.MoeError):
+        qeg.moe_workspace_layout(4, 8, E, 100, I)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="uses fake pointers; host-only check")
+def test_validation_rejects_before_touching_memory():
+    lib = qeg._lib
+    fake = 0x10000  # never dereferenced: every call below must be rejected first
+    ptrs = [fake] * 12
+    # null pointer
+    assert lib.moe_switchglu_forward_ws(*([None] + ptrs[1:]), 2, 2, 4, 128, 64, fake, fake,
+                                        1 << 20, None) == qeg.MOE_ERR_INVALID_ARG
+    # hidden not a multiple of 64
+    assert lib.moe_switchglu_forward_ws(*ptrs, 2, 2, 4, 100, 64, fake, fake, 1 << 20,
+                                        None) == qeg.MOE_ERR_INVALID_ARG
+    # non-positive sizes
+    assert lib.moe_switchglu_forward_ws(*ptrs, 0, 2, 4, 128, 64, fake, fake, 1 << 20,
+                                        None) == qeg.MOE_ERR_INVALID_ARG
+    # misaligned pointer
+    bad = list(ptrs)
+    bad[0] = fake + 2
+    assert lib.moe_switchglu_forward_ws(*bad, 2, 2, 4, 128, 64, fake, fake, 1 << 20,
+                                        None) == qeg.MOE_ERR_UNSUPPORTED
+    # workspace too small
+    assert lib.moe_switchglu_forward_ws(*ptrs, 2, 2, 4, 128, 64, fake, fake, 16,
+                                        None) == qeg.MOE_ERR_WORKSPACE
+    # too many experts / pairs
+    assert lib.moe_switchglu_forward_ws(*ptrs, 2, 2, 5000, 128, 64, fake, fake, 1 << 20,
+                                        None) == qeg.MOE_ERR_UNSUPPORTED
+    assert lib.moe_route_union(fake, 70000, 1, 8, fake, fake, fake, fake,
+                               None) == qeg.MOE_ERR_UNSUPPORTED
+    assert lib.moe_route_union(None, 2, 2, 8, fake, fake, fake, fake,
+                               None) == qeg.MOE_ERR_INVALID_ARG
