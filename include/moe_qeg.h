@@ -63,13 +63,18 @@ typedef enum {
 } moe_status;
 
 /* Supported range (checked on the host; violations return MOE_ERR_UNSUPPORTED):
- * hidden and inter multiples of 64 and <= 8192; E <= 1024; T*k <= 65536. */
+ * hidden and inter multiples of 64, hidden <= 4096, inter <= 8192; E <= 1024;
+ * T*k <= 65536. */
 #define MOE_MAX_EXPERTS 1024
 #define MOE_MAX_DIM 8192
 #define MOE_MAX_PAIRS 65536
 
 /* Human-readable name of a status code (static string). */
 const char* moe_status_str(int status);
+
+/* The CUDA runtime's message for the most recent MOE_ERR_CUDA returned on the
+ * calling thread ("no error" if none); a static string. */
+const char* moe_last_error(void);
 
 /* Bytes of workspace that moe_switchglu_forward_ws needs for this shape
  * (0 on invalid arguments).  The workspace holds the route-union arrays and

@@ -19,7 +19,8 @@ from ._build import SO, build as build_library, needs_build
 
 __all__ = ["MoeError", "MOE_OK", "moe_status_str", "moe_workspace_size", "moe_workspace_layout",
            "moe_select_path", "moe_route_union", "moe_switchglu_forward",
-           "moe_switchglu_forward_ws", "moe_read_device_status", "library_path", "QuantBank"]
+           "moe_switchglu_forward_ws", "moe_read_device_status", "moe_last_error", "library_path",
+           "QuantBank"]
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = 1
@@ -32,7 +33,8 @@ MOE_ERR_WORKSPACE = 6
 
 class MoeError(RuntimeError):
     def __init__(self, status: int, where: str):
-        super().__init__(f"{where}: {moe_status_str(status)} ({status})")
+        detail = f" [{moe_last_error()}]" if status == MOE_ERR_CUDA else ""
+        super().__init__(f"{where}: {moe_status_str(status)} ({status}){detail}")
         self.status = status
 
 
@@ -43,6 +45,8 @@ def _load():
     vp, ci, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     lib.moe_status_str.restype = ctypes.c_char_p
     lib.moe_status_str.argtypes = [ci]
+    lib.moe_last_error.restype = ctypes.c_char_p
+    lib.moe_last_error.argtypes = []
     lib.moe_workspace_size.restype = sz
     lib.moe_workspace_size.argtypes = [ci] * 5
     lib.moe_workspace_layout.restype = ci
@@ -69,6 +73,10 @@ def library_path() -> str:
 
 def moe_status_str(status: int) -> str:
     return _lib.moe_status_str(int(status)).decode()
+
+
+def moe_last_error() -> str:
+    return _lib.moe_last_error().decode()
 
 
 def _check(status: int, where: str, check: bool) -> int:

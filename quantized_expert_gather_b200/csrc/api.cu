@@ -21,29 +21,45 @@ struct DeviceInfo {
   bool ready = false;
   int sms = 0;
   int smem_optin = 0;
+  int dyn_smem[3] = {0, 0, 0};  // dynamic shared memory limit: gate_up, down, route_union
 };
 
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
+thread_local const char* g_last_error = "no error";
+
+moe_status cuda_fail(cudaError_t e) {
+  g_last_error = cudaGetErrorString(e);
+  return MOE_ERR_CUDA;
+}
 
 // Per-device state: SM count, shared-memory limit, kernel attributes set once.
 moe_status device_info(DeviceInfo** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  const cudaError_t ge = cudaGetDevice(&dev);
+  if (ge != cudaSuccess) return cuda_fail(ge);
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceInfo& d = g_dev[dev];
   if (!d.ready) {
-    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
-            cudaSuccess)
-      return MOE_ERR_CUDA;
-    if (cudaFuncSetAttribute(gate_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             d.smem_optin) != cudaSuccess ||
-        cudaFuncSetAttribute(down_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             d.smem_optin) != cudaSuccess ||
-        cudaFuncSetAttribute(route_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             d.smem_optin) != cudaSuccess)
-      return MOE_ERR_CUDA;
+    cudaError_t e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+      e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    // dynamic + static shared memory may not exceed the opt-in limit
+    const void* kernels[3] = {reinterpret_cast<const void*>(gate_up_kernel),
+                              reinterpret_cast<const void*>(down_combine_kernel),
+                              reinterpret_cast<const void*>(route_union_kernel)};
+    for (int i = 0; i < 3; ++i) {
+      cudaFuncAttributes fa;
+      cudaError_t e = cudaFuncGetAttributes(&fa, kernels[i]);
+      if (e == cudaSuccess) {
+        d.dyn_smem[i] = d.smem_optin - static_cast<int>(fa.sharedSizeBytes);
+        e = cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 d.dyn_smem[i]);
+      }
+      if (e != cudaSuccess) return cuda_fail(e);
+    }
     d.ready = true;
   }
   *out = &d;
@@ -164,7 +180,7 @@ cudaError_t launch_gemv(const uint16_t* x, const int32_t* idx, const float* w, c
   da.ncw3 = gemv_ncw3(I);
   da.rows_per_cta = gemv_rows_per_cta(H, I, d.sms);
   const K3Layout L3 = k3_layout(I, E, P, T, da.ncw3, da.rows_per_cta);
-  if (L2.total > (size_t)d.smem_optin || L3.total > (size_t)d.smem_optin) {
+  if (L2.total > (size_t)d.dyn_smem[0] || L3.total > (size_t)d.dyn_smem[1]) {
     *why = MOE_ERR_UNSUPPORTED;
     return cudaSuccess;
   }
@@ -175,7 +191,7 @@ cudaError_t launch_gemv(const uint16_t* x, const int32_t* idx, const float* w, c
 
   cudaLaunchConfig_t c2 = {};
   c2.gridDim = dim3(d.sms);
-  c2.blockDim = dim3(32 * (1 + 2 * ga.ncw));
+  c2.blockDim = dim3(32 * 2 * ga.ncw);
   c2.dynamicSmemBytes = L2.total;
   c2.stream = st;
   c2.attrs = attr;
@@ -205,6 +221,8 @@ OwnedWorkspace g_ws[kMaxDevices];
 using namespace qeg;
 
 extern "C" {
+
+const char* moe_last_error(void) { return g_last_error; }
 
 const char* moe_status_str(int s) {
   switch (s) {
@@ -252,10 +270,11 @@ moe_status moe_route_union(const int32_t* topk_idx, int T, int k, int E, int32_t
   DeviceInfo* d = nullptr;
   if (moe_status s = device_info(&d)) return s;
   const size_t smem = route_union_smem_bytes(E);
-  if (smem > (size_t)d->smem_optin) return MOE_ERR_UNSUPPORTED;
+  if (smem > (size_t)d->dyn_smem[2]) return MOE_ERR_UNSUPPORTED;
   route_union_kernel<<<1, 32 * kUnionWarps, smem, (cudaStream_t)stream>>>(
       topk_idx, T * k, E, unique, offsets, pair_list, num_unique);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
 
 moe_status moe_switchglu_forward_ws(const uint16_t* x, const int32_t* topk_idx,
@@ -285,7 +304,7 @@ moe_status moe_switchglu_forward_ws(const uint16_t* x, const int32_t* topk_idx,
                                     static_cast<unsigned char*>(workspace), *d,
                                     (cudaStream_t)stream, &why);
   if (why != MOE_OK) return why;
-  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
 
 moe_status moe_switchglu_forward(const uint16_t* x, const int32_t* topk_idx, const float* topk_w,
@@ -297,23 +316,31 @@ moe_status moe_switchglu_forward(const uint16_t* x, const int32_t* topk_idx, con
                                  int inter, uint16_t* out, void* stream) {
   if (!shape_ok(T, k, E, hidden, inter)) return MOE_ERR_INVALID_ARG;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  const cudaError_t ge = cudaGetDevice(&dev);
+  if (ge != cudaSuccess) return cuda_fail(ge);
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
   const size_t need = ws_layout(T, k, E, inter).total;
   OwnedWorkspace& w = g_ws[dev];
   {
     std::lock_guard<std::mutex> lock(g_mu);
     if (w.bytes < need) {
       cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-      if (cudaStreamIsCapturing((cudaStream_t)stream, &cs) != cudaSuccess) return MOE_ERR_CUDA;
+      const cudaError_t ce = cudaStreamIsCapturing((cudaStream_t)stream, &cs);
+      if (ce != cudaSuccess) return cuda_fail(ce);
       if (cs != cudaStreamCaptureStatusNone) return MOE_ERR_WORKSPACE;
       // The old buffer may still be in use by queued work on some stream.
       if (w.ptr) {
-        if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+        const cudaError_t se = cudaDeviceSynchronize();
+        if (se != cudaSuccess) return cuda_fail(se);
         cudaFree(w.ptr);
         w.ptr = nullptr;
         w.bytes = 0;
       }
-      if (cudaMalloc(&w.ptr, need) != cudaSuccess) return MOE_ERR_CUDA;
+      const cudaError_t me = cudaMalloc(&w.ptr, need);
+      if (me != cudaSuccess) {
+        w.ptr = nullptr;
+        return cuda_fail(me);
+      }
       w.bytes = need;
     }
   }
@@ -322,12 +349,15 @@ moe_status moe_switchglu_forward(const uint16_t* x, const int32_t* topk_idx, con
 }
 
 moe_status moe_read_device_status(void* stream) {
-  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e);
   unsigned int word = 0;
-  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return MOE_ERR_CUDA;
+  e = cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail(e);
   if (word) {
     const unsigned int zero = 0;
-    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return MOE_ERR_CUDA;
+    e = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e);
   }
   if (word & kErrTimeout) return MOE_ERR_TIMEOUT;
   if (word & kErrExpertIndex) return MOE_ERR_DEVICE_INDEX;

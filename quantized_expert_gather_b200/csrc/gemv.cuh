@@ -2,8 +2,12 @@
 //
 // K2 (gate_up_kernel): for every distinct routed expert e, stream Wg[e] and
 //   Wu[e] from HBM once, in blocks of kRows rows, through a kStages-deep ring of
-//   shared-memory buffers filled by 1-D bulk copies (one producer thread,
-//   mbarrier completion).  Consumer warps hold the activations of the expert's
+//   shared-memory buffers filled by 1-D bulk copies (mbarrier completion).
+//   Thread 0 issues the copies: the first kStages blocks up front, then block
+//   j + kStages right after the barrier that ends block j, when no warp reads
+//   its slot any more.  Every warp computes; blocks have 8 warps at most, so
+//   each SM sub-partition holds two and a thread may use up to 255 registers.
+//   The warps hold the activations of the expert's
 //   tokens in registers and compute, per row and token,
 //     G = sum_c (s*q_c + b) x_c = s * sum_c q_c x_c + b * sum_c x_c
 //   (group-sum factorisation over the 32 columns a lane owns, one group), then
@@ -32,8 +36,8 @@ constexpr int kRows = 8;       // K2: rows of gate and of up per stage
 constexpr int kStages2 = 4;    // K2: ring depth
 constexpr int kStages3 = 5;    // K3: ring depth
 constexpr int kNT = 4;         // tokens (pairs) per register pass
-constexpr int kConsWarps = 8;  // consumer warps per CTA (K2 and K3)
-constexpr int kThreads = 32 * (1 + kConsWarps);
+constexpr int kConsWarps = 8;  // warps per CTA (K2 at hidden 4096, K3); all compute
+constexpr int kThreads = 32 * kConsWarps;
 constexpr int kRowsPerWarp3 = 8;  // K3: output rows per consumer warp
 constexpr int kMaxRows3 = kConsWarps * kRowsPerWarp3;  // K3: output rows per CTA at most
 constexpr int kGemvMaxT = 256;
@@ -68,7 +72,7 @@ __host__ __device__ inline K2Layout k2_layout(int H, int E, int P, int ncw) {
   L.sb_bytes = kRows * H / 32;
   L.mat_bytes = L.q_bytes + 2 * L.sb_bytes;
   L.stage_bytes = 2 * L.mat_bytes;
-  L.bars = 0;                                   // full[kStages2], empty[kStages2]
+  L.bars = 0;  // (barriers live in static shared memory)
   L.stages = 128;
   L.part = L.stages + align_up((size_t)kStages2 * L.stage_bytes, 128);
   // partials: [2 buffers][2 matrices][ncw][kRows * kNT] floats
@@ -243,28 +247,24 @@ __device__ __forceinline__ void export_union(const UnionRefs& U, int P, int* g_u
 }
 
 // ------------------------------------------------------------------- K2 ---
-__global__ void __maxnreg__(224) gate_up_kernel(const GateUpArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) gate_up_kernel(const GateUpArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_u;
+  __shared__ __align__(8) uint64_t full[kStages2];
   const int P = a.T * a.k;
   const K2Layout L = k2_layout(a.H, a.E, P, a.ncw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
-  uint64_t* empty = full + kStages2;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_cons_warps = 2 * a.ncw;
+  const int n_threads = 2 * a.ncw * 32;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages2; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], n_cons_warps);
-    }
+    for (int s = 0; s < kStages2; ++s) mbar_init(&full[s], 1);
     fence_barrier_init();
   }
   if (a.wait_prior) grid_dep_wait();
   const UnionRefs U = block_union(a.ug, a.idx, P, a.E, smem, L.us, &s_u);
   __syncthreads();  // barrier init and union visible to every warp
   grid_dep_launch();
-  if (blockIdx.x == 0 && threadIdx.x >= 32 && threadIdx.x < 64 && a.ex_u && !a.ug.num_unique)
+  if (blockIdx.x == 0 && warp == 1 && a.ex_u && !a.ug.num_unique)
     export_union(U, P, a.ex_u, a.ex_unique, a.ex_offsets, a.ex_pair_list);
 
   const int bpe = a.I / kRows;  // row blocks per expert
@@ -273,39 +273,34 @@ __global__ void __maxnreg__(224) gate_up_kernel(const GateUpArgs a) {
   const int blk1 = (int)(nb * (blockIdx.x + 1) / gridDim.x);
   const int nblk = blk1 - blk0;
   const size_t qrow = a.H / 8, srow = a.H / 64;  // words / groups per row
+  uint64_t pol = 0;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      for (int j = 0; j < nblk; ++j) {
-        const int blk = blk0 + j, slot = blk / bpe, row0 = (blk % bpe) * kRows;
-        const int e = U.unique[slot];
-        const int st = j % kStages2;
-        if (j >= kStages2 && !mbar_wait(&empty[st], ((j / kStages2) - 1) & 1)) break;
-        unsigned char* buf = smem + L.stages + (size_t)st * L.stage_bytes;
-        mbar_arrive_expect_tx(&full[st], L.stage_bytes);
-        const size_t r0 = (size_t)e * a.I + row0;
-        bulk_g2s(buf, a.gq + r0 * qrow, L.q_bytes, &full[st], pol);
-        bulk_g2s(buf + L.q_bytes, a.gs + r0 * srow, L.sb_bytes, &full[st], pol);
-        bulk_g2s(buf + L.q_bytes + L.sb_bytes, a.gb + r0 * srow, L.sb_bytes, &full[st], pol);
-        buf += L.mat_bytes;
-        bulk_g2s(buf, a.uq + r0 * qrow, L.q_bytes, &full[st], pol);
-        bulk_g2s(buf + L.q_bytes, a.us + r0 * srow, L.sb_bytes, &full[st], pol);
-        bulk_g2s(buf + L.q_bytes + L.sb_bytes, a.ub + r0 * srow, L.sb_bytes, &full[st], pol);
-      }
-    }
-    return;
+  // thread 0: copy row block j of this CTA's range into ring slot j % kStages2
+  auto issue = [&](int j) {
+    const int blk = blk0 + j, slot = blk / bpe, row0 = (blk % bpe) * kRows;
+    const int st = j % kStages2;
+    unsigned char* buf = smem + L.stages + (size_t)st * L.stage_bytes;
+    const size_t r0 = (size_t)U.unique[slot] * a.I + row0;
+    mbar_arrive_expect_tx(&full[st], L.stage_bytes);
+    bulk_g2s(buf, a.gq + r0 * qrow, L.q_bytes, &full[st], pol);
+    bulk_g2s(buf + L.q_bytes, a.gs + r0 * srow, L.sb_bytes, &full[st], pol);
+    bulk_g2s(buf + L.q_bytes + L.sb_bytes, a.gb + r0 * srow, L.sb_bytes, &full[st], pol);
+    buf += L.mat_bytes;
+    bulk_g2s(buf, a.uq + r0 * qrow, L.q_bytes, &full[st], pol);
+    bulk_g2s(buf + L.q_bytes, a.us + r0 * srow, L.sb_bytes, &full[st], pol);
+    bulk_g2s(buf + L.q_bytes + L.sb_bytes, a.ub + r0 * srow, L.sb_bytes, &full[st], pol);
+  };
+  if (threadIdx.x == 0) {
+    pol = policy_evict_first();
+    for (int j = 0; j < nblk && j < kStages2; ++j) issue(j);
   }
 
-  // ---- consumers ----
-  const int wc = warp - 1;
-  const int m = wc / a.ncw, cw = wc % a.ncw;
+  const int m = warp / a.ncw, cw = warp % a.ncw;  // matrix (0 gate, 1 up), chunk-warp
   const int ch = cw * 32 + lane;
   const bool active = ch < a.H / 32;
   float* part = reinterpret_cast<float*>(smem + L.part);
   const int part_stride = 2 * a.ncw * kRows * kNT;  // one buffer
-  const int n_cons = n_cons_warps * 32;
-  const int ct = threadIdx.x - 32;
+  const int ct = threadIdx.x;
   float xf[kNT][32];
   float xs[kNT];
   int cur_slot = -1, cur_c0 = -1;
@@ -348,15 +343,16 @@ __global__ void __maxnreg__(224) gate_up_kernel(const GateUpArgs a) {
           for (int t = 0; t < kNT; ++t) acc[r * kNT + t] = fmaf(sc, d[t], bi * xs[t]);
         }
       }
-      if (c0 + kNT >= n_e) {  // last pass over this stage: release it
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
-      }
       int vid;
       const float v = warp_reduce_scatter<kRows * kNT>(acc, lane, vid);
       float* pbuf = part + pb * part_stride;
       pbuf[(m * a.ncw + cw) * (kRows * kNT) + vid] = v;  // V == 32: every lane owns one value
-      named_barrier(1, n_cons);
+      named_barrier(1, n_threads);
+      // every warp is past its reads of slot st: refill it with block j + kStages2
+      if (c0 + kNT >= n_e && threadIdx.x == 0 && j + kStages2 < nblk) {
+        fence_proxy_async();
+        issue(j + kStages2);
+      }
       if (ct < kRows * nt) {
         const int r = ct / nt, t = ct % nt;
         float G = 0.f, Uv = 0.f;
@@ -374,25 +370,19 @@ __global__ void __maxnreg__(224) gate_up_kernel(const GateUpArgs a) {
 }
 
 // ------------------------------------------------------------------- K3 ---
-__global__ void __maxnreg__(224) down_combine_kernel(const DownArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) down_combine_kernel(const DownArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_u;
-  __shared__ __align__(8) uint64_t bars[2 * kStages3];
+  __shared__ __align__(8) uint64_t full[kStages3];
   const int P = a.T * a.k;
   const K3Layout L = k3_layout(a.I, a.E, P, a.T, a.ncw3, a.rows_per_cta);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + kStages3;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_cons_warps = kConsWarps;
   const int row_groups = kConsWarps / a.ncw3;
   const int c0row = blockIdx.x * a.rows_per_cta;
   const int nrows = min(a.rows_per_cta, a.H - c0row);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages3; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], n_cons_warps);
-    }
+    for (int s = 0; s < kStages3; ++s) mbar_init(&full[s], 1);
     fence_barrier_init();
   }
   float* acc_out = reinterpret_cast<float*>(smem + L.acc);
@@ -401,99 +391,97 @@ __global__ void __maxnreg__(224) down_combine_kernel(const DownArgs a) {
   // grid (gate+up) started, so it is formed before waiting on that grid.
   const UnionRefs U = block_union(a.ug, a.idx, P, a.E, smem, L.us, &s_u);
   __syncthreads();  // barrier init, zeroed accumulators and union visible to every warp
+  grid_dep_launch();
   const size_t qrow = a.I / 8, srow = a.I / 64;
   const unsigned q_bytes = nrows * (a.I / 2), sb_bytes = nrows * (a.I / 32);
+  uint64_t pol = 0;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      for (int j = 0; j < U.u; ++j) {
-        const int st = j % kStages3;
-        if (j >= kStages3 && !mbar_wait(&empty[st], ((j / kStages3) - 1) & 1)) break;
-        unsigned char* buf = smem + L.stages + (size_t)st * L.stage_bytes;
-        const size_t r0 = (size_t)U.unique[j] * a.H + c0row;
-        mbar_arrive_expect_tx(&full[st], q_bytes + 2 * sb_bytes);
-        bulk_g2s(buf, a.dq + r0 * qrow, q_bytes, &full[st], pol);
-        bulk_g2s(buf + L.q_bytes, a.ds + r0 * srow, sb_bytes, &full[st], pol);
-        bulk_g2s(buf + L.q_bytes + L.sb_bytes, a.db + r0 * srow, sb_bytes, &full[st], pol);
-      }
-    }
-  } else {
-    // h comes from the preceding grid.
-    grid_dep_wait();
-    const int wc = warp - 1;
-    const int cw = wc % a.ncw3, rg = wc / a.ncw3;
-    const int ch = cw * 32 + lane;
-    const bool active = ch < a.I / 32;
-    float* part = reinterpret_cast<float*>(smem + L.part);
-    const int part_stride = a.ncw3 * kMaxRows3 * kNT;
-    const int n_cons = n_cons_warps * 32;
-    const int ct = threadIdx.x - 32;
-    float xf[kNT][32];
-    float xs[kNT];
-    int pb = 0;
-    for (int j = 0; j < U.u; ++j) {
-      const int st = j % kStages3;
-      const int pos0 = U.offsets[j], n_e = U.offsets[j + 1] - pos0;
-      const bool ok = mbar_wait(&full[st], (j / kStages3) & 1);
-      const unsigned char* bq = smem + L.stages + (size_t)st * L.stage_bytes;
-      const uint16_t* bs = reinterpret_cast<const uint16_t*>(bq + L.q_bytes);
-      const uint16_t* bb = reinterpret_cast<const uint16_t*>(bq + L.q_bytes + L.sb_bytes);
-      for (int c0 = 0; c0 < n_e; c0 += kNT) {
-        const int nt = min(kNT, n_e - c0);
+  // thread 0: copy this CTA's rows of Wd[unique[j]] into ring slot j % kStages3
+  auto issue = [&](int j) {
+    const int st = j % kStages3;
+    unsigned char* buf = smem + L.stages + (size_t)st * L.stage_bytes;
+    const size_t r0 = (size_t)U.unique[j] * a.H + c0row;
+    mbar_arrive_expect_tx(&full[st], q_bytes + 2 * sb_bytes);
+    bulk_g2s(buf, a.dq + r0 * qrow, q_bytes, &full[st], pol);
+    bulk_g2s(buf + L.q_bytes, a.ds + r0 * srow, sb_bytes, &full[st], pol);
+    bulk_g2s(buf + L.q_bytes + L.sb_bytes, a.db + r0 * srow, sb_bytes, &full[st], pol);
+  };
+  // Weights do not depend on the preceding grid: start streaming them now.
+  if (threadIdx.x == 0) {
+    pol = policy_evict_first();
+    for (int j = 0; j < U.u && j < kStages3; ++j) issue(j);
+  }
+  // h comes from the preceding grid.
+  grid_dep_wait();
+
+  const int cw = warp % a.ncw3, rg = warp / a.ncw3;
+  const int ch = cw * 32 + lane;
+  const bool active = ch < a.I / 32;
+  float* part = reinterpret_cast<float*>(smem + L.part);
+  const int part_stride = a.ncw3 * kMaxRows3 * kNT;
+  const int ct = threadIdx.x;
+  float xf[kNT][32];
+  float xs[kNT];
+  int pb = 0;
+  for (int j = 0; j < U.u; ++j) {
+    const int st = j % kStages3;
+    const int pos0 = U.offsets[j], n_e = U.offsets[j + 1] - pos0;
+    const bool ok = mbar_wait(&full[st], (j / kStages3) & 1);
+    const unsigned char* bq = smem + L.stages + (size_t)st * L.stage_bytes;
+    const uint16_t* bs = reinterpret_cast<const uint16_t*>(bq + L.q_bytes);
+    const uint16_t* bb = reinterpret_cast<const uint16_t*>(bq + L.q_bytes + L.sb_bytes);
+    for (int c0 = 0; c0 < n_e; c0 += kNT) {
+      const int nt = min(kNT, n_e - c0);
 #pragma unroll
-        for (int t = 0; t < kNT; ++t)
-          if (t < nt && active)
-            load_x32(a.h + (size_t)(pos0 + c0 + t) * a.I, ch, xf[t], xs[t]);
-        float acc[kRowsPerWarp3 * kNT];
+      for (int t = 0; t < kNT; ++t)
+        if (t < nt && active) load_x32(a.h + (size_t)(pos0 + c0 + t) * a.I, ch, xf[t], xs[t]);
+      float acc[kRowsPerWarp3 * kNT];
 #pragma unroll
-        for (int i = 0; i < kRowsPerWarp3 * kNT; ++i) acc[i] = 0.f;
-        if (active && ok) {
+      for (int i = 0; i < kRowsPerWarp3 * kNT; ++i) acc[i] = 0.f;
+      if (active && ok) {
 #pragma unroll
-          for (int i = 0; i < kRowsPerWarp3; ++i) {
-            const int r = rg + row_groups * i;
-            if (r < nrows) {
-              const uint4 wv =
-                  *reinterpret_cast<const uint4*>(bq + (size_t)r * (a.I / 2) + ch * 16);
-              const float sc = bf16_bits_to_float(bs[r * (a.I / 64) + (ch >> 1)]);
-              const float bi = bf16_bits_to_float(bb[r * (a.I / 64) + (ch >> 1)]);
-              float d[kNT];
-              dot32(wv, xf, nt, d);
-#pragma unroll
-              for (int t = 0; t < kNT; ++t) acc[i * kNT + t] = fmaf(sc, d[t], bi * xs[t]);
-            }
-          }
-        }
-        if (c0 + kNT >= n_e) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[st]);
-        }
-        int vid;
-        const float v = warp_reduce_scatter<kRowsPerWarp3 * kNT>(acc, lane, vid);
-        float* pbuf = part + pb * part_stride;
-        {
-          const int i = vid / kNT, t = vid % kNT;
+        for (int i = 0; i < kRowsPerWarp3; ++i) {
           const int r = rg + row_groups * i;
-          if (r < kMaxRows3) pbuf[(cw * kMaxRows3 + r) * kNT + t] = v;
-        }
-        named_barrier(1, n_cons);
-        if (ct < nrows) {
-          const int r = ct;
-          for (int t = 0; t < nt; ++t) {
-            float y = 0.f;
-            for (int c = 0; c < a.ncw3; ++c) y += pbuf[(c * kMaxRows3 + r) * kNT + t];
-            const int p = U.pair_list[pos0 + c0 + t];
-            acc_out[(p / a.k) * a.rows_per_cta + r] += a.w[p] * y;
+          if (r < nrows) {
+            const uint4 wv = *reinterpret_cast<const uint4*>(bq + (size_t)r * (a.I / 2) + ch * 16);
+            const float sc = bf16_bits_to_float(bs[r * (a.I / 64) + (ch >> 1)]);
+            const float bi = bf16_bits_to_float(bb[r * (a.I / 64) + (ch >> 1)]);
+            float d[kNT];
+            dot32(wv, xf, nt, d);
+#pragma unroll
+            for (int t = 0; t < kNT; ++t) acc[i * kNT + t] = fmaf(sc, d[t], bi * xs[t]);
           }
         }
-        pb ^= 1;
       }
+      int vid;
+      const float v = warp_reduce_scatter<kRowsPerWarp3 * kNT>(acc, lane, vid);
+      float* pbuf = part + pb * part_stride;
+      {
+        const int i = vid / kNT, t = vid % kNT;
+        const int r = rg + row_groups * i;
+        if (r < kMaxRows3) pbuf[(cw * kMaxRows3 + r) * kNT + t] = v;
+      }
+      named_barrier(1, kThreads);
+      if (c0 + kNT >= n_e && threadIdx.x == 0 && j + kStages3 < U.u) {
+        fence_proxy_async();
+        issue(j + kStages3);
+      }
+      if (ct < nrows) {
+        const int r = ct;
+        for (int t = 0; t < nt; ++t) {
+          float y = 0.f;
+          for (int c = 0; c < a.ncw3; ++c) y += pbuf[(c * kMaxRows3 + r) * kNT + t];
+          const int p = U.pair_list[pos0 + c0 + t];
+          acc_out[(p / a.k) * a.rows_per_cta + r] += a.w[p] * y;
+        }
+      }
+      pb ^= 1;
     }
-    named_barrier(1, n_cons);
-    for (int i = ct; i < a.T * nrows; i += n_cons) {
-      const int t = i / nrows, r = i % nrows;
-      a.out[(size_t)t * a.H + c0row + r] = float_to_bf16_bits(acc_out[t * a.rows_per_cta + r]);
-    }
+  }
+  named_barrier(1, kThreads);
+  for (int i = ct; i < a.T * nrows; i += kThreads) {
+    const int t = i / nrows, r = i % nrows;
+    a.out[(size_t)t * a.H + c0row + r] = float_to_bf16_bits(acc_out[t * a.rows_per_cta + r]);
   }
 }
 
