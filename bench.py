@@ -35,8 +35,9 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-E, K_TOP, HIDDEN, INTER = 288, 8, 4096, 2048
-LAYERS = 42
+K_TOP, HIDDEN, INTER = 8, 4096, 2048
+E = 288     # experts in the bank (--experts changes it, for small profiling cases only)
+LAYERS = 42  # chained layers per T (--layers changes it, for small profiling cases only)
 TS = (1, 4)
 SEED = 2000
 BYTES_PER_EXPERT = 3 * (INTER * HIDDEN // 2 + 2 * 2 * INTER * HIDDEN // 64)  # 14,155,776
@@ -115,9 +116,9 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except Exception:
@@ -141,9 +142,12 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], 0.0, set()
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for ln in self.lines:
-            f = [c.strip() for c in ln.split(",")]
-            if len(f) < 9:
+        rows = [[c.strip() for c in ln.split(",")] for ln in self.lines]
+        rows = [f for f in rows if len(f) >= 9]
+        indices = sorted(set(f[0] for f in rows))
+        want = str(self.gpu) if str(self.gpu) in indices else (indices[0] if indices else None)
+        for f in rows:
+            if f[0] != want:
                 continue
             try:
                 sm.append(float(f[1]))
@@ -154,17 +158,24 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(n)
         if not sm:
-            return None
+            return {"error": (self.lines[:2] if self.lines else "no nvidia-smi output")}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
 
 
 # --------------------------------------------------------------- workload ---
+ROUTING = "uniform"  # --routing markov: adjacent-overlap chain at p=0.40 (profiling)
+
+
 def routings():
     import synth
     out = {}
     for T in TS:
-        out[T] = [synth.route_uniform(T, E, K_TOP, SEED + 100 * T + l) for l in range(LAYERS)]
+        if ROUTING == "markov":
+            out[T] = [synth.route_markov(T, E, K_TOP, 0.40, SEED + 100 * T + l)
+                      for l in range(LAYERS)]
+        else:
+            out[T] = [synth.route_uniform(T, E, K_TOP, SEED + 100 * T + l) for l in range(LAYERS)]
     return out
 
 
@@ -254,6 +265,10 @@ def reference_arm(args, world, rank):
 
 
 def our_arm(args, world, rank, local):
+    global E, LAYERS, TS, ROUTING
+    E, LAYERS, ROUTING = args.experts, args.layers, args.routing
+    if args.ts:
+        TS = tuple(int(t) for t in args.ts.split(","))
     import torch
     import quantized_expert_gather_b200 as qeg
     import synth
@@ -281,8 +296,8 @@ def our_arm(args, world, rank, local):
     wts = {T: [torch.from_numpy(r[1]).to(dev) for r in routes[T]] for T in TS}
     outs = {T: [torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=dev)
                 for _ in range(LAYERS)] for T in TS}
-    ws = torch.empty(max(qeg.moe_workspace_size(T, K_TOP, E, HIDDEN, INTER) for T in TS),
-                     dtype=torch.uint8, device=dev)
+    ws = torch.zeros(max(qeg.moe_workspace_size(T, K_TOP, E, HIDDEN, INTER) for T in TS),
+                     dtype=torch.uint8, device=dev)  # barrier words must start at zero
 
     def step():
         for T in TS:
@@ -290,7 +305,7 @@ def our_arm(args, world, rank, local):
                 qeg.moe_switchglu_forward_ws(xs[T], idx[T][l], wts[T][l], bank, ws,
                                              out=outs[T][l])
 
-    launches_per_step = 2 * LAYERS * len(TS)
+    launches_per_step = LAYERS * len(TS)  # one layer kernel per layer
     step()  # first call: per-device set-up, outside any capture
     torch.cuda.synchronize()
     if qeg.moe_read_device_status() != qeg.MOE_OK:
@@ -319,6 +334,9 @@ def our_arm(args, world, rank, local):
     all_bytes = sum_over_ranks(total_bytes * args.steps, world)
     gbs = all_bytes / (ms_total * 1e-3) / 1e9
 
+    if args.quick:  # profiling runs: the timed graph replays only
+        del graph
+        return {"quick": True, "value": gbs, "ms_per_step": ms_step} if rank == 0 else None
     # per-layer times (events between layers, chained; and isolated with an L2 flush)
     per = {}
     flush = torch.empty(4 * L2_BYTES, dtype=torch.uint8, device=dev)
@@ -405,8 +423,8 @@ def our_arm(args, world, rank, local):
 
     peak, peak_kind = measured_peaks()
     layer_bytes = {T: float(np.mean(uq[T])) * BYTES_PER_EXPERT for T in TS}
-    # dominant kernel pair: gate+up and down of one layer, chained by programmatic launch;
-    # algorithmic bytes = u * 14,155,776 per layer, time = graph-replayed per-layer time
+    # dominant kernel: the layer kernel (one launch per layer); algorithmic bytes per
+    # launch = u * 14,155,776, time = its average duration inside graph replays
     tot_b = sum(layer_bytes[T] for T in TS)
     tot_us = sum(per[T]["graph_us_per_layer"] for T in TS)
     achieved = tot_b / (tot_us * 1e-6) / 1e9
@@ -436,7 +454,7 @@ def our_arm(args, world, rank, local):
             "frac_of_peak": gbs / peak, "frac_of_nominal_8TBs": gbs / 8000.0,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_source": peak_kind,
-                         "kernel": "gate_up_kernel + down_combine_kernel (one layer)",
+                         "kernel": "layer_kernel (one launch per layer)",
                          "traffic": None},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
@@ -458,6 +476,12 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--layers", type=int, default=42, help="chained layers per T (profiling)")
+    ap.add_argument("--experts", type=int, default=288, help="bank size (profiling)")
+    ap.add_argument("--quick", action="store_true", help="timed graph only (profiling)")
+    ap.add_argument("--ts", default="", help="comma-separated window sizes (profiling)")
+    ap.add_argument("--routing", default="uniform", choices=("uniform", "markov"),
+                    help="routing model (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

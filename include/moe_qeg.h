@@ -77,8 +77,12 @@ const char* moe_status_str(int status);
 const char* moe_last_error(void);
 
 /* Bytes of workspace that moe_switchglu_forward_ws needs for this shape
- * (0 on invalid arguments).  The workspace holds the route-union arrays and
- * h = bf16 [T*k, inter]; its contents are scratch between calls. */
+ * (0 on invalid arguments).  The workspace holds the kernel's progress
+ * counters, the route-union arrays, h = bf16 [T*k, inter] and y = fp32
+ * [T*k, hidden].  The counter region (the first moe_workspace_layout()[1]
+ * bytes) must be zero before the first call on a buffer; every call leaves it
+ * zero again (after a call that ends in MOE_ERR_TIMEOUT it must be zeroed
+ * again).  Zeroing the whole buffer once is enough.  The rest is scratch. */
 size_t moe_workspace_size(int T, int k, int E, int hidden, int inter);
 
 /*
@@ -103,10 +107,14 @@ moe_status moe_route_union(const int32_t* topk_idx, int T, int k, int E, int32_t
 /*
  * The fused union-of-experts SwitchGLU forward described at the top of this
  * file, using caller-provided device workspace of at least
- * moe_workspace_size(T, k, E, hidden, inter) bytes (16-byte aligned).
- * x, the weight arrays, out and workspace must be 16-byte aligned; topk_idx
- * and topk_w 4-byte aligned.  Tokens whose pairs are all invalid get a zero
- * output row.  Capturable in a CUDA graph.
+ * moe_workspace_size(T, k, E, hidden, inter) bytes (16-byte aligned, counter
+ * region zero as described there).  x, the weight arrays, out and workspace
+ * must be 16-byte aligned; topk_idx and topk_w 4-byte aligned.  Tokens whose
+ * pairs are all invalid get a zero output row.  The forward is one kernel of
+ * one CTA per SM whose CTAs wait on one another's progress through counters
+ * in the workspace (it is launched cooperatively, so all CTAs are resident);
+ * two calls that share a workspace must not run concurrently.  Capturable in a
+ * CUDA graph.
  */
 moe_status moe_switchglu_forward_ws(const uint16_t* x, const int32_t* topk_idx,
                                     const float* topk_w, const uint32_t* wg_q,
@@ -142,18 +150,20 @@ moe_status moe_read_device_status(void* stream);
 
 /*
  * Which kernel path a call with this shape takes, without launching anything:
- * 1 = expert-major dequant-GEMV path (route-union, fused gate+up, down with
- * combine), 2 = grouped tensor-core path, 0 = invalid/unsupported shape.
+ * 1 = expert-major dequant-GEMV layer kernel (T*k <= 1024), 2 = grouped
+ * tensor-core path, 0 = invalid or unsupported shape.
  */
 int moe_select_path(int T, int k, int E, int hidden, int inter);
 
 /*
  * Offsets (bytes) of the workspace regions for this shape, for inspection in
- * tests: out[0] = num_unique (int32), out[1] = unique, out[2] = offsets,
- * out[3] = pair_list, out[4] = h (bf16 [T*k, inter] in pair_list order),
- * out[5] = total bytes.  Returns MOE_ERR_INVALID_ARG on bad shapes.
+ * tests: out[0] = progress counters (zero between calls; they end where
+ * out[1] starts), out[1] = num_unique (int32), out[2] =
+ * unique, out[3] = offsets, out[4] = pair_list, out[5] = h (bf16 [T*k, inter]
+ * in pair_list order), out[6] = y (fp32 [T*k, hidden] in pair_list order),
+ * out[7] = total bytes.  Returns MOE_ERR_INVALID_ARG on bad shapes.
  */
-moe_status moe_workspace_layout(int T, int k, int E, int hidden, int inter, size_t out[6]);
+moe_status moe_workspace_layout(int T, int k, int E, int hidden, int inter, size_t out[8]);
 
 #ifdef __cplusplus
 }

@@ -19,7 +19,8 @@ from ._build import SO, build as build_library, needs_build
 
 __all__ = ["MoeError", "MOE_OK", "moe_status_str", "moe_workspace_size", "moe_workspace_layout",
            "moe_select_path", "moe_route_union", "moe_switchglu_forward",
-           "moe_switchglu_forward_ws", "moe_read_device_status", "moe_last_error", "library_path",
+           "moe_switchglu_forward_ws", "moe_read_device_status", "moe_last_error", "moe_workspace",
+           "library_path",
            "QuantBank"]
 
 MOE_OK = 0
@@ -112,10 +113,17 @@ def moe_workspace_size(T: int, k: int, E: int, hidden: int, inter: int) -> int:
 
 
 def moe_workspace_layout(T: int, k: int, E: int, hidden: int, inter: int) -> dict:
-    out = (ctypes.c_size_t * 6)()
+    out = (ctypes.c_size_t * 8)()
     _check(_lib.moe_workspace_layout(T, k, E, hidden, inter, ctypes.addressof(out)),
            "moe_workspace_layout", True)
-    return dict(zip(("num_unique", "unique", "offsets", "pair_list", "h", "total"), list(out)))
+    return dict(zip(("barrier", "num_unique", "unique", "offsets", "pair_list", "h", "y",
+                     "total"), list(out)))
+
+
+def moe_workspace(T: int, k: int, E: int, hidden: int, inter: int, device=None) -> torch.Tensor:
+    """A zeroed uint8 device workspace of the size moe_switchglu_forward_ws needs."""
+    return torch.zeros(moe_workspace_size(T, k, E, hidden, inter), dtype=torch.uint8,
+                       device=device if device is not None else "cuda")
 
 
 def moe_select_path(T: int, k: int, E: int, hidden: int, inter: int) -> int:
@@ -194,7 +202,8 @@ def moe_switchglu_forward(x, topk_idx, topk_w, bank: QuantBank, out=None, stream
 
 def moe_switchglu_forward_ws(x, topk_idx, topk_w, bank: QuantBank, workspace: torch.Tensor,
                              out=None, stream=None, check: bool = True):
-    """As moe_switchglu_forward, with a caller-owned uint8 device workspace tensor."""
+    """As moe_switchglu_forward, with a caller-owned uint8 device workspace tensor (see
+    moe_workspace: its first 16 bytes must be zero before the first call)."""
     args, dims, out = _fwd_args(x, topk_idx, topk_w, bank, out)
     st = _lib.moe_switchglu_forward_ws(*args, *dims, _ptr(out, _BF16, "out"),
                                        _ptr(workspace, (torch.uint8,), "workspace"),

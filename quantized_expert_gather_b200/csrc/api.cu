@@ -9,7 +9,7 @@
 
 #include "../../include/moe_qeg.h"
 #include "common.cuh"
-#include "gemv.cuh"
+#include "layer.cuh"
 #include "route_union.cuh"
 
 namespace qeg {
@@ -21,7 +21,7 @@ struct DeviceInfo {
   bool ready = false;
   int sms = 0;
   int smem_optin = 0;
-  int dyn_smem[3] = {0, 0, 0};  // dynamic shared memory limit: gate_up, down, route_union
+  int dyn_smem[2] = {0, 0};  // dynamic shared memory limit: layer, route_union
 };
 
 DeviceInfo g_dev[kMaxDevices];
@@ -47,10 +47,9 @@ moe_status device_info(DeviceInfo** out) {
       e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return cuda_fail(e);
     // dynamic + static shared memory may not exceed the opt-in limit
-    const void* kernels[3] = {reinterpret_cast<const void*>(gate_up_kernel),
-                              reinterpret_cast<const void*>(down_combine_kernel),
+    const void* kernels[2] = {reinterpret_cast<const void*>(layer_kernel),
                               reinterpret_cast<const void*>(route_union_kernel)};
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < 2; ++i) {
       cudaFuncAttributes fa;
       cudaError_t e = cudaFuncGetAttributes(&fa, kernels[i]);
       if (e == cudaSuccess) {
@@ -80,133 +79,89 @@ bool shape_supported(int T, int k, int E, int hidden, int inter) {
 }
 
 struct WsLayout {
-  size_t num_unique, unique, offsets, pair_list, h, total;
+  size_t barrier, num_unique, unique, offsets, pair_list, h, y, total;  // barrier = counters
 };
 
-WsLayout ws_layout(int T, int k, int E, int inter) {
+WsLayout ws_layout(int T, int k, int E, int hidden, int inter) {
   const size_t P = (size_t)T * k;
   const size_t m = P < (size_t)E ? P : (size_t)E;
   WsLayout w;
-  w.num_unique = 0;
-  w.unique = 16;
+  w.barrier = 0;
+  w.num_unique = align_up(4 * kSyncWords, 256);
+  w.unique = w.num_unique + 16;
   w.offsets = align_up(w.unique + 4 * m, 16);
   w.pair_list = align_up(w.offsets + 4 * (m + 1), 16);
   w.h = align_up(w.pair_list + 4 * P, 256);
-  w.total = align_up(w.h + 2 * P * (size_t)inter, 256);
+  w.y = align_up(w.h + 2 * P * (size_t)inter, 256);
+  w.total = align_up(w.y + 4 * P * (size_t)hidden, 256);
   return w;
-}
-
-int next_pow2(int v) {
-  int p = 1;
-  while (p < v) p <<= 1;
-  return p;
-}
-
-int gemv_ncw(int hidden) { return (hidden / 32 + 31) / 32; }
-int gemv_ncw3(int inter) { return next_pow2((inter / 32 + 31) / 32); }
-
-// Output rows per CTA of the down kernel: about one CTA per SM, a multiple of the
-// row count that keeps 1-D copies of scale/bias rows 16-byte aligned.
-int gemv_rows_per_cta(int hidden, int inter, int sms) {
-  const int sb_row = inter / 32;  // bytes of scales (or biases) per row
-  int g = 16;
-  for (int a = sb_row, b = 16; b;) {  // gcd(sb_row, 16)
-    const int t = a % b;
-    a = b;
-    b = t;
-    g = a;
-  }
-  const int gran = 16 / g;
-  const int cap = (kConsWarps / gemv_ncw3(inter)) * kRowsPerWarp3;
-  int rows = (hidden + sms - 1) / sms;
-  rows = (rows + gran - 1) / gran * gran;
-  if (rows > cap) rows = cap / gran * gran;
-  if (rows < gran) rows = gran;
-  return rows;
 }
 
 int select_path(int T, int k, int E, int hidden, int inter) {
   if (!shape_ok(T, k, E, hidden, inter) || !shape_supported(T, k, E, hidden, inter)) return 0;
-  if (T <= kGemvMaxT && T * k <= kGemvMaxPairs) return 1;
+  if (T * k <= kMaxPairsFused) return 1;
   return 0;  // the grouped tensor-core path is not available in this build
 }
 
-cudaError_t launch_gemv(const uint16_t* x, const int32_t* idx, const float* w, const uint32_t* gq,
-                        const uint16_t* gs, const uint16_t* gb, const uint32_t* uq,
-                        const uint16_t* us, const uint16_t* ub, const uint32_t* dq,
-                        const uint16_t* ds, const uint16_t* db, int T, int k, int E, int H, int I,
-                        uint16_t* out, unsigned char* ws, const DeviceInfo& d, cudaStream_t st,
-                        moe_status* why) {
-  const WsLayout wl = ws_layout(T, k, E, I);
-  const int P = T * k;
-  GateUpArgs ga;
-  ga.x = x;
-  ga.idx = idx;
-  ga.gq = gq;
-  ga.gs = gs;
-  ga.gb = gb;
-  ga.uq = uq;
-  ga.us = us;
-  ga.ub = ub;
-  ga.h = reinterpret_cast<uint16_t*>(ws + wl.h);
-  ga.ug = UnionGlobal{nullptr, nullptr, nullptr, nullptr};
-  ga.ex_u = reinterpret_cast<int*>(ws + wl.num_unique);
-  ga.ex_unique = reinterpret_cast<int*>(ws + wl.unique);
-  ga.ex_offsets = reinterpret_cast<int*>(ws + wl.offsets);
-  ga.ex_pair_list = reinterpret_cast<int*>(ws + wl.pair_list);
-  ga.T = T;
-  ga.k = k;
-  ga.E = E;
-  ga.H = H;
-  ga.I = I;
-  ga.ncw = gemv_ncw(H);
-  ga.wait_prior = 1;
-  const K2Layout L2 = k2_layout(H, E, P, ga.ncw);
-
-  DownArgs da;
-  da.idx = idx;
-  da.w = w;
-  da.dq = dq;
-  da.ds = ds;
-  da.db = db;
-  da.h = ga.h;
-  da.out = out;
-  da.ug = ga.ug;
-  da.T = T;
-  da.k = k;
-  da.E = E;
-  da.H = H;
-  da.I = I;
-  da.ncw3 = gemv_ncw3(I);
-  da.rows_per_cta = gemv_rows_per_cta(H, I, d.sms);
-  const K3Layout L3 = k3_layout(I, E, P, T, da.ncw3, da.rows_per_cta);
-  if (L2.total > (size_t)d.dyn_smem[0] || L3.total > (size_t)d.dyn_smem[1]) {
+cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
+                         const uint32_t* gq, const uint16_t* gs, const uint16_t* gb,
+                         const uint32_t* uq, const uint16_t* us, const uint16_t* ub,
+                         const uint32_t* dq, const uint16_t* ds, const uint16_t* db, int T, int k,
+                         int E, int H, int I, uint16_t* out, unsigned char* ws,
+                         const DeviceInfo& d, cudaStream_t st, moe_status* why) {
+  const WsLayout wl = ws_layout(T, k, E, H, I);
+  LayerArgs a;
+  a.x = x;
+  a.idx = idx;
+  a.w = w;
+  a.gq = gq;
+  a.gs = gs;
+  a.gb = gb;
+  a.uq = uq;
+  a.us = us;
+  a.ub = ub;
+  a.dq = dq;
+  a.ds = ds;
+  a.db = db;
+  a.h = reinterpret_cast<uint16_t*>(ws + wl.h);
+  a.y = reinterpret_cast<float*>(ws + wl.y);
+  a.sync = reinterpret_cast<unsigned*>(ws + wl.barrier);
+  a.ex_u = reinterpret_cast<int*>(ws + wl.num_unique);
+  a.ex_unique = reinterpret_cast<int*>(ws + wl.unique);
+  a.ex_offsets = reinterpret_cast<int*>(ws + wl.offsets);
+  a.ex_pair_list = reinterpret_cast<int*>(ws + wl.pair_list);
+  a.out = out;
+  a.T = T;
+  a.k = k;
+  a.E = E;
+  a.H = H;
+  a.I = I;
+  a.g = layer_geom(H, I);
+  a.wait_prior = 1;
+  const LayerSmem L = layer_smem(a.g, E, T * k, H, I);
+  if (a.g.seg < 1) {
     *why = MOE_ERR_UNSUPPORTED;
     return cudaSuccess;
   }
-
-  cudaLaunchAttribute attr[1];
+  if (L.total > (size_t)d.dyn_smem[0]) {
+    *why = MOE_ERR_UNSUPPORTED;
+    return cudaSuccess;
+  }
+  // One CTA per SM, all resident at once (the kernel has grid barriers); the
+  // launch may overlap the tail of the preceding kernel (programmatic launch).
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-
-  cudaLaunchConfig_t c2 = {};
-  c2.gridDim = dim3(d.sms);
-  c2.blockDim = dim3(32 * 2 * ga.ncw);
-  c2.dynamicSmemBytes = L2.total;
-  c2.stream = st;
-  c2.attrs = attr;
-  c2.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&c2, gate_up_kernel, ga);
-  if (e != cudaSuccess) return e;
-
-  cudaLaunchConfig_t c3 = {};
-  c3.gridDim = dim3((H + da.rows_per_cta - 1) / da.rows_per_cta);
-  c3.blockDim = dim3(kThreads);
-  c3.dynamicSmemBytes = L3.total;
-  c3.stream = st;
-  c3.attrs = attr;
-  c3.numAttrs = 1;
-  return cudaLaunchKernelEx(&c3, down_combine_kernel, da);
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
+  cudaLaunchConfig_t c = {};
+  c.gridDim = dim3(d.sms);
+  c.blockDim = dim3(kThreads);
+  c.dynamicSmemBytes = L.total;
+  c.stream = st;
+  c.attrs = attr;
+  c.numAttrs = 2;
+  return cudaLaunchKernelEx(&c, layer_kernel, a);
 }
 
 struct OwnedWorkspace {
@@ -239,18 +194,20 @@ const char* moe_status_str(int s) {
 
 size_t moe_workspace_size(int T, int k, int E, int hidden, int inter) {
   if (!shape_ok(T, k, E, hidden, inter)) return 0;
-  return ws_layout(T, k, E, inter).total;
+  return ws_layout(T, k, E, hidden, inter).total;
 }
 
-moe_status moe_workspace_layout(int T, int k, int E, int hidden, int inter, size_t out[6]) {
+moe_status moe_workspace_layout(int T, int k, int E, int hidden, int inter, size_t out[8]) {
   if (!out || !shape_ok(T, k, E, hidden, inter)) return MOE_ERR_INVALID_ARG;
-  const WsLayout w = ws_layout(T, k, E, inter);
-  out[0] = w.num_unique;
-  out[1] = w.unique;
-  out[2] = w.offsets;
-  out[3] = w.pair_list;
-  out[4] = w.h;
-  out[5] = w.total;
+  const WsLayout w = ws_layout(T, k, E, hidden, inter);
+  out[0] = w.barrier;
+  out[1] = w.num_unique;
+  out[2] = w.unique;
+  out[3] = w.offsets;
+  out[4] = w.pair_list;
+  out[5] = w.h;
+  out[6] = w.y;
+  out[7] = w.total;
   return MOE_OK;
 }
 
@@ -270,7 +227,7 @@ moe_status moe_route_union(const int32_t* topk_idx, int T, int k, int E, int32_t
   DeviceInfo* d = nullptr;
   if (moe_status s = device_info(&d)) return s;
   const size_t smem = route_union_smem_bytes(E);
-  if (smem > (size_t)d->dyn_smem[2]) return MOE_ERR_UNSUPPORTED;
+  if (smem > (size_t)d->dyn_smem[1]) return MOE_ERR_UNSUPPORTED;
   route_union_kernel<<<1, 32 * kUnionWarps, smem, (cudaStream_t)stream>>>(
       topk_idx, T * k, E, unique, offsets, pair_list, num_unique);
   const cudaError_t e = cudaGetLastError();
@@ -295,11 +252,11 @@ moe_status moe_switchglu_forward_ws(const uint16_t* x, const int32_t* topk_idx,
   if (!aligned(topk_idx, 4) || !aligned(topk_w, 4)) return MOE_ERR_UNSUPPORTED;
   const int path = select_path(T, k, E, hidden, inter);
   if (path == 0) return MOE_ERR_UNSUPPORTED;
-  if (workspace_bytes < ws_layout(T, k, E, inter).total) return MOE_ERR_WORKSPACE;
+  if (workspace_bytes < ws_layout(T, k, E, hidden, inter).total) return MOE_ERR_WORKSPACE;
   DeviceInfo* d = nullptr;
   if (moe_status s = device_info(&d)) return s;
   moe_status why = MOE_OK;
-  const cudaError_t e = launch_gemv(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q,
+  const cudaError_t e = launch_layer(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q,
                                     wd_s, wd_b, T, k, E, hidden, inter, out,
                                     static_cast<unsigned char*>(workspace), *d,
                                     (cudaStream_t)stream, &why);
@@ -319,7 +276,7 @@ moe_status moe_switchglu_forward(const uint16_t* x, const int32_t* topk_idx, con
   const cudaError_t ge = cudaGetDevice(&dev);
   if (ge != cudaSuccess) return cuda_fail(ge);
   if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
-  const size_t need = ws_layout(T, k, E, inter).total;
+  const size_t need = ws_layout(T, k, E, hidden, inter).total;
   OwnedWorkspace& w = g_ws[dev];
   {
     std::lock_guard<std::mutex> lock(g_mu);
@@ -336,8 +293,10 @@ moe_status moe_switchglu_forward(const uint16_t* x, const int32_t* topk_idx, con
         w.ptr = nullptr;
         w.bytes = 0;
       }
-      const cudaError_t me = cudaMalloc(&w.ptr, need);
+      cudaError_t me = cudaMalloc(&w.ptr, need);
+      if (me == cudaSuccess) me = cudaMemset(w.ptr, 0, need);  // grid-barrier words start at 0
       if (me != cudaSuccess) {
+        if (w.ptr) cudaFree(w.ptr);
         w.ptr = nullptr;
         return cuda_fail(me);
       }

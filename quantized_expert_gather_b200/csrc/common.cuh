@@ -50,13 +50,16 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Test phase `parity` of `bar`; a thread whose phase is not complete is suspended
+// until it completes or about kSuspendNs pass, instead of spinning on issue slots.
+constexpr unsigned kSuspendNs = 1000000;  // 1 ms
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
       " selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
       : "memory");
   return ok != 0;
 }
@@ -76,21 +79,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
 }
 
 // 1-D bulk copy global -> shared, completing `bytes` of transaction count on
-// `bar`.  dst, src and bytes must be multiples of 16.  Local memory only.
+// `bar`.  dst, src and bytes must be multiples of 16.  Local memory only, no
+// cluster multicast.  (No L2 eviction hint: on B200 an evict-first policy made
+// streaming reads slower.)
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes,
-                                         uint64_t* bar, uint64_t policy) {
+                                         uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
-}
-
-// L2 policy for data read exactly once (expert weights): evict first.
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
 }
 
 // Programmatic dependent launch controls.

@@ -23,8 +23,7 @@ def run_forward(L, ws=False):
     bank = to_dev_bank(L)
     x, idx, w = to_dev_inputs(L)
     if ws:
-        nbytes = qeg.moe_workspace_size(L.T, L.k, L.E, L.H, L.I)
-        work = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+        work = qeg.moe_workspace(L.T, L.k, L.E, L.H, L.I)
         out = qeg.moe_switchglu_forward_ws(x, idx, w, bank, work)
     else:
         out = qeg.moe_switchglu_forward(x, idx, w, bank)
@@ -113,12 +112,12 @@ def test_forward_small_shapes(cfg):
 def test_forward_ws_variant_and_union_export():
     L = make_layer(6, 4, 24, 256, 256, seed=21)
     out, (bank, x, idx, w) = run_forward(L)
-    nbytes = qeg.moe_workspace_size(L.T, L.k, L.E, L.H, L.I)
-    work = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    work = qeg.moe_workspace(L.T, L.k, L.E, L.H, L.I)
     out2 = qeg.moe_switchglu_forward_ws(x, idx, w, bank, work)
     torch.cuda.synchronize()
-    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
     lay = qeg.moe_workspace_layout(L.T, L.k, L.E, L.H, L.I)
+    assert not work[lay["barrier"]:lay["num_unique"]].any()  # progress counters back to zero
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
     wsn = work.cpu().numpy()
     u = int(wsn[lay["num_unique"]:lay["num_unique"] + 4].view(np.int32)[0])
     u_ref, o_ref, p_ref, n_ref, _ = oracle.route_union(L.idx, L.E)
@@ -246,3 +245,13 @@ def test_rejected_arguments_launch_nothing():
     assert st == qeg.MOE_ERR_INVALID_ARG
     torch.cuda.synchronize()
     assert qeg.moe_read_device_status() == qeg.MOE_OK
+
+
+def test_library_workspace_reused_across_shapes():
+    """The library-owned workspace serves calls of different shapes in any order: its
+    progress counters must stay zero between calls whatever shape came before."""
+    shapes = [(16, 8, 64, 1024, 512), (1, 2, 8, 256, 128), (9, 4, 30, 512, 1088),
+              (2, 8, 64, 256, 192), (16, 8, 64, 1024, 512)]
+    for i, (T, k, E, H, I) in enumerate(shapes):
+        L = make_layer(T, k, E, H, I, seed=900 + i, routing="uniform")
+        check_layer(L, f"reuse #{i} T={T} k={k} E={E} H={H} I={I}")

@@ -48,8 +48,9 @@ def test_status_strings():
 
 def test_path_selection_without_launch():
     # small windows -> expert-major GEMV path
-    for T in (1, 2, 4, 16, 64, 256):
+    for T in (1, 2, 4, 16, 64, 128):
         assert qeg.moe_select_path(T, 8, 256, 4096, 2048) == 1
+    assert qeg.moe_select_path(1024, 1, 256, 4096, 2048) == 1
     assert qeg.moe_select_path(2, 2, 16, 256, 128) == 1
     # invalid shapes
     assert qeg.moe_select_path(0, 8, 256, 4096, 2048) == 0
@@ -63,7 +64,11 @@ def test_workspace_size_and_layout():
     n = qeg.moe_workspace_size(T, k, E, H, I)
     lay = qeg.moe_workspace_layout(T, k, E, H, I)
     assert lay["total"] == n
-    assert lay["h"] % 256 == 0 and lay["h"] + 2 * T * k * I <= n
+    assert lay["barrier"] == 0 and lay["num_unique"] >= 4 * (1 + 1024 + 512)
+    # the counter region does not depend on the shape
+    assert qeg.moe_workspace_layout(1, 1, 4, 64, 64)["num_unique"] == lay["num_unique"]
+    assert lay["h"] % 256 == 0 and lay["h"] + 2 * T * k * I <= lay["y"]
+    assert lay["y"] % 256 == 0 and lay["y"] + 4 * T * k * H <= n
     assert lay["unique"] % 16 == 0 and lay["offsets"] % 16 == 0 and lay["pair_list"] % 16 == 0
     assert qeg.moe_workspace_size(0, 8, E, H, I) == 0
     with pytest.raises(qeg.MoeError):
