@@ -336,7 +336,8 @@ def our_arm(args, world, rank, local):
 
     if args.quick:  # profiling runs: the timed graph replays only
         del graph
-        return {"quick": True, "value": gbs, "ms_per_step": ms_step} if rank == 0 else None
+        return ({"quick": True, "value": gbs, "ms_per_step": ms_step, "clocks": clk.summary(),
+                 "us_per_layer": ms_step * 1e3 / (LAYERS * len(TS))} if rank == 0 else None)
     # per-layer times (events between layers, chained; and isolated with an L2 flush)
     per = {}
     flush = torch.empty(4 * L2_BYTES, dtype=torch.uint8, device=dev)

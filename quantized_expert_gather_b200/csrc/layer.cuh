@@ -510,11 +510,15 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
     }
   };
 
-  // out rows of row block rb for every token: sum_j w[t,j] * y[pos(t,j)][c], j ascending.
-  auto combine_rb = [&](int rb) {
-    const int c0 = rb * G.rows_b, nr = min(G.rows_b, a.H - c0);
-    for (int e = threadIdx.x; e < a.T * nr; e += kThreads) {
-      const int t = e / nr, c = c0 + e % nr;
+  // out rows of the row blocks comb[0..n) for every token:
+  // sum_j w[t,j] * y[pos(t,j)][c], j ascending.  One flat loop, so the loads of all
+  // row blocks are in flight together.
+  auto combine = [&](int n) {
+    const int per_rb = a.T * G.rows_b;
+    for (int e = threadIdx.x; e < n * per_rb; e += kThreads) {
+      const int rb = comb[e / per_rb], rem = e % per_rb;
+      const int t = rem / G.rows_b, c = rb * G.rows_b + rem % G.rows_b;
+      if (c >= a.H) continue;
       float acc = 0.f;
       for (int j = 0; j < a.k; ++j) {
         const int p = t * a.k + j;
@@ -549,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
       __threadfence();
     }
     __syncthreads();
-    for (int c = 0; c < s_ncomb; ++c) combine_rb(comb[c]);
+    combine(s_ncomb);
     seg_open = -1;
   };
 
