@@ -141,6 +141,36 @@ moe_status moe_switchglu_forward(const uint16_t* x, const int32_t* topk_idx, con
                                  int inter, uint16_t* out, void* stream);
 
 /*
+ * Same layer as moe_switchglu_forward, with no allocation of any kind: the
+ * scratch (progress counters, union arrays, h and y) is one fixed array of
+ * MOE_STATIC_SCRATCH_BYTES (4 MiB) per device, a `__device__` global of the
+ * library.  The pages describe no such entry point; it exists for callers that
+ * may not allocate (allocator-free or pre-planned memory).
+ *   - Limit: shapes whose moe_workspace_size exceeds MOE_STATIC_SCRATCH_BYTES
+ *     return MOE_ERR_WORKSPACE and moe_last_error() says so.  4 MiB holds
+ *     T*k <= 128 at hidden 4096 / inter 2048 (e.g. T <= 16 at top-8).
+ *   - Set-up: the first call on each device looks up the array's address
+ *     (cudaGetSymbolAddress, that device current) and caches it; make that
+ *     first call before any stream capture.
+ *   - Zeroing: each call clears the counter region (its first 4*1537 bytes)
+ *     with cudaMemsetAsync on `stream` before the kernel; nothing else needs
+ *     to start at zero.
+ *   - Races: all calls on one device share the one array.  Calls that overlap
+ *     (different streams, or host threads, without ordering between them)
+ *     corrupt each other's results; order them on one stream or with events.
+ * Arguments, alignment rules and results are those of moe_switchglu_forward_ws.
+ */
+#define MOE_STATIC_SCRATCH_BYTES ((size_t)4 << 20)
+moe_status moe_switchglu_forward_static(const uint16_t* x, const int32_t* topk_idx,
+                                        const float* topk_w, const uint32_t* wg_q,
+                                        const uint16_t* wg_s, const uint16_t* wg_b,
+                                        const uint32_t* wu_q, const uint16_t* wu_s,
+                                        const uint16_t* wu_b, const uint32_t* wd_q,
+                                        const uint16_t* wd_s, const uint16_t* wd_b, int T, int k,
+                                        int E, int hidden, int inter, uint16_t* out,
+                                        void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word that the
  * kernels set instead of trapping: MOE_ERR_DEVICE_INDEX if an expert id was
  * out of range, MOE_ERR_TIMEOUT if a bounded wait ran out, else MOE_OK (or

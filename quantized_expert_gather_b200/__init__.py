@@ -19,7 +19,7 @@ from ._build import SO, build as build_library, needs_build
 
 __all__ = ["MoeError", "MOE_OK", "moe_status_str", "moe_workspace_size", "moe_workspace_layout",
            "moe_select_path", "moe_route_union", "moe_switchglu_forward",
-           "moe_switchglu_forward_ws", "moe_read_device_status", "moe_last_error", "moe_workspace",
+           "moe_switchglu_forward_ws", "moe_switchglu_forward_static", "moe_read_device_status", "moe_last_error", "moe_workspace",
            "library_path",
            "QuantBank"]
 
@@ -60,6 +60,8 @@ def _load():
     lib.moe_switchglu_forward.argtypes = [vp] * 12 + [ci] * 5 + [vp, vp]
     lib.moe_switchglu_forward_ws.restype = ci
     lib.moe_switchglu_forward_ws.argtypes = [vp] * 12 + [ci] * 5 + [vp, vp, sz, vp]
+    lib.moe_switchglu_forward_static.restype = ci
+    lib.moe_switchglu_forward_static.argtypes = [vp] * 12 + [ci] * 5 + [vp, vp]
     lib.moe_read_device_status.restype = ci
     lib.moe_read_device_status.argtypes = [vp]
     return lib
@@ -210,6 +212,23 @@ def moe_switchglu_forward_ws(x, topk_idx, topk_w, bank: QuantBank, workspace: to
                                        workspace.numel(), _stream(stream))
     _check(st, "moe_switchglu_forward_ws", check)
     return out
+
+
+def moe_switchglu_forward_static(x, topk_idx, topk_w, bank: QuantBank, out=None, stream=None,
+                                 check: bool = True):
+    """As moe_switchglu_forward, with the library's fixed per-device scratch (no allocation
+    inside the call; shapes needing more than MOE_STATIC_SCRATCH_BYTES are rejected with
+    MOE_ERR_WORKSPACE; overlapping calls on one device race)."""
+    args, dims, out = _fwd_args(x, topk_idx, topk_w, bank, out)
+    st = _lib.moe_switchglu_forward_static(*args, *dims, _ptr(out, _BF16, "out"),
+                                           _stream(stream))
+    if check and st == MOE_ERR_WORKSPACE:
+        raise MoeError(st, f"moe_switchglu_forward_static [{moe_last_error()}]")
+    _check(st, "moe_switchglu_forward_static", check)
+    return out
+
+
+MOE_STATIC_SCRATCH_BYTES = 4 << 20
 
 
 def moe_read_device_status(stream=None) -> int:

@@ -170,6 +170,34 @@ struct OwnedWorkspace {
 };
 OwnedWorkspace g_ws[kMaxDevices];
 
+// Fixed scratch for moe_switchglu_forward_static: one copy per device, in the
+// module's global memory (zero at module load), so that entry never allocates.
+// 4 MiB covers T*k <= 128 pairs at hidden 4096 / inter 2048 (2,629,632 bytes
+// at T=16, k=8) and every smaller layer.
+constexpr size_t kStaticScratchBytes = MOE_STATIC_SCRATCH_BYTES;
+static_assert(kSyncWords == 1537, "the header states the counter region as 4*1537 bytes");
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+void* g_static_ptr[kMaxDevices] = {};
+
+// Device address of g_static_scratch for the current device: looked up once
+// per device (cudaGetSymbolAddress, with that device current), then cached.
+moe_status static_scratch(void** out) {
+  int dev = 0;
+  const cudaError_t ge = cudaGetDevice(&dev);
+  if (ge != cudaSuccess) return cuda_fail(ge);
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (!p) return MOE_ERR_CUDA;
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return MOE_OK;
+}
+
 }  // namespace
 }  // namespace qeg
 
@@ -305,6 +333,33 @@ moe_status moe_switchglu_forward(const uint16_t* x, const int32_t* topk_idx, con
   }
   return moe_switchglu_forward_ws(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q,
                                   wd_s, wd_b, T, k, E, hidden, inter, out, w.ptr, w.bytes, stream);
+}
+
+moe_status moe_switchglu_forward_static(const uint16_t* x, const int32_t* topk_idx,
+                                        const float* topk_w, const uint32_t* wg_q,
+                                        const uint16_t* wg_s, const uint16_t* wg_b,
+                                        const uint32_t* wu_q, const uint16_t* wu_s,
+                                        const uint16_t* wu_b, const uint32_t* wd_q,
+                                        const uint16_t* wd_s, const uint16_t* wd_b, int T, int k,
+                                        int E, int hidden, int inter, uint16_t* out,
+                                        void* stream) {
+  if (!shape_ok(T, k, E, hidden, inter)) return MOE_ERR_INVALID_ARG;
+  const size_t need = ws_layout(T, k, E, hidden, inter).total;
+  if (need > kStaticScratchBytes) {
+    g_last_error = "moe_switchglu_forward_static: this shape needs more scratch than the "
+                   "fixed 4 MiB (4194304 bytes); use moe_switchglu_forward_ws";
+    return MOE_ERR_WORKSPACE;
+  }
+  void* scratch = nullptr;
+  if (moe_status s = static_scratch(&scratch)) return s;
+  // The progress counters must be zero when the kernel starts; a call clears
+  // them again on the caller's stream (ordered after any earlier call there),
+  // so a call that ended with a device error leaves no stale counts behind.
+  const cudaError_t me = cudaMemsetAsync(scratch, 0, 4 * kSyncWords, (cudaStream_t)stream);
+  if (me != cudaSuccess) return cuda_fail(me);
+  return moe_switchglu_forward_ws(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q,
+                                  wd_s, wd_b, T, k, E, hidden, inter, out, scratch,
+                                  kStaticScratchBytes, stream);
 }
 
 moe_status moe_read_device_status(void* stream) {

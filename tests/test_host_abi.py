@@ -25,7 +25,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("moe_route_union", "moe_switchglu_forward", "moe_switchglu_forward_ws",
               "moe_workspace_size", "moe_read_device_status", "moe_status_str",
-              "moe_select_path", "moe_workspace_layout"):
+              "moe_select_path", "moe_workspace_layout", "moe_switchglu_forward_static"):
         assert n in names
 
 
