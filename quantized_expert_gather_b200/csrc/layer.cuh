@@ -35,14 +35,11 @@
 // the 32-column chunks l, l+32, ... of its rows, so one lane chunk sits inside
 // one quantisation group (64 columns):
 //     partial = s * sum_c q_c x_c + b * sum_c x_c.
-// The segment's activations sit in shared memory as fp32, laid out so that the
-// 32 lanes of a warp read 512 consecutive bytes (no bank conflicts), with the
-// per-chunk sums of x alongside.  A warp reduces its rows over its lanes once
-// per block; there is no cross-warp exchange inside a phase.
-//
-// Codes become floats without integer->float conversion: nibble j of a word
-// under exponent (150 - 4j) reads as 2^(23-4j) + q exactly; one packed fp32 add
-// removes the offset.  Products q*x are exact in fp32; sums are fp32.
+// The segment's activations sit in shared memory as 16-bit block fixed point
+// (one exponent per 32-column chunk, see below), so that sum_c q_c x_c is an
+// exact integer dot product of the 4-bit codes with the activation's two bytes
+// (dp4a), scaled once per chunk.  A warp reduces its rows over its lanes once per
+// block; there is no cross-warp exchange inside a phase.
 #pragma once
 
 #include "common.cuh"
@@ -57,7 +54,7 @@ constexpr int kMaxRowsPerWarpB = 4; // phase B: rows of Wd per warp per block
 constexpr int kStages = 4;          // ring depth
 constexpr int kNT = 4;              // pairs per segment (upper bound)
 constexpr int kMaxPairsFused = 1024;
-constexpr unsigned kXBytes = 64 * 1024;  // activation buffer (fp32)
+constexpr unsigned kXBytes = 64 * 1024;  // activation buffer (block fixed point)
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -82,7 +79,7 @@ __host__ __device__ inline LayerGeom layer_geom(int H, int I) {
   if (rb > kWarps * kMaxRowsPerWarpB) rb = kWarps * kMaxRowsPerWarpB;
   g.rows_b = rb;
   const int rmax = g.rounds_a > g.rounds_b ? g.rounds_a : g.rounds_b;
-  int s = (int)(kXBytes / (4096u * (unsigned)rmax));  // fp32 activations: rounds * 4 KB per pair
+  int s = (int)(kXBytes / (2048u * (unsigned)rmax));  // fixed point: rounds * 2 KB per pair
   g.seg = s > kNT ? kNT : s;
   g.a_q = kRowsA * H / 2;
   g.a_sb = kRowsA * H / 32;
@@ -106,7 +103,7 @@ __host__ __device__ inline LayerSmem layer_smem(const LayerGeom& g, int E, int P
   s.stages = 0;
   s.x = align_up((size_t)kStages * g.stage_bytes, 128);
   s.xsum = s.x + kXBytes;
-  s.cnt = align_up(s.xsum + sizeof(float) * kNT * rmax * 32, 16);
+  s.cnt = align_up(s.xsum + sizeof(float2) * kNT * rmax * 32, 16);
   s.rank = align_up(s.cnt + sizeof(int) * E, 16);
   s.unique = align_up(s.rank + sizeof(int) * P, 16);
   s.offsets = align_up(s.unique + sizeof(int) * m, 16);
@@ -145,78 +142,101 @@ struct LayerArgs {
   int wait_prior;     // wait for the preceding grid before reading any input
 };
 
-// ------------------------------------------------------------ code decode ---
-// Masks, exponent fields and offsets of the decode.  Masks and exponents are kept
-// in registers (hidden from constant folding) so that each nibble costs exactly
-// one LOP3, (w & mask) | exponent.
-struct DecodeConsts {
-  uint32_t m0, m1, m2, m3, m4;            // 0xF << 4j, j = 0..4
-  uint32_t e150, e146, e142, e138, e134;  // exponent (150 - 4j) << 23
-  float2 c01, c23, c45, c67;
-};
-__device__ __forceinline__ DecodeConsts decode_consts() {
-  DecodeConsts k;
-  k.m0 = 0xFu;
-  k.m1 = 0xF0u;
-  k.m2 = 0xF00u;
-  k.m3 = 0xF000u;
-  k.m4 = 0xF0000u;
-  k.e150 = 150u << 23;
-  k.e146 = 146u << 23;
-  k.e142 = 142u << 23;
-  k.e138 = 138u << 23;
-  k.e134 = 134u << 23;
-  asm volatile("" : "+r"(k.m0), "+r"(k.m1), "+r"(k.m2), "+r"(k.m3), "+r"(k.m4));
-  asm volatile("" : "+r"(k.e150), "+r"(k.e146), "+r"(k.e142), "+r"(k.e138), "+r"(k.e134));
-  k.c01 = make_float2(-8388608.f, -524288.f);
-  k.c23 = make_float2(-32768.f, -2048.f);
-  k.c45 = make_float2(-128.f, -32768.f);
-  k.c67 = make_float2(-2048.f, -128.f);
-  return k;
+// ------------------------------------------------- activations and codes ---
+// A segment's activations (x rows in phase A, h rows in phase B) are held in
+// shared memory as 16-bit block fixed point, one block per 32-column chunk:
+//   x_c = v_c * 2^(e - 14),  v_c an integer in [-32640, 32640],
+// where e is the exponent of the block's largest magnitude.  A bf16 value whose
+// exponent is within 7 of e is held exactly (8 significant bits); smaller ones are
+// rounded to the nearest multiple of 2^(e - 14), an error below 2^-15 of the
+// block's largest magnitude.  v_c is split into a low byte (unsigned) and a high
+// byte (signed), so that a chunk's sum  sum_c q_c v_c  is formed exactly in
+// integers by dp4a over 4-bit codes: the codes of a 32-bit word w are split into
+// qa = w & 0x0F0F0F0F (columns 0, 2, 4, 6 of the word, one per byte) and
+// qb = (w >> 4) & 0x0F0F0F0F (columns 1, 3, 5, 7).
+//
+// Layout: token t, chunk ch = i * 32 + l (l = lane, i < R): uint4
+// xq[((t * R + i) * 4 + m) * 32 + l] covers columns 32 ch + 8m .. +7 as
+//   .x = low bytes of columns 8m+0,2,4,6   .y = low bytes of 8m+1,3,5,7
+//   .z = high bytes of columns 8m+0,2,4,6  .w = high bytes of 8m+1,3,5,7
+// and float2 xsc[t * R * 32 + ch] = (2^(e - 14), sum of the chunk's 32 values).
+constexpr uint32_t kNibbleBytes = 0x0F0F0F0Fu;
+
+__device__ __forceinline__ int dp4a_lo(uint32_t q, uint32_t d, int c) {
+  return static_cast<int>(__dp4a(q, d, static_cast<unsigned>(c)));
+}
+__device__ __forceinline__ int dp4a_hi(uint32_t q, uint32_t d, int c) {
+  return __dp4a(static_cast<int>(q), static_cast<int>(d), c);
 }
 
-// (a & b) | c in one instruction.
-__device__ __forceinline__ float and_or_f(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return __uint_as_float(d);
-}
-
-// 8 codes of `w` (nibble j = element j) -> 4 float2 pairs (q0,q1) (q2,q3) (q4,q5) (q6,q7).
-__device__ __forceinline__ void decode8(uint32_t w, const DecodeConsts& k, float2* q) {
-  const uint32_t w2 = w >> 12;
-  q[0] = __fadd2_rn(make_float2(and_or_f(w, k.m0, k.e150), and_or_f(w, k.m1, k.e146)), k.c01);
-  q[1] = __fadd2_rn(make_float2(and_or_f(w, k.m2, k.e142), and_or_f(w, k.m3, k.e138)), k.c23);
-  q[2] = __fadd2_rn(make_float2(and_or_f(w, k.m4, k.e134), and_or_f(w2, k.m2, k.e142)), k.c45);
-  q[3] = __fadd2_rn(make_float2(and_or_f(w2, k.m3, k.e138), and_or_f(w2, k.m4, k.e134)), k.c67);
-}
-
-// The 32 codes of a uint4 (elements 8i + j = nibble j of word i) as 16 float2 pairs.
-__device__ __forceinline__ void decode32(const uint4 v, const DecodeConsts& k, float2 (&q)[16]) {
-  decode8(v.x, k, &q[0]);
-  decode8(v.y, k, &q[4]);
-  decode8(v.z, k, &q[8]);
-  decode8(v.w, k, &q[12]);
-}
-
-// sum_c q_c x_c over one 32-column chunk: x as 8 float4 (columns 4j..4j+3).
-__device__ __forceinline__ float dot32(const float2 (&q)[16], const float4 (&x)[8]) {
-  float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
+// sum_c q_c v_c over one chunk (4 code words, 4 activation uint4), exact.
+__device__ __forceinline__ int chunk_dot(const uint32_t (&qs)[8], const uint4* xp) {
+  int lo = 0, hi = 0;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    a = __ffma2_rn(q[2 * j], make_float2(x[j].x, x[j].y), a);
-    b = __ffma2_rn(q[2 * j + 1], make_float2(x[j].z, x[j].w), b);
+  for (int m = 0; m < 4; ++m) {
+    const uint4 d = xp[m * 32];
+    lo = dp4a_lo(qs[2 * m], d.x, lo);
+    lo = dp4a_lo(qs[2 * m + 1], d.y, lo);
+    hi = dp4a_hi(qs[2 * m], d.z, hi);
+    hi = dp4a_hi(qs[2 * m + 1], d.w, hi);
   }
-  return (a.x + a.y) + (b.x + b.y);
+  return hi * 256 + lo;  // |.| < 2^24: exact in fp32
 }
 
-// Activation buffer layout: float4 (t, round i, j, lane) at ((t*R + i)*8 + j)*32 + lane
-// holds columns (i*32 + lane)*32 + 4j .. +3; chunk sums at t*R*32 + i*32 + lane.
-__device__ __forceinline__ void load_xchunk(const float4* xs4, int t, int R, int i, int lane,
-                                            float4 (&x)[8]) {
-  const float4* p = xs4 + ((size_t)(t * R + i) * 8) * 32 + lane;
+// The 32 codes of a uint4, split as described above.
+__device__ __forceinline__ void split_codes(const uint4 v, uint32_t (&qs)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int j = 0; j < 8; ++j) x[j] = p[j * 32];
+  for (int m = 0; m < 4; ++m) {
+    qs[2 * m] = w[m] & kNibbleBytes;
+    qs[2 * m + 1] = (w[m] >> 4) & kNibbleBytes;
+  }
+}
+
+// One thread's quarter of a chunk: the 8 bf16 values of columns 8m .. 8m+7 (in v)
+// become this thread's uint4 of the layout above; the 4 threads of a chunk are
+// consecutive lanes (group mask gmask).  Returns the chunk's (scale, sum) in every
+// thread of the group.
+__device__ __forceinline__ float2 fixed_point_quarter(const uint4 v, unsigned gmask,
+                                                      uint4& out) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  int X[8], M[8], neg[8];
+  int xm = 0;
+  float sum = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t b = (k & 1) ? (w[k >> 1] >> 16) : (w[k >> 1] & 0xffffu);
+    const int ex = (b >> 7) & 0xff, mant = b & 0x7f;
+    M[k] = ex ? (mant | 0x80) : mant;
+    X[k] = ex ? ex : 1;
+    neg[k] = (b >> 15) & 1;
+    if (M[k]) xm = max(xm, X[k]);
+    sum += __uint_as_float(b << 16);
+  }
+  xm = max(xm, __shfl_xor_sync(gmask, xm, 1, 4));
+  xm = max(xm, __shfl_xor_sync(gmask, xm, 2, 4));
+  sum += __shfl_xor_sync(gmask, sum, 1, 4);
+  sum += __shfl_xor_sync(gmask, sum, 2, 4);
+  uint32_t lo[2] = {0u, 0u}, hi[2] = {0u, 0u};
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int sh = xm - X[k];  // >= 0 for every nonzero value
+    int mag;
+    if (sh <= 7) mag = M[k] << (7 - sh);
+    else if (sh <= 15) mag = (M[k] + (1 << (sh - 8))) >> (sh - 7);  // round half up
+    else mag = 0;
+    const int val = neg[k] ? -mag : mag;
+    const int pos = (k >> 1) * 8;  // byte within the word; k even -> .x/.z, odd -> .y/.w
+    lo[k & 1] |= (static_cast<uint32_t>(val) & 0xffu) << pos;
+    hi[k & 1] |= ((static_cast<uint32_t>(val) >> 8) & 0xffu) << pos;
+  }
+  out = make_uint4(lo[0], lo[1], hi[0], hi[1]);
+  float scale;
+  if (xm == 0) scale = 0.f;                                    // all zero
+  else if (xm == 255) scale = __uint_as_float(0x7fc00000u);   // Inf / NaN present
+  else if (xm >= 15) scale = __uint_as_float(static_cast<uint32_t>(xm - 14) << 23);
+  else scale = __uint_as_float(1u << (xm + 8));               // 2^(xm-141), subnormal
+  return make_float2(scale, sum);
 }
 
 // ---------------------------------------------------------------- counters ---
@@ -243,14 +263,14 @@ __device__ __forceinline__ bool wait_counter(const unsigned* p, unsigned target)
 
 // --------------------------------------------------------- per-warp compute ---
 // Phase A: this warp's row of Wg and of Wu, NT pairs, R rounds of 32-column chunks
-// (chunks past H/32 skipped); returns (G, U) for t < NT in every lane.
+// (chunks past H/32 skipped); returns (G, U) for t < NT in every lane.  Per chunk
+// (inside one quantisation group): s * 2^(e-14) * sum q v + b * sum x.
 template <int NT, int R>
 __device__ __forceinline__ void rows_a(const unsigned char* bg_q, const uint16_t* bg_s,
                                        const uint16_t* bg_b, const unsigned char* bu_q,
                                        const uint16_t* bu_s, const uint16_t* bu_b, int H,
-                                       const float4* xs4, const float* xsum, int lane,
-                                       const DecodeConsts& k, float (&G)[kNT],
-                                       float (&U)[kNT]) {
+                                       const uint4* xq, const float2* xsc, int lane,
+                                       float (&G)[kNT], float (&U)[kNT]) {
   float ag[NT], au[NT];
 #pragma unroll
   for (int t = 0; t < NT; ++t) ag[t] = au[t] = 0.f;
@@ -259,20 +279,19 @@ __device__ __forceinline__ void rows_a(const unsigned char* bg_q, const uint16_t
   for (int i = 0; i < R; ++i) {
     const int ch = i * 32 + lane;
     if (ch < nch) {
-      const uint4 vg = *reinterpret_cast<const uint4*>(bg_q + ch * 16);
-      const uint4 vu = *reinterpret_cast<const uint4*>(bu_q + ch * 16);
+      uint32_t qg[8], qu[8];
+      split_codes(*reinterpret_cast<const uint4*>(bg_q + ch * 16), qg);
+      split_codes(*reinterpret_cast<const uint4*>(bu_q + ch * 16), qu);
       const float sg = bf16_bits_to_float(bg_s[ch >> 1]), bgv = bf16_bits_to_float(bg_b[ch >> 1]);
       const float su = bf16_bits_to_float(bu_s[ch >> 1]), buv = bf16_bits_to_float(bu_b[ch >> 1]);
-      float2 qg[16], qu[16];
-      decode32(vg, k, qg);
-      decode32(vu, k, qu);
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
-        float4 x[8];
-        load_xchunk(xs4, t, R, i, lane, x);
-        const float xsv = xsum[t * R * 32 + ch];
-        ag[t] += fmaf(sg, dot32(qg, x), bgv * xsv);
-        au[t] += fmaf(su, dot32(qu, x), buv * xsv);
+        const uint4* xp = xq + ((size_t)(t * R + i) * 4) * 32 + lane;
+        const float2 sc = xsc[t * R * 32 + ch];
+        const float dg = static_cast<float>(chunk_dot(qg, xp));
+        const float du = static_cast<float>(chunk_dot(qu, xp));
+        ag[t] = fmaf(sg * sc.x, dg, fmaf(bgv, sc.y, ag[t]));
+        au[t] = fmaf(su * sc.x, du, fmaf(buv, sc.y, au[t]));
       }
     }
   }
@@ -289,14 +308,12 @@ __device__ __forceinline__ void rows_a(const unsigned char* bg_q, const uint16_t
 }
 
 // Phase B: rows row0 + kWarps*q (q < kMaxRowsPerWarpB, rows < nrows) of Wd, NT pairs.
-// Per 32-column round the activations of all NT pairs are loaded once, then each
-// row is decoded once and dotted with them.  Returns the value this lane holds
-// after a reduce-scatter and its index q*kNT + t in `vid` (-1 when it holds none).
+// Returns the value this lane holds after a reduce-scatter and its index
+// q*kNT + t in `vid` (-1 when it holds none).
 template <int NT, int R>
 __device__ __forceinline__ float rows_b(const unsigned char* bq, const uint16_t* bs,
                                         const uint16_t* bb, int row0, int nrows, int I,
-                                        const float4* xs4, const float* xsum, int lane,
-                                        const DecodeConsts& k, int& vid) {
+                                        const uint4* xq, const float2* xsc, int lane, int& vid) {
   constexpr int NP = (NT == 3) ? 4 : NT;
   constexpr int V = kMaxRowsPerWarpB * NP;
   float acc[V];
@@ -307,24 +324,23 @@ __device__ __forceinline__ float rows_b(const unsigned char* bq, const uint16_t*
   for (int i = 0; i < R; ++i) {
     const int ch = i * 32 + lane;
     if (ch < nch) {
-      float4 x[NT][8];
-      float xsv[NT];
+      float2 sc[NT];
 #pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        load_xchunk(xs4, t, R, i, lane, x[t]);
-        xsv[t] = xsum[t * R * 32 + ch];
-      }
+      for (int t = 0; t < NT; ++t) sc[t] = xsc[t * R * 32 + ch];
 #pragma unroll
       for (int q = 0; q < kMaxRowsPerWarpB; ++q) {
         const int r = row0 + kWarps * q;
         if (r < nrows) {
-          const uint4 v = *reinterpret_cast<const uint4*>(bq + (size_t)r * qstride + ch * 16);
-          const float sc = bf16_bits_to_float(bs[r * sstride + (ch >> 1)]);
-          const float bi = bf16_bits_to_float(bb[r * sstride + (ch >> 1)]);
-          float2 qd[16];
-          decode32(v, k, qd);
+          uint32_t qs[8];
+          split_codes(*reinterpret_cast<const uint4*>(bq + (size_t)r * qstride + ch * 16), qs);
+          const float sv = bf16_bits_to_float(bs[r * sstride + (ch >> 1)]);
+          const float bv = bf16_bits_to_float(bb[r * sstride + (ch >> 1)]);
 #pragma unroll
-          for (int t = 0; t < NT; ++t) acc[q * NP + t] += fmaf(sc, dot32(qd, x[t]), bi * xsv[t]);
+          for (int t = 0; t < NT; ++t) {
+            const uint4* xp = xq + ((size_t)(t * R + i) * 4) * 32 + lane;
+            const float d = static_cast<float>(chunk_dot(qs, xp));
+            acc[q * NP + t] = fmaf(sv * sc[t].x, d, fmaf(bv, sc[t].y, acc[q * NP + t]));
+          }
         }
       }
     }
@@ -342,23 +358,22 @@ template <int NT>
 __device__ __forceinline__ void dispatch_a(int R, const unsigned char* bgq, const uint16_t* bgs,
                                            const uint16_t* bgb, const unsigned char* buq,
                                            const uint16_t* bus, const uint16_t* bub, int H,
-                                           const float4* xs4, const float* xsum, int lane,
-                                           const DecodeConsts& k, float (&G)[kNT],
-                                           float (&U)[kNT]) {
-  if (R == 1) rows_a<NT, 1>(bgq, bgs, bgb, buq, bus, bub, H, xs4, xsum, lane, k, G, U);
-  else if (R == 2) rows_a<NT, 2>(bgq, bgs, bgb, buq, bus, bub, H, xs4, xsum, lane, k, G, U);
-  else rows_a<NT, 4>(bgq, bgs, bgb, buq, bus, bub, H, xs4, xsum, lane, k, G, U);
+                                           const uint4* xq, const float2* xsc, int lane,
+                                           float (&G)[kNT], float (&U)[kNT]) {
+  if (R == 1) rows_a<NT, 1>(bgq, bgs, bgb, buq, bus, bub, H, xq, xsc, lane, G, U);
+  else if (R == 2) rows_a<NT, 2>(bgq, bgs, bgb, buq, bus, bub, H, xq, xsc, lane, G, U);
+  else rows_a<NT, 4>(bgq, bgs, bgb, buq, bus, bub, H, xq, xsc, lane, G, U);
 }
 
 template <int NT>
 __device__ __forceinline__ float dispatch_b(int R, const unsigned char* bq, const uint16_t* bs,
                                             const uint16_t* bb, int row0, int nrows, int I,
-                                            const float4* xs4, const float* xsum, int lane,
-                                            const DecodeConsts& k, int& vid) {
-  if (R == 1) return rows_b<NT, 1>(bq, bs, bb, row0, nrows, I, xs4, xsum, lane, k, vid);
-  if (R == 2) return rows_b<NT, 2>(bq, bs, bb, row0, nrows, I, xs4, xsum, lane, k, vid);
-  if (R == 4) return rows_b<NT, 4>(bq, bs, bb, row0, nrows, I, xs4, xsum, lane, k, vid);
-  return rows_b<NT, 8>(bq, bs, bb, row0, nrows, I, xs4, xsum, lane, k, vid);
+                                            const uint4* xq, const float2* xsc, int lane,
+                                            int& vid) {
+  if (R == 1) return rows_b<NT, 1>(bq, bs, bb, row0, nrows, I, xq, xsc, lane, vid);
+  if (R == 2) return rows_b<NT, 2>(bq, bs, bb, row0, nrows, I, xq, xsc, lane, vid);
+  if (R == 4) return rows_b<NT, 4>(bq, bs, bb, row0, nrows, I, xq, xsc, lane, vid);
+  return rows_b<NT, 8>(bq, bs, bb, row0, nrows, I, xq, xsc, lane, vid);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
@@ -476,37 +491,28 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
     if (lane == 0) *a.ex_u = u;
   }
 
-  float4* xs4 = reinterpret_cast<float4*>(smem + L.x);
-  float* xsum = reinterpret_cast<float*>(smem + L.xsum);
-  const DecodeConsts dk = decode_consts();
+  uint4* xq = reinterpret_cast<uint4*>(smem + L.x);
+  float2* xsc = reinterpret_cast<float2*>(smem + L.xsum);
 
-  // Stage a segment's activations (x rows in phase A, h rows in phase B) as fp32 in
-  // the shared buffer, with per-chunk sums.  Whole CTA; called between barriers.
+  // Stage a segment's activations (x rows in phase A, h rows in phase B) in the
+  // block fixed-point layout.  Four consecutive threads share a chunk, one per
+  // 8-column quarter.  Whole CTA; called between barriers.
   auto stage_x = [&](bool phase_b, int sg) {
     const int D = phase_b ? a.I : a.H;
     const int R = phase_b ? G.rounds_b : G.rounds_a;
     const int nch = D / 32, nt = seg_nt[sg], p0 = seg_pos[sg];
-    for (int task = threadIdx.x; task < nt * nch; task += kThreads) {
-      const int t = task / nch, ch = task % nch;
+    const unsigned gmask = 0xfu << (lane & ~3);
+    for (int task = threadIdx.x; task < nt * nch * 4; task += kThreads) {
+      const int m = task & 3, tc = task >> 2, t = tc / nch, ch = tc % nch;
       const uint16_t* row = phase_b ? a.h + (size_t)(p0 + t) * a.I
                                     : a.x + (size_t)(plist[p0 + t] / a.k) * a.H;
-      const uint4* src = reinterpret_cast<const uint4*>(row + ch * 32);
-      uint4 v[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) v[q] = __ldcg(src + q);  // L2: h comes from other CTAs
+      // L2 only: h comes from other CTAs
+      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(row + ch * 32 + m * 8));
+      uint4 packed;
+      const float2 sc = fixed_point_quarter(v, gmask, packed);
       const int i = ch / 32, l = ch % 32;
-      float4* dst = xs4 + ((size_t)(t * R + i) * 8) * 32 + l;
-      float sum = 0.f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t w4[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-        const float4 f0 = make_float4(bf16_lo(w4[0]), bf16_hi(w4[0]), bf16_lo(w4[1]), bf16_hi(w4[1]));
-        const float4 f1 = make_float4(bf16_lo(w4[2]), bf16_hi(w4[2]), bf16_lo(w4[3]), bf16_hi(w4[3]));
-        dst[(2 * q) * 32] = f0;
-        dst[(2 * q + 1) * 32] = f1;
-        sum += (f0.x + f0.y) + (f0.z + f0.w) + (f1.x + f1.y) + (f1.z + f1.w);
-      }
-      xsum[t * R * 32 + ch] = sum;
+      xq[((size_t)(t * R + i) * 4 + m) * 32 + l] = packed;
+      if (m == 0) xsc[t * R * 32 + ch] = sc;
     }
   };
 
@@ -603,19 +609,19 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
       const uint16_t* bus = reinterpret_cast<const uint16_t*>(bu + G.a_q) + warp * (a.H / 64);
       const uint16_t* bub = reinterpret_cast<const uint16_t*>(bu + G.a_q + G.a_sb) + warp * (a.H / 64);
       switch (nt) {
-        case 1: dispatch_a<1>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, xs4, xsum, lane, dk, Gs, Us); break;
-        case 2: dispatch_a<2>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, xs4, xsum, lane, dk, Gs, Us); break;
-        case 3: dispatch_a<3>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, xs4, xsum, lane, dk, Gs, Us); break;
-        default: dispatch_a<4>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, xs4, xsum, lane, dk, Gs, Us); break;
+        case 1: dispatch_a<1>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, xq, xsc, lane, Gs, Us); break;
+        case 2: dispatch_a<2>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, xq, xsc, lane, Gs, Us); break;
+        case 3: dispatch_a<3>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, xq, xsc, lane, Gs, Us); break;
+        default: dispatch_a<4>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, xq, xsc, lane, Gs, Us); break;
       }
     } else if (ok) {
       const uint16_t* bs = reinterpret_cast<const uint16_t*>(buf + G.b_q);
       const uint16_t* bb = reinterpret_cast<const uint16_t*>(buf + G.b_q + G.b_sb);
       switch (nt) {
-        case 1: v = dispatch_b<1>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, xs4, xsum, lane, dk, vid); break;
-        case 2: v = dispatch_b<2>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, xs4, xsum, lane, dk, vid); break;
-        case 3: v = dispatch_b<3>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, xs4, xsum, lane, dk, vid); break;
-        default: v = dispatch_b<4>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, xs4, xsum, lane, dk, vid); break;
+        case 1: v = dispatch_b<1>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, xq, xsc, lane, vid); break;
+        case 2: v = dispatch_b<2>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, xq, xsc, lane, vid); break;
+        case 3: v = dispatch_b<3>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, xq, xsc, lane, vid); break;
+        default: v = dispatch_b<4>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, xq, xsc, lane, vid); break;
       }
     }
     // this warp is done reading stage st; the last warp to get here refills it
