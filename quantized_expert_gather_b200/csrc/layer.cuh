@@ -169,12 +169,20 @@ __device__ __forceinline__ int dp4a_hi(uint32_t q, uint32_t d, int c) {
   return __dp4a(static_cast<int>(q), static_cast<int>(d), c);
 }
 
+// A chunk's activation quarters (token t, round i) into registers.
+__device__ __forceinline__ void load_xq(const uint4* xq, int t, int R, int i, int lane,
+                                        uint4 (&d)[4]) {
+  const uint4* p = xq + ((size_t)(t * R + i) * 4) * 32 + lane;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) d[m] = p[m * 32];
+}
+
 // sum_c q_c v_c over one chunk (4 code words, 4 activation uint4), exact.
-__device__ __forceinline__ int chunk_dot(const uint32_t (&qs)[8], const uint4* xp) {
+__device__ __forceinline__ int chunk_dot(const uint32_t (&qs)[8], const uint4 (&x)[4]) {
   int lo = 0, hi = 0;
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
-    const uint4 d = xp[m * 32];
+    const uint4 d = x[m];
     lo = dp4a_lo(qs[2 * m], d.x, lo);
     lo = dp4a_lo(qs[2 * m + 1], d.y, lo);
     hi = dp4a_hi(qs[2 * m], d.z, hi);
@@ -246,6 +254,10 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   return v;
 }
 
+__device__ __forceinline__ void red_release_gpu(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Spin (bounded) until *p >= target.  Returns false and sets kErrTimeout if the
 // limit runs out.
 __device__ __forceinline__ bool wait_counter(const unsigned* p, unsigned target) {
@@ -286,10 +298,11 @@ __device__ __forceinline__ void rows_a(const unsigned char* bg_q, const uint16_t
       const float su = bf16_bits_to_float(bu_s[ch >> 1]), buv = bf16_bits_to_float(bu_b[ch >> 1]);
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
-        const uint4* xp = xq + ((size_t)(t * R + i) * 4) * 32 + lane;
+        uint4 xd[4];
+        load_xq(xq, t, R, i, lane, xd);
         const float2 sc = xsc[t * R * 32 + ch];
-        const float dg = static_cast<float>(chunk_dot(qg, xp));
-        const float du = static_cast<float>(chunk_dot(qu, xp));
+        const float dg = static_cast<float>(chunk_dot(qg, xd));
+        const float du = static_cast<float>(chunk_dot(qu, xd));
         ag[t] = fmaf(sg * sc.x, dg, fmaf(bgv, sc.y, ag[t]));
         au[t] = fmaf(su * sc.x, du, fmaf(buv, sc.y, au[t]));
       }
@@ -325,8 +338,12 @@ __device__ __forceinline__ float rows_b(const unsigned char* bq, const uint16_t*
     const int ch = i * 32 + lane;
     if (ch < nch) {
       float2 sc[NT];
+      uint4 xd[NT][4];
 #pragma unroll
-      for (int t = 0; t < NT; ++t) sc[t] = xsc[t * R * 32 + ch];
+      for (int t = 0; t < NT; ++t) {
+        sc[t] = xsc[t * R * 32 + ch];
+        load_xq(xq, t, R, i, lane, xd[t]);
+      }
 #pragma unroll
       for (int q = 0; q < kMaxRowsPerWarpB; ++q) {
         const int r = row0 + kWarps * q;
@@ -337,8 +354,7 @@ __device__ __forceinline__ float rows_b(const unsigned char* bq, const uint16_t*
           const float bv = bf16_bits_to_float(bb[r * sstride + (ch >> 1)]);
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
-            const uint4* xp = xq + ((size_t)(t * R + i) * 4) * 32 + lane;
-            const float d = static_cast<float>(chunk_dot(qs, xp));
+            const float d = static_cast<float>(chunk_dot(qs, xd[t]));
             acc[q * NP + t] = fmaf(sv * sc[t].x, d, fmaf(bv, sc[t].y, acc[q * NP + t]));
           }
         }
@@ -376,9 +392,33 @@ __device__ __forceinline__ float dispatch_b(int R, const unsigned char* bq, cons
   return rows_b<NT, 8>(bq, bs, bb, row0, nrows, I, xq, xsc, lane, vid);
 }
 
+// Estimated time of one block, in units of about 100 SM cycles: the larger of the
+// time its bytes take at the SM's share of HBM bandwidth and the time its dequant
+// work takes with nt pairs (measured on B200 for the 4096 / 2048 layer).
+__device__ __forceinline__ unsigned block_cost_a(int nt) { return max(16, 8 + 7 * nt); }
+__device__ __forceinline__ unsigned block_cost_b(int nt) { return max(16, 13 + 6 * nt); }
+
+// Index of the block at which the cumulative cost reaches `target` in a
+// segment-major block list (bpe blocks per segment, prefix sums pre[0..nseg]).
+// Monotone in target, 0 at 0 and nseg * bpe at the total, so consecutive targets
+// cut the list into contiguous, disjoint ranges.
+__device__ inline int cost_to_block(const unsigned* pre, const int* seg_nt, int nseg, int bpe,
+                                    bool phase_b, unsigned target) {
+  if (nseg == 0 || target >= pre[nseg]) return nseg * bpe;
+  int lo = 0, hi = nseg;  // largest s with pre[s] <= target, s < nseg
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (pre[mid] <= target) lo = mid;
+    else hi = mid;
+  }
+  const unsigned per = phase_b ? block_cost_b(seg_nt[lo]) : block_cost_a(seg_nt[lo]);
+  const int r = (int)min((unsigned)bpe, (target - pre[lo]) / per);
+  return lo * bpe + r;
+}
+
 __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ int s_u, s_nseg, s_ncomb;
+  __shared__ int s_u, s_nseg, s_ncomb, s_part[4];
   __shared__ __align__(8) uint64_t full[kStages];
   __shared__ int stage_cnt[kStages];
   const LayerGeom& G = a.g;
@@ -444,13 +484,54 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
   for (int i = threadIdx.x; i < n_valid; i += kThreads) pos_of[plist[i]] = i;
 
   // ---- this CTA's blocks: phase A [a0, a0+na), phase B [b0, b0+nb) ----
+  // Each phase's block list (segment-major) is cut into equal shares of estimated
+  // cost, so that CTAs holding segments with more pairs get fewer blocks.  The
+  // prefix sums live in the stage buffers, which no copy has touched yet.
   const int bpe_a = a.I / kRowsA;
   const int bpe_b = (a.H + G.rows_b - 1) / G.rows_b;
-  const long long na_tot = (long long)nseg * bpe_a, nb_tot = (long long)nseg * bpe_b;
-  const int a0 = (int)(na_tot * blockIdx.x / gridDim.x);
-  const int na = (int)(na_tot * (blockIdx.x + 1) / gridDim.x) - a0;
-  const int b0 = (int)(nb_tot * blockIdx.x / gridDim.x);
-  const int nb = (int)(nb_tot * (blockIdx.x + 1) / gridDim.x) - b0;
+  unsigned* pre_a = reinterpret_cast<unsigned*>(smem + L.stages);
+  unsigned* pre_b = pre_a + (nseg + 1);
+  if (warp == 0) {
+    unsigned run_a = 0, run_b = 0;
+    for (int c0 = 0; c0 < nseg; c0 += 32) {
+      const int sgi = c0 + lane;
+      unsigned ca = 0, cb = 0;
+      if (sgi < nseg) {
+        ca = block_cost_a(seg_nt[sgi]) * (unsigned)bpe_a;
+        cb = block_cost_b(seg_nt[sgi]) * (unsigned)bpe_b;
+      }
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const unsigned va = __shfl_up_sync(kFull, ca, d), vb = __shfl_up_sync(kFull, cb, d);
+        if (lane >= d) {
+          ca += va;
+          cb += vb;
+        }
+      }
+      if (sgi < nseg) {
+        pre_a[sgi + 1] = run_a + ca;
+        pre_b[sgi + 1] = run_b + cb;
+      }
+      run_a += __shfl_sync(kFull, ca, 31);
+      run_b += __shfl_sync(kFull, cb, 31);
+    }
+    if (lane == 0) pre_a[0] = pre_b[0] = 0;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned G_ = gridDim.x, c = blockIdx.x;
+    const unsigned long long ta = pre_a[nseg], tb = pre_b[nseg];
+    const int x0 = cost_to_block(pre_a, seg_nt, nseg, bpe_a, false, (unsigned)(ta * c / G_));
+    const int x1 = cost_to_block(pre_a, seg_nt, nseg, bpe_a, false, (unsigned)(ta * (c + 1) / G_));
+    const int y0 = cost_to_block(pre_b, seg_nt, nseg, bpe_b, true, (unsigned)(tb * c / G_));
+    const int y1 = cost_to_block(pre_b, seg_nt, nseg, bpe_b, true, (unsigned)(tb * (c + 1) / G_));
+    s_part[0] = x0;
+    s_part[1] = x1 - x0;
+    s_part[2] = y0;
+    s_part[3] = y1 - y0;
+  }
+  __syncthreads();
+  const int a0 = s_part[0], na = s_part[1], b0 = s_part[2], nb = s_part[3];
   const int ng = na + nb;
 
   // copy block g of this CTA's sequence into stage g % kStages (one thread)
@@ -481,8 +562,10 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
       bulk_g2s(buf + G.b_q + G.b_sb, a.db + r0 * srow, sb, &full[st]);
     }
   };
-  if (threadIdx.x == 0)
+  if (threadIdx.x == 0) {
+    fence_proxy_async();  // the stage buffers held the prefix sums (generic writes)
     for (int gi = 0; gi < ng && gi < kStages; ++gi) issue(gi);
+  }
 
   if (blockIdx.x == 0 && warp == 1 && a.ex_u) {
     for (int i = lane; i < u; i += 32) a.ex_unique[i] = uniq[i];
@@ -541,14 +624,21 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
   int seg_open = -1, seg_phase = 0, seg_cnt = 0, rb_first = 0;
   auto publish = [&]() {
     if (seg_open < 0) return;
-    __threadfence();  // this thread's h / y stores are visible device-wide
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      s_ncomb = 0;
-      if (seg_phase == 0) atomicAdd(&hdone[seg_open], (unsigned)seg_cnt);
+    __syncthreads();  // every warp's h / y stores of this segment are done
+    if (seg_phase == 0) {
+      // one thread releases the block's stores device-wide (the fence is cumulative
+      // over what the barrier ordered before it) and counts them; nobody waits
+      if (threadIdx.x == 0) {
+        __threadfence();
+        red_release_gpu(&hdone[seg_open], (unsigned)seg_cnt);
+      }
+      seg_open = -1;
+      return;
     }
-    __syncthreads();
-    if (seg_phase == 1 && warp == 0) {  // one lane per row block: the atomics overlap
+    if (warp == 0) {  // one lane per row block: the atomics overlap
+      if (lane == 0) s_ncomb = 0;
+      __syncwarp();
+      __threadfence();
       for (int rb = rb_first + lane; rb < rb_first + seg_cnt; rb += 32) {
         const unsigned old = atomicAdd(&ydone[rb], 1u);
         if (old == (unsigned)nseg - 1) {
