@@ -152,7 +152,7 @@ moe_status moe_switchglu_forward(const uint16_t* x, const int32_t* topk_idx, con
  *   - Set-up: the first call on each device looks up the array's address
  *     (cudaGetSymbolAddress, that device current) and caches it; make that
  *     first call before any stream capture.
- *   - Zeroing: each call clears the counter region (its first 4*1537 bytes)
+ *   - Zeroing: each call clears the counter region (its first 4*1539 bytes)
  *     with cudaMemsetAsync on `stream` before the kernel; nothing else needs
  *     to start at zero.
  *   - Races: all calls on one device share the one array.  Calls that overlap

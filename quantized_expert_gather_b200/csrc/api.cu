@@ -79,7 +79,7 @@ bool shape_supported(int T, int k, int E, int hidden, int inter) {
 }
 
 struct WsLayout {
-  size_t barrier, num_unique, unique, offsets, pair_list, h, y, total;  // barrier = counters
+  size_t barrier, num_unique, unique, offsets, pair_list, h, y, xg, hq, total;  // barrier = counters
 };
 
 WsLayout ws_layout(int T, int k, int E, int hidden, int inter) {
@@ -93,13 +93,19 @@ WsLayout ws_layout(int T, int k, int E, int hidden, int inter) {
   w.pair_list = align_up(w.offsets + 4 * (m + 1), 16);
   w.h = align_up(w.pair_list + 4 * P, 256);
   w.y = align_up(w.h + 2 * P * (size_t)inter, 256);
-  w.total = align_up(w.y + 4 * P * (size_t)hidden, 256);
+  const LayerGeom g = layer_geom(hidden, inter);
+  w.xg = align_up(w.y + 4 * P * (size_t)hidden, 256);     // x rows, fixed point
+  w.hq = align_up(w.xg + (size_t)T * act_bytes(g.rounds_a), 256);  // h rows, fixed point
+  w.total = align_up(w.hq + P * act_bytes(g.rounds_b), 256);
   return w;
 }
 
 int select_path(int T, int k, int E, int hidden, int inter) {
   if (!shape_ok(T, k, E, hidden, inter) || !shape_supported(T, k, E, hidden, inter)) return 0;
-  if (T * k <= kMaxPairsFused) return 1;
+  if (T * k <= kMaxPairsFused) {
+    LayerGeom g = layer_geom(hidden, inter);
+    if (g.seg >= 1 && fit_stages(g, E, T * k, hidden, inter, kSmemBudget)) return 1;
+  }
   return 0;  // the grouped tensor-core path is not available in this build
 }
 
@@ -125,6 +131,8 @@ cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
   a.db = db;
   a.h = reinterpret_cast<uint16_t*>(ws + wl.h);
   a.y = reinterpret_cast<float*>(ws + wl.y);
+  a.xg = ws + wl.xg;
+  a.hq = ws + wl.hq;
   a.sync = reinterpret_cast<unsigned*>(ws + wl.barrier);
   a.ex_u = reinterpret_cast<int*>(ws + wl.num_unique);
   a.ex_unique = reinterpret_cast<int*>(ws + wl.unique);
@@ -138,15 +146,11 @@ cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
   a.I = I;
   a.g = layer_geom(H, I);
   a.wait_prior = 1;
+  if (a.g.seg < 1 || !fit_stages(a.g, E, T * k, H, I, (size_t)d.dyn_smem[0])) {
+    *why = MOE_ERR_UNSUPPORTED;
+    return cudaSuccess;
+  }
   const LayerSmem L = layer_smem(a.g, E, T * k, H, I);
-  if (a.g.seg < 1) {
-    *why = MOE_ERR_UNSUPPORTED;
-    return cudaSuccess;
-  }
-  if (L.total > (size_t)d.dyn_smem[0]) {
-    *why = MOE_ERR_UNSUPPORTED;
-    return cudaSuccess;
-  }
   // One CTA per SM, all resident at once (the kernel has grid barriers); the
   // launch may overlap the tail of the preceding kernel (programmatic launch).
   cudaLaunchAttribute attr[2];
@@ -172,10 +176,10 @@ OwnedWorkspace g_ws[kMaxDevices];
 
 // Fixed scratch for moe_switchglu_forward_static: one copy per device, in the
 // module's global memory (zero at module load), so that entry never allocates.
-// 4 MiB covers T*k <= 128 pairs at hidden 4096 / inter 2048 (2,629,632 bytes
+// 4 MiB covers T*k <= 128 pairs at hidden 4096 / inter 2048 (3,366,912 bytes
 // at T=16, k=8) and every smaller layer.
 constexpr size_t kStaticScratchBytes = MOE_STATIC_SCRATCH_BYTES;
-static_assert(kSyncWords == 1537, "the header states the counter region as 4*1537 bytes");
+static_assert(kSyncWords == 1539, "the header states the counter region as 4*1539 bytes");
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 void* g_static_ptr[kMaxDevices] = {};
 

@@ -8,38 +8,40 @@
 //
 //   prologue  route-union of the window (every CTA forms the same union in
 //             shared memory from topk_idx), cut into segments: an expert and up
-//             to `seg` of its pairs;
-//   phase A   gate+up over blocks (segment, kRowsA rows of Wg and Wu):
+//             to `seg` of its pairs; the CTAs convert the window's x rows to
+//             block fixed point in the workspace, together;
+//   phase A   gate+up over items of 32 rows (segment, rows of Wg and Wu):
 //               h = bf16(silu(bf16(Wg x)) * bf16(Wu x))
 //             (the one-pass epilogue of "Apple7/8 MoE gate and up in one decode
-//             pass", splash PR 45, "What changed"), h stored per pair;
-//   phase B   down over blocks (segment, rows_b rows of Wd): y = Wd h per pair,
-//             stored fp32.  A segment's phase-B blocks start once every phase-A
-//             block of that segment has published its h (counter hdone[seg]);
-//   combine   out[t] = bf16(sum_j w[t,j] * y[t,j]), j ascending, per block of
-//             rows_b output rows, run by the CTA that completes the last segment
-//             of that row block (counter ydone[rb]) -- no grid-wide barrier.
-// Blocks are split evenly over the CTAs.  An expert with more than `seg` pairs
-// in the window forms several segments and is streamed once per segment.
-// Every spin on a counter is bounded (common.cuh); the CTA that finishes last
-// resets the counters, so the workspace counters are zero between calls.
+//             pass", splash PR 45, "What changed"); the item's 32 h values per
+//             pair are one fixed-point chunk, converted at the item's end;
+//   phase B   down over items of rows_b rows of Wd: y = Wd h per pair, fp32.
+//             A segment's phase-B items start once every phase-A item of that
+//             segment has published (counter hdone[seg]);
+//   combine   out[t] = bf16(sum_j w[t,j] * y[t,j]) per block of rows_b output
+//             rows, by CTA (row block mod grid) once every segment of the row
+//             block has published (counter ydone[rb]).
+// Work items are taken from one list (all phase-A items, segment-major, then all
+// phase-B items) through a counter in the workspace, so CTAs stay balanced and a
+// phase-B item's h is normally complete long before the item is taken.  An
+// expert with more than `seg` pairs in the window forms several segments and is
+// streamed once per segment.  Every spin on a counter or barrier is bounded
+// (common.cuh); the counters are zero again when the kernel ends.
 //
-// Memory pipeline: a ring of kStages shared-memory stages fed by 1-D bulk
-// copies (cp.async.bulk, mbarrier completion) runs through phases A and B as
-// one sequence of blocks, so the first phase-B blocks stream while phase A
-// finishes.  Every warp computes; the last warp to finish a stage (shared-memory
-// counter) issues the copy kStages blocks ahead.
+// Warps: 8 compute warps and one producer warp.  The producer takes work items,
+// issues every bulk copy (weights into a ring of stages, activation rows into
+// one of two activation buffers) and publishes finished items; the compute warps
+// wait only on mbarriers and, at the end of a phase-A item, on a named barrier.
 //
 // Compute: each warp owns whole rows (phase A: one row of Wg and the same row
 // of Wu; phase B: up to 4 rows of Wd) over the full input width.  Lane l takes
 // the 32-column chunks l, l+32, ... of its rows, so one lane chunk sits inside
 // one quantisation group (64 columns):
 //     partial = s * sum_c q_c x_c + b * sum_c x_c.
-// The segment's activations sit in shared memory as 16-bit block fixed point
-// (one exponent per 32-column chunk, see below), so that sum_c q_c x_c is an
-// exact integer dot product of the 4-bit codes with the activation's two bytes
-// (dp4a), scaled once per chunk.  A warp reduces its rows over its lanes once per
-// block; there is no cross-warp exchange inside a phase.
+// Activations are 16-bit block fixed point (one exponent per 32-column chunk,
+// see below), so that sum_c q_c x_c is an exact integer dot product of the 4-bit
+// codes with the activation's two bytes (dp4a), scaled once per chunk.  A warp
+// reduces its rows over its lanes once per block.
 #pragma once
 
 #include "common.cuh"
@@ -47,25 +49,39 @@
 
 namespace qeg {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = 32 * kWarps;
+constexpr int kWarps = 8;                    // compute warps
+constexpr int kConsumerThreads = 32 * kWarps;
+constexpr int kThreads = kConsumerThreads + 32;  // + one producer warp
 constexpr int kRowsA = kWarps;      // phase A: one row of gate and of up per warp per block
+constexpr int kBlocksPerItemA = 4;  // phase-A item: 4 blocks = 32 rows = one h chunk
+constexpr int kBlocksPerItemB = 2;  // phase-B item: row blocks
 constexpr int kMaxRowsPerWarpB = 4; // phase B: rows of Wd per warp per block
-constexpr int kStages = 4;          // ring depth
+constexpr int kMaxStages = 4;       // ring depth (fewer when shared memory is short)
 constexpr int kNT = 4;              // pairs per segment (upper bound)
 constexpr int kMaxPairsFused = 1024;
-constexpr unsigned kXBytes = 64 * 1024;  // activation buffer (block fixed point)
+constexpr unsigned kSegActBytes = 36 * 1024;  // one activation buffer (a segment's rows)
+constexpr int kItemRing = 16;       // items between compute and publication
+// Dynamic shared memory the kernel may plan for on B200 (227 KB per block, less a
+// margin for its static shared memory).
+constexpr size_t kSmemBudget = 232448 - 1024;
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Bytes of one activation row in the fixed-point layout (digits, then per-chunk
+// scale and sum; see "activations and codes"), R rounds of 32 chunks.
+__host__ __device__ constexpr unsigned act_bytes(int R) { return 2304u * (unsigned)R; }
+__host__ __device__ constexpr unsigned act_digit_bytes(int R) { return 2048u * (unsigned)R; }
 
 // ---------------------------------------------------------------- geometry ---
 struct LayerGeom {
   int rounds_a, rounds_b;  // 32-column chunks per lane per row (power of two >= H/1024, I/1024)
   int rows_b;              // phase B rows per block (multiple of kWarps, <= 32)
   int seg;                 // pairs per segment (<= kNT)
+  int stages;              // ring depth (<= kMaxStages)
   unsigned a_q, a_sb, a_mat, a_bytes;  // phase A block: per matrix codes / scale bytes
   unsigned b_q, b_sb, b_bytes;         // phase B full block
   unsigned stage_bytes;
+  unsigned act_buf;        // one activation buffer: seg rows of the wider layout
 };
 
 __host__ __device__ inline LayerGeom layer_geom(int H, int I) {
@@ -79,8 +95,9 @@ __host__ __device__ inline LayerGeom layer_geom(int H, int I) {
   if (rb > kWarps * kMaxRowsPerWarpB) rb = kWarps * kMaxRowsPerWarpB;
   g.rows_b = rb;
   const int rmax = g.rounds_a > g.rounds_b ? g.rounds_a : g.rounds_b;
-  int s = (int)(kXBytes / (2048u * (unsigned)rmax));  // fixed point: rounds * 2 KB per pair
+  int s = (int)(kSegActBytes / act_bytes(rmax));
   g.seg = s > kNT ? kNT : s;
+  g.stages = kMaxStages;
   g.a_q = kRowsA * H / 2;
   g.a_sb = kRowsA * H / 32;
   g.a_mat = g.a_q + 2 * g.a_sb;
@@ -89,21 +106,21 @@ __host__ __device__ inline LayerGeom layer_geom(int H, int I) {
   g.b_sb = g.rows_b * I / 32;
   g.b_bytes = g.b_q + 2 * g.b_sb;
   g.stage_bytes = (unsigned)align_up(g.a_bytes > g.b_bytes ? g.a_bytes : g.b_bytes, 128);
+  g.act_buf = (unsigned)align_up((size_t)(g.seg > 0 ? g.seg : 1) * act_bytes(rmax), 128);
   return g;
 }
 
 struct LayerSmem {
-  size_t stages, x, xsum, cnt, rank, unique, offsets, pair_list, pos_of, seg_slot, seg_pos,
-      seg_nt, comb, total;
+  size_t stages, act, hscr, cnt, rank, unique, offsets, pair_list, pos_of, seg_slot, seg_pos,
+      seg_nt, total;
 };
 __host__ __device__ inline LayerSmem layer_smem(const LayerGeom& g, int E, int P, int H, int I) {
   LayerSmem s;
   const int m = (E < P ? E : P) > 0 ? (E < P ? E : P) : 1;
-  const int rmax = g.rounds_a > g.rounds_b ? g.rounds_a : g.rounds_b;
   s.stages = 0;
-  s.x = align_up((size_t)kStages * g.stage_bytes, 128);
-  s.xsum = s.x + kXBytes;
-  s.cnt = align_up(s.xsum + sizeof(float2) * kNT * rmax * 32, 16);
+  s.act = align_up((size_t)g.stages * g.stage_bytes, 128);    // two activation buffers
+  s.hscr = s.act + 2 * (size_t)g.act_buf;                      // h of a phase-A item
+  s.cnt = align_up(s.hscr + sizeof(float) * 2 * kNT * 32, 16);  // two items' h
   s.rank = align_up(s.cnt + sizeof(int) * E, 16);
   s.unique = align_up(s.rank + sizeof(int) * P, 16);
   s.offsets = align_up(s.unique + sizeof(int) * m, 16);
@@ -113,17 +130,30 @@ __host__ __device__ inline LayerSmem layer_smem(const LayerGeom& g, int E, int P
   s.seg_slot = align_up(s.pos_of + sizeof(int) * P, 16);
   s.seg_pos = align_up(s.seg_slot + sizeof(int) * P, 16);
   s.seg_nt = align_up(s.seg_pos + sizeof(int) * P, 16);
-  s.comb = align_up(s.seg_nt + sizeof(int) * P, 16);  // row blocks to combine (<= rows / 8)
-  s.total = align_up(s.comb + sizeof(int) * (H / kWarps + 1), 16);
+  s.total = align_up(s.seg_nt + sizeof(int) * P, 16);
   return s;
+}
+
+// Deepest ring (kMaxStages down to 2) whose shared memory fits in `budget` bytes;
+// false if none does.
+__host__ __device__ inline bool fit_stages(LayerGeom& g, int E, int P, int H, int I,
+                                           size_t budget) {
+  for (int st = kMaxStages; st >= 2; --st) {
+    g.stages = st;
+    if (layer_smem(g, E, P, H, I).total <= budget) return true;
+  }
+  return false;
 }
 
 // Workspace counters (unsigned), a region of fixed size at the start of every
 // workspace so that calls of different shapes never see each other's data there:
 // [0] CTAs finished, [1, 1+kMaxPairsFused) hdone per segment, then ydone per
-// phase-B row block (at most kMaxRowBlocks).
+// phase-B row block (at most kMaxRowBlocks), then the work-item counter and the
+// count of CTAs that have converted their share of x.
 constexpr int kMaxRowBlocks = 4096 / kWarps;
-constexpr size_t kSyncWords = 1 + kMaxPairsFused + kMaxRowBlocks;
+constexpr size_t kSyncWords = 1 + kMaxPairsFused + kMaxRowBlocks + 2;
+constexpr size_t kSyncWorkItem = 1 + kMaxPairsFused + kMaxRowBlocks;
+constexpr size_t kSyncXDone = kSyncWorkItem + 1;
 
 // -------------------------------------------------------------- arguments ---
 struct LayerArgs {
@@ -134,7 +164,9 @@ struct LayerArgs {
   const uint16_t *gs, *gb, *us, *ub, *ds, *db;
   uint16_t* h;        // workspace [P, I] bf16, rows in pair_list order
   float* y;           // workspace [P, H] fp32, rows in pair_list order
-  unsigned* sync;     // workspace counters: [0] exit count, [1..] hdone[P], then ydone[]
+  unsigned char* xg;  // workspace: x rows in the fixed-point layout, [T] x act_bytes(rounds_a)
+  unsigned char* hq;  // workspace: h rows in the fixed-point layout, [P] x act_bytes(rounds_b)
+  unsigned* sync;     // workspace counters (kSyncWords)
   int *ex_u, *ex_unique, *ex_offsets, *ex_pair_list;  // union export (CTA 0), may be null
   uint16_t* out;      // [T, H] bf16
   int T, k, E, H, I;
@@ -155,11 +187,15 @@ struct LayerArgs {
 // qa = w & 0x0F0F0F0F (columns 0, 2, 4, 6 of the word, one per byte) and
 // qb = (w >> 4) & 0x0F0F0F0F (columns 1, 3, 5, 7).
 //
-// Layout: token t, chunk ch = i * 32 + l (l = lane, i < R): uint4
-// xq[((t * R + i) * 4 + m) * 32 + l] covers columns 32 ch + 8m .. +7 as
+// Layout of one activation row (a token's x or a pair's h) of D columns, R rounds
+// (R a power of two >= D / 1024), in act_bytes(R) = 2304 R bytes: for chunk
+// ch = i * 32 + l (i < R, l < 32) the uint4 at index (i * 4 + m) * 32 + l covers
+// columns 32 ch + 8m .. +7 as
 //   .x = low bytes of columns 8m+0,2,4,6   .y = low bytes of 8m+1,3,5,7
 //   .z = high bytes of columns 8m+0,2,4,6  .w = high bytes of 8m+1,3,5,7
-// and float2 xsc[t * R * 32 + ch] = (2^(e - 14), sum of the chunk's 32 values).
+// followed (at byte 2048 R) by float2 sc[ch] = (2^(e - 14), sum of the chunk's 32
+// values).  The same layout serves in global memory (converted once per call) and
+// in shared memory (copied per work item).
 constexpr uint32_t kNibbleBytes = 0x0F0F0F0Fu;
 
 __device__ __forceinline__ int dp4a_lo(uint32_t q, uint32_t d, int c) {
@@ -169,12 +205,16 @@ __device__ __forceinline__ int dp4a_hi(uint32_t q, uint32_t d, int c) {
   return __dp4a(static_cast<int>(q), static_cast<int>(d), c);
 }
 
-// A chunk's activation quarters (token t, round i) into registers.
-__device__ __forceinline__ void load_xq(const uint4* xq, int t, int R, int i, int lane,
+
+// Chunk (round i, lane) of an activation row into registers.
+__device__ __forceinline__ void load_xq(const unsigned char* row, int i, int lane,
                                         uint4 (&d)[4]) {
-  const uint4* p = xq + ((size_t)(t * R + i) * 4) * 32 + lane;
+  const uint4* p = reinterpret_cast<const uint4*>(row) + (i * 4) * 32 + lane;
 #pragma unroll
   for (int m = 0; m < 4; ++m) d[m] = p[m * 32];
+}
+__device__ __forceinline__ float2 load_sc(const unsigned char* row, int R, int ch) {
+  return reinterpret_cast<const float2*>(row + act_digit_bytes(R))[ch];
 }
 
 // sum_c q_c v_c over one chunk (4 code words, 4 activation uint4), exact.
@@ -254,6 +294,12 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   return v;
 }
 
+__device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ void red_release_gpu(unsigned* p, unsigned v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -274,14 +320,15 @@ __device__ __forceinline__ bool wait_counter(const unsigned* p, unsigned target)
 }
 
 // --------------------------------------------------------- per-warp compute ---
-// Phase A: this warp's row of Wg and of Wu, NT pairs, R rounds of 32-column chunks
-// (chunks past H/32 skipped); returns (G, U) for t < NT in every lane.  Per chunk
-// (inside one quantisation group): s * 2^(e-14) * sum q v + b * sum x.
+// Phase A: this warp's row of Wg and of Wu, NT pairs (activation rows act + t *
+// stride), R rounds of 32-column chunks (chunks past H/32 skipped); returns (G, U)
+// for t < NT in every lane.  Per chunk (inside one quantisation group):
+// s * 2^(e-14) * sum q v + b * sum x.
 template <int NT, int R>
 __device__ __forceinline__ void rows_a(const unsigned char* bg_q, const uint16_t* bg_s,
                                        const uint16_t* bg_b, const unsigned char* bu_q,
                                        const uint16_t* bu_s, const uint16_t* bu_b, int H,
-                                       const uint4* xq, const float2* xsc, int lane,
+                                       const unsigned char* act, unsigned stride, int lane,
                                        float (&G)[kNT], float (&U)[kNT]) {
   float ag[NT], au[NT];
 #pragma unroll
@@ -298,9 +345,10 @@ __device__ __forceinline__ void rows_a(const unsigned char* bg_q, const uint16_t
       const float su = bf16_bits_to_float(bu_s[ch >> 1]), buv = bf16_bits_to_float(bu_b[ch >> 1]);
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
+        const unsigned char* row = act + t * stride;
         uint4 xd[4];
-        load_xq(xq, t, R, i, lane, xd);
-        const float2 sc = xsc[t * R * 32 + ch];
+        load_xq(row, i, lane, xd);
+        const float2 sc = load_sc(row, R, ch);
         const float dg = static_cast<float>(chunk_dot(qg, xd));
         const float du = static_cast<float>(chunk_dot(qu, xd));
         ag[t] = fmaf(sg * sc.x, dg, fmaf(bgv, sc.y, ag[t]));
@@ -326,7 +374,8 @@ __device__ __forceinline__ void rows_a(const unsigned char* bg_q, const uint16_t
 template <int NT, int R>
 __device__ __forceinline__ float rows_b(const unsigned char* bq, const uint16_t* bs,
                                         const uint16_t* bb, int row0, int nrows, int I,
-                                        const uint4* xq, const float2* xsc, int lane, int& vid) {
+                                        const unsigned char* act, unsigned stride, int lane,
+                                        int& vid) {
   constexpr int NP = (NT == 3) ? 4 : NT;
   constexpr int V = kMaxRowsPerWarpB * NP;
   float acc[V];
@@ -341,8 +390,9 @@ __device__ __forceinline__ float rows_b(const unsigned char* bq, const uint16_t*
       uint4 xd[NT][4];
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
-        sc[t] = xsc[t * R * 32 + ch];
-        load_xq(xq, t, R, i, lane, xd[t]);
+        const unsigned char* row = act + t * stride;
+        sc[t] = load_sc(row, R, ch);
+        load_xq(row, i, lane, xd[t]);
       }
 #pragma unroll
       for (int q = 0; q < kMaxRowsPerWarpB; ++q) {
@@ -369,71 +419,93 @@ __device__ __forceinline__ float rows_b(const unsigned char* bq, const uint16_t*
   return v;
 }
 
-// ------------------------------------------------------------------ kernel ---
 template <int NT>
 __device__ __forceinline__ void dispatch_a(int R, const unsigned char* bgq, const uint16_t* bgs,
                                            const uint16_t* bgb, const unsigned char* buq,
                                            const uint16_t* bus, const uint16_t* bub, int H,
-                                           const uint4* xq, const float2* xsc, int lane,
+                                           const unsigned char* act, unsigned stride, int lane,
                                            float (&G)[kNT], float (&U)[kNT]) {
-  if (R == 1) rows_a<NT, 1>(bgq, bgs, bgb, buq, bus, bub, H, xq, xsc, lane, G, U);
-  else if (R == 2) rows_a<NT, 2>(bgq, bgs, bgb, buq, bus, bub, H, xq, xsc, lane, G, U);
-  else rows_a<NT, 4>(bgq, bgs, bgb, buq, bus, bub, H, xq, xsc, lane, G, U);
+  if (R == 1) rows_a<NT, 1>(bgq, bgs, bgb, buq, bus, bub, H, act, stride, lane, G, U);
+  else if (R == 2) rows_a<NT, 2>(bgq, bgs, bgb, buq, bus, bub, H, act, stride, lane, G, U);
+  else rows_a<NT, 4>(bgq, bgs, bgb, buq, bus, bub, H, act, stride, lane, G, U);
 }
 
 template <int NT>
 __device__ __forceinline__ float dispatch_b(int R, const unsigned char* bq, const uint16_t* bs,
                                             const uint16_t* bb, int row0, int nrows, int I,
-                                            const uint4* xq, const float2* xsc, int lane,
+                                            const unsigned char* act, unsigned stride, int lane,
                                             int& vid) {
-  if (R == 1) return rows_b<NT, 1>(bq, bs, bb, row0, nrows, I, xq, xsc, lane, vid);
-  if (R == 2) return rows_b<NT, 2>(bq, bs, bb, row0, nrows, I, xq, xsc, lane, vid);
-  if (R == 4) return rows_b<NT, 4>(bq, bs, bb, row0, nrows, I, xq, xsc, lane, vid);
-  return rows_b<NT, 8>(bq, bs, bb, row0, nrows, I, xq, xsc, lane, vid);
+  if (R == 1) return rows_b<NT, 1>(bq, bs, bb, row0, nrows, I, act, stride, lane, vid);
+  if (R == 2) return rows_b<NT, 2>(bq, bs, bb, row0, nrows, I, act, stride, lane, vid);
+  if (R == 4) return rows_b<NT, 4>(bq, bs, bb, row0, nrows, I, act, stride, lane, vid);
+  return rows_b<NT, 8>(bq, bs, bb, row0, nrows, I, act, stride, lane, vid);
 }
 
-// Estimated time of one block, in units of about 100 SM cycles: the larger of the
-// time its bytes take at the SM's share of HBM bandwidth and the time its dequant
-// work takes with nt pairs (measured on B200 for the 4096 / 2048 layer).
-__device__ __forceinline__ unsigned block_cost_a(int nt) { return max(16, 8 + 7 * nt); }
-__device__ __forceinline__ unsigned block_cost_b(int nt) { return max(16, 13 + 6 * nt); }
-
-// Index of the block at which the cumulative cost reaches `target` in a
-// segment-major block list (bpe blocks per segment, prefix sums pre[0..nseg]).
-// Monotone in target, 0 at 0 and nseg * bpe at the total, so consecutive targets
-// cut the list into contiguous, disjoint ranges.
-__device__ inline int cost_to_block(const unsigned* pre, const int* seg_nt, int nseg, int bpe,
-                                    bool phase_b, unsigned target) {
-  if (nseg == 0 || target >= pre[nseg]) return nseg * bpe;
-  int lo = 0, hi = nseg;  // largest s with pre[s] <= target, s < nseg
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (pre[mid] <= target) lo = mid;
-    else hi = mid;
-  }
-  const unsigned per = phase_b ? block_cost_b(seg_nt[lo]) : block_cost_a(seg_nt[lo]);
-  const int r = (int)min((unsigned)bpe, (target - pre[lo]) / per);
-  return lo * bpe + r;
+// mbarrier phase test without suspending (for wait loops that do other work).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, unsigned parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
+// Order this thread's generic-proxy view of global memory (data other CTAs
+// published and this thread acquired) before its following bulk copies.
+__device__ __forceinline__ void fence_proxy_async_all() {
+  asm volatile("fence.proxy.async;" ::: "memory");
+}
+
+// Lane 0's value of a condition, in every lane (keeps the producer warp's control
+// flow uniform when lanes could read a changing value at different times).
+__device__ __forceinline__ bool lane0(bool v) { return __shfl_sync(kFull, v ? 1 : 0, 0) != 0; }
+
+// Ring-slot descriptor flags (slot_info[st].x) for the compute warps.
+constexpr int kSlotEnd = 1;        // no more blocks
+constexpr int kSlotPhaseB = 2;     // a phase-B block
+constexpr int kSlotItemEnd = 4;    // last block of its work item
+constexpr int kSlotActWait = 8;    // first block of an item whose activation rows were loaded
+constexpr int kSlotActPar = 16;    // parity of that load's phase on act_full[ord % kItemRing]
+constexpr int kSlotActShift = 8;   // bits 8..: byte offset / 128 of the item's activation rows
+
+// 9 warps: 8 compute warps and one producer warp (see the top of this file).
+__global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ int s_u, s_nseg, s_ncomb, s_part[4];
-  __shared__ __align__(8) uint64_t full[kStages];
-  __shared__ int stage_cnt[kStages];
+  __shared__ int s_u, s_nseg;
+  __shared__ volatile int s_abort;
+  __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
+  __shared__ __align__(8) uint64_t act_full[kItemRing], item_done[kItemRing], hs_bar[2];
+  __shared__ unsigned long long reg_start[kItemRing];  // activation regions (producer)
+  __shared__ int reg_last[kItemRing];
+  __shared__ int4 item_info[kItemRing];  // per item ordinal: phase B, segment, first block, blocks
+  __shared__ int4 pend[kItemRing];       // queued activation loads (producer)
+  __shared__ int4 slot_info[kMaxStages];  // per ring slot: flags, segment, first row, item ordinal
   const LayerGeom& G = a.g;
   const int P = a.T * a.k;
+  const int NS = G.stages;
   const LayerSmem L = layer_smem(G, a.E, P, a.H, a.I);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned* exit_cnt = a.sync;
   unsigned* hdone = a.sync + 1;
   unsigned* ydone = a.sync + 1 + kMaxPairsFused;
+  unsigned* work_ctr = a.sync + kSyncWorkItem;
+  unsigned* xdone = a.sync + kSyncXDone;
+  const unsigned stride_a = act_bytes(G.rounds_a), stride_b = act_bytes(G.rounds_b);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      stage_cnt[s] = 0;
+      mbar_init(&empty[s], kWarps);
     }
+    for (int i = 0; i < kItemRing; ++i) {
+      mbar_init(&act_full[i], 1);
+      mbar_init(&item_done[i], kWarps);
+    }
+    for (int b = 0; b < 2; ++b) mbar_init(&hs_bar[b], kWarps);
+    s_abort = 0;
     fence_barrier_init();
   }
   if (a.wait_prior) grid_dep_wait();
@@ -446,7 +518,6 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
   int* seg_slot = reinterpret_cast<int*>(smem + L.seg_slot);
   int* seg_pos = reinterpret_cast<int*>(smem + L.seg_pos);
   int* seg_nt = reinterpret_cast<int*>(smem + L.seg_nt);
-  int* comb = reinterpret_cast<int*>(smem + L.comb);
   if (warp == 0) {
     int nv;
     const int u = warp_route_union(a.idx, P, a.E, reinterpret_cast<int*>(smem + L.cnt),
@@ -478,94 +549,31 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
   } else {
     for (int p = threadIdx.x - 32; p < P; p += kThreads - 32) pos_of[p] = -1;
   }
+
+  // ---- x rows in the fixed-point layout, converted by all CTAs together ----
+  {
+    const int nch = a.H / 32, R = G.rounds_a;
+    const long long nq = (long long)a.T * nch * 4;  // quarters of 8 columns
+    for (long long q = (long long)blockIdx.x * kThreads + threadIdx.x; q < nq + 0;
+         q += (long long)gridDim.x * kThreads) {
+      const int m = (int)(q & 3), tc = (int)(q >> 2), t = tc / nch, ch = tc % nch;
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H + ch * 32 + m * 8));
+      uint4 packed;
+      const float2 sc = fixed_point_quarter(v, 0xfu << (lane & ~3), packed);
+      unsigned char* row = a.xg + (size_t)t * stride_a;
+      reinterpret_cast<uint4*>(row)[((ch / 32) * 4 + m) * 32 + (ch % 32)] = packed;
+      if (m == 0) reinterpret_cast<float2*>(row + act_digit_bytes(R))[ch] = sc;
+    }
+  }
   __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    red_release_gpu(xdone, 1u);
+  }
   const int u = s_u, nseg = s_nseg;
   const int n_valid = offs[u];
   for (int i = threadIdx.x; i < n_valid; i += kThreads) pos_of[plist[i]] = i;
-
-  // ---- this CTA's blocks: phase A [a0, a0+na), phase B [b0, b0+nb) ----
-  // Each phase's block list (segment-major) is cut into equal shares of estimated
-  // cost, so that CTAs holding segments with more pairs get fewer blocks.  The
-  // prefix sums live in the stage buffers, which no copy has touched yet.
-  const int bpe_a = a.I / kRowsA;
-  const int bpe_b = (a.H + G.rows_b - 1) / G.rows_b;
-  unsigned* pre_a = reinterpret_cast<unsigned*>(smem + L.stages);
-  unsigned* pre_b = pre_a + (nseg + 1);
-  if (warp == 0) {
-    unsigned run_a = 0, run_b = 0;
-    for (int c0 = 0; c0 < nseg; c0 += 32) {
-      const int sgi = c0 + lane;
-      unsigned ca = 0, cb = 0;
-      if (sgi < nseg) {
-        ca = block_cost_a(seg_nt[sgi]) * (unsigned)bpe_a;
-        cb = block_cost_b(seg_nt[sgi]) * (unsigned)bpe_b;
-      }
-#pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const unsigned va = __shfl_up_sync(kFull, ca, d), vb = __shfl_up_sync(kFull, cb, d);
-        if (lane >= d) {
-          ca += va;
-          cb += vb;
-        }
-      }
-      if (sgi < nseg) {
-        pre_a[sgi + 1] = run_a + ca;
-        pre_b[sgi + 1] = run_b + cb;
-      }
-      run_a += __shfl_sync(kFull, ca, 31);
-      run_b += __shfl_sync(kFull, cb, 31);
-    }
-    if (lane == 0) pre_a[0] = pre_b[0] = 0;
-  }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    const unsigned G_ = gridDim.x, c = blockIdx.x;
-    const unsigned long long ta = pre_a[nseg], tb = pre_b[nseg];
-    const int x0 = cost_to_block(pre_a, seg_nt, nseg, bpe_a, false, (unsigned)(ta * c / G_));
-    const int x1 = cost_to_block(pre_a, seg_nt, nseg, bpe_a, false, (unsigned)(ta * (c + 1) / G_));
-    const int y0 = cost_to_block(pre_b, seg_nt, nseg, bpe_b, true, (unsigned)(tb * c / G_));
-    const int y1 = cost_to_block(pre_b, seg_nt, nseg, bpe_b, true, (unsigned)(tb * (c + 1) / G_));
-    s_part[0] = x0;
-    s_part[1] = x1 - x0;
-    s_part[2] = y0;
-    s_part[3] = y1 - y0;
-  }
-  __syncthreads();
-  const int a0 = s_part[0], na = s_part[1], b0 = s_part[2], nb = s_part[3];
-  const int ng = na + nb;
-
-  // copy block g of this CTA's sequence into stage g % kStages (one thread)
-  auto issue = [&](int gi) {
-    const int st = gi % kStages;
-    unsigned char* buf = smem + L.stages + (size_t)st * G.stage_bytes;
-    if (gi < na) {
-      const int blk = a0 + gi, sg = blk / bpe_a, row0 = (blk % bpe_a) * kRowsA;
-      const size_t r0 = (size_t)uniq[seg_slot[sg]] * a.I + row0;
-      const size_t qrow = a.H / 8, srow = a.H / 64;
-      mbar_arrive_expect_tx(&full[st], G.a_bytes);
-      bulk_g2s(buf, a.gq + r0 * qrow, G.a_q, &full[st]);
-      bulk_g2s(buf + G.a_q, a.gs + r0 * srow, G.a_sb, &full[st]);
-      bulk_g2s(buf + G.a_q + G.a_sb, a.gb + r0 * srow, G.a_sb, &full[st]);
-      buf += G.a_mat;
-      bulk_g2s(buf, a.uq + r0 * qrow, G.a_q, &full[st]);
-      bulk_g2s(buf + G.a_q, a.us + r0 * srow, G.a_sb, &full[st]);
-      bulk_g2s(buf + G.a_q + G.a_sb, a.ub + r0 * srow, G.a_sb, &full[st]);
-    } else {
-      const int blk = b0 + (gi - na), sg = blk / bpe_b, row0 = (blk % bpe_b) * G.rows_b;
-      const int nrows = min(G.rows_b, a.H - row0);
-      const size_t r0 = (size_t)uniq[seg_slot[sg]] * a.H + row0;
-      const size_t qrow = a.I / 8, srow = a.I / 64;
-      const unsigned qb = nrows * (a.I / 2), sb = nrows * (a.I / 32);
-      mbar_arrive_expect_tx(&full[st], qb + 2 * sb);
-      bulk_g2s(buf, a.dq + r0 * qrow, qb, &full[st]);
-      bulk_g2s(buf + G.b_q, a.ds + r0 * srow, sb, &full[st]);
-      bulk_g2s(buf + G.b_q + G.b_sb, a.db + r0 * srow, sb, &full[st]);
-    }
-  };
-  if (threadIdx.x == 0) {
-    fence_proxy_async();  // the stage buffers held the prefix sums (generic writes)
-    for (int gi = 0; gi < ng && gi < kStages; ++gi) issue(gi);
-  }
 
   if (blockIdx.x == 0 && warp == 1 && a.ex_u) {
     for (int i = lane; i < u; i += 32) a.ex_unique[i] = uniq[i];
@@ -574,191 +582,482 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
     if (lane == 0) *a.ex_u = u;
   }
 
-  uint4* xq = reinterpret_cast<uint4*>(smem + L.x);
-  float2* xsc = reinterpret_cast<float2*>(smem + L.xsum);
+  const int bpe_a = a.I / kRowsA;                     // phase-A blocks per segment
+  const int ipa = bpe_a / kBlocksPerItemA;            // phase-A items per segment
+  const int bpe_b = (a.H + G.rows_b - 1) / G.rows_b;  // phase-B blocks per segment
+  const int ipb = (bpe_b + kBlocksPerItemB - 1) / kBlocksPerItemB;  // phase-B items per segment
+  const int n_items_a = nseg * ipa;
+  const int n_items = n_items_a + nseg * ipb;
 
-  // Stage a segment's activations (x rows in phase A, h rows in phase B) in the
-  // block fixed-point layout.  Four consecutive threads share a chunk, one per
-  // 8-column quarter.  Whole CTA; called between barriers.
-  auto stage_x = [&](bool phase_b, int sg) {
-    const int D = phase_b ? a.I : a.H;
-    const int R = phase_b ? G.rounds_b : G.rounds_a;
-    const int nch = D / 32, nt = seg_nt[sg], p0 = seg_pos[sg];
-    const unsigned gmask = 0xfu << (lane & ~3);
-    for (int task = threadIdx.x; task < nt * nch * 4; task += kThreads) {
-      const int m = task & 3, tc = task >> 2, t = tc / nch, ch = tc % nch;
-      const uint16_t* row = phase_b ? a.h + (size_t)(p0 + t) * a.I
-                                    : a.x + (size_t)(plist[p0 + t] / a.k) * a.H;
-      // L2 only: h comes from other CTAs
-      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(row + ch * 32 + m * 8));
-      uint4 packed;
-      const float2 sc = fixed_point_quarter(v, gmask, packed);
-      const int i = ch / 32, l = ch % 32;
-      xq[((size_t)(t * R + i) * 4 + m) * 32 + l] = packed;
-      if (m == 0) xsc[t * R * 32 + ch] = sc;
-    }
-  };
-
-  // out rows of the row blocks comb[0..n) for every token:
-  // sum_j w[t,j] * y[pos(t,j)][c], j ascending.  One flat loop, so the loads of all
-  // row blocks are in flight together.
-  auto combine = [&](int n) {
-    const int per_rb = a.T * G.rows_b;
-    for (int e = threadIdx.x; e < n * per_rb; e += kThreads) {
-      const int rb = comb[e / per_rb], rem = e % per_rb;
-      const int t = rem / G.rows_b, c = rb * G.rows_b + rem % G.rows_b;
-      if (c >= a.H) continue;
-      float acc = 0.f;
-      for (int j = 0; j < a.k; ++j) {
-        const int p = t * a.k + j;
-        const int pos = pos_of[p];
-        if (pos >= 0) acc = fmaf(__ldg(a.w + p), __ldcg(a.y + (size_t)pos * a.H + c), acc);
+  if (warp == kWarps) {
+    // =============================== producer warp ===============================
+    // (every condition is lane 0's, so all lanes take the same path)
+    int pub = 0, n_rec = 0;  // next item ordinal to publish; items recorded
+    auto timed_out = [&](unsigned long long t0) -> bool {
+      if (lane0(s_abort != 0)) return true;
+      if (lane0(globaltimer() - t0 > kWaitLimitNs)) {
+        if (lane == 0) {
+          set_error(kErrTimeout);
+          s_abort = 1;
+        }
+        return true;
       }
-      a.out[(size_t)t * a.H + c] = float_to_bf16_bits(acc);
-    }
-  };
-
-  // Publish the blocks of the segment just finished: phase A adds its block count to
-  // hdone[seg]; phase B adds 1 to ydone[rb] for each of its row blocks, and the CTA
-  // that completes the last segment of a row block combines it.  Whole CTA.
-  int seg_open = -1, seg_phase = 0, seg_cnt = 0, rb_first = 0;
-  auto publish = [&]() {
-    if (seg_open < 0) return;
-    __syncthreads();  // every warp's h / y stores of this segment are done
-    if (seg_phase == 0) {
-      // one thread releases the block's stores device-wide (the fence is cumulative
-      // over what the barrier ordered before it) and counts them; nobody waits
-      if (threadIdx.x == 0) {
-        __threadfence();
-        red_release_gpu(&hdone[seg_open], (unsigned)seg_cnt);
-      }
-      seg_open = -1;
-      return;
-    }
-    if (warp == 0) {  // one lane per row block: the atomics overlap
-      if (lane == 0) s_ncomb = 0;
-      __syncwarp();
-      __threadfence();
-      for (int rb = rb_first + lane; rb < rb_first + seg_cnt; rb += 32) {
-        const unsigned old = atomicAdd(&ydone[rb], 1u);
-        if (old == (unsigned)nseg - 1) {
-          ydone[rb] = 0;  // every segment of this row block is in: reset for the next call
-          comb[atomicAdd(&s_ncomb, 1)] = rb;
+      return false;
+    };
+    // Activation rows live in a circular byte ring: an item's rows occupy a region
+    // [start, start + size) of virtual positions until the last item using them is
+    // published.  Regions are freed in order.
+    const unsigned long long ring = 2ull * G.act_buf;
+    unsigned long long head = 0, tail = 0;
+    int reg_front = 0, reg_cnt = 0;
+    // Publish every recorded item the compute warps have finished, in order.  Their
+    // mbarrier arrivals release their stores at CTA scope and the test here acquires
+    // them; the device-scope release reductions pass them on (causality order is
+    // transitive across the two scopes).
+    auto poll_publish = [&]() {
+      int n = 0;
+      while (pub + n < n_rec &&
+             lane0(mbar_test(&item_done[(pub + n) % kItemRing], ((pub + n) / kItemRing) & 1)))
+        ++n;
+      if (n == 0) return;
+      if (lane == 0) {
+        for (int i = 0; i < n; ++i) {
+          const int4 ii = item_info[(pub + i) % kItemRing];
+          if (ii.x == 0) {
+            red_release_gpu(&hdone[ii.y], (unsigned)(ii.w * 1));
+          } else {
+            for (int r = 0; r < ii.w; ++r) red_release_gpu(&ydone[ii.z + r], 1u);
+          }
         }
       }
-      __threadfence();
-    }
-    __syncthreads();
-    combine(s_ncomb);
-    seg_open = -1;
-  };
+      __syncwarp();
+      pub += n;
+      while (reg_cnt > 0 && reg_last[reg_front] < pub) {  // activation regions no one uses
+        reg_front = (reg_front + 1) % kItemRing;
+        --reg_cnt;
+        tail = reg_cnt > 0 ? reg_start[reg_front] : head;
+      }
+    };
 
-  int cur_seg_key = -1;
-  for (int gi = 0; gi < ng; ++gi) {
-    const bool phase_b = gi >= na;
-    int sg, row0, nrows;
-    if (!phase_b) {
-      const int blk = a0 + gi;
-      sg = blk / bpe_a;
-      row0 = (blk % bpe_a) * kRowsA;
-      nrows = kRowsA;
-    } else {
-      const int blk = b0 + (gi - na);
-      sg = blk / bpe_b;
-      row0 = (blk % bpe_b) * G.rows_b;
-      nrows = min(G.rows_b, a.H - row0);
-    }
-    const int key = (phase_b ? 1 : 0) * kMaxPairsFused + sg;
-    if (key != cur_seg_key) {  // new segment: publish the old one, swap the activations
-      publish();
-      if (phase_b && threadIdx.x == 0) wait_counter(&hdone[sg], (unsigned)bpe_a);
-      __syncthreads();
-      stage_x(phase_b, sg);
-      __syncthreads();
-      cur_seg_key = key;
-      seg_open = sg;
-      seg_phase = phase_b ? 1 : 0;
-      seg_cnt = 0;
-      rb_first = phase_b ? (b0 + (gi - na)) % bpe_b : 0;
-    }
-    ++seg_cnt;
-    const int nt = seg_nt[sg], p0 = seg_pos[sg];
-    const int st = gi % kStages;
-    const bool ok = mbar_wait(&full[st], (gi / kStages) & 1);
-    const unsigned char* buf = smem + L.stages + (size_t)st * G.stage_bytes;
-
-    float Gs[kNT], Us[kNT];
-    float v = 0.f;
-    int vid = -1;
-    if (ok && !phase_b) {
-      const unsigned char* bgq = buf + (size_t)warp * (a.H / 2);
-      const uint16_t* bgs = reinterpret_cast<const uint16_t*>(buf + G.a_q) + warp * (a.H / 64);
-      const uint16_t* bgb = reinterpret_cast<const uint16_t*>(buf + G.a_q + G.a_sb) + warp * (a.H / 64);
-      const unsigned char* bu = buf + G.a_mat;
-      const unsigned char* buq = bu + (size_t)warp * (a.H / 2);
-      const uint16_t* bus = reinterpret_cast<const uint16_t*>(bu + G.a_q) + warp * (a.H / 64);
-      const uint16_t* bub = reinterpret_cast<const uint16_t*>(bu + G.a_q + G.a_sb) + warp * (a.H / 64);
-      switch (nt) {
-        case 1: dispatch_a<1>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, xq, xsc, lane, Gs, Us); break;
-        case 2: dispatch_a<2>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, xq, xsc, lane, Gs, Us); break;
-        case 3: dispatch_a<3>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, xq, xsc, lane, Gs, Us); break;
-        default: dispatch_a<4>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, xq, xsc, lane, Gs, Us); break;
-      }
-    } else if (ok) {
-      const uint16_t* bs = reinterpret_cast<const uint16_t*>(buf + G.b_q);
-      const uint16_t* bb = reinterpret_cast<const uint16_t*>(buf + G.b_q + G.b_sb);
-      switch (nt) {
-        case 1: v = dispatch_b<1>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, xq, xsc, lane, vid); break;
-        case 2: v = dispatch_b<2>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, xq, xsc, lane, vid); break;
-        case 3: v = dispatch_b<3>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, xq, xsc, lane, vid); break;
-        default: v = dispatch_b<4>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, xq, xsc, lane, vid); break;
-      }
-    }
-    // this warp is done reading stage st; the last warp to get here refills it
-    __threadfence_block();
-    __syncwarp();
-    if (lane == 0) {
-      const int done = atomicAdd(&stage_cnt[st], 1);
-      if (done == kWarps - 1) {
-        stage_cnt[st] = 0;
-        __threadfence_block();
-        fence_proxy_async();
-        if (gi + kStages < ng) issue(gi + kStages);
-      }
-    }
-    if (ok && !phase_b) {
-      if (lane < nt) {
-        float gv = 0.f, uv = 0.f;
-#pragma unroll
-        for (int t = 0; t < kNT; ++t)
-          if (t == lane) {
-            gv = Gs[t];
-            uv = Us[t];
+    // Activation loads wait in a queue (in item order) until what they read is
+    // complete: every CTA's x rows (phase A), or the segment's h (phase B), so that
+    // weight copies keep flowing meanwhile.
+    int pend_front = 0, pend_cnt = 0;
+    bool x_ready = false;
+    unsigned act_par = 0;      // per item ring slot: parity of its next load's phase
+    unsigned loaded_mask = 0;  // item ring slots that have had an activation load
+    // pre_ord / pre_val: a counter value for the load of item pre_ord, read earlier
+    // (with acquire), so that the common case costs no round trip here.
+    auto try_flush = [&](int pre_ord, unsigned pre_val) {
+      while (pend_cnt > 0) {
+        const int4 pe = pend[pend_front];  // (ord, sg, byte offset, phase B)
+        const int sg = pe.y, nt = seg_nt[pe.y], p0 = seg_pos[pe.y];
+        const unsigned need = pe.w ? (unsigned)bpe_a : gridDim.x;
+        if (pe.w || !x_ready) {
+          const unsigned* ctr = pe.w ? &hdone[sg] : xdone;
+          const bool pre_ok = pe.x == pre_ord && pre_val >= need;
+          if (!pre_ok && !lane0(ld_acquire_gpu(ctr) >= need)) return;
+          if (!pe.w) x_ready = true;
+        }
+        if (lane == 0) {
+          uint64_t* bar = &act_full[pe.x % kItemRing];
+          unsigned char* dst = smem + L.act + pe.z;
+          fence_proxy_async_all();  // rows other CTAs wrote, read by the bulk copy
+          if (pe.w) {
+            const unsigned size = (unsigned)nt * stride_b;
+            mbar_arrive_expect_tx(bar, size);
+            bulk_g2s(dst, a.hq + (size_t)p0 * stride_b, size, bar);
+          } else {
+            mbar_arrive_expect_tx(bar, (unsigned)nt * stride_a);
+            for (int t = 0; t < nt; ++t)
+              bulk_g2s(dst + (size_t)t * stride_a,
+                       a.xg + (size_t)(plist[p0 + t] / a.k) * stride_a, stride_a, bar);
           }
-        const float g = round_to_bf16(gv), hu = round_to_bf16(uv);
-        const float hv = g / (1.0f + __expf(-g)) * hu;
-        a.h[(size_t)(p0 + lane) * a.I + row0 + warp] = float_to_bf16_bits(hv);
+        }
+        __syncwarp();
+        pend_front = (pend_front + 1) % kItemRing;
+        --pend_cnt;
       }
-    } else if (ok && vid >= 0) {
-      const int r = warp + kWarps * (vid / kNT), t = vid % kNT;
-      if (r < nrows) a.y[(size_t)(p0 + t) * a.H + row0 + r] = v;
+    };
+    auto wait_bar = [&](uint64_t* bar, unsigned parity) -> bool {
+      const unsigned long long t0 = globaltimer();
+      while (!lane0(mbar_test(bar, parity))) {
+        poll_publish();
+        try_flush(-1, 0);
+        if (timed_out(t0)) return false;
+        __nanosleep(64);  // leave issue slots to the compute warps
+      }
+      return true;
+    };
+
+    bool ok = true;
+    int gi = 0;                     // blocks issued into the ring
+    int cur_key = -1;               // activation set of the newest region
+    int cur_tok[kNT] = {-1, -1, -1, -1};
+    unsigned cur_off = 0;           // its byte offset in the ring
+    unsigned long long cur_start = 0;  // and its virtual position
+    int n_a_items = 0;              // phase-A items taken (scratch buffer parity)
+    // Items are taken two ahead: q1 is the next item (its counter c1, the one its
+    // activation load depends on, read one item early) and q2's atomic is in flight.
+    // Lane 0 holds the values.
+    auto dep_counter = [&](unsigned it) -> const unsigned* {
+      if ((int)it >= n_items) return nullptr;
+      if ((int)it < n_items_a) return x_ready ? nullptr : xdone;
+      return &hdone[((int)it - n_items_a) / ipb];
+    };
+    unsigned q0 = 0, q1 = 0, q2 = 0, c0 = 0, c1 = 0;
+    if (lane == 0) {
+      q0 = atomicAdd(work_ctr, 1u);
+      q1 = atomicAdd(work_ctr, 1u);
+      const unsigned* d0 = dep_counter(q0);
+      c0 = d0 ? ld_acquire_gpu(d0) : 0u;
+    }
+    for (int ord = 0; ok; ++ord) {
+      const int item = (int)__shfl_sync(kFull, q0, 0);
+      if (item >= n_items) break;
+      if (lane == 0) {
+        q2 = atomicAdd(work_ctr, 1u);
+        const unsigned* d1 = dep_counter(q1);
+        c1 = d1 ? ld_acquire_gpu(d1) : 0u;
+      }
+      const unsigned pre_val = __shfl_sync(kFull, c0, 0);
+      const bool phase_b = item >= n_items_a;
+      int sg, blk0, nblk;
+      if (!phase_b) {
+        sg = item / ipa;
+        blk0 = (item % ipa) * kBlocksPerItemA;
+        nblk = kBlocksPerItemA;
+      } else {
+        sg = (item - n_items_a) / ipb;
+        blk0 = ((item - n_items_a) % ipb) * kBlocksPerItemB;
+        nblk = min(kBlocksPerItemB, bpe_b - blk0);
+      }
+      const int nt = seg_nt[sg], p0 = seg_pos[sg];
+      // ---- its ring slot for publication (and for a pending load) must be free ----
+      {
+        const unsigned long long t0 = globaltimer();
+        while (ok && (pub <= ord - kItemRing || pend_cnt >= kItemRing)) {
+          poll_publish();
+          try_flush(-1, 0);
+          __nanosleep(64);
+          if ((pub <= ord - kItemRing || pend_cnt >= kItemRing) && timed_out(t0)) ok = false;
+        }
+      }
+      if (!ok) break;
+      // ---- the item's activation rows: the newest region again, or a new one ----
+      bool same = false;
+      if (!phase_b) {
+        same = cur_key == -2;
+        for (int t = 0; t < kNT; ++t)
+          same = same && cur_tok[t] == (t < nt ? plist[p0 + t] / a.k : -1);
+      } else {
+        same = cur_key == sg;
+      }
+      bool act_wait = false, load_par = false;
+      if (same) {  // extend the newest region's life (it may already have been freed)
+        if (lane == 0) {
+          const int r = (reg_front + reg_cnt + (reg_cnt == 0 ? 0 : -1) + kItemRing) % kItemRing;
+          if (reg_cnt == 0) reg_start[r] = cur_start;
+          reg_last[r] = ord;
+        }
+        __syncwarp();
+        if (reg_cnt == 0) {
+          tail = cur_start;
+          reg_cnt = 1;
+        }
+      } else {
+        const unsigned size = (unsigned)nt * (phase_b ? stride_b : stride_a);
+        unsigned long long start = 0;
+        {
+          const unsigned long long t0 = globaltimer();
+          for (;;) {
+            start = head;
+            if (start % ring + size > ring) start = (start / ring + 1) * ring;  // no wrap
+            if (start + size - tail <= ring && reg_cnt < kItemRing) break;
+            poll_publish();
+            try_flush(-1, 0);
+            if (timed_out(t0)) {
+              ok = false;
+              break;
+            }
+            __nanosleep(64);
+          }
+        }
+        if (!ok) break;
+        cur_off = (unsigned)(start % ring);
+        cur_start = start;
+        if (lane == 0) {
+          const int r = (reg_front + reg_cnt) % kItemRing;
+          reg_start[r] = start;
+          reg_last[r] = ord;
+          pend[(pend_front + pend_cnt) % kItemRing] = make_int4(ord, sg, (int)cur_off, phase_b ? 1 : 0);
+        }
+        __syncwarp();
+        if (reg_cnt == 0) tail = start;
+        ++reg_cnt;
+        head = start + size;
+        ++pend_cnt;
+        loaded_mask |= 1u << (ord % kItemRing);
+        load_par = (act_par >> (ord % kItemRing)) & 1u;
+        act_par ^= 1u << (ord % kItemRing);
+        act_wait = true;
+        cur_key = phase_b ? sg : -2;
+        for (int t = 0; t < kNT; ++t) cur_tok[t] = (!phase_b && t < nt) ? plist[p0 + t] / a.k : -1;
+      }
+      // ---- the item's record for publication ----
+      if (lane == 0) item_info[ord % kItemRing] = make_int4(phase_b ? 1 : 0, sg, blk0, nblk);
+      __syncwarp();
+      const int a_ord = phase_b ? 0 : n_a_items++;
+      if (act_wait) try_flush(ord, pre_val);  // at once when the early read shows it ready
+      // ---- its blocks into the ring ----
+      for (int j = 0; j < nblk && ok; ++j, ++gi) {
+        const int st = gi % NS;
+        if (gi >= NS) ok = wait_bar(&empty[st], ((gi / NS) - 1) & 1);
+        if (!ok) break;
+        if (lane == 0) {
+          const int blk = blk0 + j;
+          const int row0 = phase_b ? blk * G.rows_b : blk * kRowsA;
+          const int flags = (phase_b ? kSlotPhaseB : 0) | (j == nblk - 1 ? kSlotItemEnd : 0) |
+                            (j == 0 && act_wait ? kSlotActWait : 0) |
+                            (load_par ? kSlotActPar : 0) |
+                            (int)((cur_off >> 7) << kSlotActShift);
+          slot_info[st] = make_int4(flags, sg, row0, ord | (a_ord << 16));
+          unsigned char* buf = smem + L.stages + (size_t)st * G.stage_bytes;
+          fence_proxy_async();
+          if (!phase_b) {
+            const size_t r0 = (size_t)uniq[seg_slot[sg]] * a.I + row0;
+            const size_t qrow = a.H / 8, srow = a.H / 64;
+            mbar_arrive_expect_tx(&full[st], G.a_bytes);
+            bulk_g2s(buf, a.gq + r0 * qrow, G.a_q, &full[st]);
+            bulk_g2s(buf + G.a_q, a.gs + r0 * srow, G.a_sb, &full[st]);
+            bulk_g2s(buf + G.a_q + G.a_sb, a.gb + r0 * srow, G.a_sb, &full[st]);
+            buf += G.a_mat;
+            bulk_g2s(buf, a.uq + r0 * qrow, G.a_q, &full[st]);
+            bulk_g2s(buf + G.a_q, a.us + r0 * srow, G.a_sb, &full[st]);
+            bulk_g2s(buf + G.a_q + G.a_sb, a.ub + r0 * srow, G.a_sb, &full[st]);
+          } else {
+            const int nrows = min(G.rows_b, a.H - row0);
+            const size_t r0 = (size_t)uniq[seg_slot[sg]] * a.H + row0;
+            const size_t qrow = a.I / 8, srow = a.I / 64;
+            const unsigned qb = nrows * (a.I / 2), sb = nrows * (a.I / 32);
+            mbar_arrive_expect_tx(&full[st], qb + 2 * sb);
+            bulk_g2s(buf, a.dq + r0 * qrow, qb, &full[st]);
+            bulk_g2s(buf + G.b_q, a.ds + r0 * srow, sb, &full[st]);
+            bulk_g2s(buf + G.b_q + G.b_sb, a.db + r0 * srow, sb, &full[st]);
+          }
+        }
+        __syncwarp();
+      }
+      n_rec = ord + 1;
+      if (ok) poll_publish();
+      if (lane == 0) {
+        q0 = q1;
+        c0 = c1;
+        q1 = q2;
+      }
+    }
+    // ---- pending loads, the end marker, then publish what is left (bounded) ----
+    {
+      const unsigned long long t0 = globaltimer();
+      while (ok && pend_cnt > 0) {
+        poll_publish();
+        try_flush(-1, 0);
+        __nanosleep(64);
+        if (pend_cnt > 0 && timed_out(t0)) ok = false;
+      }
+    }
+    if (ok) {
+      const int st = gi % NS;
+      if (gi >= NS) ok = wait_bar(&empty[st], ((gi / NS) - 1) & 1);
+      if (ok && lane == 0) {
+        slot_info[st] = make_int4(kSlotEnd, 0, 0, 0);
+        mbar_arrive(&full[st]);
+      }
+      __syncwarp();
+    }
+    {
+      const unsigned long long t0 = globaltimer();
+      while (ok && pub < n_rec) {
+        poll_publish();
+        if (pub < n_rec && timed_out(t0)) ok = false;
+      }
+    }
+    // copies still in flight after an abort land before the CTA exits (bounded)
+    if (!ok && lane == 0) {
+      for (int g = (gi > NS ? gi - NS : 0); g < gi; ++g) {
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_test(&full[g % NS], (g / NS) & 1) && globaltimer() - t0 < kWaitLimitNs) {
+        }
+      }
+      for (int sl = 0; sl < kItemRing; ++sl)
+        if (loaded_mask & (1u << sl)) {  // the slot's latest load (its phase parity)
+          const unsigned par = ((act_par >> sl) & 1u) ^ 1u;
+          const unsigned long long t0 = globaltimer();
+          while (!mbar_test(&act_full[sl], par) && globaltimer() - t0 < kWaitLimitNs) {
+          }
+        }
+    }
+    __syncwarp();
+  } else {
+    // ================================ compute warps ================================
+    float* hscr = reinterpret_cast<float*>(smem + L.hscr);  // [2][kNT][32]
+    auto wait_cons = [&](uint64_t* bar, unsigned parity) -> bool {
+      if (s_abort) return false;
+      const unsigned long long t0 = globaltimer();
+      while (!mbar_try_wait(bar, parity)) {
+        if (s_abort) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+          set_error(kErrTimeout);
+          s_abort = 1;
+          return false;
+        }
+      }
+      return true;
+    };
+    for (int gi = 0;; ++gi) {
+      const int st = gi % NS;
+      if (!wait_cons(&full[st], (gi / NS) & 1)) break;
+      const int4 si = slot_info[st];
+      if (si.x & kSlotEnd) break;
+      const bool phase_b = (si.x & kSlotPhaseB) != 0;
+      const int sg = si.y, row0 = si.z, ord = si.w & 0xffff, a_ord = si.w >> 16;
+      if ((si.x & kSlotActWait) &&
+          !wait_cons(&act_full[ord % kItemRing], (si.x & kSlotActPar) ? 1u : 0u))
+        break;
+      const int nt = seg_nt[sg], p0 = seg_pos[sg];
+      const unsigned char* act = smem + L.act + ((size_t)(si.x >> kSlotActShift) << 7);
+      const unsigned char* buf = smem + L.stages + (size_t)st * G.stage_bytes;
+      float Gs[kNT], Us[kNT];
+      float v = 0.f;
+      int vid = -1, nrows = 0;
+      if (!phase_b) {
+        const unsigned char* bgq = buf + (size_t)warp * (a.H / 2);
+        const uint16_t* bgs = reinterpret_cast<const uint16_t*>(buf + G.a_q) + warp * (a.H / 64);
+        const uint16_t* bgb = reinterpret_cast<const uint16_t*>(buf + G.a_q + G.a_sb) + warp * (a.H / 64);
+        const unsigned char* bu = buf + G.a_mat;
+        const unsigned char* buq = bu + (size_t)warp * (a.H / 2);
+        const uint16_t* bus = reinterpret_cast<const uint16_t*>(bu + G.a_q) + warp * (a.H / 64);
+        const uint16_t* bub = reinterpret_cast<const uint16_t*>(bu + G.a_q + G.a_sb) + warp * (a.H / 64);
+        switch (nt) {
+          case 1: dispatch_a<1>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, act, stride_a, lane, Gs, Us); break;
+          case 2: dispatch_a<2>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, act, stride_a, lane, Gs, Us); break;
+          case 3: dispatch_a<3>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, act, stride_a, lane, Gs, Us); break;
+          default: dispatch_a<4>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, act, stride_a, lane, Gs, Us); break;
+        }
+      } else {
+        nrows = min(G.rows_b, a.H - row0);
+        const uint16_t* bs = reinterpret_cast<const uint16_t*>(buf + G.b_q);
+        const uint16_t* bb = reinterpret_cast<const uint16_t*>(buf + G.b_q + G.b_sb);
+        switch (nt) {
+          case 1: v = dispatch_b<1>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
+          case 2: v = dispatch_b<2>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
+          case 3: v = dispatch_b<3>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
+          default: v = dispatch_b<4>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
+        }
+      }
+      // this warp is done reading stage st
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+      const bool item_end = (si.x & kSlotItemEnd) != 0;
+      if (!phase_b) {
+        float* hs = hscr + (a_ord & 1) * (kNT * 32);
+        if (lane < nt) {
+          float gv = 0.f, uv = 0.f;
+#pragma unroll
+          for (int t = 0; t < kNT; ++t)
+            if (t == lane) {
+              gv = Gs[t];
+              uv = Us[t];
+            }
+          const float g = round_to_bf16(gv), hu = round_to_bf16(uv);
+          const uint16_t hb = float_to_bf16_bits(g / (1.0f + __expf(-g)) * hu);
+          a.h[(size_t)(p0 + lane) * a.I + row0 + warp] = hb;
+          hs[lane * 32 + (row0 & 31) + warp] = bf16_bits_to_float(hb);
+        }
+        if (item_end) {
+          // the item's 32 h rows per pair are one chunk of h: one warp (in turn) converts it
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&hs_bar[a_ord & 1]);
+          if (warp == (a_ord & (kWarps - 1)) && wait_cons(&hs_bar[a_ord & 1], (a_ord >> 1) & 1)) {
+            if (lane < nt * 4) {
+              const int t = lane >> 2, m = lane & 3;
+              const float* src = hs + t * 32 + m * 8;
+              uint32_t wv[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                wv[e] = (uint32_t)float_to_bf16_bits(src[2 * e]) |
+                        ((uint32_t)float_to_bf16_bits(src[2 * e + 1]) << 16);
+              uint4 packed;
+              const float2 sc = fixed_point_quarter(make_uint4(wv[0], wv[1], wv[2], wv[3]),
+                                                    0xfu << (lane & ~3), packed);
+              const int ch = row0 / 32, R = G.rounds_b;
+              unsigned char* row = a.hq + (size_t)(p0 + t) * stride_b;
+              reinterpret_cast<uint4*>(row)[((ch / 32) * 4 + m) * 32 + (ch % 32)] = packed;
+              if (m == 0) reinterpret_cast<float2*>(row + act_digit_bytes(R))[ch] = sc;
+            }
+          }
+        }
+      } else if (vid >= 0) {
+        const int r = warp + kWarps * (vid / kNT), t = vid % kNT;
+        if (r < nrows) a.y[(size_t)(p0 + t) * a.H + row0 + r] = v;
+      }
+      if (item_end) {  // this warp's stores of the item are done (released at CTA scope)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&item_done[ord % kItemRing]);
+      }
     }
   }
-  publish();
-  if (nseg == 0) {  // nothing routed anywhere valid: every output row is zero
-    const long long total = (long long)a.T * a.H;
-    const long long o0 = total * blockIdx.x / gridDim.x, o1 = total * (blockIdx.x + 1) / gridDim.x;
-    for (long long o = o0 + threadIdx.x; o < o1; o += kThreads) a.out[o] = 0;
+
+  // ---- combine: row blocks blockIdx.x, blockIdx.x + grid, ... once complete ----
+  // out[t][c] = bf16(sum_j w[t,j] * y[pos(t,j)][c]): a group of gk lanes (gk = k
+  // rounded up to a power of two, at most 32) per output, lane j of the group
+  // taking pairs j, j+gk, ...; the group sums in a fixed shuffle order.
+  __syncthreads();
+  {
+    const int n_rb = (a.H + G.rows_b - 1) / G.rows_b;
+    int gk = 1;
+    while (gk < a.k && gk < 32) gk <<= 1;
+    const int gl = lane & (gk - 1);
+    const int per_rb = a.T * G.rows_b;
+    const int groups = kThreads / gk;
+    for (int rb = blockIdx.x; rb < n_rb; rb += gridDim.x) {
+      if (threadIdx.x == 0) {
+        const unsigned long long t0 = globaltimer();
+        while (!s_abort && ld_acquire_gpu(&ydone[rb]) < (unsigned)nseg) {
+          if (globaltimer() - t0 > kWaitLimitNs) {
+            set_error(kErrTimeout);
+            s_abort = 1;
+          }
+        }
+        __threadfence();
+      }
+      __syncthreads();
+      for (int o0 = 0; o0 < per_rb; o0 += groups) {  // uniform trip count: every lane shuffles
+        const int o = o0 + (int)threadIdx.x / gk;
+        const int t = o / G.rows_b, c = rb * G.rows_b + o % G.rows_b;
+        const bool valid = o < per_rb && c < a.H;
+        float acc = 0.f;
+        if (valid)
+          for (int j = gl; j < a.k; j += gk) {
+            const int p = t * a.k + j;
+            const int pos = pos_of[p];
+            if (pos >= 0) acc = fmaf(__ldg(a.w + p), __ldcg(a.y + (size_t)pos * a.H + c), acc);
+          }
+        for (int m = gk >> 1; m >= 1; m >>= 1) acc += __shfl_xor_sync(kFull, acc, m);
+        if (valid && gl == 0) a.out[(size_t)t * a.H + c] = float_to_bf16_bits(acc);
+      }
+      if (threadIdx.x == 0) ydone[rb] = 0;  // for the next call
+    }
   }
   grid_dep_launch();
-
-  // ---- the CTA that finishes last resets the per-segment counters ----
-  __syncthreads();
+  // ---- the CTA that finishes last resets the other counters ----
   if (threadIdx.x == 0) {
     __threadfence();
     const unsigned old = atomicAdd(exit_cnt, 1u);
     if (old == gridDim.x - 1) {
       for (int sgi = 0; sgi < nseg; ++sgi) hdone[sgi] = 0;
+      *work_ctr = 0;
+      *xdone = 0;
       *exit_cnt = 0;
       __threadfence();
     }
