@@ -432,6 +432,52 @@ def our_arm(args, world, rank, local):
         per[T]["graph_gbs"] = sum(uq[T]) * BYTES_PER_EXPERT / LAYERS / (us * 1e-6) / 1e9
         del g2
 
+    # speculative-verify pair (E=256, p=0.34): a T=2 window against its first token
+    # alone, 42 chained layers each, CUDA graph; the target is T=2 <= 1.7 x T=1
+    verify = None
+    if not args.no_verify_pair:
+        E2 = 256
+        def mat2(rows, cols, mid):
+            q = torch.empty((E2, rows, cols // 8), dtype=torch.int32, device=dev)
+            s_ = torch.empty((E2, rows, cols // 64), dtype=torch.int16, device=dev)
+            b_ = torch.empty_like(s_)
+            synth.fill_bank_device(q, s_, b_, rows, cols, SEED + 1, mid)
+            return q, s_.view(torch.bfloat16), b_.view(torch.bfloat16)
+        bank2 = qeg.QuantBank(*mat2(INTER, HIDDEN, 0), *mat2(INTER, HIDDEN, 1),
+                              *mat2(HIDDEN, INTER, 2))
+        pairs = [synth.route_verify_pair(E2, K_TOP, 0.34, SEED + 500 + l) for l in range(LAYERS)]
+        x2 = torch.from_numpy(synth.x_bf16(2, HIDDEN, SEED + 2).view(np.int16)).to(dev) \
+            .view(torch.bfloat16)
+        ws2 = torch.zeros(qeg.moe_workspace_size(2, K_TOP, E2, HIDDEN, INTER), dtype=torch.uint8,
+                          device=dev)
+        runs = {}
+        for T2 in (1, 2):
+            ids = [torch.from_numpy(np.ascontiguousarray(r[0][:T2])).to(dev) for r in pairs]
+            wv = [torch.from_numpy(np.ascontiguousarray(r[1][:T2])).to(dev) for r in pairs]
+            o2 = [torch.empty((T2, HIDDEN), dtype=torch.bfloat16, device=dev) for _ in pairs]
+            xs2 = x2[:T2]
+            for l in range(LAYERS):  # warm, outside capture
+                qeg.moe_switchglu_forward_ws(xs2, ids[l], wv[l], bank2, ws2, out=o2[l])
+            g3 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g3):
+                for l in range(LAYERS):
+                    qeg.moe_switchglu_forward_ws(xs2, ids[l], wv[l], bank2, ws2, out=o2[l])
+            g3.replay()
+            a3, b3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a3.record()
+            for _ in range(5):
+                g3.replay()
+            b3.record()
+            torch.cuda.synchronize()
+            runs[T2] = a3.elapsed_time(b3) * 1e3 / (5 * LAYERS)
+            del g3
+        u2 = float(np.mean([np.unique(r[0]).size for r in pairs]))
+        verify = {"E": E2, "p": 0.34, "t1_us_per_layer": runs[1], "t2_us_per_layer": runs[2],
+                  "ratio_t2_over_t1": runs[2] / runs[1], "target_ratio": 1.7,
+                  "mean_unique_t2": u2,
+                  "t2_gbs": u2 * BYTES_PER_EXPERT / (runs[2] * 1e-6) / 1e9}
+        del bank2, ws2
+
     # end to end through the public call: pinned host inputs in, outputs back, each step
     pin_x = {T: torch.from_numpy(synth.x_bf16(T, HIDDEN, SEED + T).view(np.int16)).pin_memory()
              for T in TS}
@@ -519,6 +565,7 @@ def our_arm(args, world, rank, local):
                     "d2h_bytes_per_step": int(d2h),
                     "how": "moe_switchglu_forward per layer, pinned host inputs copied in and "
                            "all layer outputs copied back every step"},
+            "verify_pair": verify,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
         }
@@ -537,6 +584,8 @@ def main():
     ap.add_argument("--layers", type=int, default=42, help="chained layers per T (profiling)")
     ap.add_argument("--experts", type=int, default=288, help="bank size (profiling)")
     ap.add_argument("--quick", action="store_true", help="timed graph only (profiling)")
+    ap.add_argument("--no-verify-pair", action="store_true",
+                    help="skip the T=2 / T=1 speculative-verify measurement")
     ap.add_argument("--ts", default="", help="comma-separated window sizes (profiling)")
     ap.add_argument("--routing", default="uniform", choices=("uniform", "markov"),
                     help="routing model (profiling)")
