@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "layer.cuh"
 #include "route_union.cuh"
+#include "grouped.cuh"
 
 namespace qeg {
 namespace {
@@ -21,7 +22,8 @@ struct DeviceInfo {
   bool ready = false;
   int sms = 0;
   int smem_optin = 0;
-  int dyn_smem[2] = {0, 0};  // dynamic shared memory limit: layer, route_union
+  // dynamic shared memory limit: layer, route_union, grouped gate+up, grouped down, combine
+  int dyn_smem[5] = {0, 0, 0, 0, 0};
 };
 
 DeviceInfo g_dev[kMaxDevices];
@@ -47,9 +49,12 @@ moe_status device_info(DeviceInfo** out) {
       e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return cuda_fail(e);
     // dynamic + static shared memory may not exceed the opt-in limit
-    const void* kernels[2] = {reinterpret_cast<const void*>(layer_kernel),
-                              reinterpret_cast<const void*>(route_union_kernel)};
-    for (int i = 0; i < 2; ++i) {
+    const void* kernels[5] = {reinterpret_cast<const void*>(layer_kernel),
+                              reinterpret_cast<const void*>(route_union_kernel),
+                              reinterpret_cast<const void*>(grouped_kernel<0>),
+                              reinterpret_cast<const void*>(grouped_kernel<1>),
+                              reinterpret_cast<const void*>(grouped_combine_kernel)};
+    for (int i = 0; i < 5; ++i) {
       cudaFuncAttributes fa;
       cudaError_t e = cudaFuncGetAttributes(&fa, kernels[i]);
       if (e == cudaSuccess) {
@@ -100,13 +105,18 @@ WsLayout ws_layout(int T, int k, int E, int hidden, int inter) {
   return w;
 }
 
+// 1 = the persistent fused kernel (small windows), 2 = the grouped tensor-core
+// kernels (windows with more pairs; weight rows in multiples of 128), 0 = neither.
 int select_path(int T, int k, int E, int hidden, int inter) {
   if (!shape_ok(T, k, E, hidden, inter) || !shape_supported(T, k, E, hidden, inter)) return 0;
   if (T * k <= kMaxPairsFused) {
     LayerGeom g = layer_geom(hidden, inter);
     if (g.seg >= 1 && fit_stages(g, E, T * k, hidden, inter, kSmemBudget)) return 1;
   }
-  return 0;  // the grouped tensor-core path is not available in this build
+  if (hidden % kGM == 0 && inter % kGM == 0 &&
+      route_union_smem_bytes(E) <= kSmemBudget && sizeof(int) * (size_t)T * k <= kSmemBudget)
+    return 2;
+  return 0;
 }
 
 cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
@@ -166,6 +176,65 @@ cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
   c.attrs = attr;
   c.numAttrs = 2;
   return cudaLaunchKernelEx(&c, layer_kernel, a);
+}
+
+// The grouped path: route-union, gate+up, down and combine as four launches on
+// `st` (no host synchronisation).  The union arrays, h and y live in the workspace.
+cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w,
+                           const uint32_t* gq, const uint16_t* gs, const uint16_t* gb,
+                           const uint32_t* uq, const uint16_t* us, const uint16_t* ub,
+                           const uint32_t* dq, const uint16_t* ds, const uint16_t* db, int T,
+                           int k, int E, int H, int I, uint16_t* out, unsigned char* ws,
+                           const DeviceInfo& d, cudaStream_t st, moe_status* why) {
+  const WsLayout wl = ws_layout(T, k, E, H, I);
+  const int P = T * k;
+  int* nu = reinterpret_cast<int*>(ws + wl.num_unique);
+  int* uniq = reinterpret_cast<int*>(ws + wl.unique);
+  int* offs = reinterpret_cast<int*>(ws + wl.offsets);
+  int* plist = reinterpret_cast<int*>(ws + wl.pair_list);
+  uint16_t* h = reinterpret_cast<uint16_t*>(ws + wl.h);
+  float* y = reinterpret_cast<float*>(ws + wl.y);
+  const size_t usmem = route_union_smem_bytes(E);
+  const size_t csmem = sizeof(int) * (size_t)P;
+  if (usmem > (size_t)d.dyn_smem[1] || kGSmem > (unsigned)d.dyn_smem[2] ||
+      kGSmem > (unsigned)d.dyn_smem[3] || csmem > (size_t)d.dyn_smem[4]) {
+    *why = MOE_ERR_UNSUPPORTED;
+    return cudaSuccess;
+  }
+  route_union_kernel<<<1, 32 * kUnionWarps, usmem, st>>>(idx, P, E, uniq, offs, plist, nu);
+  GroupedArgs g{};
+  g.unique = uniq;
+  g.offsets = offs;
+  g.pair_list = plist;
+  g.num_unique = nu;
+  g.k = k;
+  g.H = H;
+  g.I = I;
+  g.h = h;
+  g.y = y;
+  // gate + up: weight rows I, K = H, activations x
+  g.act = x;
+  g.q0 = gq;
+  g.s0 = gs;
+  g.b0 = gb;
+  g.q1 = uq;
+  g.s1 = us;
+  g.b1 = ub;
+  g.rows = I;
+  g.K = H;
+  grouped_kernel<0><<<d.sms, kGThreads, kGSmem, st>>>(g);
+  // down: weight rows H, K = I, activations h
+  g.act = h;
+  g.q0 = dq;
+  g.s0 = ds;
+  g.b0 = db;
+  g.q1 = nullptr;
+  g.s1 = g.b1 = nullptr;
+  g.rows = H;
+  g.K = I;
+  grouped_kernel<1><<<d.sms, kGThreads, kGSmem, st>>>(g);
+  grouped_combine_kernel<<<d.sms, 256, csmem, st>>>(y, w, plist, offs, nu, T, k, H, out);
+  return cudaGetLastError();
 }
 
 struct OwnedWorkspace {
@@ -288,10 +357,15 @@ moe_status moe_switchglu_forward_ws(const uint16_t* x, const int32_t* topk_idx,
   DeviceInfo* d = nullptr;
   if (moe_status s = device_info(&d)) return s;
   moe_status why = MOE_OK;
-  const cudaError_t e = launch_layer(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q,
-                                    wd_s, wd_b, T, k, E, hidden, inter, out,
-                                    static_cast<unsigned char*>(workspace), *d,
-                                    (cudaStream_t)stream, &why);
+  const cudaError_t e =
+      path == 1 ? launch_layer(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q, wd_s,
+                               wd_b, T, k, E, hidden, inter, out,
+                               static_cast<unsigned char*>(workspace), *d, (cudaStream_t)stream,
+                               &why)
+                : launch_grouped(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q,
+                                 wd_s, wd_b, T, k, E, hidden, inter, out,
+                                 static_cast<unsigned char*>(workspace), *d, (cudaStream_t)stream,
+                                 &why);
   if (why != MOE_OK) return why;
   return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }

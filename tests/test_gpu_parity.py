@@ -294,3 +294,54 @@ def test_library_workspace_reused_across_shapes():
     for i, (T, k, E, H, I) in enumerate(shapes):
         L = make_layer(T, k, E, H, I, seed=900 + i, routing="uniform")
         check_layer(L, f"reuse #{i} T={T} k={k} E={E} H={H} I={I}")
+
+
+# ----------------------------------------------------- large windows (grouped) ---
+def test_grouped_path_selected_for_large_windows():
+    assert qeg.moe_select_path(160, 8, 64, 512, 256) == 2
+    assert qeg.moe_select_path(512, 8, 256, 4096, 2048) == 2
+    assert qeg.moe_select_path(2048, 8, 256, 4096, 2048) == 2
+    assert qeg.moe_select_path(160, 8, 64, 512, 192) == 0  # weight rows not a multiple of 128
+
+
+@pytest.mark.parametrize("cfg", [
+    # T, k, E, H, I: several experts with more than 16 pairs, ragged N tiles
+    (160, 8, 64, 512, 256),
+    (130, 8, 16, 256, 384),
+])
+def test_grouped_small(cfg):
+    T, k, E, H, I = cfg
+    L = make_layer(T, k, E, H, I, seed=700 + T, routing="uniform")
+    check_layer(L, f"grouped T={T} E={E} H={H} I={I}")
+
+
+def test_grouped_hot_expert_over_256_pairs():
+    """Expert 3 in every token: one expert with 300 pairs (two N tiles)."""
+    T, k, E, H, I = 300, 4, 32, 256, 256
+    rng = np.random.default_rng(9)
+    idx = np.stack([np.concatenate([[3], rng.choice([e for e in range(E) if e != 3], k - 1,
+                                                    replace=False)]) for _ in range(T)])
+    L = make_layer(T, k, E, H, I, seed=91, idx=idx.astype(np.int32))
+    check_layer(L, "grouped, one expert with 300 pairs")
+
+
+def test_grouped_invalid_ids_and_zero_rows():
+    T, k, E, H, I = 140, 8, 40, 256, 128
+    L = make_layer(T, k, E, H, I, seed=93, routing="uniform")
+    L.idx[5, :] = 77      # every pair of token 5 invalid -> zero row
+    L.idx[9, 3] = -1
+    out, _ = run_forward(L)
+    assert qeg.moe_read_device_status() == qeg.MOE_ERR_DEVICE_INDEX
+    ref = oracle.switchglu(L.x, L.idx, L.w, L.bank, L.E)
+    got = bf16_to_f64(out)
+    assert not np.any(got[5])
+    assert_parity(got, ref, "grouped with invalid ids")
+
+
+@pytest.mark.parametrize("T,n_check", [(512, 48), (2048, 32)])
+def test_grouped_large_window(T, n_check):
+    """The large-window configuration: E=256, top-8, 4096/2048, uniform routing; the
+    oracle checks a seeded sample of tokens."""
+    L = make_layer(T, 8, 256, 4096, 2048, seed=5000 + T, routing="uniform", draw_all=False)
+    tokens = sorted(np.random.default_rng(T).choice(T, n_check, replace=False).tolist())
+    check_layer(L, f"large window T={T}", tokens=tokens)
