@@ -476,7 +476,39 @@ def our_arm(args, world, rank, local):
                   "ratio_t2_over_t1": runs[2] / runs[1], "target_ratio": 1.7,
                   "mean_unique_t2": u2,
                   "t2_gbs": u2 * BYTES_PER_EXPERT / (runs[2] * 1e-6) / 1e9}
-        del bank2, ws2
+        del ws2
+    # large windows (the grouped tensor-core path): T=512 and T=2048 on the E=256 bank,
+    # a few layers each, CUDA events; bytes = unique experts, flops = 6 P H I
+    large = None
+    if verify is not None and not args.no_large_t:
+        large = {}
+        for TL, nl in ((512, 3), (2048, 2)):
+            rl = [synth.route_uniform(TL, E2, K_TOP, SEED + 900 + TL + l) for l in range(nl)]
+            xl = torch.from_numpy(synth.x_bf16(TL, HIDDEN, SEED + TL).view(np.int16)).to(dev) \
+                .view(torch.bfloat16)
+            il = [torch.from_numpy(r[0]).to(dev) for r in rl]
+            wl = [torch.from_numpy(r[1]).to(dev) for r in rl]
+            ol = torch.empty((TL, HIDDEN), dtype=torch.bfloat16, device=dev)
+            wsl = torch.zeros(qeg.moe_workspace_size(TL, K_TOP, E2, HIDDEN, INTER),
+                              dtype=torch.uint8, device=dev)
+            for l in range(nl):  # warm
+                qeg.moe_switchglu_forward_ws(xl, il[l], wl[l], bank2, wsl, out=ol)
+            torch.cuda.synchronize()
+            a4, b4 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a4.record()
+            for l in range(nl):
+                qeg.moe_switchglu_forward_ws(xl, il[l], wl[l], bank2, wsl, out=ol)
+            b4.record()
+            torch.cuda.synchronize()
+            us = a4.elapsed_time(b4) * 1e3 / nl
+            ul = float(np.mean([np.unique(r[0]).size for r in rl]))
+            fl = 6.0 * TL * K_TOP * HIDDEN * INTER
+            large[str(TL)] = {"us_per_layer": us, "mean_unique": ul,
+                              "unique_gbs": ul * BYTES_PER_EXPERT / (us * 1e-6) / 1e9,
+                              "tflops": fl / (us * 1e-6) / 1e12}
+            del wsl
+    if verify is not None:
+        del bank2
 
     # end to end through the public call: pinned host inputs in, outputs back, each step
     pin_x = {T: torch.from_numpy(synth.x_bf16(T, HIDDEN, SEED + T).view(np.int16)).pin_memory()
@@ -566,6 +598,7 @@ def our_arm(args, world, rank, local):
                     "how": "moe_switchglu_forward per layer, pinned host inputs copied in and "
                            "all layer outputs copied back every step"},
             "verify_pair": verify,
+            "large_window": large,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
         }
@@ -584,6 +617,8 @@ def main():
     ap.add_argument("--layers", type=int, default=42, help="chained layers per T (profiling)")
     ap.add_argument("--experts", type=int, default=288, help="bank size (profiling)")
     ap.add_argument("--quick", action="store_true", help="timed graph only (profiling)")
+    ap.add_argument("--no-large-t", action="store_true",
+                    help="skip the T=512 / T=2048 grouped-path measurement")
     ap.add_argument("--no-verify-pair", action="store_true",
                     help="skip the T=2 / T=1 speculative-verify measurement")
     ap.add_argument("--ts", default="", help="comma-separated window sizes (profiling)")

@@ -122,8 +122,59 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c) {
   return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
 }
 
-// bf16 bits of fp32 x (round to nearest even).
-__device__ __forceinline__ uint32_t bf16_rn_bits(float x) { return float_to_bf16_bits(x); }
+// Codes -> floats without integer conversion: nibble j of a word ORed under the
+// exponent (150 - 4j) reads as 2^(23-4j) + q exactly, and one packed add removes
+// the offset.  Masks and exponents live in registers (one LOP3 per nibble).
+struct NibbleConsts {
+  uint32_t m0, m1, m2, m3, m4, e150, e146, e142, e138, e134;
+};
+__device__ __forceinline__ NibbleConsts nibble_consts() {
+  NibbleConsts k{0xFu, 0xF0u, 0xF00u, 0xF000u, 0xF0000u,
+                 150u << 23, 146u << 23, 142u << 23, 138u << 23, 134u << 23};
+  asm volatile("" : "+r"(k.m0), "+r"(k.m1), "+r"(k.m2), "+r"(k.m3), "+r"(k.m4));
+  asm volatile("" : "+r"(k.e150), "+r"(k.e146), "+r"(k.e142), "+r"(k.e138), "+r"(k.e134));
+  return k;
+}
+__device__ __forceinline__ float or_and(uint32_t a, uint32_t m, uint32_t e) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(m), "r"(e));
+  return __uint_as_float(d);
+}
+// The 8 codes of w (element j = nibble j) as (q0,q1) (q2,q3) (q4,q5) (q6,q7).
+__device__ __forceinline__ void nibbles8(uint32_t w, const NibbleConsts& k, float2 (&q)[4]) {
+  const uint32_t w2 = w >> 12;
+  q[0] = __fadd2_rn(make_float2(or_and(w, k.m0, k.e150), or_and(w, k.m1, k.e146)),
+                    make_float2(-8388608.f, -524288.f));
+  q[1] = __fadd2_rn(make_float2(or_and(w, k.m2, k.e142), or_and(w, k.m3, k.e138)),
+                    make_float2(-32768.f, -2048.f));
+  q[2] = __fadd2_rn(make_float2(or_and(w, k.m4, k.e134), or_and(w2, k.m2, k.e142)),
+                    make_float2(-128.f, -32768.f));
+  q[3] = __fadd2_rn(make_float2(or_and(w2, k.m3, k.e138), or_and(w2, k.m4, k.e134)),
+                    make_float2(-2048.f, -128.f));
+}
+// Packed bf16 pair (round to nearest even) of two floats: low half = a.
+__device__ __forceinline__ uint32_t bf16x2_rn(float a, float b) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(b), "f"(a));
+  return d;
+}
+// One code word's 8 weights w = s*q + b as bf16 hi (= bf16(w)) and lo (= bf16(w - hi)).
+__device__ __forceinline__ void dequant8_hilo(uint32_t w, float2 s2, float2 b2,
+                                              const NibbleConsts& k, uint4& hi, uint4& lo) {
+  float2 q[4];
+  nibbles8(w, k, q);
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 v = __ffma2_rn(q[j], s2, b2);
+    h[j] = bf16x2_rn(v.x, v.y);
+    const float2 hv = make_float2(__uint_as_float(h[j] << 16), __uint_as_float(h[j] & 0xffff0000u));
+    const float2 r = __fadd2_rn(v, make_float2(-hv.x, -hv.y));  // exact
+    l[j] = bf16x2_rn(r.x, r.y);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
 
 // ------------------------------------------------------------------ kernels ---
 struct GroupedArgs {
@@ -172,6 +223,7 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_kernel(const GroupedArgs
   const int nslab = a.K / kGK;
   uint32_t phase_bits = 0;  // completed-phase parity of mma_done[0], [1]
   bool ok = true;
+  const NibbleConsts nk = nibble_consts();
 
   for (int tile = blockIdx.x; tile < u * mtiles && ok; tile += gridDim.x) {
     const int slot = tile / mtiles, m0 = (tile % mtiles) * kGM;
@@ -183,6 +235,41 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_kernel(const GroupedArgs
       const int np = (n + 15) & ~15;  // MMA N
       const uint32_t idesc = f16_idesc(kGM, np);
       int issued = 0;  // slabs whose MMAs were issued (in this n-chunk)
+      // Per thread: A tasks (matrix, row, half slab of 32 columns) tid and tid + 256
+      // (gate+up), B tasks (pair row, 16-byte chunk) tid + 256 i.  Their global data
+      // for slab s+1 is loaded while slab s is dequantised and multiplied.
+      constexpr int kATasks = NMAT * kGM * 2 / kGThreads;  // 2 or 1
+      constexpr int kBTasks = kGMaxN * 8 / kGThreads;      // 8
+      uint4 cw[kATasks];
+      uint16_t sraw[kATasks], braw[kATasks];
+      uint4 xv[kBTasks];
+      auto load_slab = [&](int s) {
+#pragma unroll
+        for (int i = 0; i < kATasks; ++i) {
+          const int task = tid + i * kGThreads;
+          const int mat = task / (kGM * 2), rr = (task >> 1) % kGM, half = task & 1;
+          const uint32_t* q = mat ? a.q1 : a.q0;
+          const uint16_t* sp = mat ? a.s1 : a.s0;
+          const uint16_t* bp = mat ? a.b1 : a.b0;
+          const size_t row = wrow0 + rr;
+          cw[i] = __ldg(reinterpret_cast<const uint4*>(q + row * (a.K / 8) + s * 8) + half);
+          sraw[i] = __ldg(sp + row * (a.K / 64) + s);
+          braw[i] = __ldg(bp + row * (a.K / 64) + s);
+        }
+#pragma unroll
+        for (int i = 0; i < kBTasks; ++i) {
+          const int task = tid + i * kGThreads, rr = task >> 3, c = task & 7;
+          xv[i] = make_uint4(0u, 0u, 0u, 0u);
+          if (rr < n) {
+            const int pos = n0 + rr;
+            const size_t arow = PHASE == 0 ? (size_t)(a.pair_list[pos] / a.k) : (size_t)pos;
+            const uint16_t* src = a.act + arow * a.K + s * kGK + c * 8;
+            xv[i] = PHASE == 0 ? __ldg(reinterpret_cast<const uint4*>(src))
+                               : __ldcg(reinterpret_cast<const uint4*>(src));
+          }
+        }
+      };
+      load_slab(0);
       for (int s = 0; s < nslab && ok; ++s) {
         const int buf = s & 1;
         unsigned char* base = gsm + buf * kBuf;
@@ -191,50 +278,41 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_kernel(const GroupedArgs
           phase_bits ^= 1u << buf;
           if (!ok) break;
         }
-        // --- A: dequantised weight slab(s), 128 rows x 64, swizzled ---
-        for (int task = tid; task < NMAT * kGM * 2; task += kGThreads) {
+        uint4 ccw[kATasks], cxv[kBTasks];
+        uint16_t cs[kATasks], cb[kATasks];
+#pragma unroll
+        for (int i = 0; i < kATasks; ++i) {
+          ccw[i] = cw[i];
+          cs[i] = sraw[i];
+          cb[i] = braw[i];
+        }
+#pragma unroll
+        for (int i = 0; i < kBTasks; ++i) cxv[i] = xv[i];
+        if (s + 1 < nslab) load_slab(s + 1);
+        // --- A: dequantised weight slab(s), 128 rows x 64, hi and lo, swizzled ---
+#pragma unroll
+        for (int i = 0; i < kATasks; ++i) {
+          const int task = tid + i * kGThreads;
           const int mat = task / (kGM * 2), rr = (task >> 1) % kGM, half = task & 1;
-          const uint32_t* q = mat ? a.q1 : a.q0;
-          const uint16_t* sp = mat ? a.s1 : a.s0;
-          const uint16_t* bp = mat ? a.b1 : a.b0;
-          const size_t row = wrow0 + rr;
-          // 4 code words = 32 columns (half of the slab), one group of 64
-          const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(q + row * (a.K / 8) + s * 8) + half);
-          const float sc = bf16_bits_to_float(__ldg(sp + row * (a.K / 64) + s));
-          const float bi = bf16_bits_to_float(__ldg(bp + row * (a.K / 64) + s));
-          const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+          const float sc = bf16_bits_to_float(cs[i]), bi = bf16_bits_to_float(cb[i]);
+          const float2 s2 = make_float2(sc, sc), b2 = make_float2(bi, bi);
           unsigned char* tileA = base + 2 * mat * kGATile;  // hi tile; lo tile follows
+          const uint32_t ws[4] = {ccw[i].x, ccw[i].y, ccw[i].z, ccw[i].w};
 #pragma unroll
           for (int c = 0; c < 4; ++c) {  // 16-byte chunk = 8 columns = one code word
-            uint32_t oh[4], ol[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {  // columns 2j (low half) and 2j+1 (high half)
-              const float w0 = fmaf(sc, (float)((ws[c] >> (8 * j)) & 0xf), bi);
-              const float w1 = fmaf(sc, (float)((ws[c] >> (8 * j + 4)) & 0xf), bi);
-              const uint32_t h0 = bf16_rn_bits(w0), h1 = bf16_rn_bits(w1);
-              oh[j] = h0 | (h1 << 16);
-              ol[j] = bf16_rn_bits(w0 - bf16_bits_to_float((uint16_t)h0)) |
-                      (bf16_rn_bits(w1 - bf16_bits_to_float((uint16_t)h1)) << 16);
-            }
+            uint4 hi, lo;
+            dequant8_hilo(ws[c], s2, b2, nk, hi, lo);
             const uint32_t off = sw128_off(rr, half * 4 + c);
-            *reinterpret_cast<uint4*>(tileA + off) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
-            *reinterpret_cast<uint4*>(tileA + kGATile + off) =
-                make_uint4(ol[0], ol[1], ol[2], ol[3]);
+            *reinterpret_cast<uint4*>(tileA + off) = hi;
+            *reinterpret_cast<uint4*>(tileA + kGATile + off) = lo;
           }
         }
-        // --- B: the n activation rows of the slab (zero rows up to np), swizzled ---
+        // --- B: the activation rows of the slab (zero rows up to np), swizzled ---
         unsigned char* tileB = base + 2 * NMAT * kGATile;
-        for (int task = tid; task < np * 8; task += kGThreads) {
-          const int rr = task >> 3, c = task & 7;
-          uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (rr < n) {
-            const int pos = n0 + rr;
-            const size_t arow = PHASE == 0 ? (size_t)(a.pair_list[pos] / a.k) : (size_t)pos;
-            const uint16_t* src = a.act + arow * a.K + s * kGK + c * 8;
-            v = PHASE == 0 ? __ldg(reinterpret_cast<const uint4*>(src))
-                           : __ldcg(reinterpret_cast<const uint4*>(src));
-          }
-          *reinterpret_cast<uint4*>(tileB + sw128_off(rr, c)) = v;
+#pragma unroll
+        for (int i = 0; i < kBTasks; ++i) {
+          const int task = tid + i * kGThreads, rr = task >> 3, c = task & 7;
+          if (rr < np) *reinterpret_cast<uint4*>(tileB + sw128_off(rr, c)) = cxv[i];
         }
         fence_proxy_async();  // generic smem writes -> tensor-core reads
         __syncthreads();
