@@ -51,7 +51,7 @@ namespace qeg {
 
 constexpr int kWarps = 8;                    // compute warps
 constexpr int kConsumerThreads = 32 * kWarps;
-constexpr int kThreads = kConsumerThreads + 32;  // + one producer warp
+constexpr int kThreads = kConsumerThreads + 64;  // + a producer warp and a helper warp
 constexpr int kRowsA = kWarps;      // phase A: one row of gate and of up per warp per block
 constexpr int kBlocksPerItemA = 4;  // phase-A item: 4 blocks = 32 rows = one h chunk
 constexpr int kBlocksPerItemB = 2;  // phase-B item: row blocks
@@ -119,8 +119,8 @@ __host__ __device__ inline LayerSmem layer_smem(const LayerGeom& g, int E, int P
   const int m = (E < P ? E : P) > 0 ? (E < P ? E : P) : 1;
   s.stages = 0;
   s.act = align_up((size_t)g.stages * g.stage_bytes, 128);    // two activation buffers
-  s.hscr = s.act + 2 * (size_t)g.act_buf;                      // h of a phase-A item
-  s.cnt = align_up(s.hscr + sizeof(float) * 2 * kNT * 32, 16);  // two items' h
+  s.hscr = s.act + 2 * (size_t)g.act_buf;  // bf16 h of phase-A items, per item ring slot
+  s.cnt = align_up(s.hscr + sizeof(uint16_t) * kItemRing * kNT * 32, 16);
   s.rank = align_up(s.cnt + sizeof(int) * E, 16);
   s.unique = align_up(s.rank + sizeof(int) * P, 16);
   s.offsets = align_up(s.unique + sizeof(int) * m, 16);
@@ -334,7 +334,7 @@ __device__ __forceinline__ void rows_a(const unsigned char* bg_q, const uint16_t
 #pragma unroll
   for (int t = 0; t < NT; ++t) ag[t] = au[t] = 0.f;
   const int nch = H / 32;
-#pragma unroll
+#pragma unroll 1
   for (int i = 0; i < R; ++i) {
     const int ch = i * 32 + lane;
     if (ch < nch) {
@@ -382,7 +382,7 @@ __device__ __forceinline__ float rows_b(const unsigned char* bq, const uint16_t*
 #pragma unroll
   for (int v = 0; v < V; ++v) acc[v] = 0.f;
   const int nch = I / 32, qstride = I / 2, sstride = I / 64;
-#pragma unroll
+#pragma unroll 1
   for (int i = 0; i < R; ++i) {
     const int ch = i * 32 + lane;
     if (ch < nch) {
@@ -462,6 +462,7 @@ __device__ __forceinline__ void fence_proxy_async_all() {
 // Lane 0's value of a condition, in every lane (keeps the producer warp's control
 // flow uniform when lanes could read a changing value at different times).
 __device__ __forceinline__ bool lane0(bool v) { return __shfl_sync(kFull, v ? 1 : 0, 0) != 0; }
+__device__ __forceinline__ int lane0_int(int v) { return __shfl_sync(kFull, v, 0); }
 
 // Ring-slot descriptor flags (slot_info[st].x) for the compute warps.
 constexpr int kSlotEnd = 1;        // no more blocks
@@ -476,8 +477,11 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_u, s_nseg;
   __shared__ volatile int s_abort;
+  // producer <-> helper: items recorded / published, activation loads queued / issued,
+  // producer finished
+  __shared__ volatile int s_nrec, s_pub, s_pend_tail, s_pend_head, s_prod_done;
   __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
-  __shared__ __align__(8) uint64_t act_full[kItemRing], item_done[kItemRing], hs_bar[2];
+  __shared__ __align__(8) uint64_t act_full[kItemRing], item_done[kItemRing];
   __shared__ unsigned long long reg_start[kItemRing];  // activation regions (producer)
   __shared__ int reg_last[kItemRing];
   __shared__ int4 item_info[kItemRing];  // per item ordinal: phase B, segment, first block, blocks
@@ -504,8 +508,8 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       mbar_init(&act_full[i], 1);
       mbar_init(&item_done[i], kWarps);
     }
-    for (int b = 0; b < 2; ++b) mbar_init(&hs_bar[b], kWarps);
     s_abort = 0;
+    s_nrec = s_pub = s_pend_tail = s_pend_head = s_prod_done = 0;
     fence_barrier_init();
   }
   if (a.wait_prior) grid_dep_wait();
@@ -589,10 +593,117 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
   const int n_items_a = nseg * ipa;
   const int n_items = n_items_a + nseg * ipb;
 
-  if (warp == kWarps) {
+  if (warp == kWarps + 1) {
+    // ================================ helper warp ================================
+    // Publishes finished items in order (converting each phase-A item's h chunk to
+    // the fixed-point layout first) and issues the queued activation loads once what
+    // they read is complete.  Every condition is lane 0's (uniform control flow).
+    const uint16_t* hscr_p = reinterpret_cast<const uint16_t*>(smem + L.hscr);
+    int pub = 0, ph = 0;  // items published; queued loads issued
+    bool x_ready = false;
+    unsigned long long t_prog = globaltimer();
+    for (;;) {
+      bool progressed = false;
+      // ---- publish ----
+      const int n_rec = lane0_int(s_nrec);
+      __threadfence_block();  // item_info of the recorded items is read after the count
+      int n = 0;
+      while (pub + n < n_rec &&
+             lane0(mbar_test(&item_done[(pub + n) % kItemRing], ((pub + n) / kItemRing) & 1)))
+        ++n;
+      if (n > 0) {
+        // a phase-A item's 32 h rows per pair are one chunk of h (lanes 4t..4t+3: pair t)
+        for (int i = 0; i < n; ++i) {
+          const int4 ii = item_info[(pub + i) % kItemRing];
+          if (ii.x != 0) continue;
+          const int nt = seg_nt[ii.y], p0 = seg_pos[ii.y];
+          if (lane < nt * 4) {
+            const int t = lane >> 2, m = lane & 3;
+            const uint4 v = *reinterpret_cast<const uint4*>(
+                hscr_p + ((pub + i) % kItemRing) * (kNT * 32) + t * 32 + m * 8);
+            uint4 packed;
+            const float2 sc = fixed_point_quarter(v, 0xfu << (lane & ~3), packed);
+            const int ch = ii.z / (32 / kRowsA), R = G.rounds_b;  // h chunk of the item
+            unsigned char* row = a.hq + (size_t)(p0 + t) * stride_b;
+            reinterpret_cast<uint4*>(row)[((ch / 32) * 4 + m) * 32 + (ch % 32)] = packed;
+            if (m == 0) reinterpret_cast<float2*>(row + act_digit_bytes(R))[ch] = sc;
+          }
+        }
+        __syncwarp();  // the lanes' hq writes precede lane 0's release below
+        // The compute warps' item_done arrivals released their stores at CTA scope and
+        // the tests above acquired them; the device-scope release reductions pass them
+        // on (causality order is transitive across the two scopes).
+        if (lane == 0) {
+          for (int i = 0; i < n; ++i) {
+            const int4 ii = item_info[(pub + i) % kItemRing];
+            if (ii.x == 0) {
+              red_release_gpu(&hdone[ii.y], (unsigned)ii.w);
+            } else {
+              for (int r = 0; r < ii.w; ++r) red_release_gpu(&ydone[ii.z + r], 1u);
+            }
+          }
+          __threadfence_block();
+          s_pub = pub + n;  // the producer frees ring slots and activation regions
+        }
+        __syncwarp();
+        pub += n;
+        progressed = true;
+      }
+      // ---- queued activation loads, in order ----
+      while (ph < lane0_int(s_pend_tail)) {
+        __threadfence_block();  // the entry is read after the count
+        const int4 pe = pend[ph % kItemRing];  // (ord, sg, byte offset, phase B | parity << 1)
+        const int sg = pe.y, nt = seg_nt[pe.y], p0 = seg_pos[pe.y];
+        const bool pb = (pe.w & 1) != 0;
+        if (pb) {
+          if (!lane0(ld_acquire_gpu(&hdone[sg]) >= (unsigned)bpe_a)) break;
+        } else if (!x_ready) {
+          if (!lane0(ld_acquire_gpu(xdone) >= gridDim.x)) break;
+          x_ready = true;
+        }
+        if (lane == 0) {
+          uint64_t* bar = &act_full[pe.x % kItemRing];
+          unsigned char* dst = smem + L.act + pe.z;
+          fence_proxy_async_all();  // rows other CTAs wrote, read by the bulk copy
+          if (pb) {
+            const unsigned size = (unsigned)nt * stride_b;
+            mbar_arrive_expect_tx(bar, size);
+            bulk_g2s(dst, a.hq + (size_t)p0 * stride_b, size, bar);
+          } else {
+            mbar_arrive_expect_tx(bar, (unsigned)nt * stride_a);
+            for (int t = 0; t < nt; ++t)
+              bulk_g2s(dst + (size_t)t * stride_a,
+                       a.xg + (size_t)(plist[p0 + t] / a.k) * stride_a, stride_a, bar);
+          }
+          __threadfence_block();
+          s_pend_head = ph + 1;
+        }
+        __syncwarp();
+        ++ph;
+        progressed = true;
+      }
+      // ---- done, or wait (bounded without progress) ----
+      if (lane0(s_prod_done != 0) && pub == lane0_int(s_nrec) && ph == lane0_int(s_pend_tail))
+        break;
+      if (progressed) {
+        t_prog = globaltimer();
+      } else {
+        if (lane0(s_abort != 0)) break;
+        if (lane0(globaltimer() - t_prog > kWaitLimitNs)) {
+          if (lane == 0) {
+            set_error(kErrTimeout);
+            s_abort = 1;
+          }
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+  } else if (warp == kWarps) {
     // =============================== producer warp ===============================
-    // (every condition is lane 0's, so all lanes take the same path)
-    int pub = 0, n_rec = 0;  // next item ordinal to publish; items recorded
+    // Takes items, places their activation rows in a circular byte ring (queueing
+    // the load for the helper warp) and issues their weight blocks into the stage
+    // ring.  Every condition is lane 0's (uniform control flow).
     auto timed_out = [&](unsigned long long t0) -> bool {
       if (lane0(s_abort != 0)) return true;
       if (lane0(globaltimer() - t0 > kWaitLimitNs)) {
@@ -604,123 +715,40 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       }
       return false;
     };
-    // Activation rows live in a circular byte ring: an item's rows occupy a region
-    // [start, start + size) of virtual positions until the last item using them is
-    // published.  Regions are freed in order.
+    // An item's rows occupy a region [start, start + size) of virtual positions of the
+    // ring until the last item using them is published.  Regions are freed in order.
     const unsigned long long ring = 2ull * G.act_buf;
     unsigned long long head = 0, tail = 0;
     int reg_front = 0, reg_cnt = 0;
-    // Publish every recorded item the compute warps have finished, in order.  Their
-    // mbarrier arrivals release their stores at CTA scope and the test here acquires
-    // them; the device-scope release reductions pass them on (causality order is
-    // transitive across the two scopes).
-    auto poll_publish = [&]() {
-      int n = 0;
-      while (pub + n < n_rec &&
-             lane0(mbar_test(&item_done[(pub + n) % kItemRing], ((pub + n) / kItemRing) & 1)))
-        ++n;
-      if (n == 0) return;
-      if (lane == 0) {
-        for (int i = 0; i < n; ++i) {
-          const int4 ii = item_info[(pub + i) % kItemRing];
-          if (ii.x == 0) {
-            red_release_gpu(&hdone[ii.y], (unsigned)(ii.w * 1));
-          } else {
-            for (int r = 0; r < ii.w; ++r) red_release_gpu(&ydone[ii.z + r], 1u);
-          }
-        }
-      }
-      __syncwarp();
-      pub += n;
-      while (reg_cnt > 0 && reg_last[reg_front] < pub) {  // activation regions no one uses
+    auto free_regions = [&]() {
+      const int pub = lane0_int(s_pub);
+      while (reg_cnt > 0 && reg_last[reg_front] < pub) {
         reg_front = (reg_front + 1) % kItemRing;
         --reg_cnt;
         tail = reg_cnt > 0 ? reg_start[reg_front] : head;
       }
     };
-
-    // Activation loads wait in a queue (in item order) until what they read is
-    // complete: every CTA's x rows (phase A), or the segment's h (phase B), so that
-    // weight copies keep flowing meanwhile.
-    int pend_front = 0, pend_cnt = 0;
-    bool x_ready = false;
-    unsigned act_par = 0;      // per item ring slot: parity of its next load's phase
-    unsigned loaded_mask = 0;  // item ring slots that have had an activation load
-    // pre_ord / pre_val: a counter value for the load of item pre_ord, read earlier
-    // (with acquire), so that the common case costs no round trip here.
-    auto try_flush = [&](int pre_ord, unsigned pre_val) {
-      while (pend_cnt > 0) {
-        const int4 pe = pend[pend_front];  // (ord, sg, byte offset, phase B)
-        const int sg = pe.y, nt = seg_nt[pe.y], p0 = seg_pos[pe.y];
-        const unsigned need = pe.w ? (unsigned)bpe_a : gridDim.x;
-        if (pe.w || !x_ready) {
-          const unsigned* ctr = pe.w ? &hdone[sg] : xdone;
-          const bool pre_ok = pe.x == pre_ord && pre_val >= need;
-          if (!pre_ok && !lane0(ld_acquire_gpu(ctr) >= need)) return;
-          if (!pe.w) x_ready = true;
-        }
-        if (lane == 0) {
-          uint64_t* bar = &act_full[pe.x % kItemRing];
-          unsigned char* dst = smem + L.act + pe.z;
-          fence_proxy_async_all();  // rows other CTAs wrote, read by the bulk copy
-          if (pe.w) {
-            const unsigned size = (unsigned)nt * stride_b;
-            mbar_arrive_expect_tx(bar, size);
-            bulk_g2s(dst, a.hq + (size_t)p0 * stride_b, size, bar);
-          } else {
-            mbar_arrive_expect_tx(bar, (unsigned)nt * stride_a);
-            for (int t = 0; t < nt; ++t)
-              bulk_g2s(dst + (size_t)t * stride_a,
-                       a.xg + (size_t)(plist[p0 + t] / a.k) * stride_a, stride_a, bar);
-          }
-        }
-        __syncwarp();
-        pend_front = (pend_front + 1) % kItemRing;
-        --pend_cnt;
-      }
-    };
-    auto wait_bar = [&](uint64_t* bar, unsigned parity) -> bool {
-      const unsigned long long t0 = globaltimer();
-      while (!lane0(mbar_test(bar, parity))) {
-        poll_publish();
-        try_flush(-1, 0);
-        if (timed_out(t0)) return false;
-        __nanosleep(64);  // leave issue slots to the compute warps
-      }
-      return true;
-    };
-
     bool ok = true;
     int gi = 0;                     // blocks issued into the ring
     int cur_key = -1;               // activation set of the newest region
     int cur_tok[kNT] = {-1, -1, -1, -1};
     unsigned cur_off = 0;           // its byte offset in the ring
     unsigned long long cur_start = 0;  // and its virtual position
-    int n_a_items = 0;              // phase-A items taken (scratch buffer parity)
-    // Items are taken two ahead: q1 is the next item (its counter c1, the one its
-    // activation load depends on, read one item early) and q2's atomic is in flight.
-    // Lane 0 holds the values.
-    auto dep_counter = [&](unsigned it) -> const unsigned* {
-      if ((int)it >= n_items) return nullptr;
-      if ((int)it < n_items_a) return x_ready ? nullptr : xdone;
-      return &hdone[((int)it - n_items_a) / ipb];
-    };
-    unsigned q0 = 0, q1 = 0, q2 = 0, c0 = 0, c1 = 0;
+    unsigned act_par = 0;           // per item ring slot: parity of its next load's phase
+    int pend_tail = 0;              // loads queued
+    int n_a_items = 0;              // phase-A items taken
+    unsigned q0 = 0, q1 = 0;        // items taken ahead (two atomics in flight)
     if (lane == 0) {
       q0 = atomicAdd(work_ctr, 1u);
       q1 = atomicAdd(work_ctr, 1u);
-      const unsigned* d0 = dep_counter(q0);
-      c0 = d0 ? ld_acquire_gpu(d0) : 0u;
     }
     for (int ord = 0; ok; ++ord) {
       const int item = (int)__shfl_sync(kFull, q0, 0);
       if (item >= n_items) break;
       if (lane == 0) {
-        q2 = atomicAdd(work_ctr, 1u);
-        const unsigned* d1 = dep_counter(q1);
-        c1 = d1 ? ld_acquire_gpu(d1) : 0u;
+        q0 = q1;
+        q1 = atomicAdd(work_ctr, 1u);
       }
-      const unsigned pre_val = __shfl_sync(kFull, c0, 0);
       const bool phase_b = item >= n_items_a;
       int sg, blk0, nblk;
       if (!phase_b) {
@@ -733,14 +761,12 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
         nblk = min(kBlocksPerItemB, bpe_b - blk0);
       }
       const int nt = seg_nt[sg], p0 = seg_pos[sg];
-      // ---- its ring slot for publication (and for a pending load) must be free ----
+      // ---- its ring slot for publication must be free ----
       {
         const unsigned long long t0 = globaltimer();
-        while (ok && (pub <= ord - kItemRing || pend_cnt >= kItemRing)) {
-          poll_publish();
-          try_flush(-1, 0);
+        while (ok && lane0_int(s_pub) <= ord - kItemRing) {
+          if (timed_out(t0)) ok = false;
           __nanosleep(64);
-          if ((pub <= ord - kItemRing || pend_cnt >= kItemRing) && timed_out(t0)) ok = false;
         }
       }
       if (!ok) break;
@@ -754,6 +780,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
         same = cur_key == sg;
       }
       bool act_wait = false, load_par = false;
+      free_regions();
       if (same) {  // extend the newest region's life (it may already have been freed)
         if (lane == 0) {
           const int r = (reg_front + reg_cnt + (reg_cnt == 0 ? 0 : -1) + kItemRing) % kItemRing;
@@ -773,46 +800,60 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
           for (;;) {
             start = head;
             if (start % ring + size > ring) start = (start / ring + 1) * ring;  // no wrap
-            if (start + size - tail <= ring && reg_cnt < kItemRing) break;
-            poll_publish();
-            try_flush(-1, 0);
+            if (start + size - tail <= ring && reg_cnt < kItemRing &&
+                pend_tail - lane0_int(s_pend_head) < kItemRing)
+              break;
             if (timed_out(t0)) {
               ok = false;
               break;
             }
             __nanosleep(64);
+            free_regions();
           }
         }
         if (!ok) break;
         cur_off = (unsigned)(start % ring);
         cur_start = start;
+        load_par = (act_par >> (ord % kItemRing)) & 1u;
+        act_par ^= 1u << (ord % kItemRing);
         if (lane == 0) {
           const int r = (reg_front + reg_cnt) % kItemRing;
           reg_start[r] = start;
           reg_last[r] = ord;
-          pend[(pend_front + pend_cnt) % kItemRing] = make_int4(ord, sg, (int)cur_off, phase_b ? 1 : 0);
+          pend[pend_tail % kItemRing] =
+              make_int4(ord, sg, (int)cur_off, (phase_b ? 1 : 0) | (load_par ? 2 : 0));
+          __threadfence_block();
+          s_pend_tail = pend_tail + 1;  // the helper warp issues the load
         }
         __syncwarp();
+        ++pend_tail;
         if (reg_cnt == 0) tail = start;
         ++reg_cnt;
         head = start + size;
-        ++pend_cnt;
-        loaded_mask |= 1u << (ord % kItemRing);
-        load_par = (act_par >> (ord % kItemRing)) & 1u;
-        act_par ^= 1u << (ord % kItemRing);
         act_wait = true;
         cur_key = phase_b ? sg : -2;
         for (int t = 0; t < kNT; ++t) cur_tok[t] = (!phase_b && t < nt) ? plist[p0 + t] / a.k : -1;
       }
       // ---- the item's record for publication ----
-      if (lane == 0) item_info[ord % kItemRing] = make_int4(phase_b ? 1 : 0, sg, blk0, nblk);
+      if (lane == 0) {
+        item_info[ord % kItemRing] = make_int4(phase_b ? 1 : 0, sg, blk0, nblk);
+        __threadfence_block();
+        s_nrec = ord + 1;
+      }
       __syncwarp();
       const int a_ord = phase_b ? 0 : n_a_items++;
-      if (act_wait) try_flush(ord, pre_val);  // at once when the early read shows it ready
       // ---- its blocks into the ring ----
       for (int j = 0; j < nblk && ok; ++j, ++gi) {
         const int st = gi % NS;
-        if (gi >= NS) ok = wait_bar(&empty[st], ((gi / NS) - 1) & 1);
+        if (gi >= NS) {
+          const unsigned long long t0 = globaltimer();
+          while (!lane0(mbar_test(&empty[st], ((gi / NS) - 1) & 1))) {
+            if (timed_out(t0)) {
+              ok = false;
+              break;
+            }
+          }
+        }
         if (!ok) break;
         if (lane == 0) {
           const int blk = blk0 + j;
@@ -848,39 +889,28 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
         }
         __syncwarp();
       }
-      n_rec = ord + 1;
-      if (ok) poll_publish();
-      if (lane == 0) {
-        q0 = q1;
-        c0 = c1;
-        q1 = q2;
-      }
     }
-    // ---- pending loads, the end marker, then publish what is left (bounded) ----
-    {
-      const unsigned long long t0 = globaltimer();
-      while (ok && pend_cnt > 0) {
-        poll_publish();
-        try_flush(-1, 0);
-        __nanosleep(64);
-        if (pend_cnt > 0 && timed_out(t0)) ok = false;
-      }
-    }
+    // ---- the end marker ----
     if (ok) {
       const int st = gi % NS;
-      if (gi >= NS) ok = wait_bar(&empty[st], ((gi / NS) - 1) & 1);
+      if (gi >= NS) {
+        const unsigned long long t0 = globaltimer();
+        while (!lane0(mbar_test(&empty[st], ((gi / NS) - 1) & 1))) {
+          if (timed_out(t0)) {
+            ok = false;
+            break;
+          }
+        }
+      }
       if (ok && lane == 0) {
         slot_info[st] = make_int4(kSlotEnd, 0, 0, 0);
         mbar_arrive(&full[st]);
       }
       __syncwarp();
     }
-    {
-      const unsigned long long t0 = globaltimer();
-      while (ok && pub < n_rec) {
-        poll_publish();
-        if (pub < n_rec && timed_out(t0)) ok = false;
-      }
+    if (lane == 0) {
+      __threadfence_block();
+      s_prod_done = 1;
     }
     // copies still in flight after an abort land before the CTA exits (bounded)
     if (!ok && lane == 0) {
@@ -889,18 +919,11 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
         while (!mbar_test(&full[g % NS], (g / NS) & 1) && globaltimer() - t0 < kWaitLimitNs) {
         }
       }
-      for (int sl = 0; sl < kItemRing; ++sl)
-        if (loaded_mask & (1u << sl)) {  // the slot's latest load (its phase parity)
-          const unsigned par = ((act_par >> sl) & 1u) ^ 1u;
-          const unsigned long long t0 = globaltimer();
-          while (!mbar_test(&act_full[sl], par) && globaltimer() - t0 < kWaitLimitNs) {
-          }
-        }
     }
     __syncwarp();
   } else {
     // ================================ compute warps ================================
-    float* hscr = reinterpret_cast<float*>(smem + L.hscr);  // [2][kNT][32]
+    uint16_t* hscr = reinterpret_cast<uint16_t*>(smem + L.hscr);  // [kItemRing][kNT][32]
     auto wait_cons = [&](uint64_t* bar, unsigned parity) -> bool {
       if (s_abort) return false;
       const unsigned long long t0 = globaltimer();
@@ -960,7 +983,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       if (lane == 0) mbar_arrive(&empty[st]);
       const bool item_end = (si.x & kSlotItemEnd) != 0;
       if (!phase_b) {
-        float* hs = hscr + (a_ord & 1) * (kNT * 32);
+        uint16_t* hs = hscr + (ord % kItemRing) * (kNT * 32);
         if (lane < nt) {
           float gv = 0.f, uv = 0.f;
 #pragma unroll
@@ -972,31 +995,10 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
           const float g = round_to_bf16(gv), hu = round_to_bf16(uv);
           const uint16_t hb = float_to_bf16_bits(g / (1.0f + __expf(-g)) * hu);
           a.h[(size_t)(p0 + lane) * a.I + row0 + warp] = hb;
-          hs[lane * 32 + (row0 & 31) + warp] = bf16_bits_to_float(hb);
+          hs[lane * 32 + (row0 & 31) + warp] = hb;
         }
-        if (item_end) {
-          // the item's 32 h rows per pair are one chunk of h: one warp (in turn) converts it
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&hs_bar[a_ord & 1]);
-          if (warp == (a_ord & (kWarps - 1)) && wait_cons(&hs_bar[a_ord & 1], (a_ord >> 1) & 1)) {
-            if (lane < nt * 4) {
-              const int t = lane >> 2, m = lane & 3;
-              const float* src = hs + t * 32 + m * 8;
-              uint32_t wv[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                wv[e] = (uint32_t)float_to_bf16_bits(src[2 * e]) |
-                        ((uint32_t)float_to_bf16_bits(src[2 * e + 1]) << 16);
-              uint4 packed;
-              const float2 sc = fixed_point_quarter(make_uint4(wv[0], wv[1], wv[2], wv[3]),
-                                                    0xfu << (lane & ~3), packed);
-              const int ch = row0 / 32, R = G.rounds_b;
-              unsigned char* row = a.hq + (size_t)(p0 + t) * stride_b;
-              reinterpret_cast<uint4*>(row)[((ch / 32) * 4 + m) * 32 + (ch % 32)] = packed;
-              if (m == 0) reinterpret_cast<float2*>(row + act_digit_bytes(R))[ch] = sc;
-            }
-          }
-        }
+        // (the item's 32 h rows per pair form one chunk of h; the producer converts it
+        // to the fixed-point layout when it publishes the item)
       } else if (vid >= 0) {
         const int r = warp + kWarps * (vid / kNT), t = vid % kNT;
         if (r < nrows) a.y[(size_t)(p0 + t) * a.H + row0 + r] = v;
