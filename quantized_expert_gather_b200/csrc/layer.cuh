@@ -589,9 +589,13 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
   const int bpe_a = a.I / kRowsA;                     // phase-A blocks per segment
   const int ipa = bpe_a / kBlocksPerItemA;            // phase-A items per segment
   const int bpe_b = (a.H + G.rows_b - 1) / G.rows_b;  // phase-B blocks per segment
-  const int ipb = (bpe_b + kBlocksPerItemB - 1) / kBlocksPerItemB;  // phase-B items per segment
+  // phase-B items: kBlocksPerItemB blocks each, except in the last quarter of the
+  // segments, where single blocks keep the CTAs' finishing times close
+  const int ipb = (bpe_b + kBlocksPerItemB - 1) / kBlocksPerItemB;
+  const int seg_fine = nseg - (nseg + 3) / 4;  // first segment with single-block items
   const int n_items_a = nseg * ipa;
-  const int n_items = n_items_a + nseg * ipb;
+  const int n_items_b2 = seg_fine * ipb;
+  const int n_items = n_items_a + n_items_b2 + (nseg - seg_fine) * bpe_b;
 
   if (warp == kWarps + 1) {
     // ================================ helper warp ================================
@@ -756,9 +760,16 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
         blk0 = (item % ipa) * kBlocksPerItemA;
         nblk = kBlocksPerItemA;
       } else {
-        sg = (item - n_items_a) / ipb;
-        blk0 = ((item - n_items_a) % ipb) * kBlocksPerItemB;
-        nblk = min(kBlocksPerItemB, bpe_b - blk0);
+        const int j = item - n_items_a;
+        if (j < n_items_b2) {
+          sg = j / ipb;
+          blk0 = (j % ipb) * kBlocksPerItemB;
+          nblk = min(kBlocksPerItemB, bpe_b - blk0);
+        } else {
+          sg = seg_fine + (j - n_items_b2) / bpe_b;
+          blk0 = (j - n_items_b2) % bpe_b;
+          nblk = 1;
+        }
       }
       const int nt = seg_nt[sg], p0 = seg_pos[sg];
       // ---- its ring slot for publication must be free ----
@@ -993,7 +1004,9 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
               uv = Us[t];
             }
           const float g = round_to_bf16(gv), hu = round_to_bf16(uv);
-          const uint16_t hb = float_to_bf16_bits(g / (1.0f + __expf(-g)) * hu);
+          // silu(g) = g / (1 + e^-g); the fast division's error (2 ulp of fp32) is far
+          // below the bf16 step h is rounded to
+          const uint16_t hb = float_to_bf16_bits(__fdividef(g, 1.0f + __expf(-g)) * hu);
           a.h[(size_t)(p0 + lane) * a.I + row0 + warp] = hb;
           hs[lane * 32 + (row0 & 31) + warp] = hb;
         }
