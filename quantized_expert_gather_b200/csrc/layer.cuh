@@ -217,18 +217,19 @@ __device__ __forceinline__ float2 load_sc(const unsigned char* row, int R, int c
   return reinterpret_cast<const float2*>(row + act_digit_bytes(R))[ch];
 }
 
-// sum_c q_c v_c over one chunk (4 code words, 4 activation uint4), exact.
+// sum_c q_c v_c over one chunk (4 code words, 4 activation uint4), exact.  Four
+// partial sums keep the dp4a dependency chains short.
 __device__ __forceinline__ int chunk_dot(const uint32_t (&qs)[8], const uint4 (&x)[4]) {
-  int lo = 0, hi = 0;
+  int lo0 = 0, lo1 = 0, hi0 = 0, hi1 = 0;
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
     const uint4 d = x[m];
-    lo = dp4a_lo(qs[2 * m], d.x, lo);
-    lo = dp4a_lo(qs[2 * m + 1], d.y, lo);
-    hi = dp4a_hi(qs[2 * m], d.z, hi);
-    hi = dp4a_hi(qs[2 * m + 1], d.w, hi);
+    lo0 = dp4a_lo(qs[2 * m], d.x, lo0);
+    lo1 = dp4a_lo(qs[2 * m + 1], d.y, lo1);
+    hi0 = dp4a_hi(qs[2 * m], d.z, hi0);
+    hi1 = dp4a_hi(qs[2 * m + 1], d.w, hi1);
   }
-  return hi * 256 + lo;  // |.| < 2^24: exact in fp32
+  return (hi0 + hi1) * 256 + (lo0 + lo1);  // |.| < 2^24: exact in fp32
 }
 
 // The 32 codes of a uint4, split as described above.
@@ -334,7 +335,8 @@ __device__ __forceinline__ void rows_a(const unsigned char* bg_q, const uint16_t
 #pragma unroll
   for (int t = 0; t < NT; ++t) ag[t] = au[t] = 0.f;
   const int nch = H / 32;
-#pragma unroll 1
+  constexpr int kRoundUnroll = NT == 1 ? 2 : 1;  // one pair: two chunks in flight
+#pragma unroll kRoundUnroll
   for (int i = 0; i < R; ++i) {
     const int ch = i * 32 + lane;
     if (ch < nch) {
@@ -382,7 +384,8 @@ __device__ __forceinline__ float rows_b(const unsigned char* bq, const uint16_t*
 #pragma unroll
   for (int v = 0; v < V; ++v) acc[v] = 0.f;
   const int nch = I / 32, qstride = I / 2, sstride = I / 64;
-#pragma unroll 1
+  constexpr int kRoundUnroll = NT == 1 ? 2 : 1;  // one pair: two chunks in flight
+#pragma unroll kRoundUnroll
   for (int i = 0; i < R; ++i) {
     const int ch = i * 32 + lane;
     if (ch < nch) {
