@@ -52,6 +52,11 @@ def test_path_selection_without_launch():
         assert qeg.moe_select_path(T, 8, 256, 4096, 2048) == 1
     assert qeg.moe_select_path(1024, 1, 256, 4096, 2048) == 1
     assert qeg.moe_select_path(2, 2, 16, 256, 128) == 1
+    # large windows -> grouped tensor-core path (weight rows in multiples of 128)
+    assert qeg.moe_select_path(512, 8, 256, 4096, 2048) == 2
+    assert qeg.moe_select_path(2048, 8, 256, 4096, 2048) == 2
+    assert qeg.moe_select_path(160, 8, 64, 512, 256) == 2
+    assert qeg.moe_select_path(160, 8, 64, 512, 192) == 0  # inter not a multiple of 128
     # invalid shapes
     assert qeg.moe_select_path(0, 8, 256, 4096, 2048) == 0
     assert qeg.moe_select_path(4, 8, 256, 4000, 2048) == 0
@@ -64,7 +69,7 @@ def test_workspace_size_and_layout():
     n = qeg.moe_workspace_size(T, k, E, H, I)
     lay = qeg.moe_workspace_layout(T, k, E, H, I)
     assert lay["total"] == n
-    assert lay["barrier"] == 0 and lay["num_unique"] >= 4 * (1 + 1024 + 512)
+    assert lay["barrier"] == 0 and lay["num_unique"] >= 4 * (1 + 1024 + 512 + 2)
     # the counter region does not depend on the shape
     assert qeg.moe_workspace_layout(1, 1, 4, 64, 64)["num_unique"] == lay["num_unique"]
     assert lay["h"] % 256 == 0 and lay["h"] + 2 * T * k * I <= lay["y"]
