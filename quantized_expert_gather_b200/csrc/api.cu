@@ -51,8 +51,8 @@ moe_status device_info(DeviceInfo** out) {
     // dynamic + static shared memory may not exceed the opt-in limit
     const void* kernels[5] = {reinterpret_cast<const void*>(layer_kernel),
                               reinterpret_cast<const void*>(route_union_kernel),
-                              reinterpret_cast<const void*>(grouped_kernel<0>),
-                              reinterpret_cast<const void*>(grouped_kernel<1>),
+                              reinterpret_cast<const void*>(grouped_gemm_kernel<0>),
+                              reinterpret_cast<const void*>(grouped_gemm_kernel<1>),
                               reinterpret_cast<const void*>(grouped_combine_kernel)};
     for (int i = 0; i < 5; ++i) {
       cudaFuncAttributes fa;
@@ -84,8 +84,26 @@ bool shape_supported(int T, int k, int E, int hidden, int inter) {
 }
 
 struct WsLayout {
-  size_t barrier, num_unique, unique, offsets, pair_list, h, y, xg, hq, total;  // barrier = counters
+  size_t barrier, num_unique, unique, offsets, pair_list, h, y;  // barrier = counters
+  size_t xg, hq;                         // fused kernel: x and h rows in fixed point
+  size_t padded, xs, hs, xp, hp, pcap;   // grouped path: packed activations and sums
+  size_t total;
 };
+
+// 1 = the persistent fused kernel (small windows), 2 = the grouped tensor-core
+// kernels (windows with more pairs; hidden a multiple of 256, inter of 128),
+// 0 = neither.
+int select_path(int T, int k, int E, int hidden, int inter) {
+  if (!shape_ok(T, k, E, hidden, inter) || !shape_supported(T, k, E, hidden, inter)) return 0;
+  if (T * k <= kMaxPairsFused) {
+    LayerGeom g = layer_geom(hidden, inter);
+    if (g.seg >= 1 && fit_stages(g, E, T * k, hidden, inter, kSmemBudget)) return 1;
+  }
+  if (hidden % (2 * kGM) == 0 && inter % (2 * kGK) == 0 &&
+      route_union_smem_bytes(E) <= kSmemBudget && sizeof(int) * (size_t)T * k <= kSmemBudget)
+    return 2;
+  return 0;
+}
 
 WsLayout ws_layout(int T, int k, int E, int hidden, int inter) {
   const size_t P = (size_t)T * k;
@@ -98,25 +116,22 @@ WsLayout ws_layout(int T, int k, int E, int hidden, int inter) {
   w.pair_list = align_up(w.offsets + 4 * (m + 1), 16);
   w.h = align_up(w.pair_list + 4 * P, 256);
   w.y = align_up(w.h + 2 * P * (size_t)inter, 256);
+  const size_t tail = align_up(w.y + 4 * P * (size_t)hidden, 256);
+  // fused kernel
   const LayerGeom g = layer_geom(hidden, inter);
-  w.xg = align_up(w.y + 4 * P * (size_t)hidden, 256);     // x rows, fixed point
-  w.hq = align_up(w.xg + (size_t)T * act_bytes(g.rounds_a), 256);  // h rows, fixed point
-  w.total = align_up(w.hq + P * act_bytes(g.rounds_b), 256);
+  w.xg = tail;                                                        // x rows, fixed point
+  w.hq = align_up(w.xg + (size_t)T * act_bytes(g.rounds_a), 256);     // h rows, fixed point
+  const size_t total1 = align_up(w.hq + P * act_bytes(g.rounds_b), 256);
+  // grouped path: every expert's pairs padded to 16 rows
+  w.pcap = align_up(P + 15 * m, 16);
+  w.padded = tail;
+  w.xs = align_up(w.padded + 4 * (m + 1), 256);
+  w.hs = align_up(w.xs + 4 * (size_t)(hidden / kGK) * w.pcap, 256);
+  w.xp = align_up(w.hs + 4 * (size_t)(inter / kGK) * w.pcap, 256);
+  w.hp = align_up(w.xp + 2 * (size_t)hidden * w.pcap, 256);
+  const size_t total2 = align_up(w.hp + 2 * (size_t)inter * w.pcap, 256);
+  w.total = select_path(T, k, E, hidden, inter) == 2 ? total2 : total1;
   return w;
-}
-
-// 1 = the persistent fused kernel (small windows), 2 = the grouped tensor-core
-// kernels (windows with more pairs; weight rows in multiples of 128), 0 = neither.
-int select_path(int T, int k, int E, int hidden, int inter) {
-  if (!shape_ok(T, k, E, hidden, inter) || !shape_supported(T, k, E, hidden, inter)) return 0;
-  if (T * k <= kMaxPairsFused) {
-    LayerGeom g = layer_geom(hidden, inter);
-    if (g.seg >= 1 && fit_stages(g, E, T * k, hidden, inter, kSmemBudget)) return 1;
-  }
-  if (hidden % kGM == 0 && inter % kGM == 0 &&
-      route_union_smem_bytes(E) <= kSmemBudget && sizeof(int) * (size_t)T * k <= kSmemBudget)
-    return 2;
-  return 0;
 }
 
 cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
@@ -178,8 +193,9 @@ cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
   return cudaLaunchKernelEx(&c, layer_kernel, a);
 }
 
-// The grouped path: route-union, gate+up, down and combine as four launches on
-// `st` (no host synchronisation).  The union arrays, h and y live in the workspace.
+// The grouped path: route-union (with padded offsets), x packing, gate+up, down
+// and combine as five launches on `st` (no host synchronisation).  The union
+// arrays, the packed activations, their sums and y live in the workspace.
 cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w,
                            const uint32_t* gq, const uint16_t* gs, const uint16_t* gb,
                            const uint32_t* uq, const uint16_t* us, const uint16_t* ub,
@@ -192,8 +208,14 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   int* uniq = reinterpret_cast<int*>(ws + wl.unique);
   int* offs = reinterpret_cast<int*>(ws + wl.offsets);
   int* plist = reinterpret_cast<int*>(ws + wl.pair_list);
-  uint16_t* h = reinterpret_cast<uint16_t*>(ws + wl.h);
   float* y = reinterpret_cast<float*>(ws + wl.y);
+  int* padded = reinterpret_cast<int*>(ws + wl.padded);
+  float* xs = reinterpret_cast<float*>(ws + wl.xs);
+  float* hs = reinterpret_cast<float*>(ws + wl.hs);
+  uint16_t* xp = reinterpret_cast<uint16_t*>(ws + wl.xp);
+  uint16_t* hp = reinterpret_cast<uint16_t*>(ws + wl.hp);
+  const int pcap = static_cast<int>(wl.pcap);
+  const int m = P < E ? P : E;
   const size_t usmem = route_union_smem_bytes(E);
   const size_t csmem = sizeof(int) * (size_t)P;
   if (usmem > (size_t)d.dyn_smem[1] || kGSmem > (unsigned)d.dyn_smem[2] ||
@@ -201,38 +223,45 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
     *why = MOE_ERR_UNSUPPORTED;
     return cudaSuccess;
   }
-  route_union_kernel<<<1, 32 * kUnionWarps, usmem, st>>>(idx, P, E, uniq, offs, plist, nu);
+  route_union_kernel<<<1, 32 * kUnionWarps, usmem, st>>>(idx, P, E, uniq, offs, plist, nu,
+                                                         padded);
+  grouped_pack_x_kernel<<<m < 4 * d.sms ? m : 4 * d.sms, 256, 0, st>>>(x, plist, offs, padded,
+                                                                         nu, k, H, pcap, xp, xs);
   GroupedArgs g{};
   g.unique = uniq;
   g.offsets = offs;
-  g.pair_list = plist;
+  g.padded = padded;
   g.num_unique = nu;
-  g.k = k;
+  g.pcap = pcap;
   g.H = H;
-  g.I = I;
-  g.h = h;
+  g.hp = hp;
+  g.hs = hs;
   g.y = y;
-  // gate + up: weight rows I, K = H, activations x
-  g.act = x;
-  g.q0 = gq;
-  g.s0 = gs;
-  g.b0 = gb;
-  g.q1 = uq;
-  g.s1 = us;
-  g.b1 = ub;
+  // gate + up: 128 rows of Wg and the same 128 rows of Wu per tile, K = H, packed x
+  g.bp = xp;
+  g.bs = xs;
+  g.q[0] = gq;
+  g.s[0] = gs;
+  g.b[0] = gb;
+  g.q[1] = uq;
+  g.s[1] = us;
+  g.b[1] = ub;
+  g.roff[0] = g.roff[1] = 0;
   g.rows = I;
   g.K = H;
-  grouped_kernel<0><<<d.sms, kGThreads, kGSmem, st>>>(g);
-  // down: weight rows H, K = I, activations h
-  g.act = h;
-  g.q0 = dq;
-  g.s0 = ds;
-  g.b0 = db;
-  g.q1 = nullptr;
-  g.s1 = g.b1 = nullptr;
+  g.mrows = kGM;
+  grouped_gemm_kernel<0><<<d.sms, kGThreads, kGSmem, st>>>(g);
+  // down: 256 rows of Wd per tile (two 128-row matrices), K = I, packed h
+  g.bp = hp;
+  g.bs = hs;
+  g.q[0] = g.q[1] = dq;
+  g.s[0] = g.s[1] = ds;
+  g.b[0] = g.b[1] = db;
+  g.roff[1] = kGM;
   g.rows = H;
   g.K = I;
-  grouped_kernel<1><<<d.sms, kGThreads, kGSmem, st>>>(g);
+  g.mrows = 2 * kGM;
+  grouped_gemm_kernel<1><<<d.sms, kGThreads, kGSmem, st>>>(g);
   grouped_combine_kernel<<<d.sms, 256, csmem, st>>>(y, w, plist, offs, nu, T, k, H, out);
   return cudaGetLastError();
 }

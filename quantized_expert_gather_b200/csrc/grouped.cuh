@@ -7,38 +7,80 @@
 // one matrix product (the sorted grouped path).  Here, after the route-union
 // (route_union.cuh) has grouped the pairs by expert:
 //
-//   grouped_kernel<0>  gate+up: for each (expert slot, 128 rows of Wg/Wu) tile,
-//                      G = Wg X^T and U = Wu X^T over the expert's tokens, with
-//                      h = bf16(silu(bf16 G) * bf16 U) stored per pair;
-//   grouped_kernel<1>  down: for each (expert slot, 128 rows of Wd) tile,
-//                      Y = Wd H^T over the expert's pairs, fp32 per pair;
-//   combine_kernel     out[t] = bf16(sum_j w[t,j] * y[t,j]), j ascending.
+//   grouped_pack_x_kernel   the window's x rows, one per pair, in the order and
+//                           layout the tensor cores read (below), with group sums;
+//   grouped_gemm_kernel<0>  gate+up: per (expert, 128 rows of Wg and of Wu) tile,
+//                           G = Wg X^T, U = Wu X^T, h = bf16(silu(bf16 G) * bf16 U),
+//                           h written packed for the next launch;
+//   grouped_gemm_kernel<1>  down: per (expert, 256 rows of Wd) tile, Y = Wd H^T,
+//                           fp32 per pair;
+//   grouped_combine_kernel  out[t] = bf16(sum_j w[t,j] * y[t,j]), j ascending.
 //
-// A tile is M = 128 weight rows by N = the expert's pairs (at most 256 at a
-// time, padded to a multiple of 16), K in slabs of 64.  Per slab all threads
-// dequantise the 4-bit codes, w = s * q + b in fp32, and split each weight into
-// two bf16 parts, hi = bf16(w) and lo = bf16(w - hi) (hi + lo holds w to about 16
-// significant bits), and gather the activation rows (bf16, exact), all into
-// 128-byte-swizzled K-major shared-memory tiles; one thread issues tcgen05.mma
-// (bf16 x bf16, fp32 accumulator in tensor memory) for hi and for lo into the
-// same accumulator and commits to an mbarrier.  Two slab buffers let
-// the dequantisation of slab s+1 overlap the MMAs of slab s.  The epilogue warps
-// read the accumulators with tcgen05.ld.
+// The quantisation group (64 columns of K) is the MMA's K slab.  Inside a group
+// a weight row is s * q + b, so its dot product with an activation row a splits
+// as  sum_c w_c a_c = s * (sum_c q_c a_c) + b * (sum_c a_c).  The tensor cores
+// form P = sum_c q_c a_c from bf16 operands: the codes 0..15 are exact bf16
+// integers, the activations are bf16 already, each product is exact and the sum
+// is fp32.  Every slab's P is read back from tensor memory and s * P + b * X (X
+// the activation row's group sum) is added to fp32 registers.  No weight is ever
+// rounded; the only per-weight work is turning 4-bit codes into bf16 integers.
+//
+// Roles in a CTA (one CTA per SM, looping over tiles):
+//   warp 8      producer: per stage of two slabs, 16-byte async copies of each
+//               weight row's codes (64 bytes) and 4-byte ones of its scales and
+//               biases, and 1-D bulk copies of the two packed activation slabs and
+//               of their group sums;
+//   warp 9      MMA issuer: issues tcgen05.mma (one elected lane of the converged
+//               warp) with A (the codes as bf16) in tensor memory and B (the
+//               activations) in shared memory;
+//   warps 0..7  warps 4m..4m+3 own matrix m of the tile, one weight row per
+//               thread (the row's tensor-memory lane).  Per slab they expand the
+//               row's codes to bf16 into tensor memory (the MMA's A operand), then
+//               read back the previous slab's product and accumulate it.
+// Codes expand without conversions: nibble q placed under the bf16 exponent of
+// 128 reads as 128 + q, and one packed bf16 FMA takes the 128 off exactly.  That
+// puts codes j and j + 4 of a 32-bit code word in one bf16 pair, so K runs in
+// the order (0,4,1,5,2,6,3,7) within every 8 columns; the packed activations
+// follow the same order.
+//
+// Packed activations (the B operand): [K/64][pcap][64] bf16.  Row = padded pair
+// position: expert slot i owns rows padded[i] .. padded[i] + roundup16(count_i)
+// (route_union_kernel's padded offsets), with zero rows as padding.  Each 128-byte
+// row holds one slab in the K order above, its 16-byte chunk c stored at chunk
+// (c ^ (row & 7)): the 128-byte swizzle of a K-major tile whose rows start at
+// multiples of 8.  Group sums: [K/64][pcap] fp32.
 #pragma once
 
 #include "common.cuh"
 
 namespace qeg {
 
-constexpr int kGThreads = 256;       // 8 warps
-constexpr int kGM = 128;             // weight rows per tile (MMA M)
-constexpr int kGMaxN = 256;          // pairs per MMA (MMA N, multiple of 16)
-constexpr int kGK = 64;              // K per slab (one 128-byte swizzle row of bf16)
-constexpr unsigned kGATile = kGM * kGK * 2;     // 16 KB: one matrix slab
-constexpr unsigned kGBTile = kGMaxN * kGK * 2;  // 32 KB: activation slab
-// dynamic shared memory: per buffer [A0hi | A0lo | A1hi | A1lo | B] (A1 only for
-// gate+up), 2 buffers
-constexpr unsigned kGSmem = 2 * (4 * kGATile + kGBTile) + 1024;  // + alignment slack
+constexpr int kGWorkers = 8;                         // worker warps
+constexpr int kGThreads = 32 * (kGWorkers + 2);      // + producer warp + MMA warp
+constexpr int kGM = 128;                             // weight rows per matrix (MMA M)
+constexpr int kGN = 64;                              // pairs per chunk (MMA N <= 64)
+constexpr int kGK = 64;                              // K per slab = quantisation group
+constexpr int kGSlabsPerStage = 2;
+constexpr int kGStages = 5;
+constexpr unsigned kGCodePitch = kGSlabsPerStage * 32 + 16;  // padded: no bank conflicts
+constexpr unsigned kGOffB = 2 * kGM * kGCodePitch;           // 20480, a multiple of 1024
+constexpr unsigned kGBTile = kGN * kGK * 2;                  // 8 KB per slab
+constexpr unsigned kGOffX = kGOffB + kGSlabsPerStage * kGBTile;
+constexpr unsigned kGOffS = kGOffX + kGSlabsPerStage * kGN * 4;
+constexpr unsigned kGOffBias = kGOffS + 2 * kGM * kGSlabsPerStage * 2;
+constexpr unsigned kGStageBytes = (kGOffBias + 2 * kGM * kGSlabsPerStage * 2 + 1023) & ~1023u;
+constexpr unsigned kGSmem = kGStages * kGStageBytes + 1024;  // + alignment slack
+constexpr int kGDBufs = 3;   // accumulator buffers: a slab is read back two slabs later
+constexpr int kGABufs = 2;   // A operand buffers
+constexpr uint32_t kGTmemCols = 512;
+static_assert(kGOffB % 1024 == 0 && kGBTile % 1024 == 0, "swizzled tiles need 1024-byte bases");
+static_assert(kGDBufs * 2 * kGN + kGABufs * 2 * 32 <= (int)kGTmemCols, "tensor memory map");
+
+// Tensor-memory columns: accumulator of buffer db, matrix m; A operand of buffer ab.
+__device__ __forceinline__ uint32_t g_col_d(uint32_t db, int m) { return (db * 2 + m) * kGN; }
+__device__ __forceinline__ uint32_t g_col_a(uint32_t ab, int m) {
+  return kGDBufs * 2 * kGN + (ab * 2 + m) * 32;
+}
 
 // ------------------------------------------------------------ tcgen05 helpers ---
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -60,13 +102,31 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (both operands bf16).
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16 (both operands bf16).
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// The same, issued by one elected lane of a converged warp: the whole warp runs the
+// issuing code, so its operands stay warp-uniform (issue is several times faster
+// than from a single divergent thread).
+__device__ __forceinline__ void tc_mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p, e;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit_elect(uint64_t* bar) {
+  asm volatile(
+      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}\n" ::"r"(
+          smem_u32(bar))
       : "memory");
 }
 // The mbarrier receives one arrival when every MMA this thread issued so far is done.
@@ -76,9 +136,8 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
           smem_u32(bar))
       : "memory");
 }
-// 16 consecutive fp32 columns of this thread's tensor-memory lane.
-__device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
+// 16 consecutive 32-bit columns of this thread's lane (no wait).
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t* r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
       "%15}, [%16];"
@@ -87,9 +146,30 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
         "=r"(r[14]), "=r"(r[15])
       : "r"(taddr)
       : "memory");
+}
+__device__ __forceinline__ void tc_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+// After tc_wait_ld: ties 16 loaded registers to the wait, so that no use of them
+// is scheduled before it.
+__device__ __forceinline__ void tc_regs_ready(uint32_t* r) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]));
+}
+// 16 consecutive 32-bit columns of this thread's lane <- r (no wait).
+__device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tc_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // Shared-memory matrix descriptor of a K-major, 128-byte-swizzled tile: rows of 128
@@ -117,262 +197,430 @@ __device__ __forceinline__ uint32_t f16_idesc(int M, int N) {
          ((uint32_t)(M >> 4) << 24);
 }
 
-// Byte offset of the 16-byte chunk c (0..7) of row r in a 128-byte-swizzled tile.
-__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
-  return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+// 4-byte async copy global -> shared (both 4-byte aligned).
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+// 16-byte async copy global -> shared (both 16-byte aligned), bypassing L1.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+// One arrival on `bar` once this thread's earlier cp.async copies have landed
+// (counted in the barrier's expected arrivals).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
 }
 
-// Codes -> floats without integer conversion: nibble j of a word ORed under the
-// exponent (150 - 4j) reads as 2^(23-4j) + q exactly, and one packed add removes
-// the offset.  Masks and exponents live in registers (one LOP3 per nibble).
-struct NibbleConsts {
-  uint32_t m0, m1, m2, m3, m4, e150, e146, e142, e138, e134;
-};
-__device__ __forceinline__ NibbleConsts nibble_consts() {
-  NibbleConsts k{0xFu, 0xF0u, 0xF00u, 0xF000u, 0xF0000u,
-                 150u << 23, 146u << 23, 142u << 23, 138u << 23, 134u << 23};
-  asm volatile("" : "+r"(k.m0), "+r"(k.m1), "+r"(k.m2), "+r"(k.m3), "+r"(k.m4));
-  asm volatile("" : "+r"(k.e150), "+r"(k.e146), "+r"(k.e142), "+r"(k.e138), "+r"(k.e134));
-  return k;
-}
-__device__ __forceinline__ float or_and(uint32_t a, uint32_t m, uint32_t e) {
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(m), "r"(e));
-  return __uint_as_float(d);
-}
-// The 8 codes of w (element j = nibble j) as (q0,q1) (q2,q3) (q4,q5) (q6,q7).
-__device__ __forceinline__ void nibbles8(uint32_t w, const NibbleConsts& k, float2 (&q)[4]) {
-  const uint32_t w2 = w >> 12;
-  q[0] = __fadd2_rn(make_float2(or_and(w, k.m0, k.e150), or_and(w, k.m1, k.e146)),
-                    make_float2(-8388608.f, -524288.f));
-  q[1] = __fadd2_rn(make_float2(or_and(w, k.m2, k.e142), or_and(w, k.m3, k.e138)),
-                    make_float2(-32768.f, -2048.f));
-  q[2] = __fadd2_rn(make_float2(or_and(w, k.m4, k.e134), or_and(w2, k.m2, k.e142)),
-                    make_float2(-128.f, -32768.f));
-  q[3] = __fadd2_rn(make_float2(or_and(w2, k.m3, k.e138), or_and(w2, k.m4, k.e134)),
-                    make_float2(-2048.f, -128.f));
-}
-// Packed bf16 pair (round to nearest even) of two floats: low half = a.
-__device__ __forceinline__ uint32_t bf16x2_rn(float a, float b) {
-  uint32_t d;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(b), "f"(a));
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
   return d;
 }
-// One code word's 8 weights w = s*q + b as bf16 hi (= bf16(w)) and lo (= bf16(w - hi)).
-__device__ __forceinline__ void dequant8_hilo(uint32_t w, float2 s2, float2 b2,
-                                              const NibbleConsts& k, uint4& hi, uint4& lo) {
-  float2 q[4];
-  nibbles8(w, k, q);
-  uint32_t h[4], l[4];
+
+// The 8 codes of word w as 4 bf16 pairs (low half q_j, high half q_{j+4}),
+// j = 0..3, exact.  one2 = bf16 pair (1, 1), m128 = (-128, -128).
+__device__ __forceinline__ void codes_to_bf16(uint32_t w, uint32_t one2, uint32_t m128,
+                                              uint32_t* o) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const float2 v = __ffma2_rn(q[j], s2, b2);
-    h[j] = bf16x2_rn(v.x, v.y);
-    const float2 hv = make_float2(__uint_as_float(h[j] << 16), __uint_as_float(h[j] & 0xffff0000u));
-    const float2 r = __fadd2_rn(v, make_float2(-hv.x, -hv.y));  // exact
-    l[j] = bf16x2_rn(r.x, r.y);
+    const uint32_t t = ((w >> (4 * j)) & 0x000F000Fu) | 0x43004300u;  // 128 + q
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(o[j]) : "r"(t), "r"(one2), "r"(m128));
   }
-  hi = make_uint4(h[0], h[1], h[2], h[3]);
-  lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
-// ------------------------------------------------------------------ kernels ---
+// --------------------------------------------------------------- packing ---
+// Packed x: for every padded pair position of every expert slot, the pair's token
+// row of x (zero for padding) and its group sums.  One block per slot (looping).
+__global__ void __launch_bounds__(256) grouped_pack_x_kernel(
+    const uint16_t* __restrict__ x, const int* __restrict__ pair_list,
+    const int* __restrict__ offsets, const int* __restrict__ padded,
+    const int* __restrict__ num_unique, int k, int H, int pcap, uint16_t* __restrict__ xp,
+    float* __restrict__ xs) {
+  const int u = *num_unique;
+  const int nslab = H / kGK;
+  for (int slot = blockIdx.x; slot < u; slot += gridDim.x) {
+    const int p0 = offsets[slot], cnt = offsets[slot + 1] - p0;
+    const int np = (cnt + 15) & ~15;
+    const int base = padded[slot];
+    const int units = np * nslab * 8;  // a multiple of 128: whole warps stay together
+    for (int unit = threadIdx.x; unit < units; unit += blockDim.x) {
+      const int c = unit & 7, rest = unit >> 3;
+      const int g = rest % nslab, n = rest / nslab;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (n < cnt) {
+        const int t = pair_list[p0 + n] / k;
+        v = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H + g * kGK + c * 8));
+      }
+      float s = ((bf16_lo(v.x) + bf16_hi(v.x)) + (bf16_lo(v.y) + bf16_hi(v.y))) +
+                ((bf16_lo(v.z) + bf16_hi(v.z)) + (bf16_lo(v.w) + bf16_hi(v.w)));
+      s += __shfl_xor_sync(kFull, s, 1);
+      s += __shfl_xor_sync(kFull, s, 2);
+      s += __shfl_xor_sync(kFull, s, 4);
+      uint4 o;  // K order (0,4,1,5,2,6,3,7)
+      o.x = prmt(v.x, v.z, 0x5410u);
+      o.y = prmt(v.x, v.z, 0x7632u);
+      o.z = prmt(v.y, v.w, 0x5410u);
+      o.w = prmt(v.y, v.w, 0x7632u);
+      const int pos = base + n;
+      *reinterpret_cast<uint4*>(xp + ((size_t)g * pcap + pos) * kGK + ((c ^ (pos & 7)) * 8)) = o;
+      if (c == 0) xs[(size_t)g * pcap + pos] = s;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ GEMMs ---
 struct GroupedArgs {
-  const uint16_t* act;   // phase 0: x [T, H]; phase 1: h [P, I] (pair_list order)
+  const uint16_t* bp;    // packed activations [K/64][pcap][64] (x or h)
+  const float* bs;       // their group sums [K/64][pcap]
   const int* unique;     // [u] distinct experts, ascending
   const int* offsets;    // [u + 1]
-  const int* pair_list;  // [P] pair ids grouped by expert
+  const int* padded;     // [u + 1] padded row offsets of the packed layout
   const int* num_unique; // [1]
-  const uint32_t *q0, *q1;   // codes: phase 0 gate / up, phase 1 down
-  const uint16_t *s0, *b0, *s1, *b1;
-  uint16_t* h;           // phase 0 output [P, I] bf16
-  float* y;              // phase 1 output [P, H] fp32
-  int k, rows, K;        // top-k; weight rows per expert (I or H); K (H or I)
-  int H, I;
+  const uint32_t* q[2];  // codes of matrix 0 / 1 of a tile
+  const uint16_t* s[2];  // scales
+  const uint16_t* b[2];  // biases
+  int roff[2];           // row offset of matrix m inside the tile (0/0 or 0/128)
+  uint16_t* hp;          // phase 0: packed h [I/64][pcap][64]
+  float* hs;             // phase 0: h group sums [I/64][pcap]
+  float* y;              // phase 1: [P, H] fp32 in pair_list order
+  int rows, K, mrows;    // weight rows per expert; K; weight rows per tile
+  int pcap, H;
 };
 
-// One launch per phase, one CTA per SM looping over (expert slot, 128-row tile).
 template <int PHASE>
-__global__ void __launch_bounds__(kGThreads, 1) grouped_kernel(const GroupedArgs a) {
+__global__ void __launch_bounds__(kGThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ GroupedArgs a) {
   extern __shared__ __align__(128) unsigned char gsm_raw[];
-  __shared__ __align__(8) uint64_t mma_done[2];
+  __shared__ __align__(8) uint64_t full[kGStages], empty[kGStages];
+  __shared__ __align__(8) uint64_t a_full[kGABufs], d_full[kGDBufs], d_free[kGDBufs];
   __shared__ uint32_t tmem_base_s;
+  __shared__ float red[2][2][32];
   // swizzled tiles start at 1024-byte boundaries of the shared address space
   unsigned char* gsm = gsm_raw + ((1024u - (smem_u32(gsm_raw) & 1023u)) & 1023u);
-  constexpr int NMAT = PHASE == 0 ? 2 : 1;
-  constexpr unsigned kBuf = 2 * NMAT * kGATile + kGBTile;
-  constexpr uint32_t kCols = PHASE == 0 ? 2 * kGMaxN : kGMaxN;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
-    mbar_init(&mma_done[0], 1);
-    mbar_init(&mma_done[1], 1);
+    for (int i = 0; i < kGStages; ++i) {
+      mbar_init(&full[i], 1 + 32);          // expect_tx + one cp.async arrival per lane
+      mbar_init(&empty[i], kGWorkers + 1);  // worker warps + the MMA commit
+    }
+    for (int i = 0; i < kGABufs; ++i) mbar_init(&a_full[i], kGWorkers);
+    for (int i = 0; i < kGDBufs; ++i) {
+      mbar_init(&d_full[i], 1);
+      mbar_init(&d_free[i], kGWorkers);
+    }
     fence_barrier_init();
   }
-  if (warp == 0) {
-    tmem_alloc(&tmem_base_s, kCols);
+  if (warp == kGWorkers + 1) {
+    tmem_alloc(&tmem_base_s, kGTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = tmem_base_s;
+  const uint32_t tmem = __shfl_sync(kFull, tmem_base_s, 0);  // warp-uniform
 
   const int u = *a.num_unique;
-  const int mtiles = a.rows / kGM;
+  const int mtiles = a.rows / a.mrows;
   const int nslab = a.K / kGK;
-  uint32_t phase_bits = 0;  // completed-phase parity of mma_done[0], [1]
+  const int ntiles = u * mtiles;
   bool ok = true;
-  const NibbleConsts nk = nibble_consts();
+  uint32_t sc = 0;  // stages started (the same sequence in every role)
+  uint32_t gs = 0;  // slabs started
 
-  for (int tile = blockIdx.x; tile < u * mtiles && ok; tile += gridDim.x) {
-    const int slot = tile / mtiles, m0 = (tile % mtiles) * kGM;
-    const int e = a.unique[slot];
-    const int p_begin = a.offsets[slot], p_end = a.offsets[slot + 1];
-    const size_t wrow0 = (size_t)e * a.rows + m0;  // first weight row of the tile
-    for (int n0 = p_begin; n0 < p_end && ok; n0 += kGMaxN) {
-      const int n = min(kGMaxN, p_end - n0);
-      const int np = (n + 15) & ~15;  // MMA N
-      const uint32_t idesc = f16_idesc(kGM, np);
-      int issued = 0;  // slabs whose MMAs were issued (in this n-chunk)
-      // Per thread: A tasks (matrix, row, half slab of 32 columns) tid and tid + 256
-      // (gate+up), B tasks (pair row, 16-byte chunk) tid + 256 i.  Their global data
-      // for slab s+1 is loaded while slab s is dequantised and multiplied.
-      constexpr int kATasks = NMAT * kGM * 2 / kGThreads;  // 2 or 1
-      constexpr int kBTasks = kGMaxN * 8 / kGThreads;      // 8
-      uint4 cw[kATasks];
-      uint16_t sraw[kATasks], braw[kATasks];
-      uint4 xv[kBTasks];
-      auto load_slab = [&](int s) {
-#pragma unroll
-        for (int i = 0; i < kATasks; ++i) {
-          const int task = tid + i * kGThreads;
-          const int mat = task / (kGM * 2), rr = (task >> 1) % kGM, half = task & 1;
-          const uint32_t* q = mat ? a.q1 : a.q0;
-          const uint16_t* sp = mat ? a.s1 : a.s0;
-          const uint16_t* bp = mat ? a.b1 : a.b0;
-          const size_t row = wrow0 + rr;
-          cw[i] = __ldg(reinterpret_cast<const uint4*>(q + row * (a.K / 8) + s * 8) + half);
-          sraw[i] = __ldg(sp + row * (a.K / 64) + s);
-          braw[i] = __ldg(bp + row * (a.K / 64) + s);
-        }
-#pragma unroll
-        for (int i = 0; i < kBTasks; ++i) {
-          const int task = tid + i * kGThreads, rr = task >> 3, c = task & 7;
-          xv[i] = make_uint4(0u, 0u, 0u, 0u);
-          if (rr < n) {
-            const int pos = n0 + rr;
-            const size_t arow = PHASE == 0 ? (size_t)(a.pair_list[pos] / a.k) : (size_t)pos;
-            const uint16_t* src = a.act + arow * a.K + s * kGK + c * 8;
-            xv[i] = PHASE == 0 ? __ldg(reinterpret_cast<const uint4*>(src))
-                               : __ldcg(reinterpret_cast<const uint4*>(src));
+  if (warp == kGWorkers) {
+    // ------------------------------------------------------------ producer ---
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      const int slot = tile / mtiles, m0 = (tile % mtiles) * a.mrows;
+      const int e = a.unique[slot];
+      const int cnt = a.offsets[slot + 1] - a.offsets[slot];
+      const int pp0 = a.padded[slot];
+      for (int c0 = 0; c0 < cnt && ok; c0 += kGN) {
+        const int np = (min(kGN, cnt - c0) + 15) & ~15;
+        for (int j0 = 0; j0 < nslab && ok; j0 += kGSlabsPerStage) {
+          const int st = sc % kGStages;
+          const uint32_t round = sc / kGStages;
+          if (lane == 0) {
+            if (round > 0) ok = mbar_wait(&empty[st], (round - 1) & 1);
+            if (ok)
+              mbar_arrive_expect_tx(&full[st], kGSlabsPerStage * np * (kGK * 2 + 4));
           }
-        }
-      };
-      load_slab(0);
-      for (int s = 0; s < nslab && ok; ++s) {
-        const int buf = s & 1;
-        unsigned char* base = gsm + buf * kBuf;
-        if (s >= 2) {  // the MMAs that read this buffer two slabs ago are done
-          ok = mbar_wait(&mma_done[buf], (phase_bits >> buf) & 1);
-          phase_bits ^= 1u << buf;
+          ok = __shfl_sync(kFull, ok, 0);
           if (!ok) break;
-        }
-        uint4 ccw[kATasks], cxv[kBTasks];
-        uint16_t cs[kATasks], cb[kATasks];
-#pragma unroll
-        for (int i = 0; i < kATasks; ++i) {
-          ccw[i] = cw[i];
-          cs[i] = sraw[i];
-          cb[i] = braw[i];
-        }
-#pragma unroll
-        for (int i = 0; i < kBTasks; ++i) cxv[i] = xv[i];
-        if (s + 1 < nslab) load_slab(s + 1);
-        // --- A: dequantised weight slab(s), 128 rows x 64, hi and lo, swizzled ---
-#pragma unroll
-        for (int i = 0; i < kATasks; ++i) {
-          const int task = tid + i * kGThreads;
-          const int mat = task / (kGM * 2), rr = (task >> 1) % kGM, half = task & 1;
-          const float sc = bf16_bits_to_float(cs[i]), bi = bf16_bits_to_float(cb[i]);
-          const float2 s2 = make_float2(sc, sc), b2 = make_float2(bi, bi);
-          unsigned char* tileA = base + 2 * mat * kGATile;  // hi tile; lo tile follows
-          const uint32_t ws[4] = {ccw[i].x, ccw[i].y, ccw[i].z, ccw[i].w};
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {  // 16-byte chunk = 8 columns = one code word
-            uint4 hi, lo;
-            dequant8_hilo(ws[c], s2, b2, nk, hi, lo);
-            const uint32_t off = sw128_off(rr, half * 4 + c);
-            *reinterpret_cast<uint4*>(tileA + off) = hi;
-            *reinterpret_cast<uint4*>(tileA + kGATile + off) = lo;
+          unsigned char* stg = gsm + st * kGStageBytes;
+          // codes: 16 bytes per lane, four lanes per row (64 bytes = two slabs)
+#pragma unroll 8
+          for (int i = 0; i < 2 * kGM * kGSlabsPerStage * 2 / 32; ++i) {
+            const int ci = lane + 32 * i, rr = ci >> 2, c = ci & 3;
+            const int m = rr / kGM, r = rr % kGM;
+            const size_t row = (size_t)e * a.rows + m0 + a.roff[m] + r;
+            cp_async16(stg + rr * kGCodePitch + c * 16, a.q[m] + row * (a.K / 8) + j0 * 8 + c * 4);
           }
-        }
-        // --- B: the activation rows of the slab (zero rows up to np), swizzled ---
-        unsigned char* tileB = base + 2 * NMAT * kGATile;
+          // scales and biases of the two slabs: 4 bytes per row each
 #pragma unroll
-        for (int i = 0; i < kBTasks; ++i) {
-          const int task = tid + i * kGThreads, rr = task >> 3, c = task & 7;
-          if (rr < np) *reinterpret_cast<uint4*>(tileB + sw128_off(rr, c)) = cxv[i];
-        }
-        fence_proxy_async();  // generic smem writes -> tensor-core reads
-        __syncthreads();
-        if (tid == 0) {
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(base), b_addr = smem_u32(tileB);
+          for (int i = 0; i < 2 * kGM / 32; ++i) {
+            const int rr = lane + 32 * i, m = rr / kGM, r = rr % kGM;
+            const size_t row = (size_t)e * a.rows + m0 + a.roff[m] + r;
+            cp_async4(stg + kGOffS + rr * 4, a.s[m] + row * (a.K / kGK) + j0);
+            cp_async4(stg + kGOffBias + rr * 4, a.b[m] + row * (a.K / kGK) + j0);
+          }
+          if (lane == 0) {
 #pragma unroll
-          for (int kk = 0; kk < kGK / 16; ++kk) {
-            const uint64_t bdesc = sw128_desc(b_addr + kk * 32);
-#pragma unroll
-            for (int mat = 0; mat < NMAT; ++mat) {
-              const uint32_t a_hi = a_addr + 2 * mat * kGATile + kk * 32;
-              tc_mma(tmem + mat * kGMaxN, sw128_desc(a_hi), bdesc, idesc,
-                     (s > 0 || kk > 0) ? 1u : 0u);
-              tc_mma(tmem + mat * kGMaxN, sw128_desc(a_hi + kGATile), bdesc, idesc, 1u);
+            for (int jj = 0; jj < kGSlabsPerStage; ++jj) {
+              const size_t prow = (size_t)(j0 + jj) * a.pcap + pp0 + c0;
+              bulk_g2s(stg + kGOffB + jj * kGBTile, a.bp + prow * kGK, np * kGK * 2, &full[st]);
+              bulk_g2s(stg + kGOffX + jj * kGN * 4, a.bs + prow, np * 4, &full[st]);
             }
           }
-          tc_commit(&mma_done[buf]);
+          cp_async_arrive_noinc(&full[st]);
+          ++sc;
         }
-        ++issued;
       }
-      // all MMAs of the chunk done (the last one or two commits not waited yet)
-      for (int s = (issued > 2 ? issued - 2 : 0); s < issued && ok; ++s) {
-        const int buf = s & 1;
-        ok = mbar_wait(&mma_done[buf], (phase_bits >> buf) & 1);
-        phase_bits ^= 1u << buf;
-      }
-      tc_fence_after();
-      // --- epilogue: warp w reads lanes 32 (w % 4).., columns half (w / 4) ---
-      if (ok) {
-        const int r = 32 * (warp & 3) + lane;  // tile row of this thread
-        const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-        for (int c0 = (warp >> 2) * 16; c0 < np; c0 += 32) {
-          float d0[16];
-          tc_ld16(lane_addr + c0, d0);
-          if (PHASE == 0) {
-            float d1[16];
-            tc_ld16(lane_addr + kGMaxN + c0, d1);
+    }
+    // leave no copy in flight: every stage issued has landed (at once when all went well)
+    if (lane == 0)
+      for (uint32_t i = sc > (uint32_t)kGStages ? sc - kGStages : 0; i < sc; ++i)
+        mbar_wait(&full[i % kGStages], (i / kGStages) & 1);
+  } else if (warp == kGWorkers + 1) {
+    // ---------------------------------------------------------- MMA issuer ---
+    // The whole warp runs this loop (operands warp-uniform); one elected lane issues.
+    uint32_t issued = 0;  // slabs whose MMAs were issued
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      const int slot = tile / mtiles;
+      const int cnt = a.offsets[slot + 1] - a.offsets[slot];
+      for (int c0 = 0; c0 < cnt && ok; c0 += kGN) {
+        const int np = (min(kGN, cnt - c0) + 15) & ~15;
+        const uint32_t idesc = f16_idesc(kGM, np);
+        for (int j0 = 0; j0 < nslab && ok; j0 += kGSlabsPerStage, ++sc) {
+          const int st = sc % kGStages;
+          const uint32_t round = sc / kGStages;
+          ok = __all_sync(kFull, mbar_wait(&full[st], round & 1));
+          const uint32_t bbase = smem_u32(gsm + st * kGStageBytes + kGOffB);
+          for (int jj = 0; jj < kGSlabsPerStage && ok; ++jj, ++gs) {
+            const uint32_t ab = gs % kGABufs, db = gs % kGDBufs;
+            bool w = mbar_wait(&a_full[ab], (gs / kGABufs) & 1);
+            if (w && gs >= (uint32_t)kGDBufs) w = mbar_wait(&d_free[db], (gs / kGDBufs - 1) & 1);
+            ok = __all_sync(kFull, w);
+            if (!ok) break;
+            tc_fence_after();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              if (c0 + j < n) {
-                const float g = round_to_bf16(d0[j]), uv = round_to_bf16(d1[j]);
-                a.h[(size_t)(n0 + c0 + j) * a.I + m0 + r] =
-                    float_to_bf16_bits(g / (1.0f + __expf(-g)) * uv);
+            for (int kk = 0; kk < kGK / 16; ++kk) {
+              const uint64_t bdesc = sw128_desc(bbase + jj * kGBTile + kk * 32);
+#pragma unroll
+              for (int m = 0; m < 2; ++m)
+                tc_mma_ts_elect(tmem + g_col_d(db, m), tmem + g_col_a(ab, m) + kk * 8, bdesc, idesc,
+                                kk > 0 ? 1u : 0u);
+            }
+            tc_commit_elect(&d_full[db]);
+            if (jj == kGSlabsPerStage - 1) tc_commit_elect(&empty[st]);
+            issued = gs + 1;
+          }
+        }
+      }
+    }
+    // no MMA may run past the deallocation below (at once when all went well)
+    if (issued > 0) mbar_wait(&d_full[(issued - 1) % kGDBufs], ((issued - 1) / kGDBufs) & 1);
+  } else {
+    // ------------------------------------------------------------- workers ---
+    const int m = warp >> 2, qd = warp & 3, r = 32 * qd + lane;
+    const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
+    const uint32_t one2 = 0x3F803F80u, m128 = 0xC300C300u;  // bf16 pairs (1, 1), (-128, -128)
+    float2 acc[kGN / 2];
+
+    // wait until the MMAs of slab gp are done (its accumulator is ready and the A
+    // buffer it read is free)
+    auto wait_slab = [&](uint32_t gp) {
+      ok = __all_sync(kFull, ok && mbar_wait(&d_full[gp % kGDBufs], (gp / kGDBufs) & 1));
+    };
+    // add the product of slab gp (stage st, place jj in the stage) to acc; its
+    // MMAs are known to be done
+    auto readout = [&](uint32_t gp, int st, int jj, int ng) {
+      const uint32_t ab = gp % kGDBufs;
+      tc_fence_after();
+      const unsigned char* stg = gsm + st * kGStageBytes;
+      const float sv = bf16_bits_to_float(
+          *reinterpret_cast<const uint16_t*>(stg + kGOffS + (m * kGM + r) * 4 + jj * 2));
+      const float bv = bf16_bits_to_float(
+          *reinterpret_cast<const uint16_t*>(stg + kGOffBias + (m * kGM + r) * 4 + jj * 2));
+      const float2 s2 = make_float2(sv, sv), b2 = make_float2(bv, bv);
+      const float4* X = reinterpret_cast<const float4*>(stg + kGOffX + jj * kGN * 4);
+      const uint32_t dcol = tmem + g_col_d(ab, m) + lane_base;
+#pragma unroll
+      for (int c2 = 0; c2 < kGN / 32; ++c2) {  // 32 columns per tensor-memory wait
+        if (2 * c2 < ng) {
+          uint32_t pr[32];
+          tc_ld16(dcol + c2 * 32, pr);
+          if (2 * c2 + 1 < ng) tc_ld16(dcol + c2 * 32 + 16, pr + 16);
+          tc_wait_ld();
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int cg = 2 * c2 + h;
+            if (cg < ng) {
+              tc_regs_ready(pr + 16 * h);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float4 xv = X[cg * 4 + i];
+                const int o = cg * 8 + 2 * i;
+                const uint32_t* pp = pr + 16 * h + 4 * i;
+                acc[o] = __ffma2_rn(make_float2(__uint_as_float(pp[0]), __uint_as_float(pp[1])),
+                                    s2, acc[o]);
+                acc[o + 1] = __ffma2_rn(
+                    make_float2(__uint_as_float(pp[2]), __uint_as_float(pp[3])), s2, acc[o + 1]);
+                acc[o] = __ffma2_rn(make_float2(xv.x, xv.y), b2, acc[o]);
+                acc[o + 1] = __ffma2_rn(make_float2(xv.z, xv.w), b2, acc[o + 1]);
               }
             }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              if (c0 + j < n) a.y[(size_t)(n0 + c0 + j) * a.H + m0 + r] = d0[j];
           }
         }
       }
       tc_fence_before();
-      __syncthreads();  // accumulators read before the next chunk overwrites them
-      tc_fence_after();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&d_free[ab]);
+        if (jj == kGSlabsPerStage - 1) mbar_arrive(&empty[st]);
+      }
+    };
+
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      const int slot = tile / mtiles, m0 = (tile % mtiles) * a.mrows;
+      const int p0 = a.offsets[slot], cnt = a.offsets[slot + 1] - p0;
+      const int pp0 = a.padded[slot];
+      for (int c0 = 0; c0 < cnt && ok; c0 += kGN) {
+        const int n = min(kGN, cnt - c0), np = (n + 15) & ~15, ng = np / 16;
+#pragma unroll
+        for (int i = 0; i < kGN / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+        const uint32_t gs0 = gs, sc0 = sc;  // first slab and stage of the chunk
+        // slab g of this chunk: stage (sc0 + (g - gs0) / 2) % kGStages, place (g - gs0) & 1
+        auto read_slab = [&](uint32_t g) {
+          const uint32_t jl = g - gs0;
+          readout(g, (int)((sc0 + jl / kGSlabsPerStage) % kGStages), (int)(jl % kGSlabsPerStage), ng);
+        };
+        for (int j0 = 0; j0 < nslab && ok; j0 += kGSlabsPerStage, ++sc) {
+          const int st = sc % kGStages;
+          const uint32_t round = sc / kGStages;
+          ok = __all_sync(kFull, mbar_wait(&full[st], round & 1));
+          if (!ok) break;
+          const unsigned char* stg = gsm + st * kGStageBytes;
+          for (int jj = 0; jj < kGSlabsPerStage && ok; ++jj, ++gs) {
+            const uint32_t ab = gs % kGABufs;
+            // the MMAs of slab gs - 2 are done: its accumulator is ready below and
+            // the A buffer it read is free for this slab
+            if (gs >= 2) wait_slab(gs - 2);
+            if (!ok) break;
+            tc_fence_after();  // the A buffer's earlier reads are done before these writes
+            // this row's codes of the slab -> bf16 integers -> the A operand
+            const uint4* crow =
+                reinterpret_cast<const uint4*>(stg + (m * kGM + r) * kGCodePitch + jj * 32);
+            const uint4 w0 = crow[0], w1 = crow[1];
+            uint32_t av[32];
+            codes_to_bf16(w0.x, one2, m128, av + 0);
+            codes_to_bf16(w0.y, one2, m128, av + 4);
+            codes_to_bf16(w0.z, one2, m128, av + 8);
+            codes_to_bf16(w0.w, one2, m128, av + 12);
+            codes_to_bf16(w1.x, one2, m128, av + 16);
+            codes_to_bf16(w1.y, one2, m128, av + 20);
+            codes_to_bf16(w1.z, one2, m128, av + 24);
+            codes_to_bf16(w1.w, one2, m128, av + 28);
+            const uint32_t acol = tmem + g_col_a(ab, m) + lane_base;
+            tc_st16(acol, av);
+            tc_st16(acol + 16, av + 16);
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&a_full[ab]);
+            if (gs >= gs0 + 2) read_slab(gs - 2);
+          }
+        }
+        if (!ok) break;
+        // the chunk's last two slabs
+        for (uint32_t g = gs >= gs0 + 2 ? gs - 2 : gs0; g < gs && ok; ++g) {
+          wait_slab(g);
+          if (ok) read_slab(g);
+        }
+        if (!ok) break;
+
+        if (PHASE == 0) {
+          // ---- h = bf16(silu(bf16 g) * bf16 u); matrix 0 holds g, matrix 1 u.  The
+          // two warps of a lane quarter swap halves through tensor memory (buffer 0's
+          // accumulator columns): no MMA runs now, the next one waits for every
+          // warp's next A operand.
+          const int irow = m0 + r;  // this thread's row of h's width I
+          const int gI = irow / kGK, ci = irow % kGK;
+          const int pin = (ci & ~7) + 2 * (ci & 3) + ((ci >> 2) & 1);  // K order position
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            // 16 pairs per round: this thread finishes pairs 32m + 16hh + i
+            uint32_t ex[16];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float2 v = m == 0 ? acc[16 + 8 * hh + i] : acc[8 * hh + i];
+              ex[2 * i] = __float_as_uint(v.x);
+              ex[2 * i + 1] = __float_as_uint(v.y);
+            }
+            // each warp writes only its own matrix's columns (its partner may still be
+            // reading the other matrix's): matrix 0 gives g of pairs 32 + 16hh.. at its
+            // columns 32 + 16hh.., matrix 1 gives u of pairs 16hh.. at its columns 16hh..
+            const uint32_t give = tmem + g_col_d(0, m) + (m == 0 ? 32 : 0) + 16 * hh + lane_base;
+            const uint32_t take = tmem + g_col_d(0, 1 - m) + (m == 0 ? 0 : 32) + 16 * hh + lane_base;
+            tc_st16(give, ex);
+            tc_wait_st();
+            tc_fence_before();
+            named_barrier(1 + qd, 64);
+            tc_fence_after();
+            uint32_t ot[16];
+            tc_ld16(take, ot);
+            tc_wait_ld();
+            tc_regs_ready(ot);
+            tc_fence_before();
+            float hv[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float2 mine = m == 0 ? acc[8 * hh + i / 2] : acc[16 + 8 * hh + i / 2];
+              const float own = (i & 1) ? mine.y : mine.x;
+              const float oth = __uint_as_float(ot[i]);
+              const float g = round_to_bf16(m == 0 ? own : oth);
+              const float uu = round_to_bf16(m == 0 ? oth : own);
+              const uint16_t hb = float_to_bf16_bits(g / (1.0f + __expf(-g)) * uu);
+              hv[i] = bf16_bits_to_float(hb);
+              const int nn = 32 * m + 16 * hh + i;
+              if (nn < np) {
+                const int pos = pp0 + c0 + nn;
+                a.hp[((size_t)gI * a.pcap + pos) * kGK + (((pin >> 3) ^ (pos & 7)) << 3) +
+                     (pin & 7)] = hb;
+              }
+            }
+            // group sums of h: over this warp's 32 rows (even lanes end with one
+            // pair's sum each), then over the group's two warps
+            int vid;
+            const float part = warp_reduce_scatter<16>(hv, lane, vid);
+            if ((qd & 1) && !(lane & 1)) red[m][qd >> 1][16 * hh + vid] = part;
+            named_barrier(5 + 2 * m + (qd >> 1), 64);
+            if (!(qd & 1) && !(lane & 1)) {
+              const int nn = 32 * m + 16 * hh + vid;
+              if (nn < np)
+                a.hs[(size_t)gI * a.pcap + pp0 + c0 + nn] = part + red[m][qd >> 1][16 * hh + vid];
+            }
+            named_barrier(5 + 2 * m + (qd >> 1), 64);
+          }
+        } else {
+          // ---- y rows of the chunk's pairs (pair_list order), fp32
+          float* yo = a.y + (size_t)(p0 + c0) * a.H + m0 + a.roff[m] + r;
+#pragma unroll
+          for (int i = 0; i < kGN; ++i)
+            if (i < n) yo[(size_t)i * a.H] = (i & 1) ? acc[i / 2].y : acc[i / 2].x;
+        }
+      }
     }
   }
+  tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, kCols);
+  if (warp == kGWorkers + 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kGTmemCols);
+  }
 }
 
 // out[t][c] = bf16(sum_j w[t,j] * y[pos(t,j)][c]), j ascending, for the pairs the

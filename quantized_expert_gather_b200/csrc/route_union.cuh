@@ -7,7 +7,9 @@
 //   1. per-warp histograms hist[w][e] built with __match_any_sync;
 //   2. per expert, an exclusive prefix over the warps (the slice order keeps
 //      the sort stable) and the expert's total;
-//   3. one warp turns the totals into unique[] and offsets[] (ballot + scan);
+//   3. one warp turns the totals into unique[] and offsets[] (ballot + scan),
+//      and optionally padded[], the same prefix over counts rounded up to 16
+//      (the row offsets of the grouped kernels' packed activation layout);
 //   4. each warp re-walks its slice and places every pair at
 //      offsets[slot(e)] + (pairs of e in earlier slices) + (earlier pairs of e
 //      in this slice).
@@ -26,7 +28,7 @@ __host__ __device__ inline size_t route_union_smem_bytes(int E) {
 __global__ void __launch_bounds__(32 * kUnionWarps, 1)
     route_union_kernel(const int* __restrict__ idx, int P, int E, int* __restrict__ unique,
                        int* __restrict__ offsets, int* __restrict__ pair_list,
-                       int* __restrict__ num_unique) {
+                       int* __restrict__ num_unique, int* __restrict__ padded = nullptr) {
   extern __shared__ __align__(16) int su[];
   int* hist = su;                        // [kUnionWarps][E]
   int* total = su + kUnionWarps * E;     // [E]
@@ -68,28 +70,36 @@ __global__ void __launch_bounds__(32 * kUnionWarps, 1)
 
   // 3. unique experts and offsets
   if (warp == 0) {
-    int u = 0, off = 0;
+    int u = 0, off = 0, poff = 0;
     for (int b = 0; b < E; b += 32) {
       const int e = b + lane;
       const int c = (e < E) ? total[e] : 0;
+      const int pc = (c + 15) & ~15;  // the expert's pairs rounded up to 16
       const unsigned used = __ballot_sync(kFull, c > 0);
-      int incl = c;
+      int incl = c, pincl = pc;
 #pragma unroll
       for (int d = 1; d < 32; d <<= 1) {
         const int v = __shfl_up_sync(kFull, incl, d);
-        if (lane >= d) incl += v;
+        const int pv = __shfl_up_sync(kFull, pincl, d);
+        if (lane >= d) {
+          incl += v;
+          pincl += pv;
+        }
       }
       if (c > 0) {
         const int slot = u + __popc(used & lanemask_lt());
         unique[slot] = e;
         offsets[slot] = off + incl - c;
         base[e] = off + incl - c;
+        if (padded != nullptr) padded[slot] = poff + pincl - pc;
       }
       u += __popc(used);
       off += __shfl_sync(kFull, incl, 31);
+      poff += __shfl_sync(kFull, pincl, 31);
     }
     if (lane == 0) {
       offsets[u] = off;
+      if (padded != nullptr) padded[u] = poff;
       *num_unique = u;
       s_valid = off;
     }
