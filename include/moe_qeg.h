@@ -64,7 +64,10 @@ typedef enum {
 
 /* Supported range (checked on the host; violations return MOE_ERR_UNSUPPORTED):
  * hidden and inter multiples of 64, hidden <= 4096, inter <= 8192; E <= 1024;
- * T*k <= 65536. */
+ * T*k <= 65536.  Windows of more than 1024 pairs (or whose persistent-kernel
+ * plan does not fit) take the grouped tensor-core path, which further needs
+ * hidden a multiple of 256 and inter a multiple of 128; moe_select_path tells
+ * which path a shape takes. */
 #define MOE_MAX_EXPERTS 1024
 #define MOE_MAX_DIM 8192
 #define MOE_MAX_PAIRS 65536
@@ -180,8 +183,12 @@ moe_status moe_read_device_status(void* stream);
 
 /*
  * Which kernel path a call with this shape takes, without launching anything:
- * 1 = expert-major dequant-GEMV layer kernel (T*k <= 1024), 2 = grouped
- * tensor-core path, 0 = invalid or unsupported shape.
+ * 1 = expert-major dequant-GEMV layer kernel (T*k <= 1024 and its shared-memory
+ * plan fits), 2 = grouped tensor-core path (route-union, x packing, gate+up and
+ * down GEMMs on tcgen05, combine: five launches; hidden % 256 == 0 and
+ * inter % 128 == 0), 0 = invalid or unsupported shape.  The workspace size
+ * (moe_workspace_size) follows the path: path 2 adds the packed activations,
+ * about 2*(hidden+inter)*(T*k + 15*min(E, T*k)) bytes.
  */
 int moe_select_path(int T, int k, int E, int hidden, int inter);
 
