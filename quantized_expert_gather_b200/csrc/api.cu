@@ -22,8 +22,9 @@ struct DeviceInfo {
   bool ready = false;
   int sms = 0;
   int smem_optin = 0;
-  // dynamic shared memory limit: layer, route_union, grouped gate+up, grouped down, combine
-  int dyn_smem[5] = {0, 0, 0, 0, 0};
+  // dynamic shared memory limit: layer, route_union, grouped gate+up and down (chunks of
+  // 64 pairs), combine, grouped gate+up and down (chunks of 96 pairs)
+  int dyn_smem[7] = {0, 0, 0, 0, 0, 0, 0};
 };
 
 DeviceInfo g_dev[kMaxDevices];
@@ -49,12 +50,14 @@ moe_status device_info(DeviceInfo** out) {
       e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return cuda_fail(e);
     // dynamic + static shared memory may not exceed the opt-in limit
-    const void* kernels[5] = {reinterpret_cast<const void*>(layer_kernel),
+    const void* kernels[7] = {reinterpret_cast<const void*>(layer_kernel),
                               reinterpret_cast<const void*>(route_union_kernel),
-                              reinterpret_cast<const void*>(grouped_gemm_kernel<0>),
-                              reinterpret_cast<const void*>(grouped_gemm_kernel<1>),
-                              reinterpret_cast<const void*>(grouped_combine_kernel)};
-    for (int i = 0; i < 5; ++i) {
+                              reinterpret_cast<const void*>(grouped_gemm_kernel<0, 64>),
+                              reinterpret_cast<const void*>(grouped_gemm_kernel<1, 64>),
+                              reinterpret_cast<const void*>(grouped_combine_kernel),
+                              reinterpret_cast<const void*>(grouped_gemm_kernel<0, 96>),
+                              reinterpret_cast<const void*>(grouped_gemm_kernel<1, 96>)};
+    for (int i = 0; i < 7; ++i) {
       cudaFuncAttributes fa;
       cudaError_t e = cudaFuncGetAttributes(&fa, kernels[i]);
       if (e == cudaSuccess) {
@@ -218,8 +221,12 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   const int m = P < E ? P : E;
   const size_t usmem = route_union_smem_bytes(E);
   const size_t csmem = sizeof(int) * (size_t)P;
-  if (usmem > (size_t)d.dyn_smem[1] || kGSmem > (unsigned)d.dyn_smem[2] ||
-      kGSmem > (unsigned)d.dyn_smem[3] || csmem > (size_t)d.dyn_smem[4]) {
+  // chunks of 96 pairs when experts average more than 40 pairs (fewer weight re-reads),
+  // else 64 (a deeper copy pipeline)
+  const bool wide = P > 40 * m;
+  const unsigned gsmem = wide ? GCfg<96>::kSmem : GCfg<64>::kSmem;
+  if (usmem > (size_t)d.dyn_smem[1] || csmem > (size_t)d.dyn_smem[4] ||
+      gsmem > (unsigned)d.dyn_smem[wide ? 5 : 2] || gsmem > (unsigned)d.dyn_smem[wide ? 6 : 3]) {
     *why = MOE_ERR_UNSUPPORTED;
     return cudaSuccess;
   }
@@ -250,7 +257,10 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   g.rows = I;
   g.K = H;
   g.mrows = kGM;
-  grouped_gemm_kernel<0><<<d.sms, kGThreads, kGSmem, st>>>(g);
+  if (wide)
+    grouped_gemm_kernel<0, 96><<<d.sms, kGThreads, gsmem, st>>>(g);
+  else
+    grouped_gemm_kernel<0, 64><<<d.sms, kGThreads, gsmem, st>>>(g);
   // down: 256 rows of Wd per tile (two 128-row matrices), K = I, packed h
   g.bp = hp;
   g.bs = hs;
@@ -261,7 +271,10 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   g.rows = H;
   g.K = I;
   g.mrows = 2 * kGM;
-  grouped_gemm_kernel<1><<<d.sms, kGThreads, kGSmem, st>>>(g);
+  if (wide)
+    grouped_gemm_kernel<1, 96><<<d.sms, kGThreads, gsmem, st>>>(g);
+  else
+    grouped_gemm_kernel<1, 64><<<d.sms, kGThreads, gsmem, st>>>(g);
   grouped_combine_kernel<<<d.sms, 256, csmem, st>>>(y, w, plist, offs, nu, T, k, H, out);
   return cudaGetLastError();
 }

@@ -9,11 +9,14 @@
 //
 //   grouped_pack_x_kernel   the window's x rows, one per pair, in the order and
 //                           layout the tensor cores read (below), with group sums;
-//   grouped_gemm_kernel<0>  gate+up: per (expert, 128 rows of Wg and of Wu) tile,
+//   grouped_gemm_kernel<0, N>  gate+up: per (expert, 128 rows of Wg and of Wu) tile,
 //                           G = Wg X^T, U = Wu X^T, h = bf16(silu(bf16 G) * bf16 U),
 //                           h written packed for the next launch;
-//   grouped_gemm_kernel<1>  down: per (expert, 256 rows of Wd) tile, Y = Wd H^T,
+//   grouped_gemm_kernel<1, N>  down: per (expert, 256 rows of Wd) tile, Y = Wd H^T,
 //                           fp32 per pair;
+// (N, the pairs per MMA chunk, is 64 or 96: wider chunks stream an expert's weights
+// fewer times when it has many pairs, narrower ones leave room for a deeper copy
+// pipeline.)
 //   grouped_combine_kernel  out[t] = bf16(sum_j w[t,j] * y[t,j]), j ascending.
 //
 // The quantisation group (64 columns of K) is the MMA's K slab.  Inside a group
@@ -58,29 +61,38 @@ namespace qeg {
 constexpr int kGWorkers = 8;                         // worker warps
 constexpr int kGThreads = 32 * (kGWorkers + 2);      // + producer warp + MMA warp
 constexpr int kGM = 128;                             // weight rows per matrix (MMA M)
-constexpr int kGN = 64;                              // pairs per chunk (MMA N <= 64)
 constexpr int kGK = 64;                              // K per slab = quantisation group
 constexpr int kGSlabsPerStage = 2;
-constexpr int kGStages = 5;
 constexpr unsigned kGCodePitch = kGSlabsPerStage * 32 + 16;  // padded: no bank conflicts
 constexpr unsigned kGOffB = 2 * kGM * kGCodePitch;           // 20480, a multiple of 1024
-constexpr unsigned kGBTile = kGN * kGK * 2;                  // 8 KB per slab
-constexpr unsigned kGOffX = kGOffB + kGSlabsPerStage * kGBTile;
-constexpr unsigned kGOffS = kGOffX + kGSlabsPerStage * kGN * 4;
-constexpr unsigned kGOffBias = kGOffS + 2 * kGM * kGSlabsPerStage * 2;
-constexpr unsigned kGStageBytes = (kGOffBias + 2 * kGM * kGSlabsPerStage * 2 + 1023) & ~1023u;
-constexpr unsigned kGSmem = kGStages * kGStageBytes + 1024;  // + alignment slack
-constexpr int kGDBufs = 3;   // accumulator buffers: a slab is read back two slabs later
+constexpr int kGDBufs = 2;   // accumulator buffers
+constexpr int kGLag = 1;     // a slab's accumulator is read back after the next slab's A is stored
 constexpr int kGABufs = 2;   // A operand buffers
 constexpr uint32_t kGTmemCols = 512;
-static_assert(kGOffB % 1024 == 0 && kGBTile % 1024 == 0, "swizzled tiles need 1024-byte bases");
-static_assert(kGDBufs * 2 * kGN + kGABufs * 2 * 32 <= (int)kGTmemCols, "tensor memory map");
 
-// Tensor-memory columns: accumulator of buffer db, matrix m; A operand of buffer ab.
-__device__ __forceinline__ uint32_t g_col_d(uint32_t db, int m) { return (db * 2 + m) * kGN; }
-__device__ __forceinline__ uint32_t g_col_a(uint32_t ab, int m) {
-  return kGDBufs * 2 * kGN + (ab * 2 + m) * 32;
-}
+// Per chunk width NMAX (pairs per MMA, a multiple of 32): the shared-memory stage
+// [codes | two activation slabs | their sums | scales | biases] and the tensor
+// memory map (accumulator of buffer db, matrix m; then the A operand of buffer ab).
+template <int NMAX>
+struct GCfg {
+  static constexpr int kN = NMAX;
+  static constexpr int kStages = NMAX <= 64 ? 5 : 4;
+  static constexpr unsigned kBTile = NMAX * kGK * 2;
+  static constexpr unsigned kOffX = kGOffB + kGSlabsPerStage * kBTile;
+  static constexpr unsigned kOffS = kOffX + kGSlabsPerStage * NMAX * 4;
+  static constexpr unsigned kOffBias = kOffS + 2 * kGM * kGSlabsPerStage * 2;
+  static constexpr unsigned kStageBytes =
+      (kOffBias + 2 * kGM * kGSlabsPerStage * 2 + 1023) & ~1023u;
+  static constexpr unsigned kSmem = kStages * kStageBytes + 1024;  // + alignment slack
+  static_assert(NMAX % 32 == 0 && kBTile % 1024 == 0, "swizzled tiles need 1024-byte bases");
+  static_assert(kGDBufs * 2 * NMAX + kGABufs * 2 * 32 <= (int)kGTmemCols, "tensor memory map");
+  __device__ static __forceinline__ uint32_t col_d(uint32_t db, int m) {
+    return (db * 2 + m) * NMAX;
+  }
+  __device__ static __forceinline__ uint32_t col_a(uint32_t ab, int m) {
+    return kGDBufs * 2 * NMAX + (ab * 2 + m) * 32;
+  }
+};
 
 // ------------------------------------------------------------ tcgen05 helpers ---
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -290,20 +302,21 @@ struct GroupedArgs {
   int pcap, H;
 };
 
-template <int PHASE>
+template <int PHASE, int NMAX>
 __global__ void __launch_bounds__(kGThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ GroupedArgs a) {
+  using C = GCfg<NMAX>;
   extern __shared__ __align__(128) unsigned char gsm_raw[];
-  __shared__ __align__(8) uint64_t full[kGStages], empty[kGStages];
+  __shared__ __align__(8) uint64_t full[C::kStages], empty[C::kStages];
   __shared__ __align__(8) uint64_t a_full[kGABufs], d_full[kGDBufs], d_free[kGDBufs];
   __shared__ uint32_t tmem_base_s;
-  __shared__ float red[2][2][32];
+  __shared__ float red[2][2][C::kN / 2];
   // swizzled tiles start at 1024-byte boundaries of the shared address space
   unsigned char* gsm = gsm_raw + ((1024u - (smem_u32(gsm_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
-    for (int i = 0; i < kGStages; ++i) {
+    for (int i = 0; i < C::kStages; ++i) {
       mbar_init(&full[i], 1 + 32);          // expect_tx + one cp.async arrival per lane
       mbar_init(&empty[i], kGWorkers + 1);  // worker warps + the MMA commit
     }
@@ -338,11 +351,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
       const int e = a.unique[slot];
       const int cnt = a.offsets[slot + 1] - a.offsets[slot];
       const int pp0 = a.padded[slot];
-      for (int c0 = 0; c0 < cnt && ok; c0 += kGN) {
-        const int np = (min(kGN, cnt - c0) + 15) & ~15;
+      for (int c0 = 0; c0 < cnt && ok; c0 += C::kN) {
+        const int np = (min(C::kN, cnt - c0) + 15) & ~15;
         for (int j0 = 0; j0 < nslab && ok; j0 += kGSlabsPerStage) {
-          const int st = sc % kGStages;
-          const uint32_t round = sc / kGStages;
+          const int st = sc % C::kStages;
+          const uint32_t round = sc / C::kStages;
           if (lane == 0) {
             if (round > 0) ok = mbar_wait(&empty[st], (round - 1) & 1);
             if (ok)
@@ -350,7 +363,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
           }
           ok = __shfl_sync(kFull, ok, 0);
           if (!ok) break;
-          unsigned char* stg = gsm + st * kGStageBytes;
+          unsigned char* stg = gsm + st * C::kStageBytes;
           // codes: 16 bytes per lane, four lanes per row (64 bytes = two slabs)
 #pragma unroll 8
           for (int i = 0; i < 2 * kGM * kGSlabsPerStage * 2 / 32; ++i) {
@@ -364,15 +377,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
           for (int i = 0; i < 2 * kGM / 32; ++i) {
             const int rr = lane + 32 * i, m = rr / kGM, r = rr % kGM;
             const size_t row = (size_t)e * a.rows + m0 + a.roff[m] + r;
-            cp_async4(stg + kGOffS + rr * 4, a.s[m] + row * (a.K / kGK) + j0);
-            cp_async4(stg + kGOffBias + rr * 4, a.b[m] + row * (a.K / kGK) + j0);
+            cp_async4(stg + C::kOffS + rr * 4, a.s[m] + row * (a.K / kGK) + j0);
+            cp_async4(stg + C::kOffBias + rr * 4, a.b[m] + row * (a.K / kGK) + j0);
           }
           if (lane == 0) {
 #pragma unroll
             for (int jj = 0; jj < kGSlabsPerStage; ++jj) {
               const size_t prow = (size_t)(j0 + jj) * a.pcap + pp0 + c0;
-              bulk_g2s(stg + kGOffB + jj * kGBTile, a.bp + prow * kGK, np * kGK * 2, &full[st]);
-              bulk_g2s(stg + kGOffX + jj * kGN * 4, a.bs + prow, np * 4, &full[st]);
+              bulk_g2s(stg + kGOffB + jj * C::kBTile, a.bp + prow * kGK, np * kGK * 2, &full[st]);
+              bulk_g2s(stg + C::kOffX + jj * C::kN * 4, a.bs + prow, np * 4, &full[st]);
             }
           }
           cp_async_arrive_noinc(&full[st]);
@@ -382,8 +395,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
     }
     // leave no copy in flight: every stage issued has landed (at once when all went well)
     if (lane == 0)
-      for (uint32_t i = sc > (uint32_t)kGStages ? sc - kGStages : 0; i < sc; ++i)
-        mbar_wait(&full[i % kGStages], (i / kGStages) & 1);
+      for (uint32_t i = sc > (uint32_t)C::kStages ? sc - C::kStages : 0; i < sc; ++i)
+        mbar_wait(&full[i % C::kStages], (i / C::kStages) & 1);
   } else if (warp == kGWorkers + 1) {
     // ---------------------------------------------------------- MMA issuer ---
     // The whole warp runs this loop (operands warp-uniform); one elected lane issues.
@@ -391,14 +404,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       const int slot = tile / mtiles;
       const int cnt = a.offsets[slot + 1] - a.offsets[slot];
-      for (int c0 = 0; c0 < cnt && ok; c0 += kGN) {
-        const int np = (min(kGN, cnt - c0) + 15) & ~15;
+      for (int c0 = 0; c0 < cnt && ok; c0 += C::kN) {
+        const int np = (min(C::kN, cnt - c0) + 15) & ~15;
         const uint32_t idesc = f16_idesc(kGM, np);
         for (int j0 = 0; j0 < nslab && ok; j0 += kGSlabsPerStage, ++sc) {
-          const int st = sc % kGStages;
-          const uint32_t round = sc / kGStages;
+          const int st = sc % C::kStages;
+          const uint32_t round = sc / C::kStages;
           ok = __all_sync(kFull, mbar_wait(&full[st], round & 1));
-          const uint32_t bbase = smem_u32(gsm + st * kGStageBytes + kGOffB);
+          const uint32_t bbase = smem_u32(gsm + st * C::kStageBytes + kGOffB);
           for (int jj = 0; jj < kGSlabsPerStage && ok; ++jj, ++gs) {
             const uint32_t ab = gs % kGABufs, db = gs % kGDBufs;
             bool w = mbar_wait(&a_full[ab], (gs / kGABufs) & 1);
@@ -408,10 +421,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < kGK / 16; ++kk) {
-              const uint64_t bdesc = sw128_desc(bbase + jj * kGBTile + kk * 32);
+              const uint64_t bdesc = sw128_desc(bbase + jj * C::kBTile + kk * 32);
 #pragma unroll
               for (int m = 0; m < 2; ++m)
-                tc_mma_ts_elect(tmem + g_col_d(db, m), tmem + g_col_a(ab, m) + kk * 8, bdesc, idesc,
+                tc_mma_ts_elect(tmem + C::col_d(db, m), tmem + C::col_a(ab, m) + kk * 8, bdesc, idesc,
                                 kk > 0 ? 1u : 0u);
             }
             tc_commit_elect(&d_full[db]);
@@ -428,7 +441,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const int m = warp >> 2, qd = warp & 3, r = 32 * qd + lane;
     const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
     const uint32_t one2 = 0x3F803F80u, m128 = 0xC300C300u;  // bf16 pairs (1, 1), (-128, -128)
-    float2 acc[kGN / 2];
+    float2 acc[C::kN / 2];
 
     // wait until the MMAs of slab gp are done (its accumulator is ready and the A
     // buffer it read is free)
@@ -440,16 +453,16 @@ __global__ void __launch_bounds__(kGThreads, 1)
     auto readout = [&](uint32_t gp, int st, int jj, int ng) {
       const uint32_t ab = gp % kGDBufs;
       tc_fence_after();
-      const unsigned char* stg = gsm + st * kGStageBytes;
+      const unsigned char* stg = gsm + st * C::kStageBytes;
       const float sv = bf16_bits_to_float(
-          *reinterpret_cast<const uint16_t*>(stg + kGOffS + (m * kGM + r) * 4 + jj * 2));
+          *reinterpret_cast<const uint16_t*>(stg + C::kOffS + (m * kGM + r) * 4 + jj * 2));
       const float bv = bf16_bits_to_float(
-          *reinterpret_cast<const uint16_t*>(stg + kGOffBias + (m * kGM + r) * 4 + jj * 2));
+          *reinterpret_cast<const uint16_t*>(stg + C::kOffBias + (m * kGM + r) * 4 + jj * 2));
       const float2 s2 = make_float2(sv, sv), b2 = make_float2(bv, bv);
-      const float4* X = reinterpret_cast<const float4*>(stg + kGOffX + jj * kGN * 4);
-      const uint32_t dcol = tmem + g_col_d(ab, m) + lane_base;
+      const float4* X = reinterpret_cast<const float4*>(stg + C::kOffX + jj * C::kN * 4);
+      const uint32_t dcol = tmem + C::col_d(ab, m) + lane_base;
 #pragma unroll
-      for (int c2 = 0; c2 < kGN / 32; ++c2) {  // 32 columns per tensor-memory wait
+      for (int c2 = 0; c2 < C::kN / 32; ++c2) {  // 32 columns per tensor-memory wait
         if (2 * c2 < ng) {
           uint32_t pr[32];
           tc_ld16(dcol + c2 * 32, pr);
@@ -488,27 +501,26 @@ __global__ void __launch_bounds__(kGThreads, 1)
       const int slot = tile / mtiles, m0 = (tile % mtiles) * a.mrows;
       const int p0 = a.offsets[slot], cnt = a.offsets[slot + 1] - p0;
       const int pp0 = a.padded[slot];
-      for (int c0 = 0; c0 < cnt && ok; c0 += kGN) {
-        const int n = min(kGN, cnt - c0), np = (n + 15) & ~15, ng = np / 16;
+      for (int c0 = 0; c0 < cnt && ok; c0 += C::kN) {
+        const int n = min(C::kN, cnt - c0), np = (n + 15) & ~15, ng = np / 16;
 #pragma unroll
-        for (int i = 0; i < kGN / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+        for (int i = 0; i < C::kN / 2; ++i) acc[i] = make_float2(0.f, 0.f);
         const uint32_t gs0 = gs, sc0 = sc;  // first slab and stage of the chunk
-        // slab g of this chunk: stage (sc0 + (g - gs0) / 2) % kGStages, place (g - gs0) & 1
+        // slab g of this chunk: stage (sc0 + (g - gs0) / 2) % C::kStages, place (g - gs0) & 1
         auto read_slab = [&](uint32_t g) {
           const uint32_t jl = g - gs0;
-          readout(g, (int)((sc0 + jl / kGSlabsPerStage) % kGStages), (int)(jl % kGSlabsPerStage), ng);
+          readout(g, (int)((sc0 + jl / kGSlabsPerStage) % C::kStages), (int)(jl % kGSlabsPerStage), ng);
         };
         for (int j0 = 0; j0 < nslab && ok; j0 += kGSlabsPerStage, ++sc) {
-          const int st = sc % kGStages;
-          const uint32_t round = sc / kGStages;
+          const int st = sc % C::kStages;
+          const uint32_t round = sc / C::kStages;
           ok = __all_sync(kFull, mbar_wait(&full[st], round & 1));
           if (!ok) break;
-          const unsigned char* stg = gsm + st * kGStageBytes;
+          const unsigned char* stg = gsm + st * C::kStageBytes;
           for (int jj = 0; jj < kGSlabsPerStage && ok; ++jj, ++gs) {
             const uint32_t ab = gs % kGABufs;
-            // the MMAs of slab gs - 2 are done: its accumulator is ready below and
-            // the A buffer it read is free for this slab
-            if (gs >= 2) wait_slab(gs - 2);
+            // the MMAs that read this A buffer (slab gs - 2) are done
+            if (gs >= (uint32_t)kGABufs) wait_slab(gs - kGABufs);
             if (!ok) break;
             tc_fence_after();  // the A buffer's earlier reads are done before these writes
             // this row's codes of the slab -> bf16 integers -> the A operand
@@ -524,19 +536,22 @@ __global__ void __launch_bounds__(kGThreads, 1)
             codes_to_bf16(w1.y, one2, m128, av + 20);
             codes_to_bf16(w1.z, one2, m128, av + 24);
             codes_to_bf16(w1.w, one2, m128, av + 28);
-            const uint32_t acol = tmem + g_col_a(ab, m) + lane_base;
+            const uint32_t acol = tmem + C::col_a(ab, m) + lane_base;
             tc_st16(acol, av);
             tc_st16(acol + 16, av + 16);
             tc_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&a_full[ab]);
-            if (gs >= gs0 + 2) read_slab(gs - 2);
+            if (gs >= gs0 + kGLag) {
+              wait_slab(gs - kGLag);
+              if (ok) read_slab(gs - kGLag);
+            }
           }
         }
         if (!ok) break;
-        // the chunk's last two slabs
-        for (uint32_t g = gs >= gs0 + 2 ? gs - 2 : gs0; g < gs && ok; ++g) {
+        // the chunk's last kGLag slabs
+        for (uint32_t g = gs >= gs0 + kGLag ? gs - kGLag : gs0; g < gs && ok; ++g) {
           wait_slab(g);
           if (ok) read_slab(g);
         }
@@ -550,21 +565,25 @@ __global__ void __launch_bounds__(kGThreads, 1)
           const int irow = m0 + r;  // this thread's row of h's width I
           const int gI = irow / kGK, ci = irow % kGK;
           const int pin = (ci & ~7) + 2 * (ci & 3) + ((ci >> 2) & 1);  // K order position
+          constexpr int kHalf = C::kN / 2;  // pairs finished by each matrix's warps
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            // 16 pairs per round: this thread finishes pairs 32m + 16hh + i
+          for (int hh = 0; hh < kHalf / 16; ++hh) {
+            // 16 pairs per round: this thread finishes pairs kHalf m + 16hh + i
             uint32_t ex[16];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              const float2 v = m == 0 ? acc[16 + 8 * hh + i] : acc[8 * hh + i];
+              const float2 v = m == 0 ? acc[kHalf / 2 + 8 * hh + i] : acc[8 * hh + i];
               ex[2 * i] = __float_as_uint(v.x);
               ex[2 * i + 1] = __float_as_uint(v.y);
             }
             // each warp writes only its own matrix's columns (its partner may still be
-            // reading the other matrix's): matrix 0 gives g of pairs 32 + 16hh.. at its
-            // columns 32 + 16hh.., matrix 1 gives u of pairs 16hh.. at its columns 16hh..
-            const uint32_t give = tmem + g_col_d(0, m) + (m == 0 ? 32 : 0) + 16 * hh + lane_base;
-            const uint32_t take = tmem + g_col_d(0, 1 - m) + (m == 0 ? 0 : 32) + 16 * hh + lane_base;
+            // reading the other matrix's): matrix 0 gives g of pairs kHalf + 16hh.. at
+            // its columns kHalf + 16hh.., matrix 1 gives u of pairs 16hh.. at its
+            // columns 16hh..
+            const uint32_t give =
+                tmem + C::col_d(0, m) + (m == 0 ? kHalf : 0) + 16 * hh + lane_base;
+            const uint32_t take =
+                tmem + C::col_d(0, 1 - m) + (m == 0 ? 0 : kHalf) + 16 * hh + lane_base;
             tc_st16(give, ex);
             tc_wait_st();
             tc_fence_before();
@@ -578,14 +597,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
             float hv[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float2 mine = m == 0 ? acc[8 * hh + i / 2] : acc[16 + 8 * hh + i / 2];
+              const float2 mine = m == 0 ? acc[8 * hh + i / 2] : acc[kHalf / 2 + 8 * hh + i / 2];
               const float own = (i & 1) ? mine.y : mine.x;
               const float oth = __uint_as_float(ot[i]);
               const float g = round_to_bf16(m == 0 ? own : oth);
               const float uu = round_to_bf16(m == 0 ? oth : own);
               const uint16_t hb = float_to_bf16_bits(g / (1.0f + __expf(-g)) * uu);
               hv[i] = bf16_bits_to_float(hb);
-              const int nn = 32 * m + 16 * hh + i;
+              const int nn = kHalf * m + 16 * hh + i;
               if (nn < np) {
                 const int pos = pp0 + c0 + nn;
                 a.hp[((size_t)gI * a.pcap + pos) * kGK + (((pin >> 3) ^ (pos & 7)) << 3) +
@@ -599,7 +618,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             if ((qd & 1) && !(lane & 1)) red[m][qd >> 1][16 * hh + vid] = part;
             named_barrier(5 + 2 * m + (qd >> 1), 64);
             if (!(qd & 1) && !(lane & 1)) {
-              const int nn = 32 * m + 16 * hh + vid;
+              const int nn = kHalf * m + 16 * hh + vid;
               if (nn < np)
                 a.hs[(size_t)gI * a.pcap + pp0 + c0 + nn] = part + red[m][qd >> 1][16 * hh + vid];
             }
@@ -609,7 +628,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
           // ---- y rows of the chunk's pairs (pair_list order), fp32
           float* yo = a.y + (size_t)(p0 + c0) * a.H + m0 + a.roff[m] + r;
 #pragma unroll
-          for (int i = 0; i < kGN; ++i)
+          for (int i = 0; i < C::kN; ++i)
             if (i < n) yo[(size_t)i * a.H] = (i & 1) ? acc[i / 2].y : acc[i / 2].x;
         }
       }
