@@ -23,8 +23,8 @@ struct DeviceInfo {
   int sms = 0;
   int smem_optin = 0;
   // dynamic shared memory limit: layer, route_union, grouped gate+up and down (chunks of
-  // 64 pairs), combine, grouped gate+up and down (chunks of 96 pairs)
-  int dyn_smem[7] = {0, 0, 0, 0, 0, 0, 0};
+  // 64 pairs), combine, grouped gate+up and down (chunks of 96, then of 32 pairs)
+  int dyn_smem[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
 };
 
 DeviceInfo g_dev[kMaxDevices];
@@ -50,14 +50,16 @@ moe_status device_info(DeviceInfo** out) {
       e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return cuda_fail(e);
     // dynamic + static shared memory may not exceed the opt-in limit
-    const void* kernels[7] = {reinterpret_cast<const void*>(layer_kernel),
+    const void* kernels[9] = {reinterpret_cast<const void*>(layer_kernel),
                               reinterpret_cast<const void*>(route_union_kernel),
                               reinterpret_cast<const void*>(grouped_gemm_kernel<0, 64>),
                               reinterpret_cast<const void*>(grouped_gemm_kernel<1, 64>),
                               reinterpret_cast<const void*>(grouped_combine_kernel),
                               reinterpret_cast<const void*>(grouped_gemm_kernel<0, 96>),
-                              reinterpret_cast<const void*>(grouped_gemm_kernel<1, 96>)};
-    for (int i = 0; i < 7; ++i) {
+                              reinterpret_cast<const void*>(grouped_gemm_kernel<1, 96>),
+                              reinterpret_cast<const void*>(grouped_gemm_kernel<0, 32>),
+                              reinterpret_cast<const void*>(grouped_gemm_kernel<1, 32>)};
+    for (int i = 0; i < 9; ++i) {
       cudaFuncAttributes fa;
       cudaError_t e = cudaFuncGetAttributes(&fa, kernels[i]);
       if (e == cudaSuccess) {
@@ -221,12 +223,14 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   const int m = P < E ? P : E;
   const size_t usmem = route_union_smem_bytes(E);
   const size_t csmem = sizeof(int) * (size_t)P;
-  // chunks of 96 pairs when experts average more than 40 pairs (fewer weight re-reads),
-  // else 64 (a deeper copy pipeline)
-  const bool wide = P > 40 * m;
-  const unsigned gsmem = wide ? GCfg<96>::kSmem : GCfg<64>::kSmem;
+  // pairs per MMA chunk: 96 when experts average more than 40 pairs (fewer weight
+  // re-reads), 32 when they average at most 20 (two CTAs per SM), else 64
+  const int width = P > 40 * m ? 96 : (P <= 20 * m ? 32 : 64);
+  const unsigned gsmem = width == 96 ? GCfg<96>::kSmem : width == 32 ? GCfg<32>::kSmem : GCfg<64>::kSmem;
+  const int ki = width == 96 ? 5 : width == 32 ? 7 : 2;  // dyn_smem index of gate+up
+  const int grid = width == 32 ? 2 * d.sms : d.sms;
   if (usmem > (size_t)d.dyn_smem[1] || csmem > (size_t)d.dyn_smem[4] ||
-      gsmem > (unsigned)d.dyn_smem[wide ? 5 : 2] || gsmem > (unsigned)d.dyn_smem[wide ? 6 : 3]) {
+      gsmem > (unsigned)d.dyn_smem[ki] || gsmem > (unsigned)d.dyn_smem[ki + 1]) {
     *why = MOE_ERR_UNSUPPORTED;
     return cudaSuccess;
   }
@@ -257,10 +261,12 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   g.rows = I;
   g.K = H;
   g.mrows = kGM;
-  if (wide)
-    grouped_gemm_kernel<0, 96><<<d.sms, kGThreads, gsmem, st>>>(g);
+  if (width == 96)
+    grouped_gemm_kernel<0, 96><<<grid, kGThreads, gsmem, st>>>(g);
+  else if (width == 32)
+    grouped_gemm_kernel<0, 32><<<grid, kGThreads, gsmem, st>>>(g);
   else
-    grouped_gemm_kernel<0, 64><<<d.sms, kGThreads, gsmem, st>>>(g);
+    grouped_gemm_kernel<0, 64><<<grid, kGThreads, gsmem, st>>>(g);
   // down: 256 rows of Wd per tile (two 128-row matrices), K = I, packed h
   g.bp = hp;
   g.bs = hs;
@@ -271,10 +277,12 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   g.rows = H;
   g.K = I;
   g.mrows = 2 * kGM;
-  if (wide)
-    grouped_gemm_kernel<1, 96><<<d.sms, kGThreads, gsmem, st>>>(g);
+  if (width == 96)
+    grouped_gemm_kernel<1, 96><<<grid, kGThreads, gsmem, st>>>(g);
+  else if (width == 32)
+    grouped_gemm_kernel<1, 32><<<grid, kGThreads, gsmem, st>>>(g);
   else
-    grouped_gemm_kernel<1, 64><<<d.sms, kGThreads, gsmem, st>>>(g);
+    grouped_gemm_kernel<1, 64><<<grid, kGThreads, gsmem, st>>>(g);
   grouped_combine_kernel<<<d.sms, 256, csmem, st>>>(y, w, plist, offs, nu, T, k, H, out);
   return cudaGetLastError();
 }

@@ -14,9 +14,9 @@
 //                           h written packed for the next launch;
 //   grouped_gemm_kernel<1, N>  down: per (expert, 256 rows of Wd) tile, Y = Wd H^T,
 //                           fp32 per pair;
-// (N, the pairs per MMA chunk, is 64 or 96: wider chunks stream an expert's weights
-// fewer times when it has many pairs, narrower ones leave room for a deeper copy
-// pipeline.)
+// (N, the pairs per MMA chunk, is 32, 64 or 96: wider chunks stream an expert's
+// weights fewer times when it has many pairs; with 32 two CTAs fit on an SM, which
+// doubles the warps that hide the per-slab latency.)
 //   grouped_combine_kernel  out[t] = bf16(sum_j w[t,j] * y[t,j]), j ascending.
 //
 // The quantisation group (64 columns of K) is the MMA's K slab.  Inside a group
@@ -28,7 +28,7 @@
 // the activation row's group sum) is added to fp32 registers.  No weight is ever
 // rounded; the only per-weight work is turning 4-bit codes into bf16 integers.
 //
-// Roles in a CTA (one CTA per SM, looping over tiles):
+// Roles in a CTA (one or two CTAs per SM, looping over tiles):
 //   warp 8      producer: per stage of two slabs, 16-byte async copies of each
 //               weight row's codes (64 bytes) and 4-byte ones of its scales and
 //               biases, and 1-D bulk copies of the two packed activation slabs and
@@ -68,7 +68,6 @@ constexpr unsigned kGOffB = 2 * kGM * kGCodePitch;           // 20480, a multipl
 constexpr int kGDBufs = 2;   // accumulator buffers
 constexpr int kGLag = 1;     // a slab's accumulator is read back after the next slab's A is stored
 constexpr int kGABufs = 2;   // A operand buffers
-constexpr uint32_t kGTmemCols = 512;
 
 // Per chunk width NMAX (pairs per MMA, a multiple of 32): the shared-memory stage
 // [codes | two activation slabs | their sums | scales | biases] and the tensor
@@ -76,7 +75,9 @@ constexpr uint32_t kGTmemCols = 512;
 template <int NMAX>
 struct GCfg {
   static constexpr int kN = NMAX;
-  static constexpr int kStages = NMAX <= 64 ? 5 : 4;
+  static constexpr int kStages = NMAX <= 32 ? 3 : (NMAX <= 64 ? 5 : 4);
+  static constexpr int kCtasPerSm = NMAX <= 32 ? 2 : 1;  // two CTAs share an SM's tensor memory
+  static constexpr uint32_t kTmemCols = NMAX <= 32 ? 256 : 512;
   static constexpr unsigned kBTile = NMAX * kGK * 2;
   static constexpr unsigned kOffX = kGOffB + kGSlabsPerStage * kBTile;
   static constexpr unsigned kOffS = kOffX + kGSlabsPerStage * NMAX * 4;
@@ -85,7 +86,7 @@ struct GCfg {
       (kOffBias + 2 * kGM * kGSlabsPerStage * 2 + 1023) & ~1023u;
   static constexpr unsigned kSmem = kStages * kStageBytes + 1024;  // + alignment slack
   static_assert(NMAX % 32 == 0 && kBTile % 1024 == 0, "swizzled tiles need 1024-byte bases");
-  static_assert(kGDBufs * 2 * NMAX + kGABufs * 2 * 32 <= (int)kGTmemCols, "tensor memory map");
+  static_assert(kGDBufs * 2 * NMAX + kGABufs * 2 * 32 <= (int)kTmemCols, "tensor memory map");
   __device__ static __forceinline__ uint32_t col_d(uint32_t db, int m) {
     return (db * 2 + m) * NMAX;
   }
@@ -303,7 +304,7 @@ struct GroupedArgs {
 };
 
 template <int PHASE, int NMAX>
-__global__ void __launch_bounds__(kGThreads, 1)
+__global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
     grouped_gemm_kernel(const __grid_constant__ GroupedArgs a) {
   using C = GCfg<NMAX>;
   extern __shared__ __align__(128) unsigned char gsm_raw[];
@@ -328,7 +329,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     fence_barrier_init();
   }
   if (warp == kGWorkers + 1) {
-    tmem_alloc(&tmem_base_s, kGTmemCols);
+    tmem_alloc(&tmem_base_s, C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -638,7 +639,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
   __syncthreads();
   if (warp == kGWorkers + 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kGTmemCols);
+    tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
