@@ -463,15 +463,20 @@ __global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
       const float4* X = reinterpret_cast<const float4*>(stg + C::kOffX + jj * C::kN * 4);
       const uint32_t dcol = tmem + C::col_d(ab, m) + lane_base;
 #pragma unroll
-      for (int c2 = 0; c2 < C::kN / 32; ++c2) {  // 32 columns per tensor-memory wait
-        if (2 * c2 < ng) {
-          uint32_t pr[32];
-          tc_ld16(dcol + c2 * 32, pr);
-          if (2 * c2 + 1 < ng) tc_ld16(dcol + c2 * 32 + 16, pr + 16);
+      // kRd columns per tensor-memory wait (16 where registers are scarce)
+      constexpr int kRd = C::kN <= 32 ? 16 : 32, kRg = kRd / 16;
+#pragma unroll
+      for (int c2 = 0; c2 < C::kN / kRd; ++c2) {
+        if (kRg * c2 < ng) {
+          uint32_t pr[kRd];
+          tc_ld16(dcol + c2 * kRd, pr);
+          if constexpr (kRg == 2) {
+            if (2 * c2 + 1 < ng) tc_ld16(dcol + c2 * kRd + 16, pr + 16);
+          }
           tc_wait_ld();
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int cg = 2 * c2 + h;
+          for (int h = 0; h < kRg; ++h) {
+            const int cg = kRg * c2 + h;
             if (cg < ng) {
               tc_regs_ready(pr + 16 * h);
 #pragma unroll
@@ -527,19 +532,17 @@ __global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
             // this row's codes of the slab -> bf16 integers -> the A operand
             const uint4* crow =
                 reinterpret_cast<const uint4*>(stg + (m * kGM + r) * kGCodePitch + jj * 32);
-            const uint4 w0 = crow[0], w1 = crow[1];
-            uint32_t av[32];
-            codes_to_bf16(w0.x, one2, m128, av + 0);
-            codes_to_bf16(w0.y, one2, m128, av + 4);
-            codes_to_bf16(w0.z, one2, m128, av + 8);
-            codes_to_bf16(w0.w, one2, m128, av + 12);
-            codes_to_bf16(w1.x, one2, m128, av + 16);
-            codes_to_bf16(w1.y, one2, m128, av + 20);
-            codes_to_bf16(w1.z, one2, m128, av + 24);
-            codes_to_bf16(w1.w, one2, m128, av + 28);
             const uint32_t acol = tmem + C::col_a(ab, m) + lane_base;
-            tc_st16(acol, av);
-            tc_st16(acol + 16, av + 16);
+#pragma unroll
+            for (int hw = 0; hw < 2; ++hw) {  // 32 codes (16 columns) at a time
+              const uint4 wv = crow[hw];
+              uint32_t av[16];
+              codes_to_bf16(wv.x, one2, m128, av + 0);
+              codes_to_bf16(wv.y, one2, m128, av + 4);
+              codes_to_bf16(wv.z, one2, m128, av + 8);
+              codes_to_bf16(wv.w, one2, m128, av + 12);
+              tc_st16(acol + 16 * hw, av);
+            }
             tc_wait_st();
             tc_fence_before();
             __syncwarp();
