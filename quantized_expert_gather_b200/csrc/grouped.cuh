@@ -464,7 +464,7 @@ __global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
       const uint32_t dcol = tmem + C::col_d(ab, m) + lane_base;
 #pragma unroll
       // kRd columns per tensor-memory wait (16 where registers are scarce)
-      constexpr int kRd = C::kN <= 32 ? 16 : 32, kRg = kRd / 16;
+      constexpr int kRd = C::kN == 64 ? 32 : 16, kRg = kRd / 16;
 #pragma unroll
       for (int c2 = 0; c2 < C::kN / kRd; ++c2) {
         if (kRg * c2 < ng) {
