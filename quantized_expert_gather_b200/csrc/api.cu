@@ -283,7 +283,8 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
     grouped_gemm_kernel<1, 32><<<grid, kGThreads, gsmem, st>>>(g);
   else
     grouped_gemm_kernel<1, 64><<<grid, kGThreads, gsmem, st>>>(g);
-  grouped_combine_kernel<<<d.sms, 256, csmem, st>>>(y, w, plist, offs, nu, T, k, H, out);
+  grouped_combine_kernel<<<2 * d.sms, kGCombineThreads, csmem, st>>>(y, w, plist, offs, nu, T, k,
+                                                                      H, out);
   return cudaGetLastError();
 }
 

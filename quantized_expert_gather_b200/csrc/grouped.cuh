@@ -648,8 +648,10 @@ __global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
 
 // out[t][c] = bf16(sum_j w[t,j] * y[pos(t,j)][c]), j ascending, for the pairs the
 // route-union kept (pos from pair_list); rows of tokens whose pairs were all left
-// out are zero.
-__global__ void __launch_bounds__(256) grouped_combine_kernel(
+// out are zero.  Bound by reading y: launched with two 512-thread CTAs per SM so
+// that enough loads are in flight.
+constexpr int kGCombineThreads = 512;
+__global__ void __launch_bounds__(kGCombineThreads) grouped_combine_kernel(
     const float* __restrict__ y, const float* __restrict__ w, const int* __restrict__ pair_list,
     const int* __restrict__ offsets, const int* __restrict__ num_unique, int T, int k, int H,
     uint16_t* __restrict__ out) {
