@@ -503,9 +503,11 @@ def our_arm(args, world, rank, local):
             us = a4.elapsed_time(b4) * 1e3 / nl
             ul = float(np.mean([np.unique(r[0]).size for r in rl]))
             fl = 6.0 * TL * K_TOP * HIDDEN * INTER
-            large[str(TL)] = {"us_per_layer": us, "mean_unique": ul,
-                              "unique_gbs": ul * BYTES_PER_EXPERT / (us * 1e-6) / 1e9,
-                              "tflops": fl / (us * 1e-6) / 1e12}
+            gbl = ul * BYTES_PER_EXPERT / (us * 1e-6) / 1e9
+            large[str(TL)] = {"us_per_layer": us, "mean_unique": ul, "unique_gbs": gbl,
+                              "frac_of_hbm_peak": gbl / measured_peaks()[0],
+                              "tflops": fl / (us * 1e-6) / 1e12,
+                              "path": "grouped tcgen05 kernels (5 launches per layer)"}
             del wsl
     if verify is not None:
         del bank2
