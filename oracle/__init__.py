@@ -52,6 +52,8 @@ def load(so: Optional[str] = None):
     lib.oracle_switchglu_union.argtypes = [vp] * 12 + [ci] * 5 + [vp, vp]
     lib.oracle_round_bf16.restype = ctypes.c_double
     lib.oracle_round_bf16.argtypes = [ctypes.c_double]
+    lib.oracle_router_topk.restype = None
+    lib.oracle_router_topk.argtypes = [vp, ci, ci, ci, ci, vp, vp]
     if so is None:
         _lib = lib
     return lib
@@ -137,3 +139,16 @@ def switchglu_union(x, idx, w, bank, E, want_h=False, lib=None):
 
 def round_bf16(v: float, lib=None) -> float:
     return (lib or load()).oracle_round_bf16(float(v))
+
+
+def router_topk(logits: np.ndarray, k: int, renormalize: bool = True, lib=None):
+    """(idx [T, k] int32, w [T, k] fp64): top-k of softmax over each row of the fp32
+    logits [T, E], descending, lower expert id first among equal logits; weights
+    renormalised over the k unless renormalize is False."""
+    lib = lib or load()
+    logits, pl = _c(logits, np.float32)
+    T, E = logits.shape
+    idx = np.zeros((T, k), np.int32)
+    w = np.zeros((T, k), np.float64)
+    lib.oracle_router_topk(pl, T, E, k, 1 if renormalize else 0, idx.ctypes.data, w.ctypes.data)
+    return idx, w

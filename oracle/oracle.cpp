@@ -29,6 +29,9 @@
 //   4*(c%8) .. 4*(c%8)+3, least significant first) of 32-bit word c / 8.
 // * Expert ids outside [0, E) name no expert: such a pair is left out of the
 //   union and contributes nothing.
+// * The router step before the layer (oracle_router_topk): top-k of softmax over
+//   the experts, renormalised over the k, as the tiny parity configuration routes
+//   its tokens; equal logits go to the lower expert id.
 //
 // Every sum is in fp64 in ascending index order; dequantised weights are exact
 // in fp64.  Rounding to bf16 is done directly from fp64 (one rounding).
@@ -316,5 +319,35 @@ void oracle_switchglu_union(const uint16_t* x, const int32_t* idx, const float* 
 
 // The oracle's bf16 rounding, exported so its pins can test it directly.
 double oracle_round_bf16(double v) { return round_bf16(v); }
+
+// Router step ahead of the layer, by its plain definition (the routing of the
+// tiny parity configuration: top-k of softmax over the E experts, weights
+// renormalised over the k).  For each token t: the k experts with the largest
+// logits, in descending logit order with the lower expert id first among equal
+// logits; w_j = exp(l_j - m) / D with m the row's largest logit and D the sum of
+// exp(l - m) over the k chosen experts (renormalize != 0) or over all E.
+// Logits are finite; sums in fp64, ascending order.
+void oracle_router_topk(const float* logits, int T, int E, int k, int renormalize,
+                        int32_t* idx, double* w) {
+  std::vector<int> order(E);
+  for (int t = 0; t < T; ++t) {
+    const float* row = logits + static_cast<size_t>(t) * E;
+    for (int e = 0; e < E; ++e) order[e] = e;
+    std::stable_sort(order.begin(), order.end(),
+                     [row](int a, int b) { return row[a] > row[b]; });
+    const double m = row[order[0]];
+    double denom = 0.0;
+    if (renormalize) {
+      for (int j = 0; j < k; ++j) denom += std::exp(static_cast<double>(row[order[j]]) - m);
+    } else {
+      for (int e = 0; e < E; ++e) denom += std::exp(static_cast<double>(row[e]) - m);
+    }
+    for (int j = 0; j < k; ++j) {
+      idx[static_cast<size_t>(t) * k + j] = order[j];
+      w[static_cast<size_t>(t) * k + j] =
+          std::exp(static_cast<double>(row[order[j]]) - m) / denom;
+    }
+  }
+}
 
 }  // extern "C"

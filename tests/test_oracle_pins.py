@@ -9,6 +9,9 @@ the oracle itself.
   independence;
 * E=1, k=1 reduces to a dense dequantised GEMV -> SwiGLU -> GEMV done with numpy
   matmul (library routine);
+* the router step: equal logits (ties to the lower id, weights 1/k or 1/E), a
+  logarithmic ramp (weights proportional to i + 1, a closed form), k = E against
+  scipy's softmax, torch.topk's selection, shift invariance;
 * a set of planted mistakes (in copies of the oracle source) each fail a pin.
 """
 import math
@@ -283,6 +286,12 @@ MUTANTS = {
                               "acc += Y["),
     "down_transposed": ("Y += L.down.at(e, c, r) * h[r];", "Y += L.down.at(e, r, c) * h[r];"),
     "h_product_unrounded": ("h[r] = round_bf16(g * sigmoid(g) * v);", "h[r] = g * sigmoid(g) * v;"),
+    "router_ascending": ("[row](int a, int b) { return row[a] > row[b]; }",
+                         "[row](int a, int b) { return row[a] < row[b]; }"),
+    "router_ties_to_higher_id": ("[row](int a, int b) { return row[a] > row[b]; }",
+                                 "[row](int a, int b) { return row[a] > row[b] || (row[a] == row[b] && a > b); }"),
+    "router_not_renormalised": ("    if (renormalize) {\n      for (int j = 0; j < k; ++j)",
+                                "    if (false) {\n      for (int j = 0; j < k; ++j)"),
 }
 
 _MUTANT_CHECK = r"""
@@ -300,6 +309,7 @@ def run(f):
         fails += 1
 run(P._pin_closed_forms)
 run(P._pin_textbook)
+run(P._pin_router)
 print("FAILS", fails)
 """
 
@@ -342,6 +352,52 @@ def _pin_textbook(lib):
     assert np.allclose(out[0], yref, rtol=0, atol=1e-3 * np.abs(yref).max())
 
 
+def _pin_router(lib):
+    # equal logits: the k lowest ids, weights 1/k renormalised, 1/E otherwise
+    E, k = 12, 5
+    idx, w = oracle.router_topk(np.full((2, E), 0.75, np.float32), k, True, lib=lib)
+    assert np.array_equal(idx, np.tile(np.arange(k), (2, 1)))
+    assert np.allclose(w, 1.0 / k, rtol=1e-15, atol=0)
+    _, w = oracle.router_topk(np.full((1, E), -2.5, np.float32), k, False, lib=lib)
+    assert np.allclose(w, 1.0 / E, rtol=1e-15, atol=0)
+    # logits ln(i + 1): softmax_i = (i + 1) / sum; the top k are the last k ids
+    E, k = 40, 6
+    lg = np.log(np.arange(1, E + 1, dtype=np.float64)).astype(np.float32)[None]
+    idx, w = oracle.router_topk(lg, k, True, lib=lib)
+    top = np.arange(E - 1, E - 1 - k, -1)
+    assert np.array_equal(idx[0], top)
+    assert np.allclose(w[0], (top + 1) / np.sum(top + 1), rtol=1e-6, atol=0)
+    _, w = oracle.router_topk(lg, k, False, lib=lib)
+    assert np.allclose(w[0], (top + 1) / (E * (E + 1) / 2), rtol=1e-6, atol=0)
+    # one id ahead of an equal one: a tie resolves to the lower id
+    lg = np.zeros((1, 8), np.float32)
+    lg[0, [2, 6]] = 1.0
+    idx, _ = oracle.router_topk(lg, 3, True, lib=lib)
+    assert list(idx[0]) == [2, 6, 0]
+
+
+def test_router_pins():
+    _pin_router(oracle.load())
+
+
+def test_router_against_library_routines():
+    """k = E gives the full softmax (scipy), sorted descending; the selection of
+    distinct logits equals torch.topk's; adding an exactly representable constant
+    changes nothing."""
+    from scipy.special import softmax
+    rng = np.random.default_rng(41)
+    for T, E, k in [(3, 16, 16), (5, 288, 8), (2, 1024, 32), (4, 7, 3)]:
+        lg = (rng.permutation(E * T).reshape(T, E) / 64.0 - 4.0).astype(np.float32)  # distinct
+        idx, w = oracle.router_topk(lg, k, renormalize=(k != E))
+        ti = torch.topk(torch.from_numpy(lg).double(), k, dim=1, sorted=True).indices.numpy()
+        assert np.array_equal(idx, ti)
+        if k == E:
+            ref = softmax(lg.astype(np.float64), axis=1)
+            assert np.allclose(w, np.take_along_axis(ref, idx, axis=1), rtol=1e-12, atol=0)
+        idx2, w2 = oracle.router_topk(lg + np.float32(2.0), k, renormalize=(k != E))
+        assert np.array_equal(idx, idx2) and np.allclose(w, w2, rtol=1e-12, atol=0)
+
+
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_planted_mistake_fails_a_pin(name, tmp_path):
     old, new = MUTANTS[name]
@@ -362,3 +418,4 @@ def test_unmutated_oracle_passes_mutant_pins():
     lib = oracle.load()
     _pin_closed_forms(lib)
     _pin_textbook(lib)
+    _pin_router(lib)
