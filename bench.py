@@ -512,6 +512,28 @@ def our_arm(args, world, rank, local):
     if verify is not None:
         del bank2
 
+    # the router step ahead of the layer (top-k of softmax, renormalised): a few
+    # microseconds of launch latency per call; CUDA events over 200 calls
+    router = None
+    try:
+        rt = {}
+        for TR in (1, 4, 16):
+            lg = torch.from_numpy(np.random.default_rng(SEED + 70 + TR).standard_normal(
+                (TR, E)).astype(np.float32)).to(dev)
+            for _ in range(10):
+                qeg.moe_router_topk(lg, K_TOP)
+            torch.cuda.synchronize()
+            a5, b5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a5.record()
+            for _ in range(200):
+                qeg.moe_router_topk(lg, K_TOP)
+            b5.record()
+            torch.cuda.synchronize()
+            rt[str(TR)] = a5.elapsed_time(b5) * 1e3 / 200
+        router = {"E": E, "k": K_TOP, "renormalize": True, "us_per_call": rt}
+    except Exception as ex:  # report, never lose the headline line
+        router = {"error": repr(ex)}
+
     # end to end through the public call: pinned host inputs in, outputs back, each step
     pin_x = {T: torch.from_numpy(synth.x_bf16(T, HIDDEN, SEED + T).view(np.int16)).pin_memory()
              for T in TS}
@@ -601,6 +623,7 @@ def our_arm(args, world, rank, local):
                            "all layer outputs copied back every step"},
             "verify_pair": verify,
             "large_window": large,
+            "router": router,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
         }

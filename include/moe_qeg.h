@@ -182,6 +182,25 @@ moe_status moe_switchglu_forward_static(const uint16_t* x, const int32_t* topk_i
 moe_status moe_read_device_status(void* stream);
 
 /*
+ * Router step ahead of the layer (the routing of the tiny parity configuration:
+ * top-k of softmax over the experts, renormalised over the k).  For each token t
+ * of logits [T, E] (fp32, row-major, finite values): topk_idx[t, 0..k) = the k
+ * experts with the largest logits, in descending logit order, the lower expert
+ * id first among equal logits; topk_w[t, j] = exp(l_j - m) / D, m = the row's
+ * largest logit, D = the sum of exp(l - m) over the k picks (renormalize != 0)
+ * or over all E (renormalize == 0).  The outputs are the topk_idx / topk_w
+ * arguments of moe_switchglu_forward.
+ *   logits [T*E] fp32, topk_idx [T*k] int32, topk_w [T*k] fp32: device memory
+ *   owned by the caller, 4-byte aligned.  One launch on `stream`, no host sync,
+ *   capturable.
+ * Errors: MOE_ERR_INVALID_ARG for null pointers, T, E or k <= 0, or k > E;
+ * MOE_ERR_UNSUPPORTED for E > 1024, k > 32, T*k > MOE_MAX_PAIRS or a misaligned
+ * pointer (nothing is launched); MOE_ERR_CUDA if the launch fails.
+ */
+moe_status moe_router_topk(const float* logits, int T, int E, int k, int renormalize,
+                           int32_t* topk_idx, float* topk_w, void* stream);
+
+/*
  * Which kernel path a call with this shape takes, without launching anything:
  * 1 = expert-major dequant-GEMV layer kernel (T*k <= 1024 and its shared-memory
  * plan fits), 2 = grouped tensor-core path (route-union, x packing, gate+up and

@@ -56,6 +56,8 @@ def _load():
     lib.moe_select_path.argtypes = [ci] * 5
     lib.moe_route_union.restype = ci
     lib.moe_route_union.argtypes = [vp, ci, ci, ci, vp, vp, vp, vp, vp]
+    lib.moe_router_topk.restype = ci
+    lib.moe_router_topk.argtypes = [vp, ci, ci, ci, ci, vp, vp, vp]
     lib.moe_switchglu_forward.restype = ci
     lib.moe_switchglu_forward.argtypes = [vp] * 12 + [ci] * 5 + [vp, vp]
     lib.moe_switchglu_forward_ws.restype = ci
@@ -152,6 +154,25 @@ def moe_route_union(topk_idx: torch.Tensor, E: int, unique=None, offsets=None, p
                               _ptr(num_unique, _I32, "num_unique"), _stream(stream))
     _check(st, "moe_route_union", check)
     return unique, offsets, pair_list, num_unique
+
+
+def moe_router_topk(logits: torch.Tensor, k: int, renormalize: bool = True, topk_idx=None,
+                    topk_w=None, stream=None, check: bool = True):
+    """Router step: top-k of softmax over each row of logits [T, E] (fp32, CUDA),
+    descending, lower expert id first among equal logits; weights renormalised over
+    the k unless renormalize is False.  Returns (topk_idx [T, k] int32, topk_w [T, k]
+    fp32), the inputs of moe_switchglu_forward."""
+    T, E = logits.shape
+    dev = logits.device
+    topk_idx = topk_idx if topk_idx is not None else torch.empty((T, k), dtype=torch.int32,
+                                                                 device=dev)
+    topk_w = topk_w if topk_w is not None else torch.empty((T, k), dtype=torch.float32,
+                                                           device=dev)
+    st = _lib.moe_router_topk(_ptr(logits, _F32, "logits"), T, E, k, 1 if renormalize else 0,
+                              _ptr(topk_idx, _I32, "topk_idx"), _ptr(topk_w, _F32, "topk_w"),
+                              _stream(stream))
+    _check(st, "moe_router_topk", check)
+    return topk_idx, topk_w
 
 
 class QuantBank:

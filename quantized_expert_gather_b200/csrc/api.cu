@@ -12,6 +12,7 @@
 #include "layer.cuh"
 #include "route_union.cuh"
 #include "grouped.cuh"
+#include "router.cuh"
 
 namespace qeg {
 namespace {
@@ -365,6 +366,21 @@ moe_status moe_workspace_layout(int T, int k, int E, int hidden, int inter, size
 
 int moe_select_path(int T, int k, int E, int hidden, int inter) {
   return select_path(T, k, E, hidden, inter);
+}
+
+moe_status moe_router_topk(const float* logits, int T, int E, int k, int renormalize,
+                           int32_t* topk_idx, float* topk_w, void* stream) {
+  if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (T <= 0 || E <= 0 || k <= 0 || k > E) return MOE_ERR_INVALID_ARG;
+  if (E > kRouterMaxE || k > kRouterMaxK || (long long)T * k > MOE_MAX_PAIRS)
+    return MOE_ERR_UNSUPPORTED;
+  if (!aligned(logits, 4) || !aligned(topk_idx, 4) || !aligned(topk_w, 4))
+    return MOE_ERR_UNSUPPORTED;
+  const int grid = (T + kRouterWarps - 1) / kRouterWarps;
+  router_topk_kernel<<<grid, 32 * kRouterWarps, 0, (cudaStream_t)stream>>>(
+      logits, T, E, k, renormalize ? 1 : 0, topk_idx, topk_w);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
 
 moe_status moe_route_union(const int32_t* topk_idx, int T, int k, int E, int32_t* unique,

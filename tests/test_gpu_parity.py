@@ -345,3 +345,47 @@ def test_grouped_large_window(T, n_check):
     L = make_layer(T, 8, 256, 4096, 2048, seed=5000 + T, routing="uniform", draw_all=False)
     tokens = sorted(np.random.default_rng(T).choice(T, n_check, replace=False).tolist())
     check_layer(L, f"large window T={T}", tokens=tokens)
+
+
+# ------------------------------------------------------------- router step ---
+# Weights: exp in fp32 (CUDA expf, at most 2 ulp) and fp32 sums of at most 1024 terms
+# (32 per lane, then a 5-level butterfly) against fp64: relative error below ~40 ulp
+# of fp32 (2.4e-6); the test allows 2e-5.  The picks compare the fp32 logits as given
+# on both sides, so they are compared bit for bit.
+ROUTER_RTOL = 2e-5
+
+
+@pytest.mark.parametrize("T,E,k,renorm,ties", [
+    (1, 288, 8, True, False), (4, 288, 8, True, False), (16, 256, 8, True, False),
+    (2, 16, 2, True, False), (64, 1024, 32, True, False), (33, 1, 1, True, False),
+    (7, 288, 8, False, False), (5, 1000, 32, False, False), (300, 64, 8, True, True),
+    (4096, 256, 8, True, False), (9, 32, 32, True, True),
+])
+def test_router_topk_matches_oracle(T, E, k, renorm, ties):
+    rng = np.random.default_rng(1000 + T * 7 + E + k)
+    lg = rng.standard_normal((T, E))
+    if ties:  # many equal logits: the lower expert id must come first
+        lg = np.round(lg * 2) / 2
+    lg = lg.astype(np.float32)
+    idx, w = qeg.moe_router_topk(torch.from_numpy(lg).cuda(), k, renormalize=renorm)
+    torch.cuda.synchronize()
+    ridx, rw = oracle.router_topk(lg, k, renormalize=renorm)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    np.testing.assert_allclose(w.cpu().numpy().astype(np.float64), rw, rtol=ROUTER_RTOL, atol=0)
+
+
+def test_router_feeds_the_layer():
+    """Logits -> router -> layer on the device, against the oracle's router and layer."""
+    L = tiny_layer()
+    rng = np.random.default_rng(77)
+    lg = rng.standard_normal((L.T, L.E)).astype(np.float32)
+    bank = to_dev_bank(L)
+    x, _, _ = to_dev_inputs(L)
+    idx, w = qeg.moe_router_topk(torch.from_numpy(lg).cuda(), L.k)
+    out = qeg.moe_switchglu_forward(x, idx, w, bank)
+    torch.cuda.synchronize()
+    assert qeg.moe_read_device_status() == qeg.MOE_OK
+    ridx, rw = oracle.router_topk(lg, L.k)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    ref = oracle.switchglu(L.x, ridx, rw.astype(np.float32), L.bank, L.E)
+    assert_parity(bf16_to_f64(out), ref, "router -> layer")

@@ -25,7 +25,8 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("moe_route_union", "moe_switchglu_forward", "moe_switchglu_forward_ws",
               "moe_workspace_size", "moe_read_device_status", "moe_status_str",
-              "moe_select_path", "moe_workspace_layout", "moe_switchglu_forward_static"):
+              "moe_select_path", "moe_workspace_layout", "moe_switchglu_forward_static",
+              "moe_router_topk"):
         assert n in names
 
 
@@ -109,3 +110,11 @@ def test_validation_rejects_before_touching_memory():
                                None) == qeg.MOE_ERR_UNSUPPORTED
     assert lib.moe_route_union(None, 2, 2, 8, fake, fake, fake, fake,
                                None) == qeg.MOE_ERR_INVALID_ARG
+    # router step: null pointers, bad sizes, k > E, limits, misalignment
+    assert lib.moe_router_topk(None, 4, 16, 2, 1, fake, fake, None) == qeg.MOE_ERR_INVALID_ARG
+    assert lib.moe_router_topk(fake, 4, 16, 2, 1, None, fake, None) == qeg.MOE_ERR_INVALID_ARG
+    assert lib.moe_router_topk(fake, 0, 16, 2, 1, fake, fake, None) == qeg.MOE_ERR_INVALID_ARG
+    assert lib.moe_router_topk(fake, 4, 16, 17, 1, fake, fake, None) == qeg.MOE_ERR_INVALID_ARG
+    assert lib.moe_router_topk(fake, 4, 2048, 8, 1, fake, fake, None) == qeg.MOE_ERR_UNSUPPORTED
+    assert lib.moe_router_topk(fake, 4, 64, 33, 1, fake, fake, None) == qeg.MOE_ERR_UNSUPPORTED
+    assert lib.moe_router_topk(fake + 2, 4, 16, 2, 1, fake, fake, None) == qeg.MOE_ERR_UNSUPPORTED
