@@ -6,8 +6,10 @@ import torch
 
 import quantized_expert_gather_b200 as qeg
 
-# Parity bar for the bf16 layer output (the rel-L2 bound of the target; the
-# max-abs bound is taken on the unit-RMS scale of the reference).
+# Parity bar for the bf16 layer output: rel-L2 = |out - ref| / |ref| over the whole
+# output, and max-abs measured on the unit-RMS scale of the reference (max |out - ref|
+# / rms(ref)), since the raw output of N(0,1) weights and inputs has an RMS near 1e5,
+# where one bf16 step is already far above an absolute 3e-2.
 REL_L2_TOL = 5e-3
 MAX_ABS_TOL = 3e-2
 
