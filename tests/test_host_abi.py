@@ -81,6 +81,23 @@ def test_workspace_size_and_layout():
         qeg.moe_workspace_layout(4, 8, E, 100, I)
 
 
+def test_workspace_follows_the_path():
+    """The grouped path's workspace also holds the packed activations: x and h rows
+    for every pair position padded to 16 per expert, bf16, and their fp32 group
+    sums; the persistent kernel's does not grow with them."""
+    E, H, I = 256, 4096, 2048
+    for T in (512, 2048):
+        P = T * 8
+        assert qeg.moe_select_path(T, 8, E, H, I) == 2
+        pcap = P + 15 * min(E, P)
+        packed = 2 * (H + I) * pcap + 4 * (H + I) // 64 * pcap
+        lay = qeg.moe_workspace_layout(T, 8, E, H, I)
+        assert lay["total"] >= lay["y"] + 4 * P * H + packed
+    # the small-window path stays within the 4 MiB no-allocation scratch at T=16
+    assert qeg.moe_select_path(16, 8, E, H, I) == 1
+    assert qeg.moe_workspace_size(16, 8, E, H, I) <= qeg.MOE_STATIC_SCRATCH_BYTES
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="uses fake pointers; host-only check")
 def test_validation_rejects_before_touching_memory():
     lib = qeg._lib
