@@ -66,8 +66,9 @@ typedef enum {
  * hidden and inter multiples of 64, hidden <= 4096, inter <= 8192; E <= 1024;
  * T*k <= 65536.  Windows of more than 1024 pairs (or whose persistent-kernel
  * plan does not fit) take the grouped tensor-core path, which further needs
- * hidden a multiple of 256 and inter a multiple of 128; moe_select_path tells
- * which path a shape takes. */
+ * hidden a multiple of 256, inter a multiple of 128 and T*k <= 57856 (its
+ * combine keeps a pair index per pair in shared memory); moe_select_path tells
+ * which path a shape takes (0: the call returns MOE_ERR_UNSUPPORTED). */
 #define MOE_MAX_EXPERTS 1024
 #define MOE_MAX_DIM 8192
 #define MOE_MAX_PAIRS 65536

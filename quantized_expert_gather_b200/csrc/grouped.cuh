@@ -462,7 +462,6 @@ __global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
       const float2 s2 = make_float2(sv, sv), b2 = make_float2(bv, bv);
       const float4* X = reinterpret_cast<const float4*>(stg + C::kOffX + jj * C::kN * 4);
       const uint32_t dcol = tmem + C::col_d(ab, m) + lane_base;
-#pragma unroll
       // kRd columns per tensor-memory wait (16 where registers are scarce)
       constexpr int kRd = C::kN == 64 ? 32 : 16, kRg = kRd / 16;
 #pragma unroll
