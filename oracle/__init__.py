@@ -54,6 +54,10 @@ def load(so: Optional[str] = None):
     lib.oracle_round_bf16.argtypes = [ctypes.c_double]
     lib.oracle_router_topk.restype = None
     lib.oracle_router_topk.argtypes = [vp, ci, ci, ci, ci, vp, vp]
+    lib.oracle_switchglu_mxfp4.restype = None
+    lib.oracle_switchglu_mxfp4.argtypes = [vp] * 9 + [ci] * 5 + [vp, ci, ci, vp, vp, vp]
+    lib.oracle_mxfp4_value.restype = ctypes.c_double
+    lib.oracle_mxfp4_value.argtypes = [ci, ci]
     if so is None:
         _lib = lib
     return lib
@@ -152,3 +156,35 @@ def router_topk(logits: np.ndarray, k: int, renormalize: bool = True, lib=None):
     w = np.zeros((T, k), np.float64)
     lib.oracle_router_topk(pl, T, E, k, 1 if renormalize else 0, idx.ctypes.data, w.ctypes.data)
     return idx, w
+
+
+def mxfp4_value(code: int, scale: int, lib=None) -> float:
+    """The oracle's value of one mxfp4 weight: e2m1 code (0..15) times 2^(scale - 127)."""
+    return (lib or load()).oracle_mxfp4_value(int(code), int(scale))
+
+
+def switchglu_mxfp4(x, idx, w, bank: dict, E: int, tokens=None, want_h=False, lib=None):
+    """The layer on mxfp4 banks: bank = {"gate": (q, e8), "up": (q, e8), "down": (q, e8)}
+    with q uint32 [E, rows, cols/8] (e2m1 codes) and e8 uint8 [E, rows, cols/32]
+    (e8m0 scales).  Same outputs as switchglu: out [T, H] fp64 (and h [T*k, I])."""
+    lib = lib or load()
+    x, px = _c(x, np.uint16)
+    idx, pidx = _c(idx, np.int32)
+    w, pw = _c(w, np.float32)
+    T, H = x.shape
+    k = idx.shape[1]
+    I = bank["gate"][0].shape[1]
+    arrs = []
+    for name in ("gate", "up", "down"):
+        q, e8 = bank[name]
+        arrs.append(_c(q, np.uint32))
+        arrs.append(_c(e8, np.uint8))
+    tok = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int32)
+    out = np.zeros((T, H), np.float64)
+    h = np.zeros((T * k, I), np.float64) if want_h else None
+    lib.oracle_switchglu_mxfp4(px, pidx, pw, *[a[1] for a in arrs], T, k, E, H, I,
+                               None if tok is None else tok.ctypes.data,
+                               0 if tok is None else len(tok), os.cpu_count() or 1,
+                               out.ctypes.data, None if h is None else h.ctypes.data, None)
+    return (out, h) if want_h else out
+

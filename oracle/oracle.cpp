@@ -29,6 +29,11 @@
 //   4*(c%8) .. 4*(c%8)+3, least significant first) of 32-bit word c / 8.
 // * Expert ids outside [0, E) name no expert: such a pair is left out of the
 //   union and contributes nothing.
+// * mxfp4 banks (oracle_switchglu_mxfp4): GLM-5.2's routed banks are "mxfp4 gs32"
+//   ("Small-L fused expert gather", mlx discussion 3801, the decomposition post).
+//   Reading: the OCP microscaling format, e2m1 elements (values 0, 0.5, 1, 1.5,
+//   2, 3, 4, 6 and their negatives) with one e8m0 scale 2^(e - 127) per 32
+//   input columns, packed like the affine codes; w = e2m1(q) * 2^(e - 127).
 // * The router step before the layer (oracle_router_topk): top-k of softmax over
 //   the experts, renormalised over the k, as the tiny parity configuration routes
 //   its tokens; equal logits go to the lower expert id.
@@ -69,16 +74,27 @@ double round_bf16(double v) {
 
 double sigmoid(double g) { return 1.0 / (1.0 + std::exp(-g)); }
 
-struct Matrix {  // one expert bank: q [E, rows, cols/8], s/b [E, rows, cols/64]
+// fp4 e2m1 code -> value: sign bit 3, exponent bits 2..1 (bias 1), mantissa bit 0
+// (the element format of mxfp4).
+const double kE2M1[16] = {0.0,  0.5,  1.0,  1.5,  2.0,  3.0,  4.0,  6.0,
+                          -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0};
+
+// e8m0 scale byte -> 2^(byte - 127) (the block scale of mxfp4; 255 would be NaN).
+double e8m0_value(uint8_t v) { return std::ldexp(1.0, static_cast<int>(v) - 127); }
+
+struct Matrix {  // one expert bank, q [E, rows, cols/8] and per format:
   const uint32_t* q;
-  const uint16_t* s;
-  const uint16_t* b;
+  const uint16_t* s;   // affine group 64: scales bf16 [E, rows, cols/64]
+  const uint16_t* b;   //                  biases bf16 [E, rows, cols/64]
+  const uint8_t* e8;   // mxfp4 group 32: e8m0 scales [E, rows, cols/32]
   int rows, cols;
+  bool mxfp4;
   // dequantised weight of expert e at (row, col)
   double at(int e, int row, int col) const {
     const size_t r = static_cast<size_t>(e) * rows + row;
     const uint32_t word = q[r * (cols / 8) + col / 8];
     const int nib = static_cast<int>((word >> (4 * (col % 8))) & 0xFu);
+    if (mxfp4) return kE2M1[nib] * e8m0_value(e8[r * (cols / 32) + col / 32]);
     const size_t g = r * (cols / 64) + col / 64;
     return bf16_value(s[g]) * nib + bf16_value(b[g]);
   }
@@ -144,9 +160,9 @@ Layer make_layer(const uint16_t* x, const int32_t* idx, const float* w, const ui
                  int T, int k, int E, int H, int I) {
   Layer L;
   L.x = x; L.idx = idx; L.w = w;
-  L.gate = Matrix{gq, gs, gb, I, H};
-  L.up = Matrix{uq, us, ub, I, H};
-  L.down = Matrix{dq, ds, db, H, I};
+  L.gate = Matrix{gq, gs, gb, nullptr, I, H, false};
+  L.up = Matrix{uq, us, ub, nullptr, I, H, false};
+  L.down = Matrix{dq, ds, db, nullptr, H, I, false};
   L.T = T; L.k = k; L.E = E; L.H = H; L.I = I;
   return L;
 }
@@ -185,6 +201,11 @@ void combine(const Layer& L, const std::vector<int>& pairs, const std::vector<do
   }
 }
 
+}  // namespace
+
+namespace {
+void run_switchglu(const Layer& L, const int32_t* tokens, int n_tokens, int n_threads,
+                   double* out, double* h_out, double* y_out);
 }  // namespace
 
 extern "C" {
@@ -229,7 +250,39 @@ void oracle_switchglu(const uint16_t* x, const int32_t* idx, const float* w, con
                       const uint16_t* ds, const uint16_t* db, int T, int k, int E, int H, int I,
                       const int32_t* tokens, int n_tokens, int n_threads, double* out,
                       double* h_out, double* y_out) {
-  const Layer L = make_layer(x, idx, w, gq, gs, gb, uq, us, ub, dq, ds, db, T, k, E, H, I);
+  run_switchglu(make_layer(x, idx, w, gq, gs, gb, uq, us, ub, dq, ds, db, T, k, E, H, I),
+                tokens, n_tokens, n_threads, out, h_out, y_out);
+}
+
+// The same layer on mxfp4 banks (group 32): q [E, rows, cols/8] e2m1 codes packed
+// as above, e8 [E, rows, cols/32] e8m0 scales; w = e2m1(q) * 2^(e8 - 127).
+void oracle_switchglu_mxfp4(const uint16_t* x, const int32_t* idx, const float* w,
+                            const uint32_t* gq, const uint8_t* ge8, const uint32_t* uq,
+                            const uint8_t* ue8, const uint32_t* dq, const uint8_t* de8, int T,
+                            int k, int E, int H, int I, const int32_t* tokens, int n_tokens,
+                            int n_threads, double* out, double* h_out, double* y_out) {
+  Layer L;
+  L.x = x; L.idx = idx; L.w = w;
+  L.gate = Matrix{gq, nullptr, nullptr, ge8, I, H, true};
+  L.up = Matrix{uq, nullptr, nullptr, ue8, I, H, true};
+  L.down = Matrix{dq, nullptr, nullptr, de8, H, I, true};
+  L.T = T; L.k = k; L.E = E; L.H = H; L.I = I;
+  run_switchglu(L, tokens, n_tokens, n_threads, out, h_out, y_out);
+}
+
+// One mxfp4 weight, exported so its pins can test the decoding directly.
+double oracle_mxfp4_value(int code, int scale) {
+  return kE2M1[code & 15] * e8m0_value(static_cast<uint8_t>(scale));
+}
+
+}  // extern "C"
+
+namespace {
+
+void run_switchglu(const Layer& L, const int32_t* tokens, int n_tokens, int n_threads,
+                   double* out, double* h_out, double* y_out) {
+  const int T = L.T, k = L.k, E = L.E, H = L.H, I = L.I;
+  (void)T; (void)k; (void)E;
   const std::vector<int> pairs = selected_pairs(L, tokens, n_tokens);
   const int np = static_cast<int>(pairs.size());
   std::vector<double> hbuf(static_cast<size_t>(np) * I, 0.0), ybuf(static_cast<size_t>(np) * H, 0.0);
@@ -256,6 +309,10 @@ void oracle_switchglu(const uint16_t* x, const int32_t* idx, const float* w, con
                   sizeof(double) * H);
   }
 }
+
+}  // namespace
+
+extern "C" {
 
 // Deduplicated form: take the union of experts, dequantise each distinct
 // expert's three matrices once, and apply them to every pair routed to it

@@ -12,6 +12,9 @@ the oracle itself.
 * the router step: equal logits (ties to the lower id, weights 1/k or 1/E), a
   logarithmic ramp (weights proportional to i + 1, a closed form), k = E against
   scipy's softmax, torch.topk's selection, shift invariance;
+* mxfp4 banks: the e2m1 / e8m0 decoding against ml_dtypes (a library routine), the
+  layer on weights that both formats hold exactly bit-identical to the affine form,
+  and E=1, k=1 against a dense SwiGLU of ml_dtypes-decoded matrices;
 * a set of planted mistakes (in copies of the oracle source) each fail a pin.
 """
 import math
@@ -286,6 +289,9 @@ MUTANTS = {
                               "acc += Y["),
     "down_transposed": ("Y += L.down.at(e, c, r) * h[r];", "Y += L.down.at(e, r, c) * h[r];"),
     "h_product_unrounded": ("h[r] = round_bf16(g * sigmoid(g) * v);", "h[r] = g * sigmoid(g) * v;"),
+    "mxfp4_table_swapped": ("0.0,  0.5,  1.0,  1.5,  2.0,  3.0,  4.0,  6.0,",
+                            "0.0,  0.5,  1.0,  2.0,  1.5,  3.0,  4.0,  6.0,"),
+    "mxfp4_scale_bias": ("static_cast<int>(v) - 127)", "static_cast<int>(v) - 126)"),
     "router_ascending": ("[row](int a, int b) { return row[a] > row[b]; }",
                          "[row](int a, int b) { return row[a] < row[b]; }"),
     "router_ties_to_higher_id": ("[row](int a, int b) { return row[a] > row[b]; }",
@@ -310,6 +316,7 @@ def run(f):
 run(P._pin_closed_forms)
 run(P._pin_textbook)
 run(P._pin_router)
+run(P._pin_mxfp4)
 print("FAILS", fails)
 """
 
@@ -376,6 +383,80 @@ def _pin_router(lib):
     assert list(idx[0]) == [2, 6, 0]
 
 
+def _e2m1_codes(vals: np.ndarray) -> np.ndarray:
+    """e2m1 codes of values the format holds exactly, encoded by ml_dtypes."""
+    import ml_dtypes
+    return np.asarray(vals, np.float32).astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 15
+
+
+def _shared_banks(rng, E, H, I, e8, s, b):
+    """Random weights from {0, +-0.5, +-1, +-1.5, +-2, +-3} * 2^(e8 - 127), held
+    exactly both as mxfp4 (scale e8) and as affine (scale s, bias b)."""
+    vals = np.array([0, 0.5, -0.5, 1, -1, 1.5, -1.5, 2, -2, 3, -3])
+    mx, af = {}, {}
+    for name, rows, cols in (("gate", I, H), ("up", I, H), ("down", H, I)):
+        v = rng.choice(vals, size=(E, rows, cols))
+        scale = 2.0 ** (e8 - 127)
+        mx[name] = (np.stack([pack_nibbles(_e2m1_codes(v[e])) for e in range(E)]),
+                    np.full((E, rows, cols // 32), e8, np.uint8))
+        q = np.rint((v * scale - b) / s).astype(np.int64)
+        assert q.min() >= 0 and q.max() <= 15 and np.all(q * s + b == v * scale)
+        af[name] = (np.stack([pack_nibbles(q[e]) for e in range(E)]),
+                    np.full((E, rows, cols // 64), bf16_bits(s), np.uint16),
+                    np.full((E, rows, cols // 64), bf16_bits(b), np.uint16))
+    return mx, af
+
+
+def _pin_mxfp4(lib):
+    import ml_dtypes
+    codes = np.arange(16, dtype=np.uint8)
+    ref = codes.view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    for e8 in (100, 120, 126, 127, 128, 131, 150):
+        sc = float(np.array([e8], np.uint8).view(ml_dtypes.float8_e8m0fnu).astype(np.float64)[0])
+        got = np.array([oracle.mxfp4_value(c, e8, lib=lib) for c in range(16)])
+        assert np.array_equal(got, ref * sc)
+    rng = np.random.default_rng(23)
+    T, k, E, H, I = 3, 2, 4, 128, 64
+    x = bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+    idx = np.array([[0, 3], [2, 2], [1, 0]], np.int32)
+    w = np.array([[0.25, 0.75], [0.5, 0.5], [1.0, -0.5]], np.float32)
+    for e8, s, b in ((127, 0.5, -3.0), (128, 1.0, -6.0), (125, 0.125, -0.75)):
+        mx, af = _shared_banks(rng, E, H, I, e8, s, b)
+        out_mx = oracle.switchglu_mxfp4(x, idx, w, mx, E, lib=lib)
+        out_af = oracle.switchglu(x, idx, w, af, E, lib=lib)
+        assert np.array_equal(out_mx, out_af)
+
+
+def test_mxfp4_pins():
+    _pin_mxfp4(oracle.load())
+
+
+def test_mxfp4_single_expert_is_dense_swiglu():
+    """E=1, k=1 with random codes and scales: the mxfp4 layer equals a dense SwiGLU
+    of the matrices decoded by ml_dtypes (numpy matmul)."""
+    import ml_dtypes
+    rng = np.random.default_rng(29)
+    H, I = 128, 64
+    bank, dense = {}, {}
+    for name, rows, cols in (("gate", I, H), ("up", I, H), ("down", H, I)):
+        c = rng.integers(0, 16, size=(rows, cols)).astype(np.uint8)
+        e8 = rng.integers(118, 124, size=(rows, cols // 32)).astype(np.uint8)
+        bank[name] = (pack_nibbles(c)[None], e8[None])
+        vals = c.view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+        dense[name] = vals * e8.view(ml_dtypes.float8_e8m0fnu).astype(np.float64).repeat(32, axis=1)
+    xf = rng.standard_normal(H).astype(np.float32)
+    x = bf16_bits(xf)[None]
+    out, h = oracle.switchglu_mxfp4(x, np.zeros((1, 1), np.int32), np.full((1, 1), 0.75, np.float32),
+                                    bank, 1, want_h=True)
+    xd = synth.bf16_bits_to_f32(x[0]).astype(np.float64)
+    g = bf16_round_ref(dense["gate"] @ xd)
+    v = bf16_round_ref(dense["up"] @ xd)
+    href = bf16_round_ref(g * v / (1 + np.exp(-g)))
+    assert np.mean(h[0] == href) > 0.97
+    yref = 0.75 * (dense["down"] @ href)
+    assert np.allclose(out[0], yref, rtol=0, atol=1e-3 * np.abs(yref).max())
+
+
 def test_router_pins():
     _pin_router(oracle.load())
 
@@ -419,3 +500,4 @@ def test_unmutated_oracle_passes_mutant_pins():
     _pin_closed_forms(lib)
     _pin_textbook(lib)
     _pin_router(lib)
+    _pin_mxfp4(lib)
