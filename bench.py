@@ -43,6 +43,11 @@ SEED = 2000
 BYTES_PER_EXPERT = 3 * (INTER * HIDDEN // 2 + 2 * 2 * INTER * HIDDEN // 64)  # 14,155,776
 METRIC = "us/layer and effective HBM GB/s (unique-expert bytes) at T=1..16, % of B200 peak"
 L2_BYTES = 126 * 1024 * 1024
+# what the small-window kernel computes in: 4-bit affine codes times bf16 activations held
+# as 16-bit block fixed point per 32 columns (exact for values within 8 binades of their
+# chunk's largest), integer dot products, fp32 scaling and accumulation
+DTYPE_LABEL = ("u4 affine weights x bf16 act as 16-bit block fixed point per 32 columns "
+               "(exact int dot), f32 accum")
 
 
 def measured_peaks():
@@ -198,6 +203,74 @@ class ClockSampler:
 
 # --------------------------------------------------------------- workload ---
 ROUTING = "uniform"  # --routing markov: adjacent-overlap chain at p=0.40 (profiling)
+# speculative-verify pair: adjacent-token overlap at random (3 %), in shallow layers, the
+# mean, in deep layers and the maximum of the pages' router recording
+VERIFY_PS = (0.03, 0.21, 0.34, 0.45, 0.52)
+# verify-window sweep: window sizes, and the layers of the stack (GLM-5.2's MoE depth)
+WINDOW_TS = (2, 3, 5, 8, 16)
+WINDOW_LAYERS = 78
+
+
+def graph_us_per_layer(issue, n_layers: int, reps: int = 5) -> float:
+    """Device time per layer of `issue()` (n_layers launches, no host synchronisation)
+    captured once in a CUDA graph: one warm replay, then `reps` replays between CUDA
+    events on the current stream."""
+    import torch
+    issue()  # first calls outside the capture (per-device set-up)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        issue()
+    g.replay()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b) * 1e3 / (reps * n_layers)
+    del g
+    return us
+
+
+def window_layer_seed(T: int, layer: int) -> int:
+    return SEED + 10000 + 100 * T + layer
+
+
+def window_stack(T: int, dev, qeg, synth, layers: int = None):
+    """The verify-window stack at window size T: per layer an adjacent-overlap routing at
+    p = 0.40 over E=256 experts, and a bank compacted to the u experts that window routes
+    to (drawn on the device, seed per layer; routing ids remapped to 0..u-1), its own x,
+    workspace and output buffer.  Returns {"layers": [...], "unique": [u per layer]}."""
+    import torch
+    layers = layers or WINDOW_LAYERS
+    out, uniq = [], []
+    for l in range(layers):
+        seed = window_layer_seed(T, l)
+        idx, w = synth.route_markov(T, 256, K_TOP, 0.40, seed)
+        used, remap = np.unique(idx, return_inverse=True)
+        u = int(used.size)
+        cidx = remap.reshape(idx.shape).astype(np.int32)
+
+        def mat(rows, cols, mid):
+            q = torch.empty((u, rows, cols // 8), dtype=torch.int32, device=dev)
+            s_ = torch.empty((u, rows, cols // 64), dtype=torch.int16, device=dev)
+            b_ = torch.empty_like(s_)
+            synth.fill_bank_device(q, s_, b_, rows, cols, seed, mid)
+            return q, s_.view(torch.bfloat16), b_.view(torch.bfloat16)
+        bank = qeg.QuantBank(*mat(INTER, HIDDEN, 0), *mat(INTER, HIDDEN, 1),
+                             *mat(HIDDEN, INTER, 2))
+        out.append({
+            "bank": bank, "seed": seed, "idx_host": cidx, "w_host": w,
+            "idx": torch.from_numpy(cidx).to(dev), "w": torch.from_numpy(w).to(dev),
+            "x": torch.from_numpy(synth.x_bf16(T, HIDDEN, seed).view(np.int16)).to(dev)
+            .view(torch.bfloat16),
+            "ws": torch.zeros(qeg.moe_workspace_size(T, K_TOP, u, HIDDEN, INTER),
+                              dtype=torch.uint8, device=dev),
+            "out": torch.empty((T, HIDDEN), dtype=torch.bfloat16, device=dev)})
+        uniq.append(u)
+    torch.cuda.synchronize()
+    return {"layers": out, "unique": uniq}
 
 
 def routings():
@@ -220,27 +293,44 @@ def cpu_cores():
     return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
 
 
-def run_oracle_sample(routes, budget_s: float = 15.0):
+def parity_of(got: np.ndarray, ref: np.ndarray):
+    """(rel-L2, max-abs / rms(ref)) of a layer output against the oracle's: the parity
+    measures of the GPU tests (bar: 5e-3 and 3e-2)."""
+    d = got - ref
+    rel = float(np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-300))
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    return rel, float(np.abs(d).max() / rms) if rms > 0 else float(np.abs(d).max())
+
+
+def run_oracle_sample(routes, budget_s: float = 15.0, gpu_outs=None):
     """Time the oracle (all host threads) on whole layers of the workload until about
     `budget_s` of CPU work: every layer of the chain once, then (if time is left) the
-    last T=1 and T=4 layers again.  Returns (GB/s over unique bytes, layers timed,
-    seconds, threads)."""
+    last T=1 and T=4 layers again.  Each layer the oracle computes is also compared with
+    the GPU's kept output of the same chained layer (gpu_outs[T][l], bf16 bits), outside
+    the timed call.  Returns (GB/s over unique bytes, layers timed, seconds, threads,
+    parity summary)."""
     import oracle
     import synth
     threads = cpu_cores()
     done, secs, nbytes = 0, 0.0, 0
     order = [(T, l) for l in range(LAYERS) for T in TS]
     last = {}
+    checked, worst_rel, worst_mx = [], 0.0, 0.0
 
     def timed(T, l, bank, used):
-        nonlocal done, secs, nbytes
+        nonlocal done, secs, nbytes, worst_rel, worst_mx
         idx, w = routes[T][l]
         x = synth.x_bf16(T, HIDDEN, SEED + T)
         t0 = time.perf_counter()
-        oracle.switchglu(x, idx, w, bank, E, n_threads=threads)
+        ref = oracle.switchglu(x, idx, w, bank, E, n_threads=threads)
         secs += time.perf_counter() - t0
         done += 1
         nbytes += len(used) * BYTES_PER_EXPERT
+        if gpu_outs is not None and (T, l) not in checked:
+            got = synth.bf16_bits_to_f32(gpu_outs[T][l]).astype(np.float64)
+            rel, mx = parity_of(got, ref)
+            worst_rel, worst_mx = max(worst_rel, rel), max(worst_mx, mx)
+            checked.append((T, l))
 
     for T, l in order:
         used = sorted(set(routes[T][l][0].ravel().tolist()))
@@ -255,7 +345,14 @@ def run_oracle_sample(routes, budget_s: float = 15.0):
         for T in TS:
             l, bank, used = last[T]
             timed(T, l, bank, used)
-    return nbytes / secs / 1e9, done, secs, threads
+    parity = None
+    if gpu_outs is not None:
+        parity = {"layers_checked": len(checked), "max_rel_l2": worst_rel,
+                  "max_abs_over_rms": worst_mx,
+                  "pass": bool(worst_rel <= 5e-3 and worst_mx <= 3e-2),
+                  "what": "the GPU outputs of the chained layers kept from the timed graph "
+                          "replays, against the oracle on the same inputs"}
+    return nbytes / secs / 1e9, done, secs, threads, parity
 
 
 def reference_arm(args, world, rank):
@@ -377,6 +474,8 @@ def our_arm(args, world, rank, local):
         torch.cuda.synchronize()
     barrier(world)
     ms_total = max_over_ranks(e0.elapsed_time(e1), world)
+    # every chained layer's output of the last timed replay, kept for the parity check
+    kept = {T: [o.view(torch.int16).cpu().numpy().view(np.uint16) for o in outs[T]] for T in TS}
     ms_step = ms_total / args.steps
     all_bytes = sum_over_ranks(total_bytes * args.steps, world)
     gbs = all_bytes / (ms_total * 1e-3) / 1e9
@@ -432,11 +531,13 @@ def our_arm(args, world, rank, local):
         per[T]["graph_gbs"] = sum(uq[T]) * BYTES_PER_EXPERT / LAYERS / (us * 1e-6) / 1e9
         del g2
 
-    # speculative-verify pair (E=256, p=0.34): a T=2 window against its first token
-    # alone, 42 chained layers each, CUDA graph; the target is T=2 <= 1.7 x T=1
+    # speculative-verify pair (E=256): a T=2 window against its first token alone, 42
+    # chained layers each, CUDA graph, swept over the adjacent-token overlap p of the
+    # pages' measurements; the target is T=2 <= 1.7 x T=1 at p = 0.34
     verify = None
+    E2 = 256
+    bank2 = None
     if not args.no_verify_pair:
-        E2 = 256
         def mat2(rows, cols, mid):
             q = torch.empty((E2, rows, cols // 8), dtype=torch.int32, device=dev)
             s_ = torch.empty((E2, rows, cols // 64), dtype=torch.int16, device=dev)
@@ -445,42 +546,80 @@ def our_arm(args, world, rank, local):
             return q, s_.view(torch.bfloat16), b_.view(torch.bfloat16)
         bank2 = qeg.QuantBank(*mat2(INTER, HIDDEN, 0), *mat2(INTER, HIDDEN, 1),
                               *mat2(HIDDEN, INTER, 2))
-        pairs = [synth.route_verify_pair(E2, K_TOP, 0.34, SEED + 500 + l) for l in range(LAYERS)]
         x2 = torch.from_numpy(synth.x_bf16(2, HIDDEN, SEED + 2).view(np.int16)).to(dev) \
             .view(torch.bfloat16)
         ws2 = torch.zeros(qeg.moe_workspace_size(2, K_TOP, E2, HIDDEN, INTER), dtype=torch.uint8,
                           device=dev)
-        runs = {}
-        for T2 in (1, 2):
-            ids = [torch.from_numpy(np.ascontiguousarray(r[0][:T2])).to(dev) for r in pairs]
-            wv = [torch.from_numpy(np.ascontiguousarray(r[1][:T2])).to(dev) for r in pairs]
-            o2 = [torch.empty((T2, HIDDEN), dtype=torch.bfloat16, device=dev) for _ in pairs]
-            xs2 = x2[:T2]
-            for l in range(LAYERS):  # warm, outside capture
-                qeg.moe_switchglu_forward_ws(xs2, ids[l], wv[l], bank2, ws2, out=o2[l])
-            g3 = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g3):
-                for l in range(LAYERS):
-                    qeg.moe_switchglu_forward_ws(xs2, ids[l], wv[l], bank2, ws2, out=o2[l])
-            g3.replay()
-            a3, b3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a3.record()
-            for _ in range(5):
-                g3.replay()
-            b3.record()
-            torch.cuda.synchronize()
-            runs[T2] = a3.elapsed_time(b3) * 1e3 / (5 * LAYERS)
-            del g3
-        u2 = float(np.mean([np.unique(r[0]).size for r in pairs]))
-        verify = {"E": E2, "p": 0.34, "t1_us_per_layer": runs[1], "t2_us_per_layer": runs[2],
-                  "ratio_t2_over_t1": runs[2] / runs[1], "target_ratio": 1.7,
-                  "mean_unique_t2": u2,
-                  "t2_gbs": u2 * BYTES_PER_EXPERT / (runs[2] * 1e-6) / 1e9}
+        verify = {"E": E2, "target_ratio": 1.7, "target_p": 0.34, "layers": LAYERS, "p": {}}
+        for p in VERIFY_PS:
+            pairs = [synth.route_verify_pair(E2, K_TOP, p, SEED + 500 + int(p * 1000) + l)
+                     for l in range(LAYERS)]
+            runs = {}
+            for T2 in (1, 2):
+                ids = [torch.from_numpy(np.ascontiguousarray(r[0][:T2])).to(dev) for r in pairs]
+                wv = [torch.from_numpy(np.ascontiguousarray(r[1][:T2])).to(dev) for r in pairs]
+                o2 = [torch.empty((T2, HIDDEN), dtype=torch.bfloat16, device=dev) for _ in pairs]
+                xs2 = x2[:T2]
+                runs[T2] = graph_us_per_layer(
+                    lambda: [qeg.moe_switchglu_forward_ws(xs2, ids[l], wv[l], bank2, ws2,
+                                                          out=o2[l]) for l in range(LAYERS)],
+                    LAYERS)
+            u2 = float(np.mean([np.unique(r[0]).size for r in pairs]))
+            verify["p"][str(p)] = {
+                "t1_us_per_layer": runs[1], "t2_us_per_layer": runs[2],
+                "ratio_t2_over_t1": runs[2] / runs[1], "mean_unique_t2": u2,
+                "t2_gbs": u2 * BYTES_PER_EXPERT / (runs[2] * 1e-6) / 1e9,
+                "t1_gbs": 8 * BYTES_PER_EXPERT / (runs[1] * 1e-6) / 1e9}
         del ws2
+        torch.cuda.synchronize()
+
+    # verify-window sweep: T in {2,3,5,8,16} on an adjacent-overlap chain at p = 0.40, a
+    # stack of 78 layers with independent seeded weights per layer; each layer's bank is
+    # compacted to the experts its window routes to (fresh memory per layer, ids remapped),
+    # so no expert repeats across the stack and L2 gives no reuse; graph of the stack
+    window = None
+    if not args.no_window_sweep:
+        window = {"E": E2, "p": 0.40, "layers": WINDOW_LAYERS, "per_T": {}}
+        for TW in WINDOW_TS:
+            stack = window_stack(TW, dev, qeg, synth)
+            us = graph_us_per_layer(
+                lambda: [qeg.moe_switchglu_forward_ws(st["x"], st["idx"], st["w"], st["bank"],
+                                                      st["ws"], out=st["out"])
+                         for st in stack["layers"]], len(stack["layers"]))
+            ub = stack["unique"]
+            window["per_T"][str(TW)] = {
+                "us_per_layer": us, "us_per_stack": us * len(ub),
+                "mean_unique": float(np.mean(ub)),
+                "gbs": float(np.sum(ub)) * BYTES_PER_EXPERT / (us * len(ub) * 1e-6) / 1e9,
+                "frac_of_hbm_peak": float(np.sum(ub)) * BYTES_PER_EXPERT
+                / (us * len(ub) * 1e-6) / 1e9 / measured_peaks()[0],
+                "stack_bytes": float(np.sum(ub)) * BYTES_PER_EXPERT}
+            del stack
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+        # the all-identical extreme: every token of a T=16 window routes to the same 8
+        # experts (16 pairs per expert); each expert must still stream once
+        same = np.tile(np.arange(K_TOP, dtype=np.int32) * 9, (16, 1))
+        wsame = np.full((16, K_TOP), 1.0 / K_TOP, np.float32)
+        ws3 = torch.zeros(qeg.moe_workspace_size(16, K_TOP, E2, HIDDEN, INTER), dtype=torch.uint8,
+                          device=dev)
+        xi = torch.from_numpy(synth.x_bf16(16, HIDDEN, SEED + 16).view(np.int16)).to(dev) \
+            .view(torch.bfloat16)
+        ii, wi = torch.from_numpy(same).to(dev), torch.from_numpy(wsame).to(dev)
+        oi = torch.empty((16, HIDDEN), dtype=torch.bfloat16, device=dev)
+        us = graph_us_per_layer(
+            lambda: [qeg.moe_switchglu_forward_ws(xi, ii, wi, bank2, ws3, out=oi)
+                     for _ in range(LAYERS)], LAYERS)
+        window["all_identical_T16"] = {
+            "us_per_layer": us, "unique": K_TOP, "pairs_per_expert": 16,
+            "gbs": K_TOP * BYTES_PER_EXPERT / (us * 1e-6) / 1e9,
+            "note": "42 launches of one layer (same bank, same routing) in a graph; L2 holds "
+                    "part of the 113 MB between launches"}
+        del ws3
     # large windows (the grouped tensor-core path): T=512 and T=2048 on the E=256 bank,
     # a few layers each, CUDA events; bytes = unique experts, flops = 6 P H I
     large = None
-    if verify is not None and not args.no_large_t:
+    if bank2 is not None and not args.no_large_t:
         large = {}
         for TL, nl in ((512, 3), (2048, 2)):
             rl = [synth.route_uniform(TL, E2, K_TOP, SEED + 900 + TL + l) for l in range(nl)]
@@ -509,7 +648,7 @@ def our_arm(args, world, rank, local):
                               "tflops": fl / (us * 1e-6) / 1e12,
                               "path": "grouped tcgen05 kernels (5 launches per layer)"}
             del wsl
-    if verify is not None:
+    if bank2 is not None:
         del bank2
 
     # the router step ahead of the layer (top-k of softmax, renormalised): 20 calls
@@ -601,10 +740,12 @@ def our_arm(args, world, rank, local):
     traffic = (None if tr is None else
                tr[0] * sum(float(np.mean(uq[T])) for T in TS) / len(TS) + tr[1])
     result = None
+    chained_parity = None
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            cgbs, nl, secs, thr = run_oracle_sample(routes, budget_s=args.cpu_budget)
+            cgbs, nl, secs, thr, chained_parity = run_oracle_sample(
+                routes, budget_s=args.cpu_budget, gpu_outs=kept)
             cpu = {"value": cgbs, "unit": "GB/s", "cores": thr, "kind": "oracle",
                    "sample": f"{nl} whole layers of the workload (each of the 84 layers once, "
                              f"then the last T=1 and T=4 layers again), {secs:.1f} s of "
@@ -612,7 +753,7 @@ def our_arm(args, world, rank, local):
         result = {
             "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "u4 weights x bf16 act, f32 accum",
+            "scaling": "weak", "vs_baseline": None, "dtype": DTYPE_LABEL,
             "data": "synthetic",
             "config": {"workload": "GLM-5.3-Flash-shaped union-of-experts SwitchGLU layer: "
                                    "E=288 top-8 hidden 4096 inter 2048 q4 affine g64 bf16 "
@@ -638,7 +779,9 @@ def our_arm(args, world, rank, local):
                     "d2h_bytes_per_step": int(d2h),
                     "how": "moe_switchglu_forward per layer, pinned host inputs copied in and "
                            "all layer outputs copied back every step"},
+            "chained_parity": chained_parity,
             "verify_pair": verify,
+            "verify_window": window,
             "large_window": large,
             "router": router,
             "gpu_launches": launches_per_step * args.steps,
@@ -663,6 +806,8 @@ def main():
                     help="skip the T=512 / T=2048 grouped-path measurement")
     ap.add_argument("--no-verify-pair", action="store_true",
                     help="skip the T=2 / T=1 speculative-verify measurement")
+    ap.add_argument("--no-window-sweep", action="store_true",
+                    help="skip the verify-window sweep (T=2..16, 78-layer stacks)")
     ap.add_argument("--ts", default="", help="comma-separated window sizes (profiling)")
     ap.add_argument("--routing", default="uniform", choices=("uniform", "markov"),
                     help="routing model (profiling)")

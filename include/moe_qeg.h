@@ -178,7 +178,12 @@ moe_status moe_switchglu_forward_static(const uint16_t* x, const int32_t* topk_i
  * Synchronises `stream`, then reads and clears the device error word that the
  * kernels set instead of trapping: MOE_ERR_DEVICE_INDEX if an expert id was
  * out of range, MOE_ERR_TIMEOUT if a bounded wait ran out, else MOE_OK (or
- * MOE_ERR_CUDA if the synchronisation itself failed).
+ * MOE_ERR_CUDA if the synchronisation itself failed).  On MOE_ERR_TIMEOUT it
+ * also zeroes the counter region of the workspace the library owns on the
+ * current device (the one moe_switchglu_forward uses), so that later calls
+ * start clean; work queued on other streams that uses that workspace must be
+ * complete first.  A caller-owned workspace (moe_switchglu_forward_ws) is the
+ * caller's to clear after a timeout.
  */
 moe_status moe_read_device_status(void* stream);
 

@@ -90,10 +90,19 @@ def _check(status: int, where: str, check: bool) -> int:
     return status
 
 
-def _stream(stream) -> int:
+def _stream(stream, device=None) -> int:
+    """The raw CUDA stream handle: `stream` itself, or the current stream of `device`."""
     if stream is None:
-        return torch.cuda.current_stream().cuda_stream
+        return torch.cuda.current_stream(device).cuda_stream
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _same_device(device, **tensors) -> None:
+    """The library picks its per-device state (workspace, scratch, attributes) by the
+    current device, so every tensor of a call must live on the device the call runs on."""
+    for name, t in tensors.items():
+        if t is not None and t.device != device:
+            raise ValueError(f"{name} is on {t.device}, expected {device}")
 
 
 def _ptr(t: torch.Tensor, dtypes, name: str) -> int:
@@ -148,10 +157,12 @@ def moe_route_union(topk_idx: torch.Tensor, E: int, unique=None, offsets=None, p
                                                                     device=dev)
     num_unique = num_unique if num_unique is not None else torch.zeros(1, dtype=torch.int32,
                                                                        device=dev)
-    st = _lib.moe_route_union(_ptr(topk_idx, _I32, "topk_idx"), T, k, E,
-                              _ptr(unique, _I32, "unique"), _ptr(offsets, _I32, "offsets"),
-                              _ptr(pair_list, _I32, "pair_list"),
-                              _ptr(num_unique, _I32, "num_unique"), _stream(stream))
+    _same_device(dev, unique=unique, offsets=offsets, pair_list=pair_list, num_unique=num_unique)
+    with torch.cuda.device(dev):
+        st = _lib.moe_route_union(_ptr(topk_idx, _I32, "topk_idx"), T, k, E,
+                                  _ptr(unique, _I32, "unique"), _ptr(offsets, _I32, "offsets"),
+                                  _ptr(pair_list, _I32, "pair_list"),
+                                  _ptr(num_unique, _I32, "num_unique"), _stream(stream, dev))
     _check(st, "moe_route_union", check)
     return unique, offsets, pair_list, num_unique
 
@@ -168,9 +179,11 @@ def moe_router_topk(logits: torch.Tensor, k: int, renormalize: bool = True, topk
                                                                  device=dev)
     topk_w = topk_w if topk_w is not None else torch.empty((T, k), dtype=torch.float32,
                                                            device=dev)
-    st = _lib.moe_router_topk(_ptr(logits, _F32, "logits"), T, E, k, 1 if renormalize else 0,
-                              _ptr(topk_idx, _I32, "topk_idx"), _ptr(topk_w, _F32, "topk_w"),
-                              _stream(stream))
+    _same_device(dev, topk_idx=topk_idx, topk_w=topk_w)
+    with torch.cuda.device(dev):
+        st = _lib.moe_router_topk(_ptr(logits, _F32, "logits"), T, E, k, 1 if renormalize else 0,
+                                  _ptr(topk_idx, _I32, "topk_idx"), _ptr(topk_w, _F32, "topk_w"),
+                                  _stream(stream, dev))
     _check(st, "moe_router_topk", check)
     return topk_idx, topk_w
 
@@ -209,6 +222,9 @@ def _fwd_args(x, topk_idx, topk_w, bank: QuantBank, out):
         out = torch.empty((T, hidden), dtype=torch.bfloat16, device=x.device)
     if tuple(out.shape) != (T, hidden):
         raise ValueError("out has the wrong shape")
+    _same_device(x.device, topk_idx=topk_idx, topk_w=topk_w, out=out, wg_q=bank.wg_q,
+                 wg_s=bank.wg_s, wg_b=bank.wg_b, wu_q=bank.wu_q, wu_s=bank.wu_s, wu_b=bank.wu_b,
+                 wd_q=bank.wd_q, wd_s=bank.wd_s, wd_b=bank.wd_b)
     args = [_ptr(x, _BF16, "x"), _ptr(topk_idx, _I32, "topk_idx"), _ptr(topk_w, _F32, "topk_w"),
             *bank.ptrs()]
     return args, (T, k, bank.E, hidden, bank.inter), out
@@ -218,7 +234,9 @@ def moe_switchglu_forward(x, topk_idx, topk_w, bank: QuantBank, out=None, stream
                           check: bool = True):
     """out [T, hidden] bf16 = union-of-experts SwitchGLU of x [T, hidden] bf16."""
     args, dims, out = _fwd_args(x, topk_idx, topk_w, bank, out)
-    st = _lib.moe_switchglu_forward(*args, *dims, _ptr(out, _BF16, "out"), _stream(stream))
+    with torch.cuda.device(x.device):
+        st = _lib.moe_switchglu_forward(*args, *dims, _ptr(out, _BF16, "out"),
+                                        _stream(stream, x.device))
     _check(st, "moe_switchglu_forward", check)
     return out
 
@@ -226,11 +244,15 @@ def moe_switchglu_forward(x, topk_idx, topk_w, bank: QuantBank, out=None, stream
 def moe_switchglu_forward_ws(x, topk_idx, topk_w, bank: QuantBank, workspace: torch.Tensor,
                              out=None, stream=None, check: bool = True):
     """As moe_switchglu_forward, with a caller-owned uint8 device workspace tensor (see
-    moe_workspace: its first 16 bytes must be zero before the first call)."""
+    moe_workspace).  Its counter region (the first 4 * 1539 bytes) must be zero before the
+    first call; the kernel leaves it zero again, except after a call that ended in
+    MOE_ERR_TIMEOUT, when the caller must clear it before the next call."""
     args, dims, out = _fwd_args(x, topk_idx, topk_w, bank, out)
-    st = _lib.moe_switchglu_forward_ws(*args, *dims, _ptr(out, _BF16, "out"),
-                                       _ptr(workspace, (torch.uint8,), "workspace"),
-                                       workspace.numel(), _stream(stream))
+    _same_device(x.device, workspace=workspace)
+    with torch.cuda.device(x.device):
+        st = _lib.moe_switchglu_forward_ws(*args, *dims, _ptr(out, _BF16, "out"),
+                                           _ptr(workspace, (torch.uint8,), "workspace"),
+                                           workspace.numel(), _stream(stream, x.device))
     _check(st, "moe_switchglu_forward_ws", check)
     return out
 
@@ -241,8 +263,9 @@ def moe_switchglu_forward_static(x, topk_idx, topk_w, bank: QuantBank, out=None,
     inside the call; shapes needing more than MOE_STATIC_SCRATCH_BYTES are rejected with
     MOE_ERR_WORKSPACE; overlapping calls on one device race)."""
     args, dims, out = _fwd_args(x, topk_idx, topk_w, bank, out)
-    st = _lib.moe_switchglu_forward_static(*args, *dims, _ptr(out, _BF16, "out"),
-                                           _stream(stream))
+    with torch.cuda.device(x.device):
+        st = _lib.moe_switchglu_forward_static(*args, *dims, _ptr(out, _BF16, "out"),
+                                               _stream(stream, x.device))
     if check and st == MOE_ERR_WORKSPACE:
         raise MoeError(st, f"moe_switchglu_forward_static [{moe_last_error()}]")
     _check(st, "moe_switchglu_forward_static", check)

@@ -518,7 +518,24 @@ moe_status moe_read_device_status(void* stream) {
     e = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
     if (e != cudaSuccess) return cuda_fail(e);
   }
-  if (word & kErrTimeout) return MOE_ERR_TIMEOUT;
+  if (word & kErrTimeout) {
+    // A call that gave up on a bounded wait may have left its progress counters
+    // non-zero.  The stream is idle now, so clear those of the workspace this
+    // library owns on the current device (moe_switchglu_forward's); a caller-owned
+    // workspace is the caller's to clear, and the static scratch is cleared by
+    // every call of moe_switchglu_forward_static.
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev >= 0 && dev < kMaxDevices) {
+      std::lock_guard<std::mutex> lock(g_mu);
+      if (g_ws[dev].ptr) {
+        e = cudaMemset(g_ws[dev].ptr, 0, 4 * kSyncWords);
+        if (e != cudaSuccess) return cuda_fail(e);
+      }
+    }
+    return MOE_ERR_TIMEOUT;
+  }
   if (word & kErrExpertIndex) return MOE_ERR_DEVICE_INDEX;
   return MOE_OK;
 }

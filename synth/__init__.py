@@ -5,7 +5,9 @@ oracle and the CUDA path consume what it draws.
 
 * Expert banks: ``fill_bank_host`` (C, threaded) and ``fill_bank_device``
   (CUDA) implement one counter-based generator and one quantiser and produce the
-  same bits (see ``synth_host.c`` for the definition).  The 4-bit affine
+  same bits (see ``synth_host.c`` for the definition).  ``fill_bank_mxfp4_host`` /
+  ``fill_bank_mxfp4_device`` encode the same draws as mxfp4 (e2m1 codes, one e8m0
+  scale per 32 columns).  The 4-bit affine
   group-64 format with bf16 scale and bias is the one of the ``moe_bench.py``
   script in "gather_qmm at M=1 streams 4-bit expert weights at ~half the
   bandwidth of M=4" (mlx issue 4509).
@@ -68,6 +70,11 @@ def _host_lib():
                                         ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_uint64, ctypes.c_uint64, ctypes.c_void_p,
                                         ctypes.c_int, ctypes.c_int]
+        lib.synth_fill_bank_mxfp4.restype = ctypes.c_int
+        lib.synth_fill_bank_mxfp4.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_int, ctypes.c_uint64,
+                                              ctypes.c_uint64, ctypes.c_void_p, ctypes.c_int,
+                                              ctypes.c_int]
         lib.synth_draw_row.restype = ctypes.c_int
         lib.synth_draw_row.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                        ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int,
@@ -86,6 +93,10 @@ def _dev_lib():
                                             ctypes.c_int, ctypes.c_int, ctypes.c_uint64,
                                             ctypes.c_uint64, ctypes.c_void_p, ctypes.c_int,
                                             ctypes.c_void_p]
+        lib.synth_dev_fill_bank_mxfp4.restype = ctypes.c_int
+        lib.synth_dev_fill_bank_mxfp4.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                                  ctypes.c_int, ctypes.c_uint64, ctypes.c_uint64,
+                                                  ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
         _dev = lib
     return _dev
 
@@ -121,6 +132,46 @@ def fill_bank_host(E: int, rows: int, cols: int, seed: int, matrix_id: int,
         if rc != 0:
             raise ValueError("synth_fill_bank rejected its arguments")
     return q, s, b
+
+
+def alloc_bank_mxfp4(E: int, rows: int, cols: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Zeroed host mxfp4 bank arrays q [E,rows,cols/8] u32 (e2m1 codes), e8 [E,rows,cols/32]
+    u8 (e8m0 scales)."""
+    return np.zeros((E, rows, cols // 8), np.uint32), np.zeros((E, rows, cols // 32), np.uint8)
+
+
+def fill_bank_mxfp4_host(E: int, rows: int, cols: int, seed: int, matrix_id: int,
+                         experts: Optional[Sequence[int]] = None,
+                         n_threads: Optional[int] = None, out=None):
+    """Draw experts `experts` (default: all) of one matrix of an mxfp4 bank on the host
+    (the same normal draws as fill_bank_host, encoded as e2m1 codes with one e8m0 scale
+    per 32 columns; see synth_host.c).  Returns (q, e8)."""
+    if cols % 32:
+        raise ValueError("cols must be a multiple of 32")
+    q, e8 = out if out is not None else alloc_bank_mxfp4(E, rows, cols)
+    ex = np.arange(E, dtype=np.int32) if experts is None else np.asarray(
+        sorted(set(int(e) for e in experts)), dtype=np.int32)
+    if ex.size:
+        rc = _host_lib().synth_fill_bank_mxfp4(q.ctypes.data, e8.ctypes.data, E, rows, cols, seed,
+                                               matrix_id, ex.ctypes.data, int(ex.size),
+                                               n_threads or default_threads())
+        if rc != 0:
+            raise ValueError("synth_fill_bank_mxfp4 rejected its arguments")
+    return q, e8
+
+
+def fill_bank_mxfp4_device(q, e8, rows: int, cols: int, seed: int, matrix_id: int,
+                           experts=None, n_experts: Optional[int] = None,
+                           stream: int = 0) -> None:
+    """Draw an mxfp4 bank into device tensors q (int32 [E,rows,cols/8]) and e8 (uint8
+    [E,rows,cols/32]), bit-identical to fill_bank_mxfp4_host."""
+    n = int(experts.numel()) if experts is not None else int(n_experts or q.shape[0])
+    rc = _dev_lib().synth_dev_fill_bank_mxfp4(q.data_ptr(), e8.data_ptr(), rows, cols, seed,
+                                              matrix_id,
+                                              experts.data_ptr() if experts is not None else None,
+                                              n, stream)
+    if rc != 0:
+        raise RuntimeError(f"synth_dev_fill_bank_mxfp4 failed with code {rc}")
 
 
 def draw_row(E: int, rows: int, cols: int, seed: int, matrix_id: int, expert: int,

@@ -87,6 +87,53 @@ __global__ void fill_bank_kernel(uint32_t* __restrict__ q, uint16_t* __restrict_
   }
 }
 
+// mxfp4 encoding, the device twin of synth_group_mx in synth_host.c (e8m0 scale
+// per 32 columns from the group's largest magnitude, e2m1 codes nearest, ties to
+// the even mantissa, saturating at 6).
+__device__ __forceinline__ uint32_t e2m1_code(float v) {
+  const float a = fabsf(v);
+  uint32_t m;
+  if (a <= 0.25f) m = 0;
+  else if (a < 0.75f) m = 1;
+  else if (a <= 1.25f) m = 2;
+  else if (a < 1.75f) m = 3;
+  else if (a <= 2.5f) m = 4;
+  else if (a < 3.5f) m = 5;
+  else if (a <= 5.0f) m = 6;
+  else m = 7;
+  return (v < 0.0f ? 8u : 0u) | m;
+}
+
+__global__ void fill_bank_mx_kernel(uint32_t* __restrict__ q, uint8_t* __restrict__ e8,
+                                    int rows, int cols, uint64_t key,
+                                    const int32_t* __restrict__ experts, int n_experts) {
+  const int gpr = cols / 32;
+  const uint64_t per_expert = (uint64_t)rows * gpr;
+  const uint64_t total = per_expert * (uint64_t)n_experts;
+  for (uint64_t gid = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; gid < total;
+       gid += (uint64_t)gridDim.x * blockDim.x) {
+    const int ei = (int)(gid / per_expert);
+    const uint64_t rem = gid % per_expert;
+    const int r = (int)(rem / gpr), g = (int)(rem % gpr);
+    const int e = experts ? experts[ei] : ei;
+    const uint64_t elem0 = ((uint64_t)e * rows + r) * cols + (uint64_t)g * 32;
+    float amax = 0.f;
+    for (int c = 0; c < 32; ++c) amax = fmaxf(amax, fabsf(normal_draw(key, elem0 + c)));
+    const int ex = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127 - 2 : 0;
+    const float inv = __uint_as_float((uint32_t)(127 - ex) << 23);
+    uint32_t* qrow = q + ((uint64_t)e * rows + r) * (cols / 8) + (uint64_t)g * 4;
+    for (int wd = 0; wd < 4; ++wd) {
+      uint32_t word = 0;
+      for (int j = 0; j < 8; ++j) {
+        const float w = normal_draw(key, elem0 + wd * 8 + j);
+        word |= (amax > 0.f ? e2m1_code(__fmul_rn(w, inv)) : 0u) << (4 * j);
+      }
+      qrow[wd] = word;
+    }
+    e8[((uint64_t)e * rows + r) * gpr + g] = (uint8_t)(127 + ex);
+  }
+}
+
 }  // namespace
 
 // Host-side copy of the stream key derivation (plain integer arithmetic).
@@ -112,6 +159,23 @@ int synth_dev_fill_bank(uint32_t* q, uint16_t* s, uint16_t* b, int rows, int col
   if (blocks > 148ull * 64) blocks = 148ull * 64;
   fill_bank_kernel<<<(unsigned)blocks, threads, 0, (cudaStream_t)stream>>>(
       q, s, b, rows, cols, key, experts, n_experts);
+  return (int)cudaGetLastError();
+}
+
+// The mxfp4 twin of synth_dev_fill_bank: q [E, rows, cols/8] e2m1 codes and
+// e8 [E, rows, cols/32] e8m0 scales (cols a multiple of 32), bit-identical to
+// synth_fill_bank_mxfp4 on the host.
+int synth_dev_fill_bank_mxfp4(uint32_t* q, uint8_t* e8, int rows, int cols, uint64_t seed,
+                              uint64_t matrix_id, const int32_t* experts, int n_experts,
+                              void* stream) {
+  if (!q || !e8 || rows <= 0 || cols <= 0 || cols % 32 || n_experts <= 0) return -1;
+  const uint64_t key = host_mix64(seed + (matrix_id + 1) * 0x9E3779B97F4A7C15ULL);
+  const uint64_t total = (uint64_t)rows * (cols / 32) * (uint64_t)n_experts;
+  const int threads = 256;
+  uint64_t blocks = (total + threads - 1) / threads;
+  if (blocks > 148ull * 64) blocks = 148ull * 64;
+  fill_bank_mx_kernel<<<(unsigned)blocks, threads, 0, (cudaStream_t)stream>>>(
+      q, e8, rows, cols, key, experts, n_experts);
   return (int)cudaGetLastError();
 }
 

@@ -176,6 +176,115 @@ int synth_fill_bank(uint32_t* q, uint16_t* s, uint16_t* b, int E, int rows, int 
     return 0;
 }
 
+/*
+ * mxfp4 encoding (GLM-5.2's routed banks are "mxfp4 gs32" in "Small-L fused
+ * expert gather for fine-grained MoE decode", mlx discussion 3801, the post
+ * that isolates one layer's routed bank; the pages define it no further, so
+ * the OCP microscaling format is taken): per group of 32 consecutive input
+ * columns one e8m0 scale byte X = 127 + floor(log2(max |w|)) - 2 (the largest
+ * e2m1 exponent is 2), and per element the e2m1 code nearest to w * 2^-(X-127),
+ * ties to the even mantissa, magnitudes above 6 saturating to 6.  An all-zero
+ * group gets X = 127 and zero codes.  e2m1 code: sign bit 3, magnitude index
+ * bits 2..0 for 0, 0.5, 1, 1.5, 2, 3, 4, 6.  Codes are packed like the affine
+ * ones.  Every step is exact in fp32 (power-of-two scaling, comparisons), so the
+ * device twin gives the same bits.
+ */
+static inline uint32_t synth_e2m1_code(float v) {
+    const float a = fabsf(v);
+    uint32_t m;
+    if (a <= 0.25f) m = 0;
+    else if (a < 0.75f) m = 1;
+    else if (a <= 1.25f) m = 2;
+    else if (a < 1.75f) m = 3;
+    else if (a <= 2.5f) m = 4;
+    else if (a < 3.5f) m = 5;
+    else if (a <= 5.0f) m = 6;
+    else m = 7;
+    return (v < 0.0f ? 8u : 0u) | m;
+}
+
+static void synth_group_mx(uint64_t key, uint64_t elem0, uint32_t* q4, uint8_t* e8) {
+    float w[32];
+    float amax = 0.0f;
+    for (int c = 0; c < 32; ++c) {
+        w[c] = synth_normal(key, elem0 + (uint64_t)c);
+        if (fabsf(w[c]) > amax) amax = fabsf(w[c]);
+    }
+    int e = 0;
+    if (amax > 0.0f) {
+        uint32_t u;
+        memcpy(&u, &amax, 4);
+        e = (int)((u >> 23) & 0xFF) - 127 - 2;  /* floor(log2 amax) - 2; amax is normal */
+    }
+    /* 2^-e as an fp32 bit pattern (|e| < 30 for these draws) */
+    const uint32_t inv_bits = (uint32_t)(127 - e) << 23;
+    float inv;
+    memcpy(&inv, &inv_bits, 4);
+    for (int wd = 0; wd < 4; ++wd) {
+        uint32_t word = 0;
+        for (int j = 0; j < 8; ++j)
+            word |= (amax > 0.0f ? synth_e2m1_code(w[wd * 8 + j] * inv) : 0u) << (4 * j);
+        q4[wd] = word;
+    }
+    *e8 = (uint8_t)(127 + e);
+}
+
+typedef struct {
+    uint32_t* q;
+    uint8_t* e8;
+    int rows, cols;
+    uint64_t key;
+    const int32_t* experts;
+    int n_experts;
+    int next;
+    pthread_mutex_t mu;
+} synth_job_mx;
+
+static void* synth_worker_mx(void* arg) {
+    synth_job_mx* J = (synth_job_mx*)arg;
+    for (;;) {
+        pthread_mutex_lock(&J->mu);
+        int i = J->next++;
+        pthread_mutex_unlock(&J->mu);
+        if (i >= J->n_experts) break;
+        const int e = J->experts[i], rows = J->rows, cols = J->cols, gpr = cols / 32;
+        uint32_t* q = J->q + (size_t)e * rows * (cols / 8);
+        uint8_t* e8 = J->e8 + (size_t)e * rows * gpr;
+        for (int r = 0; r < rows; ++r)
+            for (int g = 0; g < gpr; ++g)
+                synth_group_mx(J->key, ((uint64_t)e * rows + r) * cols + (uint64_t)g * 32,
+                               q + (size_t)r * (cols / 8) + g * 4, e8 + (size_t)r * gpr + g);
+    }
+    return 0;
+}
+
+/*
+ * Fill experts `experts[0..n_experts)` of an mxfp4 bank laid out as
+ *   q [E, rows, cols/8] uint32 (e2m1 codes), e8 [E, rows, cols/32] uint8,
+ * from the same normal draws as synth_fill_bank (stream (seed, matrix_id)).
+ * cols must be a multiple of 32.  Returns 0, or -1 on bad arguments.
+ */
+int synth_fill_bank_mxfp4(uint32_t* q, uint8_t* e8, int E, int rows, int cols, uint64_t seed,
+                          uint64_t matrix_id, const int32_t* experts, int n_experts,
+                          int n_threads) {
+    if (!q || !e8 || E <= 0 || rows <= 0 || cols <= 0 || cols % 32) return -1;
+    for (int i = 0; i < n_experts; ++i)
+        if (experts[i] < 0 || experts[i] >= E) return -1;
+    synth_job_mx J;
+    J.q = q; J.e8 = e8; J.rows = rows; J.cols = cols;
+    J.key = synth_stream_key(seed, matrix_id);
+    J.experts = experts; J.n_experts = n_experts; J.next = 0;
+    pthread_mutex_init(&J.mu, 0);
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > 256) n_threads = 256;
+    if (n_threads > n_experts) n_threads = n_experts > 0 ? n_experts : 1;
+    pthread_t th[256];
+    for (int i = 0; i < n_threads; ++i) pthread_create(&th[i], 0, synth_worker_mx, &J);
+    for (int i = 0; i < n_threads; ++i) pthread_join(th[i], 0);
+    pthread_mutex_destroy(&J.mu);
+    return 0;
+}
+
 /* Raw fp32 draws of one row (before quantisation); used by the quantiser's
  * round-trip test. */
 int synth_draw_row(float* out, int E, int rows, int cols, uint64_t seed, uint64_t matrix_id,

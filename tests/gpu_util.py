@@ -54,3 +54,28 @@ def assert_parity(out: np.ndarray, ref: np.ndarray, what: str = ""):
     assert rel <= REL_L2_TOL and mxn <= MAX_ABS_TOL, (
         f"{what}: rel-L2 {rel:.3e} (tol {REL_L2_TOL}), max-abs/rms {mxn:.3e} (tol {MAX_ABS_TOL}),"
         f" raw max-abs {mx:.3e}")
+
+
+def dev_bank_drawn(E: int, H: int, I: int, seed: int, device="cuda") -> qeg.QuantBank:
+    """A bank of E experts drawn on the device by the generator's CUDA twin, bit-identical
+    to tests.layers.draw_bank(E, H, I, seed) (checked by a GPU test), so that the oracle
+    can draw on the host only the experts a check needs."""
+    import synth
+
+    def mat(rows, cols, mid):
+        q = torch.empty((E, rows, cols // 8), dtype=torch.int32, device=device)
+        s = torch.empty((E, rows, cols // 64), dtype=torch.int16, device=device)
+        b = torch.empty_like(s)
+        synth.fill_bank_device(q, s, b, rows, cols, seed, mid)
+        return q, s.view(torch.bfloat16), b.view(torch.bfloat16)
+
+    bank = qeg.QuantBank(*mat(I, H, synth.MATRIX_GATE), *mat(I, H, synth.MATRIX_UP),
+                         *mat(H, I, synth.MATRIX_DOWN))
+    torch.cuda.synchronize()
+    return bank
+
+
+def bf16_tensor(bits: np.ndarray, device="cuda") -> torch.Tensor:
+    """Device bf16 tensor from raw bf16 bit patterns (uint16)."""
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device) \
+        .view(torch.bfloat16)

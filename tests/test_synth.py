@@ -106,3 +106,50 @@ def test_x_bf16_rounding():
     x = synth.x_bf16(3, 64, 2)
     f = synth.bf16_bits_to_f32(x)
     assert x.dtype == np.uint16 and np.isfinite(f).all() and abs(f.std() - 1) < 0.3
+
+
+def test_mxfp4_encoder_nearest_code_and_block_scale():
+    """The mxfp4 bank generator: per group of 32 the e8m0 scale is 127 + floor(log2 max|w|)
+    - 2, and every code is the e2m1 value nearest to w / scale (decoded by ml_dtypes, a
+    library routine), ties to the even mantissa, saturating at +-6."""
+    import ml_dtypes
+    E, rows, cols, seed = 3, 6, 256, 41
+    q, e8 = synth.fill_bank_mxfp4_host(E, rows, cols, seed, synth.MATRIX_DOWN)
+    grid = np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    for e in range(E):
+        for r in range(rows):
+            w = synth.draw_row(E, rows, cols, seed, synth.MATRIX_DOWN, e, r).astype(np.float64)
+            codes = ((q[e, r][:, None] >> (4 * np.arange(8, dtype=np.uint32))) & 15).ravel()
+            for g in range(cols // 32):
+                wg = w[32 * g:32 * g + 32]
+                amax = np.abs(wg).max()
+                ex = int(np.floor(np.log2(amax))) - 2
+                assert int(e8[e, r, g]) == 127 + ex
+                v = wg / 2.0 ** ex
+                cg = codes[32 * g:32 * g + 32]
+                got = grid[cg]
+                err = np.abs(got - np.clip(v, -6, 6))
+                best = np.abs(grid[None, :] - np.clip(v, -6, 6)[:, None]).min(axis=1)
+                assert np.all(err <= best + 1e-12)   # nearest representable value
+                assert np.all(np.sign(got) * np.sign(v) >= 0)
+
+
+def test_mxfp4_encoder_ties_and_saturation():
+    """Ties go to the even mantissa; a group's largest magnitude maps into [4, 8) and
+    values above 6 saturate (checked through the encoder on crafted draws is not possible,
+    so the decision table is checked against ml_dtypes' own rounding of the same values)."""
+    import ml_dtypes
+    vals = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.24, 0.26, 5.1, 6.0], np.float32)
+    want = vals.astype(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    # the generator's decision thresholds, restated: the e2m1 value it picks
+    table = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    th = [(0.25, True), (0.75, False), (1.25, True), (1.75, False), (2.5, True), (3.5, False),
+          (5.0, True)]
+
+    def pick(a):
+        m = 0
+        for i, (t, incl) in enumerate(th):
+            if a > t or (a == t and not incl):
+                m = i + 1
+        return table[m]
+    assert np.array_equal([pick(float(a)) for a in vals], want)
