@@ -92,7 +92,7 @@ bool shape_supported(int T, int k, int E, int hidden, int inter) {
 struct WsLayout {
   size_t barrier, num_unique, unique, offsets, pair_list, h, y;  // barrier = counters
   size_t xg, hq;                         // fused kernel: x and h rows in fixed point
-  size_t padded, xs, hs, xp, hp, pcap;   // grouped path: packed activations and sums
+  size_t padded, xp, hp, pcap;           // grouped path: padded offsets, packed activations
   size_t total;
 };
 
@@ -131,11 +131,9 @@ WsLayout ws_layout(int T, int k, int E, int hidden, int inter) {
   // grouped path: every expert's pairs padded to 16 rows
   w.pcap = align_up(P + 15 * m, 16);
   w.padded = tail;
-  w.xs = align_up(w.padded + 4 * (m + 1), 256);
-  w.hs = align_up(w.xs + 4 * (size_t)(hidden / kGK) * w.pcap, 256);
-  w.xp = align_up(w.hs + 4 * (size_t)(inter / kGK) * w.pcap, 256);
-  w.hp = align_up(w.xp + 2 * (size_t)hidden * w.pcap, 256);
-  const size_t total2 = align_up(w.hp + 2 * (size_t)inter * w.pcap, 256);
+  w.xp = align_up(w.padded + 4 * (m + 1), 1024);
+  w.hp = align_up(w.xp + 2 * (size_t)hidden * w.pcap, 1024);
+  const size_t total2 = align_up(w.hp + 2 * (size_t)inter * w.pcap, 1024);
   w.total = select_path(T, k, E, hidden, inter) == 2 ? total2 : total1;
   return w;
 }
@@ -216,8 +214,6 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   int* plist = reinterpret_cast<int*>(ws + wl.pair_list);
   float* y = reinterpret_cast<float*>(ws + wl.y);
   int* padded = reinterpret_cast<int*>(ws + wl.padded);
-  float* xs = reinterpret_cast<float*>(ws + wl.xs);
-  float* hs = reinterpret_cast<float*>(ws + wl.hs);
   uint16_t* xp = reinterpret_cast<uint16_t*>(ws + wl.xp);
   uint16_t* hp = reinterpret_cast<uint16_t*>(ws + wl.hp);
   const int pcap = static_cast<int>(wl.pcap);
@@ -229,7 +225,7 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   const int width = P > 40 * m ? 96 : (P <= 20 * m ? 32 : 64);
   const unsigned gsmem = width == 96 ? GCfg<96>::kSmem : width == 32 ? GCfg<32>::kSmem : GCfg<64>::kSmem;
   const int ki = width == 96 ? 5 : width == 32 ? 7 : 2;  // dyn_smem index of gate+up
-  const int grid = width == 32 ? 2 * d.sms : d.sms;
+  const int grid = d.sms;
   if (usmem > (size_t)d.dyn_smem[1] || csmem > (size_t)d.dyn_smem[4] ||
       gsmem > (unsigned)d.dyn_smem[ki] || gsmem > (unsigned)d.dyn_smem[ki + 1]) {
     *why = MOE_ERR_UNSUPPORTED;
@@ -238,7 +234,7 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   route_union_kernel<<<1, 32 * kUnionWarps, usmem, st>>>(idx, P, E, uniq, offs, plist, nu,
                                                          padded);
   grouped_pack_x_kernel<<<m < 4 * d.sms ? m : 4 * d.sms, 256, 0, st>>>(x, plist, offs, padded,
-                                                                         nu, k, H, pcap, xp, xs);
+                                                                         nu, k, H, pcap, xp);
   GroupedArgs g{};
   g.unique = uniq;
   g.offsets = offs;
@@ -247,11 +243,9 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   g.pcap = pcap;
   g.H = H;
   g.hp = hp;
-  g.hs = hs;
   g.y = y;
   // gate + up: 128 rows of Wg and the same 128 rows of Wu per tile, K = H, packed x
   g.bp = xp;
-  g.bs = xs;
   g.q[0] = gq;
   g.s[0] = gs;
   g.b[0] = gb;
@@ -270,7 +264,6 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
     grouped_gemm_kernel<0, 64><<<grid, kGThreads, gsmem, st>>>(g);
   // down: 256 rows of Wd per tile (two 128-row matrices), K = I, packed h
   g.bp = hp;
-  g.bs = hs;
   g.q[0] = g.q[1] = dq;
   g.s[0] = g.s[1] = ds;
   g.b[0] = g.b[1] = db;

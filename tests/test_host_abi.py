@@ -83,14 +83,14 @@ def test_workspace_size_and_layout():
 
 def test_workspace_follows_the_path():
     """The grouped path's workspace also holds the packed activations: x and h rows
-    for every pair position padded to 16 per expert, bf16, and their fp32 group
-    sums; the persistent kernel's does not grow with them."""
+    for every pair position padded to 16 per expert, bf16; the persistent kernel's
+    does not grow with them."""
     E, H, I = 256, 4096, 2048
     for T in (512, 2048):
         P = T * 8
         assert qeg.moe_select_path(T, 8, E, H, I) == 2
         pcap = P + 15 * min(E, P)
-        packed = 2 * (H + I) * pcap + 4 * (H + I) // 64 * pcap
+        packed = 2 * (H + I) * pcap
         lay = qeg.moe_workspace_layout(T, 8, E, H, I)
         assert lay["total"] >= lay["y"] + 4 * P * H + packed
     # the small-window path stays within the 4 MiB no-allocation scratch at T=16
