@@ -175,6 +175,38 @@ moe_status moe_switchglu_forward_static(const uint16_t* x, const int32_t* topk_i
                                         void* stream);
 
 /*
+ * mxfp4 banks ("Small-L fused expert gather for fine-grained MoE decode", mlx
+ * discussion 3801: GLM-5.2's routed banks are "mxfp4 gs32"; the pages define the
+ * format no further, so the OCP microscaling reading is taken).  Per matrix:
+ *   q  uint32 [E, rows, cols/8]   e2m1 codes, packed like the affine codes
+ *                                 (element c = nibble c%8 of word c/8, LSB
+ *                                 first); code bit 3 = sign, bits 2..0 index
+ *                                 0, 0.5, 1, 1.5, 2, 3, 4, 6
+ *   e  uint8  [E, rows, cols/32]  e8m0 scale bytes, 2^(e - 127) (255 = NaN)
+ *   w  = e2m1(q) * 2^(e - 127), one scale per 32 consecutive columns.
+ * Gate and up: rows = inter, cols = hidden; down: rows = hidden, cols = inter.
+ * Everything else (x, topk_idx, topk_w, out, workspace rules, errors, capture)
+ * is as for moe_switchglu_forward_ws / moe_switchglu_forward, with the workspace
+ * sized by moe_workspace_size_mxfp4.  Windows the persistent small-window kernel
+ * cannot hold (moe_select_path_mxfp4 returns 0) give MOE_ERR_UNSUPPORTED.
+ */
+size_t moe_workspace_size_mxfp4(int T, int k, int E, int hidden, int inter);
+int moe_select_path_mxfp4(int T, int k, int E, int hidden, int inter);
+moe_status moe_switchglu_forward_mxfp4_ws(const uint16_t* x, const int32_t* topk_idx,
+                                          const float* topk_w, const uint32_t* wg_q,
+                                          const uint8_t* wg_e, const uint32_t* wu_q,
+                                          const uint8_t* wu_e, const uint32_t* wd_q,
+                                          const uint8_t* wd_e, int T, int k, int E, int hidden,
+                                          int inter, uint16_t* out, void* workspace,
+                                          size_t workspace_bytes, void* stream);
+moe_status moe_switchglu_forward_mxfp4(const uint16_t* x, const int32_t* topk_idx,
+                                       const float* topk_w, const uint32_t* wg_q,
+                                       const uint8_t* wg_e, const uint32_t* wu_q,
+                                       const uint8_t* wu_e, const uint32_t* wd_q,
+                                       const uint8_t* wd_e, int T, int k, int E, int hidden,
+                                       int inter, uint16_t* out, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word that the
  * kernels set instead of trapping: MOE_ERR_DEVICE_INDEX if an expert id was
  * out of range, MOE_ERR_TIMEOUT if a bounded wait ran out, else MOE_OK (or

@@ -20,8 +20,8 @@ from ._build import SO, build as build_library, needs_build
 __all__ = ["MoeError", "MOE_OK", "moe_status_str", "moe_workspace_size", "moe_workspace_layout",
            "moe_select_path", "moe_route_union", "moe_switchglu_forward",
            "moe_switchglu_forward_ws", "moe_switchglu_forward_static", "moe_read_device_status", "moe_last_error", "moe_workspace",
-           "library_path",
-           "QuantBank"]
+           "library_path", "QuantBank", "MxBank", "moe_switchglu_forward_mxfp4",
+           "moe_switchglu_forward_mxfp4_ws", "moe_workspace_size_mxfp4", "moe_select_path_mxfp4"]
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = 1
@@ -64,6 +64,14 @@ def _load():
     lib.moe_switchglu_forward_ws.argtypes = [vp] * 12 + [ci] * 5 + [vp, vp, sz, vp]
     lib.moe_switchglu_forward_static.restype = ci
     lib.moe_switchglu_forward_static.argtypes = [vp] * 12 + [ci] * 5 + [vp, vp]
+    lib.moe_workspace_size_mxfp4.restype = sz
+    lib.moe_workspace_size_mxfp4.argtypes = [ci] * 5
+    lib.moe_select_path_mxfp4.restype = ci
+    lib.moe_select_path_mxfp4.argtypes = [ci] * 5
+    lib.moe_switchglu_forward_mxfp4.restype = ci
+    lib.moe_switchglu_forward_mxfp4.argtypes = [vp] * 9 + [ci] * 5 + [vp, vp]
+    lib.moe_switchglu_forward_mxfp4_ws.restype = ci
+    lib.moe_switchglu_forward_mxfp4_ws.argtypes = [vp] * 9 + [ci] * 5 + [vp, vp, sz, vp]
     lib.moe_read_device_status.restype = ci
     lib.moe_read_device_status.argtypes = [vp]
     return lib
@@ -119,6 +127,7 @@ _BF16 = (torch.bfloat16, torch.int16, torch.uint16)
 _Q = (torch.int32, torch.uint32)
 _I32 = (torch.int32,)
 _F32 = (torch.float32,)
+_U8 = (torch.uint8,)
 
 
 def moe_workspace_size(T: int, k: int, E: int, hidden: int, inter: int) -> int:
@@ -273,6 +282,82 @@ def moe_switchglu_forward_static(x, topk_idx, topk_w, bank: QuantBank, out=None,
 
 
 MOE_STATIC_SCRATCH_BYTES = 4 << 20
+
+
+class MxBank:
+    """Device tensors of one layer's mxfp4 bank: gate/up q [E, inter, hidden/8] (int32, e2m1
+    codes), e [E, inter, hidden/32] (uint8, e8m0 scales); down q [E, hidden, inter/8],
+    e [E, hidden, inter/32]."""
+
+    def __init__(self, wg_q, wg_e, wu_q, wu_e, wd_q, wd_e):
+        self.wg_q, self.wg_e, self.wu_q, self.wu_e, self.wd_q, self.wd_e = (
+            wg_q, wg_e, wu_q, wu_e, wd_q, wd_e)
+        self.E, self.inter, hw = wg_q.shape
+        self.hidden = hw * 8
+        for name, t, shape in (("wg_e", wg_e, (self.E, self.inter, self.hidden // 32)),
+                               ("wu_q", wu_q, wg_q.shape),
+                               ("wu_e", wu_e, (self.E, self.inter, self.hidden // 32)),
+                               ("wd_q", wd_q, (self.E, self.hidden, self.inter // 8)),
+                               ("wd_e", wd_e, (self.E, self.hidden, self.inter // 32))):
+            if tuple(t.shape) != tuple(shape):
+                raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+    def tensors(self):
+        return dict(wg_q=self.wg_q, wg_e=self.wg_e, wu_q=self.wu_q, wu_e=self.wu_e,
+                    wd_q=self.wd_q, wd_e=self.wd_e)
+
+    def ptrs(self):
+        return [_ptr(self.wg_q, _Q, "wg_q"), _ptr(self.wg_e, _U8, "wg_e"),
+                _ptr(self.wu_q, _Q, "wu_q"), _ptr(self.wu_e, _U8, "wu_e"),
+                _ptr(self.wd_q, _Q, "wd_q"), _ptr(self.wd_e, _U8, "wd_e")]
+
+
+def moe_workspace_size_mxfp4(T: int, k: int, E: int, hidden: int, inter: int) -> int:
+    return int(_lib.moe_workspace_size_mxfp4(T, k, E, hidden, inter))
+
+
+def moe_select_path_mxfp4(T: int, k: int, E: int, hidden: int, inter: int) -> int:
+    return int(_lib.moe_select_path_mxfp4(T, k, E, hidden, inter))
+
+
+def _mx_args(x, topk_idx, topk_w, bank: MxBank, out):
+    T, hidden = x.shape
+    k = topk_idx.shape[1]
+    if hidden != bank.hidden or tuple(topk_idx.shape) != (T, k) or tuple(topk_w.shape) != (T, k):
+        raise ValueError("x / topk_idx / topk_w shapes do not match the bank")
+    if out is None:
+        out = torch.empty((T, hidden), dtype=torch.bfloat16, device=x.device)
+    if tuple(out.shape) != (T, hidden):
+        raise ValueError("out has the wrong shape")
+    _same_device(x.device, topk_idx=topk_idx, topk_w=topk_w, out=out, **bank.tensors())
+    args = [_ptr(x, _BF16, "x"), _ptr(topk_idx, _I32, "topk_idx"), _ptr(topk_w, _F32, "topk_w"),
+            *bank.ptrs()]
+    return args, (T, k, bank.E, hidden, bank.inter), out
+
+
+def moe_switchglu_forward_mxfp4(x, topk_idx, topk_w, bank: MxBank, out=None, stream=None,
+                                check: bool = True):
+    """out [T, hidden] bf16 = union-of-experts SwitchGLU of x on an mxfp4 bank."""
+    args, dims, out = _mx_args(x, topk_idx, topk_w, bank, out)
+    with torch.cuda.device(x.device):
+        st = _lib.moe_switchglu_forward_mxfp4(*args, *dims, _ptr(out, _BF16, "out"),
+                                              _stream(stream, x.device))
+    _check(st, "moe_switchglu_forward_mxfp4", check)
+    return out
+
+
+def moe_switchglu_forward_mxfp4_ws(x, topk_idx, topk_w, bank: MxBank, workspace: torch.Tensor,
+                                   out=None, stream=None, check: bool = True):
+    """As moe_switchglu_forward_mxfp4 with a caller-owned zeroed uint8 workspace of
+    moe_workspace_size_mxfp4 bytes (same counter-region rules as moe_switchglu_forward_ws)."""
+    args, dims, out = _mx_args(x, topk_idx, topk_w, bank, out)
+    _same_device(x.device, workspace=workspace)
+    with torch.cuda.device(x.device):
+        st = _lib.moe_switchglu_forward_mxfp4_ws(*args, *dims, _ptr(out, _BF16, "out"),
+                                                 _ptr(workspace, (torch.uint8,), "workspace"),
+                                                 workspace.numel(), _stream(stream, x.device))
+    _check(st, "moe_switchglu_forward_mxfp4_ws", check)
+    return out
 
 
 def moe_read_device_status(stream=None) -> int:

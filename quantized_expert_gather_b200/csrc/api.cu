@@ -23,9 +23,10 @@ struct DeviceInfo {
   bool ready = false;
   int sms = 0;
   int smem_optin = 0;
-  // dynamic shared memory limit: layer, route_union, grouped gate+up and down (chunks of
-  // 64 pairs), combine, grouped gate+up and down (chunks of 96, then of 32 pairs)
-  int dyn_smem[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+  // dynamic shared memory limit: layer (affine), route_union, grouped gate+up and down
+  // (chunks of 64 pairs), combine, grouped gate+up and down (chunks of 96, then of 32
+  // pairs), layer (mxfp4)
+  int dyn_smem[10] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
 };
 
 DeviceInfo g_dev[kMaxDevices];
@@ -51,7 +52,7 @@ moe_status device_info(DeviceInfo** out) {
       e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return cuda_fail(e);
     // dynamic + static shared memory may not exceed the opt-in limit
-    const void* kernels[9] = {reinterpret_cast<const void*>(layer_kernel),
+    const void* kernels[10] = {reinterpret_cast<const void*>(layer_kernel<kFmtAffine>),
                               reinterpret_cast<const void*>(route_union_kernel),
                               reinterpret_cast<const void*>(grouped_gemm_kernel<0, 64>),
                               reinterpret_cast<const void*>(grouped_gemm_kernel<1, 64>),
@@ -59,8 +60,9 @@ moe_status device_info(DeviceInfo** out) {
                               reinterpret_cast<const void*>(grouped_gemm_kernel<0, 96>),
                               reinterpret_cast<const void*>(grouped_gemm_kernel<1, 96>),
                               reinterpret_cast<const void*>(grouped_gemm_kernel<0, 32>),
-                              reinterpret_cast<const void*>(grouped_gemm_kernel<1, 32>)};
-    for (int i = 0; i < 9; ++i) {
+                              reinterpret_cast<const void*>(grouped_gemm_kernel<1, 32>),
+                              reinterpret_cast<const void*>(layer_kernel<kFmtMx>)};
+    for (int i = 0; i < 10; ++i) {
       cudaFuncAttributes fa;
       cudaError_t e = cudaFuncGetAttributes(&fa, kernels[i]);
       if (e == cudaSuccess) {
@@ -86,32 +88,36 @@ bool shape_ok(int T, int k, int E, int hidden, int inter) {
 }
 
 bool shape_supported(int T, int k, int E, int hidden, int inter) {
-  return E <= MOE_MAX_EXPERTS && hidden <= 4096 && inter <= MOE_MAX_DIM;
+  return E <= MOE_MAX_EXPERTS && hidden <= MOE_MAX_DIM && inter <= MOE_MAX_DIM;
 }
 
 struct WsLayout {
   size_t barrier, num_unique, unique, offsets, pair_list, h, y;  // barrier = counters
   size_t xg, hq;                         // fused kernel: x and h rows in fixed point
-  size_t padded, xp, hp, pcap;           // grouped path: padded offsets, packed activations
+  size_t padded, xs, hs, xp, hp, pcap;   // grouped path: packed activations and sums
   size_t total;
 };
 
 // 1 = the persistent fused kernel (small windows), 2 = the grouped tensor-core
 // kernels (windows with more pairs; hidden a multiple of 256, inter of 128),
 // 0 = neither.
-int select_path(int T, int k, int E, int hidden, int inter) {
+// mxfp4 banks take the persistent kernel only (0 for larger windows).
+int select_path(int T, int k, int E, int hidden, int inter, int fmt = kFmtAffine) {
   if (!shape_ok(T, k, E, hidden, inter) || !shape_supported(T, k, E, hidden, inter)) return 0;
   if (T * k <= kMaxPairsFused) {
-    LayerGeom g = layer_geom(hidden, inter);
+    LayerGeom g = layer_geom(hidden, inter, fmt);
     if (g.seg >= 1 && fit_stages(g, E, T * k, hidden, inter, kSmemBudget)) return 1;
   }
-  if (hidden % (2 * kGM) == 0 && inter % (2 * kGK) == 0 &&
+  if (fmt == kFmtMx) return 0;
+  // the grouped path: hidden a multiple of 256 (down tiles) and at most 4096, inter a
+  // multiple of 128 (gate/up tiles)
+  if (hidden % (2 * kGM) == 0 && hidden <= 4096 && inter % (2 * kGK) == 0 &&
       route_union_smem_bytes(E) <= kSmemBudget && sizeof(int) * (size_t)T * k <= kSmemBudget)
     return 2;
   return 0;
 }
 
-WsLayout ws_layout(int T, int k, int E, int hidden, int inter) {
+WsLayout ws_layout(int T, int k, int E, int hidden, int inter, int fmt = kFmtAffine) {
   const size_t P = (size_t)T * k;
   const size_t m = P < (size_t)E ? P : (size_t)E;
   WsLayout w;
@@ -131,13 +137,16 @@ WsLayout ws_layout(int T, int k, int E, int hidden, int inter) {
   // grouped path: every expert's pairs padded to 16 rows
   w.pcap = align_up(P + 15 * m, 16);
   w.padded = tail;
-  w.xp = align_up(w.padded + 4 * (m + 1), 1024);
-  w.hp = align_up(w.xp + 2 * (size_t)hidden * w.pcap, 1024);
-  const size_t total2 = align_up(w.hp + 2 * (size_t)inter * w.pcap, 1024);
-  w.total = select_path(T, k, E, hidden, inter) == 2 ? total2 : total1;
+  w.xs = align_up(w.padded + 4 * (m + 1), 256);
+  w.hs = align_up(w.xs + 4 * (size_t)(hidden / kGK) * w.pcap, 256);
+  w.xp = align_up(w.hs + 4 * (size_t)(inter / kGK) * w.pcap, 256);
+  w.hp = align_up(w.xp + 2 * (size_t)hidden * w.pcap, 256);
+  const size_t total2 = align_up(w.hp + 2 * (size_t)inter * w.pcap, 256);
+  w.total = select_path(T, k, E, hidden, inter, fmt) == 2 ? total2 : total1;
   return w;
 }
 
+template <int F>
 cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
                          const uint32_t* gq, const uint16_t* gs, const uint16_t* gb,
                          const uint32_t* uq, const uint16_t* us, const uint16_t* ub,
@@ -173,9 +182,10 @@ cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
   a.E = E;
   a.H = H;
   a.I = I;
-  a.g = layer_geom(H, I);
+  a.g = layer_geom(H, I, F);
   a.wait_prior = 1;
-  if (a.g.seg < 1 || !fit_stages(a.g, E, T * k, H, I, (size_t)d.dyn_smem[0])) {
+  const int ki = F == kFmtMx ? 9 : 0;  // dyn_smem index of this layer kernel
+  if (a.g.seg < 1 || !fit_stages(a.g, E, T * k, H, I, (size_t)d.dyn_smem[ki])) {
     *why = MOE_ERR_UNSUPPORTED;
     return cudaSuccess;
   }
@@ -194,7 +204,7 @@ cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
   c.stream = st;
   c.attrs = attr;
   c.numAttrs = 2;
-  return cudaLaunchKernelEx(&c, layer_kernel, a);
+  return cudaLaunchKernelEx(&c, layer_kernel<F>, a);
 }
 
 // The grouped path: route-union (with padded offsets), x packing, gate+up, down
@@ -216,6 +226,8 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   int* padded = reinterpret_cast<int*>(ws + wl.padded);
   uint16_t* xp = reinterpret_cast<uint16_t*>(ws + wl.xp);
   uint16_t* hp = reinterpret_cast<uint16_t*>(ws + wl.hp);
+  float* xs = reinterpret_cast<float*>(ws + wl.xs);
+  float* hs = reinterpret_cast<float*>(ws + wl.hs);
   const int pcap = static_cast<int>(wl.pcap);
   const int m = P < E ? P : E;
   const size_t usmem = route_union_smem_bytes(E);
@@ -225,7 +237,7 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   const int width = P > 40 * m ? 96 : (P <= 20 * m ? 32 : 64);
   const unsigned gsmem = width == 96 ? GCfg<96>::kSmem : width == 32 ? GCfg<32>::kSmem : GCfg<64>::kSmem;
   const int ki = width == 96 ? 5 : width == 32 ? 7 : 2;  // dyn_smem index of gate+up
-  const int grid = d.sms;
+  const int grid = width == 32 ? 2 * d.sms : d.sms;
   if (usmem > (size_t)d.dyn_smem[1] || csmem > (size_t)d.dyn_smem[4] ||
       gsmem > (unsigned)d.dyn_smem[ki] || gsmem > (unsigned)d.dyn_smem[ki + 1]) {
     *why = MOE_ERR_UNSUPPORTED;
@@ -234,7 +246,7 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   route_union_kernel<<<1, 32 * kUnionWarps, usmem, st>>>(idx, P, E, uniq, offs, plist, nu,
                                                          padded);
   grouped_pack_x_kernel<<<m < 4 * d.sms ? m : 4 * d.sms, 256, 0, st>>>(x, plist, offs, padded,
-                                                                         nu, k, H, pcap, xp);
+                                                                         nu, k, H, pcap, xp, xs);
   GroupedArgs g{};
   g.unique = uniq;
   g.offsets = offs;
@@ -243,9 +255,11 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   g.pcap = pcap;
   g.H = H;
   g.hp = hp;
+  g.hs = hs;
   g.y = y;
   // gate + up: 128 rows of Wg and the same 128 rows of Wu per tile, K = H, packed x
   g.bp = xp;
+  g.bs = xs;
   g.q[0] = gq;
   g.s[0] = gs;
   g.b[0] = gb;
@@ -264,6 +278,7 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
     grouped_gemm_kernel<0, 64><<<grid, kGThreads, gsmem, st>>>(g);
   // down: 256 rows of Wd per tile (two 128-row matrices), K = I, packed h
   g.bp = hp;
+  g.bs = hs;
   g.q[0] = g.q[1] = dq;
   g.s[0] = g.s[1] = ds;
   g.b[0] = g.b[1] = db;
@@ -287,6 +302,44 @@ struct OwnedWorkspace {
   size_t bytes = 0;
 };
 OwnedWorkspace g_ws[kMaxDevices];
+
+// The library-owned workspace of the current device, grown (outside stream
+// capture only) to hold this shape; zeroed when allocated.
+moe_status owned_workspace(int T, int k, int E, int hidden, int inter, int fmt, void* stream,
+                           void** out, size_t* bytes) {
+  int dev = 0;
+  const cudaError_t ge = cudaGetDevice(&dev);
+  if (ge != cudaSuccess) return cuda_fail(ge);
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+  const size_t need = ws_layout(T, k, E, hidden, inter, fmt).total;
+  OwnedWorkspace& w = g_ws[dev];
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (w.bytes < need) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    const cudaError_t ce = cudaStreamIsCapturing((cudaStream_t)stream, &cs);
+    if (ce != cudaSuccess) return cuda_fail(ce);
+    if (cs != cudaStreamCaptureStatusNone) return MOE_ERR_WORKSPACE;
+    // The old buffer may still be in use by queued work on some stream.
+    if (w.ptr) {
+      const cudaError_t se = cudaDeviceSynchronize();
+      if (se != cudaSuccess) return cuda_fail(se);
+      cudaFree(w.ptr);
+      w.ptr = nullptr;
+      w.bytes = 0;
+    }
+    cudaError_t me = cudaMalloc(&w.ptr, need);
+    if (me == cudaSuccess) me = cudaMemset(w.ptr, 0, need);  // progress counters start at 0
+    if (me != cudaSuccess) {
+      if (w.ptr) cudaFree(w.ptr);
+      w.ptr = nullptr;
+      return cuda_fail(me);
+    }
+    w.bytes = need;
+  }
+  *out = w.ptr;
+  *bytes = w.bytes;
+  return MOE_OK;
+}
 
 // Fixed scratch for moe_switchglu_forward_static: one copy per device, in the
 // module's global memory (zero at module load), so that entry never allocates.
@@ -361,6 +414,15 @@ int moe_select_path(int T, int k, int E, int hidden, int inter) {
   return select_path(T, k, E, hidden, inter);
 }
 
+int moe_select_path_mxfp4(int T, int k, int E, int hidden, int inter) {
+  return select_path(T, k, E, hidden, inter, kFmtMx);
+}
+
+size_t moe_workspace_size_mxfp4(int T, int k, int E, int hidden, int inter) {
+  if (!shape_ok(T, k, E, hidden, inter)) return 0;
+  return ws_layout(T, k, E, hidden, inter, kFmtMx).total;
+}
+
 moe_status moe_router_topk(const float* logits, int T, int E, int k, int renormalize,
                            int32_t* topk_idx, float* topk_w, void* stream) {
   if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
@@ -418,7 +480,7 @@ moe_status moe_switchglu_forward_ws(const uint16_t* x, const int32_t* topk_idx,
   if (moe_status s = device_info(&d)) return s;
   moe_status why = MOE_OK;
   const cudaError_t e =
-      path == 1 ? launch_layer(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q, wd_s,
+      path == 1 ? launch_layer<kFmtAffine>(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q, wd_s,
                                wd_b, T, k, E, hidden, inter, out,
                                static_cast<unsigned char*>(workspace), *d, (cudaStream_t)stream,
                                &why)
@@ -438,39 +500,12 @@ moe_status moe_switchglu_forward(const uint16_t* x, const int32_t* topk_idx, con
                                  const uint16_t* wd_b, int T, int k, int E, int hidden,
                                  int inter, uint16_t* out, void* stream) {
   if (!shape_ok(T, k, E, hidden, inter)) return MOE_ERR_INVALID_ARG;
-  int dev = 0;
-  const cudaError_t ge = cudaGetDevice(&dev);
-  if (ge != cudaSuccess) return cuda_fail(ge);
-  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
-  const size_t need = ws_layout(T, k, E, hidden, inter).total;
-  OwnedWorkspace& w = g_ws[dev];
-  {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (w.bytes < need) {
-      cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-      const cudaError_t ce = cudaStreamIsCapturing((cudaStream_t)stream, &cs);
-      if (ce != cudaSuccess) return cuda_fail(ce);
-      if (cs != cudaStreamCaptureStatusNone) return MOE_ERR_WORKSPACE;
-      // The old buffer may still be in use by queued work on some stream.
-      if (w.ptr) {
-        const cudaError_t se = cudaDeviceSynchronize();
-        if (se != cudaSuccess) return cuda_fail(se);
-        cudaFree(w.ptr);
-        w.ptr = nullptr;
-        w.bytes = 0;
-      }
-      cudaError_t me = cudaMalloc(&w.ptr, need);
-      if (me == cudaSuccess) me = cudaMemset(w.ptr, 0, need);  // grid-barrier words start at 0
-      if (me != cudaSuccess) {
-        if (w.ptr) cudaFree(w.ptr);
-        w.ptr = nullptr;
-        return cuda_fail(me);
-      }
-      w.bytes = need;
-    }
-  }
+  void* ws = nullptr;
+  size_t bytes = 0;
+  if (moe_status s = owned_workspace(T, k, E, hidden, inter, kFmtAffine, stream, &ws, &bytes))
+    return s;
   return moe_switchglu_forward_ws(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q,
-                                  wd_s, wd_b, T, k, E, hidden, inter, out, w.ptr, w.bytes, stream);
+                                  wd_s, wd_b, T, k, E, hidden, inter, out, ws, bytes, stream);
 }
 
 moe_status moe_switchglu_forward_static(const uint16_t* x, const int32_t* topk_idx,
@@ -498,6 +533,52 @@ moe_status moe_switchglu_forward_static(const uint16_t* x, const int32_t* topk_i
   return moe_switchglu_forward_ws(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q,
                                   wd_s, wd_b, T, k, E, hidden, inter, out, scratch,
                                   kStaticScratchBytes, stream);
+}
+
+moe_status moe_switchglu_forward_mxfp4_ws(const uint16_t* x, const int32_t* topk_idx,
+                                          const float* topk_w, const uint32_t* wg_q,
+                                          const uint8_t* wg_e, const uint32_t* wu_q,
+                                          const uint8_t* wu_e, const uint32_t* wd_q,
+                                          const uint8_t* wd_e, int T, int k, int E, int hidden,
+                                          int inter, uint16_t* out, void* workspace,
+                                          size_t workspace_bytes, void* stream) {
+  if (!x || !topk_idx || !topk_w || !wg_q || !wg_e || !wu_q || !wu_e || !wd_q || !wd_e ||
+      !out || !workspace)
+    return MOE_ERR_INVALID_ARG;
+  if (!shape_ok(T, k, E, hidden, inter)) return MOE_ERR_INVALID_ARG;
+  const void* a16[] = {x, wg_q, wg_e, wu_q, wu_e, wd_q, wd_e, out, workspace};
+  for (const void* p : a16)
+    if (!aligned(p, 16)) return MOE_ERR_UNSUPPORTED;
+  if (!aligned(topk_idx, 4) || !aligned(topk_w, 4)) return MOE_ERR_UNSUPPORTED;
+  if (select_path(T, k, E, hidden, inter, kFmtMx) != 1) return MOE_ERR_UNSUPPORTED;
+  if (workspace_bytes < ws_layout(T, k, E, hidden, inter, kFmtMx).total) return MOE_ERR_WORKSPACE;
+  DeviceInfo* d = nullptr;
+  if (moe_status s = device_info(&d)) return s;
+  moe_status why = MOE_OK;
+  // the e8m0 scale arrays travel in the scale slots; the format has no biases
+  const uint16_t* ge = reinterpret_cast<const uint16_t*>(wg_e);
+  const uint16_t* ue = reinterpret_cast<const uint16_t*>(wu_e);
+  const uint16_t* de = reinterpret_cast<const uint16_t*>(wd_e);
+  const cudaError_t e = launch_layer<kFmtMx>(
+      x, topk_idx, topk_w, wg_q, ge, nullptr, wu_q, ue, nullptr, wd_q, de, nullptr, T, k, E,
+      hidden, inter, out, static_cast<unsigned char*>(workspace), *d, (cudaStream_t)stream, &why);
+  if (why != MOE_OK) return why;
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+moe_status moe_switchglu_forward_mxfp4(const uint16_t* x, const int32_t* topk_idx,
+                                       const float* topk_w, const uint32_t* wg_q,
+                                       const uint8_t* wg_e, const uint32_t* wu_q,
+                                       const uint8_t* wu_e, const uint32_t* wd_q,
+                                       const uint8_t* wd_e, int T, int k, int E, int hidden,
+                                       int inter, uint16_t* out, void* stream) {
+  if (!shape_ok(T, k, E, hidden, inter)) return MOE_ERR_INVALID_ARG;
+  void* ws = nullptr;
+  size_t bytes = 0;
+  if (moe_status s = owned_workspace(T, k, E, hidden, inter, kFmtMx, stream, &ws, &bytes))
+    return s;
+  return moe_switchglu_forward_mxfp4_ws(x, topk_idx, topk_w, wg_q, wg_e, wu_q, wu_e, wd_q, wd_e,
+                                        T, k, E, hidden, inter, out, ws, bytes, stream);
 }
 
 moe_status moe_read_device_status(void* stream) {

@@ -8,93 +8,90 @@
 // (route_union.cuh) has grouped the pairs by expert:
 //
 //   grouped_pack_x_kernel   the window's x rows, one per pair, in the order and
-//                           layout the tensor cores read (below);
+//                           layout the tensor cores read (below), with group sums;
 //   grouped_gemm_kernel<0, N>  gate+up: per (expert, 128 rows of Wg and of Wu) tile,
 //                           G = Wg X^T, U = Wu X^T, h = bf16(silu(bf16 G) * bf16 U),
 //                           h written packed for the next launch;
 //   grouped_gemm_kernel<1, N>  down: per (expert, 256 rows of Wd) tile, Y = Wd H^T,
 //                           fp32 per pair;
-// (N, the most pairs per MMA chunk, is 32, 64 or 96: wider chunks stream an
-// expert's weights fewer times when it has many pairs, narrower ones leave shared
-// memory for a deeper copy ring.)
+// (N, the pairs per MMA chunk, is 32, 64 or 96: wider chunks stream an expert's
+// weights fewer times when it has many pairs; with 32 two CTAs fit on an SM, which
+// doubles the warps that hide the per-slab latency.)
 //   grouped_combine_kernel  out[t] = bf16(sum_j w[t,j] * y[t,j]), j ascending.
 //
-// Arithmetic.  Each weight is dequantised once, w = bf16(s * q + b) (one fused
-// multiply-add on bf16 pairs, a single rounding of the exact s*q+b), the weight
-// rows of a tile become the MMA's A operand in shared memory, the packed bf16
-// activation rows its B operand, and the tensor cores accumulate the whole K of
-// the tile in fp32 in tensor memory.  The product is read once per tile.
+// The quantisation group (64 columns of K) is the MMA's K slab.  Inside a group
+// a weight row is s * q + b, so its dot product with an activation row a splits
+// as  sum_c w_c a_c = s * (sum_c q_c a_c) + b * (sum_c a_c).  The tensor cores
+// form P = sum_c q_c a_c from bf16 operands: the codes 0..15 are exact bf16
+// integers, the activations are bf16 already, each product is exact and the sum
+// is fp32.  Every slab's P is read back from tensor memory and s * P + b * X (X
+// the activation row's group sum) is added to fp32 registers.  No weight is ever
+// rounded; the only per-weight work is turning 4-bit codes into bf16 integers.
 //
-// Roles in a CTA (one CTA per SM, looping over tiles):
-//   warps 0..7   dequantisers: warps 4m..4m+3 own matrix m of the tile, one weight
-//                row per thread.  Per K slab of 64 columns (one quantisation group)
-//                a thread turns its row's 64 codes into bf16 weights and stores
-//                them in the A buffer (two buffers) in the MMA's layout;
-//   warps 8..11  epilogue: read a finished tile's accumulators (two buffers) from
-//                tensor memory, one row per thread, and write h (gate+up) or y
-//                (down);
-//   warp 12      producer: per stage of two slabs, 16-byte async copies of each
-//                weight row's codes (64 bytes) and 4-byte ones of its scales and
-//                biases, and 1-D bulk copies of the two packed activation slabs;
-//   warp 13      MMA issuer: tcgen05.mma (one elected lane of the converged
-//                warp) with A and B in shared memory, D in tensor memory.
+// Roles in a CTA (one or two CTAs per SM, looping over tiles):
+//   warp 8      producer: per stage of two slabs, 16-byte async copies of each
+//               weight row's codes (64 bytes) and 4-byte ones of its scales and
+//               biases, and 1-D bulk copies of the two packed activation slabs and
+//               of their group sums;
+//   warp 9      MMA issuer: issues tcgen05.mma (one elected lane of the converged
+//               warp) with A (the codes as bf16) in tensor memory and B (the
+//               activations) in shared memory;
+//   warps 0..7  warps 4m..4m+3 own matrix m of the tile, one weight row per
+//               thread (the row's tensor-memory lane).  Per slab they expand the
+//               row's codes to bf16 into tensor memory (the MMA's A operand), then
+//               read back the previous slab's product and accumulate it.
 // Codes expand without conversions: nibble q placed under the bf16 exponent of
 // 128 reads as 128 + q, and one packed bf16 FMA takes the 128 off exactly.  That
 // puts codes j and j + 4 of a 32-bit code word in one bf16 pair, so K runs in
 // the order (0,4,1,5,2,6,3,7) within every 8 columns; the packed activations
 // follow the same order.
 //
-// Operand layout (A and B alike): K-major rows of 128 bytes (one slab), 16-byte
-// chunk c of row p stored at chunk (c ^ (p & 7)), 8-row groups 1024 bytes apart:
-// the 128-byte swizzle, tiles based at 1024-byte boundaries.  Packed activations
-// in global memory: [K/64][pcap][64] bf16, row = padded pair position (expert slot
-// i owns rows padded[i] .. padded[i] + roundup16(count_i), route_union_kernel's
-// padded offsets; padding rows are zero), swizzled by the global row index.
+// Packed activations (the B operand): [K/64][pcap][64] bf16.  Row = padded pair
+// position: expert slot i owns rows padded[i] .. padded[i] + roundup16(count_i)
+// (route_union_kernel's padded offsets), with zero rows as padding.  Each 128-byte
+// row holds one slab in the K order above, its 16-byte chunk c stored at chunk
+// (c ^ (row & 7)): the 128-byte swizzle of a K-major tile whose rows start at
+// multiples of 8.  Group sums: [K/64][pcap] fp32.
 #pragma once
 
 #include "common.cuh"
 
 namespace qeg {
 
-constexpr int kGDeq = 8;                               // dequantising warps
-constexpr int kGEpi = 4;                               // epilogue warps
-constexpr int kGProducer = kGDeq + kGEpi;              // warp 12
-constexpr int kGMmaWarp = kGProducer + 1;              // warp 13
-constexpr int kGThreads = 32 * (kGMmaWarp + 1);        // 448
-constexpr int kGM = 128;                               // weight rows per matrix (MMA M)
-constexpr int kGK = 64;                                // K per slab = quantisation group
+constexpr int kGWorkers = 8;                         // worker warps
+constexpr int kGThreads = 32 * (kGWorkers + 2);      // + producer warp + MMA warp
+constexpr int kGM = 128;                             // weight rows per matrix (MMA M)
+constexpr int kGK = 64;                              // K per slab = quantisation group
 constexpr int kGSlabsPerStage = 2;
 constexpr unsigned kGCodePitch = kGSlabsPerStage * 32 + 16;  // padded: no bank conflicts
-constexpr unsigned kGCodeBytes = 2 * kGM * kGCodePitch;      // 20480
-constexpr unsigned kGSbBytes = 2 * kGM * kGSlabsPerStage * 2;  // scales (or biases) of a stage
-constexpr int kGABufs = 2;                             // A operand buffers
-constexpr unsigned kGATile = kGM * kGK * 2;            // one matrix's slab of A: 16 KB
-constexpr unsigned kGABytes = 2 * kGATile;             // one A buffer (both matrices)
-constexpr int kGAccBufs = 2;                           // accumulator buffers
-constexpr unsigned kGSmemBudget = 230400;              // dynamic shared memory planned for
+constexpr unsigned kGOffB = 2 * kGM * kGCodePitch;           // 20480, a multiple of 1024
+constexpr int kGDBufs = 2;   // accumulator buffers
+constexpr int kGLag = 1;     // a slab's accumulator is read back after the next slab's A is stored
+constexpr int kGABufs = 2;   // A operand buffers
 
-// Per chunk width NMAX (most pairs per MMA, a multiple of 32): the shared-memory
-// stage [codes | scales | biases | two activation slabs], the ring depth and the
-// tensor-memory map (accumulator buffer db, matrix m at columns (2 db + m) NMAX).
+// Per chunk width NMAX (pairs per MMA, a multiple of 32): the shared-memory stage
+// [codes | two activation slabs | their sums | scales | biases] and the tensor
+// memory map (accumulator of buffer db, matrix m; then the A operand of buffer ab).
 template <int NMAX>
 struct GCfg {
   static constexpr int kN = NMAX;
+  static constexpr int kStages = NMAX <= 32 ? 3 : (NMAX <= 64 ? 5 : 4);
+  static constexpr int kCtasPerSm = NMAX <= 32 ? 2 : 1;  // two CTAs share an SM's tensor memory
+  static constexpr uint32_t kTmemCols = NMAX <= 32 ? 256 : 512;
   static constexpr unsigned kBTile = NMAX * kGK * 2;
-  static constexpr unsigned kOffS = kGCodeBytes;
-  static constexpr unsigned kOffBias = kOffS + kGSbBytes;
-  static constexpr unsigned kOffB = kOffBias + kGSbBytes;  // 22528, a multiple of 1024
-  static constexpr unsigned kStageBytes = kOffB + kGSlabsPerStage * kBTile;
-  static constexpr unsigned kRing = kGSmemBudget - 1024 - kGABufs * kGABytes;
-  static constexpr int kStages = (int)(kRing / kStageBytes) > 6 ? 6 : (int)(kRing / kStageBytes);
-  static constexpr unsigned kSmem = kGABufs * kGABytes + kStages * kStageBytes + 1024;
-  static constexpr uint32_t kTmemCols =
-      kGAccBufs * 2 * NMAX <= 128 ? 128 : (kGAccBufs * 2 * NMAX <= 256 ? 256 : 512);
-  static_assert(NMAX % 32 == 0 && kBTile % 1024 == 0 && kOffB % 1024 == 0,
-                "swizzled tiles need 1024-byte bases");
-  static_assert(kStages >= 2 && kSmem <= kGSmemBudget, "shared-memory plan");
-  static_assert(kGAccBufs * 2 * NMAX <= 512, "tensor memory map");
+  static constexpr unsigned kOffX = kGOffB + kGSlabsPerStage * kBTile;
+  static constexpr unsigned kOffS = kOffX + kGSlabsPerStage * NMAX * 4;
+  static constexpr unsigned kOffBias = kOffS + 2 * kGM * kGSlabsPerStage * 2;
+  static constexpr unsigned kStageBytes =
+      (kOffBias + 2 * kGM * kGSlabsPerStage * 2 + 1023) & ~1023u;
+  static constexpr unsigned kSmem = kStages * kStageBytes + 1024;  // + alignment slack
+  static_assert(NMAX % 32 == 0 && kBTile % 1024 == 0, "swizzled tiles need 1024-byte bases");
+  static_assert(kGDBufs * 2 * NMAX + kGABufs * 2 * 32 <= (int)kTmemCols, "tensor memory map");
   __device__ static __forceinline__ uint32_t col_d(uint32_t db, int m) {
     return (db * 2 + m) * NMAX;
+  }
+  __device__ static __forceinline__ uint32_t col_a(uint32_t ab, int m) {
+    return kGDBufs * 2 * NMAX + (ab * 2 + m) * 32;
   }
 };
 
@@ -118,16 +115,24 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (both operands bf16),
-// issued by one elected lane of a converged warp: the whole warp runs the issuing
-// code, so its operands stay warp-uniform (issue is several times faster than from
-// a single divergent thread).
-__device__ __forceinline__ void tc_mma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16 (both operands bf16).
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// The same, issued by one elected lane of a converged warp: the whole warp runs the
+// issuing code, so its operands stay warp-uniform (issue is several times faster
+// than from a single divergent thread).
+__device__ __forceinline__ void tc_mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                                 uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n .reg .pred p, e;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
-      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 __device__ __forceinline__ void tc_commit_elect(uint64_t* bar) {
@@ -228,41 +233,32 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
-// bf16 pair fused multiply-add, one rounding: a * b + c.
-__device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-
-// The 8 codes of word w as 4 bf16 pairs of dequantised weights bf16(s q + b)
-// (low half code j, high half code j + 4), j = 0..3.  one2 = bf16 pair (1, 1),
-// m128 = (-128, -128), s2 / b2 = the group's scale / bias in both halves.
-__device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t one2, uint32_t m128,
-                                              uint32_t s2, uint32_t b2) {
-  uint32_t o[4];
+// The 8 codes of word w as 4 bf16 pairs (low half q_j, high half q_{j+4}),
+// j = 0..3, exact.  one2 = bf16 pair (1, 1), m128 = (-128, -128).
+__device__ __forceinline__ void codes_to_bf16(uint32_t w, uint32_t one2, uint32_t m128,
+                                              uint32_t* o) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const uint32_t t = ((w >> (4 * j)) & 0x000F000Fu) | 0x43004300u;  // 128 + q, exact
-    o[j] = bf16x2_fma(bf16x2_fma(t, one2, m128), s2, b2);             // q exact, then s q + b
+    const uint32_t t = ((w >> (4 * j)) & 0x000F000Fu) | 0x43004300u;  // 128 + q
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(o[j]) : "r"(t), "r"(one2), "r"(m128));
   }
-  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // --------------------------------------------------------------- packing ---
 // Packed x: for every padded pair position of every expert slot, the pair's token
-// row of x (zero for padding).  One block per slot (looping).
+// row of x (zero for padding) and its group sums.  One block per slot (looping).
 __global__ void __launch_bounds__(256) grouped_pack_x_kernel(
     const uint16_t* __restrict__ x, const int* __restrict__ pair_list,
     const int* __restrict__ offsets, const int* __restrict__ padded,
-    const int* __restrict__ num_unique, int k, int H, int pcap, uint16_t* __restrict__ xp) {
+    const int* __restrict__ num_unique, int k, int H, int pcap, uint16_t* __restrict__ xp,
+    float* __restrict__ xs) {
   const int u = *num_unique;
   const int nslab = H / kGK;
   for (int slot = blockIdx.x; slot < u; slot += gridDim.x) {
     const int p0 = offsets[slot], cnt = offsets[slot + 1] - p0;
     const int np = (cnt + 15) & ~15;
     const int base = padded[slot];
-    const int units = np * nslab * 8;
+    const int units = np * nslab * 8;  // a multiple of 128: whole warps stay together
     for (int unit = threadIdx.x; unit < units; unit += blockDim.x) {
       const int c = unit & 7, rest = unit >> 3;
       const int g = rest % nslab, n = rest / nslab;
@@ -271,6 +267,11 @@ __global__ void __launch_bounds__(256) grouped_pack_x_kernel(
         const int t = pair_list[p0 + n] / k;
         v = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H + g * kGK + c * 8));
       }
+      float s = ((bf16_lo(v.x) + bf16_hi(v.x)) + (bf16_lo(v.y) + bf16_hi(v.y))) +
+                ((bf16_lo(v.z) + bf16_hi(v.z)) + (bf16_lo(v.w) + bf16_hi(v.w)));
+      s += __shfl_xor_sync(kFull, s, 1);
+      s += __shfl_xor_sync(kFull, s, 2);
+      s += __shfl_xor_sync(kFull, s, 4);
       uint4 o;  // K order (0,4,1,5,2,6,3,7)
       o.x = prmt(v.x, v.z, 0x5410u);
       o.y = prmt(v.x, v.z, 0x7632u);
@@ -278,6 +279,7 @@ __global__ void __launch_bounds__(256) grouped_pack_x_kernel(
       o.w = prmt(v.y, v.w, 0x7632u);
       const int pos = base + n;
       *reinterpret_cast<uint4*>(xp + ((size_t)g * pcap + pos) * kGK + ((c ^ (pos & 7)) * 8)) = o;
+      if (c == 0) xs[(size_t)g * pcap + pos] = s;
     }
   }
 }
@@ -285,6 +287,7 @@ __global__ void __launch_bounds__(256) grouped_pack_x_kernel(
 // ------------------------------------------------------------------ GEMMs ---
 struct GroupedArgs {
   const uint16_t* bp;    // packed activations [K/64][pcap][64] (x or h)
+  const float* bs;       // their group sums [K/64][pcap]
   const int* unique;     // [u] distinct experts, ascending
   const int* offsets;    // [u + 1]
   const int* padded;     // [u + 1] padded row offsets of the packed layout
@@ -294,47 +297,38 @@ struct GroupedArgs {
   const uint16_t* b[2];  // biases
   int roff[2];           // row offset of matrix m inside the tile (0/0 or 0/128)
   uint16_t* hp;          // phase 0: packed h [I/64][pcap][64]
+  float* hs;             // phase 0: h group sums [I/64][pcap]
   float* y;              // phase 1: [P, H] fp32 in pair_list order
   int rows, K, mrows;    // weight rows per expert; K; weight rows per tile
   int pcap, H;
 };
 
-// Shared-memory matrix descriptor for the A tile of matrix m in A buffer ab.
-__device__ __forceinline__ uint32_t a_tile(const unsigned char* base, uint32_t ab, int m) {
-  return smem_u32(base + ab * kGABytes + m * kGATile);
-}
-
 template <int PHASE, int NMAX>
-__global__ void __launch_bounds__(kGThreads, 1)
+__global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
     grouped_gemm_kernel(const __grid_constant__ GroupedArgs a) {
   using C = GCfg<NMAX>;
   extern __shared__ __align__(128) unsigned char gsm_raw[];
-  __shared__ __align__(8) uint64_t full[C::kStages], w_empty[C::kStages];
-  __shared__ __align__(8) uint64_t a_full[kGABufs], a_empty[kGABufs];
-  __shared__ __align__(8) uint64_t acc_full[kGAccBufs], acc_empty[kGAccBufs];
+  __shared__ __align__(8) uint64_t full[C::kStages], empty[C::kStages];
+  __shared__ __align__(8) uint64_t a_full[kGABufs], d_full[kGDBufs], d_free[kGDBufs];
   __shared__ uint32_t tmem_base_s;
+  __shared__ float red[2][2][C::kN / 2];
   // swizzled tiles start at 1024-byte boundaries of the shared address space
   unsigned char* gsm = gsm_raw + ((1024u - (smem_u32(gsm_raw) & 1023u)) & 1023u);
-  unsigned char* abuf = gsm;                                // A buffers
-  unsigned char* ring = gsm + kGABufs * kGABytes;           // copy stages
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
     for (int i = 0; i < C::kStages; ++i) {
-      mbar_init(&full[i], 1 + 32);         // expect_tx + one cp.async arrival per lane
-      mbar_init(&w_empty[i], kGDeq + 1);   // dequantising warps + the MMA commit
+      mbar_init(&full[i], 1 + 32);          // expect_tx + one cp.async arrival per lane
+      mbar_init(&empty[i], kGWorkers + 1);  // worker warps + the MMA commit
     }
-    for (int i = 0; i < kGABufs; ++i) {
-      mbar_init(&a_full[i], kGDeq);
-      mbar_init(&a_empty[i], 1);
-    }
-    for (int i = 0; i < kGAccBufs; ++i) {
-      mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], kGEpi);
+    for (int i = 0; i < kGABufs; ++i) mbar_init(&a_full[i], kGWorkers);
+    for (int i = 0; i < kGDBufs; ++i) {
+      mbar_init(&d_full[i], 1);
+      mbar_init(&d_free[i], kGWorkers);
     }
     fence_barrier_init();
   }
-  if (warp == kGMmaWarp) {
+  if (warp == kGWorkers + 1) {
     tmem_alloc(&tmem_base_s, C::kTmemCols);
     tmem_relinquish();
   }
@@ -350,9 +344,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
   bool ok = true;
   uint32_t sc = 0;  // stages started (the same sequence in every role)
   uint32_t gs = 0;  // slabs started
-  uint32_t tc = 0;  // chunk tiles started
 
-  if (warp == kGProducer) {
+  if (warp == kGWorkers) {
     // ------------------------------------------------------------ producer ---
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       const int slot = tile / mtiles, m0 = (tile % mtiles) * a.mrows;
@@ -365,12 +358,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
           const int st = sc % C::kStages;
           const uint32_t round = sc / C::kStages;
           if (lane == 0) {
-            if (round > 0) ok = mbar_wait(&w_empty[st], (round - 1) & 1);
-            if (ok) mbar_arrive_expect_tx(&full[st], kGSlabsPerStage * np * (kGK * 2));
+            if (round > 0) ok = mbar_wait(&empty[st], (round - 1) & 1);
+            if (ok)
+              mbar_arrive_expect_tx(&full[st], kGSlabsPerStage * np * (kGK * 2 + 4));
           }
           ok = __shfl_sync(kFull, ok, 0);
           if (!ok) break;
-          unsigned char* stg = ring + st * C::kStageBytes;
+          unsigned char* stg = gsm + st * C::kStageBytes;
           // codes: 16 bytes per lane, four lanes per row (64 bytes = two slabs)
 #pragma unroll 8
           for (int i = 0; i < 2 * kGM * kGSlabsPerStage * 2 / 32; ++i) {
@@ -391,8 +385,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
 #pragma unroll
             for (int jj = 0; jj < kGSlabsPerStage; ++jj) {
               const size_t prow = (size_t)(j0 + jj) * a.pcap + pp0 + c0;
-              bulk_g2s(stg + C::kOffB + jj * C::kBTile, a.bp + prow * kGK, np * kGK * 2,
-                       &full[st]);
+              bulk_g2s(stg + kGOffB + jj * C::kBTile, a.bp + prow * kGK, np * kGK * 2, &full[st]);
+              bulk_g2s(stg + C::kOffX + jj * C::kN * 4, a.bs + prow, np * 4, &full[st]);
             }
           }
           cp_async_arrive_noinc(&full[st]);
@@ -404,30 +398,26 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if (lane == 0)
       for (uint32_t i = sc > (uint32_t)C::kStages ? sc - C::kStages : 0; i < sc; ++i)
         mbar_wait(&full[i % C::kStages], (i / C::kStages) & 1);
-  } else if (warp == kGMmaWarp) {
+  } else if (warp == kGWorkers + 1) {
     // ---------------------------------------------------------- MMA issuer ---
     // The whole warp runs this loop (operands warp-uniform); one elected lane issues.
-    bool issued_any = false;
-    uint32_t last_db = 0, last_tc = 0;
+    uint32_t issued = 0;  // slabs whose MMAs were issued
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       const int slot = tile / mtiles;
       const int cnt = a.offsets[slot + 1] - a.offsets[slot];
-      for (int c0 = 0; c0 < cnt && ok; c0 += C::kN, ++tc) {
+      for (int c0 = 0; c0 < cnt && ok; c0 += C::kN) {
         const int np = (min(C::kN, cnt - c0) + 15) & ~15;
         const uint32_t idesc = f16_idesc(kGM, np);
-        const uint32_t db = tc % kGAccBufs;
-        if (tc >= (uint32_t)kGAccBufs)
-          ok = __all_sync(kFull, mbar_wait(&acc_empty[db], (tc / kGAccBufs - 1) & 1));
-        if (!ok) break;
-        tc_fence_after();
-        bool first = true;
         for (int j0 = 0; j0 < nslab && ok; j0 += kGSlabsPerStage, ++sc) {
           const int st = sc % C::kStages;
-          ok = __all_sync(kFull, mbar_wait(&full[st], (sc / C::kStages) & 1));
-          const uint32_t bbase = smem_u32(ring + st * C::kStageBytes + C::kOffB);
+          const uint32_t round = sc / C::kStages;
+          ok = __all_sync(kFull, mbar_wait(&full[st], round & 1));
+          const uint32_t bbase = smem_u32(gsm + st * C::kStageBytes + kGOffB);
           for (int jj = 0; jj < kGSlabsPerStage && ok; ++jj, ++gs) {
-            const uint32_t ab = gs % kGABufs;
-            ok = __all_sync(kFull, mbar_wait(&a_full[ab], (gs / kGABufs) & 1));
+            const uint32_t ab = gs % kGABufs, db = gs % kGDBufs;
+            bool w = mbar_wait(&a_full[ab], (gs / kGABufs) & 1);
+            if (w && gs >= (uint32_t)kGDBufs) w = mbar_wait(&d_free[db], (gs / kGDBufs - 1) & 1);
+            ok = __all_sync(kFull, w);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
@@ -435,130 +425,221 @@ __global__ void __launch_bounds__(kGThreads, 1)
               const uint64_t bdesc = sw128_desc(bbase + jj * C::kBTile + kk * 32);
 #pragma unroll
               for (int m = 0; m < 2; ++m)
-                tc_mma_ss_elect(tmem + C::col_d(db, m), sw128_desc(a_tile(abuf, ab, m) + kk * 32),
-                                bdesc, idesc, (first && kk == 0) ? 0u : 1u);
+                tc_mma_ts_elect(tmem + C::col_d(db, m), tmem + C::col_a(ab, m) + kk * 8, bdesc, idesc,
+                                kk > 0 ? 1u : 0u);
             }
-            first = false;
-            tc_commit_elect(&a_empty[ab]);
-            if (jj == kGSlabsPerStage - 1) tc_commit_elect(&w_empty[st]);
+            tc_commit_elect(&d_full[db]);
+            if (jj == kGSlabsPerStage - 1) tc_commit_elect(&empty[st]);
+            issued = gs + 1;
           }
         }
-        if (!ok) break;
-        tc_commit_elect(&acc_full[db]);
-        issued_any = true;
-        last_db = db;
-        last_tc = tc;
       }
     }
     // no MMA may run past the deallocation below (at once when all went well)
-    if (issued_any) mbar_wait(&acc_full[last_db], (last_tc / kGAccBufs) & 1);
-  } else if (warp < kGDeq) {
-    // ----------------------------------------------------------- dequantise ---
-    const int m = warp >> 2, r = 32 * (warp & 3) + lane;
+    if (issued > 0) mbar_wait(&d_full[(issued - 1) % kGDBufs], ((issued - 1) / kGDBufs) & 1);
+  } else {
+    // ------------------------------------------------------------- workers ---
+    const int m = warp >> 2, qd = warp & 3, r = 32 * qd + lane;
+    const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
     const uint32_t one2 = 0x3F803F80u, m128 = 0xC300C300u;  // bf16 pairs (1, 1), (-128, -128)
-    const unsigned arow = (unsigned)((r >> 3) * 1024 + (r & 7) * 128);
-    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-      const int slot = tile / mtiles;
-      const int cnt = a.offsets[slot + 1] - a.offsets[slot];
-      for (int c0 = 0; c0 < cnt && ok; c0 += C::kN) {
-        for (int j0 = 0; j0 < nslab && ok; j0 += kGSlabsPerStage, ++sc) {
-          const int st = sc % C::kStages;
-          ok = __all_sync(kFull, mbar_wait(&full[st], (sc / C::kStages) & 1));
-          if (!ok) break;
-          const unsigned char* stg = ring + st * C::kStageBytes;
-          const uint4* crow = reinterpret_cast<const uint4*>(stg + (m * kGM + r) * kGCodePitch);
-          const uint32_t sv2 = *reinterpret_cast<const uint32_t*>(stg + C::kOffS + (m * kGM + r) * 4);
-          const uint32_t bv2 =
-              *reinterpret_cast<const uint32_t*>(stg + C::kOffBias + (m * kGM + r) * 4);
-          for (int jj = 0; jj < kGSlabsPerStage && ok; ++jj, ++gs) {
-            const uint32_t ab = gs % kGABufs;
-            if (gs >= (uint32_t)kGABufs)
-              ok = __all_sync(kFull, mbar_wait(&a_empty[ab], (gs / kGABufs - 1) & 1));
-            if (!ok) break;
-            // this slab's scale and bias in both halves of a bf16 pair
-            const uint32_t s2 = jj ? __byte_perm(sv2, 0, 0x3232) : __byte_perm(sv2, 0, 0x1010);
-            const uint32_t b2 = jj ? __byte_perm(bv2, 0, 0x3232) : __byte_perm(bv2, 0, 0x1010);
-            const uint4 w0 = crow[2 * jj], w1 = crow[2 * jj + 1];
-            unsigned char* dst = abuf + ab * kGABytes + m * kGATile + arow;
-            const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    float2 acc[C::kN / 2];
+
+    // wait until the MMAs of slab gp are done (its accumulator is ready and the A
+    // buffer it read is free)
+    auto wait_slab = [&](uint32_t gp) {
+      ok = __all_sync(kFull, ok && mbar_wait(&d_full[gp % kGDBufs], (gp / kGDBufs) & 1));
+    };
+    // add the product of slab gp (stage st, place jj in the stage) to acc; its
+    // MMAs are known to be done
+    auto readout = [&](uint32_t gp, int st, int jj, int ng) {
+      const uint32_t ab = gp % kGDBufs;
+      tc_fence_after();
+      const unsigned char* stg = gsm + st * C::kStageBytes;
+      const float sv = bf16_bits_to_float(
+          *reinterpret_cast<const uint16_t*>(stg + C::kOffS + (m * kGM + r) * 4 + jj * 2));
+      const float bv = bf16_bits_to_float(
+          *reinterpret_cast<const uint16_t*>(stg + C::kOffBias + (m * kGM + r) * 4 + jj * 2));
+      const float2 s2 = make_float2(sv, sv), b2 = make_float2(bv, bv);
+      const float4* X = reinterpret_cast<const float4*>(stg + C::kOffX + jj * C::kN * 4);
+      const uint32_t dcol = tmem + C::col_d(ab, m) + lane_base;
+      // kRd columns per tensor-memory wait (16 where registers are scarce)
+      constexpr int kRd = C::kN == 64 ? 32 : 16, kRg = kRd / 16;
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              *reinterpret_cast<uint4*>(dst + ((c ^ (r & 7)) << 4)) =
-                  dequant_word(wv[c], one2, m128, s2, b2);
-            fence_proxy_async();  // the generic-proxy stores, before the MMA reads them
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&a_full[ab]);
+      for (int c2 = 0; c2 < C::kN / kRd; ++c2) {
+        if (kRg * c2 < ng) {
+          uint32_t pr[kRd];
+          tc_ld16(dcol + c2 * kRd, pr);
+          if constexpr (kRg == 2) {
+            if (2 * c2 + 1 < ng) tc_ld16(dcol + c2 * kRd + 16, pr + 16);
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&w_empty[st]);
+          tc_wait_ld();
+#pragma unroll
+          for (int h = 0; h < kRg; ++h) {
+            const int cg = kRg * c2 + h;
+            if (cg < ng) {
+              tc_regs_ready(pr + 16 * h);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float4 xv = X[cg * 4 + i];
+                const int o = cg * 8 + 2 * i;
+                const uint32_t* pp = pr + 16 * h + 4 * i;
+                acc[o] = __ffma2_rn(make_float2(__uint_as_float(pp[0]), __uint_as_float(pp[1])),
+                                    s2, acc[o]);
+                acc[o + 1] = __ffma2_rn(
+                    make_float2(__uint_as_float(pp[2]), __uint_as_float(pp[3])), s2, acc[o + 1]);
+                acc[o] = __ffma2_rn(make_float2(xv.x, xv.y), b2, acc[o]);
+                acc[o + 1] = __ffma2_rn(make_float2(xv.z, xv.w), b2, acc[o + 1]);
+              }
+            }
+          }
         }
       }
-    }
-  } else {
-    // ------------------------------------------------------------- epilogue ---
-    const int qd = warp - kGDeq, r = 32 * qd + lane;  // tensor-memory lane quarter qd
-    const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&d_free[ab]);
+        if (jj == kGSlabsPerStage - 1) mbar_arrive(&empty[st]);
+      }
+    };
+
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       const int slot = tile / mtiles, m0 = (tile % mtiles) * a.mrows;
       const int p0 = a.offsets[slot], cnt = a.offsets[slot + 1] - p0;
       const int pp0 = a.padded[slot];
-      for (int c0 = 0; c0 < cnt && ok; c0 += C::kN, ++tc) {
-        const int n = min(C::kN, cnt - c0), np = (n + 15) & ~15;
-        const uint32_t db = tc % kGAccBufs;
-        ok = __all_sync(kFull, mbar_wait(&acc_full[db], (tc / kGAccBufs) & 1));
-        if (!ok) break;
-        tc_fence_after();
-        if (PHASE == 0) {
-          // h = bf16(silu(bf16 g) * bf16 u): matrix 0 holds g, matrix 1 u; this
-          // thread's row of the tile is column m0 + r of h
-          const int irow = m0 + r;
-          const int gI = irow / kGK, ci = irow % kGK;
-          const int pin = (ci & ~7) + 2 * (ci & 3) + ((ci >> 2) & 1);  // K order position
-#pragma unroll 1
-          for (int c16 = 0; c16 < np; c16 += 16) {
-            uint32_t gr[16], ur[16];
-            tc_ld16(tmem + C::col_d(db, 0) + c16 + lane_base, gr);
-            tc_ld16(tmem + C::col_d(db, 1) + c16 + lane_base, ur);
-            tc_wait_ld();
-            tc_regs_ready(gr);
-            tc_regs_ready(ur);
+      for (int c0 = 0; c0 < cnt && ok; c0 += C::kN) {
+        const int n = min(C::kN, cnt - c0), np = (n + 15) & ~15, ng = np / 16;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float g = round_to_bf16(__uint_as_float(gr[i]));
-              const float uu = round_to_bf16(__uint_as_float(ur[i]));
-              const uint16_t hb = float_to_bf16_bits(g / (1.0f + __expf(-g)) * uu);
-              const int pos = pp0 + c0 + c16 + i;
-              a.hp[((size_t)gI * a.pcap + pos) * kGK + (((pin >> 3) ^ (pos & 7)) << 3) +
-                   (pin & 7)] = hb;
+        for (int i = 0; i < C::kN / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+        const uint32_t gs0 = gs, sc0 = sc;  // first slab and stage of the chunk
+        // slab g of this chunk: stage (sc0 + (g - gs0) / 2) % C::kStages, place (g - gs0) & 1
+        auto read_slab = [&](uint32_t g) {
+          const uint32_t jl = g - gs0;
+          readout(g, (int)((sc0 + jl / kGSlabsPerStage) % C::kStages), (int)(jl % kGSlabsPerStage), ng);
+        };
+        for (int j0 = 0; j0 < nslab && ok; j0 += kGSlabsPerStage, ++sc) {
+          const int st = sc % C::kStages;
+          const uint32_t round = sc / C::kStages;
+          ok = __all_sync(kFull, mbar_wait(&full[st], round & 1));
+          if (!ok) break;
+          const unsigned char* stg = gsm + st * C::kStageBytes;
+          for (int jj = 0; jj < kGSlabsPerStage && ok; ++jj, ++gs) {
+            const uint32_t ab = gs % kGABufs;
+            // the MMAs that read this A buffer (slab gs - 2) are done
+            if (gs >= (uint32_t)kGABufs) wait_slab(gs - kGABufs);
+            if (!ok) break;
+            tc_fence_after();  // the A buffer's earlier reads are done before these writes
+            // this row's codes of the slab -> bf16 integers -> the A operand
+            const uint4* crow =
+                reinterpret_cast<const uint4*>(stg + (m * kGM + r) * kGCodePitch + jj * 32);
+            const uint32_t acol = tmem + C::col_a(ab, m) + lane_base;
+#pragma unroll
+            for (int hw = 0; hw < 2; ++hw) {  // 32 codes (16 columns) at a time
+              const uint4 wv = crow[hw];
+              uint32_t av[16];
+              codes_to_bf16(wv.x, one2, m128, av + 0);
+              codes_to_bf16(wv.y, one2, m128, av + 4);
+              codes_to_bf16(wv.z, one2, m128, av + 8);
+              codes_to_bf16(wv.w, one2, m128, av + 12);
+              tc_st16(acol + 16 * hw, av);
             }
-          }
-        } else {
-          // y rows of the chunk's pairs (pair_list order), fp32: rows m0 + r and
-          // m0 + 128 + r of the expert's Wd
-#pragma unroll 1
-          for (int mm = 0; mm < 2; ++mm) {
-            float* yo = a.y + (size_t)(p0 + c0) * a.H + m0 + a.roff[mm] + r;
-#pragma unroll 1
-            for (int c16 = 0; c16 < np; c16 += 16) {
-              uint32_t yr[16];
-              tc_ld16(tmem + C::col_d(db, mm) + c16 + lane_base, yr);
-              tc_wait_ld();
-              tc_regs_ready(yr);
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                if (c16 + i < n) yo[(size_t)(c16 + i) * a.H] = __uint_as_float(yr[i]);
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&a_full[ab]);
+            if (gs >= gs0 + kGLag) {
+              wait_slab(gs - kGLag);
+              if (ok) read_slab(gs - kGLag);
             }
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[db]);
+        if (!ok) break;
+        // the chunk's last kGLag slabs
+        for (uint32_t g = gs >= gs0 + kGLag ? gs - kGLag : gs0; g < gs && ok; ++g) {
+          wait_slab(g);
+          if (ok) read_slab(g);
+        }
+        if (!ok) break;
+
+        if (PHASE == 0) {
+          // ---- h = bf16(silu(bf16 g) * bf16 u); matrix 0 holds g, matrix 1 u.  The
+          // two warps of a lane quarter swap halves through tensor memory (buffer 0's
+          // accumulator columns): no MMA runs now, the next one waits for every
+          // warp's next A operand.
+          const int irow = m0 + r;  // this thread's row of h's width I
+          const int gI = irow / kGK, ci = irow % kGK;
+          const int pin = (ci & ~7) + 2 * (ci & 3) + ((ci >> 2) & 1);  // K order position
+          constexpr int kHalf = C::kN / 2;  // pairs finished by each matrix's warps
+#pragma unroll
+          for (int hh = 0; hh < kHalf / 16; ++hh) {
+            // 16 pairs per round: this thread finishes pairs kHalf m + 16hh + i
+            uint32_t ex[16];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float2 v = m == 0 ? acc[kHalf / 2 + 8 * hh + i] : acc[8 * hh + i];
+              ex[2 * i] = __float_as_uint(v.x);
+              ex[2 * i + 1] = __float_as_uint(v.y);
+            }
+            // each warp writes only its own matrix's columns (its partner may still be
+            // reading the other matrix's): matrix 0 gives g of pairs kHalf + 16hh.. at
+            // its columns kHalf + 16hh.., matrix 1 gives u of pairs 16hh.. at its
+            // columns 16hh..
+            const uint32_t give =
+                tmem + C::col_d(0, m) + (m == 0 ? kHalf : 0) + 16 * hh + lane_base;
+            const uint32_t take =
+                tmem + C::col_d(0, 1 - m) + (m == 0 ? 0 : kHalf) + 16 * hh + lane_base;
+            tc_st16(give, ex);
+            tc_wait_st();
+            tc_fence_before();
+            named_barrier(1 + qd, 64);
+            tc_fence_after();
+            uint32_t ot[16];
+            tc_ld16(take, ot);
+            tc_wait_ld();
+            tc_regs_ready(ot);
+            tc_fence_before();
+            float hv[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float2 mine = m == 0 ? acc[8 * hh + i / 2] : acc[kHalf / 2 + 8 * hh + i / 2];
+              const float own = (i & 1) ? mine.y : mine.x;
+              const float oth = __uint_as_float(ot[i]);
+              const float g = round_to_bf16(m == 0 ? own : oth);
+              const float uu = round_to_bf16(m == 0 ? oth : own);
+              const uint16_t hb = float_to_bf16_bits(g / (1.0f + __expf(-g)) * uu);
+              hv[i] = bf16_bits_to_float(hb);
+              const int nn = kHalf * m + 16 * hh + i;
+              if (nn < np) {
+                const int pos = pp0 + c0 + nn;
+                a.hp[((size_t)gI * a.pcap + pos) * kGK + (((pin >> 3) ^ (pos & 7)) << 3) +
+                     (pin & 7)] = hb;
+              }
+            }
+            // group sums of h: over this warp's 32 rows (even lanes end with one
+            // pair's sum each), then over the group's two warps
+            int vid;
+            const float part = warp_reduce_scatter<16>(hv, lane, vid);
+            if ((qd & 1) && !(lane & 1)) red[m][qd >> 1][16 * hh + vid] = part;
+            named_barrier(5 + 2 * m + (qd >> 1), 64);
+            if (!(qd & 1) && !(lane & 1)) {
+              const int nn = kHalf * m + 16 * hh + vid;
+              if (nn < np)
+                a.hs[(size_t)gI * a.pcap + pp0 + c0 + nn] = part + red[m][qd >> 1][16 * hh + vid];
+            }
+            named_barrier(5 + 2 * m + (qd >> 1), 64);
+          }
+        } else {
+          // ---- y rows of the chunk's pairs (pair_list order), fp32
+          float* yo = a.y + (size_t)(p0 + c0) * a.H + m0 + a.roff[m] + r;
+#pragma unroll
+          for (int i = 0; i < C::kN; ++i)
+            if (i < n) yo[(size_t)i * a.H] = (i & 1) ? acc[i / 2].y : acc[i / 2].x;
+        }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kGMmaWarp) {
+  if (warp == kGWorkers + 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }

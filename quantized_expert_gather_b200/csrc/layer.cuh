@@ -49,6 +49,12 @@
 
 namespace qeg {
 
+// Bank formats.  kFmtAffine: 4-bit codes, bf16 scale and bias per 64 columns
+// (w = s q + b).  kFmtMx: mxfp4, e2m1 codes and one e8m0 scale per 32 columns
+// (w = e2m1(q) 2^(e - 127)).  Codes are packed alike in both.
+constexpr int kFmtAffine = 0;
+constexpr int kFmtMx = 1;
+
 constexpr int kWarps = 8;                    // compute warps
 constexpr int kConsumerThreads = 32 * kWarps;
 constexpr int kThreads = kConsumerThreads + 64;  // + a producer warp and a helper warp
@@ -74,22 +80,28 @@ __host__ __device__ constexpr unsigned act_digit_bytes(int R) { return 2048u * (
 
 // ---------------------------------------------------------------- geometry ---
 struct LayerGeom {
-  int rounds_a, rounds_b;  // 32-column chunks per lane per row (power of two >= H/1024, I/1024)
+  int fmt;                 // kFmtAffine or kFmtMx
+  int rounds_a, rounds_b;  // 32-column chunks per lane per row (>= H/1024, I/1024; 1, 2, 4, 6, 8)
   int rows_b;              // phase B rows per block (multiple of kWarps, <= 32)
   int seg;                 // pairs per segment (<= kNT)
   int stages;              // ring depth (<= kMaxStages)
-  unsigned a_q, a_sb, a_mat, a_bytes;  // phase A block: per matrix codes / scale bytes
+  unsigned a_q, a_sb, a_mat, a_bytes;  // phase A block: per matrix codes / scale (or bias) bytes
   unsigned b_q, b_sb, b_bytes;         // phase B full block
   unsigned stage_bytes;
   unsigned act_buf;        // one activation buffer: seg rows of the wider layout
 };
 
-__host__ __device__ inline LayerGeom layer_geom(int H, int I) {
+// Chunk rounds for a row of D columns: ceil(D / 1024), rounded up to 1, 2, 4, 6 or 8.
+__host__ __device__ inline int chunk_rounds(int D) {
+  const int r = (D + 1023) / 1024;
+  return r <= 2 ? r : (r <= 4 ? 4 : (r <= 6 ? 6 : 8));
+}
+
+__host__ __device__ inline LayerGeom layer_geom(int H, int I, int fmt = kFmtAffine) {
   LayerGeom g;
-  g.rounds_a = 1;
-  while (g.rounds_a * 1024 < H) g.rounds_a <<= 1;
-  g.rounds_b = 1;
-  while (g.rounds_b * 1024 < I) g.rounds_b <<= 1;
+  g.fmt = fmt;
+  g.rounds_a = chunk_rounds(H);
+  g.rounds_b = chunk_rounds(I);
   int rb = (16 * H / I) / kWarps * kWarps;  // about one phase-A stage worth of Wd rows
   if (rb < kWarps) rb = kWarps;
   if (rb > kWarps * kMaxRowsPerWarpB) rb = kWarps * kMaxRowsPerWarpB;
@@ -99,12 +111,15 @@ __host__ __device__ inline LayerGeom layer_geom(int H, int I) {
   g.seg = s > kNT ? kNT : s;
   g.stages = kMaxStages;
   g.a_q = kRowsA * H / 2;
+  // scales: bf16 per 64 columns (affine) or one e8m0 byte per 32 (mx), H/32 bytes a
+  // row either way; the affine format adds as many bytes of biases
+  const int nsb = fmt == kFmtMx ? 1 : 2;
   g.a_sb = kRowsA * H / 32;
-  g.a_mat = g.a_q + 2 * g.a_sb;
+  g.a_mat = g.a_q + nsb * g.a_sb;
   g.a_bytes = 2 * g.a_mat;
   g.b_q = g.rows_b * I / 2;
   g.b_sb = g.rows_b * I / 32;
-  g.b_bytes = g.b_q + 2 * g.b_sb;
+  g.b_bytes = g.b_q + nsb * g.b_sb;
   g.stage_bytes = (unsigned)align_up(g.a_bytes > g.b_bytes ? g.a_bytes : g.b_bytes, 128);
   g.act_buf = (unsigned)align_up((size_t)(g.seg > 0 ? g.seg : 1) * act_bytes(rmax), 128);
   return g;
@@ -232,7 +247,7 @@ __device__ __forceinline__ int chunk_dot(const uint32_t (&qs)[8], const uint4 (&
   return (hi0 + hi1) * 256 + (lo0 + lo1);  // |.| < 2^24: exact in fp32
 }
 
-// The 32 codes of a uint4, split as described above.
+// The 32 codes of a uint4, split as described above (affine format).
 __device__ __forceinline__ void split_codes(const uint4 v, uint32_t (&qs)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -242,10 +257,66 @@ __device__ __forceinline__ void split_codes(const uint4 v, uint32_t (&qs)[8]) {
   }
 }
 
+// mxfp4 codes as bytes for dp4a.  An e2m1 code (sign bit 3, magnitude index bits
+// 2..0 for 0, 0.5, 1, 1.5, 2, 3, 4, 6) becomes q' = 2 e2m1(q) + 12, an integer in
+// [0, 24], so that  e2m1(q) = (q' - 12) / 2  and a chunk's sum is
+// (sum q' v - 12 sum v) / 2.  Two byte lookups (prmt: four selectors from the 16
+// low bits, each picking one of 8 table bytes; a selector with bit 3 set returns
+// the sign fill of its byte, 0 for these tables) give the values of the positive
+// codes and of the negative ones, each 0 where the other applies.  Bytes 0..3 of
+// qs[2m] are codes 0..3 of word m (columns 8m .. 8m+3), bytes of qs[2m+1] codes
+// 4..7: consecutive columns, the activation layout of this format.
+constexpr uint32_t kMxPos0 = 0x0F0E0D0Cu, kMxPos1 = 0x18141210u;  // 12 + 2 * (0 .. 6)
+constexpr uint32_t kMxNeg0 = 0x090A0B0Cu, kMxNeg1 = 0x00040608u;  // 12 - 2 * (0 .. 6)
+// PTX prmt in its default mode (a selector's bit 3 asks for the sign fill).
+__device__ __forceinline__ uint32_t prmt_sign(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+__device__ __forceinline__ uint32_t mx_bytes(uint32_t sel) {
+  return prmt_sign(kMxPos0, kMxPos1, sel) | prmt_sign(kMxNeg0, kMxNeg1, sel ^ 0x8888u);
+}
+__device__ __forceinline__ void split_codes_mx(const uint4 v, uint32_t (&qs)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    qs[2 * m] = mx_bytes(w[m]);
+    qs[2 * m + 1] = mx_bytes(w[m] >> 16);
+  }
+}
+
+template <int F>
+__device__ __forceinline__ void split_codes_f(const uint4 v, uint32_t (&qs)[8]) {
+  if constexpr (F == kFmtMx) split_codes_mx(v, qs);
+  else split_codes(v, qs);
+}
+
+// 2^(e - 128) for an e8m0 byte e (half the mxfp4 block scale 2^(e - 127)); NaN for 255.
+__device__ __forceinline__ float mx_half_scale(uint32_t e) {
+  if (e >= 2u && e < 255u) return __uint_as_float((e - 1u) << 23);
+  if (e == 255u) return __uint_as_float(0x7fc00000u);
+  return __uint_as_float(0x00400000u >> (1u - e));  // 2^-127, 2^-128: subnormal
+}
+
+// Scale and bias applied to a chunk's exact sum:  partial = sv * 2^(e-14) * dot +
+// bv * sum x.  Affine: the group's (s, b), group ch / 2.  mxfp4: (2^(e-128),
+// -12 * 2^(e-128)) from the chunk's own e8m0 byte (see mx_bytes).
+template <int F>
+__device__ __forceinline__ float2 chunk_sb(const uint16_t* s, const uint16_t* b, int ch) {
+  if constexpr (F == kFmtMx) {
+    const float h = mx_half_scale(reinterpret_cast<const uint8_t*>(s)[ch]);
+    return make_float2(h, -12.0f * h);
+  } else {
+    return make_float2(bf16_bits_to_float(s[ch >> 1]), bf16_bits_to_float(b[ch >> 1]));
+  }
+}
+
 // One thread's quarter of a chunk: the 8 bf16 values of columns 8m .. 8m+7 (in v)
 // become this thread's uint4 of the layout above; the 4 threads of a chunk are
 // consecutive lanes (group mask gmask).  Returns the chunk's (scale, sum) in every
 // thread of the group.
+template <int F>
 __device__ __forceinline__ float2 fixed_point_quarter(const uint4 v, unsigned gmask,
                                                       uint4& out) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -275,9 +346,12 @@ __device__ __forceinline__ float2 fixed_point_quarter(const uint4 v, unsigned gm
     else if (sh <= 15) mag = (M[k] + (1 << (sh - 8))) >> (sh - 7);  // round half up
     else mag = 0;
     const int val = neg[k] ? -mag : mag;
-    const int pos = (k >> 1) * 8;  // byte within the word; k even -> .x/.z, odd -> .y/.w
-    lo[k & 1] |= (static_cast<uint32_t>(val) & 0xffu) << pos;
-    hi[k & 1] |= ((static_cast<uint32_t>(val) >> 8) & 0xffu) << pos;
+    // affine: k even -> .x/.z, odd -> .y/.w, byte k / 2; mxfp4: k < 4 -> .x/.z,
+    // else .y/.w, byte k % 4 (the orders the two code splits produce)
+    const int wsel = F == kFmtMx ? (k >> 2) : (k & 1);
+    const int pos = F == kFmtMx ? (k & 3) * 8 : (k >> 1) * 8;
+    lo[wsel] |= (static_cast<uint32_t>(val) & 0xffu) << pos;
+    hi[wsel] |= ((static_cast<uint32_t>(val) >> 8) & 0xffu) << pos;
   }
   out = make_uint4(lo[0], lo[1], hi[0], hi[1]);
   float scale;
@@ -325,7 +399,7 @@ __device__ __forceinline__ bool wait_counter(const unsigned* p, unsigned target)
 // stride), R rounds of 32-column chunks (chunks past H/32 skipped); returns (G, U)
 // for t < NT in every lane.  Per chunk (inside one quantisation group):
 // s * 2^(e-14) * sum q v + b * sum x.
-template <int NT, int R>
+template <int NT, int R, int F>
 __device__ __forceinline__ void rows_a(const unsigned char* bg_q, const uint16_t* bg_s,
                                        const uint16_t* bg_b, const unsigned char* bu_q,
                                        const uint16_t* bu_s, const uint16_t* bu_b, int H,
@@ -341,10 +415,10 @@ __device__ __forceinline__ void rows_a(const unsigned char* bg_q, const uint16_t
     const int ch = i * 32 + lane;
     if (ch < nch) {
       uint32_t qg[8], qu[8];
-      split_codes(*reinterpret_cast<const uint4*>(bg_q + ch * 16), qg);
-      split_codes(*reinterpret_cast<const uint4*>(bu_q + ch * 16), qu);
-      const float sg = bf16_bits_to_float(bg_s[ch >> 1]), bgv = bf16_bits_to_float(bg_b[ch >> 1]);
-      const float su = bf16_bits_to_float(bu_s[ch >> 1]), buv = bf16_bits_to_float(bu_b[ch >> 1]);
+      split_codes_f<F>(*reinterpret_cast<const uint4*>(bg_q + ch * 16), qg);
+      split_codes_f<F>(*reinterpret_cast<const uint4*>(bu_q + ch * 16), qu);
+      const float2 sbg = chunk_sb<F>(bg_s, bg_b, ch), sbu = chunk_sb<F>(bu_s, bu_b, ch);
+      const float sg = sbg.x, bgv = sbg.y, su = sbu.x, buv = sbu.y;
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
         const unsigned char* row = act + t * stride;
@@ -373,7 +447,7 @@ __device__ __forceinline__ void rows_a(const unsigned char* bg_q, const uint16_t
 // Phase B: rows row0 + kWarps*q (q < kMaxRowsPerWarpB, rows < nrows) of Wd, NT pairs.
 // Returns the value this lane holds after a reduce-scatter and its index
 // q*kNT + t in `vid` (-1 when it holds none).
-template <int NT, int R>
+template <int NT, int R, int F>
 __device__ __forceinline__ float rows_b(const unsigned char* bq, const uint16_t* bs,
                                         const uint16_t* bb, int row0, int nrows, int I,
                                         const unsigned char* act, unsigned stride, int lane,
@@ -402,9 +476,10 @@ __device__ __forceinline__ float rows_b(const unsigned char* bq, const uint16_t*
         const int r = row0 + kWarps * q;
         if (r < nrows) {
           uint32_t qs[8];
-          split_codes(*reinterpret_cast<const uint4*>(bq + (size_t)r * qstride + ch * 16), qs);
-          const float sv = bf16_bits_to_float(bs[r * sstride + (ch >> 1)]);
-          const float bv = bf16_bits_to_float(bb[r * sstride + (ch >> 1)]);
+          split_codes_f<F>(*reinterpret_cast<const uint4*>(bq + (size_t)r * qstride + ch * 16), qs);
+          // a row's scales: I/64 bf16 (affine) or I/32 bytes (mxfp4), I/32 bytes either way
+          const float2 sb = chunk_sb<F>(bs + r * sstride, bb + r * sstride, ch);
+          const float sv = sb.x, bv = sb.y;
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
             const float d = static_cast<float>(chunk_dot(qs, xd[t]));
@@ -422,26 +497,29 @@ __device__ __forceinline__ float rows_b(const unsigned char* bq, const uint16_t*
   return v;
 }
 
-template <int NT>
+template <int NT, int F>
 __device__ __forceinline__ void dispatch_a(int R, const unsigned char* bgq, const uint16_t* bgs,
                                            const uint16_t* bgb, const unsigned char* buq,
                                            const uint16_t* bus, const uint16_t* bub, int H,
                                            const unsigned char* act, unsigned stride, int lane,
                                            float (&G)[kNT], float (&U)[kNT]) {
-  if (R == 1) rows_a<NT, 1>(bgq, bgs, bgb, buq, bus, bub, H, act, stride, lane, G, U);
-  else if (R == 2) rows_a<NT, 2>(bgq, bgs, bgb, buq, bus, bub, H, act, stride, lane, G, U);
-  else rows_a<NT, 4>(bgq, bgs, bgb, buq, bus, bub, H, act, stride, lane, G, U);
+  if (R == 1) rows_a<NT, 1, F>(bgq, bgs, bgb, buq, bus, bub, H, act, stride, lane, G, U);
+  else if (R == 2) rows_a<NT, 2, F>(bgq, bgs, bgb, buq, bus, bub, H, act, stride, lane, G, U);
+  else if (R == 4) rows_a<NT, 4, F>(bgq, bgs, bgb, buq, bus, bub, H, act, stride, lane, G, U);
+  else if (R == 6) rows_a<NT, 6, F>(bgq, bgs, bgb, buq, bus, bub, H, act, stride, lane, G, U);
+  else rows_a<NT, 8, F>(bgq, bgs, bgb, buq, bus, bub, H, act, stride, lane, G, U);
 }
 
-template <int NT>
+template <int NT, int F>
 __device__ __forceinline__ float dispatch_b(int R, const unsigned char* bq, const uint16_t* bs,
                                             const uint16_t* bb, int row0, int nrows, int I,
                                             const unsigned char* act, unsigned stride, int lane,
                                             int& vid) {
-  if (R == 1) return rows_b<NT, 1>(bq, bs, bb, row0, nrows, I, act, stride, lane, vid);
-  if (R == 2) return rows_b<NT, 2>(bq, bs, bb, row0, nrows, I, act, stride, lane, vid);
-  if (R == 4) return rows_b<NT, 4>(bq, bs, bb, row0, nrows, I, act, stride, lane, vid);
-  return rows_b<NT, 8>(bq, bs, bb, row0, nrows, I, act, stride, lane, vid);
+  if (R == 1) return rows_b<NT, 1, F>(bq, bs, bb, row0, nrows, I, act, stride, lane, vid);
+  if (R == 2) return rows_b<NT, 2, F>(bq, bs, bb, row0, nrows, I, act, stride, lane, vid);
+  if (R == 4) return rows_b<NT, 4, F>(bq, bs, bb, row0, nrows, I, act, stride, lane, vid);
+  if (R == 6) return rows_b<NT, 6, F>(bq, bs, bb, row0, nrows, I, act, stride, lane, vid);
+  return rows_b<NT, 8, F>(bq, bs, bb, row0, nrows, I, act, stride, lane, vid);
 }
 
 // mbarrier phase test without suspending (for wait loops that do other work).
@@ -476,6 +554,7 @@ constexpr int kSlotActPar = 16;    // parity of that load's phase on act_full[or
 constexpr int kSlotActShift = 8;   // bits 8..: byte offset / 128 of the item's activation rows
 
 // 9 warps: 8 compute warps and one producer warp (see the top of this file).
+template <int F>
 __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_u, s_nseg;
@@ -566,7 +645,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       const int m = (int)(q & 3), tc = (int)(q >> 2), t = tc / nch, ch = tc % nch;
       const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H + ch * 32 + m * 8));
       uint4 packed;
-      const float2 sc = fixed_point_quarter(v, 0xfu << (lane & ~3), packed);
+      const float2 sc = fixed_point_quarter<F>(v, 0xfu << (lane & ~3), packed);
       unsigned char* row = a.xg + (size_t)t * stride_a;
       reinterpret_cast<uint4*>(row)[((ch / 32) * 4 + m) * 32 + (ch % 32)] = packed;
       if (m == 0) reinterpret_cast<float2*>(row + act_digit_bytes(R))[ch] = sc;
@@ -629,7 +708,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
             const uint4 v = *reinterpret_cast<const uint4*>(
                 hscr_p + ((pub + i) % kItemRing) * (kNT * 32) + t * 32 + m * 8);
             uint4 packed;
-            const float2 sc = fixed_point_quarter(v, 0xfu << (lane & ~3), packed);
+            const float2 sc = fixed_point_quarter<F>(v, 0xfu << (lane & ~3), packed);
             const int ch = ii.z / (32 / kRowsA), R = G.rounds_b;  // h chunk of the item
             unsigned char* row = a.hq + (size_t)(p0 + t) * stride_b;
             reinterpret_cast<uint4*>(row)[((ch / 32) * 4 + m) * 32 + (ch % 32)] = packed;
@@ -885,20 +964,20 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
             mbar_arrive_expect_tx(&full[st], G.a_bytes);
             bulk_g2s(buf, a.gq + r0 * qrow, G.a_q, &full[st]);
             bulk_g2s(buf + G.a_q, a.gs + r0 * srow, G.a_sb, &full[st]);
-            bulk_g2s(buf + G.a_q + G.a_sb, a.gb + r0 * srow, G.a_sb, &full[st]);
+            if (F != kFmtMx) bulk_g2s(buf + G.a_q + G.a_sb, a.gb + r0 * srow, G.a_sb, &full[st]);
             buf += G.a_mat;
             bulk_g2s(buf, a.uq + r0 * qrow, G.a_q, &full[st]);
             bulk_g2s(buf + G.a_q, a.us + r0 * srow, G.a_sb, &full[st]);
-            bulk_g2s(buf + G.a_q + G.a_sb, a.ub + r0 * srow, G.a_sb, &full[st]);
+            if (F != kFmtMx) bulk_g2s(buf + G.a_q + G.a_sb, a.ub + r0 * srow, G.a_sb, &full[st]);
           } else {
             const int nrows = min(G.rows_b, a.H - row0);
             const size_t r0 = (size_t)uniq[seg_slot[sg]] * a.H + row0;
             const size_t qrow = a.I / 8, srow = a.I / 64;
             const unsigned qb = nrows * (a.I / 2), sb = nrows * (a.I / 32);
-            mbar_arrive_expect_tx(&full[st], qb + 2 * sb);
+            mbar_arrive_expect_tx(&full[st], qb + (F == kFmtMx ? 1 : 2) * sb);
             bulk_g2s(buf, a.dq + r0 * qrow, qb, &full[st]);
             bulk_g2s(buf + G.b_q, a.ds + r0 * srow, sb, &full[st]);
-            bulk_g2s(buf + G.b_q + G.b_sb, a.db + r0 * srow, sb, &full[st]);
+            if (F != kFmtMx) bulk_g2s(buf + G.b_q + G.b_sb, a.db + r0 * srow, sb, &full[st]);
           }
         }
         __syncwarp();
@@ -976,20 +1055,20 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
         const uint16_t* bus = reinterpret_cast<const uint16_t*>(bu + G.a_q) + warp * (a.H / 64);
         const uint16_t* bub = reinterpret_cast<const uint16_t*>(bu + G.a_q + G.a_sb) + warp * (a.H / 64);
         switch (nt) {
-          case 1: dispatch_a<1>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, act, stride_a, lane, Gs, Us); break;
-          case 2: dispatch_a<2>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, act, stride_a, lane, Gs, Us); break;
-          case 3: dispatch_a<3>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, act, stride_a, lane, Gs, Us); break;
-          default: dispatch_a<4>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, act, stride_a, lane, Gs, Us); break;
+          case 1: dispatch_a<1, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, act, stride_a, lane, Gs, Us); break;
+          case 2: dispatch_a<2, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, act, stride_a, lane, Gs, Us); break;
+          case 3: dispatch_a<3, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, act, stride_a, lane, Gs, Us); break;
+          default: dispatch_a<4, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, act, stride_a, lane, Gs, Us); break;
         }
       } else {
         nrows = min(G.rows_b, a.H - row0);
         const uint16_t* bs = reinterpret_cast<const uint16_t*>(buf + G.b_q);
         const uint16_t* bb = reinterpret_cast<const uint16_t*>(buf + G.b_q + G.b_sb);
         switch (nt) {
-          case 1: v = dispatch_b<1>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
-          case 2: v = dispatch_b<2>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
-          case 3: v = dispatch_b<3>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
-          default: v = dispatch_b<4>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
+          case 1: v = dispatch_b<1, F>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
+          case 2: v = dispatch_b<2, F>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
+          case 3: v = dispatch_b<3, F>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
+          default: v = dispatch_b<4, F>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
         }
       }
       // this warp is done reading stage st

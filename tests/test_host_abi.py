@@ -18,7 +18,7 @@ HEADER = os.path.join(ROOT, "include", "moe_qeg.h")
 def declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_header_declares_the_entry_points():
@@ -26,7 +26,9 @@ def test_header_declares_the_entry_points():
     for n in ("moe_route_union", "moe_switchglu_forward", "moe_switchglu_forward_ws",
               "moe_workspace_size", "moe_read_device_status", "moe_status_str",
               "moe_select_path", "moe_workspace_layout", "moe_switchglu_forward_static",
-              "moe_router_topk"):
+              "moe_router_topk", "moe_switchglu_forward_mxfp4",
+              "moe_switchglu_forward_mxfp4_ws", "moe_workspace_size_mxfp4",
+              "moe_select_path_mxfp4"):
         assert n in names
 
 
@@ -65,6 +67,18 @@ def test_path_selection_without_launch():
     assert qeg.moe_select_path(4, 8, 2048, 4096, 2048) == 0  # too many experts
 
 
+def test_mxfp4_path_and_workspace():
+    """mxfp4 banks take the persistent kernel (GLM-5.2's 6144 x 2048 bank included) and
+    nothing else; the workspace matches the affine one on that path."""
+    for T in (1, 2, 4, 16):
+        assert qeg.moe_select_path_mxfp4(T, 8, 256, 6144, 2048) == 1
+        assert qeg.moe_select_path_mxfp4(T, 8, 288, 4096, 2048) == 1
+        assert qeg.moe_workspace_size_mxfp4(T, 8, 288, 4096, 2048) == \
+            qeg.moe_workspace_size(T, 8, 288, 4096, 2048)
+    assert qeg.moe_select_path_mxfp4(512, 8, 256, 4096, 2048) == 0
+    assert qeg.moe_workspace_size_mxfp4(0, 8, 256, 4096, 2048) == 0
+
+
 def test_workspace_size_and_layout():
     T, k, E, H, I = 4, 8, 288, 4096, 2048
     n = qeg.moe_workspace_size(T, k, E, H, I)
@@ -83,14 +97,14 @@ def test_workspace_size_and_layout():
 
 def test_workspace_follows_the_path():
     """The grouped path's workspace also holds the packed activations: x and h rows
-    for every pair position padded to 16 per expert, bf16; the persistent kernel's
-    does not grow with them."""
+    for every pair position padded to 16 per expert, bf16, and their fp32 group
+    sums; the persistent kernel's does not grow with them."""
     E, H, I = 256, 4096, 2048
     for T in (512, 2048):
         P = T * 8
         assert qeg.moe_select_path(T, 8, E, H, I) == 2
         pcap = P + 15 * min(E, P)
-        packed = 2 * (H + I) * pcap
+        packed = 2 * (H + I) * pcap + 4 * (H + I) // 64 * pcap
         lay = qeg.moe_workspace_layout(T, 8, E, H, I)
         assert lay["total"] >= lay["y"] + 4 * P * H + packed
     # the small-window path stays within the 4 MiB no-allocation scratch at T=16
