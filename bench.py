@@ -616,6 +616,46 @@ def our_arm(args, world, rank, local):
             "note": "42 launches of one layer (same bank, same routing) in a graph; L2 holds "
                     "part of the 113 MB between launches"}
         del ws3
+    # mxfp4 banks: GLM-5.2's routed bank (E=256, hidden 6144, intermediate 2048, e2m1
+    # codes with one e8m0 scale per 32 columns, 20,054,016 B per expert), drawn on the
+    # device; 42 chained layers with distinct adjacent-overlap routings (p = 0.34) per
+    # window size, CUDA graph; GB/s over unique-expert mxfp4 bytes
+    mxfp4 = None
+    if not args.no_mxfp4:
+        EM, HM, IM = 256, 6144, 2048
+        bpe_mx = 3 * (IM * HM // 2 + IM * HM // 32)
+
+        def matm(rows, cols, mid):
+            q = torch.empty((EM, rows, cols // 8), dtype=torch.int32, device=dev)
+            e8 = torch.empty((EM, rows, cols // 32), dtype=torch.uint8, device=dev)
+            synth.fill_bank_mxfp4_device(q, e8, rows, cols, SEED + 3, mid)
+            return q, e8
+        bank_mx = qeg.MxBank(*matm(IM, HM, 0), *matm(IM, HM, 1), *matm(HM, IM, 2))
+        mxfp4 = {"E": EM, "hidden": HM, "inter": IM, "bytes_per_expert": bpe_mx, "p": 0.34,
+                 "layers": LAYERS, "per_T": {}}
+        for TM in (1, 2, 4, 16):
+            rts = [synth.route_markov(TM, EM, K_TOP, 0.34, SEED + 7000 + 100 * TM + l)
+                   for l in range(LAYERS)]
+            xm = torch.from_numpy(synth.x_bf16(TM, HM, SEED + 60 + TM).view(np.int16)).to(dev) \
+                .view(torch.bfloat16)
+            im = [torch.from_numpy(r[0]).to(dev) for r in rts]
+            wm = [torch.from_numpy(r[1]).to(dev) for r in rts]
+            om = [torch.empty((TM, HM), dtype=torch.bfloat16, device=dev) for _ in rts]
+            wsm = torch.zeros(qeg.moe_workspace_size_mxfp4(TM, K_TOP, EM, HM, IM),
+                              dtype=torch.uint8, device=dev)
+            us = graph_us_per_layer(
+                lambda: [qeg.moe_switchglu_forward_mxfp4_ws(xm, im[l], wm[l], bank_mx, wsm,
+                                                            out=om[l]) for l in range(LAYERS)],
+                LAYERS)
+            um = float(np.mean([np.unique(r[0]).size for r in rts]))
+            gb = um * bpe_mx / (us * 1e-6) / 1e9
+            mxfp4["per_T"][str(TM)] = {"us_per_layer": us, "mean_unique": um, "gbs": gb,
+                                       "frac_of_hbm_peak": gb / measured_peaks()[0]}
+            del wsm
+        del bank_mx
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
     # large windows (the grouped tensor-core path): T=512 and T=2048 on the E=256 bank,
     # a few layers each, CUDA events; bytes = unique experts, flops = 6 P H I
     large = None
@@ -782,6 +822,7 @@ def our_arm(args, world, rank, local):
             "chained_parity": chained_parity,
             "verify_pair": verify,
             "verify_window": window,
+            "mxfp4": mxfp4,
             "large_window": large,
             "router": router,
             "gpu_launches": launches_per_step * args.steps,
@@ -806,6 +847,8 @@ def main():
                     help="skip the T=512 / T=2048 grouped-path measurement")
     ap.add_argument("--no-verify-pair", action="store_true",
                     help="skip the T=2 / T=1 speculative-verify measurement")
+    ap.add_argument("--no-mxfp4", action="store_true",
+                    help="skip the mxfp4 (GLM-5.2 bank) measurement")
     ap.add_argument("--no-window-sweep", action="store_true",
                     help="skip the verify-window sweep (T=2..16, 78-layer stacks)")
     ap.add_argument("--ts", default="", help="comma-separated window sizes (profiling)")

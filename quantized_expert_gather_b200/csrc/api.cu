@@ -93,7 +93,6 @@ bool shape_supported(int T, int k, int E, int hidden, int inter) {
 
 struct WsLayout {
   size_t barrier, num_unique, unique, offsets, pair_list, h, y;  // barrier = counters
-  size_t xg, hq;                         // fused kernel: x and h rows in fixed point
   size_t padded, xs, hs, xp, hp, pcap;   // grouped path: packed activations and sums
   size_t total;
 };
@@ -129,11 +128,7 @@ WsLayout ws_layout(int T, int k, int E, int hidden, int inter, int fmt = kFmtAff
   w.h = align_up(w.pair_list + 4 * P, 256);
   w.y = align_up(w.h + 2 * P * (size_t)inter, 256);
   const size_t tail = align_up(w.y + 4 * P * (size_t)hidden, 256);
-  // fused kernel
-  const LayerGeom g = layer_geom(hidden, inter);
-  w.xg = tail;                                                        // x rows, fixed point
-  w.hq = align_up(w.xg + (size_t)T * act_bytes(g.rounds_a), 256);     // h rows, fixed point
-  const size_t total1 = align_up(w.hq + P * act_bytes(g.rounds_b), 256);
+  const size_t total1 = tail;  // the persistent kernel needs nothing more
   // grouped path: every expert's pairs padded to 16 rows
   w.pcap = align_up(P + 15 * m, 16);
   w.padded = tail;
@@ -169,8 +164,6 @@ cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
   a.db = db;
   a.h = reinterpret_cast<uint16_t*>(ws + wl.h);
   a.y = reinterpret_cast<float*>(ws + wl.y);
-  a.xg = ws + wl.xg;
-  a.hq = ws + wl.hq;
   a.sync = reinterpret_cast<unsigned*>(ws + wl.barrier);
   a.ex_u = reinterpret_cast<int*>(ws + wl.num_unique);
   a.ex_unique = reinterpret_cast<int*>(ws + wl.unique);
@@ -184,6 +177,8 @@ cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
   a.I = I;
   a.g = layer_geom(H, I, F);
   a.wait_prior = 1;
+  // the window's x rows fit one activation buffer: held in each CTA's shared memory
+  a.x_res = (size_t)T * act_bytes(a.g.rounds_a) <= a.g.act_buf ? 1 : 0;
   const int ki = F == kFmtMx ? 9 : 0;  // dyn_smem index of this layer kernel
   if (a.g.seg < 1 || !fit_stages(a.g, E, T * k, H, I, (size_t)d.dyn_smem[ki])) {
     *why = MOE_ERR_UNSUPPORTED;

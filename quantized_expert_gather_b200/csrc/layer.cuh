@@ -8,35 +8,38 @@
 //
 //   prologue  route-union of the window (every CTA forms the same union in
 //             shared memory from topk_idx), cut into segments: an expert and up
-//             to `seg` of its pairs; the CTAs convert the window's x rows to
-//             block fixed point in the workspace, together;
-//   phase A   gate+up over items of 32 rows (segment, rows of Wg and Wu):
+//             to `seg` of its pairs.  A window whose x rows fit one activation
+//             buffer keeps them all in shared memory (converted while the union
+//             forms);
+//   phase A   gate+up over blocks of 8 rows (segment, rows of Wg and Wu):
 //               h = bf16(silu(bf16(Wg x)) * bf16(Wu x))
 //             (the one-pass epilogue of "Apple7/8 MoE gate and up in one decode
-//             pass", splash PR 45, "What changed"); the item's 32 h values per
-//             pair are one fixed-point chunk, converted at the item's end;
-//   phase B   down over items of rows_b rows of Wd: y = Wd h per pair, fp32.
-//             A segment's phase-B items start once every phase-A item of that
+//             pass", splash PR 45, "What changed"), h written to the workspace;
+//   phase B   down over blocks of rows_b rows of Wd: y = Wd h per pair, fp32.
+//             A segment's phase-B blocks start once every phase-A block of that
 //             segment has published (counter hdone[seg]);
 //   combine   out[t] = bf16(sum_j w[t,j] * y[t,j]) per block of rows_b output
 //             rows, by CTA (row block mod grid) once every segment of the row
 //             block has published (counter ydone[rb]).
-// Work items are taken from one list (all phase-A items, segment-major, then all
-// phase-B items) through a counter in the workspace, so CTAs stay balanced and a
-// phase-B item's h is normally complete long before the item is taken.  An
+// Each CTA takes a contiguous, balanced share of all phase-A blocks (segment
+// order), then of all phase-B blocks: every block carries the same bytes at the
+// 4096/2048 shape, so the CTAs stream equal shares and finish together, and a
+// CTA's share spans few segments, so its activation sets change rarely.  An
 // expert with more than `seg` pairs in the window forms several segments and is
 // streamed once per segment.  Every spin on a counter or barrier is bounded
 // (common.cuh); the counters are zero again when the kernel ends.
 //
-// Warps: 8 compute warps and one producer warp.  The producer takes work items,
-// issues every bulk copy (weights into a ring of stages, activation rows into
-// one of two activation buffers) and publishes finished items; the compute warps
-// wait only on mbarriers and, at the end of a phase-A item, on a named barrier.
+// Warps: 8 compute warps, one producer warp and one helper warp.  The producer
+// issues this CTA's weight blocks into a ring of stages (1-D bulk copies, mbarrier
+// completion); the helper publishes finished blocks to the other CTAs (counter
+// release reductions); the compute warps convert each new activation set (the
+// segment's x rows for phase A, its h rows for phase B) into shared memory
+// together and compute.
 //
 // Compute: each warp owns whole rows (phase A: one row of Wg and the same row
 // of Wu; phase B: up to 4 rows of Wd) over the full input width.  Lane l takes
 // the 32-column chunks l, l+32, ... of its rows, so one lane chunk sits inside
-// one quantisation group (64 columns):
+// one quantisation group (64 columns affine, 32 mxfp4):
 //     partial = s * sum_c q_c x_c + b * sum_c x_c.
 // Activations are 16-bit block fixed point (one exponent per 32-column chunk,
 // see below), so that sum_c q_c x_c is an exact integer dot product of the 4-bit
@@ -59,14 +62,13 @@ constexpr int kWarps = 8;                    // compute warps
 constexpr int kConsumerThreads = 32 * kWarps;
 constexpr int kThreads = kConsumerThreads + 64;  // + a producer warp and a helper warp
 constexpr int kRowsA = kWarps;      // phase A: one row of gate and of up per warp per block
-constexpr int kBlocksPerItemA = 4;  // phase-A item: 4 blocks = 32 rows = one h chunk
-constexpr int kBlocksPerItemB = 2;  // phase-B item: row blocks
 constexpr int kMaxRowsPerWarpB = 4; // phase B: rows of Wd per warp per block
 constexpr int kMaxStages = 4;       // ring depth (fewer when shared memory is short)
 constexpr int kNT = 4;              // pairs per segment (upper bound)
 constexpr int kMaxPairsFused = 1024;
 constexpr unsigned kSegActBytes = 36 * 1024;  // one activation buffer (a segment's rows)
-constexpr int kItemRing = 16;       // items between compute and publication
+constexpr unsigned kBarUnion = 1;   // named barrier: union formed (warp 0 -> producer)
+constexpr unsigned kBarWork = 2;    // named barrier: every warp but the producer
 // Dynamic shared memory the kernel may plan for on B200 (227 KB per block, less a
 // margin for its static shared memory).
 constexpr size_t kSmemBudget = 232448 - 1024;
@@ -126,7 +128,7 @@ __host__ __device__ inline LayerGeom layer_geom(int H, int I, int fmt = kFmtAffi
 }
 
 struct LayerSmem {
-  size_t stages, act, hscr, cnt, rank, unique, offsets, pair_list, pos_of, seg_slot, seg_pos,
+  size_t stages, act, cnt, rank, unique, offsets, pair_list, pos_of, seg_slot, seg_pos,
       seg_nt, total;
 };
 __host__ __device__ inline LayerSmem layer_smem(const LayerGeom& g, int E, int P, int H, int I) {
@@ -134,8 +136,7 @@ __host__ __device__ inline LayerSmem layer_smem(const LayerGeom& g, int E, int P
   const int m = (E < P ? E : P) > 0 ? (E < P ? E : P) : 1;
   s.stages = 0;
   s.act = align_up((size_t)g.stages * g.stage_bytes, 128);    // two activation buffers
-  s.hscr = s.act + 2 * (size_t)g.act_buf;  // bf16 h of phase-A items, per item ring slot
-  s.cnt = align_up(s.hscr + sizeof(uint16_t) * kItemRing * kNT * 32, 16);
+  s.cnt = align_up(s.act + 2 * (size_t)g.act_buf, 16);
   s.rank = align_up(s.cnt + sizeof(int) * E, 16);
   s.unique = align_up(s.rank + sizeof(int) * P, 16);
   s.offsets = align_up(s.unique + sizeof(int) * m, 16);
@@ -179,14 +180,14 @@ struct LayerArgs {
   const uint16_t *gs, *gb, *us, *ub, *ds, *db;
   uint16_t* h;        // workspace [P, I] bf16, rows in pair_list order
   float* y;           // workspace [P, H] fp32, rows in pair_list order
-  unsigned char* xg;  // workspace: x rows in the fixed-point layout, [T] x act_bytes(rounds_a)
-  unsigned char* hq;  // workspace: h rows in the fixed-point layout, [P] x act_bytes(rounds_b)
   unsigned* sync;     // workspace counters (kSyncWords)
   int *ex_u, *ex_unique, *ex_offsets, *ex_pair_list;  // union export (CTA 0), may be null
   uint16_t* out;      // [T, H] bf16
   int T, k, E, H, I;
   LayerGeom g;
   int wait_prior;     // wait for the preceding grid before reading any input
+  int x_res;          // every x row of the window fits one activation buffer: each CTA
+                      // keeps them all in shared memory for phase A
 };
 
 // ------------------------------------------------- activations and codes ---
@@ -198,16 +199,18 @@ struct LayerArgs {
 // rounded to the nearest multiple of 2^(e - 14), an error below 2^-15 of the
 // block's largest magnitude.  v_c is split into a low byte (unsigned) and a high
 // byte (signed), so that a chunk's sum  sum_c q_c v_c  is formed exactly in
-// integers by dp4a over 4-bit codes: the codes of a 32-bit word w are split into
-// qa = w & 0x0F0F0F0F (columns 0, 2, 4, 6 of the word, one per byte) and
-// qb = (w >> 4) & 0x0F0F0F0F (columns 1, 3, 5, 7).
+// integers by dp4a over 4-bit codes: the affine codes of a 32-bit word w are split
+// into qa = w & 0x0F0F0F0F (columns 0, 2, 4, 6 of the word, one per byte) and
+// qb = w & 0xF0F0F0F0 (columns 1, 3, 5, 7, each as 16 q); mxfp4 codes become bytes
+// by table lookup in column order 0..3 and 4..7 (split_codes_mx).
 //
 // Layout of one activation row (a token's x or a pair's h) of D columns, R rounds
-// (R a power of two >= D / 1024), in act_bytes(R) = 2304 R bytes: for chunk
-// ch = i * 32 + l (i < R, l < 32) the uint4 at index (i * 4 + m) * 32 + l covers
-// columns 32 ch + 8m .. +7 as
+// (R >= D / 1024), in act_bytes(R) = 2304 R bytes: for chunk ch = i * 32 + l
+// (i < R, l < 32) the uint4 at index (i * 4 + m) * 32 + l covers columns
+// 32 ch + 8m .. +7 as (affine)
 //   .x = low bytes of columns 8m+0,2,4,6   .y = low bytes of 8m+1,3,5,7
 //   .z = high bytes of columns 8m+0,2,4,6  .w = high bytes of 8m+1,3,5,7
+// or (mxfp4) .x / .z = low / high bytes of columns 8m+0..3, .y / .w of 8m+4..7,
 // followed (at byte 2048 R) by float2 sc[ch] = (2^(e - 14), sum of the chunk's 32
 // values).  The same layout serves in global memory (converted once per call) and
 // in shared memory (copied per work item).
@@ -217,7 +220,9 @@ __device__ __forceinline__ int dp4a_lo(uint32_t q, uint32_t d, int c) {
   return static_cast<int>(__dp4a(q, d, static_cast<unsigned>(c)));
 }
 __device__ __forceinline__ int dp4a_hi(uint32_t q, uint32_t d, int c) {
-  return __dp4a(static_cast<int>(q), static_cast<int>(d), c);
+  int r;  // unsigned code bytes times signed activation bytes
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(r) : "r"(q), "r"(d), "r"(c));
+  return r;
 }
 
 
@@ -233,7 +238,10 @@ __device__ __forceinline__ float2 load_sc(const unsigned char* row, int R, int c
 }
 
 // sum_c q_c v_c over one chunk (4 code words, 4 activation uint4), exact.  Four
-// partial sums keep the dp4a dependency chains short.
+// partial sums keep the dp4a dependency chains short.  In the affine format the
+// odd codes stay in the high nibble of their byte (16 q, see split_codes), so the
+// affine result is 16 * sum q v (|.| < 2^28; the chunk scale carries the 1/16).
+template <int F>
 __device__ __forceinline__ int chunk_dot(const uint32_t (&qs)[8], const uint4 (&x)[4]) {
   int lo0 = 0, lo1 = 0, hi0 = 0, hi1 = 0;
 #pragma unroll
@@ -244,16 +252,19 @@ __device__ __forceinline__ int chunk_dot(const uint32_t (&qs)[8], const uint4 (&
     hi0 = dp4a_hi(qs[2 * m], d.z, hi0);
     hi1 = dp4a_hi(qs[2 * m + 1], d.w, hi1);
   }
-  return (hi0 + hi1) * 256 + (lo0 + lo1);  // |.| < 2^24: exact in fp32
+  if constexpr (F == kFmtMx) return (hi0 + hi1) * 256 + (lo0 + lo1);
+  else return (((hi0 << 4) + hi1) << 8) + ((lo0 << 4) + lo1);
 }
 
-// The 32 codes of a uint4, split as described above (affine format).
+// The 32 codes of a uint4, split as described above (affine format), except that
+// the odd codes are left in the high nibble of their byte: qs[2m+1] = w & 0xF0F0F0F0
+// holds 16 q per byte (one operation less per word; chunk_dot accounts for it).
 __device__ __forceinline__ void split_codes(const uint4 v, uint32_t (&qs)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
     qs[2 * m] = w[m] & kNibbleBytes;
-    qs[2 * m + 1] = (w[m] >> 4) & kNibbleBytes;
+    qs[2 * m + 1] = w[m] & ~kNibbleBytes;
   }
 }
 
@@ -308,7 +319,8 @@ __device__ __forceinline__ float2 chunk_sb(const uint16_t* s, const uint16_t* b,
     const float h = mx_half_scale(reinterpret_cast<const uint8_t*>(s)[ch]);
     return make_float2(h, -12.0f * h);
   } else {
-    return make_float2(bf16_bits_to_float(s[ch >> 1]), bf16_bits_to_float(b[ch >> 1]));
+    // chunk_dot returns 16 x the sum in this format
+    return make_float2(bf16_bits_to_float(s[ch >> 1]) * 0.0625f, bf16_bits_to_float(b[ch >> 1]));
   }
 }
 
@@ -403,7 +415,7 @@ template <int NT, int R, int F>
 __device__ __forceinline__ void rows_a(const unsigned char* bg_q, const uint16_t* bg_s,
                                        const uint16_t* bg_b, const unsigned char* bu_q,
                                        const uint16_t* bu_s, const uint16_t* bu_b, int H,
-                                       const unsigned char* act, unsigned stride, int lane,
+                                       const unsigned char* const (&act)[kNT], int lane,
                                        float (&G)[kNT], float (&U)[kNT]) {
   float ag[NT], au[NT];
 #pragma unroll
@@ -421,12 +433,12 @@ __device__ __forceinline__ void rows_a(const unsigned char* bg_q, const uint16_t
       const float sg = sbg.x, bgv = sbg.y, su = sbu.x, buv = sbu.y;
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
-        const unsigned char* row = act + t * stride;
+        const unsigned char* row = act[t];
         uint4 xd[4];
         load_xq(row, i, lane, xd);
         const float2 sc = load_sc(row, R, ch);
-        const float dg = static_cast<float>(chunk_dot(qg, xd));
-        const float du = static_cast<float>(chunk_dot(qu, xd));
+        const float dg = static_cast<float>(chunk_dot<F>(qg, xd));
+        const float du = static_cast<float>(chunk_dot<F>(qu, xd));
         ag[t] = fmaf(sg * sc.x, dg, fmaf(bgv, sc.y, ag[t]));
         au[t] = fmaf(su * sc.x, du, fmaf(buv, sc.y, au[t]));
       }
@@ -482,7 +494,7 @@ __device__ __forceinline__ float rows_b(const unsigned char* bq, const uint16_t*
           const float sv = sb.x, bv = sb.y;
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
-            const float d = static_cast<float>(chunk_dot(qs, xd[t]));
+            const float d = static_cast<float>(chunk_dot<F>(qs, xd[t]));
             acc[q * NP + t] = fmaf(sv * sc[t].x, d, fmaf(bv, sc[t].y, acc[q * NP + t]));
           }
         }
@@ -501,13 +513,13 @@ template <int NT, int F>
 __device__ __forceinline__ void dispatch_a(int R, const unsigned char* bgq, const uint16_t* bgs,
                                            const uint16_t* bgb, const unsigned char* buq,
                                            const uint16_t* bus, const uint16_t* bub, int H,
-                                           const unsigned char* act, unsigned stride, int lane,
+                                           const unsigned char* const (&act)[kNT], int lane,
                                            float (&G)[kNT], float (&U)[kNT]) {
-  if (R == 1) rows_a<NT, 1, F>(bgq, bgs, bgb, buq, bus, bub, H, act, stride, lane, G, U);
-  else if (R == 2) rows_a<NT, 2, F>(bgq, bgs, bgb, buq, bus, bub, H, act, stride, lane, G, U);
-  else if (R == 4) rows_a<NT, 4, F>(bgq, bgs, bgb, buq, bus, bub, H, act, stride, lane, G, U);
-  else if (R == 6) rows_a<NT, 6, F>(bgq, bgs, bgb, buq, bus, bub, H, act, stride, lane, G, U);
-  else rows_a<NT, 8, F>(bgq, bgs, bgb, buq, bus, bub, H, act, stride, lane, G, U);
+  if (R == 1) rows_a<NT, 1, F>(bgq, bgs, bgb, buq, bus, bub, H, act, lane, G, U);
+  else if (R == 2) rows_a<NT, 2, F>(bgq, bgs, bgb, buq, bus, bub, H, act, lane, G, U);
+  else if (R == 4) rows_a<NT, 4, F>(bgq, bgs, bgb, buq, bus, bub, H, act, lane, G, U);
+  else if (R == 6) rows_a<NT, 6, F>(bgq, bgs, bgb, buq, bus, bub, H, act, lane, G, U);
+  else rows_a<NT, 8, F>(bgq, bgs, bgb, buq, bus, bub, H, act, lane, G, U);
 }
 
 template <int NT, int F>
@@ -546,29 +558,49 @@ __device__ __forceinline__ bool lane0(bool v) { return __shfl_sync(kFull, v ? 1 
 __device__ __forceinline__ int lane0_int(int v) { return __shfl_sync(kFull, v, 0); }
 
 // Ring-slot descriptor flags (slot_info[st].x) for the compute warps.
-constexpr int kSlotEnd = 1;        // no more blocks
-constexpr int kSlotPhaseB = 2;     // a phase-B block
-constexpr int kSlotItemEnd = 4;    // last block of its work item
-constexpr int kSlotActWait = 8;    // first block of an item whose activation rows were loaded
-constexpr int kSlotActPar = 16;    // parity of that load's phase on act_full[ord % kItemRing]
-constexpr int kSlotActShift = 8;   // bits 8..: byte offset / 128 of the item's activation rows
+constexpr int kSlotEnd = 1;       // no more blocks
+constexpr int kSlotPhaseB = 2;    // a phase-B block
+constexpr int kSlotNewSet = 4;    // the first block that reads a new activation set
+constexpr int kPubRing = 16;      // blocks between compute and publication
 
-// 9 warps: 8 compute warps and one producer warp (see the top of this file).
+// Activation set (the rows of one segment's pairs) into `buf`, by the 8 compute warps
+// (256 threads): phase A converts the pairs' token rows of x, phase B the pairs' rows
+// of h (written by other CTAs; read around L1).  Four consecutive lanes convert one
+// 32-column chunk together.
+template <int F>
+__device__ __forceinline__ void convert_set(const LayerArgs& a, const LayerGeom& G, bool phase_b,
+                                            const int* plist, int p0, int nt,
+                                            unsigned char* buf, int lane) {
+  const int D = phase_b ? a.I : a.H, R = phase_b ? G.rounds_b : G.rounds_a, nch = D / 32;
+  const unsigned stride = act_bytes(R);
+  const int nq = nt * nch * 4;  // quarters of 8 columns
+  for (int q = threadIdx.x; q < nq; q += kConsumerThreads) {
+    const int m = q & 3, tc = q >> 2, t = tc / nch, ch = tc % nch;
+    uint4 v;
+    if (phase_b)
+      v = __ldcg(reinterpret_cast<const uint4*>(a.h + (size_t)(p0 + t) * a.I + ch * 32 + m * 8));
+    else
+      v = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)(plist[p0 + t] / a.k) * a.H +
+                                               ch * 32 + m * 8));
+    uint4 packed;
+    const float2 sc = fixed_point_quarter<F>(v, 0xfu << (lane & ~3), packed);
+    unsigned char* row = buf + (size_t)t * stride;
+    reinterpret_cast<uint4*>(row)[((ch / 32) * 4 + m) * 32 + (ch % 32)] = packed;
+    if (m == 0) reinterpret_cast<float2*>(row + act_digit_bytes(R))[ch] = sc;
+  }
+}
+
+// 10 warps: 8 compute warps, a producer warp and a helper warp (see the top of this file).
 template <int F>
 __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_u, s_nseg;
   __shared__ volatile int s_abort;
-  // producer <-> helper: items recorded / published, activation loads queued / issued,
-  // producer finished
-  __shared__ volatile int s_nrec, s_pub, s_pend_tail, s_pend_head, s_prod_done;
+  __shared__ volatile int s_pub;  // blocks published by the helper warp
   __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
-  __shared__ __align__(8) uint64_t act_full[kItemRing], item_done[kItemRing];
-  __shared__ unsigned long long reg_start[kItemRing];  // activation regions (producer)
-  __shared__ int reg_last[kItemRing];
-  __shared__ int4 item_info[kItemRing];  // per item ordinal: phase B, segment, first block, blocks
-  __shared__ int4 pend[kItemRing];       // queued activation loads (producer)
-  __shared__ int4 slot_info[kMaxStages];  // per ring slot: flags, segment, first row, item ordinal
+  __shared__ __align__(8) uint64_t done[kPubRing];           // a block's outputs written
+  __shared__ __align__(8) uint64_t set_in[1], set_out[1];    // activation-set hand-over
+  __shared__ int4 slot_info[kMaxStages];  // per ring slot: flags, segment, first row, block
   const LayerGeom& G = a.g;
   const int P = a.T * a.k;
   const int NS = G.stages;
@@ -577,8 +609,6 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
   unsigned* exit_cnt = a.sync;
   unsigned* hdone = a.sync + 1;
   unsigned* ydone = a.sync + 1 + kMaxPairsFused;
-  unsigned* work_ctr = a.sync + kSyncWorkItem;
-  unsigned* xdone = a.sync + kSyncXDone;
   const unsigned stride_a = act_bytes(G.rounds_a), stride_b = act_bytes(G.rounds_b);
 
   if (threadIdx.x == 0) {
@@ -586,12 +616,11 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kWarps);
     }
-    for (int i = 0; i < kItemRing; ++i) {
-      mbar_init(&act_full[i], 1);
-      mbar_init(&item_done[i], kWarps);
-    }
+    for (int i = 0; i < kPubRing; ++i) mbar_init(&done[i], kWarps);
+    mbar_init(&set_in[0], kWarps);
+    mbar_init(&set_out[0], kWarps);
     s_abort = 0;
-    s_nrec = s_pub = s_pend_tail = s_pend_head = s_prod_done = 0;
+    s_pub = 0;
     fence_barrier_init();
   }
   if (a.wait_prior) grid_dep_wait();
@@ -604,6 +633,9 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
   int* seg_slot = reinterpret_cast<int*>(smem + L.seg_slot);
   int* seg_pos = reinterpret_cast<int*>(smem + L.seg_pos);
   int* seg_nt = reinterpret_cast<int*>(smem + L.seg_nt);
+  // resident x rows (x_res): the start of the activation area
+  unsigned char* xres = smem + L.act;
+  const int wt = warp < kWarps ? (int)threadIdx.x : (int)threadIdx.x - 32;  // 0..287 but the producer
   if (warp == 0) {
     int nv;
     const int u = warp_route_union(a.idx, P, a.E, reinterpret_cast<int*>(smem + L.cnt),
@@ -632,34 +664,40 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       s_u = u;
       s_nseg = base;
     }
-  } else {
-    for (int p = threadIdx.x - 32; p < P; p += kThreads - 32) pos_of[p] = -1;
+    __syncwarp();
+    named_barrier_arrive(kBarUnion, 64);  // the producer may start (it waits on this)
+  } else if (warp != kWarps) {
+    // warps 1..7 and the helper: 256 threads
+    for (int p = wt - 32; p < P; p += kThreads - 64) pos_of[p] = -1;
   }
 
-  // ---- x rows in the fixed-point layout, converted by all CTAs together ----
-  {
-    const int nch = a.H / 32, R = G.rounds_a;
-    const long long nq = (long long)a.T * nch * 4;  // quarters of 8 columns
-    for (long long q = (long long)blockIdx.x * kThreads + threadIdx.x; q < nq + 0;
-         q += (long long)gridDim.x * kThreads) {
-      const int m = (int)(q & 3), tc = (int)(q >> 2), t = tc / nch, ch = tc % nch;
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H + ch * 32 + m * 8));
-      uint4 packed;
-      const float2 sc = fixed_point_quarter<F>(v, 0xfu << (lane & ~3), packed);
-      unsigned char* row = a.xg + (size_t)t * stride_a;
-      reinterpret_cast<uint4*>(row)[((ch / 32) * 4 + m) * 32 + (ch % 32)] = packed;
-      if (m == 0) reinterpret_cast<float2*>(row + act_digit_bytes(R))[ch] = sc;
+  // ---- a window whose x rows fit one activation buffer keeps them all here, converted
+  // by warps 1..7 and the helper while warp 0 forms the union ----
+  if (warp != kWarps) {
+    if (a.x_res && warp != 0) {
+      const int nch = a.H / 32, R = G.rounds_a;
+      const int nq = a.T * nch * 4;  // quarters of 8 columns
+      for (int q = wt - 32; q < nq; q += kThreads - 64) {
+        const int m = q & 3, tc = q >> 2, t = tc / nch, ch = tc % nch;
+        const uint4 v =
+            __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H + ch * 32 + m * 8));
+        uint4 packed;
+        const float2 sc = fixed_point_quarter<F>(v, 0xfu << (lane & ~3), packed);
+        unsigned char* row = xres + (size_t)t * stride_a;
+        reinterpret_cast<uint4*>(row)[((ch / 32) * 4 + m) * 32 + (ch % 32)] = packed;
+        if (m == 0) reinterpret_cast<float2*>(row + act_digit_bytes(R))[ch] = sc;
+      }
     }
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    red_release_gpu(xdone, 1u);
+    named_barrier(kBarWork, kThreads - 32);  // every warp but the producer
+  } else {
+    named_barrier(kBarUnion, 64);  // the union is formed
   }
   const int u = s_u, nseg = s_nseg;
   const int n_valid = offs[u];
-  for (int i = threadIdx.x; i < n_valid; i += kThreads) pos_of[plist[i]] = i;
-  __syncthreads();
+  if (warp != kWarps) {
+    for (int i = wt; i < n_valid; i += kThreads - 32) pos_of[plist[i]] = i;
+    named_barrier(kBarWork, kThreads - 32);
+  }
 
   if (blockIdx.x == 0 && warp == 1 && a.ex_u) {
     for (int i = lane; i < u; i += 32) a.ex_unique[i] = uniq[i];
@@ -668,110 +706,50 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
     if (lane == 0) *a.ex_u = u;
   }
 
+  // ---- this CTA's blocks: a contiguous, balanced share of the phase-A blocks (kRowsA
+  // rows of gate and of up each), then of the phase-B blocks (rows_b rows of down
+  // each), both in segment order.  Every block is 2 kRowsA H/2 + scales (A) or
+  // rows_b I/2 + scales (B) bytes; the two are equal at the 4096/2048 shape ----
   const int bpe_a = a.I / kRowsA;                     // phase-A blocks per segment
-  const int ipa = bpe_a / kBlocksPerItemA;            // phase-A items per segment
   const int bpe_b = (a.H + G.rows_b - 1) / G.rows_b;  // phase-B blocks per segment
-  // phase-B items: kBlocksPerItemB blocks each, except in the last quarter of the
-  // segments, where single blocks keep the CTAs' finishing times close
-  const int ipb = (bpe_b + kBlocksPerItemB - 1) / kBlocksPerItemB;
-  const int seg_fine = nseg - (nseg + 3) / 4;  // first segment with single-block items
-  const int n_items_a = nseg * ipa;
-  const int n_items_b2 = seg_fine * ipb;
-  const int n_items = n_items_a + n_items_b2 + (nseg - seg_fine) * bpe_b;
+  const long long NA = (long long)nseg * bpe_a, NB = (long long)nseg * bpe_b;
+  const int a0 = (int)(NA * blockIdx.x / gridDim.x), a1 = (int)(NA * (blockIdx.x + 1) / gridDim.x);
+  const int b0 = (int)(NB * blockIdx.x / gridDim.x), b1 = (int)(NB * (blockIdx.x + 1) / gridDim.x);
+  const int nA = a1 - a0, nblk = nA + (b1 - b0);
+  auto block_of = [&](int j, bool& pb, int& sg, int& row0) {
+    if (j < nA) {
+      const int blk = a0 + j;
+      pb = false;
+      sg = blk / bpe_a;
+      row0 = (blk % bpe_a) * kRowsA;
+    } else {
+      const int blk = b0 + (j - nA);
+      pb = true;
+      sg = blk / bpe_b;
+      row0 = (blk % bpe_b) * G.rows_b;
+    }
+  };
 
   if (warp == kWarps + 1) {
     // ================================ helper warp ================================
-    // Publishes finished items in order (converting each phase-A item's h chunk to
-    // the fixed-point layout first) and issues the queued activation loads once what
-    // they read is complete.  Every condition is lane 0's (uniform control flow).
-    const uint16_t* hscr_p = reinterpret_cast<const uint16_t*>(smem + L.hscr);
-    int pub = 0, ph = 0;  // items published; queued loads issued
-    bool x_ready = false;
+    // Publishes finished blocks in order: a phase-A block adds 1 to hdone of its segment
+    // (its h rows written), a phase-B block adds 1 to ydone of its row block.  The
+    // compute warps' done arrivals released their stores at CTA scope and the test
+    // below acquires them; the device-scope release reductions pass them on
+    // (causality order is transitive across the two scopes).
     unsigned long long t_prog = globaltimer();
-    for (;;) {
-      bool progressed = false;
-      // ---- publish ----
-      const int n_rec = lane0_int(s_nrec);
-      __threadfence_block();  // item_info of the recorded items is read after the count
-      int n = 0;
-      while (pub + n < n_rec &&
-             lane0(mbar_test(&item_done[(pub + n) % kItemRing], ((pub + n) / kItemRing) & 1)))
-        ++n;
-      if (n > 0) {
-        // a phase-A item's 32 h rows per pair are one chunk of h (lanes 4t..4t+3: pair t)
-        for (int i = 0; i < n; ++i) {
-          const int4 ii = item_info[(pub + i) % kItemRing];
-          if (ii.x != 0) continue;
-          const int nt = seg_nt[ii.y], p0 = seg_pos[ii.y];
-          if (lane < nt * 4) {
-            const int t = lane >> 2, m = lane & 3;
-            const uint4 v = *reinterpret_cast<const uint4*>(
-                hscr_p + ((pub + i) % kItemRing) * (kNT * 32) + t * 32 + m * 8);
-            uint4 packed;
-            const float2 sc = fixed_point_quarter<F>(v, 0xfu << (lane & ~3), packed);
-            const int ch = ii.z / (32 / kRowsA), R = G.rounds_b;  // h chunk of the item
-            unsigned char* row = a.hq + (size_t)(p0 + t) * stride_b;
-            reinterpret_cast<uint4*>(row)[((ch / 32) * 4 + m) * 32 + (ch % 32)] = packed;
-            if (m == 0) reinterpret_cast<float2*>(row + act_digit_bytes(R))[ch] = sc;
-          }
-        }
-        __syncwarp();  // the lanes' hq writes precede lane 0's release below
-        // The compute warps' item_done arrivals released their stores at CTA scope and
-        // the tests above acquired them; the device-scope release reductions pass them
-        // on (causality order is transitive across the two scopes).
+    for (int j = 0; j < nblk;) {
+      if (lane0(mbar_test(&done[j % kPubRing], (j / kPubRing) & 1))) {
+        bool pb;
+        int sg, row0;
+        block_of(j, pb, sg, row0);
         if (lane == 0) {
-          for (int i = 0; i < n; ++i) {
-            const int4 ii = item_info[(pub + i) % kItemRing];
-            if (ii.x == 0) {
-              red_release_gpu(&hdone[ii.y], (unsigned)ii.w);
-            } else {
-              for (int r = 0; r < ii.w; ++r) red_release_gpu(&ydone[ii.z + r], 1u);
-            }
-          }
-          __threadfence_block();
-          s_pub = pub + n;  // the producer frees ring slots and activation regions
+          if (!pb) red_release_gpu(&hdone[sg], 1u);
+          else red_release_gpu(&ydone[row0 / G.rows_b], 1u);
+          s_pub = j + 1;
         }
         __syncwarp();
-        pub += n;
-        progressed = true;
-      }
-      // ---- queued activation loads, in order ----
-      while (ph < lane0_int(s_pend_tail)) {
-        __threadfence_block();  // the entry is read after the count
-        const int4 pe = pend[ph % kItemRing];  // (ord, sg, byte offset, phase B | parity << 1)
-        const int sg = pe.y, nt = seg_nt[pe.y], p0 = seg_pos[pe.y];
-        const bool pb = (pe.w & 1) != 0;
-        if (pb) {
-          if (!lane0(ld_acquire_gpu(&hdone[sg]) >= (unsigned)bpe_a)) break;
-        } else if (!x_ready) {
-          if (!lane0(ld_acquire_gpu(xdone) >= gridDim.x)) break;
-          x_ready = true;
-        }
-        if (lane == 0) {
-          uint64_t* bar = &act_full[pe.x % kItemRing];
-          unsigned char* dst = smem + L.act + pe.z;
-          fence_proxy_async_all();  // rows other CTAs wrote, read by the bulk copy
-          if (pb) {
-            const unsigned size = (unsigned)nt * stride_b;
-            mbar_arrive_expect_tx(bar, size);
-            bulk_g2s(dst, a.hq + (size_t)p0 * stride_b, size, bar);
-          } else {
-            mbar_arrive_expect_tx(bar, (unsigned)nt * stride_a);
-            for (int t = 0; t < nt; ++t)
-              bulk_g2s(dst + (size_t)t * stride_a,
-                       a.xg + (size_t)(plist[p0 + t] / a.k) * stride_a, stride_a, bar);
-          }
-          __threadfence_block();
-          s_pend_head = ph + 1;
-        }
-        __syncwarp();
-        ++ph;
-        progressed = true;
-      }
-      // ---- done, or wait (bounded without progress) ----
-      if (lane0(s_prod_done != 0) && pub == lane0_int(s_nrec) && ph == lane0_int(s_pend_tail))
-        break;
-      if (progressed) {
+        ++j;
         t_prog = globaltimer();
       } else {
         if (lane0(s_abort != 0)) break;
@@ -787,9 +765,8 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
     }
   } else if (warp == kWarps) {
     // =============================== producer warp ===============================
-    // Takes items, places their activation rows in a circular byte ring (queueing
-    // the load for the helper warp) and issues their weight blocks into the stage
-    // ring.  Every condition is lane 0's (uniform control flow).
+    // Issues this CTA's blocks into the stage ring, in order.  Every condition is lane
+    // 0's (uniform control flow).
     auto timed_out = [&](unsigned long long t0) -> bool {
       if (lane0(s_abort != 0)) return true;
       if (lane0(globaltimer() - t0 > kWaitLimitNs)) {
@@ -801,213 +778,74 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       }
       return false;
     };
-    // An item's rows occupy a region [start, start + size) of virtual positions of the
-    // ring until the last item using them is published.  Regions are freed in order.
-    const unsigned long long ring = 2ull * G.act_buf;
-    unsigned long long head = 0, tail = 0;
-    int reg_front = 0, reg_cnt = 0;
-    auto free_regions = [&]() {
-      const int pub = lane0_int(s_pub);
-      while (reg_cnt > 0 && reg_last[reg_front] < pub) {
-        reg_front = (reg_front + 1) % kItemRing;
-        --reg_cnt;
-        tail = reg_cnt > 0 ? reg_start[reg_front] : head;
-      }
-    };
     bool ok = true;
-    int gi = 0;                     // blocks issued into the ring
-    int cur_key = -1;               // activation set of the newest region
-    int cur_tok[kNT] = {-1, -1, -1, -1};
-    unsigned cur_off = 0;           // its byte offset in the ring
-    unsigned long long cur_start = 0;  // and its virtual position
-    unsigned act_par = 0;           // per item ring slot: parity of its next load's phase
-    int pend_tail = 0;              // loads queued
-    int n_a_items = 0;              // phase-A items taken
-    unsigned q0 = 0, q1 = 0;        // items taken ahead (two atomics in flight)
-    if (lane == 0) {
-      q0 = atomicAdd(work_ctr, 1u);
-      q1 = atomicAdd(work_ctr, 1u);
-    }
-    for (int ord = 0; ok; ++ord) {
-      const int item = (int)__shfl_sync(kFull, q0, 0);
-      if (item >= n_items) break;
-      if (lane == 0) {
-        q0 = q1;
-        q1 = atomicAdd(work_ctr, 1u);
-      }
-      const bool phase_b = item >= n_items_a;
-      int sg, blk0, nblk;
-      if (!phase_b) {
-        sg = item / ipa;
-        blk0 = (item % ipa) * kBlocksPerItemA;
-        nblk = kBlocksPerItemA;
-      } else {
-        const int j = item - n_items_a;
-        if (j < n_items_b2) {
-          sg = j / ipb;
-          blk0 = (j % ipb) * kBlocksPerItemB;
-          nblk = min(kBlocksPerItemB, bpe_b - blk0);
-        } else {
-          sg = seg_fine + (j - n_items_b2) / bpe_b;
-          blk0 = (j - n_items_b2) % bpe_b;
-          nblk = 1;
-        }
-      }
-      const int nt = seg_nt[sg], p0 = seg_pos[sg];
-      // ---- its ring slot for publication must be free ----
-      {
+    int prev_set = -1;  // activation set of the previous block (-1: resident x)
+    int j = 0;
+    for (; j <= nblk && ok; ++j) {
+      const int st = j % NS;
+      if (j >= NS) {  // the compute warps are done with block j - NS
         const unsigned long long t0 = globaltimer();
-        while (ok && lane0_int(s_pub) <= ord - kItemRing) {
-          if (timed_out(t0)) ok = false;
-          __nanosleep(64);
-        }
-      }
-      if (!ok) break;
-      // ---- the item's activation rows: the newest region again, or a new one ----
-      bool same = false;
-      if (!phase_b) {
-        same = cur_key == -2;
-        for (int t = 0; t < kNT; ++t)
-          same = same && cur_tok[t] == (t < nt ? plist[p0 + t] / a.k : -1);
-      } else {
-        same = cur_key == sg;
-      }
-      bool act_wait = false, load_par = false;
-      free_regions();
-      if (same) {  // extend the newest region's life (it may already have been freed)
-        if (lane == 0) {
-          const int r = (reg_front + reg_cnt + (reg_cnt == 0 ? 0 : -1) + kItemRing) % kItemRing;
-          if (reg_cnt == 0) reg_start[r] = cur_start;
-          reg_last[r] = ord;
-        }
-        __syncwarp();
-        if (reg_cnt == 0) {
-          tail = cur_start;
-          reg_cnt = 1;
-        }
-      } else {
-        const unsigned size = (unsigned)nt * (phase_b ? stride_b : stride_a);
-        unsigned long long start = 0;
-        {
-          const unsigned long long t0 = globaltimer();
-          for (;;) {
-            start = head;
-            if (start % ring + size > ring) start = (start / ring + 1) * ring;  // no wrap
-            if (start + size - tail <= ring && reg_cnt < kItemRing &&
-                pend_tail - lane0_int(s_pend_head) < kItemRing)
-              break;
-            if (timed_out(t0)) {
-              ok = false;
-              break;
-            }
-            __nanosleep(64);
-            free_regions();
-          }
-        }
-        if (!ok) break;
-        cur_off = (unsigned)(start % ring);
-        cur_start = start;
-        load_par = (act_par >> (ord % kItemRing)) & 1u;
-        act_par ^= 1u << (ord % kItemRing);
-        if (lane == 0) {
-          const int r = (reg_front + reg_cnt) % kItemRing;
-          reg_start[r] = start;
-          reg_last[r] = ord;
-          pend[pend_tail % kItemRing] =
-              make_int4(ord, sg, (int)cur_off, (phase_b ? 1 : 0) | (load_par ? 2 : 0));
-          __threadfence_block();
-          s_pend_tail = pend_tail + 1;  // the helper warp issues the load
-        }
-        __syncwarp();
-        ++pend_tail;
-        if (reg_cnt == 0) tail = start;
-        ++reg_cnt;
-        head = start + size;
-        act_wait = true;
-        cur_key = phase_b ? sg : -2;
-        for (int t = 0; t < kNT; ++t) cur_tok[t] = (!phase_b && t < nt) ? plist[p0 + t] / a.k : -1;
-      }
-      // ---- the item's record for publication ----
-      if (lane == 0) {
-        item_info[ord % kItemRing] = make_int4(phase_b ? 1 : 0, sg, blk0, nblk);
-        __threadfence_block();
-        s_nrec = ord + 1;
-      }
-      __syncwarp();
-      const int a_ord = phase_b ? 0 : n_a_items++;
-      // ---- its blocks into the ring ----
-      for (int j = 0; j < nblk && ok; ++j, ++gi) {
-        const int st = gi % NS;
-        if (gi >= NS) {
-          const unsigned long long t0 = globaltimer();
-          while (!lane0(mbar_test(&empty[st], ((gi / NS) - 1) & 1))) {
-            if (timed_out(t0)) {
-              ok = false;
-              break;
-            }
-          }
-        }
-        if (!ok) break;
-        if (lane == 0) {
-          const int blk = blk0 + j;
-          const int row0 = phase_b ? blk * G.rows_b : blk * kRowsA;
-          const int flags = (phase_b ? kSlotPhaseB : 0) | (j == nblk - 1 ? kSlotItemEnd : 0) |
-                            (j == 0 && act_wait ? kSlotActWait : 0) |
-                            (load_par ? kSlotActPar : 0) |
-                            (int)((cur_off >> 7) << kSlotActShift);
-          slot_info[st] = make_int4(flags, sg, row0, ord | (a_ord << 16));
-          unsigned char* buf = smem + L.stages + (size_t)st * G.stage_bytes;
-          fence_proxy_async();
-          if (!phase_b) {
-            const size_t r0 = (size_t)uniq[seg_slot[sg]] * a.I + row0;
-            const size_t qrow = a.H / 8, srow = a.H / 64;
-            mbar_arrive_expect_tx(&full[st], G.a_bytes);
-            bulk_g2s(buf, a.gq + r0 * qrow, G.a_q, &full[st]);
-            bulk_g2s(buf + G.a_q, a.gs + r0 * srow, G.a_sb, &full[st]);
-            if (F != kFmtMx) bulk_g2s(buf + G.a_q + G.a_sb, a.gb + r0 * srow, G.a_sb, &full[st]);
-            buf += G.a_mat;
-            bulk_g2s(buf, a.uq + r0 * qrow, G.a_q, &full[st]);
-            bulk_g2s(buf + G.a_q, a.us + r0 * srow, G.a_sb, &full[st]);
-            if (F != kFmtMx) bulk_g2s(buf + G.a_q + G.a_sb, a.ub + r0 * srow, G.a_sb, &full[st]);
-          } else {
-            const int nrows = min(G.rows_b, a.H - row0);
-            const size_t r0 = (size_t)uniq[seg_slot[sg]] * a.H + row0;
-            const size_t qrow = a.I / 8, srow = a.I / 64;
-            const unsigned qb = nrows * (a.I / 2), sb = nrows * (a.I / 32);
-            mbar_arrive_expect_tx(&full[st], qb + (F == kFmtMx ? 1 : 2) * sb);
-            bulk_g2s(buf, a.dq + r0 * qrow, qb, &full[st]);
-            bulk_g2s(buf + G.b_q, a.ds + r0 * srow, sb, &full[st]);
-            if (F != kFmtMx) bulk_g2s(buf + G.b_q + G.b_sb, a.db + r0 * srow, sb, &full[st]);
-          }
-        }
-        __syncwarp();
-      }
-    }
-    // ---- the end marker ----
-    if (ok) {
-      const int st = gi % NS;
-      if (gi >= NS) {
-        const unsigned long long t0 = globaltimer();
-        while (!lane0(mbar_test(&empty[st], ((gi / NS) - 1) & 1))) {
+        while (!lane0(mbar_test(&empty[st], ((j / NS) - 1) & 1)))
           if (timed_out(t0)) {
             ok = false;
             break;
           }
+      }
+      {  // block j's publication barrier is free: block j - kPubRing was published
+        const unsigned long long t0 = globaltimer();
+        while (ok && lane0_int(s_pub) <= j - kPubRing) {
+          if (timed_out(t0)) ok = false;
+          __nanosleep(32);
         }
       }
-      if (ok && lane == 0) {
-        slot_info[st] = make_int4(kSlotEnd, 0, 0, 0);
-        mbar_arrive(&full[st]);
+      if (!ok) break;
+      if (j == nblk) {
+        if (lane == 0) {
+          slot_info[st] = make_int4(kSlotEnd, 0, 0, j);
+          mbar_arrive(&full[st]);
+        }
+        __syncwarp();
+        break;
+      }
+      bool pb;
+      int sg, row0;
+      block_of(j, pb, sg, row0);
+      const int set = pb ? nseg + sg : (a.x_res ? -1 : sg);
+      const bool new_set = set >= 0 && set != prev_set;
+      prev_set = set;
+      if (lane == 0) {
+        slot_info[st] =
+            make_int4((pb ? kSlotPhaseB : 0) | (new_set ? kSlotNewSet : 0), sg, row0, j);
+        unsigned char* buf = smem + L.stages + (size_t)st * G.stage_bytes;
+        fence_proxy_async();
+        if (!pb) {
+          const size_t r0 = (size_t)uniq[seg_slot[sg]] * a.I + row0;
+          const size_t qrow = a.H / 8, srow = a.H / 64;
+          mbar_arrive_expect_tx(&full[st], G.a_bytes);
+          bulk_g2s(buf, a.gq + r0 * qrow, G.a_q, &full[st]);
+          bulk_g2s(buf + G.a_q, a.gs + r0 * srow, G.a_sb, &full[st]);
+          if (F != kFmtMx) bulk_g2s(buf + G.a_q + G.a_sb, a.gb + r0 * srow, G.a_sb, &full[st]);
+          buf += G.a_mat;
+          bulk_g2s(buf, a.uq + r0 * qrow, G.a_q, &full[st]);
+          bulk_g2s(buf + G.a_q, a.us + r0 * srow, G.a_sb, &full[st]);
+          if (F != kFmtMx) bulk_g2s(buf + G.a_q + G.a_sb, a.ub + r0 * srow, G.a_sb, &full[st]);
+        } else {
+          const int nrows = min(G.rows_b, a.H - row0);
+          const size_t r0 = (size_t)uniq[seg_slot[sg]] * a.H + row0;
+          const size_t qrow = a.I / 8, srow = a.I / 64;
+          const unsigned qb = nrows * (a.I / 2), sb = nrows * (a.I / 32);
+          mbar_arrive_expect_tx(&full[st], qb + (F == kFmtMx ? 1 : 2) * sb);
+          bulk_g2s(buf, a.dq + r0 * qrow, qb, &full[st]);
+          bulk_g2s(buf + G.b_q, a.ds + r0 * srow, sb, &full[st]);
+          if (F != kFmtMx) bulk_g2s(buf + G.b_q + G.b_sb, a.db + r0 * srow, sb, &full[st]);
+        }
       }
       __syncwarp();
     }
-    if (lane == 0) {
-      __threadfence_block();
-      s_prod_done = 1;
-    }
     // copies still in flight after an abort land before the CTA exits (bounded)
     if (!ok && lane == 0) {
-      for (int g = (gi > NS ? gi - NS : 0); g < gi; ++g) {
+      const int issued = j < nblk ? j : nblk;
+      for (int g = (issued > NS ? issued - NS : 0); g < issued; ++g) {
         const unsigned long long t0 = globaltimer();
         while (!mbar_test(&full[g % NS], (g / NS) & 1) && globaltimer() - t0 < kWaitLimitNs) {
         }
@@ -1016,7 +854,6 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
     __syncwarp();
   } else {
     // ================================ compute warps ================================
-    uint16_t* hscr = reinterpret_cast<uint16_t*>(smem + L.hscr);  // [kItemRing][kNT][32]
     auto wait_cons = [&](uint64_t* bar, unsigned parity) -> bool {
       if (s_abort) return false;
       const unsigned long long t0 = globaltimer();
@@ -1030,18 +867,45 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       }
       return true;
     };
-    for (int gi = 0;; ++gi) {
-      const int st = gi % NS;
-      if (!wait_cons(&full[st], (gi / NS) & 1)) break;
+    int nsets = 0;                         // activation sets converted
+    const unsigned char* act = smem + L.act;  // the current set's rows
+    for (int j = 0;; ++j) {
+      const int st = j % NS;
+      if (!wait_cons(&full[st], (j / NS) & 1)) break;
       const int4 si = slot_info[st];
       if (si.x & kSlotEnd) break;
       const bool phase_b = (si.x & kSlotPhaseB) != 0;
-      const int sg = si.y, row0 = si.z, ord = si.w & 0xffff, a_ord = si.w >> 16;
-      if ((si.x & kSlotActWait) &&
-          !wait_cons(&act_full[ord % kItemRing], (si.x & kSlotActPar) ? 1u : 0u))
-        break;
+      const int sg = si.y, row0 = si.z;
       const int nt = seg_nt[sg], p0 = seg_pos[sg];
-      const unsigned char* act = smem + L.act + ((size_t)(si.x >> kSlotActShift) << 7);
+      if (si.x & kSlotNewSet) {
+        // All compute warps are past the previous set's blocks, so the buffer of the set
+        // before it is free; phase B waits (bounded) until every phase-A block of the
+        // segment has published its h rows.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&set_in[0]);
+        if (!wait_cons(&set_in[0], nsets & 1)) break;
+        if (phase_b) {
+          bool ok = true;
+          if (lane == 0) {
+            const unsigned long long t0 = globaltimer();
+            while (!s_abort && ld_acquire_gpu(&hdone[sg]) < (unsigned)bpe_a) {
+              if (globaltimer() - t0 > kWaitLimitNs) {
+                set_error(kErrTimeout);
+                s_abort = 1;
+              }
+            }
+            ok = !s_abort;
+          }
+          if (!lane0(ok)) break;
+        }
+        unsigned char* buf = smem + L.act + (size_t)(nsets & 1) * G.act_buf;
+        convert_set<F>(a, G, phase_b, plist, p0, nt, buf, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&set_out[0]);
+        if (!wait_cons(&set_out[0], nsets & 1)) break;
+        act = buf;
+        ++nsets;
+      }
       const unsigned char* buf = smem + L.stages + (size_t)st * G.stage_bytes;
       float Gs[kNT], Us[kNT];
       float v = 0.f;
@@ -1054,11 +918,18 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
         const unsigned char* buq = bu + (size_t)warp * (a.H / 2);
         const uint16_t* bus = reinterpret_cast<const uint16_t*>(bu + G.a_q) + warp * (a.H / 64);
         const uint16_t* bub = reinterpret_cast<const uint16_t*>(bu + G.a_q + G.a_sb) + warp * (a.H / 64);
+        // the activation row of each pair: the token's resident x row, or row t of the
+        // current set
+        const unsigned char* arow[kNT];
+#pragma unroll
+        for (int t = 0; t < kNT; ++t)
+          arow[t] = a.x_res ? xres + (t < nt ? plist[p0 + t] / a.k : 0) * stride_a
+                            : act + t * stride_a;
         switch (nt) {
-          case 1: dispatch_a<1, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, act, stride_a, lane, Gs, Us); break;
-          case 2: dispatch_a<2, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, act, stride_a, lane, Gs, Us); break;
-          case 3: dispatch_a<3, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, act, stride_a, lane, Gs, Us); break;
-          default: dispatch_a<4, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, act, stride_a, lane, Gs, Us); break;
+          case 1: dispatch_a<1, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us); break;
+          case 2: dispatch_a<2, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us); break;
+          case 3: dispatch_a<3, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us); break;
+          default: dispatch_a<4, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us); break;
         }
       } else {
         nrows = min(G.rows_b, a.H - row0);
@@ -1074,9 +945,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       // this warp is done reading stage st
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
-      const bool item_end = (si.x & kSlotItemEnd) != 0;
       if (!phase_b) {
-        uint16_t* hs = hscr + (ord % kItemRing) * (kNT * 32);
         if (lane < nt) {
           float gv = 0.f, uv = 0.f;
 #pragma unroll
@@ -1088,20 +957,16 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
           const float g = round_to_bf16(gv), hu = round_to_bf16(uv);
           // silu(g) = g / (1 + e^-g); the fast division's error (2 ulp of fp32) is far
           // below the bf16 step h is rounded to
-          const uint16_t hb = float_to_bf16_bits(__fdividef(g, 1.0f + __expf(-g)) * hu);
-          a.h[(size_t)(p0 + lane) * a.I + row0 + warp] = hb;
-          hs[lane * 32 + (row0 & 31) + warp] = hb;
+          a.h[(size_t)(p0 + lane) * a.I + row0 + warp] =
+              float_to_bf16_bits(__fdividef(g, 1.0f + __expf(-g)) * hu);
         }
-        // (the item's 32 h rows per pair form one chunk of h; the producer converts it
-        // to the fixed-point layout when it publishes the item)
       } else if (vid >= 0) {
         const int r = warp + kWarps * (vid / kNT), t = vid % kNT;
         if (r < nrows) a.y[(size_t)(p0 + t) * a.H + row0 + r] = v;
       }
-      if (item_end) {  // this warp's stores of the item are done (released at CTA scope)
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&item_done[ord % kItemRing]);
-      }
+      // this warp's outputs of block j are written (released at CTA scope)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&done[j % kPubRing]);
     }
   }
 
@@ -1153,8 +1018,6 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
     const unsigned old = atomicAdd(exit_cnt, 1u);
     if (old == gridDim.x - 1) {
       for (int sgi = 0; sgi < nseg; ++sgi) hdone[sgi] = 0;
-      *work_ctr = 0;
-      *xdone = 0;
       *exit_cnt = 0;
       __threadfence();
     }
