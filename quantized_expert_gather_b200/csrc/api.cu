@@ -105,7 +105,7 @@ int select_path(int T, int k, int E, int hidden, int inter, int fmt = kFmtAffine
   if (!shape_ok(T, k, E, hidden, inter) || !shape_supported(T, k, E, hidden, inter)) return 0;
   if (T * k <= kMaxPairsFused) {
     LayerGeom g = layer_geom(hidden, inter, fmt);
-    if (g.seg >= 1 && fit_stages(g, E, T * k, hidden, inter, kSmemBudget)) return 1;
+    if (layer_plan(g, E, T, k, kSmemBudget)) return 1;
   }
   if (fmt == kFmtMx) return 0;
   // the grouped path: hidden a multiple of 256 (down tiles) and at most 4096, inter a
@@ -177,14 +177,13 @@ cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
   a.I = I;
   a.g = layer_geom(H, I, F);
   a.wait_prior = 1;
-  // the window's x rows fit one activation buffer: held in each CTA's shared memory
-  a.x_res = (size_t)T * act_bytes(a.g.rounds_a) <= a.g.act_buf ? 1 : 0;
   const int ki = F == kFmtMx ? 9 : 0;  // dyn_smem index of this layer kernel
-  if (a.g.seg < 1 || !fit_stages(a.g, E, T * k, H, I, (size_t)d.dyn_smem[ki])) {
+  if (!layer_plan(a.g, E, T, k, (size_t)d.dyn_smem[ki])) {
     *why = MOE_ERR_UNSUPPORTED;
     return cudaSuccess;
   }
-  const LayerSmem L = layer_smem(a.g, E, T * k, H, I);
+  // the window's x rows fit the normal activation area: each CTA keeps them all
+  a.x_res = (size_t)T * act_bytes(a.g.rounds_a) <= a.g.act_n ? 1 : 0;
   // One CTA per SM, all resident at once (the kernel has grid barriers); the
   // launch may overlap the tail of the preceding kernel (programmatic launch).
   cudaLaunchAttribute attr[2];
@@ -195,7 +194,7 @@ cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
   cudaLaunchConfig_t c = {};
   c.gridDim = dim3(d.sms);
   c.blockDim = dim3(kThreads);
-  c.dynamicSmemBytes = L.total;
+  c.dynamicSmemBytes = a.g.total;
   c.stream = st;
   c.attrs = attr;
   c.numAttrs = 2;

@@ -66,7 +66,6 @@ constexpr int kMaxRowsPerWarpB = 4; // phase B: rows of Wd per warp per block
 constexpr int kMaxStages = 4;       // ring depth (fewer when shared memory is short)
 constexpr int kNT = 4;              // pairs per segment (upper bound)
 constexpr int kMaxPairsFused = 1024;
-constexpr unsigned kSegActBytes = 36 * 1024;  // one activation buffer (a segment's rows)
 constexpr unsigned kBarUnion = 1;   // named barrier: union formed (warp 0 -> producer)
 constexpr unsigned kBarWork = 2;    // named barrier: every warp but the producer
 // Dynamic shared memory the kernel may plan for on B200 (227 KB per block, less a
@@ -85,12 +84,17 @@ struct LayerGeom {
   int fmt;                 // kFmtAffine or kFmtMx
   int rounds_a, rounds_b;  // 32-column chunks per lane per row (>= H/1024, I/1024; 1, 2, 4, 6, 8)
   int rows_b;              // phase B rows per block (multiple of kWarps, <= 32)
-  int seg;                 // pairs per segment (<= kNT)
-  int stages;              // ring depth (<= kMaxStages)
   unsigned a_q, a_sb, a_mat, a_bytes;  // phase A block: per matrix codes / scale (or bias) bytes
   unsigned b_q, b_sb, b_bytes;         // phase B full block
   unsigned stage_bytes;
-  unsigned act_buf;        // one activation buffer: seg rows of the wider layout
+  // shared-memory plan (layer_plan): index tables at offset 0, then the stage ring,
+  // then the activation area.  Normal layout: `stages` stages and act_n bytes; wide
+  // layout (windows where one expert has more pairs than act_n holds rows of x):
+  // stages_w stages and act_w bytes, every x row of the window resident (0: none)
+  unsigned tables;
+  int stages, stages_w;
+  unsigned act_n, act_w;
+  unsigned total;          // dynamic shared memory of the launch
 };
 
 // Chunk rounds for a row of D columns: ceil(D / 1024), rounded up to 1, 2, 4, 6 or 8.
@@ -108,10 +112,6 @@ __host__ __device__ inline LayerGeom layer_geom(int H, int I, int fmt = kFmtAffi
   if (rb < kWarps) rb = kWarps;
   if (rb > kWarps * kMaxRowsPerWarpB) rb = kWarps * kMaxRowsPerWarpB;
   g.rows_b = rb;
-  const int rmax = g.rounds_a > g.rounds_b ? g.rounds_a : g.rounds_b;
-  int s = (int)(kSegActBytes / act_bytes(rmax));
-  g.seg = s > kNT ? kNT : s;
-  g.stages = kMaxStages;
   g.a_q = kRowsA * H / 2;
   // scales: bf16 per 64 columns (affine) or one e8m0 byte per 32 (mx), H/32 bytes a
   // row either way; the affine format adds as many bytes of biases
@@ -123,53 +123,79 @@ __host__ __device__ inline LayerGeom layer_geom(int H, int I, int fmt = kFmtAffi
   g.b_sb = g.rows_b * I / 32;
   g.b_bytes = g.b_q + nsb * g.b_sb;
   g.stage_bytes = (unsigned)align_up(g.a_bytes > g.b_bytes ? g.a_bytes : g.b_bytes, 128);
-  g.act_buf = (unsigned)align_up((size_t)(g.seg > 0 ? g.seg : 1) * act_bytes(rmax), 128);
+  g.tables = 0;
+  g.stages = g.stages_w = 0;
+  g.act_n = 0;
+  g.act_w = 0;
+  g.total = 0;
   return g;
 }
 
+// Index tables at the start of shared memory: union scratch and result, the pair
+// maps, and the segment tables of phase A and of phase B (at most P each).
 struct LayerSmem {
-  size_t stages, act, cnt, rank, unique, offsets, pair_list, pos_of, seg_slot, seg_pos,
-      seg_nt, total;
+  size_t cnt, rank, unique, offsets, pair_list, pos_of, tok_of, sa_slot, sa_pos, sa_nt, sb_slot,
+      sb_pos, sb_nt, end;
 };
-__host__ __device__ inline LayerSmem layer_smem(const LayerGeom& g, int E, int P, int H, int I) {
+__host__ __device__ inline LayerSmem layer_smem(int E, int P) {
   LayerSmem s;
   const int m = (E < P ? E : P) > 0 ? (E < P ? E : P) : 1;
-  s.stages = 0;
-  s.act = align_up((size_t)g.stages * g.stage_bytes, 128);    // two activation buffers
-  s.cnt = align_up(s.act + 2 * (size_t)g.act_buf, 16);
+  s.cnt = 0;
   s.rank = align_up(s.cnt + sizeof(int) * E, 16);
   s.unique = align_up(s.rank + sizeof(int) * P, 16);
   s.offsets = align_up(s.unique + sizeof(int) * m, 16);
   s.pair_list = align_up(s.offsets + sizeof(int) * (m + 1), 16);
   s.pos_of = align_up(s.pair_list + sizeof(int) * P, 16);
-  // segments: at most P of them
-  s.seg_slot = align_up(s.pos_of + sizeof(int) * P, 16);
-  s.seg_pos = align_up(s.seg_slot + sizeof(int) * P, 16);
-  s.seg_nt = align_up(s.seg_pos + sizeof(int) * P, 16);
-  s.total = align_up(s.seg_nt + sizeof(int) * P, 16);
+  s.tok_of = align_up(s.pos_of + sizeof(int) * P, 16);
+  s.sa_slot = align_up(s.tok_of + sizeof(int) * P, 16);
+  s.sa_pos = align_up(s.sa_slot + sizeof(int) * P, 16);
+  s.sa_nt = align_up(s.sa_pos + sizeof(int) * P, 16);
+  s.sb_slot = align_up(s.sa_nt + sizeof(int) * P, 16);
+  s.sb_pos = align_up(s.sb_slot + sizeof(int) * P, 16);
+  s.sb_nt = align_up(s.sb_pos + sizeof(int) * P, 16);
+  s.end = align_up(s.sb_nt + sizeof(int) * P, 128);
   return s;
 }
 
-// Deepest ring (kMaxStages down to 2) whose shared memory fits in `budget` bytes;
-// false if none does.
-__host__ __device__ inline bool fit_stages(LayerGeom& g, int E, int P, int H, int I,
-                                           size_t budget) {
+// The shared-memory plan for a window of T tokens, top-k, within `budget` bytes: the
+// deepest normal ring (kMaxStages down to 2) that leaves at least two x rows and eight
+// h rows of activations, the rest of the budget being the activation area; and a wide
+// layout holding all T x rows when that needs more than the normal area (its ring at
+// least 2 stages deep, else none).  False if not even the normal layout fits.
+__host__ __device__ inline bool layer_plan(LayerGeom& g, int E, int T, int k, size_t budget) {
+  const int P = T * k;
+  g.tables = (unsigned)layer_smem(E, P).end;
+  const size_t ra = act_bytes(g.rounds_a), rbb = act_bytes(g.rounds_b);
+  const size_t act_min = align_up(2 * ra > 8 * rbb ? 2 * ra : 8 * rbb, 128);
+  g.stages = 0;
   for (int st = kMaxStages; st >= 2; --st) {
-    g.stages = st;
-    if (layer_smem(g, E, P, H, I).total <= budget) return true;
+    const size_t used = (size_t)g.tables + (size_t)st * g.stage_bytes;
+    if (used + act_min <= budget) {
+      g.stages = st;
+      g.act_n = (unsigned)((budget - used) / 128 * 128);
+      break;
+    }
   }
-  return false;
+  if (g.stages == 0) return false;
+  g.stages_w = 0;
+  g.act_w = (unsigned)align_up((size_t)T * ra, 128);
+  if (g.act_w > g.act_n) {
+    const size_t room = budget > (size_t)g.tables + g.act_w ? budget - g.tables - g.act_w : 0;
+    int st = (int)(room / g.stage_bytes);
+    if (st > kMaxStages) st = kMaxStages;
+    if (st >= 2) g.stages_w = st;
+  }
+  g.total = (unsigned)budget;
+  return true;
 }
 
 // Workspace counters (unsigned), a region of fixed size at the start of every
 // workspace so that calls of different shapes never see each other's data there:
-// [0] CTAs finished, [1, 1+kMaxPairsFused) hdone per segment, then ydone per
-// phase-B row block (at most kMaxRowBlocks), then the work-item counter and the
-// count of CTAs that have converted their share of x.
+// [0] CTAs finished, [1, 1+kMaxPairsFused) hdone per distinct expert (phase-A
+// blocks published), then ydone per phase-B row block (at most kMaxRowBlocks),
+// then two words kept zero.
 constexpr int kMaxRowBlocks = 4096 / kWarps;
 constexpr size_t kSyncWords = 1 + kMaxPairsFused + kMaxRowBlocks + 2;
-constexpr size_t kSyncWorkItem = 1 + kMaxPairsFused + kMaxRowBlocks;
-constexpr size_t kSyncXDone = kSyncWorkItem + 1;
 
 // -------------------------------------------------------------- arguments ---
 struct LayerArgs {
@@ -569,7 +595,7 @@ constexpr int kPubRing = 16;      // blocks between compute and publication
 // 32-column chunk together.
 template <int F>
 __device__ __forceinline__ void convert_set(const LayerArgs& a, const LayerGeom& G, bool phase_b,
-                                            const int* plist, int p0, int nt,
+                                            const int* tok_of, int p0, int nt,
                                             unsigned char* buf, int lane) {
   const int D = phase_b ? a.I : a.H, R = phase_b ? G.rounds_b : G.rounds_a, nch = D / 32;
   const unsigned stride = act_bytes(R);
@@ -580,8 +606,8 @@ __device__ __forceinline__ void convert_set(const LayerArgs& a, const LayerGeom&
     if (phase_b)
       v = __ldcg(reinterpret_cast<const uint4*>(a.h + (size_t)(p0 + t) * a.I + ch * 32 + m * 8));
     else
-      v = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)(plist[p0 + t] / a.k) * a.H +
-                                               ch * 32 + m * 8));
+      v = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)tok_of[p0 + t] * a.H + ch * 32 +
+                                               m * 8));
     uint4 packed;
     const float2 sc = fixed_point_quarter<F>(v, 0xfu << (lane & ~3), packed);
     unsigned char* row = buf + (size_t)t * stride;
@@ -590,11 +616,59 @@ __device__ __forceinline__ void convert_set(const LayerArgs& a, const LayerGeom&
   }
 }
 
+// Rows of x resident in shared memory: all T tokens, by the threads [t0, t0 + nthr)
+// of this CTA (four consecutive lanes per 32-column chunk).
+template <int F>
+__device__ __forceinline__ void convert_x_all(const LayerArgs& a, const LayerGeom& G,
+                                              unsigned char* xres, int t0, int nthr, int lane) {
+  const int nch = a.H / 32, R = G.rounds_a;
+  const unsigned stride = act_bytes(R);
+  const int nq = a.T * nch * 4;  // quarters of 8 columns
+  for (int q = t0; q < nq; q += nthr) {
+    const int m = q & 3, tc = q >> 2, t = tc / nch, ch = tc % nch;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H + ch * 32 + m * 8));
+    uint4 packed;
+    const float2 sc = fixed_point_quarter<F>(v, 0xfu << (lane & ~3), packed);
+    unsigned char* row = xres + (size_t)t * stride;
+    reinterpret_cast<uint4*>(row)[((ch / 32) * 4 + m) * 32 + (ch % 32)] = packed;
+    if (m == 0) reinterpret_cast<float2*>(row + act_digit_bytes(R))[ch] = sc;
+  }
+}
+
+// Segment table: expert slot i (n_i pairs) contributes ceil(n_i / seg) segments of at
+// most `seg` pairs, in slot order.  Run by one warp; returns the number of segments.
+__device__ __forceinline__ int make_segments(const int* offs, int u, int seg, int* s_slot,
+                                             int* s_pos, int* s_nt, int lane) {
+  int base = 0;
+  for (int b0 = 0; b0 < u; b0 += 32) {
+    const int i = b0 + lane;
+    const int n_i = (i < u) ? offs[i + 1] - offs[i] : 0;
+    const int c = (n_i + seg - 1) / seg;
+    int incl = c;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(kFull, incl, d);
+      if (lane >= d) incl += v;
+    }
+    for (int j = 0; j < c; ++j) {
+      const int sidx = base + incl - c + j;
+      s_slot[sidx] = i;
+      s_pos[sidx] = offs[i] + j * seg;
+      s_nt[sidx] = min(seg, n_i - j * seg);
+    }
+    base += __shfl_sync(kFull, incl, 31);
+  }
+  return base;
+}
+
 // 10 warps: 8 compute warps, a producer warp and a helper warp (see the top of this file).
 template <int F>
 __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ int s_u, s_nseg;
+  // window plan, set by warp 0 after the union: segments of phase A and B, ring depth,
+  // resident x rows, the wide layout
+  __shared__ int s_u, s_nsa, s_nsb, s_ns, s_xres, s_wide, s_sega;
+  __shared__ unsigned s_act_off, s_act_size;
   __shared__ volatile int s_abort;
   __shared__ volatile int s_pub;  // blocks published by the helper warp
   __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
@@ -603,8 +677,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
   __shared__ int4 slot_info[kMaxStages];  // per ring slot: flags, segment, first row, block
   const LayerGeom& G = a.g;
   const int P = a.T * a.k;
-  const int NS = G.stages;
-  const LayerSmem L = layer_smem(G, a.E, P, a.H, a.I);
+  const LayerSmem L = layer_smem(a.E, P);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned* exit_cnt = a.sync;
   unsigned* hdone = a.sync + 1;
@@ -612,7 +685,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
   const unsigned stride_a = act_bytes(G.rounds_a), stride_b = act_bytes(G.rounds_b);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < kMaxStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kWarps);
     }
@@ -625,77 +698,79 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
   }
   if (a.wait_prior) grid_dep_wait();
 
-  // ---- route-union (warp 0), its segments, and the inverse map pair -> position ----
+  // ---- route-union (warp 0), segments, the window's plan, and the pair maps ----
   int* uniq = reinterpret_cast<int*>(smem + L.unique);
   int* offs = reinterpret_cast<int*>(smem + L.offsets);
   int* plist = reinterpret_cast<int*>(smem + L.pair_list);
   int* pos_of = reinterpret_cast<int*>(smem + L.pos_of);
-  int* seg_slot = reinterpret_cast<int*>(smem + L.seg_slot);
-  int* seg_pos = reinterpret_cast<int*>(smem + L.seg_pos);
-  int* seg_nt = reinterpret_cast<int*>(smem + L.seg_nt);
-  // resident x rows (x_res): the start of the activation area
-  unsigned char* xres = smem + L.act;
+  int* tok_of = reinterpret_cast<int*>(smem + L.tok_of);  // token of each pair position
+  int* sa_slot = reinterpret_cast<int*>(smem + L.sa_slot);
+  int* sa_pos = reinterpret_cast<int*>(smem + L.sa_pos);
+  int* sa_nt = reinterpret_cast<int*>(smem + L.sa_nt);
+  int* sb_slot = reinterpret_cast<int*>(smem + L.sb_slot);
+  int* sb_pos = reinterpret_cast<int*>(smem + L.sb_pos);
+  int* sb_nt = reinterpret_cast<int*>(smem + L.sb_nt);
+  unsigned char* ring = smem + G.tables;
   const int wt = warp < kWarps ? (int)threadIdx.x : (int)threadIdx.x - 32;  // 0..287 but the producer
   if (warp == 0) {
     int nv;
     const int u = warp_route_union(a.idx, P, a.E, reinterpret_cast<int*>(smem + L.cnt),
                                    reinterpret_cast<int*>(smem + L.rank), uniq, offs, plist, &nv);
-    // segments: expert slot i contributes ceil(n_i / seg) segments, in slot order
-    int base = 0;
-    for (int b0 = 0; b0 < u; b0 += 32) {
-      const int i = b0 + lane;
-      const int n_i = (i < u) ? offs[i + 1] - offs[i] : 0;
-      const int c = (n_i + G.seg - 1) / G.seg;
-      int incl = c;
+    // the plan: a window whose x rows fit the normal activation area keeps them resident;
+    // one with an expert of more pairs than that area holds x rows takes the wide layout
+    // (all x rows resident, shallower ring) when the launch planned one; phase-A
+    // segments are whole experts when x is resident, else as many pairs as the area
+    // holds rows; phase-B segments as many pairs as the area holds h rows
+    int maxn = 0;
+    for (int i = lane; i < u; i += 32) maxn = max(maxn, offs[i + 1] - offs[i]);
 #pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const int v = __shfl_up_sync(kFull, incl, d);
-        if (lane >= d) incl += v;
-      }
-      for (int j = 0; j < c; ++j) {
-        const int s = base + incl - c + j;
-        seg_slot[s] = i;
-        seg_pos[s] = offs[i] + j * G.seg;
-        seg_nt[s] = min(G.seg, n_i - j * G.seg);
-      }
-      base += __shfl_sync(kFull, incl, 31);
-    }
+    for (int d = 16; d >= 1; d >>= 1) maxn = max(maxn, __shfl_xor_sync(kFull, maxn, d));
+    const int sega_n = (int)(G.act_n / stride_a);
+    const bool wide = !a.x_res && G.stages_w >= 2 && maxn > sega_n;
+    const bool xr = a.x_res || wide;
+    const unsigned act_size = wide ? G.act_w : G.act_n;
+    const int ns = wide ? G.stages_w : G.stages;
+    const int sega = xr ? max(P, 1) : max(sega_n, 1);
+    const int segb = max((int)(act_size / stride_b), 1);
+    const int nsa = make_segments(offs, u, sega, sa_slot, sa_pos, sa_nt, lane);
+    const int nsb = make_segments(offs, u, segb, sb_slot, sb_pos, sb_nt, lane);
     if (lane == 0) {
       s_u = u;
-      s_nseg = base;
+      s_nsa = nsa;
+      s_nsb = nsb;
+      s_ns = ns;
+      s_xres = xr ? 1 : 0;
+      s_wide = wide ? 1 : 0;
+      s_sega = sega;
+      s_act_off = G.tables + (unsigned)ns * G.stage_bytes;
+      s_act_size = act_size;
     }
     __syncwarp();
     named_barrier_arrive(kBarUnion, 64);  // the producer may start (it waits on this)
   } else if (warp != kWarps) {
     // warps 1..7 and the helper: 256 threads
     for (int p = wt - 32; p < P; p += kThreads - 64) pos_of[p] = -1;
+    // a window whose x rows fit the normal activation area: converted while warp 0
+    // forms the union
+    if (a.x_res)
+      convert_x_all<F>(a, G, smem + G.tables + (unsigned)G.stages * G.stage_bytes, wt - 32,
+                       kThreads - 64, lane);
   }
-
-  // ---- a window whose x rows fit one activation buffer keeps them all here, converted
-  // by warps 1..7 and the helper while warp 0 forms the union ----
   if (warp != kWarps) {
-    if (a.x_res && warp != 0) {
-      const int nch = a.H / 32, R = G.rounds_a;
-      const int nq = a.T * nch * 4;  // quarters of 8 columns
-      for (int q = wt - 32; q < nq; q += kThreads - 64) {
-        const int m = q & 3, tc = q >> 2, t = tc / nch, ch = tc % nch;
-        const uint4 v =
-            __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H + ch * 32 + m * 8));
-        uint4 packed;
-        const float2 sc = fixed_point_quarter<F>(v, 0xfu << (lane & ~3), packed);
-        unsigned char* row = xres + (size_t)t * stride_a;
-        reinterpret_cast<uint4*>(row)[((ch / 32) * 4 + m) * 32 + (ch % 32)] = packed;
-        if (m == 0) reinterpret_cast<float2*>(row + act_digit_bytes(R))[ch] = sc;
-      }
-    }
     named_barrier(kBarWork, kThreads - 32);  // every warp but the producer
   } else {
-    named_barrier(kBarUnion, 64);  // the union is formed
+    named_barrier(kBarUnion, 64);  // the plan is made
   }
-  const int u = s_u, nseg = s_nseg;
+  const int u = s_u, nsa = s_nsa, nsb = s_nsb, NS = s_ns;
+  const bool x_res = s_xres != 0;
+  unsigned char* actp = smem + s_act_off;  // activation area (resident x rows first)
   const int n_valid = offs[u];
   if (warp != kWarps) {
-    for (int i = wt; i < n_valid; i += kThreads - 32) pos_of[plist[i]] = i;
+    for (int i = wt; i < n_valid; i += kThreads - 32) {
+      pos_of[plist[i]] = i;
+      tok_of[i] = plist[i] / a.k;
+    }
+    if (s_wide) convert_x_all<F>(a, G, actp, wt, kThreads - 32, lane);  // wide: x now
     named_barrier(kBarWork, kThreads - 32);
   }
 
@@ -707,12 +782,13 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
   }
 
   // ---- this CTA's blocks: a contiguous, balanced share of the phase-A blocks (kRowsA
-  // rows of gate and of up each), then of the phase-B blocks (rows_b rows of down
-  // each), both in segment order.  Every block is 2 kRowsA H/2 + scales (A) or
-  // rows_b I/2 + scales (B) bytes; the two are equal at the 4096/2048 shape ----
+  // rows of gate and of up each, per phase-A segment), then of the phase-B blocks
+  // (rows_b rows of down each, per phase-B segment), both in segment order.  Every
+  // block is 2 kRowsA H/2 + scales (A) or rows_b I/2 + scales (B) bytes; the two are
+  // equal at the 4096/2048 shape ----
   const int bpe_a = a.I / kRowsA;                     // phase-A blocks per segment
   const int bpe_b = (a.H + G.rows_b - 1) / G.rows_b;  // phase-B blocks per segment
-  const long long NA = (long long)nseg * bpe_a, NB = (long long)nseg * bpe_b;
+  const long long NA = (long long)nsa * bpe_a, NB = (long long)nsb * bpe_b;
   const int a0 = (int)(NA * blockIdx.x / gridDim.x), a1 = (int)(NA * (blockIdx.x + 1) / gridDim.x);
   const int b0 = (int)(NB * blockIdx.x / gridDim.x), b1 = (int)(NB * (blockIdx.x + 1) / gridDim.x);
   const int nA = a1 - a0, nblk = nA + (b1 - b0);
@@ -732,7 +808,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
 
   if (warp == kWarps + 1) {
     // ================================ helper warp ================================
-    // Publishes finished blocks in order: a phase-A block adds 1 to hdone of its segment
+    // Publishes finished blocks in order: a phase-A block adds 1 to hdone of its expert
     // (its h rows written), a phase-B block adds 1 to ydone of its row block.  The
     // compute warps' done arrivals released their stores at CTA scope and the test
     // below acquires them; the device-scope release reductions pass them on
@@ -744,7 +820,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
         int sg, row0;
         block_of(j, pb, sg, row0);
         if (lane == 0) {
-          if (!pb) red_release_gpu(&hdone[sg], 1u);
+          if (!pb) red_release_gpu(&hdone[sa_slot[sg]], 1u);
           else red_release_gpu(&ydone[row0 / G.rows_b], 1u);
           s_pub = j + 1;
         }
@@ -810,16 +886,16 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       bool pb;
       int sg, row0;
       block_of(j, pb, sg, row0);
-      const int set = pb ? nseg + sg : (a.x_res ? -1 : sg);
+      const int set = pb ? nsa + sg : (x_res ? -1 : sg);
       const bool new_set = set >= 0 && set != prev_set;
       prev_set = set;
       if (lane == 0) {
         slot_info[st] =
             make_int4((pb ? kSlotPhaseB : 0) | (new_set ? kSlotNewSet : 0), sg, row0, j);
-        unsigned char* buf = smem + L.stages + (size_t)st * G.stage_bytes;
+        unsigned char* buf = ring + (size_t)st * G.stage_bytes;
         fence_proxy_async();
         if (!pb) {
-          const size_t r0 = (size_t)uniq[seg_slot[sg]] * a.I + row0;
+          const size_t r0 = (size_t)uniq[sa_slot[sg]] * a.I + row0;
           const size_t qrow = a.H / 8, srow = a.H / 64;
           mbar_arrive_expect_tx(&full[st], G.a_bytes);
           bulk_g2s(buf, a.gq + r0 * qrow, G.a_q, &full[st]);
@@ -831,7 +907,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
           if (F != kFmtMx) bulk_g2s(buf + G.a_q + G.a_sb, a.ub + r0 * srow, G.a_sb, &full[st]);
         } else {
           const int nrows = min(G.rows_b, a.H - row0);
-          const size_t r0 = (size_t)uniq[seg_slot[sg]] * a.H + row0;
+          const size_t r0 = (size_t)uniq[sb_slot[sg]] * a.H + row0;
           const size_t qrow = a.I / 8, srow = a.I / 64;
           const unsigned qb = nrows * (a.I / 2), sb = nrows * (a.I / 32);
           mbar_arrive_expect_tx(&full[st], qb + (F == kFmtMx ? 1 : 2) * sb);
@@ -867,8 +943,8 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       }
       return true;
     };
-    int nsets = 0;                         // activation sets converted
-    const unsigned char* act = smem + L.act;  // the current set's rows
+    const int sega = s_sega;
+    int nsets = 0;  // activation sets converted
     for (int j = 0;; ++j) {
       const int st = j % NS;
       if (!wait_cons(&full[st], (j / NS) & 1)) break;
@@ -876,19 +952,23 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       if (si.x & kSlotEnd) break;
       const bool phase_b = (si.x & kSlotPhaseB) != 0;
       const int sg = si.y, row0 = si.z;
-      const int nt = seg_nt[sg], p0 = seg_pos[sg];
+      const int nt = phase_b ? sb_nt[sg] : sa_nt[sg];
+      const int p0 = phase_b ? sb_pos[sg] : sa_pos[sg];
       if (si.x & kSlotNewSet) {
-        // All compute warps are past the previous set's blocks, so the buffer of the set
-        // before it is free; phase B waits (bounded) until every phase-A block of the
-        // segment has published its h rows.
+        // All compute warps are past the previous set's blocks, so the activation area
+        // is free; phase B waits (bounded) until every phase-A block of the expert has
+        // published its h rows.
         __syncwarp();
         if (lane == 0) mbar_arrive(&set_in[0]);
         if (!wait_cons(&set_in[0], nsets & 1)) break;
         if (phase_b) {
           bool ok = true;
           if (lane == 0) {
+            const int slot = sb_slot[sg];
+            const int n_i = offs[slot + 1] - offs[slot];
+            const unsigned target = (unsigned)bpe_a * (unsigned)((n_i + sega - 1) / sega);
             const unsigned long long t0 = globaltimer();
-            while (!s_abort && ld_acquire_gpu(&hdone[sg]) < (unsigned)bpe_a) {
+            while (!s_abort && ld_acquire_gpu(&hdone[slot]) < target) {
               if (globaltimer() - t0 > kWaitLimitNs) {
                 set_error(kErrTimeout);
                 s_abort = 1;
@@ -898,75 +978,79 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
           }
           if (!lane0(ok)) break;
         }
-        unsigned char* buf = smem + L.act + (size_t)(nsets & 1) * G.act_buf;
-        convert_set<F>(a, G, phase_b, plist, p0, nt, buf, lane);
+        convert_set<F>(a, G, phase_b, tok_of, p0, nt, actp, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(&set_out[0]);
         if (!wait_cons(&set_out[0], nsets & 1)) break;
-        act = buf;
         ++nsets;
       }
-      const unsigned char* buf = smem + L.stages + (size_t)st * G.stage_bytes;
-      float Gs[kNT], Us[kNT];
-      float v = 0.f;
-      int vid = -1, nrows = 0;
-      if (!phase_b) {
-        const unsigned char* bgq = buf + (size_t)warp * (a.H / 2);
-        const uint16_t* bgs = reinterpret_cast<const uint16_t*>(buf + G.a_q) + warp * (a.H / 64);
-        const uint16_t* bgb = reinterpret_cast<const uint16_t*>(buf + G.a_q + G.a_sb) + warp * (a.H / 64);
-        const unsigned char* bu = buf + G.a_mat;
-        const unsigned char* buq = bu + (size_t)warp * (a.H / 2);
-        const uint16_t* bus = reinterpret_cast<const uint16_t*>(bu + G.a_q) + warp * (a.H / 64);
-        const uint16_t* bub = reinterpret_cast<const uint16_t*>(bu + G.a_q + G.a_sb) + warp * (a.H / 64);
-        // the activation row of each pair: the token's resident x row, or row t of the
-        // current set
-        const unsigned char* arow[kNT];
-#pragma unroll
-        for (int t = 0; t < kNT; ++t)
-          arow[t] = a.x_res ? xres + (t < nt ? plist[p0 + t] / a.k : 0) * stride_a
-                            : act + t * stride_a;
-        switch (nt) {
-          case 1: dispatch_a<1, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us); break;
-          case 2: dispatch_a<2, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us); break;
-          case 3: dispatch_a<3, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us); break;
-          default: dispatch_a<4, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us); break;
-        }
-      } else {
-        nrows = min(G.rows_b, a.H - row0);
-        const uint16_t* bs = reinterpret_cast<const uint16_t*>(buf + G.b_q);
-        const uint16_t* bb = reinterpret_cast<const uint16_t*>(buf + G.b_q + G.b_sb);
-        switch (nt) {
-          case 1: v = dispatch_b<1, F>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
-          case 2: v = dispatch_b<2, F>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
-          case 3: v = dispatch_b<3, F>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
-          default: v = dispatch_b<4, F>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
-        }
-      }
-      // this warp is done reading stage st
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
-      if (!phase_b) {
-        if (lane < nt) {
-          float gv = 0.f, uv = 0.f;
+      const unsigned char* buf = ring + (size_t)st * G.stage_bytes;
+      // the set's pairs in chunks of kNT, the block's weights read again per chunk
+      int nrows = 0;
+      for (int c0 = 0; c0 < nt; c0 += kNT) {
+        const int ntc = min(kNT, nt - c0);
+        float Gs[kNT], Us[kNT];
+        float v = 0.f;
+        int vid = -1;
+        if (!phase_b) {
+          const unsigned char* bgq = buf + (size_t)warp * (a.H / 2);
+          const uint16_t* bgs = reinterpret_cast<const uint16_t*>(buf + G.a_q) + warp * (a.H / 64);
+          const uint16_t* bgb = reinterpret_cast<const uint16_t*>(buf + G.a_q + G.a_sb) + warp * (a.H / 64);
+          const unsigned char* bu = buf + G.a_mat;
+          const unsigned char* buq = bu + (size_t)warp * (a.H / 2);
+          const uint16_t* bus = reinterpret_cast<const uint16_t*>(bu + G.a_q) + warp * (a.H / 64);
+          const uint16_t* bub = reinterpret_cast<const uint16_t*>(bu + G.a_q + G.a_sb) + warp * (a.H / 64);
+          // the activation row of each pair: the token's resident x row, or row c0 + t
+          // of the current set
+          const unsigned char* arow[kNT];
 #pragma unroll
           for (int t = 0; t < kNT; ++t)
-            if (t == lane) {
-              gv = Gs[t];
-              uv = Us[t];
-            }
-          const float g = round_to_bf16(gv), hu = round_to_bf16(uv);
-          // silu(g) = g / (1 + e^-g); the fast division's error (2 ulp of fp32) is far
-          // below the bf16 step h is rounded to
-          a.h[(size_t)(p0 + lane) * a.I + row0 + warp] =
-              float_to_bf16_bits(__fdividef(g, 1.0f + __expf(-g)) * hu);
+            arow[t] = x_res ? actp + (t < ntc ? tok_of[p0 + c0 + t] : 0) * stride_a
+                            : actp + (c0 + t) * stride_a;
+          switch (ntc) {
+            case 1: dispatch_a<1, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us); break;
+            case 2: dispatch_a<2, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us); break;
+            case 3: dispatch_a<3, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us); break;
+            default: dispatch_a<4, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us); break;
+          }
+          if (lane < ntc) {
+            float gv = 0.f, uv = 0.f;
+#pragma unroll
+            for (int t = 0; t < kNT; ++t)
+              if (t == lane) {
+                gv = Gs[t];
+                uv = Us[t];
+              }
+            const float g = round_to_bf16(gv), hu = round_to_bf16(uv);
+            // silu(g) = g / (1 + e^-g); the fast division's error (2 ulp of fp32) is far
+            // below the bf16 step h is rounded to
+            a.h[(size_t)(p0 + c0 + lane) * a.I + row0 + warp] =
+                float_to_bf16_bits(__fdividef(g, 1.0f + __expf(-g)) * hu);
+          }
+        } else {
+          nrows = min(G.rows_b, a.H - row0);
+          const uint16_t* bs = reinterpret_cast<const uint16_t*>(buf + G.b_q);
+          const uint16_t* bb = reinterpret_cast<const uint16_t*>(buf + G.b_q + G.b_sb);
+          const unsigned char* act = actp + (size_t)c0 * stride_b;
+          switch (ntc) {
+            case 1: v = dispatch_b<1, F>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
+            case 2: v = dispatch_b<2, F>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
+            case 3: v = dispatch_b<3, F>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
+            default: v = dispatch_b<4, F>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
+          }
+          if (vid >= 0) {
+            const int r = warp + kWarps * (vid / kNT), t = vid % kNT;
+            if (r < nrows) a.y[(size_t)(p0 + c0 + t) * a.H + row0 + r] = v;
+          }
         }
-      } else if (vid >= 0) {
-        const int r = warp + kWarps * (vid / kNT), t = vid % kNT;
-        if (r < nrows) a.y[(size_t)(p0 + t) * a.H + row0 + r] = v;
       }
-      // this warp's outputs of block j are written (released at CTA scope)
+      // this warp is done reading stage st, and its outputs of block j are written
+      // (released at CTA scope)
       __syncwarp();
-      if (lane == 0) mbar_arrive(&done[j % kPubRing]);
+      if (lane == 0) {
+        mbar_arrive(&empty[st]);
+        mbar_arrive(&done[j % kPubRing]);
+      }
     }
   }
 
@@ -985,7 +1069,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
     for (int rb = blockIdx.x; rb < n_rb; rb += gridDim.x) {
       if (threadIdx.x == 0) {
         const unsigned long long t0 = globaltimer();
-        while (!s_abort && ld_acquire_gpu(&ydone[rb]) < (unsigned)nseg) {
+        while (!s_abort && ld_acquire_gpu(&ydone[rb]) < (unsigned)nsb) {
           if (globaltimer() - t0 > kWaitLimitNs) {
             set_error(kErrTimeout);
             s_abort = 1;
@@ -1017,7 +1101,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
     __threadfence();
     const unsigned old = atomicAdd(exit_cnt, 1u);
     if (old == gridDim.x - 1) {
-      for (int sgi = 0; sgi < nseg; ++sgi) hdone[sgi] = 0;
+      for (int i = 0; i < u; ++i) hdone[i] = 0;
       *exit_cnt = 0;
       __threadfence();
     }
