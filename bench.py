@@ -598,23 +598,26 @@ def our_arm(args, world, rank, local):
             torch.cuda.synchronize()
             torch.cuda.empty_cache()
         # the all-identical extreme: every token of a T=16 window routes to the same 8
-        # experts (16 pairs per expert); each expert must still stream once
-        same = np.tile(np.arange(K_TOP, dtype=np.int32) * 9, (16, 1))
+        # experts (16 pairs per expert), which must still stream once; 42 chained layers,
+        # layer l on experts 8l .. 8l+7 of the E=256 bank (mod 256), so consecutive layers
+        # share no expert
         wsame = np.full((16, K_TOP), 1.0 / K_TOP, np.float32)
         ws3 = torch.zeros(qeg.moe_workspace_size(16, K_TOP, E2, HIDDEN, INTER), dtype=torch.uint8,
                           device=dev)
         xi = torch.from_numpy(synth.x_bf16(16, HIDDEN, SEED + 16).view(np.int16)).to(dev) \
             .view(torch.bfloat16)
-        ii, wi = torch.from_numpy(same).to(dev), torch.from_numpy(wsame).to(dev)
-        oi = torch.empty((16, HIDDEN), dtype=torch.bfloat16, device=dev)
+        ii = [torch.from_numpy(np.tile((np.arange(K_TOP) + K_TOP * l) % E2, (16, 1))
+                               .astype(np.int32)).to(dev) for l in range(LAYERS)]
+        wi = torch.from_numpy(wsame).to(dev)
+        oi = [torch.empty((16, HIDDEN), dtype=torch.bfloat16, device=dev) for _ in range(LAYERS)]
         us = graph_us_per_layer(
-            lambda: [qeg.moe_switchglu_forward_ws(xi, ii, wi, bank2, ws3, out=oi)
-                     for _ in range(LAYERS)], LAYERS)
+            lambda: [qeg.moe_switchglu_forward_ws(xi, ii[l], wi, bank2, ws3, out=oi[l])
+                     for l in range(LAYERS)], LAYERS)
         window["all_identical_T16"] = {
             "us_per_layer": us, "unique": K_TOP, "pairs_per_expert": 16,
             "gbs": K_TOP * BYTES_PER_EXPERT / (us * 1e-6) / 1e9,
-            "note": "42 launches of one layer (same bank, same routing) in a graph; L2 holds "
-                    "part of the 113 MB between launches"}
+            "frac_of_hbm_peak": K_TOP * BYTES_PER_EXPERT / (us * 1e-6) / 1e9
+            / measured_peaks()[0]}
         del ws3
     # mxfp4 banks: GLM-5.2's routed bank (E=256, hidden 6144, intermediate 2048, e2m1
     # codes with one e8m0 scale per 32 columns, 20,054,016 B per expert), drawn on the

@@ -220,6 +220,17 @@ moe_status moe_switchglu_forward_mxfp4(const uint16_t* x, const int32_t* topk_id
 moe_status moe_read_device_status(void* stream);
 
 /*
+ * The limit of every bounded wait in the kernels (a spin on an mbarrier or on a
+ * progress counter) on the current device, in nanoseconds: 0 restores the default of
+ * 2 s; values below 1000 are raised to 1000; above 2 s is MOE_ERR_INVALID_ARG.  A
+ * wait that runs out sets MOE_ERR_TIMEOUT in the error word and the kernel returns
+ * (a shorter limit lets a watchdog, or a test, see a stalled call sooner).  The waits
+ * that let copies and MMAs already in flight land before a CTA exits keep 2 s.  Takes
+ * effect for kernels launched after it; synchronous with respect to the device.
+ */
+moe_status moe_set_wait_limit_ns(unsigned long long ns);
+
+/*
  * Router step ahead of the layer (the routing of the tiny parity configuration:
  * top-k of softmax over the experts, renormalised over the k).  For each token t
  * of logits [T, E] (fp32, row-major, finite values): topk_idx[t, 0..k) = the k

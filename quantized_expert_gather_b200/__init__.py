@@ -72,6 +72,8 @@ def _load():
     lib.moe_switchglu_forward_mxfp4.argtypes = [vp] * 9 + [ci] * 5 + [vp, vp]
     lib.moe_switchglu_forward_mxfp4_ws.restype = ci
     lib.moe_switchglu_forward_mxfp4_ws.argtypes = [vp] * 9 + [ci] * 5 + [vp, vp, sz, vp]
+    lib.moe_set_wait_limit_ns.restype = ci
+    lib.moe_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
     lib.moe_read_device_status.restype = ci
     lib.moe_read_device_status.argtypes = [vp]
     return lib
@@ -358,6 +360,11 @@ def moe_switchglu_forward_mxfp4_ws(x, topk_idx, topk_w, bank: MxBank, workspace:
                                                  workspace.numel(), _stream(stream, x.device))
     _check(st, "moe_switchglu_forward_mxfp4_ws", check)
     return out
+
+
+def moe_set_wait_limit_ns(ns: int = 0, check: bool = True) -> int:
+    """Limit of the kernels' bounded waits on the current device (0: the default 2 s)."""
+    return _check(_lib.moe_set_wait_limit_ns(int(ns)), "moe_set_wait_limit_ns", check)
 
 
 def moe_read_device_status(stream=None) -> int:

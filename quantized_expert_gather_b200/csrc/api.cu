@@ -227,11 +227,11 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   const size_t usmem = route_union_smem_bytes(E);
   const size_t csmem = sizeof(int) * (size_t)P;
   // pairs per MMA chunk: 96 when experts average more than 40 pairs (fewer weight
-  // re-reads), 32 when they average at most 20 (two CTAs per SM), else 64
+  // re-reads), 32 when they average at most 20 (more accumulator buffers), else 64
   const int width = P > 40 * m ? 96 : (P <= 20 * m ? 32 : 64);
   const unsigned gsmem = width == 96 ? GCfg<96>::kSmem : width == 32 ? GCfg<32>::kSmem : GCfg<64>::kSmem;
   const int ki = width == 96 ? 5 : width == 32 ? 7 : 2;  // dyn_smem index of gate+up
-  const int grid = width == 32 ? 2 * d.sms : d.sms;
+  const int grid = d.sms;  // one CTA per SM (all of tensor memory, most of shared memory)
   if (usmem > (size_t)d.dyn_smem[1] || csmem > (size_t)d.dyn_smem[4] ||
       gsmem > (unsigned)d.dyn_smem[ki] || gsmem > (unsigned)d.dyn_smem[ki + 1]) {
     *why = MOE_ERR_UNSUPPORTED;
@@ -573,6 +573,13 @@ moe_status moe_switchglu_forward_mxfp4(const uint16_t* x, const int32_t* topk_id
     return s;
   return moe_switchglu_forward_mxfp4_ws(x, topk_idx, topk_w, wg_q, wg_e, wu_q, wu_e, wd_q, wd_e,
                                         T, k, E, hidden, inter, out, ws, bytes, stream);
+}
+
+moe_status moe_set_wait_limit_ns(unsigned long long ns) {
+  const unsigned long long v = ns == 0 ? kWaitLimitNs : (ns < 1000ull ? 1000ull : ns);
+  if (v > kWaitLimitNs) return MOE_ERR_INVALID_ARG;
+  const cudaError_t e = cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
 
 moe_status moe_read_device_status(void* stream) {

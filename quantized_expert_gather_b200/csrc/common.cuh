@@ -18,8 +18,16 @@ __device__ unsigned int g_error_word;
 
 __device__ __forceinline__ void set_error(unsigned bits) { atomicOr(&g_error_word, bits); }
 
-// Limit for every spin on an mbarrier: far beyond any legitimate wait.
+// Limit for every spin on an mbarrier or a counter: far beyond any legitimate wait.
+// g_wait_limit_ns is the limit in force (moe_set_wait_limit_ns may shorten it, so that
+// a test can make a wait run out); kWaitLimitNs stays the bound of the waits that let
+// copies and MMAs already in flight finish before a CTA exits.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+__device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
+
+__device__ __forceinline__ unsigned long long wait_limit() {
+  return *static_cast<volatile unsigned long long*>(&g_wait_limit_ns);
+}
 
 __device__ __forceinline__ unsigned long long globaltimer() {
   unsigned long long t;
@@ -64,13 +72,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of `bar` to complete, for at most kWaitLimitNs.
-// Returns false (and sets kErrTimeout) if the limit ran out.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
+// Wait for phase `parity` of `bar` to complete, for at most `limit` ns (the limit in
+// force by default).  Returns false (and sets kErrTimeout) if the limit ran out.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity,
+                                          unsigned long long limit = 0) {
   if (mbar_try_wait(bar, parity)) return true;
+  if (limit == 0) limit = wait_limit();
   const unsigned long long t0 = globaltimer();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit) {
       set_error(kErrTimeout);
       return false;
     }

@@ -237,9 +237,9 @@ struct LayerArgs {
 //   .x = low bytes of columns 8m+0,2,4,6   .y = low bytes of 8m+1,3,5,7
 //   .z = high bytes of columns 8m+0,2,4,6  .w = high bytes of 8m+1,3,5,7
 // or (mxfp4) .x / .z = low / high bytes of columns 8m+0..3, .y / .w of 8m+4..7,
-// followed (at byte 2048 R) by float2 sc[ch] = (2^(e - 14), sum of the chunk's 32
-// values).  The same layout serves in global memory (converted once per call) and
-// in shared memory (copied per work item).
+// followed (at byte 2048 R) by float2 sc[ch] = (2^(e - 14) (2^(e - 18) in the affine
+// layout, whose chunk sums are 16 times too large), sum of the chunk's 32
+// values).  Resident x rows and every activation set use it, in shared memory.
 constexpr uint32_t kNibbleBytes = 0x0F0F0F0Fu;
 
 __device__ __forceinline__ int dp4a_lo(uint32_t q, uint32_t d, int c) {
@@ -345,8 +345,8 @@ __device__ __forceinline__ float2 chunk_sb(const uint16_t* s, const uint16_t* b,
     const float h = mx_half_scale(reinterpret_cast<const uint8_t*>(s)[ch]);
     return make_float2(h, -12.0f * h);
   } else {
-    // chunk_dot returns 16 x the sum in this format
-    return make_float2(bf16_bits_to_float(s[ch >> 1]) * 0.0625f, bf16_bits_to_float(b[ch >> 1]));
+    // (chunk_dot returns 16 x the sum in this format; the activation scale holds 1/16)
+    return make_float2(bf16_bits_to_float(s[ch >> 1]), bf16_bits_to_float(b[ch >> 1]));
   }
 }
 
@@ -397,6 +397,9 @@ __device__ __forceinline__ float2 fixed_point_quarter(const uint4 v, unsigned gm
   else if (xm == 255) scale = __uint_as_float(0x7fc00000u);   // Inf / NaN present
   else if (xm >= 15) scale = __uint_as_float(static_cast<uint32_t>(xm - 14) << 23);
   else scale = __uint_as_float(1u << (xm + 8));               // 2^(xm-141), subnormal
+  // affine chunk sums come out 16 times too large (chunk_dot): the row's scale
+  // carries the 1/16 (exact, a power of two)
+  if (F != kFmtMx) scale *= 0.0625f;
   return make_float2(scale, sum);
 }
 
@@ -424,7 +427,7 @@ __device__ __forceinline__ bool wait_counter(const unsigned* p, unsigned target)
   const unsigned long long t0 = globaltimer();
   while (ld_acquire_gpu(p) < target) {
     __nanosleep(32);
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > wait_limit()) {
       set_error(kErrTimeout);
       return false;
     }
@@ -600,19 +603,36 @@ __device__ __forceinline__ void convert_set(const LayerArgs& a, const LayerGeom&
   const int D = phase_b ? a.I : a.H, R = phase_b ? G.rounds_b : G.rounds_a, nch = D / 32;
   const unsigned stride = act_bytes(R);
   const int nq = nt * nch * 4;  // quarters of 8 columns
-  for (int q = threadIdx.x; q < nq; q += kConsumerThreads) {
-    const int m = q & 3, tc = q >> 2, t = tc / nch, ch = tc % nch;
-    uint4 v;
-    if (phase_b)
-      v = __ldcg(reinterpret_cast<const uint4*>(a.h + (size_t)(p0 + t) * a.I + ch * 32 + m * 8));
-    else
-      v = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)tok_of[p0 + t] * a.H + ch * 32 +
-                                               m * 8));
-    uint4 packed;
-    const float2 sc = fixed_point_quarter<F>(v, 0xfu << (lane & ~3), packed);
-    unsigned char* row = buf + (size_t)t * stride;
-    reinterpret_cast<uint4*>(row)[((ch / 32) * 4 + m) * 32 + (ch % 32)] = packed;
-    if (m == 0) reinterpret_cast<float2*>(row + act_digit_bytes(R))[ch] = sc;
+  // kBatch quarters per thread at a time: their loads are all issued before the first
+  // conversion waits on one
+  constexpr int kBatch = 4;
+  for (int q0 = threadIdx.x; q0 < nq; q0 += kBatch * kConsumerThreads) {
+    uint4 v[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int q = q0 + i * kConsumerThreads;
+      v[i] = make_uint4(0u, 0u, 0u, 0u);
+      if (q < nq) {
+        const int m = q & 3, tc = q >> 2, t = tc / nch, ch = tc % nch;
+        if (phase_b)
+          v[i] = __ldcg(reinterpret_cast<const uint4*>(a.h + (size_t)(p0 + t) * a.I + ch * 32 + m * 8));
+        else
+          v[i] = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)tok_of[p0 + t] * a.H + ch * 32 +
+                                                      m * 8));
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int q = q0 + i * kConsumerThreads;
+      if (q < nq) {  // the four lanes of a chunk agree (nq is a multiple of 4)
+        const int m = q & 3, tc = q >> 2, t = tc / nch, ch = tc % nch;
+        uint4 packed;
+        const float2 sc = fixed_point_quarter<F>(v[i], 0xfu << (lane & ~3), packed);
+        unsigned char* row = buf + (size_t)t * stride;
+        reinterpret_cast<uint4*>(row)[((ch / 32) * 4 + m) * 32 + (ch % 32)] = packed;
+        if (m == 0) reinterpret_cast<float2*>(row + act_digit_bytes(R))[ch] = sc;
+      }
+    }
   }
 }
 
@@ -624,14 +644,30 @@ __device__ __forceinline__ void convert_x_all(const LayerArgs& a, const LayerGeo
   const int nch = a.H / 32, R = G.rounds_a;
   const unsigned stride = act_bytes(R);
   const int nq = a.T * nch * 4;  // quarters of 8 columns
-  for (int q = t0; q < nq; q += nthr) {
-    const int m = q & 3, tc = q >> 2, t = tc / nch, ch = tc % nch;
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H + ch * 32 + m * 8));
-    uint4 packed;
-    const float2 sc = fixed_point_quarter<F>(v, 0xfu << (lane & ~3), packed);
-    unsigned char* row = xres + (size_t)t * stride;
-    reinterpret_cast<uint4*>(row)[((ch / 32) * 4 + m) * 32 + (ch % 32)] = packed;
-    if (m == 0) reinterpret_cast<float2*>(row + act_digit_bytes(R))[ch] = sc;
+  constexpr int kBatch = 4;      // loads issued before the first conversion
+  for (int q0 = t0; q0 < nq; q0 += kBatch * nthr) {
+    uint4 v[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int q = q0 + i * nthr;
+      v[i] = make_uint4(0u, 0u, 0u, 0u);
+      if (q < nq) {
+        const int m = q & 3, tc = q >> 2, t = tc / nch, ch = tc % nch;
+        v[i] = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H + ch * 32 + m * 8));
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int q = q0 + i * nthr;
+      if (q < nq) {  // the four lanes of a chunk agree (nq and nthr are multiples of 4)
+        const int m = q & 3, tc = q >> 2, t = tc / nch, ch = tc % nch;
+        uint4 packed;
+        const float2 sc = fixed_point_quarter<F>(v[i], 0xfu << (lane & ~3), packed);
+        unsigned char* row = xres + (size_t)t * stride;
+        reinterpret_cast<uint4*>(row)[((ch / 32) * 4 + m) * 32 + (ch % 32)] = packed;
+        if (m == 0) reinterpret_cast<float2*>(row + act_digit_bytes(R))[ch] = sc;
+      }
+    }
   }
 }
 
@@ -829,7 +865,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
         t_prog = globaltimer();
       } else {
         if (lane0(s_abort != 0)) break;
-        if (lane0(globaltimer() - t_prog > kWaitLimitNs)) {
+        if (lane0(globaltimer() - t_prog > wait_limit())) {
           if (lane == 0) {
             set_error(kErrTimeout);
             s_abort = 1;
@@ -845,7 +881,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
     // 0's (uniform control flow).
     auto timed_out = [&](unsigned long long t0) -> bool {
       if (lane0(s_abort != 0)) return true;
-      if (lane0(globaltimer() - t0 > kWaitLimitNs)) {
+      if (lane0(globaltimer() - t0 > wait_limit())) {
         if (lane == 0) {
           set_error(kErrTimeout);
           s_abort = 1;
@@ -935,7 +971,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       const unsigned long long t0 = globaltimer();
       while (!mbar_try_wait(bar, parity)) {
         if (s_abort) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > wait_limit()) {
           set_error(kErrTimeout);
           s_abort = 1;
           return false;
@@ -969,7 +1005,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
             const unsigned target = (unsigned)bpe_a * (unsigned)((n_i + sega - 1) / sega);
             const unsigned long long t0 = globaltimer();
             while (!s_abort && ld_acquire_gpu(&hdone[slot]) < target) {
-              if (globaltimer() - t0 > kWaitLimitNs) {
+              if (globaltimer() - t0 > wait_limit()) {
                 set_error(kErrTimeout);
                 s_abort = 1;
               }
@@ -1070,7 +1106,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       if (threadIdx.x == 0) {
         const unsigned long long t0 = globaltimer();
         while (!s_abort && ld_acquire_gpu(&ydone[rb]) < (unsigned)nsb) {
-          if (globaltimer() - t0 > kWaitLimitNs) {
+          if (globaltimer() - t0 > wait_limit()) {
             set_error(kErrTimeout);
             s_abort = 1;
           }

@@ -186,22 +186,24 @@ def test_grouped_large_window_every_token():
 
 # ----------------------------------------------------------------- timeouts ---
 def test_bounded_wait_runs_out_and_next_call_is_clean():
-    """A workspace whose work-item counter is preset past the last item: no CTA takes any
-    item, so the combine's bounded wait for the down projection never completes.  The call
-    must return (after the wait limit) with MOE_ERR_TIMEOUT in the error word, and a call
-    on the cleared workspace must match the oracle again.  The failure is made on the host
-    (a counter value); nothing faults or hangs."""
-    T, k, E, Hs, Is = 2, 4, 16, 512, 256
+    """The kernels' wait limit shortened to 1 us: the layer's first waits (for the first
+    weight stage, about 2 us after launch) run out, the call returns with MOE_ERR_TIMEOUT
+    in the error word, and with the default limit back and the workspace's counter region
+    cleared the next call matches the oracle.  The failure is made through the limit;
+    nothing faults or hangs."""
+    T, k, E, Hs, Is = 4, 8, 64, 4096, 2048
     L = make_layer(T, k, E, Hs, Is, seed=6400)
     bank = to_dev_bank(L)
     x, idx, w = to_dev_inputs(L)
     ws = qeg.moe_workspace(T, k, E, Hs, Is)
-    # the work-item counter: word 1 + 1024 + 512 of the counter region (see the header)
-    words = ws[:4 * 1539].view(torch.int32)
-    words[1 + 1024 + 512] = 1 << 20
-    qeg.moe_switchglu_forward_ws(x, idx, w, bank, ws)
-    assert qeg.moe_read_device_status() == qeg.MOE_ERR_TIMEOUT
-    assert qeg.moe_read_device_status() == qeg.MOE_OK  # the read clears the word
+    assert qeg.moe_read_device_status() == qeg.MOE_OK
+    qeg.moe_set_wait_limit_ns(1000)
+    try:
+        qeg.moe_switchglu_forward_ws(x, idx, w, bank, ws)
+        assert qeg.moe_read_device_status() == qeg.MOE_ERR_TIMEOUT
+    finally:
+        qeg.moe_set_wait_limit_ns(0)
+    assert qeg.moe_read_device_status() == qeg.MOE_OK  # the read cleared the word
     ws[:4 * 1539].zero_()  # the caller clears its workspace after a timeout
     out = qeg.moe_switchglu_forward_ws(x, idx, w, bank, ws)
     torch.cuda.synchronize()

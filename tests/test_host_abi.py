@@ -28,7 +28,7 @@ def test_header_declares_the_entry_points():
               "moe_select_path", "moe_workspace_layout", "moe_switchglu_forward_static",
               "moe_router_topk", "moe_switchglu_forward_mxfp4",
               "moe_switchglu_forward_mxfp4_ws", "moe_workspace_size_mxfp4",
-              "moe_select_path_mxfp4"):
+              "moe_select_path_mxfp4", "moe_set_wait_limit_ns"):
         assert n in names
 
 
