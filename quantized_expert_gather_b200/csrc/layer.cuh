@@ -416,8 +416,12 @@ __device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned* p) {
   return v;
 }
 
-__device__ __forceinline__ void red_release_gpu(unsigned* p, unsigned v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+__device__ __forceinline__ void red_relaxed_gpu(unsigned* p, unsigned v) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
 
 // Spin (bounded) until *p >= target.  Returns false and sets kErrTimeout if the
@@ -563,6 +567,130 @@ __device__ __forceinline__ float dispatch_b(int R, const unsigned char* bq, cons
   return rows_b<NT, 8, F>(bq, bs, bb, row0, nrows, I, act, stride, lane, vid);
 }
 
+// Lane holding value v after warp_reduce_scatter<V> (the sum of value v is in every
+// lane whose bits 16, 8, ... down to 32 / V spell v, high bit first).
+template <int V>
+__device__ __forceinline__ constexpr int rs_holder(int v) {
+  int l = 0;
+  for (int w = V, m = 16; w > 1; w >>= 1, m >>= 1)
+    if (v & (w >> 1)) l |= m;
+  return l;
+}
+
+// Two consecutive blocks of one segment at once (at most two pairs).  Phase A takes
+// the warp's row of gate and of up from each block, four rows that share each
+// activation chunk load; phase B the warp's four rows of each block, eight rows.  The
+// rows' sums are independent dp4a chains, so a warp has two blocks' work in flight,
+// and the per-block costs (reduction, publication) are shared.  R is a run-time
+// bound (one loop body for every width).
+//
+// Phase A: rows q/s/b[0..3] = gate and up of block 0, gate and up of block 1.  Lane t
+// (t < NT) returns o[r] = row r's sum for pair t.
+template <int NT, int F>
+__device__ __forceinline__ void rows_a2(const unsigned char* const (&q)[4],
+                                        const uint16_t* const (&s)[4],
+                                        const uint16_t* const (&b)[4], int R, int H,
+                                        const unsigned char* const (&act)[kNT], int lane,
+                                        float (&o)[4]) {
+  constexpr int V = 4 * NT;
+  float acc[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) acc[v] = 0.f;
+  const int nch = H / 32;
+#pragma unroll 1
+  for (int i = 0; i < R; ++i) {
+    const int ch = i * 32 + lane;
+    if (ch < nch) {
+      uint4 w[4];
+      float2 sb[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        w[r] = *reinterpret_cast<const uint4*>(q[r] + ch * 16);
+        sb[r] = chunk_sb<F>(s[r], b[r], ch);
+      }
+      uint4 xd[NT][4];
+      float2 sc[NT];
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        load_xq(act[t], i, lane, xd[t]);
+        sc[t] = load_sc(act[t], R, ch);
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        uint32_t qs[8];
+        split_codes_f<F>(w[r], qs);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const float d = static_cast<float>(chunk_dot<F>(qs, xd[t]));
+          acc[r * NT + t] = fmaf(sb[r].x * sc[t].x, d, fmaf(sb[r].y, sc[t].y, acc[r * NT + t]));
+        }
+      }
+    }
+  }
+  int vid;
+  const float tot = warp_reduce_scatter<V>(acc, lane, vid);
+#pragma unroll
+  for (int r = 0; r < 4; ++r) o[r] = 0.f;
+#pragma unroll
+  for (int v = 0; v < V; ++v) {
+    const float x = __shfl_sync(kFull, tot, rs_holder<V>(v));
+    if (lane == v % NT) o[v / NT] = x;
+  }
+}
+
+// Phase B: rows warp + kWarps q (q < kMaxRowsPerWarpB) of block 0 (rows < n0) and of
+// block 1 (rows < n1), NT pairs.  Returns the sum this lane holds after the
+// reduce-scatter and its index q' NT + t in `vid` (q' < 4: block 0's row q', else
+// block 1's row q' - 4), -1 when it holds none.
+template <int NT, int F>
+__device__ __forceinline__ float rows_b2(const unsigned char* const (&bq)[2],
+                                         const uint16_t* const (&bs)[2],
+                                         const uint16_t* const (&bb)[2], int n0, int n1,
+                                         int R, int I, const unsigned char* act,
+                                         unsigned stride, int lane, int warp, int& vid) {
+  constexpr int Q = 2 * kMaxRowsPerWarpB;
+  constexpr int V = Q * NT;
+  float acc[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) acc[v] = 0.f;
+  const int nch = I / 32, qstride = I / 2, sstride = I / 64;
+#pragma unroll 1
+  for (int i = 0; i < R; ++i) {
+    const int ch = i * 32 + lane;
+    if (ch < nch) {
+      uint4 xd[NT][4];
+      float2 sc[NT];
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const unsigned char* row = act + t * stride;
+        sc[t] = load_sc(row, R, ch);
+        load_xq(row, i, lane, xd[t]);
+      }
+#pragma unroll
+      for (int qq = 0; qq < Q; ++qq) {
+        const int blk = qq / kMaxRowsPerWarpB;
+        const int r = warp + kWarps * (qq % kMaxRowsPerWarpB);
+        if (r < (blk ? n1 : n0)) {
+          uint32_t qs[8];
+          split_codes_f<F>(
+              *reinterpret_cast<const uint4*>(bq[blk] + (size_t)r * qstride + ch * 16), qs);
+          const float2 sb = chunk_sb<F>(bs[blk] + r * sstride, bb[blk] + r * sstride, ch);
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            const float d = static_cast<float>(chunk_dot<F>(qs, xd[t]));
+            acc[qq * NT + t] = fmaf(sb.x * sc[t].x, d, fmaf(sb.y, sc[t].y, acc[qq * NT + t]));
+          }
+        }
+      }
+    }
+  }
+  int v_id;
+  const float v = warp_reduce_scatter<V>(acc, lane, v_id);
+  constexpr int kHolderMask = (32 / V) - 1;
+  vid = (lane & kHolderMask) == 0 ? v_id : -1;
+  return v;
+}
+
 // mbarrier phase test without suspending (for wait loops that do other work).
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, unsigned parity) {
   uint32_t ok;
@@ -697,13 +825,56 @@ __device__ __forceinline__ int make_segments(const int* offs, int u, int seg, in
   return base;
 }
 
+// Balanced split of one phase's blocks among the CTAs by cost: a block of a segment of
+// nt pairs costs 2 + nt (its weights' bytes are the same for every nt; the per-pair
+// compute is about half the per-block work at one pair), so CTAs whose share has
+// segments of many pairs take fewer blocks.  Returns the first block whose cost
+// prefix reaches t (blocks in segment order, bpe per segment).  Run by one warp.
+__device__ __forceinline__ int block_at_cost(const int* s_nt, int nseg, int bpe, long long t,
+                                             int lane) {
+  if (t <= 0) return 0;
+  long long acc = 0;
+  for (int b0 = 0; b0 < nseg; b0 += 32) {
+    const int sidx = b0 + lane;
+    const long long w = sidx < nseg ? (long long)(2 + s_nt[sidx]) : 0;
+    const long long cs = w * bpe;
+    long long incl = cs;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const long long v = __shfl_up_sync(kFull, incl, d);
+      if (lane >= d) incl += v;
+    }
+    const unsigned hit = __ballot_sync(kFull, sidx < nseg && acc + incl >= t);
+    if (hit) {
+      const int L = __ffs(hit) - 1;
+      const long long excl = __shfl_sync(kFull, incl - cs, L);
+      const long long wl = __shfl_sync(kFull, w, L);
+      const long long k = (t - acc - excl + wl - 1) / wl;
+      return (b0 + L) * bpe + (int)k;
+    }
+    acc += __shfl_sync(kFull, incl, 31);
+  }
+  return nseg * bpe;
+}
+
+// This CTA's share [lo, hi) of one phase's blocks.  Run by one warp.
+__device__ __forceinline__ void cost_share(const int* s_nt, int nseg, int bpe, int lane, int& lo,
+                                           int& hi) {
+  long long tot = 0;
+  for (int sidx = lane; sidx < nseg; sidx += 32) tot += (long long)bpe * (2 + s_nt[sidx]);
+#pragma unroll
+  for (int d = 16; d >= 1; d >>= 1) tot += __shfl_xor_sync(kFull, tot, d);
+  lo = block_at_cost(s_nt, nseg, bpe, tot * blockIdx.x / gridDim.x, lane);
+  hi = block_at_cost(s_nt, nseg, bpe, tot * (blockIdx.x + 1) / gridDim.x, lane);
+}
+
 // 10 warps: 8 compute warps, a producer warp and a helper warp (see the top of this file).
 template <int F>
 __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   // window plan, set by warp 0 after the union: segments of phase A and B, ring depth,
   // resident x rows, the wide layout
-  __shared__ int s_u, s_nsa, s_nsb, s_ns, s_xres, s_wide, s_sega;
+  __shared__ int s_u, s_nsa, s_nsb, s_ns, s_xres, s_wide, s_sega, s_a0, s_a1, s_b0, s_b1;
   __shared__ unsigned s_act_off, s_act_size;
   __shared__ volatile int s_abort;
   __shared__ volatile int s_pub;  // blocks published by the helper warp
@@ -770,6 +941,10 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
     const int segb = max((int)(act_size / stride_b), 1);
     const int nsa = make_segments(offs, u, sega, sa_slot, sa_pos, sa_nt, lane);
     const int nsb = make_segments(offs, u, segb, sb_slot, sb_pos, sb_nt, lane);
+    __syncwarp();
+    int ra0, ra1, rb0, rb1;
+    cost_share(sa_nt, nsa, a.I / kRowsA, lane, ra0, ra1);
+    cost_share(sb_nt, nsb, (a.H + G.rows_b - 1) / G.rows_b, lane, rb0, rb1);
     if (lane == 0) {
       s_u = u;
       s_nsa = nsa;
@@ -780,6 +955,10 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       s_sega = sega;
       s_act_off = G.tables + (unsigned)ns * G.stage_bytes;
       s_act_size = act_size;
+      s_a0 = ra0;
+      s_a1 = ra1;
+      s_b0 = rb0;
+      s_b1 = rb1;
     }
     __syncwarp();
     named_barrier_arrive(kBarUnion, 64);  // the producer may start (it waits on this)
@@ -817,16 +996,14 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
     if (lane == 0) *a.ex_u = u;
   }
 
-  // ---- this CTA's blocks: a contiguous, balanced share of the phase-A blocks (kRowsA
-  // rows of gate and of up each, per phase-A segment), then of the phase-B blocks
-  // (rows_b rows of down each, per phase-B segment), both in segment order.  Every
-  // block is 2 kRowsA H/2 + scales (A) or rows_b I/2 + scales (B) bytes; the two are
-  // equal at the 4096/2048 shape ----
+  // ---- this CTA's blocks: a contiguous share of the phase-A blocks (kRowsA rows of
+  // gate and of up each, per phase-A segment), then of the phase-B blocks (rows_b rows
+  // of down each, per phase-B segment), both in segment order, balanced by cost
+  // (cost_share).  Every block is 2 kRowsA H/2 + scales (A) or rows_b I/2 + scales (B)
+  // bytes; the two are equal at the 4096/2048 shape ----
   const int bpe_a = a.I / kRowsA;                     // phase-A blocks per segment
   const int bpe_b = (a.H + G.rows_b - 1) / G.rows_b;  // phase-B blocks per segment
-  const long long NA = (long long)nsa * bpe_a, NB = (long long)nsb * bpe_b;
-  const int a0 = (int)(NA * blockIdx.x / gridDim.x), a1 = (int)(NA * (blockIdx.x + 1) / gridDim.x);
-  const int b0 = (int)(NB * blockIdx.x / gridDim.x), b1 = (int)(NB * (blockIdx.x + 1) / gridDim.x);
+  const int a0 = s_a0, a1 = s_a1, b0 = s_b0, b1 = s_b1;  // cost-balanced shares (cost_share)
   const int nA = a1 - a0, nblk = nA + (b1 - b0);
   auto block_of = [&](int j, bool& pb, int& sg, int& row0) {
     if (j < nA) {
@@ -848,20 +1025,38 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
     // (its h rows written), a phase-B block adds 1 to ydone of its row block.  The
     // compute warps' done arrivals released their stores at CTA scope and the test
     // below acquires them; the device-scope release reductions pass them on
-    // (causality order is transitive across the two scopes).
+    // (causality order is transitive across the two scopes).  All the finished blocks
+    // found in one pass go out behind one device-scope fence (a fence followed by
+    // relaxed reductions releases each of them), and consecutive blocks of one counter
+    // add together: one fence and a few reductions per pass, however many blocks.
     unsigned long long t_prog = globaltimer();
     for (int j = 0; j < nblk;) {
-      if (lane0(mbar_test(&done[j % kPubRing], (j / kPubRing) & 1))) {
-        bool pb;
-        int sg, row0;
-        block_of(j, pb, sg, row0);
+      int n = 0;
+      while (j + n < nblk && n < kPubRing &&
+             lane0(mbar_test(&done[(j + n) % kPubRing], ((j + n) / kPubRing) & 1)))
+        ++n;
+      if (n > 0) {
         if (lane == 0) {
-          if (!pb) red_release_gpu(&hdone[sa_slot[sg]], 1u);
-          else red_release_gpu(&ydone[row0 / G.rows_b], 1u);
-          s_pub = j + 1;
+          fence_acq_rel_gpu();
+          unsigned* cur = nullptr;
+          unsigned cnt = 0;
+          for (int q = j; q < j + n; ++q) {
+            bool pb;
+            int sg, row0;
+            block_of(q, pb, sg, row0);
+            unsigned* c = pb ? &ydone[row0 / G.rows_b] : &hdone[sa_slot[sg]];
+            if (c != cur) {
+              if (cnt) red_relaxed_gpu(cur, cnt);
+              cur = c;
+              cnt = 0;
+            }
+            ++cnt;
+          }
+          red_relaxed_gpu(cur, cnt);
+          s_pub = j + n;
         }
         __syncwarp();
-        ++j;
+        j += n;
         t_prog = globaltimer();
       } else {
         if (lane0(s_abort != 0)) break;
@@ -872,7 +1067,8 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
           }
           break;
         }
-        __nanosleep(64);
+        // suspended (not spinning on issue slots) until block j is done, or briefly
+        mbar_try_wait(&done[j % kPubRing], (j / kPubRing) & 1);
       }
     }
   } else if (warp == kWarps) {
@@ -897,7 +1093,8 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       const int st = j % NS;
       if (j >= NS) {  // the compute warps are done with block j - NS
         const unsigned long long t0 = globaltimer();
-        while (!lane0(mbar_test(&empty[st], ((j / NS) - 1) & 1)))
+        // (try_wait suspends the warp, leaving the issue slots to the compute warps)
+        while (!lane0(mbar_try_wait(&empty[st], ((j / NS) - 1) & 1)))
           if (timed_out(t0)) {
             ok = false;
             break;
@@ -994,26 +1191,27 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
         // All compute warps are past the previous set's blocks, so the activation area
         // is free; phase B waits (bounded) until every phase-A block of the expert has
         // published its h rows.
+        // For phase B one thread (warp 0's lane 0) waits, with a short back-off, until
+        // hdone[expert] counts every phase-A block of the expert; its acquire reaches
+        // the other warps through set_in (release/acquire at CTA scope), so one poller
+        // per CTA loads the counter.
+        __syncwarp();
+        if (phase_b && warp == 0 && lane == 0) {
+          const int slot = sb_slot[sg];
+          const int n_i = offs[slot + 1] - offs[slot];
+          const unsigned target = (unsigned)bpe_a * (unsigned)((n_i + sega - 1) / sega);
+          const unsigned long long t0 = globaltimer();
+          while (!s_abort && ld_acquire_gpu(&hdone[slot]) < target) {
+            if (globaltimer() - t0 > wait_limit()) {
+              set_error(kErrTimeout);
+              s_abort = 1;
+            }
+            __nanosleep(32);
+          }
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&set_in[0]);
         if (!wait_cons(&set_in[0], nsets & 1)) break;
-        if (phase_b) {
-          bool ok = true;
-          if (lane == 0) {
-            const int slot = sb_slot[sg];
-            const int n_i = offs[slot + 1] - offs[slot];
-            const unsigned target = (unsigned)bpe_a * (unsigned)((n_i + sega - 1) / sega);
-            const unsigned long long t0 = globaltimer();
-            while (!s_abort && ld_acquire_gpu(&hdone[slot]) < target) {
-              if (globaltimer() - t0 > wait_limit()) {
-                set_error(kErrTimeout);
-                s_abort = 1;
-              }
-            }
-            ok = !s_abort;
-          }
-          if (!lane0(ok)) break;
-        }
         convert_set<F>(a, G, phase_b, tok_of, p0, nt, actp, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(&set_out[0]);
@@ -1021,6 +1219,80 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
         ++nsets;
       }
       const unsigned char* buf = ring + (size_t)st * G.stage_bytes;
+      // Block j + 1 of the same segment (next rows, at most two pairs) is taken with
+      // block j (rows_a2 / rows_b2); the schedule is a pure function of j, so every
+      // compute warp makes the same choice.
+      bool paired = false;
+      if (nt <= 2 && j + 1 < nblk) {
+        bool pb1;
+        int sg1, r1;
+        block_of(j + 1, pb1, sg1, r1);
+        paired = pb1 == phase_b && sg1 == sg && r1 == row0 + (phase_b ? G.rows_b : kRowsA);
+      }
+      if (paired) {
+        const int st1 = (j + 1) % NS;
+        if (!wait_cons(&full[st1], ((j + 1) / NS) & 1)) break;
+        const unsigned char* buf1 = ring + (size_t)st1 * G.stage_bytes;
+        if (!phase_b) {
+          const unsigned char* q4[4];
+          const uint16_t* s4[4];
+          const uint16_t* b4[4];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const unsigned char* m = (r < 2 ? buf : buf1) + ((r & 1) ? G.a_mat : 0);
+            q4[r] = m + (size_t)warp * (a.H / 2);
+            s4[r] = reinterpret_cast<const uint16_t*>(m + G.a_q) + warp * (a.H / 64);
+            b4[r] = reinterpret_cast<const uint16_t*>(m + G.a_q + G.a_sb) + warp * (a.H / 64);
+          }
+          const unsigned char* arow[kNT];
+#pragma unroll
+          for (int t = 0; t < kNT; ++t)
+            arow[t] = x_res ? actp + (t < nt ? tok_of[p0 + t] : 0) * stride_a
+                            : actp + t * stride_a;
+          float o[4];
+          if (nt == 1) rows_a2<1, F>(q4, s4, b4, G.rounds_a, a.H, arow, lane, o);
+          else rows_a2<2, F>(q4, s4, b4, G.rounds_a, a.H, arow, lane, o);
+          if (lane < nt) {
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const float g = round_to_bf16(o[2 * h2]), hu = round_to_bf16(o[2 * h2 + 1]);
+              a.h[(size_t)(p0 + lane) * a.I + row0 + kRowsA * h2 + warp] =
+                  float_to_bf16_bits(__fdividef(g, 1.0f + __expf(-g)) * hu);
+            }
+          }
+        } else {
+          const int n0 = min(G.rows_b, a.H - row0);
+          const int n1 = min(G.rows_b, a.H - row0 - G.rows_b);
+          const unsigned char* bq2[2] = {buf, buf1};
+          const uint16_t* bs2[2] = {reinterpret_cast<const uint16_t*>(buf + G.b_q),
+                                    reinterpret_cast<const uint16_t*>(buf1 + G.b_q)};
+          const uint16_t* bb2[2] = {reinterpret_cast<const uint16_t*>(buf + G.b_q + G.b_sb),
+                                    reinterpret_cast<const uint16_t*>(buf1 + G.b_q + G.b_sb)};
+          int vid;
+          const float v =
+              nt == 1 ? rows_b2<1, F>(bq2, bs2, bb2, n0, n1, G.rounds_b, a.I, actp, stride_b,
+                                      lane, warp, vid)
+                      : rows_b2<2, F>(bq2, bs2, bb2, n0, n1, G.rounds_b, a.I, actp, stride_b,
+                                      lane, warp, vid);
+          if (vid >= 0) {
+            const int qq = vid / nt, t = vid % nt;
+            const int blk = qq / kMaxRowsPerWarpB;
+            const int r = warp + kWarps * (qq % kMaxRowsPerWarpB);
+            if (r < (blk ? n1 : n0))
+              a.y[(size_t)(p0 + t) * a.H + row0 + blk * G.rows_b + r] = v;
+          }
+        }
+        // done reading stages st and st1; both blocks' outputs written
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&empty[st]);
+          mbar_arrive(&done[j % kPubRing]);
+          mbar_arrive(&empty[st1]);
+          mbar_arrive(&done[(j + 1) % kPubRing]);
+        }
+        ++j;
+        continue;
+      }
       // the set's pairs in chunks of kNT, the block's weights read again per chunk
       int nrows = 0;
       for (int c0 = 0; c0 < nt; c0 += kNT) {
@@ -1110,6 +1382,7 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
             set_error(kErrTimeout);
             s_abort = 1;
           }
+          __nanosleep(32);
         }
         __threadfence();
       }

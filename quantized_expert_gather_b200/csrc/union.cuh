@@ -38,6 +38,42 @@ __device__ inline int warp_route_union(const int* __restrict__ idx, int P, int E
                                        int* rank, int* unique, int* offsets, int* pair_list,
                                        int* n_valid_out) {
   const int lane = threadIdx.x & 31;
+  if (P <= 32) {
+    // A window of at most 32 pairs: one key (expert, pair) per lane, sorted across the
+    // warp by a bitonic network (15 compare-exchange steps), so no pass over the E
+    // experts is needed.  Invalid pairs sort last and are left out.
+    const int e = lane < P ? idx[lane] : -1;
+    const bool valid = lane < P && e >= 0 && e < E;
+    if (__any_sync(kFull, lane < P && !valid)) {
+      if (lane == 0) set_error(kErrExpertIndex);
+    }
+    int key = valid ? ((e << 5) | lane) : 0x7fffffff;
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        const int other = __shfl_xor_sync(kFull, key, j);
+        const bool keep_min = ((lane & j) == 0) == ((lane & k) == 0);
+        key = keep_min ? min(key, other) : max(key, other);
+      }
+    const bool kv = key != 0x7fffffff;
+    const int ke = key >> 5;
+    const int prev = __shfl_up_sync(kFull, ke, 1);
+    const bool first = kv && (lane == 0 || prev != ke);
+    const unsigned heads = __ballot_sync(kFull, first);
+    const int nv = __popc(__ballot_sync(kFull, kv));
+    if (first) {
+      const int slot = __popc(heads & lanemask_lt());
+      unique[slot] = ke;
+      offsets[slot] = lane;
+    }
+    const int u = __popc(heads);
+    if (lane == 0) offsets[u] = nv;
+    if (lane < P) pair_list[lane] = kv ? (key & 31) : -1;
+    __syncwarp();
+    *n_valid_out = nv;
+    return u;
+  }
   for (int e = lane; e < E; e += 32) cnt[e] = 0;
   __syncwarp();
   bool bad = false;
