@@ -21,23 +21,25 @@
 //   combine   out[t] = bf16(sum_j w[t,j] * y[t,j]) per block of rows_b output
 //             rows, by CTA (row block mod grid) once every segment of the row
 //             block has published (counter ydone[rb]).
-// Each CTA takes a contiguous, balanced share of all phase-A blocks (segment
-// order), then of all phase-B blocks: every block carries the same bytes at the
-// 4096/2048 shape, so the CTAs stream equal shares and finish together, and a
-// CTA's share spans few segments, so its activation sets change rarely.  An
+// Each CTA takes a contiguous share of all phase-A blocks (segment order), then
+// of all phase-B blocks, balanced by cost (a block's bytes are the same for every
+// segment; its compute grows with the segment's pairs), so the CTAs finish
+// together, and a CTA's share spans few segments, so its activation sets change
+// rarely.  An
 // expert with more than `seg` pairs in the window forms several segments and is
 // streamed once per segment.  Every spin on a counter or barrier is bounded
 // (common.cuh); the counters are zero again when the kernel ends.
 //
-// Warps: 8 compute warps, one producer warp and one helper warp.  The producer
-// issues this CTA's weight blocks into a ring of stages (1-D bulk copies, mbarrier
-// completion); the helper publishes finished blocks to the other CTAs (counter
-// release reductions); the compute warps convert each new activation set (the
-// segment's x rows for phase A, its h rows for phase B) into shared memory
-// together and compute.
+// Warps: 16 compute warps in two teams of 8, one producer warp and one helper
+// warp.  The producer issues this CTA's weight blocks into a ring of stages (1-D
+// bulk copies, mbarrier completion); the helper publishes finished blocks to the
+// other CTAs (counter release reductions); the teams take alternate blocks, and
+// all compute warps convert each new activation set (the segment's x rows for
+// phase A, its h rows for phase B) into shared memory together.
 //
-// Compute: each warp owns whole rows (phase A: one row of Wg and the same row
-// of Wu; phase B: up to 4 rows of Wd) over the full input width.  Lane l takes
+// Compute: each warp owns whole rows of its team's block (phase A: one row of Wg
+// and the same row of Wu; phase B: up to 4 rows of Wd) over the full input width,
+// one pair at a time.  Lane l takes
 // the 32-column chunks l, l+32, ... of its rows, so one lane chunk sits inside
 // one quantisation group (64 columns affine, 32 mxfp4):
 //     partial = s * sum_c q_c x_c + b * sum_c x_c.
@@ -58,13 +60,20 @@ namespace qeg {
 constexpr int kFmtAffine = 0;
 constexpr int kFmtMx = 1;
 
-constexpr int kWarps = 8;                    // compute warps
+constexpr int kTeamWarps = 8;                // compute warps per team (rows per block)
+constexpr int kTeams = 2;                    // teams, taking alternate blocks
+constexpr int kWarps = kTeams * kTeamWarps;  // compute warps
 constexpr int kConsumerThreads = 32 * kWarps;
 constexpr int kThreads = kConsumerThreads + 64;  // + a producer warp and a helper warp
-constexpr int kRowsA = kWarps;      // phase A: one row of gate and of up per warp per block
+constexpr int kRowsA = kTeamWarps;  // phase A: one row of gate and of up per warp per block
 constexpr int kMaxRowsPerWarpB = 4; // phase B: rows of Wd per warp per block
-constexpr int kMaxStages = 4;       // ring depth (fewer when shared memory is short)
-constexpr int kNT = 4;              // pairs per segment (upper bound)
+// Ring depth: 4, or 2 when shared memory is short.  Always even: block j sits in
+// stage j % depth and belongs to team j % 2, so with an even depth every stage is
+// used by one team only, and a team's parity wait on a stage can never be more than
+// one phase ahead of that stage (an odd depth would let one team's wait for a later
+// block pass on the phase of the other team's block still in flight).
+constexpr int kMaxStages = 4;
+constexpr int kNT = 1;              // pairs per compute pass
 constexpr int kMaxPairsFused = 1024;
 constexpr unsigned kBarUnion = 1;   // named barrier: union formed (warp 0 -> producer)
 constexpr unsigned kBarWork = 2;    // named barrier: every warp but the producer
@@ -83,7 +92,7 @@ __host__ __device__ constexpr unsigned act_digit_bytes(int R) { return 2048u * (
 struct LayerGeom {
   int fmt;                 // kFmtAffine or kFmtMx
   int rounds_a, rounds_b;  // 32-column chunks per lane per row (>= H/1024, I/1024; 1, 2, 4, 6, 8)
-  int rows_b;              // phase B rows per block (multiple of kWarps, <= 32)
+  int rows_b;              // phase B rows per block (multiple of kTeamWarps, <= 32)
   unsigned a_q, a_sb, a_mat, a_bytes;  // phase A block: per matrix codes / scale (or bias) bytes
   unsigned b_q, b_sb, b_bytes;         // phase B full block
   unsigned stage_bytes;
@@ -108,9 +117,9 @@ __host__ __device__ inline LayerGeom layer_geom(int H, int I, int fmt = kFmtAffi
   g.fmt = fmt;
   g.rounds_a = chunk_rounds(H);
   g.rounds_b = chunk_rounds(I);
-  int rb = (16 * H / I) / kWarps * kWarps;  // about one phase-A stage worth of Wd rows
-  if (rb < kWarps) rb = kWarps;
-  if (rb > kWarps * kMaxRowsPerWarpB) rb = kWarps * kMaxRowsPerWarpB;
+  int rb = (16 * H / I) / kTeamWarps * kTeamWarps;  // about one phase-A stage of Wd rows
+  if (rb < kTeamWarps) rb = kTeamWarps;
+  if (rb > kTeamWarps * kMaxRowsPerWarpB) rb = kTeamWarps * kMaxRowsPerWarpB;
   g.rows_b = rb;
   g.a_q = kRowsA * H / 2;
   // scales: bf16 per 64 columns (affine) or one e8m0 byte per 32 (mx), H/32 bytes a
@@ -158,17 +167,19 @@ __host__ __device__ inline LayerSmem layer_smem(int E, int P) {
 }
 
 // The shared-memory plan for a window of T tokens, top-k, within `budget` bytes: the
-// deepest normal ring (kMaxStages down to 2) that leaves at least two x rows and eight
-// h rows of activations, the rest of the budget being the activation area; and a wide
+// deepest normal ring (kMaxStages or 2 stages) that leaves at least two x rows and
+// min(T, 8) h rows of activations, the rest of the budget being the activation area; and a wide
 // layout holding all T x rows when that needs more than the normal area (its ring at
-// least 2 stages deep, else none).  False if not even the normal layout fits.
+// least 2 stages deep and even, else none).  False if not even the normal layout fits.
 __host__ __device__ inline bool layer_plan(LayerGeom& g, int E, int T, int k, size_t budget) {
   const int P = T * k;
   g.tables = (unsigned)layer_smem(E, P).end;
   const size_t ra = act_bytes(g.rounds_a), rbb = act_bytes(g.rounds_b);
-  const size_t act_min = align_up(2 * ra > 8 * rbb ? 2 * ra : 8 * rbb, 128);
+  // an expert has at most T pairs in the window, so min(T, 8) h rows hold its set
+  const size_t hmin = (size_t)(T < 8 ? T : 8) * rbb;
+  const size_t act_min = align_up(2 * ra > hmin ? 2 * ra : hmin, 128);
   g.stages = 0;
-  for (int st = kMaxStages; st >= 2; --st) {
+  for (int st = kMaxStages; st >= 2; st -= 2) {
     const size_t used = (size_t)g.tables + (size_t)st * g.stage_bytes;
     if (used + act_min <= budget) {
       g.stages = st;
@@ -183,6 +194,7 @@ __host__ __device__ inline bool layer_plan(LayerGeom& g, int E, int T, int k, si
     const size_t room = budget > (size_t)g.tables + g.act_w ? budget - g.tables - g.act_w : 0;
     int st = (int)(room / g.stage_bytes);
     if (st > kMaxStages) st = kMaxStages;
+    st &= ~1;  // even (see kMaxStages)
     if (st >= 2) g.stages_w = st;
   }
   g.total = (unsigned)budget;
@@ -194,7 +206,7 @@ __host__ __device__ inline bool layer_plan(LayerGeom& g, int E, int T, int k, si
 // [0] CTAs finished, [1, 1+kMaxPairsFused) hdone per distinct expert (phase-A
 // blocks published), then ydone per phase-B row block (at most kMaxRowBlocks),
 // then two words kept zero.
-constexpr int kMaxRowBlocks = 4096 / kWarps;
+constexpr int kMaxRowBlocks = 4096 / kTeamWarps;
 constexpr size_t kSyncWords = 1 + kMaxPairsFused + kMaxRowBlocks + 2;
 
 // -------------------------------------------------------------- arguments ---
@@ -489,7 +501,7 @@ __device__ __forceinline__ void rows_a(const unsigned char* bg_q, const uint16_t
   }
 }
 
-// Phase B: rows row0 + kWarps*q (q < kMaxRowsPerWarpB, rows < nrows) of Wd, NT pairs.
+// Phase B: rows row0 + kTeamWarps*q (q < kMaxRowsPerWarpB, rows < nrows) of Wd, NT pairs.
 // Returns the value this lane holds after a reduce-scatter and its index
 // q*kNT + t in `vid` (-1 when it holds none).
 template <int NT, int R, int F>
@@ -518,7 +530,7 @@ __device__ __forceinline__ float rows_b(const unsigned char* bq, const uint16_t*
       }
 #pragma unroll
       for (int q = 0; q < kMaxRowsPerWarpB; ++q) {
-        const int r = row0 + kWarps * q;
+        const int r = row0 + kTeamWarps * q;
         if (r < nrows) {
           uint32_t qs[8];
           split_codes_f<F>(*reinterpret_cast<const uint4*>(bq + (size_t)r * qstride + ch * 16), qs);
@@ -567,130 +579,6 @@ __device__ __forceinline__ float dispatch_b(int R, const unsigned char* bq, cons
   return rows_b<NT, 8, F>(bq, bs, bb, row0, nrows, I, act, stride, lane, vid);
 }
 
-// Lane holding value v after warp_reduce_scatter<V> (the sum of value v is in every
-// lane whose bits 16, 8, ... down to 32 / V spell v, high bit first).
-template <int V>
-__device__ __forceinline__ constexpr int rs_holder(int v) {
-  int l = 0;
-  for (int w = V, m = 16; w > 1; w >>= 1, m >>= 1)
-    if (v & (w >> 1)) l |= m;
-  return l;
-}
-
-// Two consecutive blocks of one segment at once (at most two pairs).  Phase A takes
-// the warp's row of gate and of up from each block, four rows that share each
-// activation chunk load; phase B the warp's four rows of each block, eight rows.  The
-// rows' sums are independent dp4a chains, so a warp has two blocks' work in flight,
-// and the per-block costs (reduction, publication) are shared.  R is a run-time
-// bound (one loop body for every width).
-//
-// Phase A: rows q/s/b[0..3] = gate and up of block 0, gate and up of block 1.  Lane t
-// (t < NT) returns o[r] = row r's sum for pair t.
-template <int NT, int F>
-__device__ __forceinline__ void rows_a2(const unsigned char* const (&q)[4],
-                                        const uint16_t* const (&s)[4],
-                                        const uint16_t* const (&b)[4], int R, int H,
-                                        const unsigned char* const (&act)[kNT], int lane,
-                                        float (&o)[4]) {
-  constexpr int V = 4 * NT;
-  float acc[V];
-#pragma unroll
-  for (int v = 0; v < V; ++v) acc[v] = 0.f;
-  const int nch = H / 32;
-#pragma unroll 1
-  for (int i = 0; i < R; ++i) {
-    const int ch = i * 32 + lane;
-    if (ch < nch) {
-      uint4 w[4];
-      float2 sb[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        w[r] = *reinterpret_cast<const uint4*>(q[r] + ch * 16);
-        sb[r] = chunk_sb<F>(s[r], b[r], ch);
-      }
-      uint4 xd[NT][4];
-      float2 sc[NT];
-#pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        load_xq(act[t], i, lane, xd[t]);
-        sc[t] = load_sc(act[t], R, ch);
-      }
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        uint32_t qs[8];
-        split_codes_f<F>(w[r], qs);
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          const float d = static_cast<float>(chunk_dot<F>(qs, xd[t]));
-          acc[r * NT + t] = fmaf(sb[r].x * sc[t].x, d, fmaf(sb[r].y, sc[t].y, acc[r * NT + t]));
-        }
-      }
-    }
-  }
-  int vid;
-  const float tot = warp_reduce_scatter<V>(acc, lane, vid);
-#pragma unroll
-  for (int r = 0; r < 4; ++r) o[r] = 0.f;
-#pragma unroll
-  for (int v = 0; v < V; ++v) {
-    const float x = __shfl_sync(kFull, tot, rs_holder<V>(v));
-    if (lane == v % NT) o[v / NT] = x;
-  }
-}
-
-// Phase B: rows warp + kWarps q (q < kMaxRowsPerWarpB) of block 0 (rows < n0) and of
-// block 1 (rows < n1), NT pairs.  Returns the sum this lane holds after the
-// reduce-scatter and its index q' NT + t in `vid` (q' < 4: block 0's row q', else
-// block 1's row q' - 4), -1 when it holds none.
-template <int NT, int F>
-__device__ __forceinline__ float rows_b2(const unsigned char* const (&bq)[2],
-                                         const uint16_t* const (&bs)[2],
-                                         const uint16_t* const (&bb)[2], int n0, int n1,
-                                         int R, int I, const unsigned char* act,
-                                         unsigned stride, int lane, int warp, int& vid) {
-  constexpr int Q = 2 * kMaxRowsPerWarpB;
-  constexpr int V = Q * NT;
-  float acc[V];
-#pragma unroll
-  for (int v = 0; v < V; ++v) acc[v] = 0.f;
-  const int nch = I / 32, qstride = I / 2, sstride = I / 64;
-#pragma unroll 1
-  for (int i = 0; i < R; ++i) {
-    const int ch = i * 32 + lane;
-    if (ch < nch) {
-      uint4 xd[NT][4];
-      float2 sc[NT];
-#pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        const unsigned char* row = act + t * stride;
-        sc[t] = load_sc(row, R, ch);
-        load_xq(row, i, lane, xd[t]);
-      }
-#pragma unroll
-      for (int qq = 0; qq < Q; ++qq) {
-        const int blk = qq / kMaxRowsPerWarpB;
-        const int r = warp + kWarps * (qq % kMaxRowsPerWarpB);
-        if (r < (blk ? n1 : n0)) {
-          uint32_t qs[8];
-          split_codes_f<F>(
-              *reinterpret_cast<const uint4*>(bq[blk] + (size_t)r * qstride + ch * 16), qs);
-          const float2 sb = chunk_sb<F>(bs[blk] + r * sstride, bb[blk] + r * sstride, ch);
-#pragma unroll
-          for (int t = 0; t < NT; ++t) {
-            const float d = static_cast<float>(chunk_dot<F>(qs, xd[t]));
-            acc[qq * NT + t] = fmaf(sb.x * sc[t].x, d, fmaf(sb.y, sc[t].y, acc[qq * NT + t]));
-          }
-        }
-      }
-    }
-  }
-  int v_id;
-  const float v = warp_reduce_scatter<V>(acc, lane, v_id);
-  constexpr int kHolderMask = (32 / V) - 1;
-  vid = (lane & kHolderMask) == 0 ? v_id : -1;
-  return v;
-}
-
 // mbarrier phase test without suspending (for wait loops that do other work).
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, unsigned parity) {
   uint32_t ok;
@@ -714,14 +602,10 @@ __device__ __forceinline__ void fence_proxy_async_all() {
 __device__ __forceinline__ bool lane0(bool v) { return __shfl_sync(kFull, v ? 1 : 0, 0) != 0; }
 __device__ __forceinline__ int lane0_int(int v) { return __shfl_sync(kFull, v, 0); }
 
-// Ring-slot descriptor flags (slot_info[st].x) for the compute warps.
-constexpr int kSlotEnd = 1;       // no more blocks
-constexpr int kSlotPhaseB = 2;    // a phase-B block
-constexpr int kSlotNewSet = 4;    // the first block that reads a new activation set
 constexpr int kPubRing = 16;      // blocks between compute and publication
 
-// Activation set (the rows of one segment's pairs) into `buf`, by the 8 compute warps
-// (256 threads): phase A converts the pairs' token rows of x, phase B the pairs' rows
+// Activation set (the rows of one segment's pairs) into `buf`, by the compute warps
+// (kConsumerThreads threads): phase A converts the pairs' token rows of x, phase B the pairs' rows
 // of h (written by other CTAs; read around L1).  Four consecutive lanes convert one
 // 32-column chunk together.
 template <int F>
@@ -825,63 +709,114 @@ __device__ __forceinline__ int make_segments(const int* offs, int u, int seg, in
   return base;
 }
 
-// Balanced split of one phase's blocks among the CTAs by cost: a block of a segment of
-// nt pairs costs 2 + nt (its weights' bytes are the same for every nt; the per-pair
-// compute is about half the per-block work at one pair), so CTAs whose share has
-// segments of many pairs take fewer blocks.  Returns the first block whose cost
-// prefix reaches t (blocks in segment order, bpe per segment).  Run by one warp.
-__device__ __forceinline__ int block_at_cost(const int* s_nt, int nseg, int bpe, long long t,
-                                             int lane) {
-  if (t <= 0) return 0;
-  long long acc = 0;
+// Inclusive prefix of the segments' costs, pref[s] = sum over segments s' <= s of
+// bpe (2 + nt[s']): a block's weight bytes are the same for every segment, and its
+// compute is about two pairs' worth of fixed work plus one per pair.  Run by one warp.
+__device__ __forceinline__ unsigned prefix_costs(const int* nt, int nseg, int bpe, unsigned* pref,
+                                                 int lane) {
+  unsigned base = 0;
   for (int b0 = 0; b0 < nseg; b0 += 32) {
     const int sidx = b0 + lane;
-    const long long w = sidx < nseg ? (long long)(2 + s_nt[sidx]) : 0;
-    const long long cs = w * bpe;
-    long long incl = cs;
+    const unsigned c = sidx < nseg ? (unsigned)bpe * (2u + (unsigned)nt[sidx]) : 0u;
+    unsigned incl = c;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
-      const long long v = __shfl_up_sync(kFull, incl, d);
+      const unsigned v = __shfl_up_sync(kFull, incl, d);
       if (lane >= d) incl += v;
     }
-    const unsigned hit = __ballot_sync(kFull, sidx < nseg && acc + incl >= t);
-    if (hit) {
-      const int L = __ffs(hit) - 1;
-      const long long excl = __shfl_sync(kFull, incl - cs, L);
-      const long long wl = __shfl_sync(kFull, w, L);
-      const long long k = (t - acc - excl + wl - 1) / wl;
-      return (b0 + L) * bpe + (int)k;
-    }
-    acc += __shfl_sync(kFull, incl, 31);
+    if (sidx < nseg) pref[sidx] = base + incl;
+    base += __shfl_sync(kFull, incl, 31);
   }
-  return nseg * bpe;
+  return base;
 }
 
-// This CTA's share [lo, hi) of one phase's blocks.  Run by one warp.
-__device__ __forceinline__ void cost_share(const int* s_nt, int nseg, int bpe, int lane, int& lo,
-                                           int& hi) {
-  long long tot = 0;
-  for (int sidx = lane; sidx < nseg; sidx += 32) tot += (long long)bpe * (2 + s_nt[sidx]);
-#pragma unroll
-  for (int d = 16; d >= 1; d >>= 1) tot += __shfl_xor_sync(kFull, tot, d);
-  lo = block_at_cost(s_nt, nseg, bpe, tot * blockIdx.x / gridDim.x, lane);
-  hi = block_at_cost(s_nt, nseg, bpe, tot * (blockIdx.x + 1) / gridDim.x, lane);
+// First block (global index, segments in order, bpe blocks each) of segments [s0, s1)
+// at which the cost prefix reaches t: the start of a CTA's share.  One thread.
+__device__ __forceinline__ int block_at(const unsigned* pref, const int* nt, int s0, int s1,
+                                        int bpe, unsigned t) {
+  const unsigned before0 = s0 > 0 ? pref[s0 - 1] : 0u;
+  if (t <= before0) return s0 * bpe;
+  if (s1 <= s0 || t > pref[s1 - 1]) return s1 * bpe;
+  int lo = s0, hi = s1 - 1;  // first s in [lo, hi] with pref[s] >= t
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (pref[mid] >= t) hi = mid;
+    else lo = mid + 1;
+  }
+  const unsigned before = lo > 0 ? pref[lo - 1] : 0u, w = 2u + (unsigned)nt[lo];
+  return lo * bpe + (int)((t - before + w - 1) / w);
 }
 
-// 10 warps: 8 compute warps, a producer warp and a helper warp (see the top of this file).
+// This CTA's block ranges, r0..r7 (lane q returns rq): phase A group 1 [r0, r1) and
+// group 2 [r2, r3), phase B group 1 [r4, r5) and group 2 [r6, r7), each a
+// cost-balanced share (blockIdx of gridDim) of its group's blocks.  Group 1 is the
+// experts up to the one holding the middle of the phase-A cost, group 2 the rest.  A
+// CTA streams its phase-A share of group 1, then of group 2, then its phase-B share
+// of group 1, then of group 2: by the time it reaches group 1's phase B, every CTA
+// has long finished group 1's phase A (nobody waits for h at the turn from A to B),
+// and group 2's phase A finishes while the CTAs stream group 1's phase B.  Run by
+// one warp; prefA / prefB are scratch for nsa / nsb unsigned.
+__device__ __forceinline__ int plan_shares(const int* sa_slot, const int* sa_nt, int nsa,
+                                           int bpe_a, const int* sb_slot, const int* sb_nt,
+                                           int nsb, int bpe_b, unsigned* prefA,
+                                           unsigned* prefB, int lane) {
+  const unsigned totA = prefix_costs(sa_nt, nsa, bpe_a, prefA, lane);
+  const unsigned totB = prefix_costs(sb_nt, nsb, bpe_b, prefB, lane);
+  __syncwarp();
+  // group 1: phase-A segments up to the one holding the middle of the cost, and the
+  // phase-B segments of the same experts
+  int nsa1 = 0;
+  for (int b0 = 0; b0 < nsa; b0 += 32) {
+    const int sidx = b0 + lane;
+    const unsigned hit = __ballot_sync(kFull, sidx < nsa && 2u * prefA[sidx] >= totA);
+    if (hit) {
+      nsa1 = b0 + __ffs(hit);  // one past the middle segment
+      break;
+    }
+  }
+  const int umid = nsa1 > 0 ? sa_slot[nsa1 - 1] + 1 : 0;
+  int nsb1 = nsb;
+  for (int b0 = 0; b0 < nsb; b0 += 32) {
+    const int sidx = b0 + lane;
+    const unsigned hit = __ballot_sync(kFull, sidx < nsb && sb_slot[sidx] >= umid);
+    if (hit) {
+      nsb1 = b0 + __ffs(hit) - 1;
+      break;
+    }
+  }
+  // lane q < 8: target q = phase (q >> 2), group ((q >> 1) & 1), bound (q & 1)
+  int r = 0;
+  if (lane < 8) {
+    const bool pb = lane >= 4;
+    const int g = (lane >> 1) & 1;
+    const unsigned* pref = pb ? prefB : prefA;
+    const int* nt = pb ? sb_nt : sa_nt;
+    const int n1 = pb ? nsb1 : nsa1, n = pb ? nsb : nsa, bpe = pb ? bpe_b : bpe_a;
+    const unsigned tot = pb ? totB : totA;
+    const unsigned c1 = n1 > 0 ? pref[n1 - 1] : 0u;
+    const unsigned base = g ? c1 : 0u, cg = g ? tot - c1 : c1;
+    const unsigned k = blockIdx.x + (unsigned)(lane & 1);
+    const unsigned t = base + cg * k / gridDim.x;
+    r = g ? block_at(pref, nt, n1, n, bpe, t) : block_at(pref, nt, 0, n1, bpe, t);
+  }
+  return r;
+}
+
+// 18 warps: 16 compute warps (two teams), a producer warp and a helper warp (see the top
+// of this file).
 template <int F>
-__global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   // window plan, set by warp 0 after the union: segments of phase A and B, ring depth,
   // resident x rows, the wide layout
-  __shared__ int s_u, s_nsa, s_nsb, s_ns, s_xres, s_wide, s_sega, s_a0, s_a1, s_b0, s_b1;
+  __shared__ int s_u, s_nsa, s_nsb, s_ns, s_xres, s_wide, s_sega;
+  __shared__ int s_rng[8];  // this CTA's block ranges (plan_shares)
   __shared__ unsigned s_act_off, s_act_size;
   __shared__ volatile int s_abort;
   __shared__ volatile int s_pub;  // blocks published by the helper warp
   __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
   __shared__ __align__(8) uint64_t done[kPubRing];           // a block's outputs written
   __shared__ __align__(8) uint64_t set_in[1], set_out[1];    // activation-set hand-over
-  __shared__ int4 slot_info[kMaxStages];  // per ring slot: flags, segment, first row, block
   const LayerGeom& G = a.g;
   const int P = a.T * a.k;
   const LayerSmem L = layer_smem(a.E, P);
@@ -894,9 +829,9 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
   if (threadIdx.x == 0) {
     for (int s = 0; s < kMaxStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kWarps);
+      mbar_init(&empty[s], kTeamWarps);
     }
-    for (int i = 0; i < kPubRing; ++i) mbar_init(&done[i], kWarps);
+    for (int i = 0; i < kPubRing; ++i) mbar_init(&done[i], kTeamWarps);
     mbar_init(&set_in[0], kWarps);
     mbar_init(&set_out[0], kWarps);
     s_abort = 0;
@@ -918,7 +853,8 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
   int* sb_pos = reinterpret_cast<int*>(smem + L.sb_pos);
   int* sb_nt = reinterpret_cast<int*>(smem + L.sb_nt);
   unsigned char* ring = smem + G.tables;
-  const int wt = warp < kWarps ? (int)threadIdx.x : (int)threadIdx.x - 32;  // 0..287 but the producer
+  // every thread but the producer warp's, numbered 0 .. kThreads - 33
+  const int wt = warp < kWarps ? (int)threadIdx.x : (int)threadIdx.x - 32;
   if (warp == 0) {
     int nv;
     const int u = warp_route_union(a.idx, P, a.E, reinterpret_cast<int*>(smem + L.cnt),
@@ -942,9 +878,13 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
     const int nsa = make_segments(offs, u, sega, sa_slot, sa_pos, sa_nt, lane);
     const int nsb = make_segments(offs, u, segb, sb_slot, sb_pos, sb_nt, lane);
     __syncwarp();
-    int ra0, ra1, rb0, rb1;
-    cost_share(sa_nt, nsa, a.I / kRowsA, lane, ra0, ra1);
-    cost_share(sb_nt, nsb, (a.H + G.rows_b - 1) / G.rows_b, lane, rb0, rb1);
+    // (the union's rank scratch and tok_of, filled only after the plan, hold the cost
+    // prefixes)
+    const int rq = plan_shares(sa_slot, sa_nt, nsa, a.I / kRowsA, sb_slot, sb_nt, nsb,
+                               (a.H + G.rows_b - 1) / G.rows_b,
+                               reinterpret_cast<unsigned*>(smem + L.rank),
+                               reinterpret_cast<unsigned*>(tok_of), lane);
+    if (lane < 8) s_rng[lane] = rq;
     if (lane == 0) {
       s_u = u;
       s_nsa = nsa;
@@ -955,15 +895,11 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       s_sega = sega;
       s_act_off = G.tables + (unsigned)ns * G.stage_bytes;
       s_act_size = act_size;
-      s_a0 = ra0;
-      s_a1 = ra1;
-      s_b0 = rb0;
-      s_b1 = rb1;
     }
     __syncwarp();
     named_barrier_arrive(kBarUnion, 64);  // the producer may start (it waits on this)
   } else if (warp != kWarps) {
-    // warps 1..7 and the helper: 256 threads
+    // compute warps 1.. and the helper: kThreads - 64 threads
     for (int p = wt - 32; p < P; p += kThreads - 64) pos_of[p] = -1;
     // a window whose x rows fit the normal activation area: converted while warp 0
     // forms the union
@@ -996,23 +932,27 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
     if (lane == 0) *a.ex_u = u;
   }
 
-  // ---- this CTA's blocks: a contiguous share of the phase-A blocks (kRowsA rows of
-  // gate and of up each, per phase-A segment), then of the phase-B blocks (rows_b rows
-  // of down each, per phase-B segment), both in segment order, balanced by cost
-  // (cost_share).  Every block is 2 kRowsA H/2 + scales (A) or rows_b I/2 + scales (B)
-  // bytes; the two are equal at the 4096/2048 shape ----
+  // ---- this CTA's blocks: phase-A blocks (kRowsA rows of gate and of up each, per
+  // phase-A segment), then phase-B blocks (rows_b rows of down each, per phase-B
+  // segment), each phase in two groups of experts, each group's share contiguous in
+  // segment order and balanced by cost (plan_shares).  Every block is 2 kRowsA H/2 +
+  // scales (A) or rows_b I/2 + scales (B) bytes; the two are equal at the 4096/2048
+  // shape ----
   const int bpe_a = a.I / kRowsA;                     // phase-A blocks per segment
   const int bpe_b = (a.H + G.rows_b - 1) / G.rows_b;  // phase-B blocks per segment
-  const int a0 = s_a0, a1 = s_a1, b0 = s_b0, b1 = s_b1;  // cost-balanced shares (cost_share)
-  const int nA = a1 - a0, nblk = nA + (b1 - b0);
+  // the CTA's ranges (plan_shares): phase A group 1, group 2, phase B group 1, group 2
+  const int a0 = s_rng[0], a2 = s_rng[2], b0 = s_rng[4], b2 = s_rng[6];
+  const int nA1 = s_rng[1] - a0, nA = nA1 + (s_rng[3] - a2);
+  const int nB1 = s_rng[5] - b0, nblk = nA + nB1 + (s_rng[7] - b2);
   auto block_of = [&](int j, bool& pb, int& sg, int& row0) {
     if (j < nA) {
-      const int blk = a0 + j;
+      const int blk = j < nA1 ? a0 + j : a2 + (j - nA1);
       pb = false;
       sg = blk / bpe_a;
       row0 = (blk % bpe_a) * kRowsA;
     } else {
-      const int blk = b0 + (j - nA);
+      const int jb = j - nA;
+      const int blk = jb < nB1 ? b0 + jb : b2 + (jb - nB1);
       pb = true;
       sg = blk / bpe_b;
       row0 = (blk % bpe_b) * G.rows_b;
@@ -1087,9 +1027,8 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       return false;
     };
     bool ok = true;
-    int prev_set = -1;  // activation set of the previous block (-1: resident x)
     int j = 0;
-    for (; j <= nblk && ok; ++j) {
+    for (; j < nblk && ok; ++j) {
       const int st = j % NS;
       if (j >= NS) {  // the compute warps are done with block j - NS
         const unsigned long long t0 = globaltimer();
@@ -1108,23 +1047,10 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
         }
       }
       if (!ok) break;
-      if (j == nblk) {
-        if (lane == 0) {
-          slot_info[st] = make_int4(kSlotEnd, 0, 0, j);
-          mbar_arrive(&full[st]);
-        }
-        __syncwarp();
-        break;
-      }
       bool pb;
       int sg, row0;
       block_of(j, pb, sg, row0);
-      const int set = pb ? nsa + sg : (x_res ? -1 : sg);
-      const bool new_set = set >= 0 && set != prev_set;
-      prev_set = set;
       if (lane == 0) {
-        slot_info[st] =
-            make_int4((pb ? kSlotPhaseB : 0) | (new_set ? kSlotNewSet : 0), sg, row0, j);
         unsigned char* buf = ring + (size_t)st * G.stage_bytes;
         fence_proxy_async();
         if (!pb) {
@@ -1163,6 +1089,11 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
     __syncwarp();
   } else {
     // ================================ compute warps ================================
+    // Two teams of kTeamWarps warps: team tm takes blocks tm, tm + kTeams, ... of this
+    // CTA's sequence, warp w of a team row w of each of its blocks (phase A) or rows
+    // w, w + kTeamWarps, ... (phase B).  While one team computes a block the other
+    // computes the next, so each scheduler has twice the warps to hide latency with.
+    const int tm = warp / kTeamWarps, w = warp % kTeamWarps;
     auto wait_cons = [&](uint64_t* bar, unsigned parity) -> bool {
       if (s_abort) return false;
       const unsigned long long t0 = globaltimer();
@@ -1177,26 +1108,35 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
       return true;
     };
     const int sega = s_sega;
-    int nsets = 0;  // activation sets converted
-    for (int j = 0;; ++j) {
-      const int st = j % NS;
-      if (!wait_cons(&full[st], (j / NS) & 1)) break;
-      const int4 si = slot_info[st];
-      if (si.x & kSlotEnd) break;
-      const bool phase_b = (si.x & kSlotPhaseB) != 0;
-      const int sg = si.y, row0 = si.z;
-      const int nt = phase_b ? sb_nt[sg] : sa_nt[sg];
-      const int p0 = phase_b ? sb_pos[sg] : sa_pos[sg];
-      if (si.x & kSlotNewSet) {
-        // All compute warps are past the previous set's blocks, so the activation area
-        // is free; phase B waits (bounded) until every phase-A block of the expert has
-        // published its h rows.
-        // For phase B one thread (warp 0's lane 0) waits, with a short back-off, until
-        // hdone[expert] counts every phase-A block of the expert; its acquire reaches
-        // the other warps through set_in (release/acquire at CTA scope), so one poller
-        // per CTA loads the counter.
+    // activation set of block b: the phase-B segment (nsa + sg), the phase-A segment when
+    // x is not resident, else none (-1); a set starts where it differs from block b-1's
+    auto set_of = [&](int b) -> int {
+      if (b < 0) return -1;
+      bool pb;
+      int sg, r0;
+      block_of(b, pb, sg, r0);
+      return pb ? nsa + sg : (x_res ? -1 : sg);
+    };
+    int nsets = 0;    // activation sets converted
+    int handled = -1; // blocks up to here have had their set starts taken
+    // Every compute warp (both teams) takes every set start, in block order, before it
+    // computes a block at or after it: all warps meet at set_in (so every block of the
+    // previous set is done and the activation area is free), phase B waits (one
+    // thread, bounded) until every phase-A block of the expert has published its h
+    // rows, the compute threads convert the set, and all meet again at set_out.
+    auto take_sets = [&](int upto) -> bool {
+      for (int b = handled + 1; b <= upto; ++b) {
+        const int sb = set_of(b);
+        if (sb < 0 || sb == set_of(b - 1)) continue;
+        bool pb;
+        int sg, r0;
+        block_of(b, pb, sg, r0);
+        const int nt = pb ? sb_nt[sg] : sa_nt[sg];
+        const int p0 = pb ? sb_pos[sg] : sa_pos[sg];
+        // the poller's acquire reaches the other warps through set_in (release/acquire
+        // at CTA scope), so one thread per CTA loads the counter
         __syncwarp();
-        if (phase_b && warp == 0 && lane == 0) {
+        if (pb && warp == 0 && lane == 0) {
           const int slot = sb_slot[sg];
           const int n_i = offs[slot + 1] - offs[slot];
           const unsigned target = (unsigned)bpe_a * (unsigned)((n_i + sega - 1) / sega);
@@ -1211,144 +1151,64 @@ __global__ void __maxnreg__(168) layer_kernel(const LayerArgs a) {
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&set_in[0]);
-        if (!wait_cons(&set_in[0], nsets & 1)) break;
-        convert_set<F>(a, G, phase_b, tok_of, p0, nt, actp, lane);
+        if (!wait_cons(&set_in[0], nsets & 1)) return false;
+        convert_set<F>(a, G, pb, tok_of, p0, nt, actp, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(&set_out[0]);
-        if (!wait_cons(&set_out[0], nsets & 1)) break;
+        if (!wait_cons(&set_out[0], nsets & 1)) return false;
         ++nsets;
       }
+      handled = upto;
+      return true;
+    };
+    for (int j = tm;; j += kTeams) {
+      if (j >= nblk) {
+        take_sets(nblk - 1);  // the set starts past this team's last block
+        break;
+      }
+      if (!take_sets(j)) break;
+      const int st = j % NS;
+      if (!wait_cons(&full[st], (j / NS) & 1)) break;
+      bool phase_b;
+      int sg, row0;
+      block_of(j, phase_b, sg, row0);
+      const int nt = phase_b ? sb_nt[sg] : sa_nt[sg];
+      const int p0 = phase_b ? sb_pos[sg] : sa_pos[sg];
       const unsigned char* buf = ring + (size_t)st * G.stage_bytes;
-      // Block j + 1 of the same segment (next rows, at most two pairs) is taken with
-      // block j (rows_a2 / rows_b2); the schedule is a pure function of j, so every
-      // compute warp makes the same choice.
-      bool paired = false;
-      if (nt <= 2 && j + 1 < nblk) {
-        bool pb1;
-        int sg1, r1;
-        block_of(j + 1, pb1, sg1, r1);
-        paired = pb1 == phase_b && sg1 == sg && r1 == row0 + (phase_b ? G.rows_b : kRowsA);
-      }
-      if (paired) {
-        const int st1 = (j + 1) % NS;
-        if (!wait_cons(&full[st1], ((j + 1) / NS) & 1)) break;
-        const unsigned char* buf1 = ring + (size_t)st1 * G.stage_bytes;
-        if (!phase_b) {
-          const unsigned char* q4[4];
-          const uint16_t* s4[4];
-          const uint16_t* b4[4];
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const unsigned char* m = (r < 2 ? buf : buf1) + ((r & 1) ? G.a_mat : 0);
-            q4[r] = m + (size_t)warp * (a.H / 2);
-            s4[r] = reinterpret_cast<const uint16_t*>(m + G.a_q) + warp * (a.H / 64);
-            b4[r] = reinterpret_cast<const uint16_t*>(m + G.a_q + G.a_sb) + warp * (a.H / 64);
-          }
-          const unsigned char* arow[kNT];
-#pragma unroll
-          for (int t = 0; t < kNT; ++t)
-            arow[t] = x_res ? actp + (t < nt ? tok_of[p0 + t] : 0) * stride_a
-                            : actp + t * stride_a;
-          float o[4];
-          if (nt == 1) rows_a2<1, F>(q4, s4, b4, G.rounds_a, a.H, arow, lane, o);
-          else rows_a2<2, F>(q4, s4, b4, G.rounds_a, a.H, arow, lane, o);
-          if (lane < nt) {
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const float g = round_to_bf16(o[2 * h2]), hu = round_to_bf16(o[2 * h2 + 1]);
-              a.h[(size_t)(p0 + lane) * a.I + row0 + kRowsA * h2 + warp] =
-                  float_to_bf16_bits(__fdividef(g, 1.0f + __expf(-g)) * hu);
-            }
-          }
-        } else {
-          const int n0 = min(G.rows_b, a.H - row0);
-          const int n1 = min(G.rows_b, a.H - row0 - G.rows_b);
-          const unsigned char* bq2[2] = {buf, buf1};
-          const uint16_t* bs2[2] = {reinterpret_cast<const uint16_t*>(buf + G.b_q),
-                                    reinterpret_cast<const uint16_t*>(buf1 + G.b_q)};
-          const uint16_t* bb2[2] = {reinterpret_cast<const uint16_t*>(buf + G.b_q + G.b_sb),
-                                    reinterpret_cast<const uint16_t*>(buf1 + G.b_q + G.b_sb)};
-          int vid;
-          const float v =
-              nt == 1 ? rows_b2<1, F>(bq2, bs2, bb2, n0, n1, G.rounds_b, a.I, actp, stride_b,
-                                      lane, warp, vid)
-                      : rows_b2<2, F>(bq2, bs2, bb2, n0, n1, G.rounds_b, a.I, actp, stride_b,
-                                      lane, warp, vid);
-          if (vid >= 0) {
-            const int qq = vid / nt, t = vid % nt;
-            const int blk = qq / kMaxRowsPerWarpB;
-            const int r = warp + kWarps * (qq % kMaxRowsPerWarpB);
-            if (r < (blk ? n1 : n0))
-              a.y[(size_t)(p0 + t) * a.H + row0 + blk * G.rows_b + r] = v;
-          }
-        }
-        // done reading stages st and st1; both blocks' outputs written
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&empty[st]);
-          mbar_arrive(&done[j % kPubRing]);
-          mbar_arrive(&empty[st1]);
-          mbar_arrive(&done[(j + 1) % kPubRing]);
-        }
-        ++j;
-        continue;
-      }
-      // the set's pairs in chunks of kNT, the block's weights read again per chunk
-      int nrows = 0;
-      for (int c0 = 0; c0 < nt; c0 += kNT) {
-        const int ntc = min(kNT, nt - c0);
-        float Gs[kNT], Us[kNT];
-        float v = 0.f;
-        int vid = -1;
-        if (!phase_b) {
-          const unsigned char* bgq = buf + (size_t)warp * (a.H / 2);
-          const uint16_t* bgs = reinterpret_cast<const uint16_t*>(buf + G.a_q) + warp * (a.H / 64);
-          const uint16_t* bgb = reinterpret_cast<const uint16_t*>(buf + G.a_q + G.a_sb) + warp * (a.H / 64);
-          const unsigned char* bu = buf + G.a_mat;
-          const unsigned char* buq = bu + (size_t)warp * (a.H / 2);
-          const uint16_t* bus = reinterpret_cast<const uint16_t*>(bu + G.a_q) + warp * (a.H / 64);
-          const uint16_t* bub = reinterpret_cast<const uint16_t*>(bu + G.a_q + G.a_sb) + warp * (a.H / 64);
-          // the activation row of each pair: the token's resident x row, or row c0 + t
-          // of the current set
-          const unsigned char* arow[kNT];
-#pragma unroll
-          for (int t = 0; t < kNT; ++t)
-            arow[t] = x_res ? actp + (t < ntc ? tok_of[p0 + c0 + t] : 0) * stride_a
-                            : actp + (c0 + t) * stride_a;
-          switch (ntc) {
-            case 1: dispatch_a<1, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us); break;
-            case 2: dispatch_a<2, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us); break;
-            case 3: dispatch_a<3, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us); break;
-            default: dispatch_a<4, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us); break;
-          }
-          if (lane < ntc) {
-            float gv = 0.f, uv = 0.f;
-#pragma unroll
-            for (int t = 0; t < kNT; ++t)
-              if (t == lane) {
-                gv = Gs[t];
-                uv = Us[t];
-              }
-            const float g = round_to_bf16(gv), hu = round_to_bf16(uv);
+      // the segment's pairs one at a time, the block's weights read again per pair
+      if (!phase_b) {
+        const unsigned char* bgq = buf + (size_t)w * (a.H / 2);
+        const uint16_t* bgs = reinterpret_cast<const uint16_t*>(buf + G.a_q) + w * (a.H / 64);
+        const uint16_t* bgb = reinterpret_cast<const uint16_t*>(buf + G.a_q + G.a_sb) + w * (a.H / 64);
+        const unsigned char* bu = buf + G.a_mat;
+        const unsigned char* buq = bu + (size_t)w * (a.H / 2);
+        const uint16_t* bus = reinterpret_cast<const uint16_t*>(bu + G.a_q) + w * (a.H / 64);
+        const uint16_t* bub = reinterpret_cast<const uint16_t*>(bu + G.a_q + G.a_sb) + w * (a.H / 64);
+        for (int c = 0; c < nt; ++c) {
+          // the pair's activation row: the token's resident x row, or row c of the set
+          const unsigned char* const arow[kNT] = {x_res ? actp + tok_of[p0 + c] * stride_a
+                                                        : actp + c * stride_a};
+          float Gs[kNT], Us[kNT];
+          dispatch_a<1, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
+          if (lane == 0) {
+            const float g = round_to_bf16(Gs[0]), hu = round_to_bf16(Us[0]);
             // silu(g) = g / (1 + e^-g); the fast division's error (2 ulp of fp32) is far
             // below the bf16 step h is rounded to
-            a.h[(size_t)(p0 + c0 + lane) * a.I + row0 + warp] =
+            a.h[(size_t)(p0 + c) * a.I + row0 + w] =
                 float_to_bf16_bits(__fdividef(g, 1.0f + __expf(-g)) * hu);
           }
-        } else {
-          nrows = min(G.rows_b, a.H - row0);
-          const uint16_t* bs = reinterpret_cast<const uint16_t*>(buf + G.b_q);
-          const uint16_t* bb = reinterpret_cast<const uint16_t*>(buf + G.b_q + G.b_sb);
-          const unsigned char* act = actp + (size_t)c0 * stride_b;
-          switch (ntc) {
-            case 1: v = dispatch_b<1, F>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
-            case 2: v = dispatch_b<2, F>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
-            case 3: v = dispatch_b<3, F>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
-            default: v = dispatch_b<4, F>(G.rounds_b, buf, bs, bb, warp, nrows, a.I, act, stride_b, lane, vid); break;
-          }
+        }
+      } else {
+        const int nrows = min(G.rows_b, a.H - row0);
+        const uint16_t* bs = reinterpret_cast<const uint16_t*>(buf + G.b_q);
+        const uint16_t* bb = reinterpret_cast<const uint16_t*>(buf + G.b_q + G.b_sb);
+        for (int c = 0; c < nt; ++c) {
+          int vid;
+          const float v = dispatch_b<1, F>(G.rounds_b, buf, bs, bb, w, nrows, a.I,
+                                           actp + (size_t)c * stride_b, stride_b, lane, vid);
           if (vid >= 0) {
-            const int r = warp + kWarps * (vid / kNT), t = vid % kNT;
-            if (r < nrows) a.y[(size_t)(p0 + c0 + t) * a.H + row0 + r] = v;
+            const int r = w + kTeamWarps * vid;
+            if (r < nrows) a.y[(size_t)(p0 + c) * a.H + row0 + r] = v;
           }
         }
       }
