@@ -809,7 +809,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   // window plan, set by warp 0 after the union: segments of phase A and B, ring depth,
   // resident x rows, the wide layout
-  __shared__ int s_u, s_nsa, s_nsb, s_ns, s_xres, s_wide, s_sega;
+  __shared__ int s_u, s_nsb, s_ns, s_xres, s_wide, s_sega;
   __shared__ int s_rng[8];  // this CTA's block ranges (plan_shares)
   __shared__ unsigned s_act_off, s_act_size;
   __shared__ volatile int s_abort;
@@ -887,7 +887,6 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
     if (lane < 8) s_rng[lane] = rq;
     if (lane == 0) {
       s_u = u;
-      s_nsa = nsa;
       s_nsb = nsb;
       s_ns = ns;
       s_xres = xr ? 1 : 0;
@@ -912,7 +911,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
   } else {
     named_barrier(kBarUnion, 64);  // the plan is made
   }
-  const int u = s_u, nsa = s_nsa, nsb = s_nsb, NS = s_ns;
+  const int u = s_u, nsb = s_nsb, NS = s_ns;
   const bool x_res = s_xres != 0;
   unsigned char* actp = smem + s_act_off;  // activation area (resident x rows first)
   const int n_valid = offs[u];
@@ -944,19 +943,31 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
   const int a0 = s_rng[0], a2 = s_rng[2], b0 = s_rng[4], b2 = s_rng[6];
   const int nA1 = s_rng[1] - a0, nA = nA1 + (s_rng[3] - a2);
   const int nB1 = s_rng[5] - b0, nblk = nA + nB1 + (s_rng[7] - b2);
+  // blk / bpe as a multiply-high: m = ceil(2^40 / bpe) is exact for blk * bpe < 2^40
+  const unsigned long long mag_a = ((1ull << 40) + bpe_a - 1) / bpe_a;
+  const unsigned long long mag_b = ((1ull << 40) + bpe_b - 1) / bpe_b;
   auto block_of = [&](int j, bool& pb, int& sg, int& row0) {
     if (j < nA) {
       const int blk = j < nA1 ? a0 + j : a2 + (j - nA1);
       pb = false;
-      sg = blk / bpe_a;
-      row0 = (blk % bpe_a) * kRowsA;
+      sg = (int)(((unsigned long long)blk * mag_a) >> 40);
+      row0 = (blk - sg * bpe_a) * kRowsA;
     } else {
       const int jb = j - nA;
       const int blk = jb < nB1 ? b0 + jb : b2 + (jb - nB1);
       pb = true;
-      sg = blk / bpe_b;
-      row0 = (blk % bpe_b) * G.rows_b;
+      sg = (int)(((unsigned long long)blk * mag_b) >> 40);
+      row0 = (blk - sg * bpe_b) * G.rows_b;
     }
+  };
+  // block j starts an activation set: the first block of a segment (or of one of the
+  // four ranges) in phase B, and in phase A when x is not resident
+  auto set_start = [&](int j) -> bool {
+    bool pb;
+    int sg, r0;
+    block_of(j, pb, sg, r0);
+    if (!pb && x_res) return false;
+    return r0 == 0 || j == 0 || j == nA1 || j == nA || j == nA + nB1;
   };
 
   if (warp == kWarps + 1) {
@@ -1108,15 +1119,6 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
       return true;
     };
     const int sega = s_sega;
-    // activation set of block b: the phase-B segment (nsa + sg), the phase-A segment when
-    // x is not resident, else none (-1); a set starts where it differs from block b-1's
-    auto set_of = [&](int b) -> int {
-      if (b < 0) return -1;
-      bool pb;
-      int sg, r0;
-      block_of(b, pb, sg, r0);
-      return pb ? nsa + sg : (x_res ? -1 : sg);
-    };
     int nsets = 0;    // activation sets converted
     int handled = -1; // blocks up to here have had their set starts taken
     // Every compute warp (both teams) takes every set start, in block order, before it
@@ -1126,8 +1128,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
     // rows, the compute threads convert the set, and all meet again at set_out.
     auto take_sets = [&](int upto) -> bool {
       for (int b = handled + 1; b <= upto; ++b) {
-        const int sb = set_of(b);
-        if (sb < 0 || sb == set_of(b - 1)) continue;
+        if (!set_start(b)) continue;
         bool pb;
         int sg, r0;
         block_of(b, pb, sg, r0);
