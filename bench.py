@@ -280,6 +280,9 @@ def routings():
         if ROUTING == "markov":
             out[T] = [synth.route_markov(T, E, K_TOP, 0.40, SEED + 100 * T + l)
                       for l in range(LAYERS)]
+        elif ROUTING == "identical":  # every token on experts 8l .. 8l+7 (mod E)
+            out[T] = [(np.tile((np.arange(K_TOP) + K_TOP * l) % E, (T, 1)).astype(np.int32),
+                       np.full((T, K_TOP), 1.0 / K_TOP, np.float32)) for l in range(LAYERS)]
         else:
             out[T] = [synth.route_uniform(T, E, K_TOP, SEED + 100 * T + l) for l in range(LAYERS)]
     return out
@@ -405,6 +408,44 @@ def reference_arm(args, world, rank):
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def large_window_only(args, local):
+    """Profiling run of the grouped path alone: one T-token layer (T from --ts, default
+    512) on an E=256 bank (3.6 GB), 3 warm calls then 1 timed; for ncu captures of the
+    grouped kernels on a small device footprint."""
+    import torch
+    import quantized_expert_gather_b200 as qeg
+    import synth
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    EL = 256
+    TL = int(args.ts) if args.ts else 512
+
+    def mat(rows, cols, mid):
+        q = torch.empty((EL, rows, cols // 8), dtype=torch.int32, device=dev)
+        s = torch.empty((EL, rows, cols // 64), dtype=torch.int16, device=dev)
+        b = torch.empty_like(s)
+        synth.fill_bank_device(q, s, b, rows, cols, SEED, mid)
+        return q, s.view(torch.bfloat16), b.view(torch.bfloat16)
+    bank = qeg.QuantBank(*mat(INTER, HIDDEN, 0), *mat(INTER, HIDDEN, 1), *mat(HIDDEN, INTER, 2))
+    r = synth.route_uniform(TL, EL, K_TOP, SEED + 900 + TL)
+    x = torch.from_numpy(synth.x_bf16(TL, HIDDEN, SEED + TL).view(np.int16)).to(dev) \
+        .view(torch.bfloat16)
+    il, wl = torch.from_numpy(r[0]).to(dev), torch.from_numpy(r[1]).to(dev)
+    out = torch.empty((TL, HIDDEN), dtype=torch.bfloat16, device=dev)
+    ws = torch.zeros(qeg.moe_workspace_size(TL, K_TOP, EL, HIDDEN, INTER), dtype=torch.uint8,
+                     device=dev)
+    for _ in range(3):
+        qeg.moe_switchglu_forward_ws(x, il, wl, bank, ws, out=out)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    qeg.moe_switchglu_forward_ws(x, il, wl, bank, ws, out=out)
+    b.record()
+    torch.cuda.synchronize()
+    return {"large_window_only": True, "T": TL, "us_per_layer": a.elapsed_time(b) * 1e3,
+            "status": qeg.moe_read_device_status()}
 
 
 def our_arm(args, world, rank, local):
@@ -855,7 +896,9 @@ def main():
     ap.add_argument("--no-window-sweep", action="store_true",
                     help="skip the verify-window sweep (T=2..16, 78-layer stacks)")
     ap.add_argument("--ts", default="", help="comma-separated window sizes (profiling)")
-    ap.add_argument("--routing", default="uniform", choices=("uniform", "markov"),
+    ap.add_argument("--large-window-only", action="store_true",
+                    help="one grouped-path layer alone (T from --ts, default 512; profiling)")
+    ap.add_argument("--routing", default="uniform", choices=("uniform", "markov", "identical"),
                     help="routing model (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -864,7 +907,8 @@ def main():
     try:
         if args.impl == "reference":
             return reference_arm(args, world, rank)
-        res = our_arm(args, world, rank, local)
+        res = large_window_only(args, local) if args.large_window_only else \
+            our_arm(args, world, rank, local)
         if rank == 0 and res is not None:
             print(json.dumps(res), flush=True)
     finally:

@@ -231,7 +231,7 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   const int width = P > 40 * m ? 96 : (P <= 20 * m ? 32 : 64);
   const unsigned gsmem = width == 96 ? GCfg<96>::kSmem : width == 32 ? GCfg<32>::kSmem : GCfg<64>::kSmem;
   const int ki = width == 96 ? 5 : width == 32 ? 7 : 2;  // dyn_smem index of gate+up
-  const int grid = d.sms;  // one CTA per SM (all of tensor memory, most of shared memory)
+  const int grid = width == 32 ? 2 * d.sms : d.sms;
   if (usmem > (size_t)d.dyn_smem[1] || csmem > (size_t)d.dyn_smem[4] ||
       gsmem > (unsigned)d.dyn_smem[ki] || gsmem > (unsigned)d.dyn_smem[ki + 1]) {
     *why = MOE_ERR_UNSUPPORTED;

@@ -28,24 +28,18 @@
 // the activation row's group sum) is added to fp32 registers.  No weight is ever
 // rounded; the only per-weight work is turning 4-bit codes into bf16 integers.
 //
-// Roles in a CTA (one CTA per SM, looping over tiles):
-//   warp 12     producer: per stage of two slabs, 16-byte async copies of each
+// Roles in a CTA (one or two CTAs per SM, looping over tiles):
+//   warp 8      producer: per stage of two slabs, 16-byte async copies of each
 //               weight row's codes (64 bytes) and 4-byte ones of its scales and
 //               biases, and 1-D bulk copies of the two packed activation slabs and
 //               of their group sums;
-//   warp 13     MMA issuer: issues tcgen05.mma (one elected lane of the converged
+//   warp 9      MMA issuer: issues tcgen05.mma (one elected lane of the converged
 //               warp) with A (the codes as bf16) in tensor memory and B (the
-//               activations) in shared memory, each slab into its own accumulator
-//               buffer (two to four of them);
-//   warps 0..3  expanders: one tensor-memory lane each (row r of both matrices of
-//               the tile); per slab they expand the rows' codes to bf16 into an A
-//               buffer (two to four), ahead of the MMAs;
-//   warps 4..11 read-back: warps 4 + 4m .. 4 + 4m + 3 own matrix m, one weight row
-//               per thread; per slab they read the slab's product back and add
-//               s * P + b * X in fp32 registers, behind the MMAs; at a chunk's end
-//               they finish h (gate+up) or y (down).
-// The three roles meet only at buffer barriers, so expansion, the MMAs and the read-
-// back of different slabs overlap.
+//               activations) in shared memory;
+//   warps 0..7  warps 4m..4m+3 own matrix m of the tile, one weight row per
+//               thread (the row's tensor-memory lane).  Per slab they expand the
+//               row's codes to bf16 into tensor memory (the MMA's A operand), then
+//               read back the previous slab's product and accumulate it.
 // Codes expand without conversions: nibble q placed under the bf16 exponent of
 // 128 reads as 128 + q, and one packed bf16 FMA takes the 128 off exactly.  That
 // puts codes j and j + 4 of a 32-bit code word in one bf16 pair, so K runs in
@@ -64,46 +58,40 @@
 
 namespace qeg {
 
-constexpr int kGExp = 4;                             // expander warps
-constexpr int kGRead = 8;                            // read-back warps
-constexpr int kGProducer = kGExp + kGRead;           // warp 12
-constexpr int kGMmaWarp = kGProducer + 1;            // warp 13
-constexpr int kGThreads = 32 * (kGMmaWarp + 1);      // 448
+constexpr int kGWorkers = 8;                         // worker warps
+constexpr int kGThreads = 32 * (kGWorkers + 2);      // + producer warp + MMA warp
 constexpr int kGM = 128;                             // weight rows per matrix (MMA M)
 constexpr int kGK = 64;                              // K per slab = quantisation group
 constexpr int kGSlabsPerStage = 2;
 constexpr unsigned kGCodePitch = kGSlabsPerStage * 32 + 16;  // padded: no bank conflicts
 constexpr unsigned kGOffB = 2 * kGM * kGCodePitch;           // 20480, a multiple of 1024
-constexpr unsigned kGXchg = 2 * kGM * 16 * 4;                // h exchange: 16 pairs a round
-constexpr unsigned kGSmemBudget = 230400;                    // dynamic shared memory planned for
+constexpr int kGDBufs = 2;   // accumulator buffers
+constexpr int kGLag = 1;     // a slab's accumulator is read back after the next slab's A is stored
+constexpr int kGABufs = 2;   // A operand buffers
 
 // Per chunk width NMAX (pairs per MMA, a multiple of 32): the shared-memory stage
-// [codes | two activation slabs | their sums | scales | biases], the ring depth, and
-// the tensor-memory map: kND accumulator buffers of both matrices' NMAX columns,
-// then kNA A buffers of both matrices' 32 columns (64 bf16 codes), 512 columns.
+// [codes | two activation slabs | their sums | scales | biases] and the tensor
+// memory map (accumulator of buffer db, matrix m; then the A operand of buffer ab).
 template <int NMAX>
 struct GCfg {
   static constexpr int kN = NMAX;
-  static constexpr int kND = NMAX <= 32 ? 4 : (NMAX <= 64 ? 3 : 2);
-  static constexpr int kNA = (512 - kND * 2 * NMAX) / 64 > 4 ? 4 : (512 - kND * 2 * NMAX) / 64;
-  static constexpr uint32_t kTmemCols = 512;
+  static constexpr int kStages = NMAX <= 32 ? 3 : (NMAX <= 64 ? 5 : 4);
+  static constexpr int kCtasPerSm = NMAX <= 32 ? 2 : 1;  // two CTAs share an SM's tensor memory
+  static constexpr uint32_t kTmemCols = NMAX <= 32 ? 256 : 512;
   static constexpr unsigned kBTile = NMAX * kGK * 2;
   static constexpr unsigned kOffX = kGOffB + kGSlabsPerStage * kBTile;
   static constexpr unsigned kOffS = kOffX + kGSlabsPerStage * NMAX * 4;
   static constexpr unsigned kOffBias = kOffS + 2 * kGM * kGSlabsPerStage * 2;
   static constexpr unsigned kStageBytes =
       (kOffBias + 2 * kGM * kGSlabsPerStage * 2 + 1023) & ~1023u;
-  static constexpr unsigned kRing = kGSmemBudget - 1024 - kGXchg;
-  static constexpr int kStages = (int)(kRing / kStageBytes) > 6 ? 6 : (int)(kRing / kStageBytes);
-  static constexpr unsigned kSmem = kStages * kStageBytes + kGXchg + 1024;  // + alignment slack
+  static constexpr unsigned kSmem = kStages * kStageBytes + 1024;  // + alignment slack
   static_assert(NMAX % 32 == 0 && kBTile % 1024 == 0, "swizzled tiles need 1024-byte bases");
-  static_assert(kNA >= 2 && kND * 2 * NMAX + kNA * 64 <= 512, "tensor memory map");
-  static_assert(kStages >= 3, "copy ring depth");
+  static_assert(kGDBufs * 2 * NMAX + kGABufs * 2 * 32 <= (int)kTmemCols, "tensor memory map");
   __device__ static __forceinline__ uint32_t col_d(uint32_t db, int m) {
     return (db * 2 + m) * NMAX;
   }
   __device__ static __forceinline__ uint32_t col_a(uint32_t ab, int m) {
-    return kND * 2 * NMAX + (ab * 2 + m) * 32;
+    return kGDBufs * 2 * NMAX + (ab * 2 + m) * 32;
   }
 };
 
@@ -316,46 +304,31 @@ struct GroupedArgs {
 };
 
 template <int PHASE, int NMAX>
-__global__ void __launch_bounds__(kGThreads, 1)
+__global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
     grouped_gemm_kernel(const __grid_constant__ GroupedArgs a) {
   using C = GCfg<NMAX>;
   extern __shared__ __align__(128) unsigned char gsm_raw[];
   __shared__ __align__(8) uint64_t full[C::kStages], empty[C::kStages];
-  __shared__ __align__(8) uint64_t a_full[C::kNA], a_free[C::kNA];
-  __shared__ __align__(8) uint64_t d_full[C::kND], d_free[C::kND];
-  // epilogue hand-overs between read-back warps (bounded waits, two arrivals each): the
-  // h exchange of a lane quarter's two warps, and the group-sum exchange of the two
-  // warps of one matrix that cover a 64-row group
-  __shared__ __align__(8) uint64_t xa[4], xb[4], ra[2][2], rb[2][2];
+  __shared__ __align__(8) uint64_t a_full[kGABufs], d_full[kGDBufs], d_free[kGDBufs];
   __shared__ uint32_t tmem_base_s;
   __shared__ float red[2][2][C::kN / 2];
   // swizzled tiles start at 1024-byte boundaries of the shared address space
   unsigned char* gsm = gsm_raw + ((1024u - (smem_u32(gsm_raw) & 1023u)) & 1023u);
-  float* xchg = reinterpret_cast<float*>(gsm + C::kStages * C::kStageBytes);  // [2][128][16]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
     for (int i = 0; i < C::kStages; ++i) {
-      mbar_init(&full[i], 1 + 32);                 // expect_tx + one cp.async arrival per lane
-      mbar_init(&empty[i], kGExp + kGRead + 1);    // expanders, read-back warps, MMA commit
+      mbar_init(&full[i], 1 + 32);          // expect_tx + one cp.async arrival per lane
+      mbar_init(&empty[i], kGWorkers + 1);  // worker warps + the MMA commit
     }
-    for (int i = 0; i < C::kNA; ++i) {
-      mbar_init(&a_full[i], kGExp);
-      mbar_init(&a_free[i], 1);
-    }
-    for (int i = 0; i < C::kND; ++i) {
+    for (int i = 0; i < kGABufs; ++i) mbar_init(&a_full[i], kGWorkers);
+    for (int i = 0; i < kGDBufs; ++i) {
       mbar_init(&d_full[i], 1);
-      mbar_init(&d_free[i], kGRead);
-    }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&xa[i], 2);
-      mbar_init(&xb[i], 2);
-      mbar_init(&ra[i >> 1][i & 1], 2);
-      mbar_init(&rb[i >> 1][i & 1], 2);
+      mbar_init(&d_free[i], kGWorkers);
     }
     fence_barrier_init();
   }
-  if (warp == kGMmaWarp) {
+  if (warp == kGWorkers + 1) {
     tmem_alloc(&tmem_base_s, C::kTmemCols);
     tmem_relinquish();
   }
@@ -372,7 +345,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
   uint32_t sc = 0;  // stages started (the same sequence in every role)
   uint32_t gs = 0;  // slabs started
 
-  if (warp == kGProducer) {
+  if (warp == kGWorkers) {
     // ------------------------------------------------------------ producer ---
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       const int slot = tile / mtiles, m0 = (tile % mtiles) * a.mrows;
@@ -424,8 +397,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
     // leave no copy in flight: every stage issued has landed (at once when all went well)
     if (lane == 0)
       for (uint32_t i = sc > (uint32_t)C::kStages ? sc - C::kStages : 0; i < sc; ++i)
-        mbar_wait(&full[i % C::kStages], (i / C::kStages) & 1, kWaitLimitNs);
-  } else if (warp == kGMmaWarp) {
+        mbar_wait(&full[i % C::kStages], (i / C::kStages) & 1);
+  } else if (warp == kGWorkers + 1) {
     // ---------------------------------------------------------- MMA issuer ---
     // The whole warp runs this loop (operands warp-uniform); one elected lane issues.
     uint32_t issued = 0;  // slabs whose MMAs were issued
@@ -441,9 +414,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
           ok = __all_sync(kFull, mbar_wait(&full[st], round & 1));
           const uint32_t bbase = smem_u32(gsm + st * C::kStageBytes + kGOffB);
           for (int jj = 0; jj < kGSlabsPerStage && ok; ++jj, ++gs) {
-            const uint32_t ab = gs % C::kNA, db = gs % C::kND;
-            bool w = mbar_wait(&a_full[ab], (gs / C::kNA) & 1);
-            if (w && gs >= (uint32_t)C::kND) w = mbar_wait(&d_free[db], (gs / C::kND - 1) & 1);
+            const uint32_t ab = gs % kGABufs, db = gs % kGDBufs;
+            bool w = mbar_wait(&a_full[ab], (gs / kGABufs) & 1);
+            if (w && gs >= (uint32_t)kGDBufs) w = mbar_wait(&d_free[db], (gs / kGDBufs - 1) & 1);
             ok = __all_sync(kFull, w);
             if (!ok) break;
             tc_fence_after();
@@ -452,11 +425,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
               const uint64_t bdesc = sw128_desc(bbase + jj * C::kBTile + kk * 32);
 #pragma unroll
               for (int m = 0; m < 2; ++m)
-                tc_mma_ts_elect(tmem + C::col_d(db, m), tmem + C::col_a(ab, m) + kk * 8, bdesc,
-                                idesc, kk > 0 ? 1u : 0u);
+                tc_mma_ts_elect(tmem + C::col_d(db, m), tmem + C::col_a(ab, m) + kk * 8, bdesc, idesc,
+                                kk > 0 ? 1u : 0u);
             }
             tc_commit_elect(&d_full[db]);
-            tc_commit_elect(&a_free[ab]);
             if (jj == kGSlabsPerStage - 1) tc_commit_elect(&empty[st]);
             issued = gs + 1;
           }
@@ -464,71 +436,72 @@ __global__ void __launch_bounds__(kGThreads, 1)
       }
     }
     // no MMA may run past the deallocation below (at once when all went well)
-    if (issued > 0)
-      mbar_wait(&d_full[(issued - 1) % C::kND], ((issued - 1) / C::kND) & 1, kWaitLimitNs);
-  } else if (warp < kGExp) {
-    // ------------------------------------------------------------- expanders ---
-    // Lane r of the tensor memory: row r of both matrices.  Per slab, the rows' codes
-    // as bf16 integers into an A buffer, ahead of the MMAs.
-    const int r = 32 * warp + lane;
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    if (issued > 0) mbar_wait(&d_full[(issued - 1) % kGDBufs], ((issued - 1) / kGDBufs) & 1);
+  } else {
+    // ------------------------------------------------------------- workers ---
+    const int m = warp >> 2, qd = warp & 3, r = 32 * qd + lane;
+    const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
     const uint32_t one2 = 0x3F803F80u, m128 = 0xC300C300u;  // bf16 pairs (1, 1), (-128, -128)
-    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-      const int slot = tile / mtiles;
-      const int cnt = a.offsets[slot + 1] - a.offsets[slot];
-      for (int c0 = 0; c0 < cnt && ok; c0 += C::kN) {
-        for (int j0 = 0; j0 < nslab && ok; j0 += kGSlabsPerStage, ++sc) {
-          const int st = sc % C::kStages;
-          ok = __all_sync(kFull, mbar_wait(&full[st], (sc / C::kStages) & 1));
-          if (!ok) break;
-          const unsigned char* stg = gsm + st * C::kStageBytes;
-          for (int jj = 0; jj < kGSlabsPerStage && ok; ++jj, ++gs) {
-            const uint32_t ab = gs % C::kNA;
-            // the MMAs that read this A buffer (slab gs - kNA) are done
-            if (gs >= (uint32_t)C::kNA)
-              ok = __all_sync(kFull, mbar_wait(&a_free[ab], (gs / C::kNA - 1) & 1));
-            if (!ok) break;
-            tc_fence_after();
+    float2 acc[C::kN / 2];
+
+    // wait until the MMAs of slab gp are done (its accumulator is ready and the A
+    // buffer it read is free)
+    auto wait_slab = [&](uint32_t gp) {
+      ok = __all_sync(kFull, ok && mbar_wait(&d_full[gp % kGDBufs], (gp / kGDBufs) & 1));
+    };
+    // add the product of slab gp (stage st, place jj in the stage) to acc; its
+    // MMAs are known to be done
+    auto readout = [&](uint32_t gp, int st, int jj, int ng) {
+      const uint32_t ab = gp % kGDBufs;
+      tc_fence_after();
+      const unsigned char* stg = gsm + st * C::kStageBytes;
+      const float sv = bf16_bits_to_float(
+          *reinterpret_cast<const uint16_t*>(stg + C::kOffS + (m * kGM + r) * 4 + jj * 2));
+      const float bv = bf16_bits_to_float(
+          *reinterpret_cast<const uint16_t*>(stg + C::kOffBias + (m * kGM + r) * 4 + jj * 2));
+      const float2 s2 = make_float2(sv, sv), b2 = make_float2(bv, bv);
+      const float4* X = reinterpret_cast<const float4*>(stg + C::kOffX + jj * C::kN * 4);
+      const uint32_t dcol = tmem + C::col_d(ab, m) + lane_base;
+      // kRd columns per tensor-memory wait (16 where registers are scarce)
+      constexpr int kRd = C::kN == 64 ? 32 : 16, kRg = kRd / 16;
 #pragma unroll
-            for (int m = 0; m < 2; ++m) {
-              const uint4* crow =
-                  reinterpret_cast<const uint4*>(stg + (m * kGM + r) * kGCodePitch + jj * 32);
-              const uint32_t acol = tmem + C::col_a(ab, m) + lane_base;
+      for (int c2 = 0; c2 < C::kN / kRd; ++c2) {
+        if (kRg * c2 < ng) {
+          uint32_t pr[kRd];
+          tc_ld16(dcol + c2 * kRd, pr);
+          if constexpr (kRg == 2) {
+            if (2 * c2 + 1 < ng) tc_ld16(dcol + c2 * kRd + 16, pr + 16);
+          }
+          tc_wait_ld();
 #pragma unroll
-              for (int hw = 0; hw < 2; ++hw) {  // 32 codes (16 columns) at a time
-                const uint4 wv = crow[hw];
-                uint32_t av[16];
-                codes_to_bf16(wv.x, one2, m128, av + 0);
-                codes_to_bf16(wv.y, one2, m128, av + 4);
-                codes_to_bf16(wv.z, one2, m128, av + 8);
-                codes_to_bf16(wv.w, one2, m128, av + 12);
-                tc_st16(acol + 16 * hw, av);
+          for (int h = 0; h < kRg; ++h) {
+            const int cg = kRg * c2 + h;
+            if (cg < ng) {
+              tc_regs_ready(pr + 16 * h);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float4 xv = X[cg * 4 + i];
+                const int o = cg * 8 + 2 * i;
+                const uint32_t* pp = pr + 16 * h + 4 * i;
+                acc[o] = __ffma2_rn(make_float2(__uint_as_float(pp[0]), __uint_as_float(pp[1])),
+                                    s2, acc[o]);
+                acc[o + 1] = __ffma2_rn(
+                    make_float2(__uint_as_float(pp[2]), __uint_as_float(pp[3])), s2, acc[o + 1]);
+                acc[o] = __ffma2_rn(make_float2(xv.x, xv.y), b2, acc[o]);
+                acc[o + 1] = __ffma2_rn(make_float2(xv.z, xv.w), b2, acc[o + 1]);
               }
             }
-            tc_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&a_full[ab]);
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[st]);
         }
       }
-    }
-  } else {
-    // ------------------------------------------------------------- read-back ---
-    const int w8 = warp - kGExp;  // 0..7
-    const int m = w8 >> 2, qd = warp & 3, r = 32 * qd + lane;
-    const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
-    float2 acc[C::kN / 2];
-    uint32_t xr = 0;  // epilogue rounds so far (phase parity of the hand-over barriers)
-    // one hand-over: arrive (lane 0, after the warp's shared-memory writes), then wait,
-    // bounded, for the partner warp's arrival
-    auto hand_over = [&](uint64_t* bar) {
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar);
-      ok = __all_sync(kFull, ok && mbar_wait(bar, xr & 1));
+      if (lane == 0) {
+        mbar_arrive(&d_free[ab]);
+        if (jj == kGSlabsPerStage - 1) mbar_arrive(&empty[st]);
+      }
     };
+
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       const int slot = tile / mtiles, m0 = (tile % mtiles) * a.mrows;
       const int p0 = a.offsets[slot], cnt = a.offsets[slot + 1] - p0;
@@ -537,80 +510,99 @@ __global__ void __launch_bounds__(kGThreads, 1)
         const int n = min(C::kN, cnt - c0), np = (n + 15) & ~15, ng = np / 16;
 #pragma unroll
         for (int i = 0; i < C::kN / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+        const uint32_t gs0 = gs, sc0 = sc;  // first slab and stage of the chunk
+        // slab g of this chunk: stage (sc0 + (g - gs0) / 2) % C::kStages, place (g - gs0) & 1
+        auto read_slab = [&](uint32_t g) {
+          const uint32_t jl = g - gs0;
+          readout(g, (int)((sc0 + jl / kGSlabsPerStage) % C::kStages), (int)(jl % kGSlabsPerStage), ng);
+        };
         for (int j0 = 0; j0 < nslab && ok; j0 += kGSlabsPerStage, ++sc) {
           const int st = sc % C::kStages;
-          ok = __all_sync(kFull, mbar_wait(&full[st], (sc / C::kStages) & 1));
+          const uint32_t round = sc / C::kStages;
+          ok = __all_sync(kFull, mbar_wait(&full[st], round & 1));
           if (!ok) break;
           const unsigned char* stg = gsm + st * C::kStageBytes;
           for (int jj = 0; jj < kGSlabsPerStage && ok; ++jj, ++gs) {
-            const uint32_t db = gs % C::kND;
-            ok = __all_sync(kFull, mbar_wait(&d_full[db], (gs / C::kND) & 1));
+            const uint32_t ab = gs % kGABufs;
+            // the MMAs that read this A buffer (slab gs - 2) are done
+            if (gs >= (uint32_t)kGABufs) wait_slab(gs - kGABufs);
             if (!ok) break;
-            tc_fence_after();
-            const float sv = bf16_bits_to_float(
-                *reinterpret_cast<const uint16_t*>(stg + C::kOffS + (m * kGM + r) * 4 + jj * 2));
-            const float bv = bf16_bits_to_float(
-                *reinterpret_cast<const uint16_t*>(stg + C::kOffBias + (m * kGM + r) * 4 + jj * 2));
-            const float2 s2 = make_float2(sv, sv), b2 = make_float2(bv, bv);
-            const float4* X = reinterpret_cast<const float4*>(stg + C::kOffX + jj * C::kN * 4);
-            const uint32_t dcol = tmem + C::col_d(db, m) + lane_base;
+            tc_fence_after();  // the A buffer's earlier reads are done before these writes
+            // this row's codes of the slab -> bf16 integers -> the A operand
+            const uint4* crow =
+                reinterpret_cast<const uint4*>(stg + (m * kGM + r) * kGCodePitch + jj * 32);
+            const uint32_t acol = tmem + C::col_a(ab, m) + lane_base;
 #pragma unroll
-            for (int cg = 0; cg < C::kN / 16; ++cg) {
-              if (cg < ng) {
-                uint32_t pr[16];
-                tc_ld16(dcol + cg * 16, pr);
-                tc_wait_ld();
-                tc_regs_ready(pr);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const float4 xv = X[cg * 4 + i];
-                  const int o = cg * 8 + 2 * i;
-                  const uint32_t* pp = pr + 4 * i;
-                  acc[o] = __ffma2_rn(make_float2(__uint_as_float(pp[0]), __uint_as_float(pp[1])),
-                                      s2, acc[o]);
-                  acc[o + 1] = __ffma2_rn(
-                      make_float2(__uint_as_float(pp[2]), __uint_as_float(pp[3])), s2, acc[o + 1]);
-                  acc[o] = __ffma2_rn(make_float2(xv.x, xv.y), b2, acc[o]);
-                  acc[o + 1] = __ffma2_rn(make_float2(xv.z, xv.w), b2, acc[o + 1]);
-                }
-              }
+            for (int hw = 0; hw < 2; ++hw) {  // 32 codes (16 columns) at a time
+              const uint4 wv = crow[hw];
+              uint32_t av[16];
+              codes_to_bf16(wv.x, one2, m128, av + 0);
+              codes_to_bf16(wv.y, one2, m128, av + 4);
+              codes_to_bf16(wv.z, one2, m128, av + 8);
+              codes_to_bf16(wv.w, one2, m128, av + 12);
+              tc_st16(acol + 16 * hw, av);
             }
+            tc_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&d_free[db]);
+            if (lane == 0) mbar_arrive(&a_full[ab]);
+            if (gs >= gs0 + kGLag) {
+              wait_slab(gs - kGLag);
+              if (ok) read_slab(gs - kGLag);
+            }
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[st]);
+        }
+        if (!ok) break;
+        // the chunk's last kGLag slabs
+        for (uint32_t g = gs >= gs0 + kGLag ? gs - kGLag : gs0; g < gs && ok; ++g) {
+          wait_slab(g);
+          if (ok) read_slab(g);
         }
         if (!ok) break;
 
         if (PHASE == 0) {
           // ---- h = bf16(silu(bf16 g) * bf16 u); matrix 0 holds g, matrix 1 u.  The
-          // two warps of a lane quarter swap halves through shared memory, 16 pairs a
-          // round: this thread finishes pairs kHalf m + 16 hh + i.
+          // two warps of a lane quarter swap halves through tensor memory (buffer 0's
+          // accumulator columns): no MMA runs now, the next one waits for every
+          // warp's next A operand.
           const int irow = m0 + r;  // this thread's row of h's width I
           const int gI = irow / kGK, ci = irow % kGK;
           const int pin = (ci & ~7) + 2 * (ci & 3) + ((ci >> 2) & 1);  // K order position
-          constexpr int kHalf = C::kN / 2;
-          float* mine_x = xchg + ((size_t)m * kGM + r) * 16;
-          const float* other_x = xchg + ((size_t)(1 - m) * kGM + r) * 16;
+          constexpr int kHalf = C::kN / 2;  // pairs finished by each matrix's warps
 #pragma unroll
-          for (int hh = 0; hh < kHalf / 16; ++hh, ++xr) {
-            // matrix 0 gives g of pairs kHalf + 16hh.., matrix 1 gives u of pairs 16hh..
+          for (int hh = 0; hh < kHalf / 16; ++hh) {
+            // 16 pairs per round: this thread finishes pairs kHalf m + 16hh + i
+            uint32_t ex[16];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               const float2 v = m == 0 ? acc[kHalf / 2 + 8 * hh + i] : acc[8 * hh + i];
-              mine_x[2 * i] = v.x;
-              mine_x[2 * i + 1] = v.y;
+              ex[2 * i] = __float_as_uint(v.x);
+              ex[2 * i + 1] = __float_as_uint(v.y);
             }
-            hand_over(&xa[qd]);
-            if (!ok) break;
+            // each warp writes only its own matrix's columns (its partner may still be
+            // reading the other matrix's): matrix 0 gives g of pairs kHalf + 16hh.. at
+            // its columns kHalf + 16hh.., matrix 1 gives u of pairs 16hh.. at its
+            // columns 16hh..
+            const uint32_t give =
+                tmem + C::col_d(0, m) + (m == 0 ? kHalf : 0) + 16 * hh + lane_base;
+            const uint32_t take =
+                tmem + C::col_d(0, 1 - m) + (m == 0 ? 0 : kHalf) + 16 * hh + lane_base;
+            tc_st16(give, ex);
+            tc_wait_st();
+            tc_fence_before();
+            named_barrier(1 + qd, 64);
+            tc_fence_after();
+            uint32_t ot[16];
+            tc_ld16(take, ot);
+            tc_wait_ld();
+            tc_regs_ready(ot);
+            tc_fence_before();
             float hv[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float2 mv = m == 0 ? acc[8 * hh + i / 2] : acc[kHalf / 2 + 8 * hh + i / 2];
-              const float own = (i & 1) ? mv.y : mv.x;
-              const float oth = other_x[i];
+              const float2 mine = m == 0 ? acc[8 * hh + i / 2] : acc[kHalf / 2 + 8 * hh + i / 2];
+              const float own = (i & 1) ? mine.y : mine.x;
+              const float oth = __uint_as_float(ot[i]);
               const float g = round_to_bf16(m == 0 ? own : oth);
               const float uu = round_to_bf16(m == 0 ? oth : own);
               const uint16_t hb = float_to_bf16_bits(g / (1.0f + __expf(-g)) * uu);
@@ -622,22 +614,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
                      (pin & 7)] = hb;
               }
             }
-            hand_over(&xb[qd]);  // the exchange buffer is free again
-            if (!ok) break;
             // group sums of h: over this warp's 32 rows (even lanes end with one
             // pair's sum each), then over the group's two warps
             int vid;
             const float part = warp_reduce_scatter<16>(hv, lane, vid);
             if ((qd & 1) && !(lane & 1)) red[m][qd >> 1][16 * hh + vid] = part;
-            hand_over(&ra[m][qd >> 1]);
-            if (!ok) break;
+            named_barrier(5 + 2 * m + (qd >> 1), 64);
             if (!(qd & 1) && !(lane & 1)) {
               const int nn = kHalf * m + 16 * hh + vid;
               if (nn < np)
                 a.hs[(size_t)gI * a.pcap + pp0 + c0 + nn] = part + red[m][qd >> 1][16 * hh + vid];
             }
-            hand_over(&rb[m][qd >> 1]);
-            if (!ok) break;
+            named_barrier(5 + 2 * m + (qd >> 1), 64);
           }
         } else {
           // ---- y rows of the chunk's pairs (pair_list order), fp32
@@ -651,7 +639,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kGMmaWarp) {
+  if (warp == kGWorkers + 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }

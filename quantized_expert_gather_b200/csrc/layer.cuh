@@ -73,7 +73,7 @@ constexpr int kMaxRowsPerWarpB = 4; // phase B: rows of Wd per warp per block
 // one phase ahead of that stage (an odd depth would let one team's wait for a later
 // block pass on the phase of the other team's block still in flight).
 constexpr int kMaxStages = 4;
-constexpr int kNT = 1;              // pairs per compute pass
+constexpr int kNT = 2;              // pairs per compute pass (phase A; phase B takes one)
 constexpr int kMaxPairsFused = 1024;
 constexpr unsigned kBarUnion = 1;   // named barrier: union formed (warp 0 -> producer)
 constexpr unsigned kBarWork = 2;    // named barrier: every warp but the producer
@@ -1185,17 +1185,26 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
         const unsigned char* buq = bu + (size_t)w * (a.H / 2);
         const uint16_t* bus = reinterpret_cast<const uint16_t*>(bu + G.a_q) + w * (a.H / 64);
         const uint16_t* bub = reinterpret_cast<const uint16_t*>(bu + G.a_q + G.a_sb) + w * (a.H / 64);
-        for (int c = 0; c < nt; ++c) {
-          // the pair's activation row: the token's resident x row, or row c of the set
-          const unsigned char* const arow[kNT] = {x_res ? actp + tok_of[p0 + c] * stride_a
-                                                        : actp + c * stride_a};
+        // the segment's pairs two at a time (the codes split once for both), the last
+        // one alone
+        for (int c = 0; c < nt; c += kNT) {
+          const int ntc = min(kNT, nt - c);
+          // each pair's activation row: the token's resident x row, or its row of the set
+          const unsigned char* arow[kNT];
+#pragma unroll
+          for (int t = 0; t < kNT; ++t) {
+            const int q = c + (t < ntc ? t : 0);
+            arow[t] = x_res ? actp + tok_of[p0 + q] * stride_a : actp + q * stride_a;
+          }
           float Gs[kNT], Us[kNT];
-          dispatch_a<1, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
-          if (lane == 0) {
-            const float g = round_to_bf16(Gs[0]), hu = round_to_bf16(Us[0]);
+          if (ntc == 2) dispatch_a<2, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
+          else dispatch_a<1, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
+          if (lane < ntc) {
+            const float g = round_to_bf16(lane == 0 ? Gs[0] : Gs[1]);
+            const float hu = round_to_bf16(lane == 0 ? Us[0] : Us[1]);
             // silu(g) = g / (1 + e^-g); the fast division's error (2 ulp of fp32) is far
             // below the bf16 step h is rounded to
-            a.h[(size_t)(p0 + c) * a.I + row0 + w] =
+            a.h[(size_t)(p0 + c + lane) * a.I + row0 + w] =
                 float_to_bf16_bits(__fdividef(g, 1.0f + __expf(-g)) * hu);
           }
         }
@@ -1208,7 +1217,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
           const float v = dispatch_b<1, F>(G.rounds_b, buf, bs, bb, w, nrows, a.I,
                                            actp + (size_t)c * stride_b, stride_b, lane, vid);
           if (vid >= 0) {
-            const int r = w + kTeamWarps * vid;
+            const int r = w + kTeamWarps * (vid / kNT);
             if (r < nrows) a.y[(size_t)(p0 + c) * a.H + row0 + r] = v;
           }
         }
