@@ -769,8 +769,35 @@ def our_arm(args, world, rank, local):
             torch.cuda.synchronize()
             rt[str(TR)] = a5.elapsed_time(b5) * 1e3 / 400
             del g5
+        # the router fused into the layer (one launch) against the router kernel then the
+        # layer (two), 42 chained layers each on the bench bank, CUDA graph; per layer
+        fused, two = {}, {}
+        for TR in (1, 4, 16):
+            lgs = [torch.from_numpy(np.random.default_rng(SEED + 80 + 100 * TR + l)
+                                    .standard_normal((TR, E)).astype(np.float32)).to(dev)
+                   for l in range(LAYERS)]
+            xr = torch.from_numpy(synth.x_bf16(TR, HIDDEN, SEED + TR).view(np.int16)).to(dev) \
+                .view(torch.bfloat16)
+            orr = torch.empty((TR, HIDDEN), dtype=torch.bfloat16, device=dev)
+            ri = torch.empty((TR, K_TOP), dtype=torch.int32, device=dev)
+            rw = torch.empty((TR, K_TOP), dtype=torch.float32, device=dev)
+            wsr = torch.zeros(qeg.moe_workspace_size(TR, K_TOP, E, HIDDEN, INTER),
+                              dtype=torch.uint8, device=dev)
+            fused[str(TR)] = graph_us_per_layer(
+                lambda: [qeg.moe_switchglu_forward_routed(xr, lgs[l], K_TOP, bank, workspace=wsr,
+                                                          out=orr, topk_idx=ri, topk_w=rw)
+                         for l in range(LAYERS)], LAYERS)
+
+            def two_step():
+                for l in range(LAYERS):
+                    qeg.moe_router_topk(lgs[l], K_TOP, topk_idx=ri, topk_w=rw)
+                    qeg.moe_switchglu_forward_ws(xr, ri, rw, bank, wsr, out=orr)
+            two[str(TR)] = graph_us_per_layer(two_step, LAYERS)
+            del wsr
         router = {"E": E, "k": K_TOP, "renormalize": True, "us_per_call_graph": rt,
-                  "us_per_call_python": rt_host}
+                  "us_per_call_python": rt_host,
+                  "router_and_layer_us_per_layer_graph": {"fused_one_launch": fused,
+                                                          "router_then_layer": two}}
     except Exception as ex:  # report, never lose the headline line
         router = {"error": repr(ex)}
 

@@ -250,6 +250,42 @@ moe_status moe_router_topk(const float* logits, int T, int E, int k, int renorma
                            int32_t* topk_idx, float* topk_w, void* stream);
 
 /*
+ * The router step and the layer in one call: the experts of each token are picked
+ * from router logits exactly as moe_router_topk does (top-k of softmax, descending,
+ * lower id first among equal logits, weights renormalised over the k when
+ * renormalize != 0), then the layer of moe_switchglu_forward_ws runs on those picks.
+ * On the persistent path (moe_select_path == 1 with the picks' shared-memory room)
+ * every CTA makes the picks in its own prologue, so there is one launch for the
+ * router and the layer; on the grouped path the router kernel runs first (two
+ * launches more than the layer's own).  Both write the picks and weights to
+ * topk_idx / topk_w ([T*k] int32 / fp32, device, 4-byte aligned, caller-owned),
+ * which equal moe_router_topk's on the same logits bit for bit.
+ *   logits [T*E] fp32 (finite), x, bank and out as for moe_switchglu_forward_ws;
+ *   workspace of moe_workspace_size(T, k, E, hidden, inter) bytes.
+ * "Small-L fused expert gather for fine-grained MoE decode" (mlx discussion 3801):
+ * the picks feed the union of the window directly.
+ * Errors: those of moe_switchglu_forward_ws and moe_router_topk (E > 1024 or k > 32
+ * is MOE_ERR_UNSUPPORTED, k > E is MOE_ERR_INVALID_ARG).
+ */
+moe_status moe_switchglu_forward_routed_ws(
+    const uint16_t* x, const float* logits, int renormalize, const uint32_t* wg_q,
+    const uint16_t* wg_s, const uint16_t* wg_b, const uint32_t* wu_q, const uint16_t* wu_s,
+    const uint16_t* wu_b, const uint32_t* wd_q, const uint16_t* wd_s, const uint16_t* wd_b, int T,
+    int k, int E, int hidden, int inter, uint16_t* out, int32_t* topk_idx, float* topk_w,
+    void* workspace, size_t workspace_bytes, void* stream);
+
+/* moe_switchglu_forward_routed_ws with a library-owned workspace per device (as for
+ * moe_switchglu_forward). */
+moe_status moe_switchglu_forward_routed(const uint16_t* x, const float* logits, int renormalize,
+                                        const uint32_t* wg_q, const uint16_t* wg_s,
+                                        const uint16_t* wg_b, const uint32_t* wu_q,
+                                        const uint16_t* wu_s, const uint16_t* wu_b,
+                                        const uint32_t* wd_q, const uint16_t* wd_s,
+                                        const uint16_t* wd_b, int T, int k, int E, int hidden,
+                                        int inter, uint16_t* out, int32_t* topk_idx,
+                                        float* topk_w, void* stream);
+
+/*
  * Which kernel path a call with this shape takes, without launching anything:
  * 1 = expert-major dequant-GEMV layer kernel (T*k <= 1024 and its shared-memory
  * plan fits), 2 = grouped tensor-core path (route-union, x packing, gate+up and

@@ -64,6 +64,13 @@ def _load():
     lib.moe_switchglu_forward_ws.argtypes = [vp] * 12 + [ci] * 5 + [vp, vp, sz, vp]
     lib.moe_switchglu_forward_static.restype = ci
     lib.moe_switchglu_forward_static.argtypes = [vp] * 12 + [ci] * 5 + [vp, vp]
+    # (x, logits, renormalize, 9 bank pointers, T, k, E, hidden, inter, out, topk_idx,
+    # topk_w, [workspace, bytes,] stream)
+    lib.moe_switchglu_forward_routed.restype = ci
+    lib.moe_switchglu_forward_routed.argtypes = [vp, vp, ci] + [vp] * 9 + [ci] * 5 + [vp] * 4
+    lib.moe_switchglu_forward_routed_ws.restype = ci
+    lib.moe_switchglu_forward_routed_ws.argtypes = ([vp, vp, ci] + [vp] * 9 + [ci] * 5 +
+                                                    [vp] * 4 + [sz, vp])
     lib.moe_workspace_size_mxfp4.restype = sz
     lib.moe_workspace_size_mxfp4.argtypes = [ci] * 5
     lib.moe_select_path_mxfp4.restype = ci
@@ -281,6 +288,53 @@ def moe_switchglu_forward_static(x, topk_idx, topk_w, bank: QuantBank, out=None,
         raise MoeError(st, f"moe_switchglu_forward_static [{moe_last_error()}]")
     _check(st, "moe_switchglu_forward_static", check)
     return out
+
+
+def _routed_args(x, logits, k, bank: QuantBank, out, topk_idx, topk_w):
+    T, hidden = x.shape
+    if hidden != bank.hidden or logits.dim() != 2 or logits.shape[0] != T \
+            or logits.shape[1] != bank.E:
+        raise ValueError("x / logits shapes do not match the bank")
+    dev = x.device
+    out = out if out is not None else torch.empty((T, hidden), dtype=torch.bfloat16, device=dev)
+    topk_idx = topk_idx if topk_idx is not None else torch.empty((T, k), dtype=torch.int32,
+                                                                 device=dev)
+    topk_w = topk_w if topk_w is not None else torch.empty((T, k), dtype=torch.float32,
+                                                           device=dev)
+    if tuple(out.shape) != (T, hidden) or tuple(topk_idx.shape) != (T, k) \
+            or tuple(topk_w.shape) != (T, k):
+        raise ValueError("out / topk_idx / topk_w have the wrong shape")
+    _same_device(dev, logits=logits, out=out, topk_idx=topk_idx, topk_w=topk_w, wg_q=bank.wg_q,
+                 wd_q=bank.wd_q)
+    return out, topk_idx, topk_w
+
+
+def moe_switchglu_forward_routed(x, logits, k: int, bank: QuantBank, renormalize: bool = True,
+                                 workspace=None, out=None, topk_idx=None, topk_w=None,
+                                 stream=None, check: bool = True):
+    """The router step and the layer in one call: picks of top-k of softmax over each row of
+    logits [T, E] (fp32, CUDA) as moe_router_topk makes them, then the layer on those picks.
+    Returns (out [T, hidden] bf16, topk_idx [T, k] int32, topk_w [T, k] fp32).  With
+    `workspace` (see moe_workspace) the call uses it, else the library-owned one."""
+    out, topk_idx, topk_w = _routed_args(x, logits, k, bank, out, topk_idx, topk_w)
+    T, hidden = x.shape
+    dims = (T, k, bank.E, hidden, bank.inter)
+    head = [_ptr(x, _BF16, "x"), _ptr(logits, _F32, "logits"), 1 if renormalize else 0,
+            *bank.ptrs()]
+    tail = [_ptr(out, _BF16, "out"), _ptr(topk_idx, _I32, "topk_idx"),
+            _ptr(topk_w, _F32, "topk_w")]
+    with torch.cuda.device(x.device):
+        if workspace is None:
+            st = _lib.moe_switchglu_forward_routed(*head, *dims, *tail, _stream(stream, x.device))
+            name = "moe_switchglu_forward_routed"
+        else:
+            _same_device(x.device, workspace=workspace)
+            st = _lib.moe_switchglu_forward_routed_ws(
+                *head, *dims, *tail, _ptr(workspace, (torch.uint8,), "workspace"),
+                workspace.numel(), _stream(stream, x.device))
+            name = "moe_switchglu_forward_routed_ws"
+    _check(st, name, check)
+    return out, topk_idx, topk_w
 
 
 MOE_STATIC_SCRATCH_BYTES = 4 << 20

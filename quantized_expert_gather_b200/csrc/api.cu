@@ -101,11 +101,14 @@ struct WsLayout {
 // kernels (windows with more pairs; hidden a multiple of 256, inter of 128),
 // 0 = neither.
 // mxfp4 banks take the persistent kernel only (0 for larger windows).
-int select_path(int T, int k, int E, int hidden, int inter, int fmt = kFmtAffine) {
+// `routed`: the router step runs inside the persistent kernel (its picks and weights
+// take shared memory too).
+int select_path(int T, int k, int E, int hidden, int inter, int fmt = kFmtAffine,
+                bool routed = false) {
   if (!shape_ok(T, k, E, hidden, inter) || !shape_supported(T, k, E, hidden, inter)) return 0;
   if (T * k <= kMaxPairsFused) {
     LayerGeom g = layer_geom(hidden, inter, fmt);
-    if (layer_plan(g, E, T, k, kSmemBudget)) return 1;
+    if (layer_plan(g, E, T, k, kSmemBudget, routed)) return 1;
   }
   if (fmt == kFmtMx) return 0;
   // the grouped path: hidden a multiple of 256 (down tiles) and at most 4096, inter a
@@ -147,9 +150,15 @@ cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
                          const uint32_t* uq, const uint16_t* us, const uint16_t* ub,
                          const uint32_t* dq, const uint16_t* ds, const uint16_t* db, int T, int k,
                          int E, int H, int I, uint16_t* out, unsigned char* ws,
-                         const DeviceInfo& d, cudaStream_t st, moe_status* why) {
+                         const DeviceInfo& d, cudaStream_t st, moe_status* why,
+                         const float* logits = nullptr, int renorm = 0,
+                         int32_t* ridx_out = nullptr, float* rw_out = nullptr) {
   const WsLayout wl = ws_layout(T, k, E, H, I);
   LayerArgs a;
+  a.logits = logits;  // the fused router step (idx and w unused then)
+  a.renorm = renorm;
+  a.ridx_out = ridx_out;
+  a.rw_out = rw_out;
   a.x = x;
   a.idx = idx;
   a.w = w;
@@ -178,7 +187,12 @@ cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
   a.g = layer_geom(H, I, F);
   a.wait_prior = 1;
   const int ki = F == kFmtMx ? 9 : 0;  // dyn_smem index of this layer kernel
-  if (!layer_plan(a.g, E, T, k, (size_t)d.dyn_smem[ki])) {
+  if (!layer_plan(a.g, E, T, k, (size_t)d.dyn_smem[ki], logits != nullptr)) {
+    *why = MOE_ERR_UNSUPPORTED;
+    return cudaSuccess;
+  }
+  // the fused router stages one logit row per routing warp behind the tables
+  if (logits && (size_t)kRouteWarps * ((5u * (unsigned)E + 15u) & ~15u) > a.g.total - a.g.tables) {
     *why = MOE_ERR_UNSUPPORTED;
     return cudaSuccess;
   }
@@ -500,6 +514,67 @@ moe_status moe_switchglu_forward(const uint16_t* x, const int32_t* topk_idx, con
     return s;
   return moe_switchglu_forward_ws(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q,
                                   wd_s, wd_b, T, k, E, hidden, inter, out, ws, bytes, stream);
+}
+
+moe_status moe_switchglu_forward_routed_ws(
+    const uint16_t* x, const float* logits, int renormalize, const uint32_t* wg_q,
+    const uint16_t* wg_s, const uint16_t* wg_b, const uint32_t* wu_q, const uint16_t* wu_s,
+    const uint16_t* wu_b, const uint32_t* wd_q, const uint16_t* wd_s, const uint16_t* wd_b, int T,
+    int k, int E, int hidden, int inter, uint16_t* out, int32_t* topk_idx, float* topk_w,
+    void* workspace, size_t workspace_bytes, void* stream) {
+  if (!x || !logits || !wg_q || !wg_s || !wg_b || !wu_q || !wu_s || !wu_b || !wd_q || !wd_s ||
+      !wd_b || !out || !topk_idx || !topk_w || !workspace)
+    return MOE_ERR_INVALID_ARG;
+  if (!shape_ok(T, k, E, hidden, inter) || k > E) return MOE_ERR_INVALID_ARG;
+  if (E > kRouterMaxE || k > kRouterMaxK) return MOE_ERR_UNSUPPORTED;
+  const void* a16[] = {x, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q, wd_s, wd_b, out, workspace};
+  for (const void* p : a16)
+    if (!aligned(p, 16)) return MOE_ERR_UNSUPPORTED;
+  if (!aligned(logits, 4) || !aligned(topk_idx, 4) || !aligned(topk_w, 4))
+    return MOE_ERR_UNSUPPORTED;
+  const int path = select_path(T, k, E, hidden, inter, kFmtAffine, true);
+  if (path == 0) return MOE_ERR_UNSUPPORTED;
+  if (workspace_bytes < ws_layout(T, k, E, hidden, inter).total) return MOE_ERR_WORKSPACE;
+  DeviceInfo* d = nullptr;
+  if (moe_status s = device_info(&d)) return s;
+  const cudaStream_t st = (cudaStream_t)stream;
+  moe_status why = MOE_OK;
+  cudaError_t e;
+  if (path == 1) {
+    e = launch_layer<kFmtAffine>(x, nullptr, nullptr, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q,
+                                 wd_s, wd_b, T, k, E, hidden, inter, out,
+                                 static_cast<unsigned char*>(workspace), *d, st, &why, logits,
+                                 renormalize ? 1 : 0, topk_idx, topk_w);
+  } else {
+    // the grouped path takes the picks from the router kernel, then its five launches
+    router_topk_kernel<<<(T + kRouterWarps - 1) / kRouterWarps, 32 * kRouterWarps, 0, st>>>(
+        logits, T, E, k, renormalize ? 1 : 0, topk_idx, topk_w);
+    e = cudaGetLastError();
+    if (e == cudaSuccess)
+      e = launch_grouped(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q, wd_s,
+                         wd_b, T, k, E, hidden, inter, out,
+                         static_cast<unsigned char*>(workspace), *d, st, &why);
+  }
+  if (why != MOE_OK) return why;
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+moe_status moe_switchglu_forward_routed(const uint16_t* x, const float* logits, int renormalize,
+                                        const uint32_t* wg_q, const uint16_t* wg_s,
+                                        const uint16_t* wg_b, const uint32_t* wu_q,
+                                        const uint16_t* wu_s, const uint16_t* wu_b,
+                                        const uint32_t* wd_q, const uint16_t* wd_s,
+                                        const uint16_t* wd_b, int T, int k, int E, int hidden,
+                                        int inter, uint16_t* out, int32_t* topk_idx,
+                                        float* topk_w, void* stream) {
+  if (!shape_ok(T, k, E, hidden, inter)) return MOE_ERR_INVALID_ARG;
+  void* ws = nullptr;
+  size_t bytes = 0;
+  if (moe_status s = owned_workspace(T, k, E, hidden, inter, kFmtAffine, stream, &ws, &bytes))
+    return s;
+  return moe_switchglu_forward_routed_ws(x, logits, renormalize, wg_q, wg_s, wg_b, wu_q, wu_s,
+                                         wu_b, wd_q, wd_s, wd_b, T, k, E, hidden, inter, out,
+                                         topk_idx, topk_w, ws, bytes, stream);
 }
 
 moe_status moe_switchglu_forward_static(const uint16_t* x, const int32_t* topk_idx,

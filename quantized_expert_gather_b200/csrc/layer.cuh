@@ -50,6 +50,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "router.cuh"
 #include "union.cuh"
 
 namespace qeg {
@@ -71,12 +72,15 @@ constexpr int kMaxRowsPerWarpB = 4; // phase B: rows of Wd per warp per block
 // stage j % depth and belongs to team j % 2, so with an even depth every stage is
 // used by one team only, and a team's parity wait on a stage can never be more than
 // one phase ahead of that stage (an odd depth would let one team's wait for a later
-// block pass on the phase of the other team's block still in flight).
+// block pass on the phase of the other team's block still in flight; waiting first
+// for the stage's previous block to be consumed avoids that, but couples the teams
+// and measured slower with 5 stages than with 4).
 constexpr int kMaxStages = 4;
 constexpr int kNT = 2;              // pairs per compute pass (phase A; phase B takes one)
 constexpr int kMaxPairsFused = 1024;
 constexpr unsigned kBarUnion = 1;   // named barrier: union formed (warp 0 -> producer)
 constexpr unsigned kBarWork = 2;    // named barrier: every warp but the producer
+constexpr int kRouteWarps = kWarps;  // warps picking the experts when the router is fused
 // Dynamic shared memory the kernel may plan for on B200 (227 KB per block, less a
 // margin for its static shared memory).
 constexpr size_t kSmemBudget = 232448 - 1024;
@@ -144,9 +148,11 @@ __host__ __device__ inline LayerGeom layer_geom(int H, int I, int fmt = kFmtAffi
 // maps, and the segment tables of phase A and of phase B (at most P each).
 struct LayerSmem {
   size_t cnt, rank, unique, offsets, pair_list, pos_of, tok_of, sa_slot, sa_pos, sa_nt, sb_slot,
-      sb_pos, sb_nt, end;
+      sb_pos, sb_nt, ridx, rw, end;
 };
-__host__ __device__ inline LayerSmem layer_smem(int E, int P) {
+// `routed`: the kernel picks the experts itself from router logits, and the picks and
+// their weights (P ints, P floats) are kept here too.
+__host__ __device__ inline LayerSmem layer_smem(int E, int P, bool routed = false) {
   LayerSmem s;
   const int m = (E < P ? E : P) > 0 ? (E < P ? E : P) : 1;
   s.cnt = 0;
@@ -162,7 +168,9 @@ __host__ __device__ inline LayerSmem layer_smem(int E, int P) {
   s.sb_slot = align_up(s.sa_nt + sizeof(int) * P, 16);
   s.sb_pos = align_up(s.sb_slot + sizeof(int) * P, 16);
   s.sb_nt = align_up(s.sb_pos + sizeof(int) * P, 16);
-  s.end = align_up(s.sb_nt + sizeof(int) * P, 128);
+  s.ridx = align_up(s.sb_nt + sizeof(int) * P, 16);
+  s.rw = align_up(s.ridx + (routed ? sizeof(int) * P : 0), 16);
+  s.end = align_up(s.rw + (routed ? sizeof(float) * P : 0), 128);
   return s;
 }
 
@@ -171,9 +179,10 @@ __host__ __device__ inline LayerSmem layer_smem(int E, int P) {
 // min(T, 8) h rows of activations, the rest of the budget being the activation area; and a wide
 // layout holding all T x rows when that needs more than the normal area (its ring at
 // least 2 stages deep and even, else none).  False if not even the normal layout fits.
-__host__ __device__ inline bool layer_plan(LayerGeom& g, int E, int T, int k, size_t budget) {
+__host__ __device__ inline bool layer_plan(LayerGeom& g, int E, int T, int k, size_t budget,
+                                           bool routed = false) {
   const int P = T * k;
-  g.tables = (unsigned)layer_smem(E, P).end;
+  g.tables = (unsigned)layer_smem(E, P, routed).end;
   const size_t ra = act_bytes(g.rounds_a), rbb = act_bytes(g.rounds_b);
   // an expert has at most T pairs in the window, so min(T, 8) h rows hold its set
   const size_t hmin = (size_t)(T < 8 ? T : 8) * rbb;
@@ -226,6 +235,13 @@ struct LayerArgs {
   int wait_prior;     // wait for the preceding grid before reading any input
   int x_res;          // every x row of the window fits one activation buffer: each CTA
                       // keeps them all in shared memory for phase A
+  // Router step fused ahead of the union (idx and w unused): [T, E] fp32 logits, top-k
+  // of their softmax per token, renormalised over the k when renorm is set; CTA 0
+  // writes the picks and weights to ridx_out / rw_out ([T, k]).
+  const float* logits;
+  int renorm;
+  int* ridx_out;
+  float* rw_out;
 };
 
 // ------------------------------------------------- activations and codes ---
@@ -611,18 +627,19 @@ constexpr int kPubRing = 16;      // blocks between compute and publication
 template <int F>
 __device__ __forceinline__ void convert_set(const LayerArgs& a, const LayerGeom& G, bool phase_b,
                                             const int* tok_of, int p0, int nt,
-                                            unsigned char* buf, int lane) {
+                                            unsigned char* buf, int lane, int tid = threadIdx.x,
+                                            int nthreads = kConsumerThreads) {
   const int D = phase_b ? a.I : a.H, R = phase_b ? G.rounds_b : G.rounds_a, nch = D / 32;
   const unsigned stride = act_bytes(R);
   const int nq = nt * nch * 4;  // quarters of 8 columns
   // kBatch quarters per thread at a time: their loads are all issued before the first
   // conversion waits on one
   constexpr int kBatch = 4;
-  for (int q0 = threadIdx.x; q0 < nq; q0 += kBatch * kConsumerThreads) {
+  for (int q0 = tid; q0 < nq; q0 += kBatch * nthreads) {
     uint4 v[kBatch];
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
-      const int q = q0 + i * kConsumerThreads;
+      const int q = q0 + i * nthreads;
       v[i] = make_uint4(0u, 0u, 0u, 0u);
       if (q < nq) {
         const int m = q & 3, tc = q >> 2, t = tc / nch, ch = tc % nch;
@@ -635,7 +652,7 @@ __device__ __forceinline__ void convert_set(const LayerArgs& a, const LayerGeom&
     }
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
-      const int q = q0 + i * kConsumerThreads;
+      const int q = q0 + i * nthreads;
       if (q < nq) {  // the four lanes of a chunk agree (nq is a multiple of 4)
         const int m = q & 3, tc = q >> 2, t = tc / nch, ch = tc % nch;
         uint4 packed;
@@ -812,14 +829,17 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
   __shared__ int s_u, s_nsb, s_ns, s_xres, s_wide, s_sega;
   __shared__ int s_rng[8];  // this CTA's block ranges (plan_shares)
   __shared__ unsigned s_act_off, s_act_size;
+  __shared__ unsigned s_bbase, s_bhalf;  // per-team phase-B set halves: offset, size
+  __shared__ int s_bsep;                 // the halves do not overlap the x rows
   __shared__ volatile int s_abort;
   __shared__ volatile int s_pub;  // blocks published by the helper warp
   __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
   __shared__ __align__(8) uint64_t done[kPubRing];           // a block's outputs written
   __shared__ __align__(8) uint64_t set_in[1], set_out[1];    // activation-set hand-over
+  __shared__ __align__(8) uint64_t team_in[kTeams], team_out[kTeams];  // per-team phase-B sets
   const LayerGeom& G = a.g;
   const int P = a.T * a.k;
-  const LayerSmem L = layer_smem(a.E, P);
+  const LayerSmem L = layer_smem(a.E, P, a.logits != nullptr);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned* exit_cnt = a.sync;
   unsigned* hdone = a.sync + 1;
@@ -834,6 +854,10 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
     for (int i = 0; i < kPubRing; ++i) mbar_init(&done[i], kTeamWarps);
     mbar_init(&set_in[0], kWarps);
     mbar_init(&set_out[0], kWarps);
+    for (int t = 0; t < kTeams; ++t) {
+      mbar_init(&team_in[t], kTeamWarps);
+      mbar_init(&team_out[t], kTeamWarps);
+    }
     s_abort = 0;
     s_pub = 0;
     fence_barrier_init();
@@ -855,9 +879,32 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
   unsigned char* ring = smem + G.tables;
   // every thread but the producer warp's, numbered 0 .. kThreads - 33
   const int wt = warp < kWarps ? (int)threadIdx.x : (int)threadIdx.x - 32;
+  // ---- the router step, when fused: warps 0 .. kRouteWarps-1 take one token each in
+  // turn (router.cuh), staging its logits in the ring and activation area, which are
+  // unused until the plan is made; the picks and weights stay in shared memory ----
+  const bool routed = a.logits != nullptr;
+  int* ridx = reinterpret_cast<int*>(smem + L.ridx);
+  float* rw = reinterpret_cast<float*>(smem + L.rw);
+  if (routed) {
+    if (warp < kRouteWarps) {
+      const unsigned stride = (5u * (unsigned)a.E + 15u) & ~15u;
+      float* v = reinterpret_cast<float*>(ring + (size_t)warp * stride);
+      unsigned char* taken = reinterpret_cast<unsigned char*>(v + a.E);
+      for (int t = warp; t < a.T; t += kRouteWarps) {
+        int pi;
+        float pw;
+        router_row(a.logits + (size_t)t * a.E, a.E, a.k, a.renorm, v, taken, lane, &pi, &pw);
+        if (lane < a.k) {
+          ridx[t * a.k + lane] = pi;
+          rw[t * a.k + lane] = pw;
+        }
+      }
+    }
+    if (warp != kWarps) named_barrier(kBarWork, kThreads - 32);  // every warp but the producer
+  }
   if (warp == 0) {
     int nv;
-    const int u = warp_route_union(a.idx, P, a.E, reinterpret_cast<int*>(smem + L.cnt),
+    const int u = warp_route_union(routed ? ridx : a.idx, P, a.E, reinterpret_cast<int*>(smem + L.cnt),
                                    reinterpret_cast<int*>(smem + L.rank), uniq, offs, plist, &nv);
     // the plan: a window whose x rows fit the normal activation area keeps them resident;
     // one with an expert of more pairs than that area holds x rows takes the wide layout
@@ -874,7 +921,17 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
     const unsigned act_size = wide ? G.act_w : G.act_n;
     const int ns = wide ? G.stages_w : G.stages;
     const int sega = xr ? max(P, 1) : max(sega_n, 1);
-    const int segb = max((int)(act_size / stride_b), 1);
+    // phase-B sets are per team, each in half of the area; when the resident x rows
+    // leave room for halves that hold as many pairs as an expert can have (at most T),
+    // the halves follow the x rows, and no team waits for the other at the turn from
+    // phase A to phase B
+    const unsigned xbytes = xr ? (unsigned)(((size_t)a.T * stride_a + 15) & ~(size_t)15) : 0u;
+    const unsigned half_all = (act_size / 2) & ~15u;
+    const unsigned half_sep = xbytes < act_size ? ((act_size - xbytes) / 2) & ~15u : 0u;
+    const int need = max(min(a.T, (int)(half_all / stride_b)), 1);
+    const bool bsep = xr && (int)(half_sep / stride_b) >= need;
+    const unsigned bhalf = bsep ? half_sep : half_all;
+    const int segb = max((int)(bhalf / stride_b), 1);
     const int nsa = make_segments(offs, u, sega, sa_slot, sa_pos, sa_nt, lane);
     const int nsb = make_segments(offs, u, segb, sb_slot, sb_pos, sb_nt, lane);
     __syncwarp();
@@ -894,6 +951,9 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
       s_sega = sega;
       s_act_off = G.tables + (unsigned)ns * G.stage_bytes;
       s_act_size = act_size;
+      s_bbase = bsep ? xbytes : 0u;
+      s_bhalf = bhalf;
+      s_bsep = bsep ? 1 : 0;
     }
     __syncwarp();
     named_barrier_arrive(kBarUnion, 64);  // the producer may start (it waits on this)
@@ -924,6 +984,12 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
     named_barrier(kBarWork, kThreads - 32);
   }
 
+  if (blockIdx.x == 0 && warp == 2 && routed && a.ridx_out) {
+    for (int i = lane; i < P; i += 32) {
+      a.ridx_out[i] = ridx[i];
+      a.rw_out[i] = rw[i];
+    }
+  }
   if (blockIdx.x == 0 && warp == 1 && a.ex_u) {
     for (int i = lane; i < u; i += 32) a.ex_unique[i] = uniq[i];
     for (int i = lane; i <= u; i += 32) a.ex_offsets[i] = offs[i];
@@ -1068,22 +1134,22 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
           const size_t r0 = (size_t)uniq[sa_slot[sg]] * a.I + row0;
           const size_t qrow = a.H / 8, srow = a.H / 64;
           mbar_arrive_expect_tx(&full[st], G.a_bytes);
-          bulk_g2s(buf, a.gq + r0 * qrow, G.a_q, &full[st]);
-          bulk_g2s(buf + G.a_q, a.gs + r0 * srow, G.a_sb, &full[st]);
-          if (F != kFmtMx) bulk_g2s(buf + G.a_q + G.a_sb, a.gb + r0 * srow, G.a_sb, &full[st]);
+          bulk_g2s_stream(buf, a.gq + r0 * qrow, G.a_q, &full[st]);
+          bulk_g2s_stream(buf + G.a_q, a.gs + r0 * srow, G.a_sb, &full[st]);
+          if (F != kFmtMx) bulk_g2s_stream(buf + G.a_q + G.a_sb, a.gb + r0 * srow, G.a_sb, &full[st]);
           buf += G.a_mat;
-          bulk_g2s(buf, a.uq + r0 * qrow, G.a_q, &full[st]);
-          bulk_g2s(buf + G.a_q, a.us + r0 * srow, G.a_sb, &full[st]);
-          if (F != kFmtMx) bulk_g2s(buf + G.a_q + G.a_sb, a.ub + r0 * srow, G.a_sb, &full[st]);
+          bulk_g2s_stream(buf, a.uq + r0 * qrow, G.a_q, &full[st]);
+          bulk_g2s_stream(buf + G.a_q, a.us + r0 * srow, G.a_sb, &full[st]);
+          if (F != kFmtMx) bulk_g2s_stream(buf + G.a_q + G.a_sb, a.ub + r0 * srow, G.a_sb, &full[st]);
         } else {
           const int nrows = min(G.rows_b, a.H - row0);
           const size_t r0 = (size_t)uniq[sb_slot[sg]] * a.H + row0;
           const size_t qrow = a.I / 8, srow = a.I / 64;
           const unsigned qb = nrows * (a.I / 2), sb = nrows * (a.I / 32);
           mbar_arrive_expect_tx(&full[st], qb + (F == kFmtMx ? 1 : 2) * sb);
-          bulk_g2s(buf, a.dq + r0 * qrow, qb, &full[st]);
-          bulk_g2s(buf + G.b_q, a.ds + r0 * srow, sb, &full[st]);
-          if (F != kFmtMx) bulk_g2s(buf + G.b_q + G.b_sb, a.db + r0 * srow, sb, &full[st]);
+          bulk_g2s_stream(buf, a.dq + r0 * qrow, qb, &full[st]);
+          bulk_g2s_stream(buf + G.b_q, a.ds + r0 * srow, sb, &full[st]);
+          if (F != kFmtMx) bulk_g2s_stream(buf + G.b_q + G.b_sb, a.db + r0 * srow, sb, &full[st]);
         }
       }
       __syncwarp();
@@ -1119,13 +1185,22 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
       return true;
     };
     const int sega = s_sega;
-    int nsets = 0;    // activation sets converted
+    int nsets = 0;    // all-warp meetings at set starts
+    int nteam = 0;    // this team's phase-B sets converted
     int handled = -1; // blocks up to here have had their set starts taken
-    // Every compute warp (both teams) takes every set start, in block order, before it
-    // computes a block at or after it: all warps meet at set_in (so every block of the
-    // previous set is done and the activation area is free), phase B waits (one
-    // thread, bounded) until every phase-A block of the expert has published its h
-    // rows, the compute threads convert the set, and all meet again at set_out.
+    // this team's phase-B set buffer: half the activation area
+    unsigned char* bset = actp + s_bbase + (size_t)tm * s_bhalf;
+    const bool bsep = s_bsep != 0;
+    // Set starts, in block order, before a block at or after them is computed.
+    // Phase A (x not resident): every compute warp takes it; all meet at set_in (the
+    // previous set's blocks are done, the area is free), the 512 compute threads
+    // convert the x rows into the area, and all meet at set_out.
+    // Phase B: each team keeps its own copy of the set's h rows in its half of the area,
+    // so the teams do not wait for each other; the first phase-B set start is also an
+    // all-warp meeting when the halves overlap the x rows or phase-A sets.  One thread
+    // per team waits (bounded, with back-off) until hdone[expert] counts every phase-A
+    // block of the expert, its acquire reaching the team's warps through team_in, then
+    // the team's 256 threads convert the rows and meet at team_out.
     auto take_sets = [&](int upto) -> bool {
       for (int b = handled + 1; b <= upto; ++b) {
         if (!set_start(b)) continue;
@@ -1134,10 +1209,21 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
         block_of(b, pb, sg, r0);
         const int nt = pb ? sb_nt[sg] : sa_nt[sg];
         const int p0 = pb ? sb_pos[sg] : sa_pos[sg];
-        // the poller's acquire reaches the other warps through set_in (release/acquire
-        // at CTA scope), so one thread per CTA loads the counter
+        if (!pb || (b == nA && !bsep)) {  // all-warp meeting
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&set_in[0]);
+          if (!wait_cons(&set_in[0], nsets & 1)) return false;
+          if (!pb) {
+            convert_set<F>(a, G, false, tok_of, p0, nt, actp, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&set_out[0]);
+            if (!wait_cons(&set_out[0], nsets & 1)) return false;
+          }
+          ++nsets;
+          if (!pb) continue;
+        }
         __syncwarp();
-        if (pb && warp == 0 && lane == 0) {
+        if (w == 0 && lane == 0) {
           const int slot = sb_slot[sg];
           const int n_i = offs[slot + 1] - offs[slot];
           const unsigned target = (unsigned)bpe_a * (unsigned)((n_i + sega - 1) / sega);
@@ -1151,13 +1237,13 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
           }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&set_in[0]);
-        if (!wait_cons(&set_in[0], nsets & 1)) return false;
-        convert_set<F>(a, G, pb, tok_of, p0, nt, actp, lane);
+        if (lane == 0) mbar_arrive(&team_in[tm]);
+        if (!wait_cons(&team_in[tm], nteam & 1)) return false;
+        convert_set<F>(a, G, true, tok_of, p0, nt, bset, lane, w * 32 + lane, kTeamWarps * 32);
         __syncwarp();
-        if (lane == 0) mbar_arrive(&set_out[0]);
-        if (!wait_cons(&set_out[0], nsets & 1)) return false;
-        ++nsets;
+        if (lane == 0) mbar_arrive(&team_out[tm]);
+        if (!wait_cons(&team_out[tm], nteam & 1)) return false;
+        ++nteam;
       }
       handled = upto;
       return true;
@@ -1215,7 +1301,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
         for (int c = 0; c < nt; ++c) {
           int vid;
           const float v = dispatch_b<1, F>(G.rounds_b, buf, bs, bb, w, nrows, a.I,
-                                           actp + (size_t)c * stride_b, stride_b, lane, vid);
+                                           bset + (size_t)c * stride_b, stride_b, lane, vid);
           if (vid >= 0) {
             const int r = w + kTeamWarps * (vid / kNT);
             if (r < nrows) a.y[(size_t)(p0 + c) * a.H + row0 + r] = v;
@@ -1266,7 +1352,8 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
           for (int j = gl; j < a.k; j += gk) {
             const int p = t * a.k + j;
             const int pos = pos_of[p];
-            if (pos >= 0) acc = fmaf(__ldg(a.w + p), __ldcg(a.y + (size_t)pos * a.H + c), acc);
+            if (pos >= 0)
+              acc = fmaf(routed ? rw[p] : __ldg(a.w + p), __ldcg(a.y + (size_t)pos * a.H + c), acc);
           }
         for (int m = gk >> 1; m >= 1; m >>= 1) acc += __shfl_xor_sync(kFull, acc, m);
         if (valid && gl == 0) a.out[(size_t)t * a.H + c] = float_to_bf16_bits(acc);

@@ -20,17 +20,12 @@ constexpr int kRouterWarps = 8;      // tokens per CTA
 constexpr int kRouterMaxE = 1024;    // experts (the library's limit)
 constexpr int kRouterMaxK = 32;      // picks per token: one lane each
 
-__global__ void __launch_bounds__(32 * kRouterWarps)
-    router_topk_kernel(const float* __restrict__ logits, int T, int E, int k, int renormalize,
-                       int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
-  __shared__ float s_val[kRouterWarps][kRouterMaxE];
-  __shared__ unsigned char s_taken[kRouterWarps][kRouterMaxE];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kRouterWarps + warp;
-  if (t >= T) return;  // warp-uniform
-  float* v = s_val[warp];
-  unsigned char* taken = s_taken[warp];
-  const float* row = logits + (size_t)t * E;
+// One token's picks by one warp: the row `row` (E logits, global) is staged in v / taken
+// (E floats and E bytes of this warp's scratch); lane j < k returns the j-th pick in
+// *idx (-1 if none) and its probability in *w.  Run by all 32 lanes.
+__device__ __forceinline__ void router_row(const float* __restrict__ row, int E, int k,
+                                           int renormalize, float* v, unsigned char* taken,
+                                           int lane, int* idx, float* w) {
   for (int e = lane; e < E; e += 32) {
     v[e] = __ldg(row + e);
     taken[e] = 0;
@@ -78,9 +73,26 @@ __global__ void __launch_bounds__(32 * kRouterWarps)
   }
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) denom += __shfl_xor_sync(kFull, denom, off);
+  *idx = my_idx;
+  *w = ex / denom;
+  __syncwarp();  // v and taken may be reused for the next row
+}
+
+__global__ void __launch_bounds__(32 * kRouterWarps)
+    router_topk_kernel(const float* __restrict__ logits, int T, int E, int k, int renormalize,
+                       int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  __shared__ float s_val[kRouterWarps][kRouterMaxE];
+  __shared__ unsigned char s_taken[kRouterWarps][kRouterMaxE];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kRouterWarps + warp;
+  if (t >= T) return;  // warp-uniform
+  int pi;
+  float pw;
+  router_row(logits + (size_t)t * E, E, k, renormalize, s_val[warp], s_taken[warp], lane, &pi,
+             &pw);
   if (lane < k) {
-    topk_idx[(size_t)t * k + lane] = my_idx;
-    topk_w[(size_t)t * k + lane] = ex / denom;
+    topk_idx[(size_t)t * k + lane] = pi;
+    topk_w[(size_t)t * k + lane] = pw;
   }
 }
 

@@ -13,6 +13,9 @@
 * Every token of the T=512 large window (grouped tensor-core path).
 * A bounded wait that runs out: the call reports MOE_ERR_TIMEOUT and returns, and the
   next call is correct again.
+* The router step fused into the layer (moe_switchglu_forward_routed): the same picks,
+  weights and output, bit for bit, as the router kernel followed by the layer, on the
+  persistent path and on the grouped path, and the oracle's router and layer.
 """
 import numpy as np
 import pytest
@@ -210,3 +213,57 @@ def test_bounded_wait_runs_out_and_next_call_is_clean():
     assert qeg.moe_read_device_status() == qeg.MOE_OK
     assert_parity(bf16_to_f64(out), oracle.switchglu(L.x, L.idx, L.w, L.bank, E),
                   "after a timeout")
+
+
+# ------------------------------------------------------ router fused with the layer ---
+@pytest.mark.parametrize("T,E,renorm", [(1, 288, True), (4, 288, True), (16, 288, False),
+                                        (64, 288, True)])
+def test_router_fused_into_the_layer(T, E, renorm):
+    """Logits -> picks -> layer in one launch, against the router kernel then the layer (bit
+    for bit: the same picks, weights and arithmetic) and against the oracle on sampled
+    tokens; ties in the logits (equal values, the lower id first) included."""
+    k, seed = 8, 4100 + T
+    rng = np.random.default_rng(seed)
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    lg[:, 5] = lg[:, 6] = lg[:, 200] = 3.0  # equal logits among the top picks
+    bank = dev_bank_drawn(E, H, I, seed)
+    x_bits = synth.x_bf16(T, H, seed)
+    x = bf16_tensor(x_bits)
+    lgd = torch.from_numpy(lg).cuda()
+    ws = qeg.moe_workspace(T, k, E, H, I)
+    out, idx, w = qeg.moe_switchglu_forward_routed(x, lgd, k, bank, renormalize=renorm,
+                                                   workspace=ws)
+    idx2, w2 = qeg.moe_router_topk(lgd, k, renormalize=renorm)
+    out2 = qeg.moe_switchglu_forward(x, idx2, w2, bank)
+    torch.cuda.synchronize()
+    assert qeg.moe_read_device_status() == qeg.MOE_OK
+    assert torch.equal(idx, idx2) and torch.equal(w, w2)
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+    ridx, rw = oracle.router_topk(lg, k, renormalize=renorm)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=2e-5, atol=0)
+    tokens = sample_tokens(T, 4, seed)
+    used = sorted(set(int(e) for e in ridx[tokens].ravel()))
+    hb = draw_bank(E, H, I, seed, used)
+    ref = oracle.switchglu(x_bits, ridx, rw.astype(np.float32), hb, E, tokens=tokens)
+    assert_parity(bf16_to_f64(out)[tokens], ref[tokens], f"router fused, T={T}")
+
+
+def test_router_fused_grouped_path():
+    """A window that takes the grouped path: the router kernel runs first, then the five
+    grouped launches; the picks and output equal the two-call sequence's bit for bit."""
+    T, k, E, Hs, Is = 160, 8, 64, 512, 256
+    assert qeg.moe_select_path(T, k, E, Hs, Is) == 2
+    L = make_layer(T, k, E, Hs, Is, 4300)
+    bank = to_dev_bank(L)
+    x, _, _ = to_dev_inputs(L)
+    lg = torch.from_numpy(np.random.default_rng(4301).standard_normal((T, E))
+                          .astype(np.float32)).cuda()
+    out, idx, w = qeg.moe_switchglu_forward_routed(x, lg, k, bank)
+    idx2, w2 = qeg.moe_router_topk(lg, k)
+    out2 = qeg.moe_switchglu_forward(x, idx2, w2, bank)
+    torch.cuda.synchronize()
+    assert qeg.moe_read_device_status() == qeg.MOE_OK
+    assert torch.equal(idx, idx2) and torch.equal(w, w2)
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+

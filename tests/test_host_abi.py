@@ -28,7 +28,8 @@ def test_header_declares_the_entry_points():
               "moe_select_path", "moe_workspace_layout", "moe_switchglu_forward_static",
               "moe_router_topk", "moe_switchglu_forward_mxfp4",
               "moe_switchglu_forward_mxfp4_ws", "moe_workspace_size_mxfp4",
-              "moe_select_path_mxfp4", "moe_set_wait_limit_ns"):
+              "moe_select_path_mxfp4", "moe_set_wait_limit_ns", "moe_switchglu_forward_routed",
+              "moe_switchglu_forward_routed_ws"):
         assert n in names
 
 
@@ -149,3 +150,15 @@ def test_validation_rejects_before_touching_memory():
     assert lib.moe_router_topk(fake, 4, 2048, 8, 1, fake, fake, None) == qeg.MOE_ERR_UNSUPPORTED
     assert lib.moe_router_topk(fake, 4, 64, 33, 1, fake, fake, None) == qeg.MOE_ERR_UNSUPPORTED
     assert lib.moe_router_topk(fake + 2, 4, 16, 2, 1, fake, fake, None) == qeg.MOE_ERR_UNSUPPORTED
+    # router fused with the layer: null logits, k > E, E over the router's limit,
+    # misaligned logits, too-small workspace
+    bank = [fake] * 9
+    def routed(logits, T, k, E, ws_bytes=1 << 30, out=fake, idx=fake, w=fake):
+        return lib.moe_switchglu_forward_routed_ws(fake, logits, 1, *bank, T, k, E, 128, 64, out,
+                                                   idx, w, fake, ws_bytes, None)
+    assert routed(None, 2, 2, 4) == qeg.MOE_ERR_INVALID_ARG
+    assert routed(fake, 2, 2, 4, idx=None) == qeg.MOE_ERR_INVALID_ARG
+    assert routed(fake, 2, 5, 4) == qeg.MOE_ERR_INVALID_ARG
+    assert routed(fake, 2, 2, 2000) == qeg.MOE_ERR_UNSUPPORTED
+    assert routed(fake + 2, 2, 2, 4) == qeg.MOE_ERR_UNSUPPORTED
+    assert routed(fake, 2, 2, 4, ws_bytes=16) == qeg.MOE_ERR_WORKSPACE
