@@ -1009,20 +1009,21 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
   const int a0 = s_rng[0], a2 = s_rng[2], b0 = s_rng[4], b2 = s_rng[6];
   const int nA1 = s_rng[1] - a0, nA = nA1 + (s_rng[3] - a2);
   const int nB1 = s_rng[5] - b0, nblk = nA + nB1 + (s_rng[7] - b2);
-  // blk / bpe as a multiply-high: m = ceil(2^40 / bpe) is exact for blk * bpe < 2^40
-  const unsigned long long mag_a = ((1ull << 40) + bpe_a - 1) / bpe_a;
-  const unsigned long long mag_b = ((1ull << 40) + bpe_b - 1) / bpe_b;
+  // blk / bpe as a multiply-high by m = ceil(2^32 / bpe), exact while blk * bpe < 2^32
+  // (here blk < 2^20 and 2 <= bpe <= 2^10)
+  const unsigned mag_a = 0xFFFFFFFFu / (unsigned)bpe_a + 1u;
+  const unsigned mag_b = 0xFFFFFFFFu / (unsigned)bpe_b + 1u;
   auto block_of = [&](int j, bool& pb, int& sg, int& row0) {
     if (j < nA) {
       const int blk = j < nA1 ? a0 + j : a2 + (j - nA1);
       pb = false;
-      sg = (int)(((unsigned long long)blk * mag_a) >> 40);
+      sg = (int)__umulhi((unsigned)blk, mag_a);
       row0 = (blk - sg * bpe_a) * kRowsA;
     } else {
       const int jb = j - nA;
       const int blk = jb < nB1 ? b0 + jb : b2 + (jb - nB1);
       pb = true;
-      sg = (int)(((unsigned long long)blk * mag_b) >> 40);
+      sg = (int)__umulhi((unsigned)blk, mag_b);
       row0 = (blk - sg * bpe_b) * G.rows_b;
     }
   };
