@@ -820,8 +820,10 @@ __device__ __forceinline__ int plan_shares(const int* sa_slot, const int* sa_nt,
 }
 
 // 18 warps: 16 compute warps (two teams), a producer warp and a helper warp (see the top
-// of this file).
-template <int F>
+// of this file).  RA / RB: the chunk rounds of phase A / B fixed at compile time (the
+// widths the launch sees most, 4096 / 2048: 4 / 2), or 0 for any width (a run-time
+// switch over the instances); the fixed instances carry only the code the width uses.
+template <int F, int RA = 0, int RB = 0>
 __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   // window plan, set by warp 0 after the union: segments of phase A and B, ring depth,
@@ -1284,8 +1286,13 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
             arow[t] = x_res ? actp + tok_of[p0 + q] * stride_a : actp + q * stride_a;
           }
           float Gs[kNT], Us[kNT];
-          if (ntc == 2) dispatch_a<2, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
-          else dispatch_a<1, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
+          if constexpr (RA > 0) {
+            if (ntc == 2) rows_a<2, RA, F>(bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
+            else rows_a<1, RA, F>(bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
+          } else {
+            if (ntc == 2) dispatch_a<2, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
+            else dispatch_a<1, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
+          }
           if (lane < ntc) {
             const float g = round_to_bf16(lane == 0 ? Gs[0] : Gs[1]);
             const float hu = round_to_bf16(lane == 0 ? Us[0] : Us[1]);
@@ -1301,8 +1308,13 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
         const uint16_t* bb = reinterpret_cast<const uint16_t*>(buf + G.b_q + G.b_sb);
         for (int c = 0; c < nt; ++c) {
           int vid;
-          const float v = dispatch_b<1, F>(G.rounds_b, buf, bs, bb, w, nrows, a.I,
-                                           bset + (size_t)c * stride_b, stride_b, lane, vid);
+          float v;
+          if constexpr (RB > 0)
+            v = rows_b<1, RB, F>(buf, bs, bb, w, nrows, a.I, bset + (size_t)c * stride_b,
+                                 stride_b, lane, vid);
+          else
+            v = dispatch_b<1, F>(G.rounds_b, buf, bs, bb, w, nrows, a.I,
+                                 bset + (size_t)c * stride_b, stride_b, lane, vid);
           if (vid >= 0) {
             const int r = w + kTeamWarps * (vid / kNT);
             if (r < nrows) a.y[(size_t)(p0 + c) * a.H + row0 + r] = v;
