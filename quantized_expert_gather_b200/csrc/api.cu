@@ -26,8 +26,9 @@ struct DeviceInfo {
   // dynamic shared memory limit: layer (affine), route_union, grouped gate+up and down
   // (chunks of 64 pairs), combine, grouped gate+up and down (chunks of 96, then of 32
   // pairs), layer (mxfp4); then the layer instances for fixed widths (affine 4096/2048,
-  // mxfp4 6144/2048 and 4096/2048), which share the general instances' limits
-  int dyn_smem[13] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
+  // mxfp4 6144/2048 and 4096/2048, each also with resident x rows), which share the
+  // general instances' limits
+  int dyn_smem[16] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
 };
 
 DeviceInfo g_dev[kMaxDevices];
@@ -53,7 +54,7 @@ moe_status device_info(DeviceInfo** out) {
       e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return cuda_fail(e);
     // dynamic + static shared memory may not exceed the opt-in limit
-    const void* kernels[13] = {reinterpret_cast<const void*>(layer_kernel<kFmtAffine>),
+    const void* kernels[16] = {reinterpret_cast<const void*>(layer_kernel<kFmtAffine>),
                               reinterpret_cast<const void*>(route_union_kernel),
                               reinterpret_cast<const void*>(grouped_gemm_kernel<0, 64>),
                               reinterpret_cast<const void*>(grouped_gemm_kernel<1, 64>),
@@ -65,8 +66,11 @@ moe_status device_info(DeviceInfo** out) {
                               reinterpret_cast<const void*>(layer_kernel<kFmtMx>),
                               reinterpret_cast<const void*>(layer_kernel<kFmtAffine, 4, 2>),
                               reinterpret_cast<const void*>(layer_kernel<kFmtMx, 6, 2>),
-                              reinterpret_cast<const void*>(layer_kernel<kFmtMx, 4, 2>)};
-    for (int i = 0; i < 13; ++i) {
+                              reinterpret_cast<const void*>(layer_kernel<kFmtMx, 4, 2>),
+                              reinterpret_cast<const void*>(layer_kernel<kFmtAffine, 4, 2, 1>),
+                              reinterpret_cast<const void*>(layer_kernel<kFmtMx, 6, 2, 1>),
+                              reinterpret_cast<const void*>(layer_kernel<kFmtMx, 4, 2, 1>)};
+    for (int i = 0; i < 16; ++i) {
       cudaFuncAttributes fa;
       cudaError_t e = cudaFuncGetAttributes(&fa, kernels[i]);
       if (e == cudaSuccess) {
@@ -217,10 +221,15 @@ cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
   c.attrs = attr;
   c.numAttrs = 2;
   // the instance with the chunk rounds fixed, for the widths that have one
+  // (and x resident: the instance without phase-A activation sets)
   const int ra = a.g.rounds_a, rb = a.g.rounds_b;
-  if (ra == 4 && rb == 2) return cudaLaunchKernelEx(&c, layer_kernel<F, 4, 2>, a);
+  if (ra == 4 && rb == 2)
+    return a.x_res ? cudaLaunchKernelEx(&c, layer_kernel<F, 4, 2, 1>, a)
+                   : cudaLaunchKernelEx(&c, layer_kernel<F, 4, 2>, a);
   if constexpr (F == kFmtMx) {
-    if (ra == 6 && rb == 2) return cudaLaunchKernelEx(&c, layer_kernel<F, 6, 2>, a);
+    if (ra == 6 && rb == 2)
+      return a.x_res ? cudaLaunchKernelEx(&c, layer_kernel<F, 6, 2, 1>, a)
+                     : cudaLaunchKernelEx(&c, layer_kernel<F, 6, 2>, a);
   }
   return cudaLaunchKernelEx(&c, layer_kernel<F>, a);
 }

@@ -822,8 +822,10 @@ __device__ __forceinline__ int plan_shares(const int* sa_slot, const int* sa_nt,
 // 18 warps: 16 compute warps (two teams), a producer warp and a helper warp (see the top
 // of this file).  RA / RB: the chunk rounds of phase A / B fixed at compile time (the
 // widths the launch sees most, 4096 / 2048: 4 / 2), or 0 for any width (a run-time
-// switch over the instances); the fixed instances carry only the code the width uses.
-template <int F, int RA = 0, int RB = 0>
+// switch over the instances); XR = 1: the window's x rows are resident (the launch's
+// x_res), so phase A has no activation sets, or -1: decided per window.  The fixed
+// instances carry only the code their windows use.
+template <int F, int RA = 0, int RB = 0, int XR = -1>
 __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   // window plan, set by warp 0 after the union: segments of phase A and B, ring depth,
@@ -974,7 +976,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
     named_barrier(kBarUnion, 64);  // the plan is made
   }
   const int u = s_u, nsb = s_nsb, NS = s_ns;
-  const bool x_res = s_xres != 0;
+  const bool x_res = XR == 1 ? true : s_xres != 0;
   unsigned char* actp = smem + s_act_off;  // activation area (resident x rows first)
   const int n_valid = offs[u];
   if (warp != kWarps) {
@@ -1212,18 +1214,24 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
         block_of(b, pb, sg, r0);
         const int nt = pb ? sb_nt[sg] : sa_nt[sg];
         const int p0 = pb ? sb_pos[sg] : sa_pos[sg];
-        if (!pb || (b == nA && !bsep)) {  // all-warp meeting
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&set_in[0]);
-          if (!wait_cons(&set_in[0], nsets & 1)) return false;
-          if (!pb) {
+        if constexpr (XR != 1) {
+          if (!pb) {  // phase-A set (x not resident): all-warp meeting and conversion
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&set_in[0]);
+            if (!wait_cons(&set_in[0], nsets & 1)) return false;
             convert_set<F>(a, G, false, tok_of, p0, nt, actp, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&set_out[0]);
             if (!wait_cons(&set_out[0], nsets & 1)) return false;
+            ++nsets;
+            continue;
           }
+        }
+        if (b == nA && !bsep) {  // the turn to phase B over the x rows: all-warp meeting
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&set_in[0]);
+          if (!wait_cons(&set_in[0], nsets & 1)) return false;
           ++nsets;
-          if (!pb) continue;
         }
         __syncwarp();
         if (w == 0 && lane == 0) {
