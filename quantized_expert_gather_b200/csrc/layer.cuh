@@ -1259,84 +1259,109 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const LayerArgs a) {
       handled = upto;
       return true;
     };
-    for (int j = tm;; j += kTeams) {
-      if (j >= nblk) {
-        take_sets(nblk - 1);  // the set starts past this team's last block
-        break;
-      }
-      if (!take_sets(j)) break;
-      const int st = j % NS;
-      if (!wait_cons(&full[st], (j / NS) & 1)) break;
-      bool phase_b;
-      int sg, row0;
-      block_of(j, phase_b, sg, row0);
-      const int nt = phase_b ? sb_nt[sg] : sa_nt[sg];
-      const int p0 = phase_b ? sb_pos[sg] : sa_pos[sg];
-      const unsigned char* buf = ring + (size_t)st * G.stage_bytes;
-      // the segment's pairs one at a time, the block's weights read again per pair
-      if (!phase_b) {
-        const unsigned char* bgq = buf + (size_t)w * (a.H / 2);
-        const uint16_t* bgs = reinterpret_cast<const uint16_t*>(buf + G.a_q) + w * (a.H / 64);
-        const uint16_t* bgb = reinterpret_cast<const uint16_t*>(buf + G.a_q + G.a_sb) + w * (a.H / 64);
-        const unsigned char* bu = buf + G.a_mat;
-        const unsigned char* buq = bu + (size_t)w * (a.H / 2);
-        const uint16_t* bus = reinterpret_cast<const uint16_t*>(bu + G.a_q) + w * (a.H / 64);
-        const uint16_t* bub = reinterpret_cast<const uint16_t*>(bu + G.a_q + G.a_sb) + w * (a.H / 64);
-        // the segment's pairs two at a time (the codes split once for both), the last
-        // one alone
-        for (int c = 0; c < nt; c += kNT) {
-          const int ntc = min(kNT, nt - c);
-          // each pair's activation row: the token's resident x row, or its row of the set
-          const unsigned char* arow[kNT];
-#pragma unroll
-          for (int t = 0; t < kNT; ++t) {
-            const int q = c + (t < ntc ? t : 0);
-            arow[t] = x_res ? actp + tok_of[p0 + q] * stride_a : actp + q * stride_a;
-          }
-          float Gs[kNT], Us[kNT];
-          if constexpr (RA > 0) {
-            if (ntc == 2) rows_a<2, RA, F>(bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
-            else rows_a<1, RA, F>(bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
-          } else {
-            if (ntc == 2) dispatch_a<2, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
-            else dispatch_a<1, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
-          }
-          if (lane < ntc) {
-            const float g = round_to_bf16(lane == 0 ? Gs[0] : Gs[1]);
-            const float hu = round_to_bf16(lane == 0 ? Us[0] : Us[1]);
-            // silu(g) = g / (1 + e^-g); the fast division's error (2 ulp of fp32) is far
-            // below the bf16 step h is rounded to
-            a.h[(size_t)(p0 + c + lane) * a.I + row0 + w] =
-                float_to_bf16_bits(__fdividef(g, 1.0f + __expf(-g)) * hu);
-          }
-        }
-      } else {
-        const int nrows = min(G.rows_b, a.H - row0);
-        const uint16_t* bs = reinterpret_cast<const uint16_t*>(buf + G.b_q);
-        const uint16_t* bb = reinterpret_cast<const uint16_t*>(buf + G.b_q + G.b_sb);
-        for (int c = 0; c < nt; ++c) {
-          int vid;
-          float v;
-          if constexpr (RB > 0)
-            v = rows_b<1, RB, F>(buf, bs, bb, w, nrows, a.I, bset + (size_t)c * stride_b,
-                                 stride_b, lane, vid);
-          else
-            v = dispatch_b<1, F>(G.rounds_b, buf, bs, bb, w, nrows, a.I,
-                                 bset + (size_t)c * stride_b, stride_b, lane, vid);
-          if (vid >= 0) {
-            const int r = w + kTeamWarps * (vid / kNT);
-            if (r < nrows) a.y[(size_t)(p0 + c) * a.H + row0 + r] = v;
-          }
-        }
-      }
-      // this warp is done reading stage st, and its outputs of block j are written
-      // (released at CTA scope)
+    // this warp is done reading stage st, and its outputs of block jb are written
+    // (released at CTA scope)
+    auto finish = [&](int st, int jb) {
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&empty[st]);
-        mbar_arrive(&done[j % kPubRing]);
+        mbar_arrive(&done[jb % kPubRing]);
       }
+    };
+    // the phase-A blocks, then the phase-B blocks, in two loops (each loop's code holds
+    // only its phase's core)
+    int j = tm;
+    bool go = true;
+    for (; j < nA; j += kTeams) {
+      if (!take_sets(j)) {
+        go = false;
+        break;
+      }
+      const int st = j % NS;
+      if (!wait_cons(&full[st], (j / NS) & 1)) {
+        go = false;
+        break;
+      }
+      bool phase_b;
+      int sg, row0;
+      block_of(j, phase_b, sg, row0);
+      const int nt = sa_nt[sg];
+      const int p0 = sa_pos[sg];
+      const unsigned char* buf = ring + (size_t)st * G.stage_bytes;
+      const unsigned char* bgq = buf + (size_t)w * (a.H / 2);
+      const uint16_t* bgs = reinterpret_cast<const uint16_t*>(buf + G.a_q) + w * (a.H / 64);
+      const uint16_t* bgb = reinterpret_cast<const uint16_t*>(buf + G.a_q + G.a_sb) + w * (a.H / 64);
+      const unsigned char* bu = buf + G.a_mat;
+      const unsigned char* buq = bu + (size_t)w * (a.H / 2);
+      const uint16_t* bus = reinterpret_cast<const uint16_t*>(bu + G.a_q) + w * (a.H / 64);
+      const uint16_t* bub = reinterpret_cast<const uint16_t*>(bu + G.a_q + G.a_sb) + w * (a.H / 64);
+      // the segment's pairs two at a time (the codes split once for both), the last one
+      // alone; the block's weights read again per pass
+      for (int c = 0; c < nt; c += kNT) {
+        const int ntc = min(kNT, nt - c);
+        // each pair's activation row: the token's resident x row, or its row of the set
+        const unsigned char* arow[kNT];
+#pragma unroll
+        for (int t = 0; t < kNT; ++t) {
+          const int q = c + (t < ntc ? t : 0);
+          arow[t] = x_res ? actp + tok_of[p0 + q] * stride_a : actp + q * stride_a;
+        }
+        float Gs[kNT], Us[kNT];
+        if constexpr (RA > 0) {
+          if (ntc == 2) rows_a<2, RA, F>(bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
+          else rows_a<1, RA, F>(bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
+        } else {
+          if (ntc == 2) dispatch_a<2, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
+          else dispatch_a<1, F>(G.rounds_a, bgq, bgs, bgb, buq, bus, bub, a.H, arow, lane, Gs, Us);
+        }
+        if (lane < ntc) {
+          const float g = round_to_bf16(lane == 0 ? Gs[0] : Gs[1]);
+          const float hu = round_to_bf16(lane == 0 ? Us[0] : Us[1]);
+          // silu(g) = g / (1 + e^-g); the fast division's error (2 ulp of fp32) is far
+          // below the bf16 step h is rounded to
+          a.h[(size_t)(p0 + c + lane) * a.I + row0 + w] =
+              float_to_bf16_bits(__fdividef(g, 1.0f + __expf(-g)) * hu);
+        }
+      }
+      finish(st, j);
     }
+    for (; go && j < nblk; j += kTeams) {
+      if (!take_sets(j)) {
+        go = false;
+        break;
+      }
+      const int st = j % NS;
+      if (!wait_cons(&full[st], (j / NS) & 1)) {
+        go = false;
+        break;
+      }
+      bool phase_b;
+      int sg, row0;
+      block_of(j, phase_b, sg, row0);
+      const int nt = sb_nt[sg];
+      const int p0 = sb_pos[sg];
+      const unsigned char* buf = ring + (size_t)st * G.stage_bytes;
+      const int nrows = min(G.rows_b, a.H - row0);
+      const uint16_t* bs = reinterpret_cast<const uint16_t*>(buf + G.b_q);
+      const uint16_t* bb = reinterpret_cast<const uint16_t*>(buf + G.b_q + G.b_sb);
+      // the segment's pairs one at a time, the block's weights read again per pair
+      for (int c = 0; c < nt; ++c) {
+        int vid;
+        float v;
+        if constexpr (RB > 0)
+          v = rows_b<1, RB, F>(buf, bs, bb, w, nrows, a.I, bset + (size_t)c * stride_b,
+                               stride_b, lane, vid);
+        else
+          v = dispatch_b<1, F>(G.rounds_b, buf, bs, bb, w, nrows, a.I,
+                               bset + (size_t)c * stride_b, stride_b, lane, vid);
+        if (vid >= 0) {
+          const int r = w + kTeamWarps * (vid / kNT);
+          if (r < nrows) a.y[(size_t)(p0 + c) * a.H + row0 + r] = v;
+        }
+      }
+      finish(st, j);
+    }
+    if (go) take_sets(nblk - 1);  // the set starts past this team's last block
   }
 
   // ---- combine: row blocks blockIdx.x, blockIdx.x + grid, ... once complete ----
