@@ -267,3 +267,15 @@ def test_router_fused_grouped_path():
     assert torch.equal(idx, idx2) and torch.equal(w, w2)
     assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
 
+
+def test_one_token_with_repeated_experts_full_width():
+    """A one-token window whose row names some experts more than once (segments of two
+    and three pairs) at hidden 4096 / inter 2048: the one-token instance runs such a
+    segment one pair per pass."""
+    E, seed = 288, 4400
+    idx = np.array([[5, 5, 17, 17, 17, 40, 41, 287]], np.int32)
+    w = np.array([[0.2, 0.1, 0.15, 0.05, 0.1, 0.2, 0.1, 0.1]], np.float32)
+    bank = dev_bank_drawn(E, H, I, seed)
+    x_bits = synth.x_bf16(1, H, seed)
+    check_sampled(x_bits, idx, w, bank, E, seed, [0], "one token, repeated experts")
+
