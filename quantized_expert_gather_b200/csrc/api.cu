@@ -370,7 +370,7 @@ moe_status owned_workspace(int T, int k, int E, int hidden, int inter, int fmt, 
 
 // Fixed scratch for moe_switchglu_forward_static: one copy per device, in the
 // module's global memory (zero at module load), so that entry never allocates.
-// 4 MiB covers T*k <= 128 pairs at hidden 4096 / inter 2048 (3,366,912 bytes
+// 4 MiB covers T*k <= 128 pairs at hidden 4096 / inter 2048 (2,629,632 bytes
 // at T=16, k=8) and every smaller layer.
 constexpr size_t kStaticScratchBytes = MOE_STATIC_SCRATCH_BYTES;
 static_assert(kSyncWords == 1539, "the header states the counter region as 4*1539 bytes");
