@@ -726,15 +726,29 @@ __device__ __forceinline__ int make_segments(const int* offs, int u, int seg, in
   return base;
 }
 
+// Cost of one block of a segment of nt pairs, in units of about 10 ns of a team's time
+// (fitted to per-block timings on B200 at hidden 4096 / inter 2048): phase A runs its
+// pairs two per pass over the block's codes, phase B one per pass.  Only costs within
+// one phase are compared with each other.
+__device__ __forceinline__ unsigned block_cost(bool phase_b, int nt) {
+  return phase_b ? 36u + 119u * (unsigned)nt
+                 : 26u + 73u * (unsigned)nt + 64u * (unsigned)((nt + 1) >> 1);
+}
+// A CTA whose share of a phase-B range crosses a segment start converts one more
+// activation set than the others: about 2.5 us for each team, both teams at once, in
+// the units of the summed block costs of both teams.  Half of it is charged to the
+// segment's first block and half to its last, so that a share that starts or ends at
+// a segment start, and converts nothing extra, is charged half.
+constexpr unsigned kSetCost = 500u;
+
 // Inclusive prefix of the segments' costs, pref[s] = sum over segments s' <= s of
-// bpe (2 + nt[s']): a block's weight bytes are the same for every segment, and its
-// compute is about two pairs' worth of fixed work plus one per pair.  Run by one warp.
-__device__ __forceinline__ unsigned prefix_costs(const int* nt, int nseg, int bpe, unsigned* pref,
-                                                 int lane) {
+// bpe block_cost(nt[s']) + sig.  Run by one warp.
+__device__ __forceinline__ unsigned prefix_costs(const int* nt, int nseg, int bpe, bool phase_b,
+                                                 unsigned sig, unsigned* pref, int lane) {
   unsigned base = 0;
   for (int b0 = 0; b0 < nseg; b0 += 32) {
     const int sidx = b0 + lane;
-    const unsigned c = sidx < nseg ? (unsigned)bpe * (2u + (unsigned)nt[sidx]) : 0u;
+    const unsigned c = sidx < nseg ? (unsigned)bpe * block_cost(phase_b, nt[sidx]) + sig : 0u;
     unsigned incl = c;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -747,10 +761,20 @@ __device__ __forceinline__ unsigned prefix_costs(const int* nt, int nseg, int bp
   return base;
 }
 
-// First block (global index, segments in order, bpe blocks each) of segments [s0, s1)
-// at which the cost prefix reaches t: the start of a CTA's share.  One thread.
+// Cost of the blocks before block b (global index, segments in order, bpe blocks each):
+// a segment's first block carries sig / 2 more, its last block the rest of sig.  One
+// thread.
+__device__ __forceinline__ unsigned cost_before(const unsigned* pref, const int* nt, int b, int bpe,
+                                                bool phase_b, unsigned sig) {
+  const int sg = b / bpe, i = b - sg * bpe;
+  const unsigned before = sg > 0 ? pref[sg - 1] : 0u;
+  return i == 0 ? before : before + sig / 2u + (unsigned)i * block_cost(phase_b, nt[sg]);
+}
+
+// First block (global index) of segments [s0, s1) whose cost_before reaches t: the
+// start of a CTA's share.  One thread.
 __device__ __forceinline__ int block_at(const unsigned* pref, const int* nt, int s0, int s1,
-                                        int bpe, unsigned t) {
+                                        int bpe, unsigned t, bool phase_b, unsigned sig) {
   const unsigned before0 = s0 > 0 ? pref[s0 - 1] : 0u;
   if (t <= before0) return s0 * bpe;
   if (s1 <= s0 || t > pref[s1 - 1]) return s1 * bpe;
@@ -760,25 +784,32 @@ __device__ __forceinline__ int block_at(const unsigned* pref, const int* nt, int
     if (pref[mid] >= t) hi = mid;
     else lo = mid + 1;
   }
-  const unsigned before = lo > 0 ? pref[lo - 1] : 0u, w = 2u + (unsigned)nt[lo];
-  return lo * bpe + (int)((t - before + w - 1) / w);
+  const unsigned before = lo > 0 ? pref[lo - 1] : 0u, w = block_cost(phase_b, nt[lo]);
+  const unsigned d = t - before, h = sig / 2u;  // 0 < d <= sig + bpe w
+  return lo * bpe + (d <= h + w ? 1 : min(bpe, (int)((d - h + w - 1) / w)));
 }
 
 // This CTA's block ranges, r0..r7 (lane q returns rq): phase A group 1 [r0, r1) and
-// group 2 [r2, r3), phase B group 1 [r4, r5) and group 2 [r6, r7), each a
-// cost-balanced share (blockIdx of gridDim) of its group's blocks.  Group 1 is the
-// experts up to the one holding the middle of the phase-A cost, group 2 the rest.  A
-// CTA streams its phase-A share of group 1, then of group 2, then its phase-B share
-// of group 1, then of group 2: by the time it reaches group 1's phase B, every CTA
-// has long finished group 1's phase A (nobody waits for h at the turn from A to B),
-// and group 2's phase A finishes while the CTAs stream group 1's phase B.  Run by
-// one warp; prefA / prefB are scratch for nsa / nsb unsigned.
+// group 2 [r2, r3), phase B group 1 [r4, r5) and group 2 [r6, r7), each a share of its
+// group's blocks, the shares in blockIdx order.  Group 1 is the experts up to the one
+// holding the middle of the phase-A cost, group 2 the rest.  A CTA streams its phase-A
+// share of group 1, then of group 2, then its phase-B share of group 1, then of group
+// 2: by the time it reaches group 1's phase B, every CTA has long finished group 1's
+// phase A (nobody waits for h at the turn from A to B), and group 2's phase A finishes
+// while the CTAs stream group 1's phase B.
+// Each range is cut where its cost prefix reaches a CTA's ideal share, corrected by the
+// cost the ranges cut before it gave the CTAs before this one beyond their ideal (the
+// rounding error carried from range to range): a CTA's total stays within about a block
+// of the mean instead of collecting the rounding of all four ranges.  The correction is
+// at most half of a CTA's ideal share of the range, which keeps the cuts in blockIdx
+// order.  Lanes 0 and 1 cut at blockIdx and blockIdx + 1.  Run by one warp; prefA /
+// prefB are scratch for nsa / nsb unsigned.
 __device__ __forceinline__ int plan_shares(const int* sa_slot, const int* sa_nt, int nsa,
                                            int bpe_a, const int* sb_slot, const int* sb_nt,
-                                           int nsb, int bpe_b, unsigned* prefA,
-                                           unsigned* prefB, int lane) {
-  const unsigned totA = prefix_costs(sa_nt, nsa, bpe_a, prefA, lane);
-  const unsigned totB = prefix_costs(sb_nt, nsb, bpe_b, prefB, lane);
+                                           int nsb, int bpe_b, unsigned* prefA, unsigned* prefB,
+                                           int lane) {
+  const unsigned totA = prefix_costs(sa_nt, nsa, bpe_a, false, 0u, prefA, lane);
+  const unsigned totB = prefix_costs(sb_nt, nsb, bpe_b, true, kSetCost, prefB, lane);
   __syncwarp();
   // group 1: phase-A segments up to the one holding the middle of the cost, and the
   // phase-B segments of the same experts
@@ -801,20 +832,36 @@ __device__ __forceinline__ int plan_shares(const int* sa_slot, const int* sa_nt,
       break;
     }
   }
-  // lane q < 8: target q = phase (q >> 2), group ((q >> 1) & 1), bound (q & 1)
+  int cut[4] = {0, 0, 0, 0};  // range q = 2 phase + group: A1, A2, B1, B2
+  if (lane < 2) {
+    const unsigned long long k = blockIdx.x + (unsigned)lane, G = gridDim.x;
+    long long err = 0;  // cost the ranges cut so far gave CTAs 0 .. k-1 beyond their ideal
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int q = (i + 2) & 3;  // B1, B2, A1, A2
+      const bool pb = q >= 2;
+      const int g = q & 1;
+      const unsigned* pref = pb ? prefB : prefA;
+      const int* nt = pb ? sb_nt : sa_nt;
+      const int n1 = pb ? nsb1 : nsa1, n = pb ? nsb : nsa, bpe = pb ? bpe_b : bpe_a;
+      const unsigned tot = pb ? totB : totA, sig = pb ? kSetCost : 0u;
+      const unsigned c1 = n1 > 0 ? pref[n1 - 1] : 0u;
+      const unsigned base = g ? c1 : 0u, cg = g ? tot - c1 : c1;
+      const long long ideal = (long long)base + (long long)((unsigned long long)cg * k / G);
+      const long long lim = (long long)((unsigned long long)cg / (2ull * G));
+      const long long t = ideal - max(-lim, min(lim, err));
+      const int s0 = g ? n1 : 0, s1 = g ? n : n1;
+      const int c = block_at(pref, nt, s0, s1, bpe, (unsigned)t, pb, sig);
+      err += (long long)cost_before(pref, nt, c, bpe, pb, sig) - ideal;
+      cut[q] = c;
+    }
+  }
+  // lane q < 8 returns the cut of range q >> 1 at bound q & 1
   int r = 0;
-  if (lane < 8) {
-    const bool pb = lane >= 4;
-    const int g = (lane >> 1) & 1;
-    const unsigned* pref = pb ? prefB : prefA;
-    const int* nt = pb ? sb_nt : sa_nt;
-    const int n1 = pb ? nsb1 : nsa1, n = pb ? nsb : nsa, bpe = pb ? bpe_b : bpe_a;
-    const unsigned tot = pb ? totB : totA;
-    const unsigned c1 = n1 > 0 ? pref[n1 - 1] : 0u;
-    const unsigned base = g ? c1 : 0u, cg = g ? tot - c1 : c1;
-    const unsigned k = blockIdx.x + (unsigned)(lane & 1);
-    const unsigned t = base + cg * k / gridDim.x;
-    r = g ? block_at(pref, nt, n1, n, bpe, t) : block_at(pref, nt, 0, n1, bpe, t);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int v = __shfl_sync(kFull, cut[q], lane & 1);
+    if ((lane >> 1) == q) r = v;
   }
   return r;
 }
