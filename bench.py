@@ -696,6 +696,37 @@ def our_arm(args, world, rank, local):
             mxfp4["per_T"][str(TM)] = {"us_per_layer": us, "mean_unique": um, "gbs": gb,
                                        "frac_of_hbm_peak": gb / measured_peaks()[0]}
             del wsm
+        # a large window on the same bank: T=512, uniform top-8 routing (every expert
+        # used), the grouped tensor-core path; 3 layers between CUDA events after a warm
+        # pass; bytes = unique experts, flops = 6 P H I
+        if not args.no_large_t:
+            TL, nl = 512, 3
+            rl = [synth.route_uniform(TL, EM, K_TOP, SEED + 7900 + l) for l in range(nl)]
+            xl = torch.from_numpy(synth.x_bf16(TL, HM, SEED + 79).view(np.int16)).to(dev) \
+                .view(torch.bfloat16)
+            il = [torch.from_numpy(r[0]).to(dev) for r in rl]
+            wl = [torch.from_numpy(r[1]).to(dev) for r in rl]
+            ol = torch.empty((TL, HM), dtype=torch.bfloat16, device=dev)
+            wsl = torch.zeros(qeg.moe_workspace_size_mxfp4(TL, K_TOP, EM, HM, IM),
+                              dtype=torch.uint8, device=dev)
+            for l in range(nl):  # warm
+                qeg.moe_switchglu_forward_mxfp4_ws(xl, il[l], wl[l], bank_mx, wsl, out=ol)
+            torch.cuda.synchronize()
+            a5, b5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a5.record()
+            for l in range(nl):
+                qeg.moe_switchglu_forward_mxfp4_ws(xl, il[l], wl[l], bank_mx, wsl, out=ol)
+            b5.record()
+            torch.cuda.synchronize()
+            us = a5.elapsed_time(b5) * 1e3 / nl
+            ul = float(np.mean([np.unique(r[0]).size for r in rl]))
+            gbl = ul * bpe_mx / (us * 1e-6) / 1e9
+            mxfp4["large_window"] = {
+                "T": TL, "us_per_layer": us, "mean_unique": ul, "gbs": gbl,
+                "frac_of_hbm_peak": gbl / measured_peaks()[0],
+                "tflops": 6.0 * TL * K_TOP * HM * IM / (us * 1e-6) / 1e12,
+                "path": "grouped tcgen05 kernels (5 launches per layer)"}
+            del wsl
         del bank_mx
         torch.cuda.synchronize()
         torch.cuda.empty_cache()

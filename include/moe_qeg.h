@@ -63,7 +63,7 @@ typedef enum {
 } moe_status;
 
 /* Supported range (checked on the host; violations return MOE_ERR_UNSUPPORTED):
- * hidden and inter multiples of 64, hidden <= 4096, inter <= 8192; E <= 1024;
+ * hidden and inter multiples of 64, hidden <= 8192, inter <= 8192; E <= 1024;
  * T*k <= 65536.  Windows of more than 1024 pairs (or whose persistent-kernel
  * plan does not fit) take the grouped tensor-core path, which further needs
  * hidden a multiple of 256, inter a multiple of 128 and T*k <= 57856 (its
@@ -187,8 +187,11 @@ moe_status moe_switchglu_forward_static(const uint16_t* x, const int32_t* topk_i
  * Gate and up: rows = inter, cols = hidden; down: rows = hidden, cols = inter.
  * Everything else (x, topk_idx, topk_w, out, workspace rules, errors, capture)
  * is as for moe_switchglu_forward_ws / moe_switchglu_forward, with the workspace
- * sized by moe_workspace_size_mxfp4.  Windows the persistent small-window kernel
- * cannot hold (moe_select_path_mxfp4 returns 0) give MOE_ERR_UNSUPPORTED.
+ * sized by moe_workspace_size_mxfp4.  Small windows take the persistent kernel,
+ * larger ones the grouped tensor-core path (moe_select_path_mxfp4 returns 1 or 2,
+ * under the same shape rules as the affine format); a shape neither takes
+ * (moe_select_path_mxfp4 returns 0) gives MOE_ERR_UNSUPPORTED.  On the grouped
+ * path each weight e2m1(q) 2^(e - 127) is exact in bf16 and is the MMA's operand.
  */
 size_t moe_workspace_size_mxfp4(int T, int k, int E, int hidden, int inter);
 int moe_select_path_mxfp4(int T, int k, int E, int hidden, int inter);

@@ -18,6 +18,7 @@ namespace qeg {
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr int kNumKernels = 22;
 
 struct DeviceInfo {
   bool ready = false;
@@ -27,8 +28,9 @@ struct DeviceInfo {
   // (chunks of 64 pairs), combine, grouped gate+up and down (chunks of 96, then of 32
   // pairs), layer (mxfp4); then the layer instances for fixed widths (affine 4096/2048,
   // mxfp4 6144/2048 and 4096/2048, each also with resident x rows), which share the
-  // general instances' limits
-  int dyn_smem[16] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
+  // general instances' limits; then the grouped kernels for mxfp4 banks (chunks of 64,
+  // 96, 32 pairs), which share the affine ones'
+  int dyn_smem[kNumKernels] = {};
 };
 
 DeviceInfo g_dev[kMaxDevices];
@@ -54,7 +56,8 @@ moe_status device_info(DeviceInfo** out) {
       e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return cuda_fail(e);
     // dynamic + static shared memory may not exceed the opt-in limit
-    const void* kernels[16] = {reinterpret_cast<const void*>(layer_kernel<kFmtAffine>),
+    const void* kernels[kNumKernels] = {
+                              reinterpret_cast<const void*>(layer_kernel<kFmtAffine>),
                               reinterpret_cast<const void*>(route_union_kernel),
                               reinterpret_cast<const void*>(grouped_gemm_kernel<0, 64>),
                               reinterpret_cast<const void*>(grouped_gemm_kernel<1, 64>),
@@ -69,8 +72,14 @@ moe_status device_info(DeviceInfo** out) {
                               reinterpret_cast<const void*>(layer_kernel<kFmtMx, 4, 2>),
                               reinterpret_cast<const void*>(layer_kernel<kFmtAffine, 4, 2, 1>),
                               reinterpret_cast<const void*>(layer_kernel<kFmtMx, 6, 2, 1>),
-                              reinterpret_cast<const void*>(layer_kernel<kFmtMx, 4, 2, 1>)};
-    for (int i = 0; i < 16; ++i) {
+                              reinterpret_cast<const void*>(layer_kernel<kFmtMx, 4, 2, 1>),
+                              reinterpret_cast<const void*>(grouped_gemm_kernel<0, 64, kFmtMx>),
+                              reinterpret_cast<const void*>(grouped_gemm_kernel<1, 64, kFmtMx>),
+                              reinterpret_cast<const void*>(grouped_gemm_kernel<0, 96, kFmtMx>),
+                              reinterpret_cast<const void*>(grouped_gemm_kernel<1, 96, kFmtMx>),
+                              reinterpret_cast<const void*>(grouped_gemm_kernel<0, 32, kFmtMx>),
+                              reinterpret_cast<const void*>(grouped_gemm_kernel<1, 32, kFmtMx>)};
+    for (int i = 0; i < kNumKernels; ++i) {
       cudaFuncAttributes fa;
       cudaError_t e = cudaFuncGetAttributes(&fa, kernels[i]);
       if (e == cudaSuccess) {
@@ -107,8 +116,7 @@ struct WsLayout {
 
 // 1 = the persistent fused kernel (small windows), 2 = the grouped tensor-core
 // kernels (windows with more pairs; hidden a multiple of 256, inter of 128),
-// 0 = neither.
-// mxfp4 banks take the persistent kernel only (0 for larger windows).
+// 0 = neither.  Both bank formats take both paths.
 // `routed`: the router step runs inside the persistent kernel (its picks and weights
 // take shared memory too).
 int select_path(int T, int k, int E, int hidden, int inter, int fmt = kFmtAffine,
@@ -118,10 +126,9 @@ int select_path(int T, int k, int E, int hidden, int inter, int fmt = kFmtAffine
     LayerGeom g = layer_geom(hidden, inter, fmt);
     if (layer_plan(g, E, T, k, kSmemBudget, routed)) return 1;
   }
-  if (fmt == kFmtMx) return 0;
-  // the grouped path: hidden a multiple of 256 (down tiles) and at most 4096, inter a
-  // multiple of 128 (gate/up tiles)
-  if (hidden % (2 * kGM) == 0 && hidden <= 4096 && inter % (2 * kGK) == 0 &&
+  // the grouped path: hidden a multiple of 256 (down tiles), inter a multiple of 128
+  // (gate/up tiles)
+  if (hidden % (2 * kGM) == 0 && inter % (2 * kGK) == 0 &&
       route_union_smem_bytes(E) <= kSmemBudget && sizeof(int) * (size_t)T * k <= kSmemBudget)
     return 2;
   return 0;
@@ -237,13 +244,14 @@ cudaError_t launch_layer(const uint16_t* x, const int32_t* idx, const float* w,
 // The grouped path: route-union (with padded offsets), x packing, gate+up, down
 // and combine as five launches on `st` (no host synchronisation).  The union
 // arrays, the packed activations, their sums and y live in the workspace.
+template <int F>
 cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w,
                            const uint32_t* gq, const uint16_t* gs, const uint16_t* gb,
                            const uint32_t* uq, const uint16_t* us, const uint16_t* ub,
                            const uint32_t* dq, const uint16_t* ds, const uint16_t* db, int T,
                            int k, int E, int H, int I, uint16_t* out, unsigned char* ws,
                            const DeviceInfo& d, cudaStream_t st, moe_status* why) {
-  const WsLayout wl = ws_layout(T, k, E, H, I);
+  const WsLayout wl = ws_layout(T, k, E, H, I, F);
   const int P = T * k;
   int* nu = reinterpret_cast<int*>(ws + wl.num_unique);
   int* uniq = reinterpret_cast<int*>(ws + wl.unique);
@@ -263,7 +271,9 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   // re-reads), 32 when they average at most 20 (more accumulator buffers), else 64
   const int width = P > 40 * m ? 96 : (P <= 20 * m ? 32 : 64);
   const unsigned gsmem = width == 96 ? GCfg<96>::kSmem : width == 32 ? GCfg<32>::kSmem : GCfg<64>::kSmem;
-  const int ki = width == 96 ? 5 : width == 32 ? 7 : 2;  // dyn_smem index of gate+up
+  // dyn_smem index of the gate+up kernel (down: the next one)
+  const int ki = F == kFmtMx ? (width == 96 ? 18 : width == 32 ? 20 : 16)
+                             : (width == 96 ? 5 : width == 32 ? 7 : 2);
   const int grid = width == 32 ? 2 * d.sms : d.sms;
   if (usmem > (size_t)d.dyn_smem[1] || csmem > (size_t)d.dyn_smem[4] ||
       gsmem > (unsigned)d.dyn_smem[ki] || gsmem > (unsigned)d.dyn_smem[ki + 1]) {
@@ -298,11 +308,11 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   g.K = H;
   g.mrows = kGM;
   if (width == 96)
-    grouped_gemm_kernel<0, 96><<<grid, kGThreads, gsmem, st>>>(g);
+    grouped_gemm_kernel<0, 96, F><<<grid, kGThreads, gsmem, st>>>(g);
   else if (width == 32)
-    grouped_gemm_kernel<0, 32><<<grid, kGThreads, gsmem, st>>>(g);
+    grouped_gemm_kernel<0, 32, F><<<grid, kGThreads, gsmem, st>>>(g);
   else
-    grouped_gemm_kernel<0, 64><<<grid, kGThreads, gsmem, st>>>(g);
+    grouped_gemm_kernel<0, 64, F><<<grid, kGThreads, gsmem, st>>>(g);
   // down: 256 rows of Wd per tile (two 128-row matrices), K = I, packed h
   g.bp = hp;
   g.bs = hs;
@@ -314,11 +324,11 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   g.K = I;
   g.mrows = 2 * kGM;
   if (width == 96)
-    grouped_gemm_kernel<1, 96><<<grid, kGThreads, gsmem, st>>>(g);
+    grouped_gemm_kernel<1, 96, F><<<grid, kGThreads, gsmem, st>>>(g);
   else if (width == 32)
-    grouped_gemm_kernel<1, 32><<<grid, kGThreads, gsmem, st>>>(g);
+    grouped_gemm_kernel<1, 32, F><<<grid, kGThreads, gsmem, st>>>(g);
   else
-    grouped_gemm_kernel<1, 64><<<grid, kGThreads, gsmem, st>>>(g);
+    grouped_gemm_kernel<1, 64, F><<<grid, kGThreads, gsmem, st>>>(g);
   grouped_combine_kernel<<<2 * d.sms, kGCombineThreads, csmem, st>>>(y, w, plist, offs, nu, T, k,
                                                                       H, out);
   return cudaGetLastError();
@@ -506,15 +516,14 @@ moe_status moe_switchglu_forward_ws(const uint16_t* x, const int32_t* topk_idx,
   DeviceInfo* d = nullptr;
   if (moe_status s = device_info(&d)) return s;
   moe_status why = MOE_OK;
+  unsigned char* wsp = static_cast<unsigned char*>(workspace);
   const cudaError_t e =
-      path == 1 ? launch_layer<kFmtAffine>(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q, wd_s,
-                               wd_b, T, k, E, hidden, inter, out,
-                               static_cast<unsigned char*>(workspace), *d, (cudaStream_t)stream,
-                               &why)
-                : launch_grouped(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q,
-                                 wd_s, wd_b, T, k, E, hidden, inter, out,
-                                 static_cast<unsigned char*>(workspace), *d, (cudaStream_t)stream,
-                                 &why);
+      path == 1 ? launch_layer<kFmtAffine>(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s,
+                                           wu_b, wd_q, wd_s, wd_b, T, k, E, hidden, inter, out,
+                                           wsp, *d, (cudaStream_t)stream, &why)
+                : launch_grouped<kFmtAffine>(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s,
+                                             wu_b, wd_q, wd_s, wd_b, T, k, E, hidden, inter, out,
+                                             wsp, *d, (cudaStream_t)stream, &why);
   if (why != MOE_OK) return why;
   return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
@@ -570,9 +579,9 @@ moe_status moe_switchglu_forward_routed_ws(
         logits, T, E, k, renormalize ? 1 : 0, topk_idx, topk_w);
     e = cudaGetLastError();
     if (e == cudaSuccess)
-      e = launch_grouped(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b, wd_q, wd_s,
-                         wd_b, T, k, E, hidden, inter, out,
-                         static_cast<unsigned char*>(workspace), *d, st, &why);
+      e = launch_grouped<kFmtAffine>(x, topk_idx, topk_w, wg_q, wg_s, wg_b, wu_q, wu_s, wu_b,
+                                     wd_q, wd_s, wd_b, T, k, E, hidden, inter, out,
+                                     static_cast<unsigned char*>(workspace), *d, st, &why);
   }
   if (why != MOE_OK) return why;
   return e == cudaSuccess ? MOE_OK : cuda_fail(e);
@@ -638,7 +647,8 @@ moe_status moe_switchglu_forward_mxfp4_ws(const uint16_t* x, const int32_t* topk
   for (const void* p : a16)
     if (!aligned(p, 16)) return MOE_ERR_UNSUPPORTED;
   if (!aligned(topk_idx, 4) || !aligned(topk_w, 4)) return MOE_ERR_UNSUPPORTED;
-  if (select_path(T, k, E, hidden, inter, kFmtMx) != 1) return MOE_ERR_UNSUPPORTED;
+  const int path = select_path(T, k, E, hidden, inter, kFmtMx);
+  if (path == 0) return MOE_ERR_UNSUPPORTED;
   if (workspace_bytes < ws_layout(T, k, E, hidden, inter, kFmtMx).total) return MOE_ERR_WORKSPACE;
   DeviceInfo* d = nullptr;
   if (moe_status s = device_info(&d)) return s;
@@ -647,9 +657,14 @@ moe_status moe_switchglu_forward_mxfp4_ws(const uint16_t* x, const int32_t* topk
   const uint16_t* ge = reinterpret_cast<const uint16_t*>(wg_e);
   const uint16_t* ue = reinterpret_cast<const uint16_t*>(wu_e);
   const uint16_t* de = reinterpret_cast<const uint16_t*>(wd_e);
-  const cudaError_t e = launch_layer<kFmtMx>(
-      x, topk_idx, topk_w, wg_q, ge, nullptr, wu_q, ue, nullptr, wd_q, de, nullptr, T, k, E,
-      hidden, inter, out, static_cast<unsigned char*>(workspace), *d, (cudaStream_t)stream, &why);
+  unsigned char* wsp = static_cast<unsigned char*>(workspace);
+  const cudaError_t e =
+      path == 1 ? launch_layer<kFmtMx>(x, topk_idx, topk_w, wg_q, ge, nullptr, wu_q, ue, nullptr,
+                                       wd_q, de, nullptr, T, k, E, hidden, inter, out, wsp, *d,
+                                       (cudaStream_t)stream, &why)
+                : launch_grouped<kFmtMx>(x, topk_idx, topk_w, wg_q, ge, nullptr, wu_q, ue,
+                                         nullptr, wd_q, de, nullptr, T, k, E, hidden, inter, out,
+                                         wsp, *d, (cudaStream_t)stream, &why);
   if (why != MOE_OK) return why;
   return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }

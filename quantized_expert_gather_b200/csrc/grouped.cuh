@@ -46,6 +46,12 @@
 // the order (0,4,1,5,2,6,3,7) within every 8 columns; the packed activations
 // follow the same order.
 //
+// mxfp4 banks (F = kFmtMx: e2m1 codes, one e8m0 scale 2^(e-127) per 32 columns, no
+// bias): a weight e2m1(q) 2^(e-127) is itself exact in bf16, so the expansion writes
+// the weights (two byte lookups give 2 e2m1(q) + 12 per code, placed under the bf16
+// exponent of 128 as above, and one packed FMA scales and offsets them exactly) and
+// the read-back adds each slab's product with no scale and no bias term.
+//
 // Packed activations (the B operand): [K/64][pcap][64] bf16.  Row = padded pair
 // position: expert slot i owns rows padded[i] .. padded[i] + roundup16(count_i)
 // (route_union_kernel's padded offsets), with zero rows as padding.  Each 128-byte
@@ -55,6 +61,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "layer.cuh"  // kFmtMx, mx_bytes, mx_half_scale: the mxfp4 code and scale lookups
 
 namespace qeg {
 
@@ -244,6 +251,31 @@ __device__ __forceinline__ void codes_to_bf16(uint32_t w, uint32_t one2, uint32_
   }
 }
 
+// The 8 mxfp4 codes of word w as 4 bf16 pairs of weights e2m1(q) 2^(e-127) (low
+// half code j, high half code j + 4), j = 0..3, exact.  s2 = bf16 pair (h, h) and
+// c2 = (-140 h, -140 h) for h = 2^(e-128) of the group's scale byte e: the bytes
+// q' = 2 e2m1(q) + 12 read as 128 + q' under the bf16 exponent of 128, and
+// (128 + q') h - 140 h = 2 e2m1(q) h.
+__device__ __forceinline__ void mx_codes_to_bf16(uint32_t w, uint32_t s2, uint32_t c2,
+                                                 uint32_t* o) {
+  const uint32_t lo = mx_bytes(w), hi = mx_bytes(w >> 16);  // codes 0..3, 4..7
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    // bytes (lo[j], 0, hi[j], 0): selectors j and 4 + j, the others the sign fill of a
+    // byte below 128
+    const uint32_t sel = (uint32_t)j | ((8u | j) << 4) | ((4u + j) << 8) | ((12u + j) << 12);
+    const uint32_t t = prmt_sign(lo, hi, sel) | 0x43004300u;  // 128 + q'
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(o[j]) : "r"(t), "r"(s2), "r"(c2));
+  }
+}
+// The bf16 pairs (h, h) and (-140 h, -140 h), h = 2^(e - 128), for an e8m0 byte e.
+__device__ __forceinline__ void mx_scale_pairs(uint32_t e, uint32_t& s2, uint32_t& c2) {
+  const float h = mx_half_scale(e);
+  const uint32_t hb = float_to_bf16_bits(h), cb = float_to_bf16_bits(-140.0f * h);
+  s2 = hb | (hb << 16);
+  c2 = cb | (cb << 16);
+}
+
 // --------------------------------------------------------------- packing ---
 // Packed x: for every padded pair position of every expert slot, the pair's token
 // row of x (zero for padding) and its group sums.  One block per slot (looping).
@@ -293,8 +325,8 @@ struct GroupedArgs {
   const int* padded;     // [u + 1] padded row offsets of the packed layout
   const int* num_unique; // [1]
   const uint32_t* q[2];  // codes of matrix 0 / 1 of a tile
-  const uint16_t* s[2];  // scales
-  const uint16_t* b[2];  // biases
+  const uint16_t* s[2];  // scales (mxfp4: the e8m0 bytes)
+  const uint16_t* b[2];  // biases (mxfp4: none)
   int roff[2];           // row offset of matrix m inside the tile (0/0 or 0/128)
   uint16_t* hp;          // phase 0: packed h [I/64][pcap][64]
   float* hs;             // phase 0: h group sums [I/64][pcap]
@@ -303,7 +335,7 @@ struct GroupedArgs {
   int pcap, H;
 };
 
-template <int PHASE, int NMAX>
+template <int PHASE, int NMAX, int F = kFmtAffine>
 __global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
     grouped_gemm_kernel(const __grid_constant__ GroupedArgs a) {
   using C = GCfg<NMAX>;
@@ -378,8 +410,13 @@ __global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
           for (int i = 0; i < 2 * kGM / 32; ++i) {
             const int rr = lane + 32 * i, m = rr / kGM, r = rr % kGM;
             const size_t row = (size_t)e * a.rows + m0 + a.roff[m] + r;
-            cp_async4(stg + C::kOffS + rr * 4, a.s[m] + row * (a.K / kGK) + j0);
-            cp_async4(stg + C::kOffBias + rr * 4, a.b[m] + row * (a.K / kGK) + j0);
+            if constexpr (F == kFmtMx) {  // the stage's four e8m0 bytes; no biases
+              cp_async4(stg + C::kOffS + rr * 4,
+                        reinterpret_cast<const unsigned char*>(a.s[m]) + row * (a.K / 32) + 2 * j0);
+            } else {
+              cp_async4(stg + C::kOffS + rr * 4, a.s[m] + row * (a.K / kGK) + j0);
+              cp_async4(stg + C::kOffBias + rr * 4, a.b[m] + row * (a.K / kGK) + j0);
+            }
           }
           if (lane == 0) {
 #pragma unroll
@@ -455,10 +492,13 @@ __global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
       const uint32_t ab = gp % kGDBufs;
       tc_fence_after();
       const unsigned char* stg = gsm + st * C::kStageBytes;
-      const float sv = bf16_bits_to_float(
-          *reinterpret_cast<const uint16_t*>(stg + C::kOffS + (m * kGM + r) * 4 + jj * 2));
-      const float bv = bf16_bits_to_float(
-          *reinterpret_cast<const uint16_t*>(stg + C::kOffBias + (m * kGM + r) * 4 + jj * 2));
+      float sv = 1.0f, bv = 0.0f;  // mxfp4: the weights carry their scale, no bias
+      if constexpr (F != kFmtMx) {
+        sv = bf16_bits_to_float(
+            *reinterpret_cast<const uint16_t*>(stg + C::kOffS + (m * kGM + r) * 4 + jj * 2));
+        bv = bf16_bits_to_float(
+            *reinterpret_cast<const uint16_t*>(stg + C::kOffBias + (m * kGM + r) * 4 + jj * 2));
+      }
       const float2 s2 = make_float2(sv, sv), b2 = make_float2(bv, bv);
       const float4* X = reinterpret_cast<const float4*>(stg + C::kOffX + jj * C::kN * 4);
       const uint32_t dcol = tmem + C::col_d(ab, m) + lane_base;
@@ -487,8 +527,10 @@ __global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
                                     s2, acc[o]);
                 acc[o + 1] = __ffma2_rn(
                     make_float2(__uint_as_float(pp[2]), __uint_as_float(pp[3])), s2, acc[o + 1]);
-                acc[o] = __ffma2_rn(make_float2(xv.x, xv.y), b2, acc[o]);
-                acc[o + 1] = __ffma2_rn(make_float2(xv.z, xv.w), b2, acc[o + 1]);
+                if constexpr (F != kFmtMx) {
+                  acc[o] = __ffma2_rn(make_float2(xv.x, xv.y), b2, acc[o]);
+                  acc[o + 1] = __ffma2_rn(make_float2(xv.z, xv.w), b2, acc[o + 1]);
+                }
               }
             }
           }
@@ -536,10 +578,19 @@ __global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
             for (int hw = 0; hw < 2; ++hw) {  // 32 codes (16 columns) at a time
               const uint4 wv = crow[hw];
               uint32_t av[16];
-              codes_to_bf16(wv.x, one2, m128, av + 0);
-              codes_to_bf16(wv.y, one2, m128, av + 4);
-              codes_to_bf16(wv.z, one2, m128, av + 8);
-              codes_to_bf16(wv.w, one2, m128, av + 12);
+              if constexpr (F == kFmtMx) {  // one e8m0 group: this slab's byte hw
+                uint32_t s2, c2;
+                mx_scale_pairs(stg[C::kOffS + (m * kGM + r) * 4 + jj * 2 + hw], s2, c2);
+                mx_codes_to_bf16(wv.x, s2, c2, av + 0);
+                mx_codes_to_bf16(wv.y, s2, c2, av + 4);
+                mx_codes_to_bf16(wv.z, s2, c2, av + 8);
+                mx_codes_to_bf16(wv.w, s2, c2, av + 12);
+              } else {
+                codes_to_bf16(wv.x, one2, m128, av + 0);
+                codes_to_bf16(wv.y, one2, m128, av + 4);
+                codes_to_bf16(wv.z, one2, m128, av + 8);
+                codes_to_bf16(wv.w, one2, m128, av + 12);
+              }
               tc_st16(acol + 16 * hw, av);
             }
             tc_wait_st();

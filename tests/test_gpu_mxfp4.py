@@ -90,3 +90,39 @@ def test_mxfp4_glm52_bank(T):
     used = sorted(set(int(e) for e in idx.ravel()))
     ref = oracle.switchglu_mxfp4(x, idx, w, host_bank(E, H, I, seed, used), E)
     assert_parity(bf16_to_f64(out), ref, f"mxfp4 GLM-5.2 bank T={T}")
+
+
+@pytest.mark.parametrize("cfg", [
+    # T, k, E, H, I: more than 1024 pairs, so the grouped tensor-core path
+    (160, 8, 64, 512, 256),
+    (200, 6, 32, 768, 384),
+    (600, 2, 3, 256, 128),   # about 400 pairs per expert: several chunks of 96
+])
+def test_mxfp4_grouped_small_shapes(cfg):
+    T, k, E, H, I = cfg
+    assert qeg.moe_select_path_mxfp4(T, k, E, H, I) == 2
+    seed = 7200 + sum(cfg)
+    idx, w = synth.route_uniform(T, E, k, seed)
+    hb = host_bank(E, H, I, seed)
+    x = synth.x_bf16(T, H, seed)
+    out = run(x, idx, w, upload(hb))
+    assert qeg.moe_read_device_status() == qeg.MOE_OK
+    assert_parity(bf16_to_f64(out), oracle.switchglu_mxfp4(x, idx, w, hb, E),
+                  f"mxfp4 grouped T={T} k={k} E={E} H={H} I={I}")
+
+
+def test_mxfp4_glm52_bank_large_window():
+    """GLM-5.2's routed bank (E=256, 6144 x 2048) at T=512 with uniform top-8 routing: the
+    grouped path; sampled tokens against the oracle."""
+    E, H, I, T, seed = 256, 6144, 2048, 512, 7300
+    assert qeg.moe_select_path_mxfp4(T, 8, E, H, I) == 2
+    bank = dev_bank(E, H, I, seed)
+    idx, w = synth.route_uniform(T, E, 8, seed)
+    x = synth.x_bf16(T, H, seed)
+    out = run(x, idx, w, bank)
+    assert qeg.moe_read_device_status() == qeg.MOE_OK
+    tokens = sorted(np.random.default_rng(seed).choice(T, 8, replace=False).tolist())
+    used = sorted(set(int(e) for e in idx[tokens].ravel()))
+    ref = oracle.switchglu_mxfp4(x[tokens], idx[tokens], w[tokens],
+                                 host_bank(E, H, I, seed, used), E)
+    assert_parity(bf16_to_f64(out)[tokens], ref, "mxfp4 GLM-5.2 bank T=512 (sampled tokens)")

@@ -301,6 +301,7 @@ def test_grouped_path_selected_for_large_windows():
     assert qeg.moe_select_path(160, 8, 64, 512, 256) == 2
     assert qeg.moe_select_path(512, 8, 256, 4096, 2048) == 2
     assert qeg.moe_select_path(2048, 8, 256, 4096, 2048) == 2
+    assert qeg.moe_select_path(512, 8, 256, 6144, 2048) == 2
     assert qeg.moe_select_path(160, 8, 64, 512, 192) == 0  # weight rows not a multiple of 128
 
 
@@ -308,6 +309,7 @@ def test_grouped_path_selected_for_large_windows():
     # T, k, E, H, I: several experts with more than 16 pairs, ragged N tiles
     (160, 8, 64, 512, 256),
     (130, 8, 16, 256, 384),
+    (130, 8, 16, 6144, 256),  # hidden 6144 (GLM-5.2's width)
 ])
 def test_grouped_small(cfg):
     T, k, E, H, I = cfg

@@ -69,14 +69,19 @@ def test_path_selection_without_launch():
 
 
 def test_mxfp4_path_and_workspace():
-    """mxfp4 banks take the persistent kernel (GLM-5.2's 6144 x 2048 bank included) and
-    nothing else; the workspace matches the affine one on that path."""
+    """mxfp4 banks take the persistent kernel for small windows and the grouped path for
+    large ones (GLM-5.2's 6144 x 2048 bank included); the workspace matches the affine one
+    on both paths."""
     for T in (1, 2, 4, 16):
         assert qeg.moe_select_path_mxfp4(T, 8, 256, 6144, 2048) == 1
         assert qeg.moe_select_path_mxfp4(T, 8, 288, 4096, 2048) == 1
         assert qeg.moe_workspace_size_mxfp4(T, 8, 288, 4096, 2048) == \
             qeg.moe_workspace_size(T, 8, 288, 4096, 2048)
-    assert qeg.moe_select_path_mxfp4(512, 8, 256, 4096, 2048) == 0
+    for H in (4096, 6144):
+        assert qeg.moe_select_path_mxfp4(512, 8, 256, H, 2048) == 2
+        assert qeg.moe_workspace_size_mxfp4(512, 8, 256, H, 2048) == \
+            qeg.moe_workspace_size(512, 8, 256, H, 2048)
+    assert qeg.moe_select_path_mxfp4(160, 8, 64, 512, 192) == 0  # rows not a multiple of 128
     assert qeg.moe_workspace_size_mxfp4(0, 8, 256, 4096, 2048) == 0
 
 
