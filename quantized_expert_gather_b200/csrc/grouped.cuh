@@ -49,8 +49,8 @@
 // mxfp4 banks (F = kFmtMx: e2m1 codes, one e8m0 scale 2^(e-127) per 32 columns, no
 // bias): a weight e2m1(q) 2^(e-127) is itself exact in bf16, so the expansion writes
 // the weights (two byte lookups give 2 e2m1(q) + 12 per code, placed under the bf16
-// exponent of 128 as above, and one packed FMA scales and offsets them exactly) and
-// the read-back adds each slab's product with no scale and no bias term.
+// exponent of 128 as above, and one packed FMA scales and offsets them exactly), and
+// a chunk's whole K accumulates in tensor memory, read back once per chunk.
 //
 // Packed activations (the B operand): [K/64][pcap][64] bf16.  Row = padded pair
 // position: expert slot i owns rows padded[i] .. padded[i] + roundup16(count_i)
@@ -342,6 +342,7 @@ __global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
   extern __shared__ __align__(128) unsigned char gsm_raw[];
   __shared__ __align__(8) uint64_t full[C::kStages], empty[C::kStages];
   __shared__ __align__(8) uint64_t a_full[kGABufs], d_full[kGDBufs], d_free[kGDBufs];
+  __shared__ __align__(8) uint64_t c_full[kGDBufs];  // mxfp4: a chunk's product complete
   __shared__ uint32_t tmem_base_s;
   __shared__ float red[2][2][C::kN / 2];
   // swizzled tiles start at 1024-byte boundaries of the shared address space
@@ -357,6 +358,7 @@ __global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
     for (int i = 0; i < kGDBufs; ++i) {
       mbar_init(&d_full[i], 1);
       mbar_init(&d_free[i], kGWorkers);
+      mbar_init(&c_full[i], 1);
     }
     fence_barrier_init();
   }
@@ -439,12 +441,48 @@ __global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
     // ---------------------------------------------------------- MMA issuer ---
     // The whole warp runs this loop (operands warp-uniform); one elected lane issues.
     uint32_t issued = 0;  // slabs whose MMAs were issued
+    uint32_t tcn = 0;     // chunks started (mxfp4)
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       const int slot = tile / mtiles;
       const int cnt = a.offsets[slot + 1] - a.offsets[slot];
       for (int c0 = 0; c0 < cnt && ok; c0 += C::kN) {
         const int np = (min(C::kN, cnt - c0) + 15) & ~15;
         const uint32_t idesc = f16_idesc(kGM, np);
+        if constexpr (F == kFmtMx) {
+          // The weights are exact in bf16: the chunk's whole K accumulates in
+          // accumulator buffer tcn % 2, read back once (c_full); d_full[slab % 2] only
+          // says that a slab's MMAs are done, so that its A buffer may be rewritten.
+          const uint32_t db = tcn % kGDBufs;
+          if (tcn >= (uint32_t)kGDBufs)
+            ok = __all_sync(kFull, mbar_wait(&d_free[db], (tcn / kGDBufs - 1) & 1));
+          bool first = true;
+          for (int j0 = 0; j0 < nslab && ok; j0 += kGSlabsPerStage, ++sc) {
+            const int st = sc % C::kStages;
+            ok = __all_sync(kFull, mbar_wait(&full[st], (sc / C::kStages) & 1));
+            const uint32_t bbase = smem_u32(gsm + st * C::kStageBytes + kGOffB);
+            for (int jj = 0; jj < kGSlabsPerStage && ok; ++jj, ++gs) {
+              const uint32_t ab = gs % kGABufs;
+              ok = __all_sync(kFull, mbar_wait(&a_full[ab], (gs / kGABufs) & 1));
+              if (!ok) break;
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < kGK / 16; ++kk) {
+                const uint64_t bdesc = sw128_desc(bbase + jj * C::kBTile + kk * 32);
+#pragma unroll
+                for (int m = 0; m < 2; ++m)
+                  tc_mma_ts_elect(tmem + C::col_d(db, m), tmem + C::col_a(ab, m) + kk * 8, bdesc,
+                                  idesc, (first && kk == 0) ? 0u : 1u);
+              }
+              first = false;
+              tc_commit_elect(&d_full[ab]);
+              if (jj == kGSlabsPerStage - 1) tc_commit_elect(&empty[st]);
+              issued = gs + 1;
+            }
+          }
+          if (ok) tc_commit_elect(&c_full[db]);
+          ++tcn;
+          continue;
+        }
         for (int j0 = 0; j0 < nslab && ok; j0 += kGSlabsPerStage, ++sc) {
           const int st = sc % C::kStages;
           const uint32_t round = sc / C::kStages;
@@ -544,6 +582,29 @@ __global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
       }
     };
 
+    // mxfp4: acc = the chunk's product in accumulator buffer db (its MMAs are known to
+    // be done), then the buffer is free again
+    auto read_chunk = [&](uint32_t db, int ng) {
+      tc_fence_after();
+      const uint32_t dcol = tmem + C::col_d(db, m) + lane_base;
+#pragma unroll
+      for (int cg = 0; cg < C::kN / 16; ++cg) {
+        if (cg < ng) {
+          uint32_t pr[16];
+          tc_ld16(dcol + cg * 16, pr);
+          tc_wait_ld();
+          tc_regs_ready(pr);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            acc[cg * 8 + i] = make_float2(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&d_free[db]);
+    };
+    uint32_t tcn = 0;  // chunks finished (mxfp4)
+
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       const int slot = tile / mtiles, m0 = (tile % mtiles) * a.mrows;
       const int p0 = a.offsets[slot], cnt = a.offsets[slot + 1] - p0;
@@ -597,17 +658,30 @@ __global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&a_full[ab]);
-            if (gs >= gs0 + kGLag) {
+            if constexpr (F == kFmtMx) {
+              // the stage's codes and scale bytes are read: release it (the MMA warp's
+              // commit is the other arrival)
+              if (jj == kGSlabsPerStage - 1 && lane == 0) mbar_arrive(&empty[st]);
+            } else if (gs >= gs0 + kGLag) {
               wait_slab(gs - kGLag);
               if (ok) read_slab(gs - kGLag);
             }
           }
         }
         if (!ok) break;
-        // the chunk's last kGLag slabs
-        for (uint32_t g = gs >= gs0 + kGLag ? gs - kGLag : gs0; g < gs && ok; ++g) {
-          wait_slab(g);
-          if (ok) read_slab(g);
+        if constexpr (F == kFmtMx) {
+          // the chunk's whole product, accumulated over K in tensor memory, read once
+          const uint32_t db = tcn % kGDBufs;
+          ok = __all_sync(kFull, mbar_wait(&c_full[db], (tcn / kGDBufs) & 1));
+          if (!ok) break;
+          read_chunk(db, ng);
+          ++tcn;
+        } else {
+          // the chunk's last kGLag slabs
+          for (uint32_t g = gs >= gs0 + kGLag ? gs - kGLag : gs0; g < gs && ok; ++g) {
+            wait_slab(g);
+            if (ok) read_slab(g);
+          }
         }
         if (!ok) break;
 
