@@ -481,31 +481,31 @@ __global__ void __launch_bounds__(kGThreads, GCfg<NMAX>::kCtasPerSm)
           }
           if (ok) tc_commit_elect(&c_full[db]);
           ++tcn;
-          continue;
-        }
-        for (int j0 = 0; j0 < nslab && ok; j0 += kGSlabsPerStage, ++sc) {
-          const int st = sc % C::kStages;
-          const uint32_t round = sc / C::kStages;
-          ok = __all_sync(kFull, mbar_wait(&full[st], round & 1));
-          const uint32_t bbase = smem_u32(gsm + st * C::kStageBytes + kGOffB);
-          for (int jj = 0; jj < kGSlabsPerStage && ok; ++jj, ++gs) {
-            const uint32_t ab = gs % kGABufs, db = gs % kGDBufs;
-            bool w = mbar_wait(&a_full[ab], (gs / kGABufs) & 1);
-            if (w && gs >= (uint32_t)kGDBufs) w = mbar_wait(&d_free[db], (gs / kGDBufs - 1) & 1);
-            ok = __all_sync(kFull, w);
-            if (!ok) break;
-            tc_fence_after();
+        } else {
+          for (int j0 = 0; j0 < nslab && ok; j0 += kGSlabsPerStage, ++sc) {
+            const int st = sc % C::kStages;
+            const uint32_t round = sc / C::kStages;
+            ok = __all_sync(kFull, mbar_wait(&full[st], round & 1));
+            const uint32_t bbase = smem_u32(gsm + st * C::kStageBytes + kGOffB);
+            for (int jj = 0; jj < kGSlabsPerStage && ok; ++jj, ++gs) {
+              const uint32_t ab = gs % kGABufs, db = gs % kGDBufs;
+              bool w = mbar_wait(&a_full[ab], (gs / kGABufs) & 1);
+              if (w && gs >= (uint32_t)kGDBufs) w = mbar_wait(&d_free[db], (gs / kGDBufs - 1) & 1);
+              ok = __all_sync(kFull, w);
+              if (!ok) break;
+              tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < kGK / 16; ++kk) {
-              const uint64_t bdesc = sw128_desc(bbase + jj * C::kBTile + kk * 32);
+              for (int kk = 0; kk < kGK / 16; ++kk) {
+                const uint64_t bdesc = sw128_desc(bbase + jj * C::kBTile + kk * 32);
 #pragma unroll
-              for (int m = 0; m < 2; ++m)
-                tc_mma_ts_elect(tmem + C::col_d(db, m), tmem + C::col_a(ab, m) + kk * 8, bdesc, idesc,
-                                kk > 0 ? 1u : 0u);
+                for (int m = 0; m < 2; ++m)
+                  tc_mma_ts_elect(tmem + C::col_d(db, m), tmem + C::col_a(ab, m) + kk * 8, bdesc,
+                                  idesc, kk > 0 ? 1u : 0u);
+              }
+              tc_commit_elect(&d_full[db]);
+              if (jj == kGSlabsPerStage - 1) tc_commit_elect(&empty[st]);
+              issued = gs + 1;
             }
-            tc_commit_elect(&d_full[db]);
-            if (jj == kGSlabsPerStage - 1) tc_commit_elect(&empty[st]);
-            issued = gs + 1;
           }
         }
       }
