@@ -412,8 +412,9 @@ def reference_arm(args, world, rank):
 
 def large_window_only(args, local):
     """Profiling run of the grouped path alone: one T-token layer (T from --ts, default
-    512) on an E=256 bank (3.6 GB), 3 warm calls then 1 timed; for ncu captures of the
-    grouped kernels on a small device footprint."""
+    512) on an E=256 bank (3.6 GB; with --mxfp4 an mxfp4 bank of the same shape, 3.4 GB),
+    3 warm calls then 1 timed; for ncu captures of the grouped kernels on a small device
+    footprint."""
     import torch
     import quantized_expert_gather_b200 as qeg
     import synth
@@ -428,24 +429,41 @@ def large_window_only(args, local):
         b = torch.empty_like(s)
         synth.fill_bank_device(q, s, b, rows, cols, SEED, mid)
         return q, s.view(torch.bfloat16), b.view(torch.bfloat16)
-    bank = qeg.QuantBank(*mat(INTER, HIDDEN, 0), *mat(INTER, HIDDEN, 1), *mat(HIDDEN, INTER, 2))
+    def matm(rows, cols, mid):
+        q = torch.empty((EL, rows, cols // 8), dtype=torch.int32, device=dev)
+        e8 = torch.empty((EL, rows, cols // 32), dtype=torch.uint8, device=dev)
+        synth.fill_bank_mxfp4_device(q, e8, rows, cols, SEED, mid)
+        return q, e8
+    if args.mxfp4:  # the same shape on an mxfp4 bank (3.4 GB)
+        bank = qeg.MxBank(*matm(INTER, HIDDEN, 0), *matm(INTER, HIDDEN, 1),
+                          *matm(HIDDEN, INTER, 2))
+        size = qeg.moe_workspace_size_mxfp4
+
+        def call(x, il, wl, ws, out):
+            qeg.moe_switchglu_forward_mxfp4_ws(x, il, wl, bank, ws, out=out)
+    else:
+        bank = qeg.QuantBank(*mat(INTER, HIDDEN, 0), *mat(INTER, HIDDEN, 1),
+                             *mat(HIDDEN, INTER, 2))
+        size = qeg.moe_workspace_size
+
+        def call(x, il, wl, ws, out):
+            qeg.moe_switchglu_forward_ws(x, il, wl, bank, ws, out=out)
     r = synth.route_uniform(TL, EL, K_TOP, SEED + 900 + TL)
     x = torch.from_numpy(synth.x_bf16(TL, HIDDEN, SEED + TL).view(np.int16)).to(dev) \
         .view(torch.bfloat16)
     il, wl = torch.from_numpy(r[0]).to(dev), torch.from_numpy(r[1]).to(dev)
     out = torch.empty((TL, HIDDEN), dtype=torch.bfloat16, device=dev)
-    ws = torch.zeros(qeg.moe_workspace_size(TL, K_TOP, EL, HIDDEN, INTER), dtype=torch.uint8,
-                     device=dev)
+    ws = torch.zeros(size(TL, K_TOP, EL, HIDDEN, INTER), dtype=torch.uint8, device=dev)
     for _ in range(3):
-        qeg.moe_switchglu_forward_ws(x, il, wl, bank, ws, out=out)
+        call(x, il, wl, ws, out)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
-    qeg.moe_switchglu_forward_ws(x, il, wl, bank, ws, out=out)
+    call(x, il, wl, ws, out)
     b.record()
     torch.cuda.synchronize()
-    return {"large_window_only": True, "T": TL, "us_per_layer": a.elapsed_time(b) * 1e3,
-            "status": qeg.moe_read_device_status()}
+    return {"large_window_only": True, "T": TL, "mxfp4": bool(args.mxfp4),
+            "us_per_layer": a.elapsed_time(b) * 1e3, "status": qeg.moe_read_device_status()}
 
 
 def our_arm(args, world, rank, local):
@@ -954,6 +972,8 @@ def main():
     ap.add_argument("--no-window-sweep", action="store_true",
                     help="skip the verify-window sweep (T=2..16, 78-layer stacks)")
     ap.add_argument("--ts", default="", help="comma-separated window sizes (profiling)")
+    ap.add_argument("--mxfp4", action="store_true",
+                    help="with --large-window-only: the same shape on an mxfp4 bank")
     ap.add_argument("--large-window-only", action="store_true",
                     help="one grouped-path layer alone (T from --ts, default 512; profiling)")
     ap.add_argument("--routing", default="uniform", choices=("uniform", "markov", "identical"),
