@@ -282,8 +282,9 @@ cudaError_t launch_grouped(const uint16_t* x, const int32_t* idx, const float* w
   }
   route_union_kernel<<<1, 32 * kUnionWarps, usmem, st>>>(idx, P, E, uniq, offs, plist, nu,
                                                          padded);
-  grouped_pack_x_kernel<<<m < 4 * d.sms ? m : 4 * d.sms, 256, 0, st>>>(x, plist, offs, padded,
-                                                                         nu, k, H, pcap, xp, xs);
+  // blocks (slot, slice): up to two per SM along the slots, four slices of each slot
+  const dim3 pgrid(m < 2 * d.sms ? m : 2 * d.sms, 4);
+  grouped_pack_x_kernel<<<pgrid, 256, 0, st>>>(x, plist, offs, padded, nu, k, H, pcap, xp, xs);
   GroupedArgs g{};
   g.unique = uniq;
   g.offsets = offs;

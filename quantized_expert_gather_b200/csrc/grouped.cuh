@@ -286,32 +286,49 @@ __global__ void __launch_bounds__(256) grouped_pack_x_kernel(
     float* __restrict__ xs) {
   const int u = *num_unique;
   const int nslab = H / kGK;
+  // blocks (slot, y) share a slot's units in strides of gridDim.y * blockDim.x, each
+  // thread with kPackBatch loads in flight before the first is used
+  constexpr int kPackBatch = 4;
+  const int step = gridDim.y * blockDim.x;
   for (int slot = blockIdx.x; slot < u; slot += gridDim.x) {
     const int p0 = offsets[slot], cnt = offsets[slot + 1] - p0;
     const int np = (cnt + 15) & ~15;
     const int base = padded[slot];
     const int units = np * nslab * 8;  // a multiple of 128: whole warps stay together
-    for (int unit = threadIdx.x; unit < units; unit += blockDim.x) {
-      const int c = unit & 7, rest = unit >> 3;
-      const int g = rest % nslab, n = rest / nslab;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (n < cnt) {
-        const int t = pair_list[p0 + n] / k;
-        v = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H + g * kGK + c * 8));
+    for (int u0 = blockIdx.y * blockDim.x + threadIdx.x; u0 < units; u0 += kPackBatch * step) {
+      uint4 v[kPackBatch];
+#pragma unroll
+      for (int i = 0; i < kPackBatch; ++i) {
+        const int unit = u0 + i * step;
+        const int rest = unit >> 3, n = rest / nslab;
+        v[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (unit < units && n < cnt) {
+          const int c = unit & 7, g = rest % nslab;
+          const int t = pair_list[p0 + n] / k;
+          v[i] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H + g * kGK + c * 8));
+        }
       }
-      float s = ((bf16_lo(v.x) + bf16_hi(v.x)) + (bf16_lo(v.y) + bf16_hi(v.y))) +
-                ((bf16_lo(v.z) + bf16_hi(v.z)) + (bf16_lo(v.w) + bf16_hi(v.w)));
-      s += __shfl_xor_sync(kFull, s, 1);
-      s += __shfl_xor_sync(kFull, s, 2);
-      s += __shfl_xor_sync(kFull, s, 4);
-      uint4 o;  // K order (0,4,1,5,2,6,3,7)
-      o.x = prmt(v.x, v.z, 0x5410u);
-      o.y = prmt(v.x, v.z, 0x7632u);
-      o.z = prmt(v.y, v.w, 0x5410u);
-      o.w = prmt(v.y, v.w, 0x7632u);
-      const int pos = base + n;
-      *reinterpret_cast<uint4*>(xp + ((size_t)g * pcap + pos) * kGK + ((c ^ (pos & 7)) * 8)) = o;
-      if (c == 0) xs[(size_t)g * pcap + pos] = s;
+#pragma unroll
+      for (int i = 0; i < kPackBatch; ++i) {
+        const int unit = u0 + i * step;
+        if (unit < units) {  // uniform over the warp (units and step are multiples of 32)
+          const int c = unit & 7, rest = unit >> 3;
+          const int g = rest % nslab, n = rest / nslab;
+          float s = ((bf16_lo(v[i].x) + bf16_hi(v[i].x)) + (bf16_lo(v[i].y) + bf16_hi(v[i].y))) +
+                    ((bf16_lo(v[i].z) + bf16_hi(v[i].z)) + (bf16_lo(v[i].w) + bf16_hi(v[i].w)));
+          s += __shfl_xor_sync(kFull, s, 1);
+          s += __shfl_xor_sync(kFull, s, 2);
+          s += __shfl_xor_sync(kFull, s, 4);
+          uint4 o;  // K order (0,4,1,5,2,6,3,7)
+          o.x = prmt(v[i].x, v[i].z, 0x5410u);
+          o.y = prmt(v[i].x, v[i].z, 0x7632u);
+          o.z = prmt(v[i].y, v[i].w, 0x5410u);
+          o.w = prmt(v[i].y, v[i].w, 0x7632u);
+          const int pos = base + n;
+          *reinterpret_cast<uint4*>(xp + ((size_t)g * pcap + pos) * kGK + ((c ^ (pos & 7)) * 8)) = o;
+          if (c == 0) xs[(size_t)g * pcap + pos] = s;
+        }
+      }
     }
   }
 }
@@ -786,16 +803,29 @@ __global__ void __launch_bounds__(kGCombineThreads) grouped_combine_kernel(
   const int nv = offsets[*num_unique];
   for (int i = threadIdx.x; i < nv; i += blockDim.x) pos_of[pair_list[i]] = i;
   __syncthreads();
-  const long long total = (long long)T * H;
+  // four consecutive columns per thread (H is a multiple of 4): one 16-byte load of y
+  // per pair; each column's sum runs over j in ascending order as a chain of fmaf
+  const int H4 = H / 4;
+  const long long total = (long long)T * H4;
   for (long long o = (long long)blockIdx.x * blockDim.x + threadIdx.x; o < total;
        o += (long long)gridDim.x * blockDim.x) {
-    const int t = (int)(o / H), c = (int)(o % H);
-    float acc = 0.f;
+    const int t = (int)(o / H4), c4 = (int)(o % H4);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < k; ++j) {
       const int pos = pos_of[t * k + j];
-      if (pos >= 0) acc = fmaf(__ldg(w + t * k + j), __ldcg(y + (size_t)pos * H + c), acc);
+      if (pos >= 0) {
+        const float wj = __ldg(w + t * k + j);
+        const float4 yv = __ldcg(reinterpret_cast<const float4*>(y + (size_t)pos * H) + c4);
+        acc.x = fmaf(wj, yv.x, acc.x);
+        acc.y = fmaf(wj, yv.y, acc.y);
+        acc.z = fmaf(wj, yv.z, acc.z);
+        acc.w = fmaf(wj, yv.w, acc.w);
+      }
     }
-    out[o] = float_to_bf16_bits(acc);
+    uint2 ob;
+    ob.x = (uint32_t)float_to_bf16_bits(acc.x) | ((uint32_t)float_to_bf16_bits(acc.y) << 16);
+    ob.y = (uint32_t)float_to_bf16_bits(acc.z) | ((uint32_t)float_to_bf16_bits(acc.w) << 16);
+    reinterpret_cast<uint2*>(out + (size_t)t * H)[c4] = ob;
   }
 }
 
