@@ -310,6 +310,7 @@ def test_grouped_path_selected_for_large_windows():
     (160, 8, 64, 512, 256),
     (130, 8, 16, 256, 384),
     (130, 8, 16, 6144, 256),  # hidden 6144 (GLM-5.2's width)
+    (130, 8, 8, 8192, 128),   # the widest hidden the library takes
 ])
 def test_grouped_small(cfg):
     T, k, E, H, I = cfg
